@@ -1,0 +1,161 @@
+/*
+ * oracle.c -- plain, slow CPU oracle for the element-wise recurrence scans.
+ *
+ * TEST INFRASTRUCTURE.  Only the test suite, the package's smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The product path (the
+ * CUDA library under scan_gated_rnns_b200/) never links, loads or calls it, and
+ * the two share no code: no headers, no helpers, no constants.
+ *
+ * Everything here is written for a reader to check by eye against the method:
+ *   - minGRU (the layer profiled on the page "Mingru Pytorch", sections
+ *     "Requirements & limits" and "Install and apply the minGRU layer"): a
+ *     gated recurrence over the time axis of a (B, T, D) tensor,
+ *         z_t       = sigmoid(k_t)
+ *         htilde_t  = g(hx_t),   g(x) = x + 0.5 for x >= 0, sigmoid(x) otherwise
+ *         h_t       = (1 - z_t) * h_{t-1} + z_t * htilde_t,
+ *     with an optional carried state h_0 (absent => h_0 = 0).  The page states
+ *     that the implementation is the "log-space" numerically stable version;
+ *     that version evaluates the same h_t as
+ *         h_t = exp( a*_t + logcumsumexp_{s<=t}( log z_s + log htilde_s - a*_s ) ),
+ *         a*_t = cumsum_{r<=t}( -softplus(k_r) ),
+ *     where a carried h_0 > 0 joins the logcumsumexp as an s = 0 term log h_0
+ *     with a*_0 = 0.  Two oracles are provided, one per formulation, so that
+ *     each pins the other.
+ *   - the MinMax neuron (page "MinMax Recurrent Neural Cascades", section
+ *     "The model", item 3):  x_{t+1} = max(min(r_t, x_t), s_t), element-wise.
+ *
+ * Conventions (the pages are silent on them; these are the plainest readings):
+ *   - layout (B, T, D) row-major, D fastest, like the page's torch.randn(2, 1024, 512);
+ *   - output index t holds the state after consuming token t (T outputs; the
+ *     carried initial state is not echoed);
+ *   - optional initial states are (B, D) with a batch stride in elements;
+ *   - all arithmetic is IEEE binary64; inputs given in fp32/bf16 are widened
+ *     exactly by the caller.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+
+/* ---------------------------------------------------------------- helpers */
+
+/* logistic sigmoid, evaluated on the side where exp() cannot overflow */
+static double sigmoid(double x)
+{
+    if (x >= 0.0) {
+        return 1.0 / (1.0 + exp(-x));
+    }
+    double e = exp(x);
+    return e / (1.0 + e);
+}
+
+/* minGRU candidate activation g */
+static double g_act(double x)
+{
+    return (x >= 0.0) ? x + 0.5 : sigmoid(x);
+}
+
+/* softplus(x) = log(1 + e^x), without overflow */
+static double softplus(double x)
+{
+    return fmax(x, 0.0) + log1p(exp(-fabs(x)));
+}
+
+/* --------------------------------------------------------- minGRU, linear */
+
+/*
+ * The recurrence h_t = (1 - z_t) h_{t-1} + z_t g(hx_t), one channel at a time,
+ * sequentially in t.  1 - z_t is written as sigmoid(-k_t), which is the same
+ * number without the cancellation of 1 - sigmoid(k_t) when z_t is near 1.
+ */
+int oracle_mingru_linear(const double *k, const double *hx,
+                         const double *h0, int64_t h0_bs,
+                         double *h, int64_t B, int64_t T, int64_t D)
+{
+    if (B < 0 || T < 0 || D < 0) return 1;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t d = 0; d < D; ++d) {
+            double state = h0 ? h0[b * h0_bs + d] : 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                int64_t i = (b * T + t) * D + d;
+                double z = sigmoid(k[i]);
+                double one_minus_z = sigmoid(-k[i]);
+                state = one_minus_z * state + z * g_act(hx[i]);
+                h[i] = state;
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------ minGRU, log space */
+
+/*
+ * The log-space formula, term by term:
+ *   log(1 - z_t)   = -softplus(k_t)           (accumulated into a*_t)
+ *   log z_t        = -softplus(-k_t)
+ *   log htilde_t   = log(hx_t + 0.5) if hx_t >= 0, else -softplus(-hx_t)
+ *   v_s            = log z_s + log htilde_s - a*_s
+ *   h_t            = exp(a*_t + logcumsumexp_{s<=t} v_s)
+ * The running logcumsumexp is kept as (m, acc) with value m + log(acc), m the
+ * running maximum, which is the usual overflow-free way to add exponentials.
+ * A carried h0 contributes v_0 = log h0 (a*_0 = 0); it must be > 0.  Finite k
+ * only: k = +-inf makes a*_t infinite and the formula undefined.
+ */
+int oracle_mingru_log(const double *k, const double *hx,
+                      const double *h0, int64_t h0_bs,
+                      double *h, int64_t B, int64_t T, int64_t D)
+{
+    if (B < 0 || T < 0 || D < 0) return 1;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t d = 0; d < D; ++d) {
+            double a_star = 0.0;
+            double m = -INFINITY; /* running max of v_s */
+            double acc = 0.0;     /* sum of exp(v_s - m) */
+            if (h0) {
+                m = log(h0[b * h0_bs + d]);
+                acc = 1.0;
+            }
+            for (int64_t t = 0; t < T; ++t) {
+                int64_t i = (b * T + t) * D + d;
+                a_star += -softplus(k[i]);
+                double log_z = -softplus(-k[i]);
+                double x = hx[i];
+                double log_ht = (x >= 0.0) ? log(x + 0.5) : -softplus(-x);
+                double v = log_z + log_ht - a_star;
+                if (v > m) {
+                    acc = acc * exp(m - v) + 1.0;
+                    m = v;
+                } else {
+                    acc += exp(v - m);
+                }
+                h[i] = exp(a_star + m + log(acc));
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------- MinMax */
+
+/*
+ * x_{t+1} = max(min(r_t, x_t), s_t), sequentially in t; out[t] = x_{t+1}.
+ * x0 absent => +0.  min/max only select one of their operands, so the result
+ * is exactly one of the input values whatever the working precision.
+ */
+int oracle_minmax(const double *r, const double *s,
+                  const double *x0, int64_t x0_bs,
+                  double *x, int64_t B, int64_t T, int64_t D)
+{
+    if (B < 0 || T < 0 || D < 0) return 1;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t d = 0; d < D; ++d) {
+            double state = x0 ? x0[b * x0_bs + d] : 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                int64_t i = (b * T + t) * D + d;
+                state = fmax(fmin(r[i], state), s[i]);
+                x[i] = state;
+            }
+        }
+    }
+    return 0;
+}

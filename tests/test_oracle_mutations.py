@@ -1,0 +1,94 @@
+"""Plant plausible mistakes in a copy of the oracle's C source, on the CPU, and
+check that the pin suite catches every one of them.
+
+Each mutant is oracle.c with one textual edit (a swapped operand, a dropped
+term, a wrong sign, an off-by-one in the output index), compiled to a scratch
+library; the pin tests of test_oracle_pins.py then run against it and at
+least one of them must fail.  This is what makes the pins a check of the
+oracle rather than a restatement of it.
+"""
+import math
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(os.path.abspath(oracle.__file__)), "oracle.c")
+
+MUTANTS = {
+    # minGRU, linear
+    "z_and_one_minus_z_swapped": ("double one_minus_z = sigmoid(-k[i]);",
+                                  "double one_minus_z = sigmoid(k[i]);"),
+    "g_branches_swapped": ("return (x >= 0.0) ? x + 0.5 : sigmoid(x);",
+                           "return (x >= 0.0) ? sigmoid(x) : x + 0.5;"),
+    "g_offset_sign": ("return (x >= 0.0) ? x + 0.5 : sigmoid(x);",
+                      "return (x >= 0.0) ? x - 0.5 : sigmoid(x);"),
+    "sigmoid_sign": ("return 1.0 / (1.0 + exp(-x));", "return 1.0 / (1.0 + exp(x));"),
+    "h0_dropped": ("double state = h0 ? h0[b * h0_bs + d] : 0.0;\n            for (int64_t t = 0; t < T; ++t) {\n                int64_t i = (b * T + t) * D + d;\n                double z",
+                   "double state = 0.0;\n            for (int64_t t = 0; t < T; ++t) {\n                int64_t i = (b * T + t) * D + d;\n                double z"),
+    "output_before_update": ("state = one_minus_z * state + z * g_act(hx[i]);\n                h[i] = state;",
+                             "h[i] = state;\n                state = one_minus_z * state + z * g_act(hx[i]);"),
+    # minGRU, log space
+    "log_astar_sign": ("a_star += -softplus(k[i]);", "a_star += softplus(k[i]);"),
+    "log_z_sign": ("double log_z = -softplus(-k[i]);", "double log_z = -softplus(k[i]);"),
+    "log_h0_term_dropped": ("m = log(h0[b * h0_bs + d]);\n                acc = 1.0;",
+                            "m = -INFINITY;\n                acc = 0.0;"),
+    "log_candidate_branch": ("(x >= 0.0) ? log(x + 0.5) : -softplus(-x);",
+                             "(x >= 0.0) ? log(x + 0.5) : -softplus(x);"),
+    "log_lse_update": ("acc = acc * exp(m - v) + 1.0;", "acc = acc + 1.0;"),
+    # MinMax
+    "minmax_min_max_swapped": ("state = fmax(fmin(r[i], state), s[i]);",
+                               "state = fmin(fmax(r[i], state), s[i]);"),
+    "minmax_r_s_swapped": ("state = fmax(fmin(r[i], state), s[i]);",
+                           "state = fmax(fmin(s[i], state), r[i]);"),
+    "minmax_x0_dropped": ("double state = x0 ? x0[b * x0_bs + d] : 0.0;",
+                          "double state = 0.0;"),
+}
+
+
+def _pin_checks():
+    """Every pin of test_oracle_pins.py, with its parameters spelled out."""
+    out = []
+    for name in ("mingru_worked_example.txt", "mingru_worked_example_noh0.txt"):
+        out.append(lambda n=name: pins.test_mingru_linear_golden(n))
+        out.append(lambda n=name: pins.test_mingru_log_golden(n))
+    out.append(pins.test_minmax_golden)
+    for wh in (False, True):
+        for km in (0.0, 2.0, -2.0):
+            out.append(lambda a=wh, b=km: pins.test_linear_and_log_space_agree(a, b))
+    out += [pins.test_gate_one_gives_candidate, pins.test_large_gate_is_near_candidate,
+            pins.test_gate_zero_holds_state, pins.test_small_gate_is_near_state,
+            pins.test_sigmoid_branches_match_library, pins.test_positive_and_inside_hull,
+            pins.test_minmax_selection_bound_monotone_hold, pins.test_minmax_default_state_is_zero]
+    for args in [(math.log(3.0), 0.5, 0.2), (0.3, -1.7, 0.9), (-1.1, 2.25, 0.5)]:
+        out.append(lambda a=args: pins.test_constant_inputs_closed_form(*a))
+    for T in (1, 2):
+        out.append(lambda t=T: pins.test_minmax_brute_force(t))
+    return out
+
+
+def test_unmutated_oracle_passes_every_check():
+    for check in _pin_checks():
+        check()
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_planted_mistake_is_caught(mutant, tmp_path):
+    before, after = MUTANTS[mutant]
+    src = open(SRC).read()
+    assert src.count(before) >= 1, f"mutation anchor for {mutant} not found"
+    msrc = tmp_path / "mutant.c"
+    msrc.write_text(src.replace(before, after, 1))
+    lib = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", *oracle.CFLAGS, "-o", str(lib), str(msrc), "-lm"], check=True)
+    failures = 0
+    with oracle.use_library(str(lib)):
+        for check in _pin_checks():
+            try:
+                check()
+            except (AssertionError, ValueError, FloatingPointError):
+                failures += 1
+    assert failures > 0, f"no pin caught mutant {mutant}"
