@@ -1,0 +1,513 @@
+#!/usr/bin/env python
+"""Throughput of the element-wise recurrence scans on B200, one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl b200|reference] [--no-rows]
+
+A step is one minGRU scan (activations, in-chunk scan, chunk hand-off,
+fix-up, store) over one batch of the workload, with inputs resident in HBM.
+The default workload is the minGRU scan with carried state,
+B=8 T=4096 D=1024 fp32 (k, hx ~ N(0,1), h0 ~ U(0.1,1)).  Its inputs (268 MB)
+and output (134 MB) are larger than the 126 MB L2, so back-to-back steps do
+not hit in L2.
+
+Metric: scan HBM GB/s = algorithmic bytes (inputs read once + output written
+once + initial state) per step / time per step, summed over GPUs.  Also
+reported: Gelem/s, the dominant kernel's roofline fraction against the
+measured HBM copy bandwidth, the end-to-end figure through the public API
+with the inputs in pinned host memory (host<->device copies timed), the CPU
+oracle on a bounded sample of the same workload, and one line per other hot
+path row (MinMax scan, long sequence, bf16 I/O, small shape, decode step).
+
+Multi-GPU (torchrun): every rank scans its own batch shard of the same size
+(weak scaling); channels are independent, so there is no data-path
+collective.  Timing is the max over ranks of device-measured time.
+
+--impl reference times the CPU oracle (the reference arm of this method) on
+the host cores, on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from scan_gated_rnns_b200.synth import BENCH_WORKLOAD, WORKLOADS, generate  # noqa: E402
+
+METRIC = "scan HBM GB/s (fraction of B200 peak) and Gelem/s at BxTxD, vs CPU oracle"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["scan_gated_rnns_b200/csrc/scan_engine.cuh", "scan_gated_rnns_b200/csrc/sgr_api.cu"]
+
+
+# ------------------------------------------------------------------ helpers
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier pool measurement)"
+
+
+def recorded_traffic(workload: str):
+    """dram bytes per launch from the committed ncu summary of this kernel and
+    workload, if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"scan_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    try:
+        return int(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """SM clock, power and clock-event reasons via NVML, polled from a thread
+    every `period` seconds; samples are kept with host timestamps so the ones
+    inside the timed window can be selected."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index: int, period: float = 0.002):
+        self.samples = []
+        self.period = period
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            self.nv = pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            handle = None
+            for cand in (uuid, "GPU-" + uuid):
+                try:
+                    handle = pynvml.nvmlDeviceGetHandleByUUID(cand)
+                    break
+                except Exception:
+                    continue
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.h = handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report the clocks as unknown
+            self.err = str(e)
+
+    def _read(self):
+        nv = self.nv
+        sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        try:
+            pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+        except Exception:
+            pw = None
+        return sm, rs, pw
+
+    def start(self):
+        if not self.ok:
+            return self
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    sm, rs, pw = self._read()
+                    self.samples.append((time.time(), sm, rs, pw))
+                except Exception:
+                    pass
+                time.sleep(self.period)
+
+        self._t = threading.Thread(target=loop, daemon=True)
+        self._t.start()
+        return self
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": "unavailable: " + getattr(self, "err", "")}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        used = inside
+        where = "timed region"
+        if not inside:   # region shorter than one poll: the nearest samples around it
+            used = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+            where = "nearest to the timed region (shorter than the poll period)"
+        reasons = set()
+        for _, _, rs, _ in used:
+            for name, bit in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        sm = [s[1] for s in used]
+        pw = [s[3] for s in used if s[3] is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(used), "window": where,
+                "power_w_max": max(pw) if pw else None, "source": "nvml"}
+
+
+# ------------------------------------------------------------ distribution
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Each rank scans its own batch shard: same shape, its own seeded draws."""
+    return base_seed + 1000 * rank
+
+
+def reduce_max(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None) -> None:
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate(bytes_per_step: int, elems_per_step: int, steps: int, max_seconds: float, world: int):
+    """Whole-job throughput: every rank moved bytes_per_step per step."""
+    return {
+        "gbs": world * bytes_per_step * steps / max_seconds / 1e9,
+        "gelems": world * elems_per_step * steps / max_seconds / 1e9,
+        "ms_per_step": max_seconds * 1e3 / steps,
+    }
+
+
+# ---------------------------------------------------------------- GPU timing
+
+def timed_launches(fn, steps: int, stream):
+    """Time `steps` calls of fn with CUDA events on the launching stream: the
+    whole region and each launch.  Returns (total_s, mean_launch_s)."""
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        starts[i].record(stream)
+        fn()
+        ends[i].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    total = t0.elapsed_time(t1) / 1e3
+    per = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends)) / 1e3
+    return total, per
+
+
+def scan_fn(w, p, q, init, out, ws):
+    import scan_gated_rnns_b200 as sgr
+    f = sgr.mingru_scan if w.op == "mingru" else sgr.minmax_scan
+    return lambda: f(p, q, init, out=out, workspace=ws)
+
+
+def measure_row(w, device, steps=10, warmup=3):
+    """One other hot-path row, timed alone (inputs larger than L2 except the
+    small shape, which is launch-latency bound)."""
+    import scan_gated_rnns_b200 as sgr
+    p, q, init = generate(w, device=device)
+    out = torch.empty_like(p)
+    ws = sgr.Workspace(sgr.workspace_size(w.op, w.B, w.T, w.D, p.dtype), device)
+    fn = scan_fn(w, p, q, init, out, ws)
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(device)
+    total, per = timed_launches(fn, steps, stream)
+    bytes_ = w.algorithmic_bytes()
+    peak, _ = hbm_peak()
+    gbs = bytes_ / per / 1e9
+    plan = sgr._abi.plan(0 if w.op == "mingru" else 1, w.B, w.T, w.D,
+                         0 if w.dtype == "f32" else 1, True)
+    del p, q, init, out, ws
+    return {"op": f"{w.op}_scan", "B": w.B, "T": w.T, "D": w.D, "io_dtype": w.dtype,
+            "us_per_launch": round(per * 1e6, 2), "gbs": round(gbs, 1),
+            "gelem_per_s": round(w.n_elems / per / 1e9, 2), "roofline_frac": round(gbs / peak, 4),
+            "bytes_per_launch": bytes_,
+            "tile": f"{plan['tile_rows']}x{plan['tile_channels']}", "n_tiles": plan["n_tiles"]}
+
+
+def measure_step_row(device, B=8, D=1024, calls=200, warmup=10):
+    """Decode step on (B, D): latency-bound; microseconds per call."""
+    import scan_gated_rnns_b200 as sgr
+    g = torch.Generator(device=device).manual_seed(77)
+    k = torch.randn(B, D, device=device, generator=g)
+    hx = torch.randn(B, D, device=device, generator=g)
+    h = torch.rand(B, D, device=device, generator=g) + 0.1
+    fn = lambda: sgr.mingru_step(k, hx, h, out=h)   # noqa: E731
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    total, per = timed_launches(fn, calls, torch.cuda.current_stream(device))
+    return {"op": "mingru_step", "B": B, "D": D, "io_dtype": "f32",
+            "us_per_call": round(total / calls * 1e6, 2),
+            "us_per_launch_event": round(per * 1e6, 2), "bytes_per_call": 4 * 4 * B * D}
+
+
+def cpu_baseline(w, p, q, init, budget_s: float = 12.0):
+    """The fp64 CPU oracle as it stands, on a bounded sample of the workload:
+    whole batch rows (all T and D of each), threads over rows."""
+    import oracle
+    cores = max(1, min(os.cpu_count() or 1, 32))
+    row = w.T * w.D
+    # time one row first, then size the sample to about `budget_s` of wall time
+    p1, q1 = p[:1].cpu(), q[:1].cpu()
+    i1 = init[:1].cpu() if init is not None else None
+    t = time.perf_counter()
+    oracle.mingru_linear(p1, q1, i1) if w.op == "mingru" else oracle.minmax(p1, q1, i1)
+    one = time.perf_counter() - t
+    rows = int(max(1, min(w.B, budget_s / max(one, 1e-6) * min(cores, w.B))))
+    threads = min(cores, rows)
+    ps, qs = p[:rows].cpu(), q[:rows].cpu()
+    ins = init[:rows].cpu() if init is not None else None
+    fn = oracle.mingru_linear if w.op == "mingru" else oracle.minmax
+    t = time.perf_counter()
+    fn(ps, qs, ins, threads=threads)
+    wall = time.perf_counter() - t
+    bytes_ = 3 * rows * row * w.elem_bytes + (rows * w.D * w.elem_bytes if init is not None else 0)
+    return {"value": round(bytes_ / wall / 1e9, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "gelem_per_s": round(rows * row / wall / 1e9, 5), "seconds": round(wall, 2),
+            "sample": f"batch rows 0..{rows - 1} of the workload ({rows}x{w.T}x{w.D} elements), "
+                      f"fp64 {'linear-space minGRU' if w.op == 'mingru' else 'MinMax'} oracle, "
+                      f"{threads} thread(s) over rows; host has {os.cpu_count()} logical CPUs"}
+
+
+# ------------------------------------------------------------------- arms
+
+def run_b200(args):
+    import scan_gated_rnns_b200 as sgr
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the scans have no CPU path)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    w = WORKLOADS[args.workload]
+    p, q, init = generate(w, seed=shard_seed(w.seed, rank), device=device)
+    out = torch.empty_like(p)
+    ws = sgr.Workspace(sgr.workspace_size(w.op, w.B, w.T, w.D, p.dtype), device)
+    fn = scan_fn(w, p, q, init, out, ws)
+    stream = torch.cuda.current_stream(device)
+    bytes_step = w.algorithmic_bytes()
+
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local).start()
+    barrier(world, device)
+    torch.cuda.synchronize()
+    h0 = time.time()
+    total, per_launch = timed_launches(fn, args.steps, stream)
+    h1 = time.time()
+    barrier(world, device)
+    clocks.stop()
+    if ws.status() != 0:
+        raise SystemExit("bench.py: a chunk timed out waiting for its carry (workspace status)")
+    t_max = reduce_max(total, world, device)
+    launch_max = reduce_max(per_launch, world, device)
+    agg = aggregate(bytes_step, w.n_elems, args.steps, t_max, world)
+
+    # end to end through the public API: pinned host inputs, copies timed
+    e2e = None
+    if not args.no_e2e:
+        hp = p.cpu().pin_memory()
+        hq = q.cpu().pin_memory()
+        hi = init.cpu().pin_memory() if init is not None else None
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dp, dq = torch.empty_like(p), torch.empty_like(q)
+        di = torch.empty_like(init) if init is not None else None
+
+        def e2e_step():
+            dp.copy_(hp, non_blocking=True)
+            dq.copy_(hq, non_blocking=True)
+            if di is not None:
+                di.copy_(hi, non_blocking=True)
+            y = (sgr.mingru_scan if w.op == "mingru" else sgr.minmax_scan)(dp, dq, di, out=out, workspace=ws)
+            hout.copy_(y, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world, device)
+        e_steps = max(1, min(args.steps, 5))
+        et, _ = timed_launches(e2e_step, e_steps, stream)
+        barrier(world, device)
+        et = reduce_max(et, world, device)
+        h2d = hp.numel() * hp.element_size() + hq.numel() * hq.element_size() + \
+            (hi.numel() * hi.element_size() if hi is not None else 0)
+        d2h = hout.numel() * hout.element_size()
+        e2e = {"value": round(world * bytes_step * e_steps / et / 1e9, 2), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(et * 1e3 / e_steps, 3), "steps": e_steps}
+        del hp, hq, hi, hout, dp, dq, di
+
+    peak, peak_src = hbm_peak()
+    achieved = bytes_step / launch_max / 1e9
+    plan = sgr._abi.plan(0 if w.op == "mingru" else 1, w.B, w.T, w.D, 0 if w.dtype == "f32" else 1, True)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": UNIT,
+                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name),
+                "peak_source": peak_src, "kernel": "sgr::scan_kernel",
+                "bytes_per_launch": bytes_step,
+                "launch_us": round(launch_max * 1e6, 2)}
+    line = {
+        "metric": METRIC, "value": round(agg["gbs"], 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(agg["ms_per_step"], 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded torch generator on the device)",
+        "config": {"workload": w.name, "op": f"{w.op}_scan", "B": w.B, "T": w.T, "D": w.D,
+                   "io_dtype": w.dtype, "initial_state": init is not None,
+                   "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
+                   "tile": f"{plan['tile_rows']}x{plan['tile_channels']}", "n_tiles": plan["n_tiles"],
+                   "l2": "inputs larger than L2 (inputs + output per step "
+                         f"{bytes_step / 1e6:.0f} MB vs 126 MB L2); no flush"},
+        "gelem_per_s": round(agg["gelems"], 2),
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(h0, h1),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(w, p, q, init)
+    del p, q, init, out, ws
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_rows:
+        rows = {}
+        for name in WORKLOADS:
+            if name != w.name:
+                rows[name] = measure_row(WORKLOADS[name], device)
+                torch.cuda.empty_cache()
+        rows["mingru_step_b8_d1024_f32"] = measure_step_row(device)
+        line["rows"] = rows
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args):
+    """The CPU oracle timed as the reference arm, on bounded samples."""
+    import oracle
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    if dev.type == "cuda":
+        p, q, init = generate(w, device=dev)
+    else:
+        p, q, init = generate(w.scaled(B=1))
+    cores = max(1, min(os.cpu_count() or 1, 32))
+    # one step = the oracle over one batch row (T x D elements) per thread
+    rows = max(1, min(w.B, cores))
+    ps, qs = p[:rows].cpu(), q[:rows].cpu()
+    ins = init[:rows].cpu() if init is not None else None
+    del p, q, init
+    fn = oracle.mingru_linear if w.op == "mingru" else oracle.minmax
+    for _ in range(args.warmup):
+        fn(ps[:1, : max(1, w.T // 64)], qs[:1, : max(1, w.T // 64)],
+           ins[:1] if ins is not None else None)
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        fn(ps, qs, ins, threads=rows)
+        times.append(time.perf_counter() - t)
+    wall = sum(times)
+    bytes_step = 3 * rows * w.T * w.D * w.elem_bytes + (rows * w.D * w.elem_bytes if ins is not None else 0)
+    value = bytes_step * args.steps / wall / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(wall / args.steps * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded torch generator)", "impl": "reference",
+        "config": {"workload": w.name, "op": f"{w.op}_scan", "B": w.B, "T": w.T, "D": w.D,
+                   "io_dtype": w.dtype, "initial_state": ins is not None, "global_batch": w.B,
+                   "seq_len": w.T, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": rows, "kind": "oracle",
+                         "sample": f"each step: batch rows 0..{rows - 1} ({rows}x{w.T}x{w.D} elements) "
+                                   f"of the workload, fp64 oracle, {rows} thread(s)"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-rows", action="store_true", help="skip the other hot-path rows")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    _, world, _ = dist_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_b200(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,227 @@
+/*
+ * scan_gated_rnns.h -- C ABI of the B200 element-wise recurrence scans.
+ *
+ * Three operations, all element-wise over channels and sequential in time:
+ *
+ *   mingru_scan   minGRU over a whole sequence (page "Mingru Pytorch", sections
+ *                 "Requirements & limits" -- the log-space numerically stable
+ *                 minGRU -- and "Install and apply the minGRU layer": a batched
+ *                 (B, T, D) tensor in, a tensor of the same shape out):
+ *                     z_t = sigmoid(k_t),  htilde_t = g(hx_t),
+ *                     g(x) = x + 0.5 (x >= 0), sigmoid(x) (x < 0),
+ *                     h_t = (1 - z_t) h_{t-1} + z_t htilde_t,
+ *                 which the log-space form writes as
+ *                     h_t = exp(a*_t + logcumsumexp_{s<=t}(log z_s + log htilde_s - a*_s)),
+ *                     a*_t = sum_{r<=t} -softplus(k_r),
+ *                 with an optional carried state h_0 (absent: h_0 = 0).
+ *   mingru_step   one token of the same recurrence, for token-by-token decoding
+ *                 with the hidden state carried between calls (page "Mingru
+ *                 Pytorch", guide "Process a sequence sequentially with carried
+ *                 hidden state").  It returns only the new state.
+ *   minmax_scan   MinMax neuron x_{t+1} = max(min(r_t, x_t), s_t) over a whole
+ *                 sequence (page "MinMax Recurrent Neural Cascades", section
+ *                 "The model", item 3), with an optional carried state x_0
+ *                 (absent: +0).  Exact: the result is bitwise one of the inputs.
+ *
+ * The input projections that produce k, hx (or r, s) are not part of this
+ * library: callers pass pre-activation tensors.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Layout: (B, T, D) row-major, D fastest, contiguous; output index t holds
+ *    the state after token t (T outputs; the initial state is not echoed).
+ *    Initial states and step operands are (B, D) rows with a batch stride in
+ *    ELEMENTS; stride 0 broadcasts one D-vector to every batch row (inputs only).
+ *  - Pointers are DEVICE pointers (cudaMalloc / caching-allocator memory of the
+ *    current device).  The caller owns every buffer; the library keeps no
+ *    pointer after a call returns and allocates nothing.
+ *  - dtype selects the storage type of every tensor of a call (inputs, initial
+ *    state, output).  Arithmetic is fp32 on the device in both cases; bf16
+ *    inputs widen exactly and outputs round to nearest-even.
+ *  - Every call is asynchronous on `stream`.  Host-detectable errors return
+ *    before anything is enqueued.  A launch failure returns SGR_ERR_CUDA.
+ *  - Outputs must not overlap inputs (checked on the address ranges), except
+ *    that mingru_step may update its state in place (h_out == h_prev with the
+ *    same batch stride).
+ *  - A size of 0 in any dimension is a valid no-op; negative sizes are
+ *    SGR_ERR_INVALID_ARG.
+ *  - Fast path: 16-byte aligned base pointers and D a multiple of 4 (fp32) or
+ *    8 (bf16) take 128-bit vector loads; anything else runs a scalar GPU
+ *    variant.  Results do not depend on the variant beyond fp32 rounding order.
+ *  - minGRU inputs are NaN-free; h_0 > 0 where the log-space reading matters
+ *    (the linear recurrence the kernels evaluate is defined for any h_0).
+ *    MinMax inputs are NaN-free; with no -0.0 among the inputs the result is
+ *    bit-identical to the sequential loop, otherwise equal as a value.
+ *
+ * Workspace (mingru_scan, minmax_scan)
+ * ------------------------------------
+ *  Long sequences are cut into chunks of T that run on different thread
+ *  blocks; each chunk receives its carried state from the chunks before it
+ *  through a small device workspace (flags and per-chunk summaries) that stays
+ *  in L2.  sgr_workspace_size() gives the bytes a call needs (0 when the whole
+ *  sequence fits one chunk, in which case workspace may be NULL).  Before its
+ *  first use a workspace must be zero-filled once (sgr_workspace_init or
+ *  cudaMemset); afterwards calls keep it valid.  One workspace must not be used
+ *  by two calls that can run at the same time (e.g. on two streams).
+ *  Calls may be captured in a CUDA graph; a captured call zero-fills the flag
+ *  region itself inside the graph.
+ */
+#ifndef SCAN_GATED_RNNS_H
+#define SCAN_GATED_RNNS_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define SGR_API __attribute__((visibility("default")))
+#else
+#define SGR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sgr_status {
+    SGR_OK = 0,
+    SGR_ERR_INVALID_ARG = 1,  /* null pointer with data to move, negative size or
+                                 stride, unknown dtype/op, overlapping output      */
+    SGR_ERR_UNSUPPORTED = 2,  /* sizes beyond what the kernels index (grid > 2^31-1,
+                                 byte counts overflowing int64)                    */
+    SGR_ERR_WORKSPACE = 3,    /* workspace needed but NULL, too small or not
+                                 16-byte aligned                                   */
+    SGR_ERR_CUDA = 4,         /* a CUDA runtime call or a kernel launch failed     */
+    SGR_ERR_TIMEOUT = 5       /* device side: a chunk waited too long (~0.3 s) for
+                                 the state of the chunk before it and gave up; its
+                                 outputs are NaN.  Reported by sgr_workspace_status */
+} sgr_status_t;
+
+typedef enum sgr_dtype { SGR_F32 = 0, SGR_BF16 = 1 } sgr_dtype_t;
+
+typedef enum sgr_op { SGR_OP_MINGRU = 0, SGR_OP_MINMAX = 1 } sgr_op_t;
+
+/* ---------------------------------------------------------------- scans */
+
+/*
+ * mingru_scan -- h[b, t, :] for t = 0..T-1 from k, hx (B, T, D).
+ *   k, hx    : gate and candidate pre-activations, (B, T, D), dtype.
+ *   h0       : optional initial state rows (B, D) with batch stride
+ *              h0_batch_stride (elements, >= 0); NULL means h_0 = 0.
+ *   h        : output (B, T, D), dtype; must not overlap k, hx or h0.
+ *   workspace: see above; ws_bytes >= sgr_workspace_size(SGR_OP_MINGRU, ...).
+ */
+SGR_API sgr_status_t mingru_scan(const void *k, const void *hx,
+                         const void *h0, int64_t h0_batch_stride,
+                         void *h, int64_t B, int64_t T, int64_t D,
+                         sgr_dtype_t dtype, void *workspace, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/*
+ * minmax_scan -- x[b, t, :] = x_{t+1} for t = 0..T-1 from r, s (B, T, D).
+ *   x0 : optional initial state rows (B, D), batch stride x0_batch_stride;
+ *        NULL means x_0 = +0.
+ *   x  : output (B, T, D), dtype; must not overlap r, s or x0.
+ */
+SGR_API sgr_status_t minmax_scan(const void *r, const void *s,
+                         const void *x0, int64_t x0_batch_stride,
+                         void *x, int64_t B, int64_t T, int64_t D,
+                         sgr_dtype_t dtype, void *workspace, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/*
+ * mingru_step -- one token: h_out = (1 - z) h_prev + z g(hx_t), z = sigmoid(k_t).
+ *   k_t, hx_t : (B, D) rows with batch strides (elements; e.g. k[:, t, :] of a
+ *               (B, T, D) tensor has stride T*D).
+ *   h_prev    : (B, D) rows with batch stride, or NULL for a zero state.
+ *   h_out     : (B, D) rows with batch stride (>= D when B > 1).  May equal
+ *               h_prev (same pointer and stride) for an in-place update; any
+ *               other overlap with an operand is SGR_ERR_INVALID_ARG.
+ * No workspace.  The arithmetic per element is the one mingru_scan uses, so a
+ * prefix scanned in parallel followed by step calls matches the full scan to
+ * fp32 rounding.
+ */
+SGR_API sgr_status_t mingru_step(const void *k_t, int64_t k_batch_stride,
+                         const void *hx_t, int64_t hx_batch_stride,
+                         const void *h_prev, int64_t h_prev_batch_stride,
+                         void *h_out, int64_t h_out_batch_stride,
+                         int64_t B, int64_t D, sgr_dtype_t dtype,
+                         cudaStream_t stream);
+
+/* ------------------------------------------------------------ workspace */
+
+/* Bytes of workspace a scan of this shape needs (0: none).  Pure host code. */
+SGR_API size_t sgr_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D,
+                          sgr_dtype_t dtype);
+
+/* Zero-fill a workspace on `stream` (asynchronous). */
+SGR_API sgr_status_t sgr_workspace_init(void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Synchronize `stream`, then read the device-side status word of a workspace:
+ * SGR_OK, or SGR_ERR_TIMEOUT if any chunk gave up waiting since the word was
+ * last cleared.  clear != 0 resets the word to SGR_OK afterwards.
+ */
+SGR_API sgr_status_t sgr_workspace_status(void *workspace, size_t ws_bytes, int clear,
+                                  cudaStream_t stream);
+
+/* ------------------------------------------------------------- misc */
+
+SGR_API const char *sgr_status_string(sgr_status_t status);
+SGR_API const char *sgr_version(void);
+
+/*
+ * Tuning/testing knob, process-wide: force the chunk shape the scans use.
+ * channel_lanes in {8, 32} lanes across D per warp (0: automatic), rows_per_thread
+ * in {1, 2, 4, 8} (0: automatic; bf16 vector tiles cap it at 4).  Shapes the
+ * fast path cannot take fall back to automatic choices.  The chunk shape
+ * changes the workspace size: query sgr_workspace_size after changing it.
+ * Returns SGR_ERR_INVALID_ARG for other values.
+ */
+SGR_API sgr_status_t sgr_set_tile_override(int channel_lanes, int rows_per_thread);
+
+/* ------------------------------------------------------- introspection */
+
+/* How a scan of this shape is cut into tiles (rows x channels per block). */
+typedef struct sgr_plan {
+    int32_t vector_path;        /* 1: 128-bit loads; 0: scalar variant         */
+    int32_t channels_per_thread;
+    int32_t channel_lanes;      /* lanes across D per warp                      */
+    int32_t rows_per_thread;
+    int32_t warps;              /* data warps per block (plus one carry warp)   */
+    int32_t threads;            /* threads per block                            */
+    int64_t tile_rows;          /* rows of T per block                          */
+    int64_t tile_channels;      /* channels of D per block                      */
+    int64_t n_channel_tiles;    /* per batch row                                */
+    int64_t n_chains;           /* B * n_channel_tiles                          */
+    int64_t n_chunks;           /* tiles along T                                */
+    int64_t n_tiles;            /* blocks launched                              */
+    uint64_t workspace_bytes;   /* 0 when n_chunks == 1                         */
+    uint64_t off_flags, off_agg, off_pref;  /* workspace layout (bytes)         */
+} sgr_plan_t;
+
+/* Fill *plan for a scan; `aligned` says whether the operands would be 16-byte
+ * aligned.  Pure host code. */
+SGR_API sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D,
+                                   sgr_dtype_t dtype, int aligned, sgr_plan_t *plan);
+
+/* ------------------------------------------------------- testing hooks */
+
+/*
+ * Both hooks are process-wide and exist to exercise the bounded wait of the
+ * chunk hand-off without faulting or hanging a GPU.
+ * sgr_set_wait_limit: polls a chunk makes before it gives up waiting for an
+ *   earlier chunk (0 restores the default of 2^18 polls, a fraction of a second).
+ * sgr_set_drop_publish: the block with this tile index (chunk * n_chains +
+ *   chain) skips publishing its state, so the chunk after it in the same
+ *   channels waits until the limit, records SGR_ERR_TIMEOUT in the workspace
+ *   status word and writes NaN for its outputs; -1 (the default) disables it.
+ */
+SGR_API sgr_status_t sgr_set_wait_limit(uint32_t polls);
+SGR_API sgr_status_t sgr_set_drop_publish(int64_t tile);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SCAN_GATED_RNNS_H */

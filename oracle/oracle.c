@@ -35,6 +35,7 @@
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 /* ---------------------------------------------------------------- helpers */
 
@@ -63,9 +64,10 @@ static double softplus(double x)
 /* --------------------------------------------------------- minGRU, linear */
 
 /*
- * The recurrence h_t = (1 - z_t) h_{t-1} + z_t g(hx_t), one channel at a time,
- * sequentially in t.  1 - z_t is written as sigmoid(-k_t), which is the same
- * number without the cancellation of 1 - sigmoid(k_t) when z_t is near 1.
+ * The recurrence h_t = (1 - z_t) h_{t-1} + z_t g(hx_t), sequentially in t,
+ * for every channel (b, d); the state h_{t-1} is the previous output row.
+ * 1 - z_t is written as sigmoid(-k_t), which is the same number without the
+ * cancellation of 1 - sigmoid(k_t) when z_t is near 1.
  */
 int oracle_mingru_linear(const double *k, const double *hx,
                          const double *h0, int64_t h0_bs,
@@ -73,14 +75,18 @@ int oracle_mingru_linear(const double *k, const double *hx,
 {
     if (B < 0 || T < 0 || D < 0) return 1;
     for (int64_t b = 0; b < B; ++b) {
-        for (int64_t d = 0; d < D; ++d) {
-            double state = h0 ? h0[b * h0_bs + d] : 0.0;
-            for (int64_t t = 0; t < T; ++t) {
+        for (int64_t t = 0; t < T; ++t) {
+            for (int64_t d = 0; d < D; ++d) {
                 int64_t i = (b * T + t) * D + d;
+                double prev;
+                if (t > 0) {
+                    prev = h[i - D];
+                } else {
+                    prev = h0 ? h0[b * h0_bs + d] : 0.0;
+                }
                 double z = sigmoid(k[i]);
                 double one_minus_z = sigmoid(-k[i]);
-                state = one_minus_z * state + z * g_act(hx[i]);
-                h[i] = state;
+                h[i] = one_minus_z * prev + z * g_act(hx[i]);
             }
         }
     }
@@ -100,47 +106,61 @@ int oracle_mingru_linear(const double *k, const double *hx,
  * running maximum, which is the usual overflow-free way to add exponentials.
  * A carried h0 contributes v_0 = log h0 (a*_0 = 0); it must be > 0.  Finite k
  * only: k = +-inf makes a*_t infinite and the formula undefined.
+ * Per-channel running values (a*, m, acc) live in arrays over d so that the
+ * loops walk the (B, T, D) arrays row by row.
  */
 int oracle_mingru_log(const double *k, const double *hx,
                       const double *h0, int64_t h0_bs,
                       double *h, int64_t B, int64_t T, int64_t D)
 {
     if (B < 0 || T < 0 || D < 0) return 1;
+    if (D == 0) return 0;
+    double *a_star = malloc(sizeof(double) * (size_t)D);
+    double *m = malloc(sizeof(double) * (size_t)D);    /* running max of v_s */
+    double *acc = malloc(sizeof(double) * (size_t)D);  /* sum of exp(v_s - m) */
+    if (!a_star || !m || !acc) {
+        free(a_star); free(m); free(acc);
+        return 2;
+    }
     for (int64_t b = 0; b < B; ++b) {
         for (int64_t d = 0; d < D; ++d) {
-            double a_star = 0.0;
-            double m = -INFINITY; /* running max of v_s */
-            double acc = 0.0;     /* sum of exp(v_s - m) */
+            a_star[d] = 0.0;
+            m[d] = -INFINITY;
+            acc[d] = 0.0;
             if (h0) {
-                m = log(h0[b * h0_bs + d]);
-                acc = 1.0;
+                m[d] = log(h0[b * h0_bs + d]);
+                acc[d] = 1.0;
             }
-            for (int64_t t = 0; t < T; ++t) {
+        }
+        for (int64_t t = 0; t < T; ++t) {
+            for (int64_t d = 0; d < D; ++d) {
                 int64_t i = (b * T + t) * D + d;
-                a_star += -softplus(k[i]);
+                a_star[d] += -softplus(k[i]);
                 double log_z = -softplus(-k[i]);
                 double x = hx[i];
                 double log_ht = (x >= 0.0) ? log(x + 0.5) : -softplus(-x);
-                double v = log_z + log_ht - a_star;
-                if (v > m) {
-                    acc = acc * exp(m - v) + 1.0;
-                    m = v;
+                double v = log_z + log_ht - a_star[d];
+                if (v > m[d]) {
+                    acc[d] = acc[d] * exp(m[d] - v) + 1.0;
+                    m[d] = v;
                 } else {
-                    acc += exp(v - m);
+                    acc[d] += exp(v - m[d]);
                 }
-                h[i] = exp(a_star + m + log(acc));
+                h[i] = exp(a_star[d] + m[d] + log(acc[d]));
             }
         }
     }
+    free(a_star); free(m); free(acc);
     return 0;
 }
 
 /* ------------------------------------------------------------- MinMax */
 
 /*
- * x_{t+1} = max(min(r_t, x_t), s_t), sequentially in t; out[t] = x_{t+1}.
- * x0 absent => +0.  min/max only select one of their operands, so the result
- * is exactly one of the input values whatever the working precision.
+ * x_{t+1} = max(min(r_t, x_t), s_t), sequentially in t, for every channel;
+ * out[t] = x_{t+1} and the state x_t is the previous output row.  x0 absent
+ * => +0.  min/max only select one of their operands, so the result is
+ * exactly one of the input values whatever the working precision.
  */
 int oracle_minmax(const double *r, const double *s,
                   const double *x0, int64_t x0_bs,
@@ -148,12 +168,16 @@ int oracle_minmax(const double *r, const double *s,
 {
     if (B < 0 || T < 0 || D < 0) return 1;
     for (int64_t b = 0; b < B; ++b) {
-        for (int64_t d = 0; d < D; ++d) {
-            double state = x0 ? x0[b * x0_bs + d] : 0.0;
-            for (int64_t t = 0; t < T; ++t) {
+        for (int64_t t = 0; t < T; ++t) {
+            for (int64_t d = 0; d < D; ++d) {
                 int64_t i = (b * T + t) * D + d;
-                state = fmax(fmin(r[i], state), s[i]);
-                x[i] = state;
+                double state;
+                if (t > 0) {
+                    state = x[i - D];
+                } else {
+                    state = x0 ? x0[b * x0_bs + d] : 0.0;
+                }
+                x[i] = fmax(fmin(r[i], state), s[i]);
             }
         }
     }

@@ -1,0 +1,16 @@
+"""B200 (sm_100a) element-wise recurrence scans over the time axis.
+
+    mingru_scan(k, hx, h0=None)     minGRU, whole sequence (B, T, D)
+    mingru_step(k_t, hx_t, h_prev)  minGRU, one token (B, D)
+    minmax_scan(r, s, x0=None)      MinMax neuron, whole sequence (B, T, D)
+
+All three run in the CUDA library ``libsgr.so`` (C ABI:
+include/scan_gated_rnns.h); this package only marshals PyTorch tensors into
+it.  Build the library with ``python -m scan_gated_rnns_b200.build``.
+"""
+from ._abi import ScanError
+from .ops import (Workspace, default_workspace, mingru_scan, mingru_step, minmax_scan,
+                  set_tile_override, version, workspace_size)
+
+__all__ = ["ScanError", "Workspace", "default_workspace", "mingru_scan", "mingru_step",
+           "minmax_scan", "set_tile_override", "version", "workspace_size"]

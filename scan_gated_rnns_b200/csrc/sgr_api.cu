@@ -1,0 +1,343 @@
+// sgr_api.cu -- host side of the C ABI declared in include/scan_gated_rnns.h:
+// argument checks, the choice of chunk shape, the workspace layout and the
+// kernel launches.  No allocation, no synchronisation on the scan paths.
+#include "scan_gated_rnns.h"
+#include "scan_engine.cuh"
+
+#include <atomic>
+#include <cstring>
+#include <limits>
+
+namespace {
+
+using namespace sgr;
+
+constexpr int kWarps = 8;           // warps per tile block
+constexpr int64_t kTargetTiles = 4 * 148;  // prefer >= 4 tiles per SM before shrinking chunks
+constexpr size_t kAlign = 256;
+
+std::atomic<int> g_override_cg{0};
+std::atomic<int> g_override_r{0};
+// Launch epochs tag the chunk status words.  1 is reserved for launches
+// captured into CUDA graphs (those zero the flags first, inside the graph).
+std::atomic<uint64_t> g_epoch{2};
+std::atomic<uint32_t> g_spin_limit{sgr::kSpinLimit};
+std::atomic<int64_t> g_drop_tile{-1};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Plan {
+    int esz = 4;          // bytes per stored element
+    bool vec = false;     // 128-bit path
+    int V = 1;            // channels per thread
+    int cg = 32;          // lanes across channels
+    int r = 2;            // rows per thread
+    int TR = 0, TC = 0;   // tile rows / channels
+    int64_t n_dt = 0, n_chains = 0, n_chunks = 0, n_tiles = 0;
+    size_t off_flags = 0, off_agg = 0, off_pref = 0, ws_bytes = 0;
+};
+
+bool mul_ok(int64_t a, int64_t b, int64_t *out) {
+    if (a < 0 || b < 0) return false;
+    if (a != 0 && b > std::numeric_limits<int64_t>::max() / a) return false;
+    *out = a * b;
+    return true;
+}
+
+// Chunk shape for a scan: vector width from dtype and alignment, CG lanes
+// across channels (8 => 128-byte row segments for fp32/bf16 rows), and the
+// largest rows-per-thread that still leaves >= kTargetTiles tiles.
+Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned) {
+    Plan p;
+    p.esz = (dtype == SGR_BF16) ? 2 : 4;
+    const int vw = 16 / p.esz;
+    p.vec = aligned && (D % vw == 0);
+    p.V = p.vec ? vw : 1;
+    int cg = p.vec ? 8 : 32;
+    const int ocg = g_override_cg.load();
+    if (p.vec && (ocg == 8 || ocg == 32)) cg = ocg;
+    p.cg = cg;
+    p.TC = p.cg * p.V;
+    const int J = 32 / p.cg;
+    p.n_dt = (D + p.TC - 1) / p.TC;
+    p.n_chains = B * p.n_dt;
+    // rows per thread: the automatic choice keeps a data thread within 72
+    // registers without spilling (16 elements of each operand), so three
+    // blocks fit per SM; the override may go up to 32 elements per operand
+    const int rmax_auto = p.vec ? (p.V >= 8 ? 2 : 4) : 8;
+    const int rmax = p.V >= 8 ? 4 : 8;
+    const int orr = g_override_r.load();
+    int r = 1;
+    if (orr == 1 || orr == 2 || orr == 4 || orr == 8) {
+        r = orr < rmax ? orr : rmax;
+    } else {
+        for (int cand : {8, 4, 2, 1}) {
+            if (cand > rmax_auto) continue;
+            const int64_t tr = int64_t(kWarps) * J * cand;
+            const int64_t chunks = (T + tr - 1) / tr;
+            if (p.n_chains * chunks >= kTargetTiles || cand == 1) { r = cand; break; }
+        }
+    }
+    p.r = r;
+    p.TR = kWarps * J * r;
+    p.n_chunks = (T + p.TR - 1) / p.TR;
+    p.n_tiles = p.n_chains * p.n_chunks;
+    if (p.n_chunks > 1) {
+        p.off_flags = kAlign;                                   // [0, 256): status word
+        p.off_agg = align_up(p.off_flags + 8 * size_t(p.n_tiles), kAlign);
+        p.off_pref = align_up(p.off_agg + 8 * size_t(p.n_tiles) * p.TC, kAlign);
+        p.ws_bytes = align_up(p.off_pref + 4 * size_t(p.n_tiles) * p.TC, kAlign);
+    }
+    return p;
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+// bytes spanned by B rows of D elements with a batch stride (stride 0 = one row)
+size_t rows_span(int64_t B, int64_t D, int64_t bs, int esz) {
+    if (B <= 0 || D <= 0) return 0;
+    return size_t((B - 1) * bs + D) * esz;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <class Op, typename IO, int V, int CG, int R>
+cudaError_t launch_scan(const ScanParams &sp, int64_t n_tiles, cudaStream_t s) {
+    if constexpr (R * V > 32) {
+        return cudaErrorInvalidConfiguration;   // never planned (see make_plan)
+    } else {
+        // registers a data thread keeps live: its tile (2RV), one pair per
+        // channel (2V) and about 24 for addressing; blocks of 288 threads
+        constexpr int NEED = 2 * R * V + 2 * V + 24;
+        constexpr int MINB = NEED <= 56 ? 4 : (NEED <= 72 ? 3 : 2);
+        scan_kernel<Op, IO, V, CG, R, kWarps, MINB>
+            <<<dim3(unsigned(n_tiles)), (kWarps + 1) * 32, 0, s>>>(sp);
+        return cudaGetLastError();
+    }
+}
+
+template <class Op, typename IO, int V, int CG>
+cudaError_t dispatch_r(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
+    switch (pl.r) {
+        case 1: return launch_scan<Op, IO, V, CG, 1>(sp, pl.n_tiles, s);
+        case 2: return launch_scan<Op, IO, V, CG, 2>(sp, pl.n_tiles, s);
+        case 4: return launch_scan<Op, IO, V, CG, 4>(sp, pl.n_tiles, s);
+        default: return launch_scan<Op, IO, V, CG, 8>(sp, pl.n_tiles, s);
+    }
+}
+
+template <class Op, typename IO>
+cudaError_t dispatch(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
+    constexpr int VW = 16 / int(sizeof(IO));
+    if (!pl.vec) return dispatch_r<Op, IO, 1, 32>(pl, sp, s);
+    if (pl.cg == 32) return dispatch_r<Op, IO, VW, 32>(pl, sp, s);
+    return dispatch_r<Op, IO, VW, 8>(pl, sp, s);
+}
+
+sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void *init,
+                      int64_t init_bs, void *out, int64_t B, int64_t T, int64_t D,
+                      sgr_dtype_t dtype, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
+    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return SGR_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || D < 0 || init_bs < 0) return SGR_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || D == 0) return SGR_OK;
+    if (!in0 || !in1 || !out) return SGR_ERR_INVALID_ARG;
+    const int esz = dtype == SGR_BF16 ? 2 : 4;
+    int64_t n = 0, nbytes = 0;
+    if (!mul_ok(B, T, &n) || !mul_ok(n, D, &n) || !mul_ok(n, esz, &nbytes)) return SGR_ERR_UNSUPPORTED;
+    int64_t init_span_elems = 0;
+    if (init && !mul_ok(B - 1, init_bs, &init_span_elems)) return SGR_ERR_UNSUPPORTED;
+    const size_t tb = size_t(nbytes);
+    const size_t ib = init ? rows_span(B, D, init_bs, esz) : 0;
+    if (overlaps(out, tb, in0, tb) || overlaps(out, tb, in1, tb) || overlaps(out, tb, init, ib))
+        return SGR_ERR_INVALID_ARG;
+
+    const bool aligned = aligned16(in0) && aligned16(in1) && aligned16(out);
+    const Plan pl = make_plan(B, T, D, dtype, aligned);
+    if (pl.n_tiles > int64_t(std::numeric_limits<int>::max())) return SGR_ERR_UNSUPPORTED;
+
+    ScanParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.in0 = in0; sp.in1 = in1; sp.init = init; sp.init_bs = init_bs; sp.out = out;
+    sp.B = B; sp.T = T; sp.D = D;
+    sp.n_dt = pl.n_dt; sp.n_chains = pl.n_chains; sp.n_chunks = pl.n_chunks;
+    sp.epoch = 0;
+    sp.spin_limit = g_spin_limit.load();
+    sp.drop_tile = g_drop_tile.load();
+    if (pl.n_chunks > 1) {
+        if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)) return SGR_ERR_WORKSPACE;
+        char *w = static_cast<char *>(ws);
+        sp.status = reinterpret_cast<uint32_t *>(w);
+        sp.flags = reinterpret_cast<uint64_t *>(w + pl.off_flags);
+        sp.agg = reinterpret_cast<float2 *>(w + pl.off_agg);
+        sp.pref = reinterpret_cast<float *>(w + pl.off_pref);
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return SGR_ERR_CUDA;
+        if (cs == cudaStreamCaptureStatusActive) {
+            // a graph replays its launch arguments: clear the flags inside the
+            // graph so the fixed epoch of captured launches never sees stale words
+            if (cudaMemsetAsync(sp.flags, 0, 8 * size_t(pl.n_tiles), stream) != cudaSuccess)
+                return SGR_ERR_CUDA;
+            sp.epoch = 1;
+        } else {
+            sp.epoch = g_epoch.fetch_add(1);
+        }
+    }
+    cudaError_t e;
+    if (op == SGR_OP_MINGRU) {
+        e = dtype == SGR_F32 ? dispatch<MinGRUOp, float>(pl, sp, stream)
+                             : dispatch<MinGRUOp, __nv_bfloat16>(pl, sp, stream);
+    } else {
+        e = dtype == SGR_F32 ? dispatch<MinMaxOp, float>(pl, sp, stream)
+                             : dispatch<MinMaxOp, __nv_bfloat16>(pl, sp, stream);
+    }
+    return e == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+sgr_status_t mingru_scan(const void *k, const void *hx, const void *h0, int64_t h0_batch_stride,
+                         void *h, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
+                         void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    return run_scan(SGR_OP_MINGRU, k, hx, h0, h0_batch_stride, h, B, T, D, dtype, workspace,
+                    ws_bytes, stream);
+}
+
+sgr_status_t minmax_scan(const void *r, const void *s, const void *x0, int64_t x0_batch_stride,
+                         void *x, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
+                         void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    return run_scan(SGR_OP_MINMAX, r, s, x0, x0_batch_stride, x, B, T, D, dtype, workspace,
+                    ws_bytes, stream);
+}
+
+sgr_status_t mingru_step(const void *k_t, int64_t k_bs, const void *hx_t, int64_t hx_bs,
+                         const void *h_prev, int64_t hp_bs, void *h_out, int64_t ho_bs,
+                         int64_t B, int64_t D, sgr_dtype_t dtype, cudaStream_t stream) {
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
+    if (B < 0 || D < 0 || k_bs < 0 || hx_bs < 0 || hp_bs < 0 || ho_bs < 0) return SGR_ERR_INVALID_ARG;
+    if (B == 0 || D == 0) return SGR_OK;
+    if (!k_t || !hx_t || !h_out) return SGR_ERR_INVALID_ARG;
+    if (B > 1 && ho_bs < D) return SGR_ERR_INVALID_ARG;   // output rows would overlap
+    const int esz = dtype == SGR_BF16 ? 2 : 4;
+    int64_t tmp = 0;
+    for (int64_t bs : {k_bs, hx_bs, hp_bs, ho_bs})
+        if (!mul_ok(B - 1, bs, &tmp) || !mul_ok(tmp + D, esz, &tmp)) return SGR_ERR_UNSUPPORTED;
+    const size_t ob = rows_span(B, D, ho_bs, esz);
+    if (overlaps(h_out, ob, k_t, rows_span(B, D, k_bs, esz)) ||
+        overlaps(h_out, ob, hx_t, rows_span(B, D, hx_bs, esz)))
+        return SGR_ERR_INVALID_ARG;
+    const bool in_place = (h_prev == h_out) && (hp_bs == ho_bs);
+    if (h_prev && !in_place && overlaps(h_out, ob, h_prev, rows_span(B, D, hp_bs, esz)))
+        return SGR_ERR_INVALID_ARG;
+    const int64_t n = B * D;
+    const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 16);
+    if (dtype == SGR_F32) {
+        mingru_step_kernel<float><<<unsigned(blocks), 256, 0, stream>>>(
+            static_cast<const float *>(k_t), k_bs, static_cast<const float *>(hx_t), hx_bs,
+            static_cast<const float *>(h_prev), hp_bs, static_cast<float *>(h_out), ho_bs, B, D);
+    } else {
+        mingru_step_kernel<__nv_bfloat16><<<unsigned(blocks), 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16 *>(k_t), k_bs,
+            static_cast<const __nv_bfloat16 *>(hx_t), hx_bs,
+            static_cast<const __nv_bfloat16 *>(h_prev), hp_bs,
+            static_cast<__nv_bfloat16 *>(h_out), ho_bs, B, D);
+    }
+    return cudaGetLastError() == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
+}
+
+size_t sgr_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype) {
+    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return 0;
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return 0;
+    if (B <= 0 || T <= 0 || D <= 0) return 0;
+    // the vector and the scalar variant may cut T differently: cover both
+    const Plan a = make_plan(B, T, D, dtype, true);
+    const Plan b = make_plan(B, T, D, dtype, false);
+    return a.ws_bytes > b.ws_bytes ? a.ws_bytes : b.ws_bytes;
+}
+
+sgr_status_t sgr_workspace_init(void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (ws_bytes == 0) return SGR_OK;
+    if (!workspace) return SGR_ERR_INVALID_ARG;
+    return cudaMemsetAsync(workspace, 0, ws_bytes, stream) == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
+}
+
+sgr_status_t sgr_workspace_status(void *workspace, size_t ws_bytes, int clear, cudaStream_t stream) {
+    if (!workspace || ws_bytes < sizeof(uint32_t)) return SGR_ERR_INVALID_ARG;
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return SGR_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return SGR_ERR_CUDA;
+    if (clear) {
+        if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), stream) != cudaSuccess) return SGR_ERR_CUDA;
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return SGR_ERR_CUDA;
+    }
+    return (word & sgr::kTimeoutBit) ? SGR_ERR_TIMEOUT : SGR_OK;
+}
+
+const char *sgr_status_string(sgr_status_t s) {
+    switch (s) {
+        case SGR_OK: return "ok";
+        case SGR_ERR_INVALID_ARG: return "invalid argument";
+        case SGR_ERR_UNSUPPORTED: return "unsupported size";
+        case SGR_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+        case SGR_ERR_CUDA: return "CUDA error";
+        case SGR_ERR_TIMEOUT: return "timed out waiting for an earlier chunk's state";
+    }
+    return "unknown status";
+}
+
+const char *sgr_version(void) { return "scan_gated_rnns_b200 0.1.0 sm_100a"; }
+
+sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
+                           int aligned, sgr_plan_t *plan) {
+    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return SGR_ERR_INVALID_ARG;
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || D < 0 || !plan) return SGR_ERR_INVALID_ARG;
+    const Plan p = make_plan(B, T, D, dtype, aligned != 0);
+    plan->vector_path = p.vec ? 1 : 0;
+    plan->channels_per_thread = p.V;
+    plan->channel_lanes = p.cg;
+    plan->rows_per_thread = p.r;
+    plan->warps = kWarps;
+    plan->threads = (kWarps + 1) * 32;
+    plan->tile_rows = p.TR;
+    plan->tile_channels = p.TC;
+    plan->n_channel_tiles = p.n_dt;
+    plan->n_chains = p.n_chains;
+    plan->n_chunks = p.n_chunks;
+    plan->n_tiles = p.n_tiles;
+    plan->workspace_bytes = p.ws_bytes;
+    plan->off_flags = p.off_flags;
+    plan->off_agg = p.off_agg;
+    plan->off_pref = p.off_pref;
+    return SGR_OK;
+}
+
+sgr_status_t sgr_set_wait_limit(uint32_t polls) {
+    g_spin_limit.store(polls == 0 ? sgr::kSpinLimit : polls);
+    return SGR_OK;
+}
+
+sgr_status_t sgr_set_drop_publish(int64_t tile) {
+    if (tile < -1) return SGR_ERR_INVALID_ARG;
+    g_drop_tile.store(tile);
+    return SGR_OK;
+}
+
+sgr_status_t sgr_set_tile_override(int channel_lanes, int rows_per_thread) {
+    if (!(channel_lanes == 0 || channel_lanes == 8 || channel_lanes == 32)) return SGR_ERR_INVALID_ARG;
+    if (!(rows_per_thread == 0 || rows_per_thread == 1 || rows_per_thread == 2 ||
+          rows_per_thread == 4 || rows_per_thread == 8))
+        return SGR_ERR_INVALID_ARG;
+    g_override_cg.store(channel_lanes);
+    g_override_r.store(rows_per_thread);
+    return SGR_OK;
+}
+
+}  // extern "C"

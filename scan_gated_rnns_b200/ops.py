@@ -1,0 +1,167 @@
+"""Torch-facing wrappers of the C ABI: argument marshalling only.
+
+Every operation runs in the CUDA library (``libsgr.so``).  These wrappers check
+shapes, dtypes and devices, allocate outputs and the workspace with PyTorch's
+allocator, pass raw device pointers and PyTorch's current stream, and turn a
+non-zero status into an exception.  There is no CPU path.
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from . import _abi
+from ._abi import check, lib
+
+_DT = {torch.float32: _abi.SGR_F32, torch.bfloat16: _abi.SGR_BF16}
+
+
+def _dtype_code(t: torch.Tensor, name: str) -> int:
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise TypeError(f"{name}: dtype {t.dtype} is not supported (float32 or bfloat16)") from None
+
+
+def _need_cuda(t: torch.Tensor, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the scans have no CPU path)")
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _seq(t: torch.Tensor, name: str) -> None:
+    _need_cuda(t, name)
+    if t.dim() != 3:
+        raise ValueError(f"{name} must be (B, T, D), got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (B, T, D)")
+
+
+def _rows(t: Optional[torch.Tensor], B: int, D: int, like: torch.Tensor, name: str) -> Tuple[int, int]:
+    """(pointer, batch stride in elements) of a (B, D) or (D,) operand."""
+    if t is None:
+        return 0, 0
+    _need_cuda(t, name)
+    if t.dtype != like.dtype or t.device != like.device:
+        raise ValueError(f"{name} must have dtype {like.dtype} on {like.device}")
+    if t.dim() == 1:
+        if t.shape[0] != D or (D > 1 and t.stride(0) != 1):
+            raise ValueError(f"{name} must be a contiguous (D,) vector")
+        return t.data_ptr(), 0
+    if t.dim() != 2 or tuple(t.shape) != (B, D):
+        raise ValueError(f"{name} must be (B, D) = ({B}, {D}), got {tuple(t.shape)}")
+    if D > 1 and t.stride(1) != 1:
+        raise ValueError(f"{name} rows must be contiguous along D")
+    return t.data_ptr(), (t.stride(0) if B > 1 else D)
+
+
+class Workspace:
+    """Device workspace of the chunked scans, zero-filled when allocated (the
+    library keeps it valid from call to call).  Use one per stream."""
+
+    def __init__(self, nbytes: int, device) -> None:
+        self.nbytes = max(int(nbytes), 256)
+        self.buf = torch.zeros(self.nbytes, dtype=torch.uint8, device=device)
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+    def status(self, clear: bool = True) -> int:
+        """Synchronise the current stream and return the device status word
+        (0 = ok, SGR_ERR_TIMEOUT if a chunk gave up waiting)."""
+        return lib().sgr_workspace_status(self.ptr, self.nbytes, int(clear), _stream(self.buf.device))
+
+
+_cache = {}
+
+
+def workspace_size(op: str, B: int, T: int, D: int, dtype: torch.dtype) -> int:
+    opc = {"mingru": _abi.SGR_OP_MINGRU, "minmax": _abi.SGR_OP_MINMAX}[op]
+    return int(lib().sgr_workspace_size(opc, B, T, D, _DT[dtype]))
+
+
+def default_workspace(device: torch.device, nbytes: int) -> Workspace:
+    """The per-(device, stream) workspace the wrappers use when none is given."""
+    key = (device.index, _stream(device))
+    ws = _cache.get(key)
+    if ws is None or ws.nbytes < nbytes:
+        ws = Workspace(nbytes, device)
+        _cache[key] = ws
+    return ws
+
+
+def _scan(fn: str, op: int, p: torch.Tensor, q: torch.Tensor, init, out, workspace):
+    _seq(p, fn + ": first operand")
+    _seq(q, fn + ": second operand")
+    if p.shape != q.shape or p.dtype != q.dtype or p.device != q.device:
+        raise ValueError(f"{fn}: operands must share shape, dtype and device")
+    dt = _dtype_code(p, fn)
+    B, T, D = p.shape
+    ip, ibs = _rows(init, B, D, p, fn + ": initial state")
+    if out is None:
+        out = torch.empty_like(p)
+    else:
+        _seq(out, fn + ": out")
+        if out.shape != p.shape or out.dtype != p.dtype or out.device != p.device:
+            raise ValueError(f"{fn}: out must match the operands")
+    need = int(lib().sgr_workspace_size(op, B, T, D, dt))
+    wp, wn = 0, 0
+    if need:
+        ws = workspace if workspace is not None else default_workspace(p.device, need)
+        wp, wn = ws.ptr, ws.nbytes
+    with torch.cuda.device(p.device):
+        code = getattr(lib(), fn)(p.data_ptr(), q.data_ptr(), ip, ibs, out.data_ptr(),
+                                  B, T, D, dt, wp, wn, _stream(p.device))
+    check(fn, code)
+    return out
+
+
+def mingru_scan(k: torch.Tensor, hx: torch.Tensor, h0: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, workspace: Optional[Workspace] = None) -> torch.Tensor:
+    """h (B, T, D): minGRU over the time axis of pre-activations k, hx (B, T, D),
+    with optional initial state h0 (B, D) or (D,)."""
+    return _scan("mingru_scan", _abi.SGR_OP_MINGRU, k, hx, h0, out, workspace)
+
+
+def minmax_scan(r: torch.Tensor, s: torch.Tensor, x0: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, workspace: Optional[Workspace] = None) -> torch.Tensor:
+    """x (B, T, D), x[:, t] = x_{t+1} = max(min(r_t, x_t), s_t), x_0 = x0 or +0."""
+    return _scan("minmax_scan", _abi.SGR_OP_MINMAX, r, s, x0, out, workspace)
+
+
+def mingru_step(k_t: torch.Tensor, hx_t: torch.Tensor, h_prev: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One token: (B, D) rows in (any batch stride, contiguous along D), new
+    state (B, D) out.  ``out`` may be ``h_prev`` for an in-place update."""
+    for t, n in ((k_t, "k_t"), (hx_t, "hx_t")):
+        _need_cuda(t, n)
+        if t.dim() != 2:
+            raise ValueError(f"mingru_step: {n} must be (B, D)")
+    if k_t.shape != hx_t.shape or k_t.dtype != hx_t.dtype or k_t.device != hx_t.device:
+        raise ValueError("mingru_step: k_t and hx_t must share shape, dtype and device")
+    dt = _dtype_code(k_t, "mingru_step")
+    B, D = k_t.shape
+    kp, kbs = _rows(k_t, B, D, k_t, "k_t")
+    hp, hbs = _rows(hx_t, B, D, k_t, "hx_t")
+    pp, pbs = _rows(h_prev, B, D, k_t, "h_prev")
+    if out is None:
+        out = torch.empty((B, D), dtype=k_t.dtype, device=k_t.device)
+    op, obs = _rows(out, B, D, k_t, "out")
+    with torch.cuda.device(k_t.device):
+        code = lib().mingru_step(kp, kbs, hp, hbs, pp, pbs, op, obs, B, D, dt, _stream(k_t.device))
+    check("mingru_step", code)
+    return out
+
+
+def set_tile_override(channel_lanes: int = 0, rows_per_thread: int = 0) -> None:
+    """Force the chunk shape of the scans (0, 0 restores the automatic choice)."""
+    check("sgr_set_tile_override", lib().sgr_set_tile_override(channel_lanes, rows_per_thread))
+
+
+def version() -> str:
+    return lib().sgr_version().decode()

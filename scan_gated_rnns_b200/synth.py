@@ -2,12 +2,16 @@
 
 This module is shared by the tests, the benchmark and the smoke check, and
 feeds both the CUDA library and the CPU oracle.  It holds none of the scans'
-arithmetic: it only draws random numbers on the CPU with a seeded
-``torch.Generator`` and rounds them to the I/O dtype.
+arithmetic: it only draws random numbers with a seeded ``torch.Generator``
+and rounds them to the I/O dtype.
 
 Draw order per workload: first operand (k or r), second operand (hx or s),
 then the optional initial state.  bf16 inputs are fp32 draws rounded to
 nearest-even by ``Tensor.to``; the identical bits go to the GPU and the oracle.
+Draws are made on the device asked for (a CPU or a CUDA ``torch.Generator``
+seeded the same way); the two devices give different numbers for one seed,
+so a run that checks GPU results copies the GPU-drawn inputs to the host for
+the oracle rather than drawing them twice.
 
 The named workloads are the shapes and distributions of the minGRU layer
 example on the page "Mingru Pytorch" (batched (B, T, D) tensors such as
@@ -74,24 +78,25 @@ WORKLOADS = {
 BENCH_WORKLOAD = "mingru_b8_t4096_d1024_f32_h0"
 
 
-def generate(w: Workload, seed: Optional[int] = None):
-    """Return (p, q, init) CPU tensors in the workload's I/O dtype.
+def generate(w: Workload, seed: Optional[int] = None, device="cpu"):
+    """Return (p, q, init) tensors on `device` in the workload's I/O dtype.
 
     p, q are (B, T, D): (k, hx) for minGRU with k ~ N(k_mean, 1), hx ~ N(0, 1);
     (r, s) for MinMax with r, s ~ N(0, 1).  init is (B, D) or None.
     """
-    g = torch.Generator(device="cpu")
+    device = torch.device(device)
+    g = torch.Generator(device=device)
     g.manual_seed(w.seed if seed is None else seed)
     shape = (w.B, w.T, w.D)
-    p = torch.randn(shape, generator=g, dtype=torch.float32)
+    p = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
     if w.k_mean:
         p += w.k_mean
-    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    q = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
     init = None
     if w.init == "u01_1":
-        init = torch.rand((w.B, w.D), generator=g, dtype=torch.float32) * 0.9 + 0.1
+        init = torch.rand((w.B, w.D), generator=g, dtype=torch.float32, device=device) * 0.9 + 0.1
     elif w.init == "zero":
-        init = torch.zeros((w.B, w.D), dtype=torch.float32)
+        init = torch.zeros((w.B, w.D), dtype=torch.float32, device=device)
     dt = _DTYPES[w.dtype]
     p, q = p.to(dt), q.to(dt)
     if init is not None:

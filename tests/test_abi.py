@@ -1,0 +1,193 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+- the library loads and exports every function include/scan_gated_rnns.h declares;
+- argument errors are reported before anything is enqueued;
+- the tile plan's index arithmetic, replayed here for every block and thread of
+  the benchmark and parity shapes, stays inside the buffers it addresses and
+  covers every output element exactly once.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from scan_gated_rnns_b200 import _abi
+from scan_gated_rnns_b200.synth import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "scan_gated_rnns.h")
+
+F32, BF16 = _abi.SGR_F32, _abi.SGR_BF16
+MINGRU, MINMAX = _abi.SGR_OP_MINGRU, _abi.SGR_OP_MINMAX
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^SGR_API\s+[\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_three_operations():
+    names = declared_functions()
+    for n in ("mingru_scan", "mingru_step", "minmax_scan"):
+        assert n in names
+
+
+def test_every_declared_function_is_exported_and_typed():
+    lib = _abi.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _abi.SIGNATURES, f"{name} has no ctypes signature"
+
+
+def test_version_and_status_strings():
+    assert "sm_100a" in _abi.lib().sgr_version().decode()
+    for code in range(6):
+        assert _abi.status_string(code)
+    assert _abi.status_string(99) == "unknown status"
+
+
+# ----------------------------------------------------- argument validation
+# Fake device addresses: validation must reject these calls before touching CUDA.
+A, Bp, C = 0x10000000, 0x20000000, 0x30000000
+
+
+def scan(fn, *args):
+    return getattr(_abi.lib(), fn)(*args)
+
+
+@pytest.mark.parametrize("fn", ["mingru_scan", "minmax_scan"])
+def test_scan_argument_errors(fn):
+    E = _abi.SGR_ERR_INVALID_ARG
+    # negative sizes / strides, unknown dtype
+    assert scan(fn, A, Bp, None, 0, C, -1, 4, 4, F32, None, 0, None) == E
+    assert scan(fn, A, Bp, None, 0, C, 1, -4, 4, F32, None, 0, None) == E
+    assert scan(fn, A, Bp, 0x40000000, -1, C, 1, 4, 4, F32, None, 0, None) == E
+    assert scan(fn, A, Bp, None, 0, C, 1, 4, 4, 7, None, 0, None) == E
+    # null operands with data to move
+    assert scan(fn, None, Bp, None, 0, C, 1, 4, 4, F32, None, 0, None) == E
+    assert scan(fn, A, None, None, 0, C, 1, 4, 4, F32, None, 0, None) == E
+    assert scan(fn, A, Bp, None, 0, None, 1, 4, 4, F32, None, 0, None) == E
+    # output overlapping an input
+    assert scan(fn, A, Bp, None, 0, A + 16, 1, 4, 4, F32, None, 0, None) == E
+    assert scan(fn, A, Bp, C + 8, 4, C, 1, 4, 4, F32, None, 0, None) == E
+    # empty shapes are no-ops, even with null pointers
+    for shp in [(0, 4, 4), (2, 0, 4), (2, 4, 0)]:
+        assert scan(fn, None, None, None, 0, None, *shp, F32, None, 0, None) == _abi.SGR_OK
+    # a long sequence needs a workspace
+    assert scan(fn, A, Bp, None, 0, C, 1, 1 << 16, 64, F32, None, 0, None) == _abi.SGR_ERR_WORKSPACE
+    need = _abi.plan(MINGRU, 1, 1 << 16, 64, F32, True)["workspace_bytes"]
+    assert 0 < need <= _abi.lib().sgr_workspace_size(MINGRU, 1, 1 << 16, 64, F32)
+    assert scan(fn, A, Bp, None, 0, C, 1, 1 << 16, 64, F32, 0x50000000, need - 1, None) \
+        == _abi.SGR_ERR_WORKSPACE
+    assert scan(fn, A, Bp, None, 0, C, 1, 1 << 16, 64, F32, 0x50000008, need, None) \
+        == _abi.SGR_ERR_WORKSPACE   # misaligned
+    # byte counts that overflow int64
+    assert scan(fn, A, Bp, None, 0, C, 1 << 40, 1 << 20, 1 << 10, F32, None, 0, None) \
+        == _abi.SGR_ERR_UNSUPPORTED
+
+
+def test_step_argument_errors():
+    lib = _abi.lib()
+    E = _abi.SGR_ERR_INVALID_ARG
+    assert lib.mingru_step(A, 8, Bp, 8, None, 0, C, 8, 2, 8, 5, None) == E          # dtype
+    assert lib.mingru_step(A, 8, Bp, 8, None, 0, C, 4, 2, 8, F32, None) == E        # out rows overlap
+    assert lib.mingru_step(A, -8, Bp, 8, None, 0, C, 8, 2, 8, F32, None) == E       # stride
+    assert lib.mingru_step(None, 8, Bp, 8, None, 0, C, 8, 2, 8, F32, None) == E
+    assert lib.mingru_step(A, 8, Bp, 8, None, 0, A + 4, 8, 2, 8, F32, None) == E    # out on k
+    assert lib.mingru_step(A, 8, Bp, 8, C + 4, 8, C, 8, 2, 8, F32, None) == E       # partial overlap
+    assert lib.mingru_step(A, 8, Bp, 8, None, 0, C, 8, 0, 8, F32, None) == _abi.SGR_OK
+
+
+def test_workspace_size_and_hooks():
+    lib = _abi.lib()
+    assert lib.sgr_workspace_size(MINGRU, 2, 1, 512, F32) == 0      # one chunk
+    assert lib.sgr_workspace_size(9, 2, 4096, 512, F32) == 0
+    assert lib.sgr_workspace_size(MINGRU, 8, 4096, 1024, F32) > 0
+    assert lib.sgr_set_tile_override(3, 0) == _abi.SGR_ERR_INVALID_ARG
+    assert lib.sgr_set_tile_override(0, 3) == _abi.SGR_ERR_INVALID_ARG
+    assert lib.sgr_set_drop_publish(-2) == _abi.SGR_ERR_INVALID_ARG
+    assert lib.sgr_set_wait_limit(0) == _abi.SGR_OK
+    assert lib.sgr_set_drop_publish(-1) == _abi.SGR_OK
+    assert lib.sgr_workspace_init(None, 0, None) == _abi.SGR_OK
+    assert lib.sgr_workspace_init(None, 64, None) == _abi.SGR_ERR_INVALID_ARG
+    assert lib.sgr_workspace_status(None, 64, 0, None) == _abi.SGR_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------- index arithmetic
+# The kernel's address formulas, replayed for every block and thread.
+
+def check_plan_indices(B, T, D, dtype, aligned, check_cover):
+    pl = _abi.plan(MINGRU, B, T, D, dtype, aligned)
+    esz = 4 if dtype == F32 else 2
+    V, cg, R, W = pl["channels_per_thread"], pl["channel_lanes"], pl["rows_per_thread"], pl["warps"]
+    J = 32 // cg
+    TR, TC = pl["tile_rows"], pl["tile_channels"]
+    n_dt, n_chains, n_chunks, n_tiles = pl["n_channel_tiles"], pl["n_chains"], pl["n_chunks"], pl["n_tiles"]
+    assert TR == W * J * R and TC == cg * V and TC % 32 == 0
+    assert n_dt == -(-D // TC) and n_chains == B * n_dt and n_chunks == -(-T // TR)
+    assert n_tiles == n_chains * n_chunks and n_tiles < 2 ** 31
+    if pl["vector_path"]:
+        assert aligned and D % V == 0 and V * esz == 16
+    tile = np.arange(n_tiles, dtype=np.int64)[:, None, None]
+    warp = np.arange(W, dtype=np.int64)[None, :, None]
+    lane = np.arange(32, dtype=np.int64)[None, None, :]
+    chain, c = tile % n_chains, tile // n_chains
+    b, dt = chain // n_dt, chain % n_dt
+    g, j = lane % cg, lane // cg
+    d0 = dt * TC + g * V
+    row0 = c * TR + (warp * J + j) * R
+    N = B * T * D
+    cover = np.zeros(N, dtype=np.int32) if check_cover else None
+    for r in range(R):
+        t = row0 + r
+        valid = (d0 < D) & (t < T)
+        idx = ((b * T + t) * D + d0)[np.broadcast_to(valid, np.broadcast_shapes(valid.shape, d0.shape))]
+        if idx.size:
+            assert idx.min() >= 0 and idx.max() + V <= N
+            dv = np.broadcast_to(d0, valid.shape)[valid]
+            assert (dv + V <= D).all()
+            if pl["vector_path"]:
+                assert ((idx * esz) % 16 == 0).all()
+            if check_cover:
+                for v in range(V):
+                    np.add.at(cover, idx + v, 1)
+    if check_cover:
+        assert (cover == 1).all(), "every output element is written exactly once"
+    # carry warp: channel slots, flags and summaries inside their regions
+    CV = TC // 32
+    assert (np.arange(32) * CV + CV - 1 < TC).all()
+    if n_chunks > 1:
+        assert pl["off_flags"] >= 4
+        assert pl["off_flags"] + 8 * n_tiles <= pl["off_agg"]
+        assert pl["off_agg"] + 8 * n_tiles * TC <= pl["off_pref"]
+        assert pl["off_pref"] + 4 * n_tiles * TC <= pl["workspace_bytes"]
+        assert pl["off_agg"] % 16 == 0 and pl["off_pref"] % 16 == 0 and pl["off_flags"] % 8 == 0
+        assert _abi.lib().sgr_workspace_size(MINGRU, B, T, D, dtype) >= pl["workspace_bytes"]
+    else:
+        assert pl["workspace_bytes"] == 0
+
+
+SMALL_SHAPES = [(2, 1024, 512), (3, 1000, 96), (1, 777, 36), (2, 300, 7), (1, 1, 1), (5, 1, 64),
+                (1, 4097, 32), (2, 129, 40), (4, 63, 8), (1, 2000, 1)]
+
+
+@pytest.mark.parametrize("shape", SMALL_SHAPES)
+@pytest.mark.parametrize("dtype", [F32, BF16])
+@pytest.mark.parametrize("aligned", [True, False])
+@pytest.mark.parametrize("override", [(0, 0), (8, 1), (8, 8), (32, 2), (32, 4)])
+def test_plan_indices_small(shape, dtype, aligned, override):
+    lib = _abi.lib()
+    assert lib.sgr_set_tile_override(*override) == 0
+    try:
+        check_plan_indices(*shape, dtype, aligned, check_cover=True)
+    finally:
+        lib.sgr_set_tile_override(0, 0)
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_plan_indices_workloads(name):
+    w = WORKLOADS[name]
+    check_plan_indices(w.B, w.T, w.D, F32 if w.dtype == "f32" else BF16, True, check_cover=False)

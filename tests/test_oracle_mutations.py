@@ -27,25 +27,24 @@ MUTANTS = {
     "g_offset_sign": ("return (x >= 0.0) ? x + 0.5 : sigmoid(x);",
                       "return (x >= 0.0) ? x - 0.5 : sigmoid(x);"),
     "sigmoid_sign": ("return 1.0 / (1.0 + exp(-x));", "return 1.0 / (1.0 + exp(x));"),
-    "h0_dropped": ("double state = h0 ? h0[b * h0_bs + d] : 0.0;\n            for (int64_t t = 0; t < T; ++t) {\n                int64_t i = (b * T + t) * D + d;\n                double z",
-                   "double state = 0.0;\n            for (int64_t t = 0; t < T; ++t) {\n                int64_t i = (b * T + t) * D + d;\n                double z"),
-    "output_before_update": ("state = one_minus_z * state + z * g_act(hx[i]);\n                h[i] = state;",
-                             "h[i] = state;\n                state = one_minus_z * state + z * g_act(hx[i]);"),
+    "h0_dropped": ("prev = h0 ? h0[b * h0_bs + d] : 0.0;", "prev = 0.0;"),
+    "state_from_wrong_row": ("prev = h[i - D];", "prev = h[i - 1 < 0 ? 0 : i - 1];"),
+    "output_shifted_by_one": ("h[i] = one_minus_z * prev + z * g_act(hx[i]);",
+                              "h[i] = prev; (void)(one_minus_z * prev + z * g_act(hx[i]));"),
     # minGRU, log space
-    "log_astar_sign": ("a_star += -softplus(k[i]);", "a_star += softplus(k[i]);"),
+    "log_astar_sign": ("a_star[d] += -softplus(k[i]);", "a_star[d] += softplus(k[i]);"),
     "log_z_sign": ("double log_z = -softplus(-k[i]);", "double log_z = -softplus(k[i]);"),
-    "log_h0_term_dropped": ("m = log(h0[b * h0_bs + d]);\n                acc = 1.0;",
-                            "m = -INFINITY;\n                acc = 0.0;"),
+    "log_h0_term_dropped": ("m[d] = log(h0[b * h0_bs + d]);\n                acc[d] = 1.0;",
+                            "m[d] = -INFINITY;\n                acc[d] = 0.0;"),
     "log_candidate_branch": ("(x >= 0.0) ? log(x + 0.5) : -softplus(-x);",
                              "(x >= 0.0) ? log(x + 0.5) : -softplus(x);"),
-    "log_lse_update": ("acc = acc * exp(m - v) + 1.0;", "acc = acc + 1.0;"),
+    "log_lse_update": ("acc[d] = acc[d] * exp(m[d] - v) + 1.0;", "acc[d] = acc[d] + 1.0;"),
     # MinMax
-    "minmax_min_max_swapped": ("state = fmax(fmin(r[i], state), s[i]);",
-                               "state = fmin(fmax(r[i], state), s[i]);"),
-    "minmax_r_s_swapped": ("state = fmax(fmin(r[i], state), s[i]);",
-                           "state = fmax(fmin(s[i], state), r[i]);"),
-    "minmax_x0_dropped": ("double state = x0 ? x0[b * x0_bs + d] : 0.0;",
-                          "double state = 0.0;"),
+    "minmax_min_max_swapped": ("x[i] = fmax(fmin(r[i], state), s[i]);",
+                               "x[i] = fmin(fmax(r[i], state), s[i]);"),
+    "minmax_r_s_swapped": ("x[i] = fmax(fmin(r[i], state), s[i]);",
+                           "x[i] = fmax(fmin(s[i], state), r[i]);"),
+    "minmax_x0_dropped": ("state = x0 ? x0[b * x0_bs + d] : 0.0;", "state = 0.0;"),
 }
 
 
