@@ -172,32 +172,45 @@ SGR_API const char *sgr_version(void);
 
 /*
  * Tuning/testing knob, process-wide: force the chunk shape the scans use.
- * channel_lanes in {8, 32} lanes across D per warp (0: automatic), rows_per_thread
- * in {1, 2, 4, 8} (0: automatic; bf16 vector tiles cap it at 4).  Shapes the
- * fast path cannot take fall back to automatic choices.  The chunk shape
- * changes the workspace size: query sgr_workspace_size after changing it.
- * Returns SGR_ERR_INVALID_ARG for other values.
+ * rows_per_thread: tile kernel {1, 2, 4, 8} (bf16 vector tiles cap it at 4),
+ * pipelined kernel {2, 4}; 0 or a value a kernel does not take means
+ * automatic.  channel_lanes is accepted for compatibility (0, 8 or 32) and
+ * ignored: the lane layout follows from the kernel and the alignment.  The
+ * chunk shape changes the workspace size: query sgr_workspace_size after
+ * changing it.  Returns SGR_ERR_INVALID_ARG for other values.
  */
 SGR_API sgr_status_t sgr_set_tile_override(int channel_lanes, int rows_per_thread);
+
+/*
+ * Tuning/testing knob, process-wide: 0 automatic (pipelined kernel for
+ * aligned vector-width rows, tile kernel otherwise), 1 force the tile kernel,
+ * 2 pipelined wherever the fast path applies.
+ */
+SGR_API sgr_status_t sgr_set_kernel_override(int kernel);
 
 /* ------------------------------------------------------- introspection */
 
 /* How a scan of this shape is cut into tiles (rows x channels per block). */
 typedef struct sgr_plan {
-    int32_t vector_path;        /* 1: 128-bit loads; 0: scalar variant         */
+    int32_t vector_path;        /* 1: 128-bit loads; 0: scalar variant            */
+    int32_t kernel;             /* 1: one block per tile; 2: pipelined persistent  */
     int32_t channels_per_thread;
-    int32_t channel_lanes;      /* lanes across D per warp                      */
+    int32_t channel_lanes;      /* lanes across D per warp                         */
     int32_t rows_per_thread;
-    int32_t warps;              /* data warps per block (plus one carry warp)   */
-    int32_t threads;            /* threads per block                            */
-    int64_t tile_rows;          /* rows of T per block                          */
-    int64_t tile_channels;      /* channels of D per block                      */
-    int64_t n_channel_tiles;    /* per batch row                                */
-    int64_t n_chains;           /* B * n_channel_tiles                          */
-    int64_t n_chunks;           /* tiles along T                                */
-    int64_t n_tiles;            /* blocks launched                              */
-    uint64_t workspace_bytes;   /* 0 when n_chunks == 1                         */
-    uint64_t off_flags, off_agg, off_pref;  /* workspace layout (bytes)         */
+    int32_t warps;              /* data warps per block (plus one carry warp)      */
+    int32_t threads;            /* threads per block                               */
+    int32_t stages;             /* pipelined: tiles in flight per block            */
+    int64_t tile_rows;          /* rows of T per tile                              */
+    int64_t tile_channels;      /* channels of D per tile                          */
+    int64_t n_channel_tiles;    /* per batch row                                   */
+    int64_t n_chains;           /* B * n_channel_tiles                             */
+    int64_t n_chunks;           /* tiles along T                                   */
+    int64_t n_tiles;            /* n_chains * n_chunks                             */
+    uint64_t smem_bytes;        /* dynamic shared memory per block                 */
+    uint64_t workspace_bytes;   /* 0 when n_chunks == 1                            */
+    uint64_t off_words;         /* workspace offset of the hand-off words          */
+    uint32_t div_chains_m, div_chains_s;  /* tile -> chunk division constants   */
+    uint32_t div_dt_m, div_dt_s;          /* chain -> batch division constants  */
 } sgr_plan_t;
 
 /* Fill *plan for a scan; `aligned` says whether the operands would be 16-byte

@@ -10,7 +10,7 @@ it.  Build the library with ``python -m scan_gated_rnns_b200.build``.
 """
 from ._abi import ScanError
 from .ops import (Workspace, default_workspace, mingru_scan, mingru_step, minmax_scan,
-                  set_tile_override, version, workspace_size)
+                  set_kernel_override, set_tile_override, version, workspace_size)
 
 __all__ = ["ScanError", "Workspace", "default_workspace", "mingru_scan", "mingru_step",
-           "minmax_scan", "set_tile_override", "version", "workspace_size"]
+           "minmax_scan", "set_kernel_override", "set_tile_override", "version", "workspace_size"]

@@ -45,14 +45,17 @@ SIGNATURES = {
 
 
 class Plan(ctypes.Structure):
-    _fields_ = [("vector_path", ctypes.c_int32), ("channels_per_thread", ctypes.c_int32),
-                ("channel_lanes", ctypes.c_int32), ("rows_per_thread", ctypes.c_int32),
-                ("warps", ctypes.c_int32), ("threads", ctypes.c_int32),
+    _fields_ = [("vector_path", ctypes.c_int32), ("kernel", ctypes.c_int32),
+                ("channels_per_thread", ctypes.c_int32), ("channel_lanes", ctypes.c_int32),
+                ("rows_per_thread", ctypes.c_int32), ("warps", ctypes.c_int32),
+                ("threads", ctypes.c_int32), ("stages", ctypes.c_int32),
                 ("tile_rows", ctypes.c_int64), ("tile_channels", ctypes.c_int64),
                 ("n_channel_tiles", ctypes.c_int64), ("n_chains", ctypes.c_int64),
                 ("n_chunks", ctypes.c_int64), ("n_tiles", ctypes.c_int64),
-                ("workspace_bytes", ctypes.c_uint64), ("off_flags", ctypes.c_uint64),
-                ("off_agg", ctypes.c_uint64), ("off_pref", ctypes.c_uint64)]
+                ("smem_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
+                ("off_words", ctypes.c_uint64),
+                ("div_chains_m", ctypes.c_uint32), ("div_chains_s", ctypes.c_uint32),
+                ("div_dt_m", ctypes.c_uint32), ("div_dt_s", ctypes.c_uint32)]
 
     def as_dict(self):
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -62,7 +65,11 @@ SIGNATURES.update({
     "sgr_scan_plan": (_int, [_int, _i64, _i64, _i64, _int, _int, ctypes.POINTER(Plan)]),
     "sgr_set_wait_limit": (_int, [ctypes.c_uint32]),
     "sgr_set_drop_publish": (_int, [_i64]),
+    "sgr_set_kernel_override": (_int, [_int]),
 })
+
+KERNEL_TILE = 1
+KERNEL_PIPELINED = 2
 
 _lock = threading.Lock()
 _lib = None

@@ -43,6 +43,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 namespace sgr {
 
 // ------------------------------------------------------------- operators
@@ -60,21 +62,23 @@ struct MinGRUOp {
     static __device__ __forceinline__ float pad0() { return -INFINITY; }
     static __device__ __forceinline__ float pad1() { return 0.f; }
     // fused activations: (k, hx) -> (a, b) = (sigmoid(-k), sigmoid(k) * g(hx)).
-    // Both sigmoids come from e = exp(-|x|) in (0, 1]: sigmoid(|x|) = 1/(1+e),
-    // sigmoid(-|x|) = e/(1+e); the two reciprocals share one division.
+    // With e = exp(-|x|) in [0, 1]: sigmoid(-|x|) = e/(1+e) =: s <= 1/2 and
+    // sigmoid(|x|) = 1 - s (no cancellation since s <= 1/2; exactly 1 - 0 = 1
+    // when e underflows, so k = -inf gives a = 1 and k = +inf gives z = 1).
+    // The two reciprocals 1/(1+ek), 1/(1+eh) share one division:
+    // inv = 1/((1+ek)(1+eh)).  MUFU work: 2 exp2 + 1 reciprocal.
     static __device__ __forceinline__ void element(float k, float hx, float &a, float &b) {
         const float ek = __expf(-fabsf(k));
         const float eh = __expf(-fabsf(hx));
         const float dk = 1.f + ek;
         const float dh = 1.f + eh;
-        const float inv = __frcp_rn(dk * dh);
-        const float rk = dh * inv;   // 1 / (1 + ek)
-        const float rh = dk * inv;   // 1 / (1 + eh)
-        const float ekr = ek * rk;
+        const float inv = __fdividef(1.f, dk * dh);
+        const float sk = ek * (dh * inv);    // sigmoid(-|k|)
+        const float kbig = 1.f - sk;          // sigmoid(|k|)
         const bool kpos = k >= 0.f;
-        const float z = kpos ? rk : ekr;
-        a = kpos ? ekr : rk;
-        const float g = (hx >= 0.f) ? hx + 0.5f : eh * rh;
+        const float z = kpos ? kbig : sk;
+        a = kpos ? sk : kbig;
+        const float g = (hx >= 0.f) ? hx + 0.5f : eh * (dk * inv);
         b = z * g;
     }
     // one step of phase 3
@@ -139,6 +143,22 @@ template <> struct Access<__nv_bfloat16, 8> {
     }
 };
 
+template <> struct Access<__nv_bfloat16, 4> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&x)[4]) {
+        const uint2 t = __ldcs(reinterpret_cast<const uint2 *>(p));
+        x[0] = __uint_as_float(t.x << 16);
+        x[1] = __uint_as_float(t.x & 0xffff0000u);
+        x[2] = __uint_as_float(t.y << 16);
+        x[3] = __uint_as_float(t.y & 0xffff0000u);
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&x)[4]) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(x[0], x[1]);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(x[2], x[3]);
+        __stcs(reinterpret_cast<uint2 *>(p),
+               make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi)));
+    }
+};
+
 template <> struct Access<__nv_bfloat16, 1> {
     static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&x)[1]) {
         const unsigned short u = __ldcs(reinterpret_cast<const unsigned short *>(p));
@@ -158,26 +178,64 @@ template <> __device__ __forceinline__ float load_scalar<__nv_bfloat16>(const __
     return __bfloat162float(*p);
 }
 
-// ------------------------------------------------------- look-back plumbing
 
-__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t *p) {
+// One vector of V elements from shared memory, widened to fp32.
+template <typename IO, int V> struct VecOf;
+template <> struct VecOf<float, 4> { using type = uint4; };
+template <> struct VecOf<__nv_bfloat16, 4> { using type = uint2; };
+
+__device__ __forceinline__ void unpack(const uint4 &t, float (&x)[4]) {
+    x[0] = __uint_as_float(t.x); x[1] = __uint_as_float(t.y);
+    x[2] = __uint_as_float(t.z); x[3] = __uint_as_float(t.w);
+}
+__device__ __forceinline__ void unpack(const uint2 &t, float (&x)[4]) {   // 4 x bf16
+    x[0] = __uint_as_float(t.x << 16);
+    x[1] = __uint_as_float(t.x & 0xffff0000u);
+    x[2] = __uint_as_float(t.y << 16);
+    x[3] = __uint_as_float(t.y & 0xffff0000u);
+}
+
+// ------------------------------------------------------- chunk hand-off
+//
+// Each chunk (tile) publishes, per channel, three 64-bit words in the
+// workspace: its summary pair (A, B) and, once known, its final state S.
+// Every word carries the launch epoch in its high half next to the fp32 value
+// in its low half, and is written and read as one 64-bit access, so a reader
+// sees either the whole current word or a stale one with another epoch.
+// No flag, no fence and no second round trip is needed: a word is valid
+// exactly when its epoch matches.  Layout: words[(tile * 3 + kind) * TC + ch],
+// kind 0 = A, 1 = B, 2 = S.
+
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t *p) {
     uint64_t v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 
-__device__ __forceinline__ void st_release_u64(uint64_t *p, uint64_t v) {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+__device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// Chunk status word: (epoch << 2) | state.  The epoch is new for every launch,
-// so words left by earlier launches read as "not ready".
-enum : uint32_t { ST_NONE = 0, ST_AGG = 1, ST_PREFIX = 2 };
+__device__ __forceinline__ uint64_t pack_word(uint32_t epoch, float v) {
+    return (uint64_t(epoch) << 32) | uint64_t(__float_as_uint(v));
+}
+__device__ __forceinline__ bool word_valid(uint64_t w, uint32_t epoch) { return uint32_t(w >> 32) == epoch; }
+__device__ __forceinline__ float word_value(uint64_t w) { return __uint_as_float(uint32_t(w)); }
 
 // bounded waiting: 2^18 polls with back-off capped at 1 us => a fraction of a
 // second, far above the microseconds a chunk waits for a running predecessor
 constexpr uint32_t kSpinLimit = 1u << 18;
 constexpr uint32_t kTimeoutBit = 1u;
+
+// Division by a divisor fixed at launch, for values below 2^31: the
+// multiply-high / add / shift form of division by invariant integers
+// (Granlund and Montgomery, 1994), round-up variant.  The host picks
+// s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1; then
+// n / d = (umulhi(n, m) + n) >> s for every n < 2^31 (the sum fits 32 bits).
+struct FastDiv {
+    uint32_t d, m, s;
+    __device__ __forceinline__ uint32_t div(uint32_t n) const { return (__umulhi(n, m) + n) >> s; }
+};
 
 struct ScanParams {
     const void *in0;      // k or r, (B, T, D)
@@ -189,39 +247,205 @@ struct ScanParams {
     int64_t n_dt;         // channel tiles per batch row
     int64_t n_chains;     // B * n_dt
     int64_t n_chunks;     // chunks along T
-    uint64_t *flags;      // [n_chunks * n_chains] status words (workspace)
-    float2 *agg;          // [n_chunks * n_chains * TC] chunk summaries
-    float *pref;          // [n_chunks * n_chains * TC] state at the end of each chunk
+    int64_t n_tiles;      // n_chains * n_chunks (< 2^31)
+    FastDiv by_chains;    // tile  -> (chunk, chain)
+    FastDiv by_dt;        // chain -> (b, dt)
+    uint64_t *words;      // [n_tiles][3][TC] hand-off words (workspace)
     uint32_t *status;     // device status word
-    uint64_t epoch;
+    uint32_t epoch;
     uint32_t spin_limit;  // polls before a chunk gives up waiting
     int64_t drop_tile;    // testing: this tile does not publish (-1: none)
 };
 
-// ----------------------------------------------------------------- kernel
-//
-// Template parameters: Op (operator), IO (storage type), V (channels per thread,
-// one 16-byte vector or 1), CG (lanes across channels), R (rows per thread),
-// W (data warps).  J = 32 / CG row groups per warp.  Tile = TR x TC with
-// TR = W * J * R rows and TC = CG * V channels.
-//
-// The block has W data warps and one carry warp.  Data warps hold the tile in
-// registers; the carry warp holds none and does the cross-chunk work (publish
-// the chunk summary, look back, publish the chunk's final state).  The two
-// roles sit in disjoint branches that meet only at named barriers, so their
-// register live ranges never add up.
-//
-// Tiles are numbered chain-fastest: blockIdx.x = chunk * n_chains + chain,
-// chain = b * n_dt + dt.  Blocks are dispatched in increasing index order, so
-// every chunk a block waits for belongs to a block that started earlier; a
-// block publishes its summary before it waits, so waits never form a cycle.
+// Position of a tile: chunk c along T, chain = b * n_dt + dt.  All < 2^31.
+struct TileCoord {
+    uint32_t c, chain, b, dt;
+};
+__device__ __forceinline__ TileCoord tile_coord(const ScanParams &p, uint32_t tile) {
+    TileCoord t;
+    t.c = p.by_chains.div(tile);
+    t.chain = tile - t.c * p.by_chains.d;
+    t.b = p.by_dt.div(t.chain);
+    t.dt = t.chain - t.b * p.by_dt.d;
+    return t;
+}
 
-__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
+template <typename IO>
+__device__ __forceinline__ float load_init(const ScanParams &p, int64_t b, int64_t d, float dflt) {
+    if (p.init == nullptr || d >= p.D) return dflt;
+    return load_scalar<IO>(static_cast<const IO *>(p.init) + b * p.init_bs + d);
+}
+
+// Publish this chunk's summary pairs for CV channels starting at ch.
+template <int CV, int TC>
+__device__ __forceinline__ void publish_summary(const ScanParams &p, int64_t tile, int ch,
+                                                const float2 (&tot)[CV]) {
+    uint64_t *w = p.words + tile * 3 * TC + ch;
+#pragma unroll
+    for (int v = 0; v < CV; ++v) {
+        st_relaxed_u64(w + v, pack_word(p.epoch, tot[v].x));
+        st_relaxed_u64(w + TC + v, pack_word(p.epoch, tot[v].y));
+    }
+}
+
+template <int CV, int TC>
+__device__ __forceinline__ void publish_state(const ScanParams &p, int64_t tile, int ch,
+                                              const float (&st)[CV]) {
+    uint64_t *w = p.words + tile * 3 * TC + 2 * TC + ch;
+#pragma unroll
+    for (int v = 0; v < CV; ++v) st_relaxed_u64(w + v, pack_word(p.epoch, st[v]));
+}
+
+// Decoupled look-back for CV channels of one lane: the state entering chunk c
+// of `chain`.  Walks back over chunks c-1, c-2, ... reading K of them per
+// round trip: a chunk whose final state S is published ends the walk; a chunk
+// with only its summary (A, B) is folded in and the walk goes on; a chunk with
+// neither is waited for (bounded, with back-off).  Before chunk 0 the state is
+// the initial state.  Each lane works alone: its channels' words carry their
+// own validity.
+template <class Op, typename IO, int CV, int TC>
+__device__ void look_back(const ScanParams &p, int64_t c, int64_t chain, int64_t b, int64_t d_first,
+                          int ch, float (&hin)[CV]) {
+    constexpr int K = CV >= 4 ? 1 : (CV == 2 ? 2 : 4);
+    float2 M[CV];
+#pragma unroll
+    for (int v = 0; v < CV; ++v) M[v] = Op::identity();
+    int64_t q = c - 1;
+    uint32_t polls = 0, ns = 32;
+    while (true) {
+        uint64_t wa[K][CV], wb[K][CV], ws[K][CV];
+#pragma unroll
+        for (int i = 0; i < K; ++i) {
+            const int64_t qq = q - i;
+            if (qq >= 0) {
+                const uint64_t *w = p.words + (qq * p.n_chains + chain) * 3 * TC + ch;
+#pragma unroll
+                for (int v = 0; v < CV; ++v) {
+                    ws[i][v] = ld_relaxed_u64(w + 2 * TC + v);
+                    wa[i][v] = ld_relaxed_u64(w + v);
+                    wb[i][v] = ld_relaxed_u64(w + TC + v);
+                }
+            }
+        }
+        int consumed = 0;
+        bool done = false, stop = false;
+#pragma unroll
+        for (int i = 0; i < K; ++i) {
+            if (done || stop) continue;
+            const int64_t qq = q - i;
+            if (qq < 0) {
+#pragma unroll
+                for (int v = 0; v < CV; ++v)
+                    hin[v] = Op::apply(M[v], load_init<IO>(p, b, d_first + v, Op::default_init()));
+                done = true;
+                continue;
+            }
+            bool s_ok = true, ab_ok = true;
+#pragma unroll
+            for (int v = 0; v < CV; ++v) {
+                s_ok = s_ok && word_valid(ws[i][v], p.epoch);
+                ab_ok = ab_ok && word_valid(wa[i][v], p.epoch) && word_valid(wb[i][v], p.epoch);
+            }
+            if (s_ok) {
+#pragma unroll
+                for (int v = 0; v < CV; ++v) hin[v] = Op::apply(M[v], word_value(ws[i][v]));
+                done = true;
+            } else if (ab_ok) {
+#pragma unroll
+                for (int v = 0; v < CV; ++v)
+                    M[v] = Op::combine(make_float2(word_value(wa[i][v]), word_value(wb[i][v])), M[v]);
+                consumed = i + 1;
+            } else {
+                stop = true;
+            }
+        }
+        if (done) return;
+        if (consumed > 0) {
+            q -= consumed;
+            ns = 32;
+            continue;
+        }
+        if (++polls > p.spin_limit) {
+            atomicOr(p.status, kTimeoutBit);
+#pragma unroll
+            for (int v = 0; v < CV; ++v) hin[v] = __int_as_float(0x7fffffff);
+            return;
+        }
+        __nanosleep(ns);
+        ns = ns < 1024 ? ns * 2 : 1024;
+    }
+}
+
+// The carry of one tile, as done by the carry warp: fold the W warp totals in
+// s_tot (replaced in place by each warp's incoming state), publish the chunk
+// summary, look back, publish the chunk's final state.  `between` runs after
+// the per-warp states are in shared memory and before the final state is
+// published (it releases the data warps).
+template <class Op, typename IO, int CV, int TC, int W, class Between>
+__device__ __forceinline__ void carry_tile(const ScanParams &p, int64_t tile, float2 (*s_tot)[TC],
+                                           int lane, Between between) {
+    const TileCoord tc = tile_coord(p, uint32_t(tile));
+    const int64_t chain = tc.chain;
+    const int64_t c = tc.c;
+    const int64_t b = tc.b;
+    const int ch = lane * CV;
+    const int64_t dl = int64_t(tc.dt) * TC + ch;
+    float2 total[CV];
+#pragma unroll
+    for (int v = 0; v < CV; ++v) total[v] = Op::identity();
+    for (int w = 0; w < W; ++w) {
+#pragma unroll
+        for (int v = 0; v < CV; ++v) {
+            const float2 t = s_tot[w][ch + v];
+            s_tot[w][ch + v] = total[v];          // exclusive prefix over warps
+            total[v] = Op::combine(total[v], t);
+        }
+    }
+    const bool publish = (p.n_chunks > 1) && (c < p.n_chunks - 1) && (tile != p.drop_tile);
+    float hin[CV];
+    if (c == 0) {
+#pragma unroll
+        for (int v = 0; v < CV; ++v) hin[v] = load_init<IO>(p, b, dl + v, Op::default_init());
+    } else {
+        if (publish) publish_summary<CV, TC>(p, tile, ch, total);
+        look_back<Op, IO, CV, TC>(p, c, chain, b, dl, ch, hin);
+    }
+    // state entering each warp's rows, written over the prefix pair's .x
+    for (int w = 0; w < W; ++w) {
+#pragma unroll
+        for (int v = 0; v < CV; ++v) s_tot[w][ch + v].x = Op::apply(s_tot[w][ch + v], hin[v]);
+    }
+    between();
+    if (publish) {
+        float fin[CV];
+#pragma unroll
+        for (int v = 0; v < CV; ++v) fin[v] = Op::apply(total[v], hin[v]);
+        publish_state<CV, TC>(p, tile, ch, fin);
+    }
+}
+
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// -------------------------------------------------------- tile kernel
+//
+// One block per tile (TR rows x TC channels), W data warps + 1 carry warp.
+// Template parameters: Op, IO (storage type), V (channels per thread: one
+// 16-byte vector, or 1 for the scalar variant), CG (lanes across channels),
+// R (rows per thread), W (data warps).  J = 32 / CG row groups per warp,
+// TR = W * J * R, TC = CG * V.  Tiles are numbered chain-fastest:
+// blockIdx.x = chunk * n_chains + chain, chain = b * n_dt + dt.  Blocks are
+// dispatched in increasing index order and a block publishes its summary
+// before it waits, so every wait is for a block that started earlier and waits
+// never form a cycle.  Used for the scalar (unaligned) variant and as a
+// cross-check of the pipelined kernel.
 template <class Op, typename IO, int V, int CG, int R, int W, int MINB>
-__global__ void __launch_bounds__((W + 1) * 32, MINB) scan_kernel(const ScanParams p) {
+__global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const ScanParams p) {
     constexpr int J = 32 / CG;
     constexpr int TR = W * J * R;
     constexpr int TC = CG * V;
@@ -230,20 +454,17 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_kernel(const ScanPara
     static_assert(CG * J == 32, "CG must divide 32");
     static_assert(TC % 32 == 0, "a tile spans a multiple of 32 channels");
 
-    __shared__ float2 s_tot[W][TC];   // per-warp totals, then per-warp exclusive prefixes
-    __shared__ float s_win[W][TC];    // state entering each warp's rows
+    __shared__ float2 s_tot[W][TC];   // per-warp totals -> per-warp incoming states (.x)
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-
     const int64_t tile = blockIdx.x;
-    const int64_t chain = tile % p.n_chains;
-    const int64_t c = tile / p.n_chains;
-    const int64_t b = chain / p.n_dt;
-    const int64_t dt = chain - b * p.n_dt;
 
     if (warp < W) {
-        // ================================================= data warps
+        const TileCoord tc = tile_coord(p, uint32_t(tile));
+        const int64_t c = tc.c;
+        const int64_t b = tc.b;
+        const int64_t dt = tc.dt;
         const int g = lane % CG;
         const int j = lane / CG;
         const int64_t d0 = dt * TC + int64_t(g) * V;
@@ -254,7 +475,6 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_kernel(const ScanPara
         IO *out = static_cast<IO *>(p.out);
         const int64_t base = (b * p.T) * p.D + d0;
 
-        // ---- load R rows x V channels of both operands (all in flight at once)
         float x0[R][V], x1[R][V];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
@@ -267,8 +487,6 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_kernel(const ScanPara
                 for (int v = 0; v < V; ++v) { x0[r][v] = Op::pad0(); x1[r][v] = Op::pad1(); }
             }
         }
-
-        // ---- phase 1: activations and the thread's own fold
         float2 incl[V];
 #pragma unroll
         for (int v = 0; v < V; ++v) incl[v] = Op::identity();
@@ -283,8 +501,6 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_kernel(const ScanPara
                 incl[v] = Op::combine(incl[v], make_float2(e0, e1));
             }
         }
-
-        // ---- phase 2a: inclusive scan across the J row groups of the warp
 #pragma unroll
         for (int off = 1; off < J; off <<= 1) {
 #pragma unroll
@@ -307,13 +523,12 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_kernel(const ScanPara
             o.y = __shfl_up_sync(0xffffffffu, incl[v].y, CG);
             excl[v] = (J > 1 && j > 0) ? o : Op::identity();
         }
-        named_barrier(1, NT);   // totals are in shared memory
-        named_barrier(2, NT);   // the carry warp has filled s_win
+        named_barrier_sync(1, NT);   // totals are in shared memory
+        named_barrier_sync(2, NT);   // the carry warp has written the warp states
 
-        // ---- phase 3: replay the thread's steps from its incoming state, store
         float st[V];
 #pragma unroll
-        for (int v = 0; v < V; ++v) st[v] = Op::apply(excl[v], s_win[warp][g * V + v]);
+        for (int v = 0; v < V; ++v) st[v] = Op::apply(excl[v], s_tot[warp][g * V + v].x);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             float y[V];
@@ -326,114 +541,234 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_kernel(const ScanPara
             if (dvalid && t < p.T) Access<IO, V>::store(out + base + t * p.D, y);
         }
     } else {
-        // ================================================= carry warp
-        // lane owns tile channels [lane * CV, lane * CV + CV)
-        const int ch = lane * CV;
-        const int64_t dl = dt * TC + ch;   // first global channel
-        float init[CV];
-#pragma unroll
-        for (int v = 0; v < CV; ++v) {
-            init[v] = Op::default_init();
-            if (p.init != nullptr && dl + v < p.D)
-                init[v] = load_scalar<IO>(static_cast<const IO *>(p.init) + b * p.init_bs + dl + v);
-        }
-        named_barrier(1, NT);
+        named_barrier_sync(1, NT);
+        carry_tile<Op, IO, CV, TC, W>(p, tile, s_tot, lane, [&] { named_barrier_sync(2, NT); });
+    }
+}
 
-        // exclusive prefix over the warps (in place) and the tile total
-        float2 total[CV];
-#pragma unroll
-        for (int v = 0; v < CV; ++v) total[v] = Op::identity();
-        for (int w = 0; w < W; ++w) {
-#pragma unroll
-            for (int v = 0; v < CV; ++v) {
-                const float2 t = s_tot[w][ch + v];
-                s_tot[w][ch + v] = total[v];
-                total[v] = Op::combine(total[v], t);
-            }
-        }
+// --------------------------------------------------- pipelined kernel
+//
+// Persistent blocks (co-resident, cooperative launch), each owning tiles
+// blockIdx.x, blockIdx.x + gridDim.x, ... in order.  A tile is TR x TC with
+// TC = CG * V channels and TR = W * J * R rows (J = 32 / CG row groups per
+// warp): lane (g, j) = (lane % CG, lane / CG) of warp w owns channels
+// [g V, g V + V) of rows [(w J + j) R, (w J + j) R + R).  V = 4 (16-byte fp32
+// or 8-byte bf16 vectors).  Narrow tiles keep the chunk hand-off cheap: the
+// chunks of one channel tile that are in flight at once number about
+// gridDim.x / n_chains, and a look-back folds that many summaries of TC
+// channels each.
+//
+// Loads: each data thread streams its own vector pieces of the next S tiles
+// into a private slice of a shared-memory ring with cp.async (no registers
+// held, no cross-thread hand-off: a thread only reads what it copied), one
+// commit group per tile, so S tiles of HBM reads are always in flight.
+//
+// Compute, with a one-tile lag: phase A of tile n (activations, the thread's
+// fold over its R rows, the scan across the warp's J row groups, the warp's
+// summary to shared memory; pairs and the thread's exclusive prefix stay in
+// registers), then phase B of tile n-1 (replay from the thread's incoming
+// state, store).  The carry warp runs the hand-off of tile n while the data
+// warps are in phase A of tile n+1, so the look-back latency is overlapped
+// with loads and compute.  Shared summaries and named barriers are
+// double-buffered by tile parity:
+//   barrier 1 + (n & 1): data warps arrive (summaries of tile n written),
+//                        carry warp waits;
+//   barrier 3 + (n & 1): carry warp arrives (incoming states of tile n
+//                        written), data warps wait.
+// Every wait is for a tile with a smaller index and blocks are co-resident,
+// so the smallest unfinished tile can always progress.
+template <typename IO, int V, int CG, int R, int S, int W>
+struct PipeShape {
+    static constexpr int NTD = W * 32;                       // data threads
+    static constexpr int J = 32 / CG;
+    static constexpr int TC = CG * V;
+    static constexpr int TR = W * J * R;
+    static constexpr int VB = V * int(sizeof(IO));           // bytes per vector
+    static constexpr size_t stage_bytes = size_t(R) * 2 * NTD * VB;
+    static constexpr size_t tot_bytes = size_t(2) * W * TC * sizeof(float2);
+    static constexpr size_t smem_bytes = S * stage_bytes + tot_bytes;
+};
 
-        float hin[CV];
+template <int BYTES> __device__ __forceinline__ void cp_async(void *smem, const void *gmem);
+template <> __device__ __forceinline__ void cp_async<16>(void *smem, const void *gmem) {
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+template <> __device__ __forceinline__ void cp_async<8>(void *smem, const void *gmem) {
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <class Op, typename IO, int V, int CG, int R, int S, int W, int MINB>
+__global__ void __launch_bounds__((W + 1) * 32, MINB) scan_pipelined_kernel(const ScanParams p) {
+    using Shape = PipeShape<IO, V, CG, R, S, W>;
+    using Vec = typename VecOf<IO, V>::type;
+    constexpr int J = Shape::J;
+    constexpr int TC = Shape::TC;
+    constexpr int TR = Shape::TR;
+    constexpr int NTD = Shape::NTD;
+    constexpr int VB = Shape::VB;
+    constexpr int CV = TC / 32;
+    constexpr uint32_t NT = (W + 1) * 32;
+    static_assert(sizeof(Vec) == VB, "vector type matches the vector width");
+    static_assert(CG * J == 32 && TC % 32 == 0, "lane layout");
+
+    extern __shared__ __align__(16) unsigned char smem[];
+    Vec *ring = reinterpret_cast<Vec *>(smem);                             // [S][R][2][NTD]
+    float2 (*s_tot)[W][TC] = reinterpret_cast<float2 (*)[W][TC]>(smem + S * Shape::stage_bytes);
+
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t G = gridDim.x;
+    const int64_t first = blockIdx.x;
+    const int n_local = int((p.n_tiles - first + G - 1) / G);
+
+    if (warp < W) {
+        // ============================================== data warps
+        const int tid = threadIdx.x;
+        const int g = lane % CG;
+        const int j = lane / CG;
+        const IO *in0 = static_cast<const IO *>(p.in0);
+        const IO *in1 = static_cast<const IO *>(p.in1);
+        IO *out = static_cast<IO *>(p.out);
+
+        // global position of this thread's piece of tile n
+        auto locate = [&](int n, int64_t &base, int64_t &row0, bool &dvalid) {
+            const TileCoord tc = tile_coord(p, uint32_t(first + int64_t(n) * G));
+            const int64_t d0 = int64_t(tc.dt) * TC + g * V;
+            dvalid = d0 < p.D;
+            row0 = int64_t(tc.c) * TR + (warp * J + j) * R;
+            base = (int64_t(tc.b) * p.T) * p.D + d0;
+        };
+        auto issue = [&](int n) {
+            if (n < n_local) {
+                int64_t base, row0;
+                bool dvalid;
+                locate(n, base, row0, dvalid);
+                Vec *slot = ring + (n % S) * (R * 2 * NTD) + tid;
 #pragma unroll
-        for (int v = 0; v < CV; ++v) hin[v] = init[v];
-        const int64_t slot = tile;
-        const bool publish = (p.n_chunks > 1) && (c < p.n_chunks - 1) && (tile != p.drop_tile);
-        const uint64_t tag = p.epoch << 2;
-        if (c > 0) {
-            // publish this chunk's summary so later chunks need not wait for its carry
-            if (publish) {
-#pragma unroll
-                for (int v = 0; v < CV; ++v) __stcg(&p.agg[slot * TC + ch + v], total[v]);
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) st_release_u64(&p.flags[slot], tag | ST_AGG);
-            }
-            // decoupled look-back: lane i watches chunk pos - i
-            float2 M[CV];
-#pragma unroll
-            for (int v = 0; v < CV; ++v) M[v] = Op::identity();
-            int64_t pos = c - 1;
-            uint32_t polls = 0;
-            bool timed_out = false;
-            while (true) {
-                const int64_t q = pos - lane;
-                int first = 32;
-                uint32_t ns = 32;
-                while (true) {
-                    uint32_t stt = ST_PREFIX;   // before chunk 0: the initial state
-                    if (q >= 0) {
-                        const uint64_t f = ld_acquire_u64(&p.flags[q * p.n_chains + chain]);
-                        stt = ((f >> 2) == p.epoch) ? uint32_t(f & 3u) : ST_NONE;
+                for (int r = 0; r < R; ++r) {
+                    const int64_t t = row0 + r;
+                    if (dvalid && t < p.T) {
+                        cp_async<VB>(slot + (r * 2 + 0) * NTD, in0 + base + t * p.D);
+                        cp_async<VB>(slot + (r * 2 + 1) * NTD, in1 + base + t * p.D);
                     }
-                    const uint32_t pm = __ballot_sync(0xffffffffu, stt == ST_PREFIX);
-                    const uint32_t rm = __ballot_sync(0xffffffffu, stt != ST_NONE);
-                    first = pm ? (__ffs(pm) - 1) : 32;
-                    const uint32_t need = (first >= 31) ? 0xffffffffu : ((2u << first) - 1u);
-                    if ((rm & need) == need) break;
-                    if (++polls > p.spin_limit) { timed_out = true; break; }
-                    __nanosleep(ns);
-                    ns = ns < 1024 ? ns * 2 : 1024;
                 }
-                __syncwarp();
-                if (timed_out) break;
-                for (int i = 0; i < first; ++i) {
-                    const int64_t qq = pos - i;
-#pragma unroll
-                    for (int v = 0; v < CV; ++v) {
-                        const float2 a = __ldcg(&p.agg[(qq * p.n_chains + chain) * TC + ch + v]);
-                        M[v] = Op::combine(a, M[v]);
-                    }
-                }
-                if (first < 32) {
-                    const int64_t qq = pos - first;
-#pragma unroll
-                    for (int v = 0; v < CV; ++v) {
-                        const float s = (qq >= 0)
-                            ? __ldcg(&p.pref[(qq * p.n_chains + chain) * TC + ch + v])
-                            : init[v];
-                        hin[v] = Op::apply(M[v], s);
-                    }
-                    break;
-                }
-                pos -= 32;
             }
-            if (timed_out) {
-                if (lane == 0) atomicOr(p.status, kTimeoutBit);
+            cp_async_commit();   // one group per tile, empty past the end
+        };
+
+        float2 P[2][R][V];   // pairs of the two tiles in flight (tile parity)
+        float2 E[2][V];      // the thread's exclusive prefix within its warp
+
+        // phase A of tile n into register buffer BUF
+        auto phaseA = [&](int n, auto bufc) {
+            constexpr int BUF = decltype(bufc)::value;
+            cp_async_wait<S - 1>();   // this thread's pieces of tile n have landed
+            int64_t base, row0;
+            bool dvalid;
+            locate(n, base, row0, dvalid);
+            const Vec *slot = ring + (n % S) * (R * 2 * NTD) + tid;
+            float2 incl[V];
 #pragma unroll
-                for (int v = 0; v < CV; ++v) hin[v] = __int_as_float(0x7fffffff);
+            for (int v = 0; v < V; ++v) incl[v] = Op::identity();
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                float x0[V], x1[V];
+                const int64_t t = row0 + r;
+                if (dvalid && t < p.T) {
+                    unpack(slot[(r * 2 + 0) * NTD], x0);
+                    unpack(slot[(r * 2 + 1) * NTD], x1);
+                } else {
+#pragma unroll
+                    for (int v = 0; v < V; ++v) { x0[v] = Op::pad0(); x1[v] = Op::pad1(); }
+                }
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    float e0, e1;
+                    Op::element(x0[v], x1[v], e0, e1);
+                    P[BUF][r][v] = make_float2(e0, e1);
+                    incl[v] = Op::combine(incl[v], P[BUF][r][v]);
+                }
             }
+            // the ring slot is consumed: refill it with tile n + S
+            issue(n + S);
+            // scan across the J row groups of the warp
+#pragma unroll
+            for (int off = 1; off < J; off <<= 1) {
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    float2 o;
+                    o.x = __shfl_up_sync(0xffffffffu, incl[v].x, off * CG);
+                    o.y = __shfl_up_sync(0xffffffffu, incl[v].y, off * CG);
+                    if (j >= off) incl[v] = Op::combine(o, incl[v]);
+                }
+            }
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                float2 o;
+                o.x = __shfl_up_sync(0xffffffffu, incl[v].x, CG);
+                o.y = __shfl_up_sync(0xffffffffu, incl[v].y, CG);
+                E[BUF][v] = (J > 1 && j > 0) ? o : Op::identity();
+            }
+            if (j == J - 1) {
+#pragma unroll
+                for (int v = 0; v < V; ++v) s_tot[BUF][warp][g * V + v] = incl[v];
+            }
+            named_barrier_arrive(1 + BUF, NT);
+        };
+
+        // phase B of tile n from register buffer BUF
+        auto phaseB = [&](int n, auto bufc) {
+            constexpr int BUF = decltype(bufc)::value;
+            int64_t base, row0;
+            bool dvalid;
+            locate(n, base, row0, dvalid);
+            named_barrier_sync(3 + BUF, NT);
+            float st[V];
+#pragma unroll
+            for (int v = 0; v < V; ++v) st[v] = Op::apply(E[BUF][v], s_tot[BUF][warp][g * V + v].x);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                float y[V];
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    st[v] = Op::step(P[BUF][r][v].x, P[BUF][r][v].y, st[v]);
+                    y[v] = st[v];
+                }
+                const int64_t t = row0 + r;
+                if (dvalid && t < p.T) Access<IO, V>::store(out + base + t * p.D, y);
+            }
+        };
+
+        using B0 = std::integral_constant<int, 0>;
+        using B1 = std::integral_constant<int, 1>;
+        for (int s = 0; s < S; ++s) issue(s);
+        int n = 0;
+        for (; n + 1 < n_local; n += 2) {
+            phaseA(n, B0{});
+            if (n >= 1) phaseB(n - 1, B1{});
+            phaseA(n + 1, B1{});
+            phaseB(n, B0{});
         }
-        // state entering each warp's rows
-        for (int w = 0; w < W; ++w) {
-#pragma unroll
-            for (int v = 0; v < CV; ++v) s_win[w][ch + v] = Op::apply(s_tot[w][ch + v], hin[v]);
+        if (n < n_local) {
+            phaseA(n, B0{});
+            if (n >= 1) phaseB(n - 1, B1{});
+            phaseB(n, B0{});
+        } else if (n_local >= 1) {
+            phaseB(n - 1, B1{});
         }
-        named_barrier(2, NT);
-        if (publish) {
-#pragma unroll
-            for (int v = 0; v < CV; ++v) __stcg(&p.pref[slot * TC + ch + v], Op::apply(total[v], hin[v]));
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) st_release_u64(&p.flags[slot], tag | ST_PREFIX);
+        cp_async_wait<0>();
+    } else {
+        // ============================================== carry warp
+        for (int n = 0; n < n_local; ++n) {
+            const int buf = n & 1;
+            named_barrier_sync(1 + buf, NT);
+            carry_tile<Op, IO, CV, TC, W>(p, first + int64_t(n) * G, s_tot[buf], lane,
+                                          [&] { named_barrier_arrive(3 + buf, NT); });
         }
     }
 }

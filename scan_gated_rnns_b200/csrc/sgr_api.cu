@@ -4,6 +4,7 @@
 #include "scan_gated_rnns.h"
 #include "scan_engine.cuh"
 
+#include <algorithm>
 #include <atomic>
 #include <cstring>
 #include <limits>
@@ -12,29 +13,47 @@ namespace {
 
 using namespace sgr;
 
-constexpr int kWarps = 8;           // warps per tile block
-constexpr int64_t kTargetTiles = 4 * 148;  // prefer >= 4 tiles per SM before shrinking chunks
+// Both kernels use 7 data warps + 1 carry warp = 8 warps per block, so blocks
+// spread evenly over the SM's 4 sub-partitions, each of which has its own
+// register file (two pipelined blocks per SM: 128 registers per thread).
+constexpr int kWarps = 7;
+constexpr int kPipeWarps = 7;
+constexpr int kStages = 3;
+constexpr int64_t kTargetTiles = 4 * 148;  // tile kernel: prefer >= 4 tiles per SM
 constexpr size_t kAlign = 256;
+
+enum Kind { KIND_AUTO = 0, KIND_TILE = 1, KIND_PIPELINED = 2 };
 
 std::atomic<int> g_override_cg{0};
 std::atomic<int> g_override_r{0};
-// Launch epochs tag the chunk status words.  1 is reserved for launches
-// captured into CUDA graphs (those zero the flags first, inside the graph).
+std::atomic<int> g_override_kind{KIND_AUTO};
+// Launch epochs tag the hand-off words (32 bits in each word).  0 never tags a
+// word (zeroed memory) and 1 is reserved for launches captured into CUDA
+// graphs, which zero the words inside the graph first.
 std::atomic<uint64_t> g_epoch{2};
 std::atomic<uint32_t> g_spin_limit{sgr::kSpinLimit};
 std::atomic<int64_t> g_drop_tile{-1};
+
+uint32_t next_epoch() {
+    uint32_t e;
+    do { e = uint32_t(g_epoch.fetch_add(1)); } while (e < 2);
+    return e;
+}
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Plan {
     int esz = 4;          // bytes per stored element
     bool vec = false;     // 128-bit path
+    int kind = KIND_TILE;
     int V = 1;            // channels per thread
     int cg = 32;          // lanes across channels
     int r = 2;            // rows per thread
+    int stages = 0;       // pipelined: tiles in flight per block
     int TR = 0, TC = 0;   // tile rows / channels
     int64_t n_dt = 0, n_chains = 0, n_chunks = 0, n_tiles = 0;
-    size_t off_flags = 0, off_agg = 0, off_pref = 0, ws_bytes = 0;
+    size_t smem = 0;      // dynamic shared memory per block
+    size_t off_words = 0, ws_bytes = 0;
 };
 
 bool mul_ok(int64_t a, int64_t b, int64_t *out) {
@@ -44,51 +63,82 @@ bool mul_ok(int64_t a, int64_t b, int64_t *out) {
     return true;
 }
 
-// Chunk shape for a scan: vector width from dtype and alignment, CG lanes
-// across channels (8 => 128-byte row segments for fp32/bf16 rows), and the
-// largest rows-per-thread that still leaves >= kTargetTiles tiles.
+// pipelined lane layout: fp32 8 lanes x 4 channels (32-channel tiles, 128-byte
+// rows), bf16 16 lanes x 4 channels (64-channel tiles, 128-byte rows)
+template <typename IO> constexpr int pipe_cg() { return sizeof(IO) == 4 ? 8 : 16; }
+
+template <typename IO, int R>
+constexpr size_t pipe_smem() { return PipeShape<IO, 4, pipe_cg<IO>(), R, kStages, kPipeWarps>::smem_bytes; }
+
+// Tile shape of a scan.  Aligned vector-width rows take the pipelined kernel
+// (fp32: 7 x 4 x R rows x 32 channels; bf16: 7 x 2 x R rows x 64 channels;
+// 128-byte row segments); anything else takes the tile kernel's scalar
+// variant.  The override knobs select the kernel and the rows per thread.
 Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned) {
     Plan p;
     p.esz = (dtype == SGR_BF16) ? 2 : 4;
     const int vw = 16 / p.esz;
     p.vec = aligned && (D % vw == 0);
-    p.V = p.vec ? vw : 1;
-    int cg = p.vec ? 8 : 32;
-    const int ocg = g_override_cg.load();
-    if (p.vec && (ocg == 8 || ocg == 32)) cg = ocg;
-    p.cg = cg;
-    p.TC = p.cg * p.V;
-    const int J = 32 / p.cg;
+    const int ok = g_override_kind.load();
+    p.kind = (p.vec && ok != KIND_TILE) ? KIND_PIPELINED : KIND_TILE;
+    const int orr = g_override_r.load();
+    if (p.kind == KIND_PIPELINED) {
+        // 4 channels per lane (16-byte fp32 / 8-byte bf16 vectors)
+        p.V = 4;
+        p.cg = p.esz == 4 ? 8 : 16;
+        p.TC = p.cg * p.V;
+        // rows per thread {2, 4}, automatic 4
+        p.r = (orr == 2 || orr == 4) ? orr : 4;
+        p.stages = kStages;
+        p.TR = kPipeWarps * (32 / p.cg) * p.r;
+        if (p.esz == 4) p.smem = p.r == 4 ? pipe_smem<float, 4>() : pipe_smem<float, 2>();
+        else p.smem = p.r == 4 ? pipe_smem<__nv_bfloat16, 4>() : pipe_smem<__nv_bfloat16, 2>();
+    } else {
+        // tile kernel: 8 lanes x one vector (32 fp32 / 64 bf16 channels,
+        // 128-byte row segments) or, unaligned, 32 lanes x 1 channel
+        p.V = p.vec ? vw : 1;
+        p.cg = p.vec ? 8 : 32;
+        p.TC = p.cg * p.V;
+        const int J = 32 / p.cg;
+        const int64_t n_chains = B * ((D + p.TC - 1) / p.TC);
+        // rows per thread: the automatic choice keeps a data thread within 72
+        // registers (16 elements of each operand); the override may go to 32
+        const int rmax_auto = p.vec ? (p.V >= 8 ? 2 : 4) : 8;
+        const int rmax = p.V >= 8 ? 4 : 8;
+        int r = 1;
+        if (orr == 1 || orr == 2 || orr == 4 || orr == 8) {
+            r = orr < rmax ? orr : rmax;
+        } else {
+            for (int cand : {8, 4, 2, 1}) {
+                if (cand > rmax_auto) continue;
+                const int64_t tr = int64_t(kWarps) * J * cand;
+                const int64_t chunks = (T + tr - 1) / tr;
+                if (n_chains * chunks >= kTargetTiles || cand == 1) { r = cand; break; }
+            }
+        }
+        p.r = r;
+        p.TR = kWarps * J * r;
+    }
     p.n_dt = (D + p.TC - 1) / p.TC;
     p.n_chains = B * p.n_dt;
-    // rows per thread: the automatic choice keeps a data thread within 72
-    // registers without spilling (16 elements of each operand), so three
-    // blocks fit per SM; the override may go up to 32 elements per operand
-    const int rmax_auto = p.vec ? (p.V >= 8 ? 2 : 4) : 8;
-    const int rmax = p.V >= 8 ? 4 : 8;
-    const int orr = g_override_r.load();
-    int r = 1;
-    if (orr == 1 || orr == 2 || orr == 4 || orr == 8) {
-        r = orr < rmax ? orr : rmax;
-    } else {
-        for (int cand : {8, 4, 2, 1}) {
-            if (cand > rmax_auto) continue;
-            const int64_t tr = int64_t(kWarps) * J * cand;
-            const int64_t chunks = (T + tr - 1) / tr;
-            if (p.n_chains * chunks >= kTargetTiles || cand == 1) { r = cand; break; }
-        }
-    }
-    p.r = r;
-    p.TR = kWarps * J * r;
     p.n_chunks = (T + p.TR - 1) / p.TR;
     p.n_tiles = p.n_chains * p.n_chunks;
     if (p.n_chunks > 1) {
-        p.off_flags = kAlign;                                   // [0, 256): status word
-        p.off_agg = align_up(p.off_flags + 8 * size_t(p.n_tiles), kAlign);
-        p.off_pref = align_up(p.off_agg + 8 * size_t(p.n_tiles) * p.TC, kAlign);
-        p.ws_bytes = align_up(p.off_pref + 4 * size_t(p.n_tiles) * p.TC, kAlign);
+        p.off_words = kAlign;                                   // [0, 256): status word
+        p.ws_bytes = align_up(p.off_words + size_t(p.n_tiles) * 3 * p.TC * 8, kAlign);
     }
     return p;
+}
+
+// divisor constants for FastDiv (see scan_engine.cuh); 1 <= d < 2^31
+FastDiv make_fastdiv(uint32_t d) {
+    FastDiv f;
+    f.d = d;
+    uint32_t s = 0;
+    while ((uint64_t(1) << s) < d) ++s;
+    f.s = s;
+    f.m = uint32_t(((uint64_t(1) << 32) * ((uint64_t(1) << s) - d)) / d + 1);
+    return f;
 }
 
 bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
@@ -105,37 +155,98 @@ size_t rows_span(int64_t B, int64_t D, int64_t bs, int esz) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// ---- tile kernel launch
 template <class Op, typename IO, int V, int CG, int R>
-cudaError_t launch_scan(const ScanParams &sp, int64_t n_tiles, cudaStream_t s) {
+cudaError_t launch_tile(const ScanParams &sp, cudaStream_t s) {
     if constexpr (R * V > 32) {
         return cudaErrorInvalidConfiguration;   // never planned (see make_plan)
     } else {
         // registers a data thread keeps live: its tile (2RV), one pair per
-        // channel (2V) and about 24 for addressing; blocks of 288 threads
+        // channel (2V) and about 24 for addressing; blocks of 256 threads
         constexpr int NEED = 2 * R * V + 2 * V + 24;
         constexpr int MINB = NEED <= 56 ? 4 : (NEED <= 72 ? 3 : 2);
-        scan_kernel<Op, IO, V, CG, R, kWarps, MINB>
-            <<<dim3(unsigned(n_tiles)), (kWarps + 1) * 32, 0, s>>>(sp);
+        scan_tile_kernel<Op, IO, V, CG, R, kWarps, MINB>
+            <<<dim3(unsigned(sp.n_tiles)), (kWarps + 1) * 32, 0, s>>>(sp);
         return cudaGetLastError();
     }
 }
 
 template <class Op, typename IO, int V, int CG>
-cudaError_t dispatch_r(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
+cudaError_t dispatch_tile_r(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
     switch (pl.r) {
-        case 1: return launch_scan<Op, IO, V, CG, 1>(sp, pl.n_tiles, s);
-        case 2: return launch_scan<Op, IO, V, CG, 2>(sp, pl.n_tiles, s);
-        case 4: return launch_scan<Op, IO, V, CG, 4>(sp, pl.n_tiles, s);
-        default: return launch_scan<Op, IO, V, CG, 8>(sp, pl.n_tiles, s);
+        case 1: return launch_tile<Op, IO, V, CG, 1>(sp, s);
+        case 2: return launch_tile<Op, IO, V, CG, 2>(sp, s);
+        case 4: return launch_tile<Op, IO, V, CG, 4>(sp, s);
+        default: return launch_tile<Op, IO, V, CG, 8>(sp, s);
     }
+}
+
+// ---- pipelined kernel launch: persistent, co-resident blocks
+struct DeviceInfo {
+    int sms = 0;
+};
+DeviceInfo device_info(int dev) {
+    static std::atomic<int> cache[64];
+    DeviceInfo d;
+    if (dev >= 0 && dev < 64) {
+        int v = cache[dev].load();
+        if (v == 0) {
+            if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) v = 0;
+            cache[dev].store(v);
+        }
+        d.sms = v;
+    }
+    return d;
+}
+
+template <class Op, typename IO, int V, int R>
+cudaError_t launch_pipelined(const ScanParams &sp_in, cudaStream_t s, int64_t *grid_out) {
+    constexpr int CG = pipe_cg<IO>();
+    auto kernel = scan_pipelined_kernel<Op, IO, V, CG, R, kStages, kPipeWarps, 2>;
+    constexpr size_t smem = PipeShape<IO, V, CG, R, kStages, kPipeWarps>::smem_bytes;
+    constexpr int NT = (kPipeWarps + 1) * 32;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    // per-device one-time set-up of the shared-memory limit and occupancy
+    static std::atomic<int> occ_cache[64];
+    int occ = (dev >= 0 && dev < 64) ? occ_cache[dev].load() : 0;
+    if (occ == 0) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, NT, smem);
+        if (e != cudaSuccess) return e;
+        if (occ <= 0) return cudaErrorInvalidConfiguration;
+        if (dev >= 0 && dev < 64) occ_cache[dev].store(occ);
+    }
+    const DeviceInfo di = device_info(dev);
+    if (di.sms <= 0) return cudaErrorInvalidDevice;
+    const int64_t grid = std::min<int64_t>(sp_in.n_tiles, int64_t(di.sms) * occ);
+    if (grid_out) *grid_out = grid;
+    ScanParams sp = sp_in;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(grid));
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, sp);
+    return e;
 }
 
 template <class Op, typename IO>
 cudaError_t dispatch(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
     constexpr int VW = 16 / int(sizeof(IO));
-    if (!pl.vec) return dispatch_r<Op, IO, 1, 32>(pl, sp, s);
-    if (pl.cg == 32) return dispatch_r<Op, IO, VW, 32>(pl, sp, s);
-    return dispatch_r<Op, IO, VW, 8>(pl, sp, s);
+    if (pl.kind == KIND_PIPELINED) {
+        return pl.r == 2 ? launch_pipelined<Op, IO, 4, 2>(sp, s, nullptr)
+                         : launch_pipelined<Op, IO, 4, 4>(sp, s, nullptr);
+    }
+    if (!pl.vec) return dispatch_tile_r<Op, IO, 1, 32>(pl, sp, s);
+    return dispatch_tile_r<Op, IO, VW, 8>(pl, sp, s);
 }
 
 sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void *init,
@@ -164,7 +275,9 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
     std::memset(&sp, 0, sizeof(sp));
     sp.in0 = in0; sp.in1 = in1; sp.init = init; sp.init_bs = init_bs; sp.out = out;
     sp.B = B; sp.T = T; sp.D = D;
-    sp.n_dt = pl.n_dt; sp.n_chains = pl.n_chains; sp.n_chunks = pl.n_chunks;
+    sp.n_dt = pl.n_dt; sp.n_chains = pl.n_chains; sp.n_chunks = pl.n_chunks; sp.n_tiles = pl.n_tiles;
+    sp.by_chains = make_fastdiv(uint32_t(pl.n_chains));
+    sp.by_dt = make_fastdiv(uint32_t(pl.n_dt));
     sp.epoch = 0;
     sp.spin_limit = g_spin_limit.load();
     sp.drop_tile = g_drop_tile.load();
@@ -172,19 +285,17 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
         if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)) return SGR_ERR_WORKSPACE;
         char *w = static_cast<char *>(ws);
         sp.status = reinterpret_cast<uint32_t *>(w);
-        sp.flags = reinterpret_cast<uint64_t *>(w + pl.off_flags);
-        sp.agg = reinterpret_cast<float2 *>(w + pl.off_agg);
-        sp.pref = reinterpret_cast<float *>(w + pl.off_pref);
+        sp.words = reinterpret_cast<uint64_t *>(w + pl.off_words);
         cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
         if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return SGR_ERR_CUDA;
         if (cs == cudaStreamCaptureStatusActive) {
-            // a graph replays its launch arguments: clear the flags inside the
-            // graph so the fixed epoch of captured launches never sees stale words
-            if (cudaMemsetAsync(sp.flags, 0, 8 * size_t(pl.n_tiles), stream) != cudaSuccess)
+            // a graph replays its launch arguments: clear the words inside the
+            // graph so the fixed epoch of captured launches never sees stale ones
+            if (cudaMemsetAsync(sp.words, 0, pl.ws_bytes - pl.off_words, stream) != cudaSuccess)
                 return SGR_ERR_CUDA;
             sp.epoch = 1;
         } else {
-            sp.epoch = g_epoch.fetch_add(1);
+            sp.epoch = next_epoch();
         }
     }
     cudaError_t e;
@@ -301,21 +412,29 @@ sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dty
     if (B < 0 || T < 0 || D < 0 || !plan) return SGR_ERR_INVALID_ARG;
     const Plan p = make_plan(B, T, D, dtype, aligned != 0);
     plan->vector_path = p.vec ? 1 : 0;
+    plan->kernel = p.kind;
     plan->channels_per_thread = p.V;
     plan->channel_lanes = p.cg;
     plan->rows_per_thread = p.r;
-    plan->warps = kWarps;
-    plan->threads = (kWarps + 1) * 32;
+    plan->warps = p.kind == KIND_PIPELINED ? kPipeWarps : kWarps;
+    plan->threads = (plan->warps + 1) * 32;
+    plan->stages = p.stages;
     plan->tile_rows = p.TR;
     plan->tile_channels = p.TC;
     plan->n_channel_tiles = p.n_dt;
     plan->n_chains = p.n_chains;
     plan->n_chunks = p.n_chunks;
     plan->n_tiles = p.n_tiles;
+    plan->smem_bytes = p.smem;
     plan->workspace_bytes = p.ws_bytes;
-    plan->off_flags = p.off_flags;
-    plan->off_agg = p.off_agg;
-    plan->off_pref = p.off_pref;
+    plan->off_words = p.off_words;
+    if (p.n_chains > 0 && p.n_dt > 0 && p.n_chains < (int64_t(1) << 31)) {
+        const FastDiv a = make_fastdiv(uint32_t(p.n_chains)), b = make_fastdiv(uint32_t(p.n_dt));
+        plan->div_chains_m = a.m; plan->div_chains_s = a.s;
+        plan->div_dt_m = b.m; plan->div_dt_s = b.s;
+    } else {
+        plan->div_chains_m = plan->div_chains_s = plan->div_dt_m = plan->div_dt_s = 0;
+    }
     return SGR_OK;
 }
 
@@ -327,6 +446,12 @@ sgr_status_t sgr_set_wait_limit(uint32_t polls) {
 sgr_status_t sgr_set_drop_publish(int64_t tile) {
     if (tile < -1) return SGR_ERR_INVALID_ARG;
     g_drop_tile.store(tile);
+    return SGR_OK;
+}
+
+sgr_status_t sgr_set_kernel_override(int kernel) {
+    if (kernel < KIND_AUTO || kernel > KIND_PIPELINED) return SGR_ERR_INVALID_ARG;
+    g_override_kind.store(kernel);
     return SGR_OK;
 }
 

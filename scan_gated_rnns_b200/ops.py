@@ -163,5 +163,10 @@ def set_tile_override(channel_lanes: int = 0, rows_per_thread: int = 0) -> None:
     check("sgr_set_tile_override", lib().sgr_set_tile_override(channel_lanes, rows_per_thread))
 
 
+def set_kernel_override(kernel: int = 0) -> None:
+    """0 automatic, 1 tile kernel, 2 pipelined kernel (where the fast path applies)."""
+    check("sgr_set_kernel_override", lib().sgr_set_kernel_override(kernel))
+
+
 def version() -> str:
     return lib().sgr_version().decode()

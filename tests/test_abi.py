@@ -109,6 +109,7 @@ def test_workspace_size_and_hooks():
     assert lib.sgr_set_tile_override(3, 0) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_tile_override(0, 3) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_drop_publish(-2) == _abi.SGR_ERR_INVALID_ARG
+    assert lib.sgr_set_kernel_override(3) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_wait_limit(0) == _abi.SGR_OK
     assert lib.sgr_set_drop_publish(-1) == _abi.SGR_OK
     assert lib.sgr_workspace_init(None, 0, None) == _abi.SGR_OK
@@ -129,8 +130,23 @@ def check_plan_indices(B, T, D, dtype, aligned, check_cover):
     assert TR == W * J * R and TC == cg * V and TC % 32 == 0
     assert n_dt == -(-D // TC) and n_chains == B * n_dt and n_chunks == -(-T // TR)
     assert n_tiles == n_chains * n_chunks and n_tiles < 2 ** 31
+    assert pl["threads"] == (W + 1) * 32
+    if pl["kernel"] == _abi.KERNEL_PIPELINED:
+        # persistent blocks: lane l owns channels l V.., warp w owns rows w R..
+        assert pl["vector_path"] and cg * V * esz == 128 and V == 4 and pl["stages"] >= 2
+        assert pl["threads"] % 128 == 0      # whole warps per SM sub-partition
+        assert pl["smem_bytes"] <= 227 * 1024 // 2
     if pl["vector_path"]:
-        assert aligned and D % V == 0 and V * esz == 16
+        assert aligned and D % V == 0 and V * esz in (8, 16)
+    # the kernels divide tile -> (chunk, chain) -> (b, dt) by multiply-high,
+    # add and shift with the host's constants: exact for every tile index
+    ti = np.arange(n_tiles, dtype=np.uint64)
+    fd = lambda n, m, s: ((n * np.uint64(m)) >> np.uint64(32)) + n >> np.uint64(s)
+    cq = fd(ti, pl["div_chains_m"], pl["div_chains_s"])
+    assert (cq == ti // np.uint64(n_chains)).all()
+    ch = np.arange(n_chains, dtype=np.uint64)
+    assert (fd(ch, pl["div_dt_m"], pl["div_dt_s"]) == ch // np.uint64(n_dt)).all()
+    # every (tile, warp, lane) piece, whichever block processes the tile
     tile = np.arange(n_tiles, dtype=np.int64)[:, None, None]
     warp = np.arange(W, dtype=np.int64)[None, :, None]
     lane = np.arange(32, dtype=np.int64)[None, None, :]
@@ -150,21 +166,18 @@ def check_plan_indices(B, T, D, dtype, aligned, check_cover):
             dv = np.broadcast_to(d0, valid.shape)[valid]
             assert (dv + V <= D).all()
             if pl["vector_path"]:
-                assert ((idx * esz) % 16 == 0).all()
+                assert ((idx * esz) % (V * esz) == 0).all()
             if check_cover:
                 for v in range(V):
                     np.add.at(cover, idx + v, 1)
     if check_cover:
         assert (cover == 1).all(), "every output element is written exactly once"
-    # carry warp: channel slots, flags and summaries inside their regions
+    # carry warp: lane l owns channels [l CV, l CV + CV); hand-off words inside the workspace
     CV = TC // 32
     assert (np.arange(32) * CV + CV - 1 < TC).all()
     if n_chunks > 1:
-        assert pl["off_flags"] >= 4
-        assert pl["off_flags"] + 8 * n_tiles <= pl["off_agg"]
-        assert pl["off_agg"] + 8 * n_tiles * TC <= pl["off_pref"]
-        assert pl["off_pref"] + 4 * n_tiles * TC <= pl["workspace_bytes"]
-        assert pl["off_agg"] % 16 == 0 and pl["off_pref"] % 16 == 0 and pl["off_flags"] % 8 == 0
+        assert pl["off_words"] >= 4 and pl["off_words"] % 8 == 0
+        assert pl["off_words"] + 8 * 3 * TC * n_tiles <= pl["workspace_bytes"]
         assert _abi.lib().sgr_workspace_size(MINGRU, B, T, D, dtype) >= pl["workspace_bytes"]
     else:
         assert pl["workspace_bytes"] == 0
@@ -177,14 +190,17 @@ SMALL_SHAPES = [(2, 1024, 512), (3, 1000, 96), (1, 777, 36), (2, 300, 7), (1, 1,
 @pytest.mark.parametrize("shape", SMALL_SHAPES)
 @pytest.mark.parametrize("dtype", [F32, BF16])
 @pytest.mark.parametrize("aligned", [True, False])
-@pytest.mark.parametrize("override", [(0, 0), (8, 1), (8, 8), (32, 2), (32, 4)])
+@pytest.mark.parametrize("override", [(0, 0, 0), (1, 0, 1), (1, 0, 2), (1, 0, 4), (1, 0, 8),
+                                      (2, 0, 2), (2, 0, 4)])
 def test_plan_indices_small(shape, dtype, aligned, override):
     lib = _abi.lib()
-    assert lib.sgr_set_tile_override(*override) == 0
+    assert lib.sgr_set_kernel_override(override[0]) == 0
+    assert lib.sgr_set_tile_override(*override[1:]) == 0
     try:
         check_plan_indices(*shape, dtype, aligned, check_cover=True)
     finally:
         lib.sgr_set_tile_override(0, 0)
+        lib.sgr_set_kernel_override(0)
 
 
 @pytest.mark.parametrize("name", sorted(WORKLOADS))

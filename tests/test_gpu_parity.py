@@ -58,8 +58,13 @@ def _reset_hooks():
     yield
     lib = _abi.lib()
     lib.sgr_set_tile_override(0, 0)
+    lib.sgr_set_kernel_override(0)
     lib.sgr_set_wait_limit(0)
     lib.sgr_set_drop_publish(-1)
+
+
+# (kernel, rows per thread): the tile kernel and the pipelined kernel, every R
+VARIANTS = [(1, 1), (1, 2), (1, 4), (1, 8), (2, 2), (2, 4)]
 
 
 # ------------------------------------------------------------------ minGRU
@@ -78,11 +83,15 @@ def test_mingru_matches_oracle(shape, dtype, init):
     assert rel_err(h, ref_log) <= TOL[dtype]
 
 
-@pytest.mark.parametrize("cg,r", [(8, 1), (8, 2), (8, 4), (8, 8), (32, 1), (32, 2), (32, 4), (32, 8)])
+@pytest.mark.parametrize("kernel,r", VARIANTS)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_mingru_every_tile_shape(cg, r, dtype):
-    sgr.set_tile_override(cg, r)
-    k, hx, h0 = small("mingru", 3, 1500, 160, dtype, "u01_1", seed=cg * 10 + r)
+@pytest.mark.parametrize("shape", [(3, 1500, 160), (2, 3001, 384)])
+def test_mingru_every_kernel_and_tile_shape(kernel, r, dtype, shape):
+    sgr.set_kernel_override(kernel)
+    sgr.set_tile_override(0, r)
+    k, hx, h0 = small("mingru", *shape, dtype, "u01_1", seed=kernel * 10 + r)
+    pl = _abi.plan(0, *shape, 0 if dtype == "f32" else 1, True)
+    assert pl["kernel"] == kernel and pl["n_chunks"] > 1
     h = run("mingru", k, hx, h0)
     assert rel_err(h, oracle.mingru_linear(k, hx, h0, threads=8)) <= TOL[dtype]
 
@@ -186,15 +195,17 @@ def test_graph_capture_replays():
         assert rel_err(y, oracle.mingru_linear(k, hx, h0, threads=8)) <= TOL["f32"]
 
 
-def test_bounded_wait_reports_timeout():
+@pytest.mark.parametrize("kernel,D", [(1, 64), (2, 64)])
+def test_bounded_wait_reports_timeout(kernel, D):
     # chunk 0 of channel tile 0 skips publishing its state: the next chunk of the
     # same channels waits until the poll limit, records the timeout and writes
     # NaN; every other channel tile is unaffected
-    B, T, D = 1, 2048, 64
+    B, T = 1, 2048
     k, hx, h0 = small("mingru", B, T, D, "f32", "u01_1", seed=31)
-    sgr.set_tile_override(8, 1)                   # 32 channels x 32 rows per tile
+    sgr.set_kernel_override(kernel)
+    sgr.set_tile_override(0, 1 if kernel == 1 else 2)
     pl = _abi.plan(0, B, T, D, 0, True)
-    assert pl["n_chunks"] > 2 and pl["n_chains"] == 2
+    assert pl["kernel"] == kernel and pl["n_chunks"] > 2 and pl["n_chains"] == 2
     ws = sgr.Workspace(pl["workspace_bytes"], DEV)
     lib = _abi.lib()
     lib.sgr_set_wait_limit(2000)
@@ -253,10 +264,12 @@ def test_minmax_bit_exact(shape, dtype, init):
     assert exact(x, oracle.minmax(r, s, x0, threads=8))
 
 
-@pytest.mark.parametrize("cg,rr", [(8, 1), (8, 4), (8, 8), (32, 1), (32, 8)])
-def test_minmax_every_tile_shape(cg, rr):
-    sgr.set_tile_override(cg, rr)
-    r, s, x0 = small("minmax", 3, 1500, 160, "f32", "u01_1", seed=cg + rr)
+@pytest.mark.parametrize("kernel,rr", VARIANTS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_minmax_every_kernel_and_tile_shape(kernel, rr, dtype):
+    sgr.set_kernel_override(kernel)
+    sgr.set_tile_override(0, rr)
+    r, s, x0 = small("minmax", 3, 2500, 160, dtype, "u01_1", seed=kernel + rr)
     assert exact(run("minmax", r, s, x0), oracle.minmax(r, s, x0, threads=8))
 
 
