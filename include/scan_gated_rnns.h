@@ -148,6 +148,25 @@ SGR_API sgr_status_t mingru_step(const void *k_t, int64_t k_batch_stride,
                          int64_t B, int64_t D, sgr_dtype_t dtype,
                          cudaStream_t stream);
 
+/*
+ * mingru_scan_noalloc -- mingru_scan for callers that cannot allocate device
+ * memory where they call it (an inference runtime's plugin whose enqueue step
+ * must not allocate, a process with a fixed device-memory plan, code running
+ * while its stream is captured).  There is no counterpart on the pages: this
+ * is a deployment convenience of this library.  Arguments and result are those
+ * of mingru_scan minus the workspace: the scratch comes from a 16 MiB array
+ * inside the library (held by every GPU that loads it, until exit).  Shapes
+ * whose scratch (sgr_workspace_size) exceeds 16 MiB return
+ * SGR_ERR_WORKSPACE.  The first call on a device looks up the array's device
+ * address and zero-fills it on `stream`, so make it before any stream capture.
+ * All calls on a device share the array: calls whose kernels can overlap on
+ * the GPU race and must not be made.
+ */
+SGR_API sgr_status_t mingru_scan_noalloc(const void *k, const void *hx,
+                                         const void *h0, int64_t h0_batch_stride,
+                                         void *h, int64_t B, int64_t T, int64_t D,
+                                         sgr_dtype_t dtype, cudaStream_t stream);
+
 /* ------------------------------------------------------------ workspace */
 
 /* Bytes of workspace a scan of this shape needs (0: none).  Pure host code. */

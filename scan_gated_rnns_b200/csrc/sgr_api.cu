@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cstring>
 #include <limits>
+#include <mutex>
 
 namespace {
 
@@ -466,3 +467,61 @@ sgr_status_t sgr_set_tile_override(int channel_lanes, int rows_per_thread) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// mingru_scan without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// scan: an inference runtime's plugin whose enqueue step must not call the
+// allocator (allocation can block or fail in the middle of a run), a process
+// with a fixed, pre-planned device-memory budget, or code that runs while its
+// stream is being captured and must not make allocation calls there.  For
+// them this entry point takes its scratch (the chunk hand-off words and the
+// status word) from a fixed array that lives in the library itself.
+//
+// The array is kNoAllocScratchBytes (16 MiB) of device memory, held by every
+// GPU that loads the library until the process exits.  The first call on a
+// device looks up the array's device address (cudaGetSymbolAddress, with that
+// device current) and zero-fills it on the caller's stream; that first call
+// should therefore come before any stream capture.  All calls on a device
+// share the one array and it keeps the last call's contents; every launch tags
+// its words with a fresh epoch, so nothing needs clearing between calls, but
+// calls whose kernels can overlap on the GPU (e.g. on two streams without an
+// ordering between them) race on the array and must not be made.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[64] = {};
+
+}  // namespace
+
+extern "C" sgr_status_t mingru_scan_noalloc(const void *k, const void *hx, const void *h0,
+                                            int64_t h0_batch_stride, void *h, int64_t B,
+                                            int64_t T, int64_t D, sgr_dtype_t dtype,
+                                            cudaStream_t stream) {
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || D < 0 || h0_batch_stride < 0) return SGR_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || D == 0) return SGR_OK;
+    // scratch this shape needs, for whichever kernel variant the call takes
+    const size_t need = sgr_workspace_size(SGR_OP_MINGRU, B, T, D, dtype);
+    if (need > kNoAllocScratchBytes) return SGR_ERR_WORKSPACE;
+    void *ws = nullptr;
+    if (need > 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SGR_ERR_CUDA;
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (g_noalloc_ptr[dev] == nullptr) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+                return SGR_ERR_CUDA;
+            if (cudaMemsetAsync(p, 0, kNoAllocScratchBytes, stream) != cudaSuccess) return SGR_ERR_CUDA;
+            g_noalloc_ptr[dev] = p;
+        }
+        ws = g_noalloc_ptr[dev];
+    }
+    return mingru_scan(k, hx, h0, h0_batch_stride, h, B, T, D, dtype, ws,
+                       ws ? kNoAllocScratchBytes : 0, stream);
+}
