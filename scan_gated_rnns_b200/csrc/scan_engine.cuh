@@ -41,6 +41,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda.h>
 #include <stdint.h>
 
 #include <type_traits>
@@ -303,77 +304,111 @@ __device__ __forceinline__ void publish_state(const ScanParams &p, int64_t tile,
 // neither is waited for (bounded, with back-off).  Before chunk 0 the state is
 // the initial state.  Each lane works alone: its channels' words carry their
 // own validity.
+template <int CV>
+constexpr int window_len() { return CV >= 4 ? 1 : (CV == 2 ? 2 : 4); }
+
+template <int CV, int TC>
+struct LookWindow {
+    static constexpr int K = window_len<CV>();
+    uint64_t wa[K][CV], wb[K][CV], ws[K][CV];
+};
+
+// issue the loads of the words of chunks q, q-1, ..., q-K+1
+template <int CV, int TC>
+__device__ __forceinline__ void load_window(const ScanParams &p, int64_t q, int64_t chain, int ch,
+                                            LookWindow<CV, TC> &win) {
+#pragma unroll
+    for (int i = 0; i < LookWindow<CV, TC>::K; ++i) {
+        const int64_t qq = q - i;
+        if (qq >= 0) {
+            const uint64_t *w = p.words + (qq * p.n_chains + chain) * 3 * TC + ch;
+#pragma unroll
+            for (int v = 0; v < CV; ++v) {
+                win.ws[i][v] = ld_relaxed_u64(w + 2 * TC + v);
+                win.wa[i][v] = ld_relaxed_u64(w + v);
+                win.wb[i][v] = ld_relaxed_u64(w + TC + v);
+            }
+        }
+    }
+}
+
+// Walk a loaded window starting at chunk q with the running composite M.
+// Returns true when the incoming state is known (hin set); otherwise the
+// number of chunks folded in is in `consumed`.
 template <class Op, typename IO, int CV, int TC>
-__device__ void look_back(const ScanParams &p, int64_t c, int64_t chain, int64_t b, int64_t d_first,
-                          int ch, float (&hin)[CV]) {
-    constexpr int K = CV >= 4 ? 1 : (CV == 2 ? 2 : 4);
+__device__ __forceinline__ bool resolve_window(const ScanParams &p, int64_t q, const LookWindow<CV, TC> &win,
+                                               int64_t b, int64_t d_first, float2 (&M)[CV],
+                                               float (&hin)[CV], int &consumed) {
+    consumed = 0;
+    bool done = false, stop = false;
+#pragma unroll
+    for (int i = 0; i < LookWindow<CV, TC>::K; ++i) {
+        if (done || stop) continue;
+        const int64_t qq = q - i;
+        if (qq < 0) {
+#pragma unroll
+            for (int v = 0; v < CV; ++v)
+                hin[v] = Op::apply(M[v], load_init<IO>(p, b, d_first + v, Op::default_init()));
+            done = true;
+            continue;
+        }
+        bool s_ok = true, ab_ok = true;
+#pragma unroll
+        for (int v = 0; v < CV; ++v) {
+            s_ok = s_ok && word_valid(win.ws[i][v], p.epoch);
+            ab_ok = ab_ok && word_valid(win.wa[i][v], p.epoch) && word_valid(win.wb[i][v], p.epoch);
+        }
+        if (s_ok) {
+#pragma unroll
+            for (int v = 0; v < CV; ++v) hin[v] = Op::apply(M[v], word_value(win.ws[i][v]));
+            done = true;
+        } else if (ab_ok) {
+#pragma unroll
+            for (int v = 0; v < CV; ++v)
+                M[v] = Op::combine(make_float2(word_value(win.wa[i][v]), word_value(win.wb[i][v])), M[v]);
+            consumed = i + 1;
+        } else {
+            stop = true;
+        }
+    }
+    return done;
+}
+
+// Finish a look-back whose first window (chunks c-1 ...) is already loaded.
+template <class Op, typename IO, int CV, int TC>
+__device__ void look_back_from(const ScanParams &p, int64_t c, int64_t chain, int64_t b, int64_t d_first,
+                               int ch, LookWindow<CV, TC> &win, float (&hin)[CV]) {
     float2 M[CV];
 #pragma unroll
     for (int v = 0; v < CV; ++v) M[v] = Op::identity();
     int64_t q = c - 1;
     uint32_t polls = 0, ns = 32;
     while (true) {
-        uint64_t wa[K][CV], wb[K][CV], ws[K][CV];
-#pragma unroll
-        for (int i = 0; i < K; ++i) {
-            const int64_t qq = q - i;
-            if (qq >= 0) {
-                const uint64_t *w = p.words + (qq * p.n_chains + chain) * 3 * TC + ch;
-#pragma unroll
-                for (int v = 0; v < CV; ++v) {
-                    ws[i][v] = ld_relaxed_u64(w + 2 * TC + v);
-                    wa[i][v] = ld_relaxed_u64(w + v);
-                    wb[i][v] = ld_relaxed_u64(w + TC + v);
-                }
-            }
-        }
-        int consumed = 0;
-        bool done = false, stop = false;
-#pragma unroll
-        for (int i = 0; i < K; ++i) {
-            if (done || stop) continue;
-            const int64_t qq = q - i;
-            if (qq < 0) {
-#pragma unroll
-                for (int v = 0; v < CV; ++v)
-                    hin[v] = Op::apply(M[v], load_init<IO>(p, b, d_first + v, Op::default_init()));
-                done = true;
-                continue;
-            }
-            bool s_ok = true, ab_ok = true;
-#pragma unroll
-            for (int v = 0; v < CV; ++v) {
-                s_ok = s_ok && word_valid(ws[i][v], p.epoch);
-                ab_ok = ab_ok && word_valid(wa[i][v], p.epoch) && word_valid(wb[i][v], p.epoch);
-            }
-            if (s_ok) {
-#pragma unroll
-                for (int v = 0; v < CV; ++v) hin[v] = Op::apply(M[v], word_value(ws[i][v]));
-                done = true;
-            } else if (ab_ok) {
-#pragma unroll
-                for (int v = 0; v < CV; ++v)
-                    M[v] = Op::combine(make_float2(word_value(wa[i][v]), word_value(wb[i][v])), M[v]);
-                consumed = i + 1;
-            } else {
-                stop = true;
-            }
-        }
-        if (done) return;
+        int consumed;
+        if (resolve_window<Op, IO, CV, TC>(p, q, win, b, d_first, M, hin, consumed)) return;
         if (consumed > 0) {
             q -= consumed;
             ns = 32;
-            continue;
-        }
-        if (++polls > p.spin_limit) {
-            atomicOr(p.status, kTimeoutBit);
+        } else {
+            if (++polls > p.spin_limit) {
+                atomicOr(p.status, kTimeoutBit);
 #pragma unroll
-            for (int v = 0; v < CV; ++v) hin[v] = __int_as_float(0x7fffffff);
-            return;
+                for (int v = 0; v < CV; ++v) hin[v] = __int_as_float(0x7fffffff);
+                return;
+            }
+            __nanosleep(ns);
+            ns = ns < 256 ? ns * 2 : 256;
         }
-        __nanosleep(ns);
-        ns = ns < 1024 ? ns * 2 : 1024;
+        load_window<CV, TC>(p, q, chain, ch, win);
     }
+}
+
+template <class Op, typename IO, int CV, int TC>
+__device__ __forceinline__ void look_back(const ScanParams &p, int64_t c, int64_t chain, int64_t b,
+                                          int64_t d_first, int ch, float (&hin)[CV]) {
+    LookWindow<CV, TC> win;
+    load_window<CV, TC>(p, c - 1, chain, ch, win);
+    look_back_from<Op, IO, CV, TC>(p, c, chain, b, d_first, ch, win, hin);
 }
 
 // The carry of one tile, as done by the carry warp: fold the W warp totals in
@@ -548,77 +583,115 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const Sca
 
 // --------------------------------------------------- pipelined kernel
 //
-// Persistent blocks (co-resident, cooperative launch), each owning tiles
-// blockIdx.x, blockIdx.x + gridDim.x, ... in order.  A tile is TR x TC with
-// TC = CG * V channels and TR = W * J * R rows (J = 32 / CG row groups per
-// warp): lane (g, j) = (lane % CG, lane / CG) of warp w owns channels
-// [g V, g V + V) of rows [(w J + j) R, (w J + j) R + R).  V = 4 (16-byte fp32
-// or 8-byte bf16 vectors).  Narrow tiles keep the chunk hand-off cheap: the
-// chunks of one channel tile that are in flight at once number about
-// gridDim.x / n_chains, and a look-back folds that many summaries of TC
-// channels each.
+// Persistent blocks (co-resident, cooperative launch, two per SM), each owning
+// tiles blockIdx.x, blockIdx.x + gridDim.x, ... in order.  7 data warps and
+// one carry warp.  A tile is TR x TC with TC = CG * V channels (V = 4) and
+// TR = W * J * R rows (J = 32 / CG row groups per warp): lane (g, j) =
+// (lane % CG, lane / CG) of warp w owns channels [g V, g V + V) of rows
+// [(w J + j) R, (w J + j) R + R).  Narrow tiles (128-byte rows) keep the chunk
+// hand-off cheap: about gridDim.x / n_chains chunks of one channel tile are in
+// flight at once, and a look-back folds that many summaries of TC channels.
 //
-// Loads: each data thread streams its own vector pieces of the next S tiles
-// into a private slice of a shared-memory ring with cp.async (no registers
-// held, no cross-thread hand-off: a thread only reads what it copied), one
-// commit group per tile, so S tiles of HBM reads are always in flight.
+// Loads: the tensor memory accelerator copies whole tiles (box TC x TR x 1 of
+// the (D, T, B) tensor) of both operands into an S-slot shared-memory ring,
+// an mbarrier per slot counting the bytes in.  The carry warp issues the
+// first S tiles; afterwards the last data warp to finish reading a slot (a
+// shared counter per slot) issues the next tile into it at once.  Rows past T
+// and channels past D arrive as zeros and are replaced by the operator's
+// identity inputs in registers.  No multicast.
 //
 // Compute, with a one-tile lag: phase A of tile n (activations, the thread's
 // fold over its R rows, the scan across the warp's J row groups, the warp's
 // summary to shared memory; pairs and the thread's exclusive prefix stay in
 // registers), then phase B of tile n-1 (replay from the thread's incoming
-// state, store).  The carry warp runs the hand-off of tile n while the data
-// warps are in phase A of tile n+1, so the look-back latency is overlapped
-// with loads and compute.  Shared summaries and named barriers are
-// double-buffered by tile parity:
+// state, streaming stores).
+//
+// Carry warp: the hand-off of tile n runs while the data warps are in phase A
+// of tile n+1; the loads of tile n+1's look-back window are issued as soon as
+// tile n is released, so the round trip overlaps the wait for tile n+1's
+// summaries.  Named barriers and summaries are double-buffered by tile parity:
 //   barrier 1 + (n & 1): data warps arrive (summaries of tile n written),
 //                        carry warp waits;
 //   barrier 3 + (n & 1): carry warp arrives (incoming states of tile n
-//                        written), data warps wait.
-// Every wait is for a tile with a smaller index and blocks are co-resident,
-// so the smallest unfinished tile can always progress.
+//                        written), data warps wait (phase B of n).
+// Data warps reach phase A of n only after phase B of n-2, which the carry
+// warp released before it waited for tile n-1: no cycle.  Every look-back
+// wait is for a tile with a smaller index and blocks are co-resident, so the
+// smallest unfinished tile can always progress.
 template <typename IO, int V, int CG, int R, int S, int W>
 struct PipeShape {
-    static constexpr int NTD = W * 32;                       // data threads
     static constexpr int J = 32 / CG;
     static constexpr int TC = CG * V;
     static constexpr int TR = W * J * R;
-    static constexpr int VB = V * int(sizeof(IO));           // bytes per vector
-    static constexpr size_t stage_bytes = size_t(R) * 2 * NTD * VB;
-    static constexpr size_t tot_bytes = size_t(2) * W * TC * sizeof(float2);
-    static constexpr size_t smem_bytes = S * stage_bytes + tot_bytes;
+    static constexpr size_t op_bytes = size_t(TR) * TC * sizeof(IO);     // one operand of a tile
+    static constexpr size_t slot_bytes = 2 * op_bytes;
+    static constexpr size_t bar_offset = S * slot_bytes;
+    static constexpr size_t cnt_offset = bar_offset + S * 8;          // per-slot reader counts
+    static constexpr size_t tot_offset = (cnt_offset + S * 4 + 15) / 16 * 16;
+    static constexpr size_t smem_bytes = tot_offset + size_t(2) * W * TC * sizeof(float2);
 };
 
-template <int BYTES> __device__ __forceinline__ void cp_async(void *smem, const void *gmem);
-template <> __device__ __forceinline__ void cp_async<16>(void *smem, const void *gmem) {
-    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-template <> __device__ __forceinline__ void cp_async<8>(void *smem, const void *gmem) {
-    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(s), "l"(gmem) : "memory");
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+// bounded wait for a phase of an mbarrier; false if it did not complete
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+// 3-D tiled tensor load into this block's shared memory, completion counted
+// on an mbarrier (plain load: no cluster multicast)
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+// bound on mbarrier polls (each try_wait may suspend the thread for up to a
+// microsecond or so); after one wait has run out, later waits of the thread
+// make a single poll, so a broken copy cannot stretch the kernel to n_local
+// full bounds
+constexpr uint32_t kMbarLimit = 1u << 16;
 
 template <class Op, typename IO, int V, int CG, int R, int S, int W, int MINB>
-__global__ void __launch_bounds__((W + 1) * 32, MINB) scan_pipelined_kernel(const ScanParams p) {
+__global__ void __launch_bounds__((W + 1) * 32, MINB)
+scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap map0,
+                      const __grid_constant__ CUtensorMap map1) {
     using Shape = PipeShape<IO, V, CG, R, S, W>;
     using Vec = typename VecOf<IO, V>::type;
     constexpr int J = Shape::J;
     constexpr int TC = Shape::TC;
     constexpr int TR = Shape::TR;
-    constexpr int NTD = Shape::NTD;
-    constexpr int VB = Shape::VB;
     constexpr int CV = TC / 32;
     constexpr uint32_t NT = (W + 1) * 32;
-    static_assert(sizeof(Vec) == VB, "vector type matches the vector width");
+    static_assert(sizeof(Vec) == V * sizeof(IO), "vector type matches the vector width");
     static_assert(CG * J == 32 && TC % 32 == 0, "lane layout");
+    static_assert(TC * sizeof(IO) % 16 == 0 && TC <= 256 && TR <= 256, "TMA box");
 
-    extern __shared__ __align__(16) unsigned char smem[];
-    Vec *ring = reinterpret_cast<Vec *>(smem);                             // [S][R][2][NTD]
-    float2 (*s_tot)[W][TC] = reinterpret_cast<float2 (*)[W][TC]>(smem + S * Shape::stage_bytes);
+    extern __shared__ __align__(128) unsigned char smem[];
+    float2 (*s_tot)[W][TC] = reinterpret_cast<float2 (*)[W][TC]>(smem + Shape::tot_offset);
+    unsigned int *s_cnt = reinterpret_cast<unsigned int *>(smem + Shape::cnt_offset);
+    const uint32_t ring = smem_addr(smem);
+    const uint32_t bars = ring + uint32_t(Shape::bar_offset);
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -626,76 +699,86 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_pipelined_kernel(cons
     const int64_t first = blockIdx.x;
     const int n_local = int((p.n_tiles - first + G - 1) / G);
 
+    // TMA copy of tile n into ring slot n % S (one thread)
+    auto issue_tile = [&](int n) {
+        const TileCoord tc = tile_coord(p, uint32_t(first + int64_t(n) * G));
+        const uint32_t slot = ring + uint32_t((n % S) * Shape::slot_bytes);
+        const uint32_t bar = bars + 8u * uint32_t(n % S);
+        const int x = int(tc.dt) * TC, y = int(tc.c) * TR, z = int(tc.b);
+        mbar_expect_tx(bar, uint32_t(Shape::slot_bytes));
+        tma_load_3d(slot, &map0, x, y, z, bar);
+        tma_load_3d(slot + uint32_t(Shape::op_bytes), &map1, x, y, z, bar);
+    };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(bars + 8u * s, 1);
+            s_cnt[s] = 0;
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (warp == W && lane == 0) {
+        for (int s = 0; s < S && s < n_local; ++s) issue_tile(s);
+    }
+
     if (warp < W) {
         // ============================================== data warps
-        const int tid = threadIdx.x;
         const int g = lane % CG;
         const int j = lane / CG;
-        const IO *in0 = static_cast<const IO *>(p.in0);
-        const IO *in1 = static_cast<const IO *>(p.in1);
         IO *out = static_cast<IO *>(p.out);
-
-        // global position of this thread's piece of tile n
-        auto locate = [&](int n, int64_t &base, int64_t &row0, bool &dvalid) {
-            const TileCoord tc = tile_coord(p, uint32_t(first + int64_t(n) * G));
-            const int64_t d0 = int64_t(tc.dt) * TC + g * V;
-            dvalid = d0 < p.D;
-            row0 = int64_t(tc.c) * TR + (warp * J + j) * R;
-            base = (int64_t(tc.b) * p.T) * p.D + d0;
-        };
-        auto issue = [&](int n) {
-            if (n < n_local) {
-                int64_t base, row0;
-                bool dvalid;
-                locate(n, base, row0, dvalid);
-                Vec *slot = ring + (n % S) * (R * 2 * NTD) + tid;
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const int64_t t = row0 + r;
-                    if (dvalid && t < p.T) {
-                        cp_async<VB>(slot + (r * 2 + 0) * NTD, in0 + base + t * p.D);
-                        cp_async<VB>(slot + (r * 2 + 1) * NTD, in1 + base + t * p.D);
-                    }
-                }
-            }
-            cp_async_commit();   // one group per tile, empty past the end
-        };
 
         float2 P[2][R][V];   // pairs of the two tiles in flight (tile parity)
         float2 E[2][V];      // the thread's exclusive prefix within its warp
+        int64_t base[2];     // global offset of the thread's first element of the tile
+        int row0[2];         // first row (along T) of the thread's rows
+        bool dvalid[2];
+        uint32_t wait_limit = kMbarLimit;
 
-        // phase A of tile n into register buffer BUF
         auto phaseA = [&](int n, auto bufc) {
             constexpr int BUF = decltype(bufc)::value;
-            cp_async_wait<S - 1>();   // this thread's pieces of tile n have landed
-            int64_t base, row0;
-            bool dvalid;
-            locate(n, base, row0, dvalid);
-            const Vec *slot = ring + (n % S) * (R * 2 * NTD) + tid;
+            const TileCoord tc = tile_coord(p, uint32_t(first + int64_t(n) * G));
+            const int64_t d0 = int64_t(tc.dt) * TC + g * V;
+            dvalid[BUF] = d0 < p.D;
+            row0[BUF] = int(tc.c) * TR + (warp * J + j) * R;
+            base[BUF] = (int64_t(tc.b) * p.T) * p.D + d0;
+            if (!mbar_wait(bars + 8u * uint32_t(n % S), uint32_t((n / S) & 1), wait_limit)) {
+                wait_limit = 1;
+                if (lane == 0) atomicOr(p.status, kTimeoutBit);
+            }
+            const IO *t0 = reinterpret_cast<const IO *>(smem + (n % S) * Shape::slot_bytes);
+            const IO *t1 = t0 + TR * TC;
+            const int lr = (warp * J + j) * R;      // first local row
             float2 incl[V];
 #pragma unroll
             for (int v = 0; v < V; ++v) incl[v] = Op::identity();
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 float x0[V], x1[V];
-                const int64_t t = row0 + r;
-                if (dvalid && t < p.T) {
-                    unpack(slot[(r * 2 + 0) * NTD], x0);
-                    unpack(slot[(r * 2 + 1) * NTD], x1);
-                } else {
-#pragma unroll
-                    for (int v = 0; v < V; ++v) { x0[v] = Op::pad0(); x1[v] = Op::pad1(); }
-                }
+                const bool ok = dvalid[BUF] && (row0[BUF] + r < p.T);
+                unpack(*reinterpret_cast<const Vec *>(t0 + (lr + r) * TC + g * V), x0);
+                unpack(*reinterpret_cast<const Vec *>(t1 + (lr + r) * TC + g * V), x1);
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
                     float e0, e1;
-                    Op::element(x0[v], x1[v], e0, e1);
+                    Op::element(ok ? x0[v] : Op::pad0(), ok ? x1[v] : Op::pad1(), e0, e1);
                     P[BUF][r][v] = make_float2(e0, e1);
                     incl[v] = Op::combine(incl[v], P[BUF][r][v]);
                 }
             }
-            // the ring slot is consumed: refill it with tile n + S
-            issue(n + S);
+            // the warp is done with the slot; the last of the W warps refills it
+            // with tile n + S (its values are in registers, consumed above)
+            __syncwarp();
+            if (lane == 0) {
+                const unsigned int seen = atomicAdd(&s_cnt[n % S], 1u);
+                if (seen == W - 1) {
+                    s_cnt[n % S] = 0;
+                    if (n + S < n_local) {
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        issue_tile(n + S);
+                    }
+                }
+            }
             // scan across the J row groups of the warp
 #pragma unroll
             for (int off = 1; off < J; off <<= 1) {
@@ -721,12 +804,8 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_pipelined_kernel(cons
             named_barrier_arrive(1 + BUF, NT);
         };
 
-        // phase B of tile n from register buffer BUF
-        auto phaseB = [&](int n, auto bufc) {
+        auto phaseB = [&](auto bufc) {
             constexpr int BUF = decltype(bufc)::value;
-            int64_t base, row0;
-            bool dvalid;
-            locate(n, base, row0, dvalid);
             named_barrier_sync(3 + BUF, NT);
             float st[V];
 #pragma unroll
@@ -739,36 +818,88 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_pipelined_kernel(cons
                     st[v] = Op::step(P[BUF][r][v].x, P[BUF][r][v].y, st[v]);
                     y[v] = st[v];
                 }
-                const int64_t t = row0 + r;
-                if (dvalid && t < p.T) Access<IO, V>::store(out + base + t * p.D, y);
+                if (dvalid[BUF] && row0[BUF] + r < p.T)
+                    Access<IO, V>::store(out + base[BUF] + int64_t(row0[BUF] + r) * p.D, y);
             }
         };
 
         using B0 = std::integral_constant<int, 0>;
         using B1 = std::integral_constant<int, 1>;
-        for (int s = 0; s < S; ++s) issue(s);
         int n = 0;
         for (; n + 1 < n_local; n += 2) {
             phaseA(n, B0{});
-            if (n >= 1) phaseB(n - 1, B1{});
+            if (n >= 1) phaseB(B1{});
             phaseA(n + 1, B1{});
-            phaseB(n, B0{});
+            phaseB(B0{});
         }
         if (n < n_local) {
             phaseA(n, B0{});
-            if (n >= 1) phaseB(n - 1, B1{});
-            phaseB(n, B0{});
+            if (n >= 1) phaseB(B1{});
+            phaseB(B0{});
         } else if (n_local >= 1) {
-            phaseB(n - 1, B1{});
+            phaseB(B1{});
         }
-        cp_async_wait<0>();
     } else {
         // ============================================== carry warp
+        // Per tile: fold the warp summaries, publish the chunk summary,
+        // resolve the incoming state from the look-back window, write each
+        // warp's incoming state, release the data warps, publish the chunk's
+        // final state, and issue the loads of the next tile's look-back window
+        // (they read other blocks' words, so they fly while this warp waits
+        // for the next tile's summaries).
+        const int ch = lane * CV;
+        LookWindow<CV, TC> win;
+        float init[CV];
+        auto prefetch = [&](int n) {
+            const TileCoord tc = tile_coord(p, uint32_t(first + int64_t(n) * G));
+            if (tc.c == 0) {
+#pragma unroll
+                for (int v = 0; v < CV; ++v)
+                    init[v] = load_init<IO>(p, tc.b, int64_t(tc.dt) * TC + ch + v, Op::default_init());
+            } else {
+                load_window<CV, TC>(p, int64_t(tc.c) - 1, tc.chain, ch, win);
+            }
+        };
+        if (n_local > 0) prefetch(0);
         for (int n = 0; n < n_local; ++n) {
-            const int buf = n & 1;
-            named_barrier_sync(1 + buf, NT);
-            carry_tile<Op, IO, CV, TC, W>(p, first + int64_t(n) * G, s_tot[buf], lane,
-                                          [&] { named_barrier_arrive(3 + buf, NT); });
+            const int PB = n & 1;
+            named_barrier_sync(1 + PB, NT);
+            const int64_t tile = first + int64_t(n) * G;
+            const TileCoord tc = tile_coord(p, uint32_t(tile));
+            const int64_t c = tc.c;
+            const int64_t dl = int64_t(tc.dt) * TC + ch;
+            float2 total[CV];
+#pragma unroll
+            for (int v = 0; v < CV; ++v) total[v] = Op::identity();
+            for (int w = 0; w < W; ++w) {
+#pragma unroll
+                for (int v = 0; v < CV; ++v) {
+                    const float2 t = s_tot[PB][w][ch + v];
+                    s_tot[PB][w][ch + v] = total[v];       // exclusive prefix over warps
+                    total[v] = Op::combine(total[v], t);
+                }
+            }
+            const bool publish = (p.n_chunks > 1) && (c < p.n_chunks - 1) && (tile != p.drop_tile);
+            float hin[CV];
+            if (c == 0) {
+#pragma unroll
+                for (int v = 0; v < CV; ++v) hin[v] = init[v];
+            } else {
+                if (publish) publish_summary<CV, TC>(p, tile, ch, total);
+                look_back_from<Op, IO, CV, TC>(p, c, tc.chain, tc.b, dl, ch, win, hin);
+            }
+            for (int w = 0; w < W; ++w) {
+#pragma unroll
+                for (int v = 0; v < CV; ++v) s_tot[PB][w][ch + v].x = Op::apply(s_tot[PB][w][ch + v], hin[v]);
+            }
+            named_barrier_arrive(3 + PB, NT);
+            if (publish) {
+                float fin[CV];
+#pragma unroll
+                for (int v = 0; v < CV; ++v) fin[v] = Op::apply(total[v], hin[v]);
+                publish_state<CV, TC>(p, tile, ch, fin);
+            }
+            if (n + 1 < n_local) prefetch(n + 1);
         }
     }
 }

@@ -71,6 +71,43 @@ template <typename IO> constexpr int pipe_cg() { return sizeof(IO) == 4 ? 8 : 16
 template <typename IO, int R>
 constexpr size_t pipe_smem() { return PipeShape<IO, 4, pipe_cg<IO>(), R, kStages, kPipeWarps>::smem_bytes; }
 
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime
+// (no link-time dependency on the driver library)
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn() {
+    static std::atomic<EncodeTiledFn> fn{nullptr};
+    EncodeTiledFn f = fn.load();
+    if (f == nullptr) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || ptr == nullptr)
+            return nullptr;
+        f = reinterpret_cast<EncodeTiledFn>(ptr);
+        fn.store(f);
+    }
+    return f;
+}
+
+// Tensor map of one (B, T, D) operand for boxes of TC channels x TR rows x 1
+// batch row; elements past the tensor's edges read as zero.
+bool make_operand_map(CUtensorMap *map, const void *ptr, int64_t B, int64_t T, int64_t D, int esz,
+                      int TC, int TR) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(T), cuuint64_t(B)};
+    const cuuint64_t strides[2] = {cuuint64_t(D) * esz, cuuint64_t(T) * cuuint64_t(D) * esz};
+    const cuuint32_t box[3] = {cuuint32_t(TC), cuuint32_t(TR), 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    const CUtensorMapDataType dt = esz == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    return enc(map, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Tile shape of a scan.  Aligned vector-width rows take the pipelined kernel
 // (fp32: 7 x 4 x R rows x 32 channels; bf16: 7 x 2 x R rows x 64 channels;
 // 128-byte row segments); anything else takes the tile kernel's scalar
@@ -203,8 +240,13 @@ DeviceInfo device_info(int dev) {
 template <class Op, typename IO, int V, int R>
 cudaError_t launch_pipelined(const ScanParams &sp_in, cudaStream_t s, int64_t *grid_out) {
     constexpr int CG = pipe_cg<IO>();
+    using Shape = PipeShape<IO, V, CG, R, kStages, kPipeWarps>;
     auto kernel = scan_pipelined_kernel<Op, IO, V, CG, R, kStages, kPipeWarps, 2>;
-    constexpr size_t smem = PipeShape<IO, V, CG, R, kStages, kPipeWarps>::smem_bytes;
+    constexpr size_t smem = Shape::smem_bytes;
+    alignas(64) CUtensorMap map0, map1;
+    if (!make_operand_map(&map0, sp_in.in0, sp_in.B, sp_in.T, sp_in.D, int(sizeof(IO)), Shape::TC, Shape::TR) ||
+        !make_operand_map(&map1, sp_in.in1, sp_in.B, sp_in.T, sp_in.D, int(sizeof(IO)), Shape::TC, Shape::TR))
+        return cudaErrorInvalidValue;
     constexpr int NT = (kPipeWarps + 1) * 32;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -235,7 +277,7 @@ cudaError_t launch_pipelined(const ScanParams &sp_in, cudaStream_t s, int64_t *g
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kernel, sp);
+    e = cudaLaunchKernelEx(&cfg, kernel, sp, map0, map1);
     return e;
 }
 

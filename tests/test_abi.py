@@ -134,6 +134,10 @@ def check_plan_indices(B, T, D, dtype, aligned, check_cover):
     if pl["kernel"] == _abi.KERNEL_PIPELINED:
         # persistent blocks: lane l owns channels l V.., warp w owns rows w R..
         assert pl["vector_path"] and cg * V * esz == 128 and V == 4 and pl["stages"] >= 2
+        # tensor-memory-accelerator boxes of TC x TR x 1: inner extent a multiple of
+        # 16 bytes, every box dimension <= 256, the x coordinate (dt TC) 16-byte aligned
+        assert (TC * esz) % 16 == 0 and TC <= 256 and TR <= 256
+        assert (D * esz) % 16 == 0 and (T * D * esz) % 16 == 0
         assert pl["threads"] % 128 == 0      # whole warps per SM sub-partition
         assert pl["smem_bytes"] <= 227 * 1024 // 2
     if pl["vector_path"]:
