@@ -48,6 +48,23 @@
 
 namespace sgr {
 
+// --------------------------------------------------- hardware approximations
+//
+// exp(x) = 2^(x log2 e) with the MUFU's 2^x and 1/x approximations (ftz:
+// results below the normal range flush to 0, which only ever replaces a gate
+// below 1e-38 by 0).
+constexpr float kNegLog2e = -1.4426950408889634f;
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float fast_rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ------------------------------------------------------------- operators
 
 struct MinGRUOp {
@@ -67,21 +84,28 @@ struct MinGRUOp {
     // sigmoid(|x|) = 1 - s (no cancellation since s <= 1/2; exactly 1 - 0 = 1
     // when e underflows, so k = -inf gives a = 1 and k = +inf gives z = 1).
     // The two reciprocals 1/(1+ek), 1/(1+eh) share one division:
-    // inv = 1/((1+ek)(1+eh)).  MUFU work: 2 exp2 + 1 reciprocal.
+    // inv = 1/((1+ek)(1+eh)).  MUFU work: 2 exp2 + 1 reciprocal (hardware
+    // approximations, relative error ~2^-22), the rest in packed fp32x2 pairs.
     static __device__ __forceinline__ void element(float k, float hx, float &a, float &b) {
-        const float ek = __expf(-fabsf(k));
-        const float eh = __expf(-fabsf(hx));
-        const float dk = 1.f + ek;
-        const float dh = 1.f + eh;
-        const float inv = __fdividef(1.f, dk * dh);
-        const float sk = ek * (dh * inv);    // sigmoid(-|k|)
-        const float kbig = 1.f - sk;          // sigmoid(|k|)
+        const float2 e = make_float2(fast_exp2(fabsf(k) * kNegLog2e), fast_exp2(fabsf(hx) * kNegLog2e));
+        const float2 d = __fadd2_rn(e, make_float2(1.f, 1.f));               // (1+ek, 1+eh)
+        const float inv = fast_rcp(d.x * d.y);
+        const float2 rr = __fmul2_rn(make_float2(d.y, d.x), make_float2(inv, inv));  // (1/(1+ek), 1/(1+eh))
+        const float2 sg = __fmul2_rn(e, rr);     // (sigmoid(-|k|), sigmoid(-|hx|))
+        const float kbig = 1.f - sg.x;          // sigmoid(|k|)
         const bool kpos = k >= 0.f;
-        const float z = kpos ? kbig : sk;
-        a = kpos ? sk : kbig;
-        const float g = (hx >= 0.f) ? hx + 0.5f : eh * (dk * inv);
+        const float z = kpos ? kbig : sg.x;
+        a = kpos ? sg.x : kbig;
+        const float g = (hx >= 0.f) ? hx + 0.5f : sg.y;
         b = z * g;
     }
+    // fold a step into a running pair, two channels at once: (A, B) <- (A a, B a + b)
+    static __device__ __forceinline__ void fold2(float2 &A, float2 &B, float2 a, float2 b) {
+        B = __ffma2_rn(B, a, b);
+        A = __fmul2_rn(A, a);
+    }
+    // replay one step for two channels: h <- a h + b
+    static __device__ __forceinline__ float2 step2(float2 a, float2 b, float2 h) { return __ffma2_rn(a, h, b); }
     // one step of phase 3
     static __device__ __forceinline__ float step(float a, float b, float x) { return fmaf(a, x, b); }
     // initial state when none is given
@@ -100,6 +124,13 @@ struct MinMaxOp {
     static __device__ __forceinline__ void element(float r, float s, float &u, float &l) { u = r; l = s; }
     static __device__ __forceinline__ float step(float u, float l, float x) { return fmaxf(fminf(x, u), l); }
     static __device__ __forceinline__ float default_init() { return 0.f; }
+    static __device__ __forceinline__ void fold2(float2 &U, float2 &L, float2 u, float2 l) {
+        L = make_float2(fmaxf(fminf(L.x, u.x), l.x), fmaxf(fminf(L.y, u.y), l.y));
+        U = make_float2(fminf(U.x, u.x), fminf(U.y, u.y));
+    }
+    static __device__ __forceinline__ float2 step2(float2 u, float2 l, float2 x) {
+        return make_float2(fmaxf(fminf(x.x, u.x), l.x), fmaxf(fminf(x.y, u.y), l.y));
+    }
 };
 
 // ------------------------------------------------------------ memory access
@@ -727,11 +758,14 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
         const int g = lane % CG;
         const int j = lane / CG;
         IO *out = static_cast<IO *>(p.out);
+        constexpr int V2 = V / 2;
 
-        float2 P[2][R][V];   // pairs of the two tiles in flight (tile parity)
-        float2 E[2][V];      // the thread's exclusive prefix within its warp
+        // pairs of the two tiles in flight (tile parity), two channels per float2
+        float2 PA[2][R][V2], PB[2][R][V2];
+        float2 E[2][V];      // the thread's exclusive prefix within its warp, per channel
         int64_t base[2];     // global offset of the thread's first element of the tile
         int row0[2];         // first row (along T) of the thread's rows
+        bool full[2];        // all R rows and V channels of the thread inside the tensor
         bool dvalid[2];
         uint32_t wait_limit = kMbarLimit;
 
@@ -741,31 +775,49 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
             const int64_t d0 = int64_t(tc.dt) * TC + g * V;
             dvalid[BUF] = d0 < p.D;
             row0[BUF] = int(tc.c) * TR + (warp * J + j) * R;
+            full[BUF] = dvalid[BUF] && (row0[BUF] + R <= p.T);
             base[BUF] = (int64_t(tc.b) * p.T) * p.D + d0;
             if (!mbar_wait(bars + 8u * uint32_t(n % S), uint32_t((n / S) & 1), wait_limit)) {
                 wait_limit = 1;
                 if (lane == 0) atomicOr(p.status, kTimeoutBit);
             }
-            const IO *t0 = reinterpret_cast<const IO *>(smem + (n % S) * Shape::slot_bytes);
+            const IO *t0 = reinterpret_cast<const IO *>(smem + (n % S) * Shape::slot_bytes) +
+                           ((warp * J + j) * R) * TC + g * V;
             const IO *t1 = t0 + TR * TC;
-            const int lr = (warp * J + j) * R;      // first local row
-            float2 incl[V];
+            float2 IA[V2], IB[V2];
 #pragma unroll
-            for (int v = 0; v < V; ++v) incl[v] = Op::identity();
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                float x0[V], x1[V];
-                const bool ok = dvalid[BUF] && (row0[BUF] + r < p.T);
-                unpack(*reinterpret_cast<const Vec *>(t0 + (lr + r) * TC + g * V), x0);
-                unpack(*reinterpret_cast<const Vec *>(t1 + (lr + r) * TC + g * V), x1);
-#pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    float e0, e1;
-                    Op::element(ok ? x0[v] : Op::pad0(), ok ? x1[v] : Op::pad1(), e0, e1);
-                    P[BUF][r][v] = make_float2(e0, e1);
-                    incl[v] = Op::combine(incl[v], P[BUF][r][v]);
-                }
+            for (int i = 0; i < V2; ++i) {
+                IA[i] = make_float2(Op::identity().x, Op::identity().x);
+                IB[i] = make_float2(Op::identity().y, Op::identity().y);
             }
+            auto rows = [&](auto fullc) {
+                constexpr bool FULL = decltype(fullc)::value;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    float x0[V], x1[V];
+                    unpack(*reinterpret_cast<const Vec *>(t0 + r * TC), x0);
+                    unpack(*reinterpret_cast<const Vec *>(t1 + r * TC), x1);
+                    if (!FULL) {
+                        const bool ok = dvalid[BUF] && (row0[BUF] + r < p.T);
+#pragma unroll
+                        for (int v = 0; v < V; ++v) {
+                            x0[v] = ok ? x0[v] : Op::pad0();
+                            x1[v] = ok ? x1[v] : Op::pad1();
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < V2; ++i) {
+                        float a0, b0, a1, b1;
+                        Op::element(x0[2 * i], x1[2 * i], a0, b0);
+                        Op::element(x0[2 * i + 1], x1[2 * i + 1], a1, b1);
+                        PA[BUF][r][i] = make_float2(a0, a1);
+                        PB[BUF][r][i] = make_float2(b0, b1);
+                        Op::fold2(IA[i], IB[i], PA[BUF][r][i], PB[BUF][r][i]);
+                    }
+                }
+            };
+            if (full[BUF]) rows(std::true_type{});
+            else rows(std::false_type{});
             // the warp is done with the slot; the last of the W warps refills it
             // with tile n + S (its values are in registers, consumed above)
             __syncwarp();
@@ -778,6 +830,12 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                         issue_tile(n + S);
                     }
                 }
+            }
+            float2 incl[V];
+#pragma unroll
+            for (int i = 0; i < V2; ++i) {
+                incl[2 * i] = make_float2(IA[i].x, IB[i].x);
+                incl[2 * i + 1] = make_float2(IA[i].y, IB[i].y);
             }
             // scan across the J row groups of the warp
 #pragma unroll
@@ -807,19 +865,23 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
         auto phaseB = [&](auto bufc) {
             constexpr int BUF = decltype(bufc)::value;
             named_barrier_sync(3 + BUF, NT);
-            float st[V];
+            float2 st[V2];
 #pragma unroll
-            for (int v = 0; v < V; ++v) st[v] = Op::apply(E[BUF][v], s_tot[BUF][warp][g * V + v].x);
+            for (int i = 0; i < V2; ++i)
+                st[i] = make_float2(Op::apply(E[BUF][2 * i], s_tot[BUF][warp][g * V + 2 * i].x),
+                                    Op::apply(E[BUF][2 * i + 1], s_tot[BUF][warp][g * V + 2 * i + 1].x));
+            IO *dst = out + base[BUF] + int64_t(row0[BUF]) * p.D;
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 float y[V];
 #pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    st[v] = Op::step(P[BUF][r][v].x, P[BUF][r][v].y, st[v]);
-                    y[v] = st[v];
+                for (int i = 0; i < V2; ++i) {
+                    st[i] = Op::step2(PA[BUF][r][i], PB[BUF][r][i], st[i]);
+                    y[2 * i] = st[i].x;
+                    y[2 * i + 1] = st[i].y;
                 }
-                if (dvalid[BUF] && row0[BUF] + r < p.T)
-                    Access<IO, V>::store(out + base[BUF] + int64_t(row0[BUF] + r) * p.D, y);
+                if (full[BUF] || (dvalid[BUF] && row0[BUF] + r < p.T)) Access<IO, V>::store(dst, y);
+                dst += p.D;
             }
         };
 
