@@ -335,21 +335,25 @@ __device__ __forceinline__ void publish_state(const ScanParams &p, int64_t tile,
 // neither is waited for (bounded, with back-off).  Before chunk 0 the state is
 // the initial state.  Each lane works alone: its channels' words carry their
 // own validity.
+// chunks read per round trip: short windows for the tile kernel (few
+// registers), longer ones for the pipelined kernel's carry warp
 template <int CV>
-constexpr int window_len() { return CV >= 4 ? 1 : (CV == 2 ? 2 : 4); }
+constexpr int window_short() { return CV >= 4 ? 1 : (CV == 2 ? 2 : 4); }
+template <int CV>
+constexpr int window_long() { return CV >= 4 ? 1 : (CV == 2 ? 4 : 8); }
 
-template <int CV, int TC>
+template <int CV, int TC, int KW>
 struct LookWindow {
-    static constexpr int K = window_len<CV>();
+    static constexpr int K = KW;
     uint64_t wa[K][CV], wb[K][CV], ws[K][CV];
 };
 
 // issue the loads of the words of chunks q, q-1, ..., q-K+1
-template <int CV, int TC>
+template <int CV, int TC, int KW>
 __device__ __forceinline__ void load_window(const ScanParams &p, int64_t q, int64_t chain, int ch,
-                                            LookWindow<CV, TC> &win) {
+                                            LookWindow<CV, TC, KW> &win) {
 #pragma unroll
-    for (int i = 0; i < LookWindow<CV, TC>::K; ++i) {
+    for (int i = 0; i < KW; ++i) {
         const int64_t qq = q - i;
         if (qq >= 0) {
             const uint64_t *w = p.words + (qq * p.n_chains + chain) * 3 * TC + ch;
@@ -366,14 +370,14 @@ __device__ __forceinline__ void load_window(const ScanParams &p, int64_t q, int6
 // Walk a loaded window starting at chunk q with the running composite M.
 // Returns true when the incoming state is known (hin set); otherwise the
 // number of chunks folded in is in `consumed`.
-template <class Op, typename IO, int CV, int TC>
-__device__ __forceinline__ bool resolve_window(const ScanParams &p, int64_t q, const LookWindow<CV, TC> &win,
+template <class Op, typename IO, int CV, int TC, int KW>
+__device__ __forceinline__ bool resolve_window(const ScanParams &p, int64_t q, const LookWindow<CV, TC, KW> &win,
                                                int64_t b, int64_t d_first, float2 (&M)[CV],
                                                float (&hin)[CV], int &consumed) {
     consumed = 0;
     bool done = false, stop = false;
 #pragma unroll
-    for (int i = 0; i < LookWindow<CV, TC>::K; ++i) {
+    for (int i = 0; i < KW; ++i) {
         if (done || stop) continue;
         const int64_t qq = q - i;
         if (qq < 0) {
@@ -406,9 +410,9 @@ __device__ __forceinline__ bool resolve_window(const ScanParams &p, int64_t q, c
 }
 
 // Finish a look-back whose first window (chunks c-1 ...) is already loaded.
-template <class Op, typename IO, int CV, int TC>
+template <class Op, typename IO, int CV, int TC, int KW>
 __device__ void look_back_from(const ScanParams &p, int64_t c, int64_t chain, int64_t b, int64_t d_first,
-                               int ch, LookWindow<CV, TC> &win, float (&hin)[CV]) {
+                               int ch, LookWindow<CV, TC, KW> &win, float (&hin)[CV]) {
     float2 M[CV];
 #pragma unroll
     for (int v = 0; v < CV; ++v) M[v] = Op::identity();
@@ -416,7 +420,7 @@ __device__ void look_back_from(const ScanParams &p, int64_t c, int64_t chain, in
     uint32_t polls = 0, ns = 32;
     while (true) {
         int consumed;
-        if (resolve_window<Op, IO, CV, TC>(p, q, win, b, d_first, M, hin, consumed)) return;
+        if (resolve_window<Op, IO, CV, TC, KW>(p, q, win, b, d_first, M, hin, consumed)) return;
         if (consumed > 0) {
             q -= consumed;
             ns = 32;
@@ -430,16 +434,17 @@ __device__ void look_back_from(const ScanParams &p, int64_t c, int64_t chain, in
             __nanosleep(ns);
             ns = ns < 256 ? ns * 2 : 256;
         }
-        load_window<CV, TC>(p, q, chain, ch, win);
+        load_window<CV, TC, KW>(p, q, chain, ch, win);
     }
 }
 
 template <class Op, typename IO, int CV, int TC>
 __device__ __forceinline__ void look_back(const ScanParams &p, int64_t c, int64_t chain, int64_t b,
                                           int64_t d_first, int ch, float (&hin)[CV]) {
-    LookWindow<CV, TC> win;
-    load_window<CV, TC>(p, c - 1, chain, ch, win);
-    look_back_from<Op, IO, CV, TC>(p, c, chain, b, d_first, ch, win, hin);
+    constexpr int KW = window_short<CV>();
+    LookWindow<CV, TC, KW> win;
+    load_window<CV, TC, KW>(p, c - 1, chain, ch, win);
+    look_back_from<Op, IO, CV, TC, KW>(p, c, chain, b, d_first, ch, win, hin);
 }
 
 // The carry of one tile, as done by the carry warp: fold the W warp totals in
@@ -496,6 +501,23 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthread
 
 __device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Fold the W warp summaries of CV channels (starting at ch) into the tile
+// total, replacing each summary by the exclusive prefix of the warps before it.
+template <class Op, int CV, int TC, int W>
+__device__ __forceinline__ void fold_warps(float2 (*s_tot)[TC], int ch, float2 (&total)[CV]) {
+#pragma unroll
+    for (int v = 0; v < CV; ++v) total[v] = Op::identity();
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+#pragma unroll
+        for (int v = 0; v < CV; ++v) {
+            const float2 t = s_tot[w][ch + v];
+            s_tot[w][ch + v] = total[v];
+            total[v] = Op::combine(total[v], t);
+        }
+    }
 }
 
 // -------------------------------------------------------- tile kernel
@@ -658,8 +680,10 @@ struct PipeShape {
     static constexpr size_t slot_bytes = 2 * op_bytes;
     static constexpr size_t bar_offset = S * slot_bytes;
     static constexpr size_t cnt_offset = bar_offset + S * 8;          // per-slot reader counts
-    static constexpr size_t tot_offset = (cnt_offset + S * 4 + 15) / 16 * 16;
-    static constexpr size_t smem_bytes = tot_offset + size_t(2) * W * TC * sizeof(float2);
+    static constexpr size_t tot_offset = (cnt_offset + S * 4 + 15) / 16 * 16;        // [2][W][TC] float2
+    static constexpr size_t total_offset = tot_offset + size_t(2) * W * TC * sizeof(float2);  // [2][TC] float2
+    static constexpr size_t hin_offset = total_offset + size_t(2) * TC * sizeof(float2);     // [2][TC] float
+    static constexpr size_t smem_bytes = hin_offset + size_t(2) * TC * sizeof(float);
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
@@ -714,12 +738,20 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
     constexpr int TR = Shape::TR;
     constexpr int CV = TC / 32;
     constexpr uint32_t NT = (W + 1) * 32;
+    // Who folds the W warp summaries into the tile total and publishes the
+    // chunk summary: with fp32 I/O the carry warp's per-tile work is the
+    // limit, so the last data warp of the tile does it; with bf16 I/O (half
+    // the bytes per element) the data warps' instruction issue is the limit,
+    // so the carry warp does it.
+    constexpr bool kFoldInData = sizeof(IO) == 4;
     static_assert(sizeof(Vec) == V * sizeof(IO), "vector type matches the vector width");
     static_assert(CG * J == 32 && TC % 32 == 0, "lane layout");
     static_assert(TC * sizeof(IO) % 16 == 0 && TC <= 256 && TR <= 256, "TMA box");
 
     extern __shared__ __align__(128) unsigned char smem[];
     float2 (*s_tot)[W][TC] = reinterpret_cast<float2 (*)[W][TC]>(smem + Shape::tot_offset);
+    float2 (*s_total)[TC] = reinterpret_cast<float2 (*)[TC]>(smem + Shape::total_offset);
+    float (*s_hin)[TC] = reinterpret_cast<float (*)[TC]>(smem + Shape::hin_offset);
     unsigned int *s_cnt = reinterpret_cast<unsigned int *>(smem + Shape::cnt_offset);
     const uint32_t ring = smem_addr(smem);
     const uint32_t bars = ring + uint32_t(Shape::bar_offset);
@@ -818,19 +850,6 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
             };
             if (full[BUF]) rows(std::true_type{});
             else rows(std::false_type{});
-            // the warp is done with the slot; the last of the W warps refills it
-            // with tile n + S (its values are in registers, consumed above)
-            __syncwarp();
-            if (lane == 0) {
-                const unsigned int seen = atomicAdd(&s_cnt[n % S], 1u);
-                if (seen == W - 1) {
-                    s_cnt[n % S] = 0;
-                    if (n + S < n_local) {
-                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                        issue_tile(n + S);
-                    }
-                }
-            }
             float2 incl[V];
 #pragma unroll
             for (int i = 0; i < V2; ++i) {
@@ -859,6 +878,37 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
 #pragma unroll
                 for (int v = 0; v < V; ++v) s_tot[BUF][warp][g * V + v] = incl[v];
             }
+            // The warp is done with the slot and has written its summary.  The
+            // last of the W warps (a shared counter per slot) refills the slot
+            // with tile n + S and, for fp32 I/O, folds the W warp summaries
+            // into per-warp exclusive prefixes and the tile total and publishes
+            // the chunk summary, so the carry warp only has the look-back left.
+            __threadfence_block();
+            __syncwarp();
+            unsigned int seen = 0;
+            if (lane == 0) seen = atomicAdd(&s_cnt[n % S], 1u);
+            seen = __shfl_sync(0xffffffffu, seen, 0);
+            if (seen == W - 1) {
+                __threadfence_block();
+                if (lane == 0) {
+                    s_cnt[n % S] = 0;
+                    if (n + S < n_local) {
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        issue_tile(n + S);
+                    }
+                }
+                if constexpr (kFoldInData) {
+                    const int ch = lane * CV;
+                    float2 total[CV];
+                    fold_warps<Op, CV, TC, W>(s_tot[BUF], ch, total);
+#pragma unroll
+                    for (int v = 0; v < CV; ++v) s_total[BUF][ch + v] = total[v];
+                    const int64_t tile = first + int64_t(n) * G;
+                    const bool publish =
+                        (p.n_chunks > 1) && (int64_t(tc.c) < p.n_chunks - 1) && (tile != p.drop_tile);
+                    if (publish && tc.c > 0) publish_summary<CV, TC>(p, tile, ch, total);
+                }
+            }
             named_barrier_arrive(1 + BUF, NT);
         };
 
@@ -867,9 +917,12 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
             named_barrier_sync(3 + BUF, NT);
             float2 st[V2];
 #pragma unroll
-            for (int i = 0; i < V2; ++i)
-                st[i] = make_float2(Op::apply(E[BUF][2 * i], s_tot[BUF][warp][g * V + 2 * i].x),
-                                    Op::apply(E[BUF][2 * i + 1], s_tot[BUF][warp][g * V + 2 * i + 1].x));
+            for (int i = 0; i < V2; ++i) {
+                const int c0 = g * V + 2 * i;
+                const float w0 = Op::apply(s_tot[BUF][warp][c0], s_hin[BUF][c0]);
+                const float w1 = Op::apply(s_tot[BUF][warp][c0 + 1], s_hin[BUF][c0 + 1]);
+                st[i] = make_float2(Op::apply(E[BUF][2 * i], w0), Op::apply(E[BUF][2 * i + 1], w1));
+            }
             IO *dst = out + base[BUF] + int64_t(row0[BUF]) * p.D;
 #pragma unroll
             for (int r = 0; r < R; ++r) {
@@ -903,14 +956,15 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
         }
     } else {
         // ============================================== carry warp
-        // Per tile: fold the warp summaries, publish the chunk summary,
-        // resolve the incoming state from the look-back window, write each
-        // warp's incoming state, release the data warps, publish the chunk's
-        // final state, and issue the loads of the next tile's look-back window
-        // (they read other blocks' words, so they fly while this warp waits
-        // for the next tile's summaries).
+        // Per tile: (bf16 I/O: fold the warp summaries and publish the chunk
+        // summary,) resolve the incoming state from the look-back window,
+        // write it to shared memory, release the data warps, publish the
+        // chunk's final state, and issue the loads of the next tile's
+        // look-back window (they read other blocks' words, so they fly while
+        // this warp waits for the next tile's summaries).
         const int ch = lane * CV;
-        LookWindow<CV, TC> win;
+        constexpr int KW = window_long<CV>();
+        LookWindow<CV, TC, KW> win;
         float init[CV];
         auto prefetch = [&](int n) {
             const TileCoord tc = tile_coord(p, uint32_t(first + int64_t(n) * G));
@@ -919,7 +973,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                 for (int v = 0; v < CV; ++v)
                     init[v] = load_init<IO>(p, tc.b, int64_t(tc.dt) * TC + ch + v, Op::default_init());
             } else {
-                load_window<CV, TC>(p, int64_t(tc.c) - 1, tc.chain, ch, win);
+                load_window<CV, TC, KW>(p, int64_t(tc.c) - 1, tc.chain, ch, win);
             }
         };
         if (n_local > 0) prefetch(0);
@@ -930,35 +984,28 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
             const TileCoord tc = tile_coord(p, uint32_t(tile));
             const int64_t c = tc.c;
             const int64_t dl = int64_t(tc.dt) * TC + ch;
-            float2 total[CV];
-#pragma unroll
-            for (int v = 0; v < CV; ++v) total[v] = Op::identity();
-            for (int w = 0; w < W; ++w) {
-#pragma unroll
-                for (int v = 0; v < CV; ++v) {
-                    const float2 t = s_tot[PB][w][ch + v];
-                    s_tot[PB][w][ch + v] = total[v];       // exclusive prefix over warps
-                    total[v] = Op::combine(total[v], t);
-                }
-            }
             const bool publish = (p.n_chunks > 1) && (c < p.n_chunks - 1) && (tile != p.drop_tile);
+            if constexpr (!kFoldInData) {
+                float2 total[CV];
+                fold_warps<Op, CV, TC, W>(s_tot[PB], ch, total);
+#pragma unroll
+                for (int v = 0; v < CV; ++v) s_total[PB][ch + v] = total[v];
+                if (publish && c > 0) publish_summary<CV, TC>(p, tile, ch, total);
+            }
             float hin[CV];
             if (c == 0) {
 #pragma unroll
                 for (int v = 0; v < CV; ++v) hin[v] = init[v];
             } else {
-                if (publish) publish_summary<CV, TC>(p, tile, ch, total);
-                look_back_from<Op, IO, CV, TC>(p, c, tc.chain, tc.b, dl, ch, win, hin);
+                look_back_from<Op, IO, CV, TC, KW>(p, c, tc.chain, tc.b, dl, ch, win, hin);
             }
-            for (int w = 0; w < W; ++w) {
 #pragma unroll
-                for (int v = 0; v < CV; ++v) s_tot[PB][w][ch + v].x = Op::apply(s_tot[PB][w][ch + v], hin[v]);
-            }
+            for (int v = 0; v < CV; ++v) s_hin[PB][ch + v] = hin[v];
             named_barrier_arrive(3 + PB, NT);
             if (publish) {
                 float fin[CV];
 #pragma unroll
-                for (int v = 0; v < CV; ++v) fin[v] = Op::apply(total[v], hin[v]);
+                for (int v = 0; v < CV; ++v) fin[v] = Op::apply(s_total[PB][ch + v], hin[v]);
                 publish_state<CV, TC>(p, tile, ch, fin);
             }
             if (n + 1 < n_local) prefetch(n + 1);
