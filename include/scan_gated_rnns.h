@@ -203,7 +203,9 @@ SGR_API sgr_status_t sgr_set_tile_override(int channel_lanes, int rows_per_threa
 /*
  * Tuning/testing knob, process-wide: 0 automatic (pipelined kernel for
  * aligned vector-width rows, tile kernel otherwise), 1 force the tile kernel,
- * 2 pipelined wherever the fast path applies.
+ * 2 pipelined with 7 data warps per block (two blocks per SM), 3 pipelined
+ * with 15 data warps (one block per SM, tiles twice as long), both wherever
+ * the fast path applies.
  */
 SGR_API sgr_status_t sgr_set_kernel_override(int kernel);
 
@@ -212,7 +214,8 @@ SGR_API sgr_status_t sgr_set_kernel_override(int kernel);
 /* How a scan of this shape is cut into tiles (rows x channels per block). */
 typedef struct sgr_plan {
     int32_t vector_path;        /* 1: 128-bit loads; 0: scalar variant            */
-    int32_t kernel;             /* 1: one block per tile; 2: pipelined persistent  */
+    int32_t kernel;             /* 1: one block per tile; 2: pipelined persistent,
+                                   7 data warps; 3: pipelined, 15 data warps       */
     int32_t channels_per_thread;
     int32_t channel_lanes;      /* lanes across D per warp                         */
     int32_t rows_per_thread;

@@ -14,16 +14,19 @@ namespace {
 
 using namespace sgr;
 
-// Both kernels use 7 data warps + 1 carry warp = 8 warps per block, so blocks
-// spread evenly over the SM's 4 sub-partitions, each of which has its own
-// register file (two pipelined blocks per SM: 128 registers per thread).
+// Blocks are whole multiples of 4 warps (7 or 15 data warps + 1 carry warp),
+// so they spread evenly over the SM's 4 sub-partitions, each of which has its
+// own register file: 128 registers per thread with two 8-warp pipelined
+// blocks or one 16-warp block per SM.
 constexpr int kWarps = 7;
-constexpr int kPipeWarps = 7;
+constexpr int kPipeWarps = 7;        // two blocks per SM
+constexpr int kPipeWarpsWide = 15;   // one block per SM, tiles twice as long
 constexpr int kStages = 3;
+constexpr int kAssumedSMs = 148;     // B200; only used to pick a tile shape
 constexpr int64_t kTargetTiles = 4 * 148;  // tile kernel: prefer >= 4 tiles per SM
 constexpr size_t kAlign = 256;
 
-enum Kind { KIND_AUTO = 0, KIND_TILE = 1, KIND_PIPELINED = 2 };
+enum Kind { KIND_AUTO = 0, KIND_TILE = 1, KIND_PIPELINED = 2, KIND_PIPELINED_WIDE = 3 };
 
 std::atomic<int> g_override_cg{0};
 std::atomic<int> g_override_r{0};
@@ -51,6 +54,7 @@ struct Plan {
     int cg = 32;          // lanes across channels
     int r = 2;            // rows per thread
     int stages = 0;       // pipelined: tiles in flight per block
+    int warps = kWarps;   // data warps per block
     int TR = 0, TC = 0;   // tile rows / channels
     int64_t n_dt = 0, n_chains = 0, n_chunks = 0, n_tiles = 0;
     size_t smem = 0;      // dynamic shared memory per block
@@ -68,8 +72,8 @@ bool mul_ok(int64_t a, int64_t b, int64_t *out) {
 // rows), bf16 16 lanes x 4 channels (64-channel tiles, 128-byte rows)
 template <typename IO> constexpr int pipe_cg() { return sizeof(IO) == 4 ? 8 : 16; }
 
-template <typename IO, int R>
-constexpr size_t pipe_smem() { return PipeShape<IO, 4, pipe_cg<IO>(), R, kStages, kPipeWarps>::smem_bytes; }
+template <typename IO, int R, int W>
+constexpr size_t pipe_smem() { return PipeShape<IO, 4, pipe_cg<IO>(), R, kStages, W>::smem_bytes; }
 
 // cuTensorMapEncodeTiled, fetched once from the driver through the runtime
 // (no link-time dependency on the driver library)
@@ -128,9 +132,29 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned)
         // rows per thread {2, 4}, automatic 4
         p.r = (orr == 2 || orr == 4) ? orr : 4;
         p.stages = kStages;
-        p.TR = kPipeWarps * (32 / p.cg) * p.r;
-        if (p.esz == 4) p.smem = p.r == 4 ? pipe_smem<float, 4>() : pipe_smem<float, 2>();
-        else p.smem = p.r == 4 ? pipe_smem<__nv_bfloat16, 4>() : pipe_smem<__nv_bfloat16, 2>();
+        // Block shape: about (blocks in flight) / n_chains chunks of one
+        // channel tile are processed at once and a look-back folds that many
+        // summaries; when that depth reaches 8 with two 8-warp blocks per SM,
+        // one 16-warp block per SM with tiles twice as long halves it.
+        // Only when the wide tiles still give every SM at least 4 of them.
+        const int64_t n_chains = B * ((D + p.TC - 1) / p.TC);
+        const int64_t tr_wide = int64_t(kPipeWarpsWide) * (32 / p.cg) * p.r;
+        const int64_t tiles_wide = n_chains * ((T + tr_wide - 1) / tr_wide);
+        bool wide = n_chains > 0 && 2 * kAssumedSMs >= 8 * n_chains && tiles_wide >= 4 * kAssumedSMs;
+        if (ok == KIND_PIPELINED) wide = false;
+        if (ok == KIND_PIPELINED_WIDE) wide = true;
+        p.kind = wide ? KIND_PIPELINED_WIDE : KIND_PIPELINED;
+        p.warps = wide ? kPipeWarpsWide : kPipeWarps;
+        p.TR = p.warps * (32 / p.cg) * p.r;
+        if (p.esz == 4) {
+            p.smem = wide ? (p.r == 4 ? pipe_smem<float, 4, kPipeWarpsWide>() : pipe_smem<float, 2, kPipeWarpsWide>())
+                          : (p.r == 4 ? pipe_smem<float, 4, kPipeWarps>() : pipe_smem<float, 2, kPipeWarps>());
+        } else {
+            p.smem = wide ? (p.r == 4 ? pipe_smem<__nv_bfloat16, 4, kPipeWarpsWide>()
+                                      : pipe_smem<__nv_bfloat16, 2, kPipeWarpsWide>())
+                          : (p.r == 4 ? pipe_smem<__nv_bfloat16, 4, kPipeWarps>()
+                                      : pipe_smem<__nv_bfloat16, 2, kPipeWarps>());
+        }
     } else {
         // tile kernel: 8 lanes x one vector (32 fp32 / 64 bf16 channels,
         // 128-byte row segments) or, unaligned, 32 lanes x 1 channel
@@ -237,17 +261,18 @@ DeviceInfo device_info(int dev) {
     return d;
 }
 
-template <class Op, typename IO, int V, int R>
+template <class Op, typename IO, int V, int R, int W>
 cudaError_t launch_pipelined(const ScanParams &sp_in, cudaStream_t s, int64_t *grid_out) {
     constexpr int CG = pipe_cg<IO>();
-    using Shape = PipeShape<IO, V, CG, R, kStages, kPipeWarps>;
-    auto kernel = scan_pipelined_kernel<Op, IO, V, CG, R, kStages, kPipeWarps, 2>;
+    using Shape = PipeShape<IO, V, CG, R, kStages, W>;
+    constexpr int MINB = W == kPipeWarps ? 2 : 1;
+    auto kernel = scan_pipelined_kernel<Op, IO, V, CG, R, kStages, W, MINB>;
     constexpr size_t smem = Shape::smem_bytes;
     alignas(64) CUtensorMap map0, map1;
     if (!make_operand_map(&map0, sp_in.in0, sp_in.B, sp_in.T, sp_in.D, int(sizeof(IO)), Shape::TC, Shape::TR) ||
         !make_operand_map(&map1, sp_in.in1, sp_in.B, sp_in.T, sp_in.D, int(sizeof(IO)), Shape::TC, Shape::TR))
         return cudaErrorInvalidValue;
-    constexpr int NT = (kPipeWarps + 1) * 32;
+    constexpr int NT = (W + 1) * 32;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -285,8 +310,12 @@ template <class Op, typename IO>
 cudaError_t dispatch(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
     constexpr int VW = 16 / int(sizeof(IO));
     if (pl.kind == KIND_PIPELINED) {
-        return pl.r == 2 ? launch_pipelined<Op, IO, 4, 2>(sp, s, nullptr)
-                         : launch_pipelined<Op, IO, 4, 4>(sp, s, nullptr);
+        return pl.r == 2 ? launch_pipelined<Op, IO, 4, 2, kPipeWarps>(sp, s, nullptr)
+                         : launch_pipelined<Op, IO, 4, 4, kPipeWarps>(sp, s, nullptr);
+    }
+    if (pl.kind == KIND_PIPELINED_WIDE) {
+        return pl.r == 2 ? launch_pipelined<Op, IO, 4, 2, kPipeWarpsWide>(sp, s, nullptr)
+                         : launch_pipelined<Op, IO, 4, 4, kPipeWarpsWide>(sp, s, nullptr);
     }
     if (!pl.vec) return dispatch_tile_r<Op, IO, 1, 32>(pl, sp, s);
     return dispatch_tile_r<Op, IO, VW, 8>(pl, sp, s);
@@ -459,7 +488,7 @@ sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dty
     plan->channels_per_thread = p.V;
     plan->channel_lanes = p.cg;
     plan->rows_per_thread = p.r;
-    plan->warps = p.kind == KIND_PIPELINED ? kPipeWarps : kWarps;
+    plan->warps = p.warps;
     plan->threads = (plan->warps + 1) * 32;
     plan->stages = p.stages;
     plan->tile_rows = p.TR;
@@ -493,7 +522,7 @@ sgr_status_t sgr_set_drop_publish(int64_t tile) {
 }
 
 sgr_status_t sgr_set_kernel_override(int kernel) {
-    if (kernel < KIND_AUTO || kernel > KIND_PIPELINED) return SGR_ERR_INVALID_ARG;
+    if (kernel < KIND_AUTO || kernel > KIND_PIPELINED_WIDE) return SGR_ERR_INVALID_ARG;
     g_override_kind.store(kernel);
     return SGR_OK;
 }

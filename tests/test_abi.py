@@ -109,7 +109,7 @@ def test_workspace_size_and_hooks():
     assert lib.sgr_set_tile_override(3, 0) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_tile_override(0, 3) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_drop_publish(-2) == _abi.SGR_ERR_INVALID_ARG
-    assert lib.sgr_set_kernel_override(3) == _abi.SGR_ERR_INVALID_ARG
+    assert lib.sgr_set_kernel_override(4) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_wait_limit(0) == _abi.SGR_OK
     assert lib.sgr_set_drop_publish(-1) == _abi.SGR_OK
     assert lib.sgr_workspace_init(None, 0, None) == _abi.SGR_OK
@@ -131,7 +131,7 @@ def check_plan_indices(B, T, D, dtype, aligned, check_cover):
     assert n_dt == -(-D // TC) and n_chains == B * n_dt and n_chunks == -(-T // TR)
     assert n_tiles == n_chains * n_chunks and n_tiles < 2 ** 31
     assert pl["threads"] == (W + 1) * 32
-    if pl["kernel"] == _abi.KERNEL_PIPELINED:
+    if pl["kernel"] in (_abi.KERNEL_PIPELINED, _abi.KERNEL_PIPELINED_WIDE):
         # persistent blocks: lane l owns channels l V.., warp w owns rows w R..
         assert pl["vector_path"] and cg * V * esz == 128 and V == 4 and pl["stages"] >= 2
         # tensor-memory-accelerator boxes of TC x TR x 1: inner extent a multiple of
@@ -139,7 +139,8 @@ def check_plan_indices(B, T, D, dtype, aligned, check_cover):
         assert (TC * esz) % 16 == 0 and TC <= 256 and TR <= 256
         assert (D * esz) % 16 == 0 and (T * D * esz) % 16 == 0
         assert pl["threads"] % 128 == 0      # whole warps per SM sub-partition
-        assert pl["smem_bytes"] <= 227 * 1024 // 2
+        per_sm = 2 if pl["kernel"] == _abi.KERNEL_PIPELINED else 1
+        assert pl["smem_bytes"] <= 227 * 1024 // per_sm
     if pl["vector_path"]:
         assert aligned and D % V == 0 and V * esz in (8, 16)
     # the kernels divide tile -> (chunk, chain) -> (b, dt) by multiply-high,
@@ -195,7 +196,7 @@ SMALL_SHAPES = [(2, 1024, 512), (3, 1000, 96), (1, 777, 36), (2, 300, 7), (1, 1,
 @pytest.mark.parametrize("dtype", [F32, BF16])
 @pytest.mark.parametrize("aligned", [True, False])
 @pytest.mark.parametrize("override", [(0, 0, 0), (1, 0, 1), (1, 0, 2), (1, 0, 4), (1, 0, 8),
-                                      (2, 0, 2), (2, 0, 4)])
+                                      (2, 0, 2), (2, 0, 4), (3, 0, 2), (3, 0, 4)])
 def test_plan_indices_small(shape, dtype, aligned, override):
     lib = _abi.lib()
     assert lib.sgr_set_kernel_override(override[0]) == 0

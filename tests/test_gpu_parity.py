@@ -64,7 +64,7 @@ def _reset_hooks():
 
 
 # (kernel, rows per thread): the tile kernel and the pipelined kernel, every R
-VARIANTS = [(1, 1), (1, 2), (1, 4), (1, 8), (2, 2), (2, 4)]
+VARIANTS = [(1, 1), (1, 2), (1, 4), (1, 8), (2, 2), (2, 4), (3, 2), (3, 4)]
 
 
 # ------------------------------------------------------------------ minGRU
@@ -195,7 +195,7 @@ def test_graph_capture_replays():
         assert rel_err(y, oracle.mingru_linear(k, hx, h0, threads=8)) <= TOL["f32"]
 
 
-@pytest.mark.parametrize("kernel,D", [(1, 64), (2, 64)])
+@pytest.mark.parametrize("kernel,D", [(1, 64), (2, 64), (3, 64)])
 def test_bounded_wait_reports_timeout(kernel, D):
     # chunk 0 of channel tile 0 skips publishing its state: the next chunk of the
     # same channels waits until the poll limit, records the timeout and writes
