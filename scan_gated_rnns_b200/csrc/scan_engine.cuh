@@ -659,10 +659,11 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const Sca
 // registers), then phase B of tile n-1 (replay from the thread's incoming
 // state, streaming stores).
 //
-// Carry warp: the hand-off of tile n runs while the data warps are in phase A
-// of tile n+1; the loads of tile n+1's look-back window are issued as soon as
-// tile n is released, so the round trip overlaps the wait for tile n+1's
-// summaries.  Named barriers and summaries are double-buffered by tile parity:
+// Carry warp: it resolves tile n's incoming state (a look-back over earlier
+// chunks only) while the data warps are still in phase A of tile n, so once
+// tile n's summaries are in it only writes the state and releases them; the
+// loads of tile n+1's look-back window are issued as soon as tile n is
+// released.  Named barriers and summaries are double-buffered by tile parity:
 //   barrier 1 + (n & 1): data warps arrive (summaries of tile n written),
 //                        carry warp waits;
 //   barrier 3 + (n & 1): carry warp arrives (incoming states of tile n
@@ -956,12 +957,13 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
         }
     } else {
         // ============================================== carry warp
-        // Per tile: (bf16 I/O: fold the warp summaries and publish the chunk
-        // summary,) resolve the incoming state from the look-back window,
-        // write it to shared memory, release the data warps, publish the
-        // chunk's final state, and issue the loads of the next tile's
-        // look-back window (they read other blocks' words, so they fly while
-        // this warp waits for the next tile's summaries).
+        // Per tile: resolve the incoming state from the look-back window
+        // (issued when the previous tile was done) while the data warps are in
+        // phase A; wait for the tile's warp summaries; (bf16 I/O: fold them and
+        // publish the chunk summary;) write the incoming state, release the
+        // data warps, publish the chunk's final state, and issue the next
+        // tile's look-back loads.  A look-back only ever waits for chunks with
+        // smaller tile indices, whose blocks never wait on this one.
         const int ch = lane * CV;
         constexpr int KW = window_long<CV>();
         LookWindow<CV, TC, KW> win;
@@ -979,25 +981,27 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
         if (n_local > 0) prefetch(0);
         for (int n = 0; n < n_local; ++n) {
             const int PB = n & 1;
-            named_barrier_sync(1 + PB, NT);
             const int64_t tile = first + int64_t(n) * G;
             const TileCoord tc = tile_coord(p, uint32_t(tile));
             const int64_t c = tc.c;
             const int64_t dl = int64_t(tc.dt) * TC + ch;
             const bool publish = (p.n_chunks > 1) && (c < p.n_chunks - 1) && (tile != p.drop_tile);
-            if constexpr (!kFoldInData) {
-                float2 total[CV];
-                fold_warps<Op, CV, TC, W>(s_tot[PB], ch, total);
-#pragma unroll
-                for (int v = 0; v < CV; ++v) s_total[PB][ch + v] = total[v];
-                if (publish && c > 0) publish_summary<CV, TC>(p, tile, ch, total);
-            }
+            // The incoming state depends only on earlier chunks: resolve it
+            // while the data warps are still in phase A of this tile.
             float hin[CV];
             if (c == 0) {
 #pragma unroll
                 for (int v = 0; v < CV; ++v) hin[v] = init[v];
             } else {
                 look_back_from<Op, IO, CV, TC, KW>(p, c, tc.chain, tc.b, dl, ch, win, hin);
+            }
+            named_barrier_sync(1 + PB, NT);
+            if constexpr (!kFoldInData) {
+                float2 total[CV];
+                fold_warps<Op, CV, TC, W>(s_tot[PB], ch, total);
+#pragma unroll
+                for (int v = 0; v < CV; ++v) s_total[PB][ch + v] = total[v];
+                if (publish && c > 0) publish_summary<CV, TC>(p, tile, ch, total);
             }
 #pragma unroll
             for (int v = 0; v < CV; ++v) s_hin[PB][ch + v] = hin[v];
