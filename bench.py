@@ -363,39 +363,38 @@ def run_b200(args):
     launch_max = reduce_max(per_launch, world, device)
     agg = aggregate(bytes_step, w.n_elems, args.steps, t_max, world)
 
-    # end to end through the public API: pinned host inputs, copies timed
+    # end to end through the public API: pinned host inputs and output, the
+    # library's time-sliced host scan (uploads, scans and downloads overlap)
     e2e = None
     if not args.no_e2e:
         hp = p.cpu().pin_memory()
         hq = q.cpu().pin_memory()
         hi = init.cpu().pin_memory() if init is not None else None
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        dp, dq = torch.empty_like(p), torch.empty_like(q)
-        di = torch.empty_like(init) if init is not None else None
+        host_fn = sgr.mingru_scan_host if w.op == "mingru" else sgr.minmax_scan_host
 
         def e2e_step():
-            dp.copy_(hp, non_blocking=True)
-            dq.copy_(hq, non_blocking=True)
-            if di is not None:
-                di.copy_(hi, non_blocking=True)
-            y = (sgr.mingru_scan if w.op == "mingru" else sgr.minmax_scan)(dp, dq, di, out=out, workspace=ws)
-            hout.copy_(y, non_blocking=True)
+            host_fn(hp, hq, hi, out=hout, blocking=False)
 
-        for _ in range(2):
+        for _ in range(3):
             e2e_step()
         torch.cuda.synchronize()
         barrier(world, device)
-        e_steps = max(1, min(args.steps, 5))
+        e_steps = max(1, min(args.steps, 10))
         et, _ = timed_launches(e2e_step, e_steps, stream)
         barrier(world, device)
         et = reduce_max(et, world, device)
         h2d = hp.numel() * hp.element_size() + hq.numel() * hq.element_size() + \
             (hi.numel() * hi.element_size() if hi is not None else 0)
         d2h = hout.numel() * hout.element_size()
+        nbytes = sgr.staging_size(w.op, w.B, w.T, w.D, p.dtype)
         e2e = {"value": round(world * bytes_step * e_steps / et / 1e9, 2), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": round(et * 1e3 / e_steps, 3), "steps": e_steps}
-        del hp, hq, hi, hout, dp, dq, di
+               "ms_per_step": round(et * 1e3 / e_steps, 3), "steps": e_steps,
+               "api": f"{host_fn.__name__} (pinned host tensors in and out, time slices of "
+                      "~8 MB of inputs, uploads/scans/downloads overlapped)",
+               "staging_bytes": nbytes}
+        del hp, hq, hi, hout
 
     peak, peak_src = hbm_peak()
     achieved = bytes_step / launch_max / 1e9

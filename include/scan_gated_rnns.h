@@ -167,6 +167,54 @@ SGR_API sgr_status_t mingru_scan_noalloc(const void *k, const void *hx,
                                          void *h, int64_t B, int64_t T, int64_t D,
                                          sgr_dtype_t dtype, cudaStream_t stream);
 
+/* ---------------------------------------------------- host-buffer scans */
+
+/*
+ * mingru_scan_host / minmax_scan_host -- the same scans for operands that sit
+ * in HOST memory: k, hx (r, s), the optional initial state and the output h
+ * (x) are host pointers, same layout, strides and dtype rules as above.  There
+ * is no counterpart on the pages; this is the library's end-to-end path for
+ * data that does not already live on the GPU.
+ *
+ * The time axis is cut into slices of Tc = ceil(T / n) rows, n = `chunks`
+ * (0 picks n so that one slice's inputs are about 8 MB).  Slice i is copied to
+ * the device on a library-owned copy stream, scanned on `stream` with the
+ * last row of slice i-1's output as its initial state, and copied back on a
+ * second library-owned stream, with two sets of device buffers, so the
+ * upload of slice i+1, the scan of slice i and the download of slice i-1
+ * overlap.  The result equals that of one device scan up to fp32 rounding
+ * order (MinMax: bit-identical).
+ *
+ * staging: DEVICE memory of at least sgr_host_staging_size(...) bytes, 16-byte
+ *   aligned, owned by the caller; its contents need no initialisation (its
+ *   first bytes hold the scan workspace, which each call clears, so
+ *   sgr_workspace_status(staging, ...) reports a timed-out chunk of the call).
+ *   One staging buffer serves one call at a time.
+ * Ordering: the call returns once everything is enqueued.  The copies wait
+ *   for the work already on `stream`, and `stream` waits for the last copy, so
+ *   the host output is complete when `stream` reaches the point after the
+ *   call (cudaStreamSynchronize(stream)).  Host buffers must stay valid until
+ *   then.  Page-locked host memory gives asynchronous, overlapped copies;
+ *   pageable memory gives correct results with copies that block the host.
+ * Errors: as mingru_scan, plus SGR_ERR_WORKSPACE for a missing, small or
+ *   misaligned staging buffer and SGR_ERR_INVALID_ARG for a capturing stream
+ *   (these calls are not graph-capturable) or overlapping host buffers.
+ */
+SGR_API size_t sgr_host_staging_size(sgr_op_t op, int64_t B, int64_t T, int64_t D,
+                                     sgr_dtype_t dtype, int chunks);
+SGR_API sgr_status_t mingru_scan_host(const void *k, const void *hx,
+                                      const void *h0, int64_t h0_batch_stride,
+                                      void *h, int64_t B, int64_t T, int64_t D,
+                                      sgr_dtype_t dtype, int chunks,
+                                      void *staging, size_t staging_bytes,
+                                      cudaStream_t stream);
+SGR_API sgr_status_t minmax_scan_host(const void *r, const void *s,
+                                      const void *x0, int64_t x0_batch_stride,
+                                      void *x, int64_t B, int64_t T, int64_t D,
+                                      sgr_dtype_t dtype, int chunks,
+                                      void *staging, size_t staging_bytes,
+                                      cudaStream_t stream);
+
 /* ------------------------------------------------------------ workspace */
 
 /* Bytes of workspace a scan of this shape needs (0: none).  Pure host code. */

@@ -3,14 +3,18 @@
     mingru_scan(k, hx, h0=None)     minGRU, whole sequence (B, T, D)
     mingru_step(k_t, hx_t, h_prev)  minGRU, one token (B, D)
     minmax_scan(r, s, x0=None)      MinMax neuron, whole sequence (B, T, D)
+    mingru_scan_host / minmax_scan_host   the same for CPU tensors, with the
+                                    copies to and from the GPU overlapped
 
 All three run in the CUDA library ``libsgr.so`` (C ABI:
 include/scan_gated_rnns.h); this package only marshals PyTorch tensors into
 it.  Build the library with ``python -m scan_gated_rnns_b200.build``.
 """
 from ._abi import ScanError
+from .host import mingru_scan_host, minmax_scan_host, staging_size
 from .ops import (Workspace, default_workspace, mingru_scan, mingru_step, minmax_scan,
                   set_kernel_override, set_tile_override, version, workspace_size)
 
-__all__ = ["ScanError", "Workspace", "default_workspace", "mingru_scan", "mingru_step",
-           "minmax_scan", "set_kernel_override", "set_tile_override", "version", "workspace_size"]
+__all__ = ["ScanError", "Workspace", "default_workspace", "mingru_scan", "mingru_scan_host",
+           "mingru_step", "minmax_scan", "minmax_scan_host", "set_kernel_override",
+           "set_tile_override", "staging_size", "version", "workspace_size"]

@@ -212,3 +212,48 @@ def test_plan_indices_small(shape, dtype, aligned, override):
 def test_plan_indices_workloads(name):
     w = WORKLOADS[name]
     check_plan_indices(w.B, w.T, w.D, F32 if w.dtype == "f32" else BF16, True, check_cover=False)
+
+
+# ------------------------------------------------------- host-buffer scans
+
+@pytest.mark.parametrize("fn", ["mingru_scan_host", "minmax_scan_host"])
+def test_host_scan_argument_errors(fn):
+    E = _abi.SGR_ERR_INVALID_ARG
+
+    def call(p, q, init, ibs, out, B, T, D, dt=F32, chunks=0):
+        return scan(fn, p, q, init, ibs, out, B, T, D, dt, chunks, None, 0, None)
+
+    assert call(A, Bp, None, 0, C, -1, 4, 4) == E
+    assert call(A, Bp, None, 0, C, 1, 4, 4, dt=7) == E
+    assert call(A, Bp, None, 0, C, 1, 4, 4, chunks=-2) == E
+    assert call(A, Bp, 0x40000000, -1, C, 1, 4, 4) == E
+    assert call(None, Bp, None, 0, C, 1, 4, 4) == E
+    assert call(A, Bp, None, 0, A + 16, 1, 4, 4) == E           # output on an input
+    assert call(A, Bp, C + 8, 4, C, 1, 4, 4) == E               # output on the state
+    for shp in [(0, 4, 4), (2, 0, 4), (2, 4, 0)]:
+        assert call(None, None, None, 0, None, *shp) == _abi.SGR_OK
+    assert call(A, Bp, None, 0, C, 1 << 40, 1 << 20, 1 << 10) == _abi.SGR_ERR_UNSUPPORTED
+
+
+def test_host_staging_size():
+    lib = _abi.lib()
+    size = lambda B, T, D, dt=F32, chunks=0, op=MINGRU: lib.sgr_host_staging_size(op, B, T, D, dt, chunks)
+    assert size(0, 4, 4) == 0 and size(1, 4, 4, dt=9) == 0 and size(1, 4, 4, chunks=-1) == 0
+    assert size(1, 4, 4, op=5) == 0
+    B, T, D = 8, 4096, 1024
+    whole = B * T * D * 4
+    # one slice: two sets of (two operands + output) of the whole tensor, plus state and workspace
+    assert size(B, T, D, chunks=1) >= 6 * whole + B * D * 4
+    prev = None
+    for n in (1, 2, 3, 8, 64, T):
+        s = size(B, T, D, chunks=n)
+        tc = -(-T // n)
+        assert s >= 6 * B * tc * D * 4
+        if prev is not None:
+            assert s <= prev
+        prev = s
+    assert size(B, T, D, chunks=T) == size(B, T, D, chunks=10 * T)    # at most one row per slice
+    # automatic slices hold about 8 MB of inputs: staging stays far below the tensor
+    auto = size(B, T, D)
+    assert 6 * (8 << 20) // 2 <= auto <= 6 * (8 << 20) // 2 + (4 << 20)
+    assert size(2, 5, 3, op=MINMAX, chunks=2) > 0
