@@ -409,14 +409,12 @@ __device__ __forceinline__ bool resolve_window(const ScanParams &p, int64_t q, c
     return done;
 }
 
-// Finish a look-back whose first window (chunks c-1 ...) is already loaded.
+// Continue a look-back at chunk q with the running composite M (the chunks
+// after q already folded in); the window of chunks q, q-1, ... is loaded.
 template <class Op, typename IO, int CV, int TC, int KW>
-__device__ void look_back_from(const ScanParams &p, int64_t c, int64_t chain, int64_t b, int64_t d_first,
-                               int ch, LookWindow<CV, TC, KW> &win, float (&hin)[CV]) {
-    float2 M[CV];
-#pragma unroll
-    for (int v = 0; v < CV; ++v) M[v] = Op::identity();
-    int64_t q = c - 1;
+__device__ void look_back_continue(const ScanParams &p, int64_t q, int64_t chain, int64_t b,
+                                   int64_t d_first, int ch, LookWindow<CV, TC, KW> &win,
+                                   float2 (&M)[CV], float (&hin)[CV]) {
     uint32_t polls = 0, ns = 32;
     while (true) {
         int consumed;
@@ -436,6 +434,16 @@ __device__ void look_back_from(const ScanParams &p, int64_t c, int64_t chain, in
         }
         load_window<CV, TC, KW>(p, q, chain, ch, win);
     }
+}
+
+// Finish a look-back whose first window (chunks c-1 ...) is already loaded.
+template <class Op, typename IO, int CV, int TC, int KW>
+__device__ void look_back_from(const ScanParams &p, int64_t c, int64_t chain, int64_t b, int64_t d_first,
+                               int ch, LookWindow<CV, TC, KW> &win, float (&hin)[CV]) {
+    float2 M[CV];
+#pragma unroll
+    for (int v = 0; v < CV; ++v) M[v] = Op::identity();
+    look_back_continue<Op, IO, CV, TC, KW>(p, c - 1, chain, b, d_first, ch, win, M, hin);
 }
 
 template <class Op, typename IO, int CV, int TC>
@@ -657,7 +665,8 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const Sca
 // fold over its R rows, the scan across the warp's J row groups, the warp's
 // summary to shared memory; pairs and the thread's exclusive prefix stay in
 // registers), then phase B of tile n-1 (replay from the thread's incoming
-// state, streaming stores).
+// state, streaming stores).  With R = 8 rows per thread two tiles' pairs no
+// longer fit in registers, and phase B of tile n follows its own phase A.
 //
 // Carry warp: it resolves tile n's incoming state (a look-back over earlier
 // chunks only) while the data warps are still in phase A of tile n, so once
@@ -745,6 +754,13 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
     // the bytes per element) the data warps' instruction issue is the limit,
     // so the carry warp does it.
     constexpr bool kFoldInData = sizeof(IO) == 4;
+    // Phase B of a tile runs one tile late (LAG) so the data warps never wait
+    // for the carry warp, at the price of holding two tiles' pairs in
+    // registers; with 8 rows per thread that no longer fits, so those tiles
+    // replay right after their own phase A and the per-tile work (warp scan,
+    // barriers, tile coordinates) is spread over twice the elements.
+    constexpr bool LAG = R < 8;
+    constexpr int NB = LAG ? 2 : 1;
     static_assert(sizeof(Vec) == V * sizeof(IO), "vector type matches the vector width");
     static_assert(CG * J == 32 && TC % 32 == 0, "lane layout");
     static_assert(TC * sizeof(IO) % 16 == 0 && TC <= 256 && TR <= 256, "TMA box");
@@ -793,23 +809,25 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
         IO *out = static_cast<IO *>(p.out);
         constexpr int V2 = V / 2;
 
-        // pairs of the two tiles in flight (tile parity), two channels per float2
-        float2 PA[2][R][V2], PB[2][R][V2];
-        float2 E[2][V];      // the thread's exclusive prefix within its warp, per channel
-        int64_t base[2];     // global offset of the thread's first element of the tile
-        int row0[2];         // first row (along T) of the thread's rows
-        bool full[2];        // all R rows and V channels of the thread inside the tensor
-        bool dvalid[2];
+        // pairs of the tiles in flight (two with the lag, by tile parity), two
+        // channels per float2
+        float2 PA[NB][R][V2], PB[NB][R][V2];
+        float2 E[NB][V];     // the thread's exclusive prefix within its warp, per channel
+        int64_t base[NB];    // global offset of the thread's first element of the tile
+        int row0[NB];        // first row (along T) of the thread's rows
+        bool full[NB];       // all R rows and V channels of the thread inside the tensor
+        bool dvalid[NB];
         uint32_t wait_limit = kMbarLimit;
 
         auto phaseA = [&](int n, auto bufc) {
             constexpr int BUF = decltype(bufc)::value;
+            constexpr int SB = LAG ? BUF : 0;
             const TileCoord tc = tile_coord(p, uint32_t(first + int64_t(n) * G));
             const int64_t d0 = int64_t(tc.dt) * TC + g * V;
-            dvalid[BUF] = d0 < p.D;
-            row0[BUF] = int(tc.c) * TR + (warp * J + j) * R;
-            full[BUF] = dvalid[BUF] && (row0[BUF] + R <= p.T);
-            base[BUF] = (int64_t(tc.b) * p.T) * p.D + d0;
+            dvalid[SB] = d0 < p.D;
+            row0[SB] = int(tc.c) * TR + (warp * J + j) * R;
+            full[SB] = dvalid[SB] && (row0[SB] + R <= p.T);
+            base[SB] = (int64_t(tc.b) * p.T) * p.D + d0;
             if (!mbar_wait(bars + 8u * uint32_t(n % S), uint32_t((n / S) & 1), wait_limit)) {
                 wait_limit = 1;
                 if (lane == 0) atomicOr(p.status, kTimeoutBit);
@@ -831,7 +849,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                     unpack(*reinterpret_cast<const Vec *>(t0 + r * TC), x0);
                     unpack(*reinterpret_cast<const Vec *>(t1 + r * TC), x1);
                     if (!FULL) {
-                        const bool ok = dvalid[BUF] && (row0[BUF] + r < p.T);
+                        const bool ok = dvalid[SB] && (row0[SB] + r < p.T);
 #pragma unroll
                         for (int v = 0; v < V; ++v) {
                             x0[v] = ok ? x0[v] : Op::pad0();
@@ -843,13 +861,13 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                         float a0, b0, a1, b1;
                         Op::element(x0[2 * i], x1[2 * i], a0, b0);
                         Op::element(x0[2 * i + 1], x1[2 * i + 1], a1, b1);
-                        PA[BUF][r][i] = make_float2(a0, a1);
-                        PB[BUF][r][i] = make_float2(b0, b1);
-                        Op::fold2(IA[i], IB[i], PA[BUF][r][i], PB[BUF][r][i]);
+                        PA[SB][r][i] = make_float2(a0, a1);
+                        PB[SB][r][i] = make_float2(b0, b1);
+                        Op::fold2(IA[i], IB[i], PA[SB][r][i], PB[SB][r][i]);
                     }
                 }
             };
-            if (full[BUF]) rows(std::true_type{});
+            if (full[SB]) rows(std::true_type{});
             else rows(std::false_type{});
             float2 incl[V];
 #pragma unroll
@@ -873,7 +891,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                 float2 o;
                 o.x = __shfl_up_sync(0xffffffffu, incl[v].x, CG);
                 o.y = __shfl_up_sync(0xffffffffu, incl[v].y, CG);
-                E[BUF][v] = (J > 1 && j > 0) ? o : Op::identity();
+                E[SB][v] = (J > 1 && j > 0) ? o : Op::identity();
             }
             if (j == J - 1) {
 #pragma unroll
@@ -915,6 +933,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
 
         auto phaseB = [&](auto bufc) {
             constexpr int BUF = decltype(bufc)::value;
+            constexpr int SB = LAG ? BUF : 0;
             named_barrier_sync(3 + BUF, NT);
             float2 st[V2];
 #pragma unroll
@@ -922,19 +941,19 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                 const int c0 = g * V + 2 * i;
                 const float w0 = Op::apply(s_tot[BUF][warp][c0], s_hin[BUF][c0]);
                 const float w1 = Op::apply(s_tot[BUF][warp][c0 + 1], s_hin[BUF][c0 + 1]);
-                st[i] = make_float2(Op::apply(E[BUF][2 * i], w0), Op::apply(E[BUF][2 * i + 1], w1));
+                st[i] = make_float2(Op::apply(E[SB][2 * i], w0), Op::apply(E[SB][2 * i + 1], w1));
             }
-            IO *dst = out + base[BUF] + int64_t(row0[BUF]) * p.D;
+            IO *dst = out + base[SB] + int64_t(row0[SB]) * p.D;
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 float y[V];
 #pragma unroll
                 for (int i = 0; i < V2; ++i) {
-                    st[i] = Op::step2(PA[BUF][r][i], PB[BUF][r][i], st[i]);
+                    st[i] = Op::step2(PA[SB][r][i], PB[SB][r][i], st[i]);
                     y[2 * i] = st[i].x;
                     y[2 * i + 1] = st[i].y;
                 }
-                if (full[BUF] || (dvalid[BUF] && row0[BUF] + r < p.T)) Access<IO, V>::store(dst, y);
+                if (full[SB] || (dvalid[SB] && row0[SB] + r < p.T)) Access<IO, V>::store(dst, y);
                 dst += p.D;
             }
         };
@@ -942,18 +961,31 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
         using B0 = std::integral_constant<int, 0>;
         using B1 = std::integral_constant<int, 1>;
         int n = 0;
-        for (; n + 1 < n_local; n += 2) {
-            phaseA(n, B0{});
-            if (n >= 1) phaseB(B1{});
-            phaseA(n + 1, B1{});
-            phaseB(B0{});
-        }
-        if (n < n_local) {
-            phaseA(n, B0{});
-            if (n >= 1) phaseB(B1{});
-            phaseB(B0{});
-        } else if (n_local >= 1) {
-            phaseB(B1{});
+        if constexpr (LAG) {
+            for (; n + 1 < n_local; n += 2) {
+                phaseA(n, B0{});
+                if (n >= 1) phaseB(B1{});
+                phaseA(n + 1, B1{});
+                phaseB(B0{});
+            }
+            if (n < n_local) {
+                phaseA(n, B0{});
+                if (n >= 1) phaseB(B1{});
+                phaseB(B0{});
+            } else if (n_local >= 1) {
+                phaseB(B1{});
+            }
+        } else {
+            for (; n + 1 < n_local; n += 2) {
+                phaseA(n, B0{});
+                phaseB(B0{});
+                phaseA(n + 1, B1{});
+                phaseB(B1{});
+            }
+            if (n < n_local) {
+                phaseA(n, B0{});
+                phaseB(B0{});
+            }
         }
     } else {
         // ============================================== carry warp
@@ -987,13 +1019,27 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
             const int64_t dl = int64_t(tc.dt) * TC + ch;
             const bool publish = (p.n_chunks > 1) && (c < p.n_chunks - 1) && (tile != p.drop_tile);
             // The incoming state depends only on earlier chunks: resolve it
-            // while the data warps are still in phase A of this tile.
+            // while the data warps are still in phase A of this tile.  When
+            // this warp publishes the tile's summary itself (bf16), it must not
+            // wait for earlier chunks first -- the next chunk's look-back may
+            // be waiting for that summary, and waiting here would chain the
+            // chunks of a channel tile one after another -- so it only walks
+            // the window already loaded and finishes the walk after publishing.
             float hin[CV];
+            float2 M[CV];
+            int64_t q = c - 1;
+            bool resolved = true;
             if (c == 0) {
 #pragma unroll
                 for (int v = 0; v < CV; ++v) hin[v] = init[v];
-            } else {
+            } else if constexpr (kFoldInData) {
                 look_back_from<Op, IO, CV, TC, KW>(p, c, tc.chain, tc.b, dl, ch, win, hin);
+            } else {
+#pragma unroll
+                for (int v = 0; v < CV; ++v) M[v] = Op::identity();
+                int consumed;
+                resolved = resolve_window<Op, IO, CV, TC, KW>(p, q, win, tc.b, dl, M, hin, consumed);
+                q -= consumed;
             }
             named_barrier_sync(1 + PB, NT);
             if constexpr (!kFoldInData) {
@@ -1002,6 +1048,10 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
 #pragma unroll
                 for (int v = 0; v < CV; ++v) s_total[PB][ch + v] = total[v];
                 if (publish && c > 0) publish_summary<CV, TC>(p, tile, ch, total);
+                if (!resolved) {
+                    load_window<CV, TC, KW>(p, q, tc.chain, ch, win);
+                    look_back_continue<Op, IO, CV, TC, KW>(p, q, tc.chain, tc.b, dl, ch, win, M, hin);
+                }
             }
 #pragma unroll
             for (int v = 0; v < CV; ++v) s_hin[PB][ch + v] = hin[v];

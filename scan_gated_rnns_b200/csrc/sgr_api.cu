@@ -75,6 +75,13 @@ template <typename IO> constexpr int pipe_cg() { return sizeof(IO) == 4 ? 8 : 16
 template <typename IO, int R, int W>
 constexpr size_t pipe_smem() { return PipeShape<IO, 4, pipe_cg<IO>(), R, kStages, W>::smem_bytes; }
 
+template <typename IO>
+size_t pipe_smem_for(int r, bool wide) {
+    if (r == 8) return wide ? pipe_smem<IO, 8, kPipeWarpsWide>() : pipe_smem<IO, 8, kPipeWarps>();
+    if (wide) return r == 2 ? pipe_smem<IO, 2, kPipeWarpsWide>() : pipe_smem<IO, 4, kPipeWarpsWide>();
+    return r == 2 ? pipe_smem<IO, 2, kPipeWarps>() : pipe_smem<IO, 4, kPipeWarps>();
+}
+
 // cuTensorMapEncodeTiled, fetched once from the driver through the runtime
 // (no link-time dependency on the driver library)
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -129,8 +136,11 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned)
         p.V = 4;
         p.cg = p.esz == 4 ? 8 : 16;
         p.TC = p.cg * p.V;
-        // rows per thread {2, 4}, automatic 4
-        p.r = (orr == 2 || orr == 4) ? orr : 4;
+        // rows per thread {2, 4, 8}; automatic: 4 for fp32, 8 for bf16, whose
+        // elements are half the bytes, so per-tile work (warp scan, barriers,
+        // hand-off) weighs twice as much per byte and is spread over twice
+        // the rows (replayed without the one-tile lag, see the kernel)
+        p.r = (orr == 2 || orr == 4 || orr == 8) ? orr : (p.esz == 2 ? 8 : 4);
         p.stages = kStages;
         // Block shape: about (blocks in flight) / n_chains chunks of one
         // channel tile are processed at once and a look-back folds that many
@@ -143,18 +153,13 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned)
         bool wide = n_chains > 0 && 2 * kAssumedSMs >= 8 * n_chains && tiles_wide >= 4 * kAssumedSMs;
         if (ok == KIND_PIPELINED) wide = false;
         if (ok == KIND_PIPELINED_WIDE) wide = true;
+        // 8 rows: bf16 only (fp32 tiles of 8 rows exceed the TMA box with 15
+        // warps and leave shared memory for one 7-warp block per SM)
+        if (p.r == 8 && p.esz == 4) p.r = 4;
         p.kind = wide ? KIND_PIPELINED_WIDE : KIND_PIPELINED;
         p.warps = wide ? kPipeWarpsWide : kPipeWarps;
         p.TR = p.warps * (32 / p.cg) * p.r;
-        if (p.esz == 4) {
-            p.smem = wide ? (p.r == 4 ? pipe_smem<float, 4, kPipeWarpsWide>() : pipe_smem<float, 2, kPipeWarpsWide>())
-                          : (p.r == 4 ? pipe_smem<float, 4, kPipeWarps>() : pipe_smem<float, 2, kPipeWarps>());
-        } else {
-            p.smem = wide ? (p.r == 4 ? pipe_smem<__nv_bfloat16, 4, kPipeWarpsWide>()
-                                      : pipe_smem<__nv_bfloat16, 2, kPipeWarpsWide>())
-                          : (p.r == 4 ? pipe_smem<__nv_bfloat16, 4, kPipeWarps>()
-                                      : pipe_smem<__nv_bfloat16, 2, kPipeWarps>());
-        }
+        p.smem = p.esz == 4 ? pipe_smem_for<float>(p.r, wide) : pipe_smem_for<__nv_bfloat16>(p.r, wide);
     } else {
         // tile kernel: 8 lanes x one vector (32 fp32 / 64 bf16 channels,
         // 128-byte row segments) or, unaligned, 32 lanes x 1 channel
@@ -310,10 +315,16 @@ template <class Op, typename IO>
 cudaError_t dispatch(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
     constexpr int VW = 16 / int(sizeof(IO));
     if (pl.kind == KIND_PIPELINED) {
+        if constexpr (sizeof(IO) == 2) {
+            if (pl.r == 8) return launch_pipelined<Op, IO, 4, 8, kPipeWarps>(sp, s, nullptr);
+        }
         return pl.r == 2 ? launch_pipelined<Op, IO, 4, 2, kPipeWarps>(sp, s, nullptr)
                          : launch_pipelined<Op, IO, 4, 4, kPipeWarps>(sp, s, nullptr);
     }
     if (pl.kind == KIND_PIPELINED_WIDE) {
+        if constexpr (sizeof(IO) == 2) {
+            if (pl.r == 8) return launch_pipelined<Op, IO, 4, 8, kPipeWarpsWide>(sp, s, nullptr);
+        }
         return pl.r == 2 ? launch_pipelined<Op, IO, 4, 2, kPipeWarpsWide>(sp, s, nullptr)
                          : launch_pipelined<Op, IO, 4, 4, kPipeWarpsWide>(sp, s, nullptr);
     }

@@ -64,7 +64,7 @@ def _reset_hooks():
 
 
 # (kernel, rows per thread): the tile kernel and the pipelined kernel, every R
-VARIANTS = [(1, 1), (1, 2), (1, 4), (1, 8), (2, 2), (2, 4), (3, 2), (3, 4)]
+VARIANTS = [(1, 1), (1, 2), (1, 4), (1, 8), (2, 2), (2, 4), (2, 8), (3, 2), (3, 4)]
 
 
 # ------------------------------------------------------------------ minGRU
