@@ -22,6 +22,11 @@ Functions (all inputs are widened exactly to float64 first):
 ``minmax(r, s, x0=None)``
     MinMax neuron x_{t+1} = max(min(r_t, x_t), s_t); page "MinMax Recurrent
     Neural Cascades" (The model, item 3).
+``mingru_backward(k, hx, h0, gy)`` / ``minmax_backward(r, s, x0, gy)``
+    gradients of a loss with dL/d out = gy with respect to both inputs and the
+    initial state, by the chain rule through the sequential loop (forward
+    recomputed in fp64); MinMax ties share the gradient evenly, as PyTorch's
+    elementwise minimum/maximum do.
 
 Arrays are (B, T, D); optional states are (B, D).  ``threads`` splits the batch
 over Python threads (ctypes releases the GIL during the C call).
@@ -65,6 +70,10 @@ def _open(path: str):
         fn = getattr(lib, name)
         fn.restype = ctypes.c_int
         fn.argtypes = [dp, dp, dp, i64, dp, i64, i64, i64]
+    for name in ("oracle_mingru_backward", "oracle_minmax_backward"):
+        fn = getattr(lib, name)
+        fn.restype = ctypes.c_int
+        fn.argtypes = [dp, dp, dp, i64, dp, dp, dp, dp, i64, i64, i64]
     return lib
 
 
@@ -154,3 +163,44 @@ def mingru_step(k_t, hx_t, h_prev=None) -> np.ndarray:
     B, D = k_t.shape
     h = mingru_linear(k_t.reshape(B, 1, D), hx_t.reshape(B, 1, D), h_prev)
     return h.reshape(B, D)
+
+
+def _run_backward(name: str, p, q, init, gy, threads: int):
+    p, q, gy = _as_f64(p), _as_f64(q), _as_f64(gy)
+    if p.ndim != 3 or p.shape != q.shape or p.shape != gy.shape:
+        raise ValueError(f"inputs must be three (B, T, D) arrays of one shape, got {p.shape} {q.shape} {gy.shape}")
+    B, T, D = p.shape
+    dp, dq = np.empty_like(p), np.empty_like(p)
+    dinit = np.empty((B, D), dtype=np.float64)
+    if init is not None:
+        init = _as_f64(init).reshape(B, D)
+    fn = getattr(_load(), name)
+
+    def one(b0: int, b1: int) -> None:
+        if b1 <= b0:
+            return
+        ip = _ptr(init[b0:b1]) if init is not None else None
+        rc = fn(_ptr(p[b0:b1]), _ptr(q[b0:b1]), ip, D, _ptr(gy[b0:b1]), _ptr(dp[b0:b1]),
+                _ptr(dq[b0:b1]), _ptr(dinit[b0:b1]), b1 - b0, T, D)
+        if rc != 0:
+            raise RuntimeError(f"{name} returned {rc}")
+
+    threads = max(1, min(int(threads), B)) if B > 0 else 1
+    if threads == 1:
+        one(0, B)
+    else:
+        bounds = np.linspace(0, B, threads + 1).astype(int)
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(lambda i: one(bounds[i], bounds[i + 1]), range(threads)))
+    return dp, dq, dinit
+
+
+def mingru_backward(k, hx, h0, gy, threads: int = 1):
+    """(dk, dhx, dh0) of a loss with dL/dh = gy (fp64; dh0 is (B, D) whether
+    or not h0 is given: the gradient with respect to the initial state)."""
+    return _run_backward("oracle_mingru_backward", k, hx, h0, gy, threads)
+
+
+def minmax_backward(r, s, x0, gy, threads: int = 1):
+    """(dr, ds, dx0) of a loss with dL/d out = gy (fp64; ties share evenly)."""
+    return _run_backward("oracle_minmax_backward", r, s, x0, gy, threads)

@@ -183,3 +183,115 @@ int oracle_minmax(const double *r, const double *s,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------ gradients */
+
+/*
+ * Reverse mode through the same recurrences, for a loss L whose gradient
+ * with respect to every output row is given: gy[b, t, d] = dL/d out[b, t, d].
+ * The pages name training with bounded gradients as a property of the
+ * MinMax model (page "MinMax Recurrent Neural Cascades", Key properties) and
+ * show the minGRU layer as a trainable torch module (page "Mingru
+ * Pytorch"); neither prints the derivative, so it is taken here from the
+ * chain rule through the sequential loop, channel by channel:
+ *   lam       = dL/d state_t flowing back from steps after t (0 after the last)
+ *   delta_t   = gy_t + lam                           (total dL/d out_t)
+ *   d input_t = delta_t * d out_t / d input_t
+ *   lam       = delta_t * d out_t / d state_{t-1}     (moves one step back)
+ * and after t = 0, lam is the gradient with respect to the initial state.
+ * The forward states are recomputed here in fp64; dinit may be NULL.
+ */
+
+/*
+ * minGRU: out_t = h_t = (1 - z_t) h_{t-1} + z_t g(hx_t), z_t = sigmoid(k_t).
+ *   dh_t/dk_t     = z_t (1 - z_t) (g(hx_t) - h_{t-1})
+ *                   (d sigmoid(k)/dk = z (1 - z), d (1 - z)/dk = -z (1 - z))
+ *   dh_t/dhx_t    = z_t g'(hx_t),  g'(x) = 1 (x >= 0), sigmoid(x) sigmoid(-x) (x < 0)
+ *   dh_t/dh_{t-1} = 1 - z_t
+ */
+int oracle_mingru_backward(const double *k, const double *hx,
+                           const double *h0, int64_t h0_bs, const double *gy,
+                           double *dk, double *dhx, double *dh0,
+                           int64_t B, int64_t T, int64_t D)
+{
+    if (B < 0 || T < 0 || D < 0) return 1;
+    double *h = malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    if (!h) return 2;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t d = 0; d < D; ++d) {
+            double init = h0 ? h0[b * h0_bs + d] : 0.0;
+            /* forward, this channel only */
+            double prev = init;
+            for (int64_t t = 0; t < T; ++t) {
+                int64_t i = (b * T + t) * D + d;
+                prev = sigmoid(-k[i]) * prev + sigmoid(k[i]) * g_act(hx[i]);
+                h[t] = prev;
+            }
+            /* backward */
+            double lam = 0.0;
+            for (int64_t t = T - 1; t >= 0; --t) {
+                int64_t i = (b * T + t) * D + d;
+                double delta = gy[i] + lam;
+                double hprev = (t > 0) ? h[t - 1] : init;
+                double z = sigmoid(k[i]);
+                double one_minus_z = sigmoid(-k[i]);
+                double x = hx[i];
+                double g = g_act(x);
+                double gprime = (x >= 0.0) ? 1.0 : sigmoid(x) * sigmoid(-x);
+                dk[i] = delta * z * one_minus_z * (g - hprev);
+                dhx[i] = delta * z * gprime;
+                lam = delta * one_minus_z;
+            }
+            if (dh0) dh0[b * D + d] = lam;
+        }
+    }
+    free(h);
+    return 0;
+}
+
+/*
+ * MinMax: out_t = x_{t+1} = max(m_t, s_t), m_t = min(r_t, x_t).  min and max
+ * are differentiated the way PyTorch's elementwise minimum/maximum are: the
+ * selected operand gets the whole gradient and equal operands share it
+ * evenly (the plainest reading for a model trained with autograd; the pages
+ * do not state a rule for ties).
+ *   dm/dr = 1 if r < x, 1/2 if r == x, 0 if r > x;   dm/dx = 1 - dm/dr
+ *   dout/dm = 1 if m > s, 1/2 if m == s, 0 if m < s;  dout/ds = 1 - dout/dm
+ */
+int oracle_minmax_backward(const double *r, const double *s,
+                           const double *x0, int64_t x0_bs, const double *gy,
+                           double *dr, double *ds, double *dx0,
+                           int64_t B, int64_t T, int64_t D)
+{
+    if (B < 0 || T < 0 || D < 0) return 1;
+    double *x = malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    if (!x) return 2;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t d = 0; d < D; ++d) {
+            double init = x0 ? x0[b * x0_bs + d] : 0.0;
+            double state = init;
+            for (int64_t t = 0; t < T; ++t) {
+                int64_t i = (b * T + t) * D + d;
+                state = fmax(fmin(r[i], state), s[i]);
+                x[t] = state;
+            }
+            double lam = 0.0;
+            for (int64_t t = T - 1; t >= 0; --t) {
+                int64_t i = (b * T + t) * D + d;
+                double delta = gy[i] + lam;
+                double xprev = (t > 0) ? x[t - 1] : init;
+                double m = fmin(r[i], xprev);
+                double dm_dr = (r[i] < xprev) ? 1.0 : ((r[i] == xprev) ? 0.5 : 0.0);
+                double dm_dx = 1.0 - dm_dr;
+                double dout_dm = (m > s[i]) ? 1.0 : ((m == s[i]) ? 0.5 : 0.0);
+                double dout_ds = 1.0 - dout_dm;
+                dr[i] = delta * dout_dm * dm_dr;
+                ds[i] = delta * dout_ds;
+                lam = delta * dout_dm * dm_dx;
+            }
+            if (dx0) dx0[b * D + d] = lam;
+        }
+    }
+    free(x);
+    return 0;
+}

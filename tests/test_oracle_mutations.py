@@ -14,6 +14,7 @@ import subprocess
 import pytest
 
 import oracle
+import test_oracle_backward_pins as bpins
 import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(os.path.abspath(oracle.__file__)), "oracle.c")
@@ -45,6 +46,27 @@ MUTANTS = {
     "minmax_r_s_swapped": ("x[i] = fmax(fmin(r[i], state), s[i]);",
                            "x[i] = fmax(fmin(s[i], state), r[i]);"),
     "minmax_x0_dropped": ("state = x0 ? x0[b * x0_bs + d] : 0.0;", "state = 0.0;"),
+    # minGRU gradient
+    "bwd_dk_sign": ("dk[i] = delta * z * one_minus_z * (g - hprev);",
+                    "dk[i] = delta * z * one_minus_z * (hprev - g);"),
+    "bwd_dk_missing_gate": ("dk[i] = delta * z * one_minus_z * (g - hprev);",
+                            "dk[i] = delta * z * (g - hprev);"),
+    "bwd_hprev_off_by_one": ("double hprev = (t > 0) ? h[t - 1] : init;",
+                             "double hprev = h[t];"),
+    "bwd_gprime_branch": ("double gprime = (x >= 0.0) ? 1.0 : sigmoid(x) * sigmoid(-x);",
+                          "double gprime = (x >= 0.0) ? 1.0 : sigmoid(x);"),
+    "bwd_state_gradient_gate": ("lam = delta * one_minus_z;", "lam = delta * z;"),
+    "bwd_direct_gradient_dropped": ("double delta = gy[i] + lam;\n                double hprev",
+                                    "double delta = lam + (t == T - 1 ? gy[i] : 0.0);\n                double hprev"),
+    "bwd_forward_without_h0": ("            double prev = init;", "            double prev = 0.0;"),
+    # MinMax gradient
+    "bwd_minmax_tie_to_r": ("double dm_dr = (r[i] < xprev) ? 1.0 : ((r[i] == xprev) ? 0.5 : 0.0);",
+                            "double dm_dr = (r[i] <= xprev) ? 1.0 : 0.0;"),
+    "bwd_minmax_tie_to_s": ("double dout_dm = (m > s[i]) ? 1.0 : ((m == s[i]) ? 0.5 : 0.0);",
+                            "double dout_dm = (m > s[i]) ? 1.0 : 0.0;"),
+    "bwd_minmax_state_path": ("lam = delta * dout_dm * dm_dx;", "lam = delta * dm_dx;"),
+    "bwd_minmax_r_s_swapped": ("dr[i] = delta * dout_dm * dm_dr;\n                ds[i] = delta * dout_ds;",
+                               "ds[i] = delta * dout_dm * dm_dr;\n                dr[i] = delta * dout_ds;"),
 }
 
 
@@ -66,6 +88,19 @@ def _pin_checks():
         out.append(lambda a=args: pins.test_constant_inputs_closed_form(*a))
     for T in (1, 2):
         out.append(lambda t=T: pins.test_minmax_brute_force(t))
+    # gradient pins
+    for shape in [(1, 1, 1), (2, 7, 3)]:
+        for wh in (False, True):
+            out.append(lambda a=shape, b=wh: bpins.test_mingru_backward_matches_autograd(a, b, 0.0))
+    out += [bpins.test_mingru_backward_one_step_closed_form,
+            bpins.test_mingru_backward_state_gradient_is_product_of_gates,
+            bpins.test_mingru_backward_convex_combination_conserves_gradient,
+            bpins.test_mingru_backward_saturated_gates,
+            bpins.test_minmax_backward_default_state_is_zero,
+            bpins.test_minmax_backward_gradient_weights_are_bounded]
+    for seed in range(2):
+        out.append(lambda sd=seed: bpins.test_minmax_backward_matches_autograd_with_ties(sd))
+        out.append(lambda sd=seed: bpins.test_minmax_backward_conserves_gradient(sd))
     return out
 
 
