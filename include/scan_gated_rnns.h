@@ -167,6 +167,62 @@ SGR_API sgr_status_t mingru_scan_noalloc(const void *k, const void *hx,
                                          void *h, int64_t B, int64_t T, int64_t D,
                                          sgr_dtype_t dtype, cudaStream_t stream);
 
+/* ------------------------------------------------------------ gradients */
+
+/*
+ * mingru_scan_backward -- gradients of a loss L through mingru_scan, given the
+ * upstream gradient dh = dL/dh (B, T, D) for every output row.  The pages
+ * show the minGRU layer as a trainable module (page "Mingru Pytorch") but
+ * print no derivative; this is the chain rule through the recurrence
+ * h_t = (1 - z_t) h_{t-1} + z_t g(hx_t):
+ *     delta_t = dh_t + (1 - z_{t+1}) delta_{t+1}          (delta_T+1 = 0)
+ *     dk_t    = delta_t z_t (1 - z_t) (g(hx_t) - h_{t-1})
+ *     dhx_t   = delta_t z_t g'(hx_t),  g'(x) = 1 (x >= 0), sigmoid(x) sigmoid(-x)
+ *     dh0     = (1 - z_1) delta_1  (gradient with respect to the initial state)
+ * computed as a reverse-time chunked scan (one kernel, decoupled look-back).
+ *   k, hx, h0, h0_batch_stride : the forward call's inputs (h0 may be NULL)
+ *   h     : the forward call's output (B, T, D); h_{t-1} is read from it
+ *   dh    : dL/dh (B, T, D)
+ *   dk, dhx : outputs (B, T, D)
+ *   dh0   : optional output rows (B, D), batch stride dh0_batch_stride
+ *           (>= D when B > 1); written whether or not h0 was given (the
+ *           gradient with respect to a zero initial state); NULL: not written
+ *   workspace: ws_bytes >= sgr_backward_workspace_size(SGR_OP_MINGRU, ...),
+ *           same rules as the forward workspace (zero-filled once).
+ * All tensors share dtype; arithmetic is fp32.  Outputs must not overlap any
+ * input or each other (SGR_ERR_INVALID_ARG).  T = 0 writes dh0 = 0.
+ */
+SGR_API sgr_status_t mingru_scan_backward(const void *k, const void *hx,
+                                          const void *h0, int64_t h0_batch_stride,
+                                          const void *h, const void *dh,
+                                          void *dk, void *dhx,
+                                          void *dh0, int64_t dh0_batch_stride,
+                                          int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
+                                          void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * minmax_scan_backward -- gradients through minmax_scan for dx = dL/dx
+ * (B, T, D), x the forward output (x[t] = x_{t+1}).  The neuron selects one
+ * operand per step, x_{t+1} = max(m_t, s_t), m_t = min(r_t, x_t); the gradient
+ * flows to the selected operand, and equal operands of a min or a max share
+ * it evenly (the rule of PyTorch's elementwise minimum / maximum, the
+ * framework the page's package is written in; the page "MinMax Recurrent
+ * Neural Cascades" gives no rule for ties).  Arguments as
+ * mingru_scan_backward: r, s, x0 (NULL: +0) the forward inputs; dr, ds, dx0
+ * the outputs.
+ */
+SGR_API sgr_status_t minmax_scan_backward(const void *r, const void *s,
+                                          const void *x0, int64_t x0_batch_stride,
+                                          const void *x, const void *dx,
+                                          void *dr, void *ds,
+                                          void *dx0, int64_t dx0_batch_stride,
+                                          int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
+                                          void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Bytes of workspace a gradient call of this shape needs (0: none).  Pure host code. */
+SGR_API size_t sgr_backward_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D,
+                                           sgr_dtype_t dtype);
+
 /* ---------------------------------------------------- host-buffer scans */
 
 /*

@@ -68,6 +68,11 @@ SIGNATURES.update({
     "sgr_set_kernel_override": (_int, [_int]),
     "mingru_scan_noalloc": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _i64, _i64, _int, _vp]),
     "sgr_host_staging_size": (_sz, [_int, _i64, _i64, _i64, _int, _int]),
+    "mingru_scan_backward": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _i64,
+                                    _i64, _i64, _i64, _int, _vp, _sz, _vp]),
+    "minmax_scan_backward": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _i64,
+                                    _i64, _i64, _i64, _int, _vp, _sz, _vp]),
+    "sgr_backward_workspace_size": (_sz, [_int, _i64, _i64, _i64, _int]),
     "mingru_scan_host": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _i64, _i64, _int, _int, _vp, _sz, _vp]),
     "minmax_scan_host": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _i64, _i64, _int, _int, _vp, _sz, _vp]),
 })

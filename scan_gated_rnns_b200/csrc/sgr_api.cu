@@ -2,6 +2,7 @@
 // argument checks, the choice of chunk shape, the workspace layout and the
 // kernel launches.  No allocation, no synchronisation on the scan paths.
 #include "scan_gated_rnns.h"
+#include "scan_backward.cuh"
 #include "scan_engine.cuh"
 
 #include <algorithm>
@@ -123,13 +124,16 @@ bool make_operand_map(CUtensorMap *map, const void *ptr, int64_t B, int64_t T, i
 // (fp32: 7 x 4 x R rows x 32 channels; bf16: 7 x 2 x R rows x 64 channels;
 // 128-byte row segments); anything else takes the tile kernel's scalar
 // variant.  The override knobs select the kernel and the rows per thread.
-Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned) {
+// force_tile: the tile kernel whatever the alignment (the gradient kernel,
+// which keeps four values per element live, also caps a thread at 16 elements)
+Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
+               bool force_tile = false) {
     Plan p;
     p.esz = (dtype == SGR_BF16) ? 2 : 4;
     const int vw = 16 / p.esz;
     p.vec = aligned && (D % vw == 0);
     const int ok = g_override_kind.load();
-    p.kind = (p.vec && ok != KIND_TILE) ? KIND_PIPELINED : KIND_TILE;
+    p.kind = (p.vec && ok != KIND_TILE && !force_tile) ? KIND_PIPELINED : KIND_TILE;
     const int orr = g_override_r.load();
     if (p.kind == KIND_PIPELINED) {
         // 4 channels per lane (16-byte fp32 / 8-byte bf16 vectors)
@@ -182,6 +186,9 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned)
                 const int64_t chunks = (T + tr - 1) / tr;
                 if (n_chains * chunks >= kTargetTiles || cand == 1) { r = cand; break; }
             }
+        }
+        if (force_tile) {
+            while (r > 1 && r * p.V > 16) r /= 2;
         }
         p.r = r;
         p.TR = kWarps * J * r;
@@ -392,6 +399,125 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
     return e == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
 }
 
+// ---- gradients: the reverse-time tile kernel (scan_backward.cuh)
+template <class BOp, typename IO, int V, int CG, int R>
+cudaError_t launch_bwd_tile(const BwdParams &bp, cudaStream_t s) {
+    if constexpr (R * V > 16) {
+        return cudaErrorInvalidConfiguration;   // never planned (see make_plan)
+    } else {
+        // registers a data thread keeps live: four values per element, the
+        // pair per channel and about 24 for addressing; blocks of 256 threads
+        constexpr int NEED = 4 * R * V + 2 * V + 24;
+        constexpr int MINB = NEED <= 56 ? 4 : (NEED <= 72 ? 3 : 2);
+        scan_backward_kernel<BOp, IO, V, CG, R, kWarps, MINB>
+            <<<unsigned(bp.s.n_tiles), (kWarps + 1) * 32, 0, s>>>(bp);
+        return cudaGetLastError();
+    }
+}
+
+template <class BOp, typename IO, int V, int CG>
+cudaError_t dispatch_bwd_r(const Plan &pl, const BwdParams &bp, cudaStream_t s) {
+    switch (pl.r) {
+        case 1: return launch_bwd_tile<BOp, IO, V, CG, 1>(bp, s);
+        case 2: return launch_bwd_tile<BOp, IO, V, CG, 2>(bp, s);
+        case 4: return launch_bwd_tile<BOp, IO, V, CG, 4>(bp, s);
+        default: return launch_bwd_tile<BOp, IO, V, CG, 8>(bp, s);
+    }
+}
+
+template <class BOp, typename IO>
+cudaError_t dispatch_bwd(const Plan &pl, const BwdParams &bp, cudaStream_t s) {
+    constexpr int VW = 16 / int(sizeof(IO));
+    if (!pl.vec) return dispatch_bwd_r<BOp, IO, 1, 32>(pl, bp, s);
+    return dispatch_bwd_r<BOp, IO, VW, 8>(pl, bp, s);
+}
+
+sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, const void *init,
+                               int64_t init_bs, const void *fwd, const void *gy, void *out0,
+                               void *out1, void *dinit, int64_t dinit_bs, int64_t B, int64_t T,
+                               int64_t D, sgr_dtype_t dtype, void *ws, size_t ws_bytes,
+                               cudaStream_t stream) {
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
+    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return SGR_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || D < 0 || init_bs < 0 || dinit_bs < 0) return SGR_ERR_INVALID_ARG;
+    if (B == 0 || D == 0) return SGR_OK;
+    if (dinit && B > 1 && dinit_bs < D) return SGR_ERR_INVALID_ARG;   // rows would overlap
+    const int esz = dtype == SGR_BF16 ? 2 : 4;
+    int64_t n = 0, nbytes = 0, tmp = 0;
+    if (!mul_ok(B, T, &n) || !mul_ok(n, D, &n) || !mul_ok(n, esz, &nbytes)) return SGR_ERR_UNSUPPORTED;
+    for (int64_t bs : {init_bs, dinit_bs})
+        if (!mul_ok(B - 1, bs, &tmp) || !mul_ok(tmp + D, esz, &tmp)) return SGR_ERR_UNSUPPORTED;
+    const size_t db = dinit ? rows_span(B, D, dinit_bs, esz) : 0;
+    if (T == 0) {
+        // no steps: the gradient reaching the initial state is zero
+        if (dinit) {
+            if (dinit_bs == D || B == 1) {
+                if (cudaMemsetAsync(dinit, 0, size_t(D) * esz * (B == 1 ? 1 : B), stream) != cudaSuccess)
+                    return SGR_ERR_CUDA;
+            } else if (cudaMemset2DAsync(dinit, size_t(dinit_bs) * esz, 0, size_t(D) * esz, size_t(B),
+                                         stream) != cudaSuccess) {
+                return SGR_ERR_CUDA;
+            }
+        }
+        return SGR_OK;
+    }
+    if (!in0 || !in1 || !fwd || !gy || !out0 || !out1) return SGR_ERR_INVALID_ARG;
+    const size_t tb = size_t(nbytes);
+    const size_t ib = init ? rows_span(B, D, init_bs, esz) : 0;
+    const void *ins[5] = {in0, in1, fwd, gy, init};
+    const size_t in_bytes[5] = {tb, tb, tb, tb, ib};
+    for (int i = 0; i < 5; ++i) {
+        if (overlaps(out0, tb, ins[i], in_bytes[i]) || overlaps(out1, tb, ins[i], in_bytes[i]) ||
+            overlaps(dinit, db, ins[i], in_bytes[i]))
+            return SGR_ERR_INVALID_ARG;
+    }
+    if (overlaps(out0, tb, out1, tb) || overlaps(out0, tb, dinit, db) || overlaps(out1, tb, dinit, db))
+        return SGR_ERR_INVALID_ARG;
+
+    const bool aligned = aligned16(in0) && aligned16(in1) && aligned16(fwd) && aligned16(gy) &&
+                         aligned16(out0) && aligned16(out1);
+    const Plan pl = make_plan(B, T, D, dtype, aligned, true);
+    if (pl.n_tiles > int64_t(std::numeric_limits<int>::max())) return SGR_ERR_UNSUPPORTED;
+
+    BwdParams bp;
+    std::memset(&bp, 0, sizeof(bp));
+    ScanParams &sp = bp.s;
+    sp.in0 = in0; sp.in1 = in1; sp.init = nullptr; sp.init_bs = 0; sp.out = out0;
+    sp.B = B; sp.T = T; sp.D = D;
+    sp.n_dt = pl.n_dt; sp.n_chains = pl.n_chains; sp.n_chunks = pl.n_chunks; sp.n_tiles = pl.n_tiles;
+    sp.by_chains = make_fastdiv(uint32_t(pl.n_chains));
+    sp.by_dt = make_fastdiv(uint32_t(pl.n_dt));
+    sp.epoch = 0;
+    sp.spin_limit = g_spin_limit.load();
+    sp.drop_tile = g_drop_tile.load();
+    bp.fwd = fwd; bp.gy = gy; bp.init = init; bp.init_bs = init_bs;
+    bp.out1 = out1; bp.dinit = dinit; bp.dinit_bs = dinit_bs;
+    if (pl.n_chunks > 1) {
+        if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)) return SGR_ERR_WORKSPACE;
+        char *w = static_cast<char *>(ws);
+        sp.status = reinterpret_cast<uint32_t *>(w);
+        sp.words = reinterpret_cast<uint64_t *>(w + pl.off_words);
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return SGR_ERR_CUDA;
+        if (cs == cudaStreamCaptureStatusActive) {
+            if (cudaMemsetAsync(sp.words, 0, pl.ws_bytes - pl.off_words, stream) != cudaSuccess)
+                return SGR_ERR_CUDA;
+            sp.epoch = 1;
+        } else {
+            sp.epoch = next_epoch();
+        }
+    }
+    cudaError_t e;
+    if (op == SGR_OP_MINGRU) {
+        e = dtype == SGR_F32 ? dispatch_bwd<MinGRUBwd, float>(pl, bp, stream)
+                             : dispatch_bwd<MinGRUBwd, __nv_bfloat16>(pl, bp, stream);
+    } else {
+        e = dtype == SGR_F32 ? dispatch_bwd<MinMaxBwd, float>(pl, bp, stream)
+                             : dispatch_bwd<MinMaxBwd, __nv_bfloat16>(pl, bp, stream);
+    }
+    return e == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -443,6 +569,33 @@ sgr_status_t mingru_step(const void *k_t, int64_t k_bs, const void *hx_t, int64_
             static_cast<__nv_bfloat16 *>(h_out), ho_bs, B, D);
     }
     return cudaGetLastError() == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
+}
+
+sgr_status_t mingru_scan_backward(const void *k, const void *hx, const void *h0,
+                                  int64_t h0_batch_stride, const void *h, const void *dh, void *dk,
+                                  void *dhx, void *dh0, int64_t dh0_batch_stride, int64_t B,
+                                  int64_t T, int64_t D, sgr_dtype_t dtype, void *workspace,
+                                  size_t ws_bytes, cudaStream_t stream) {
+    return run_scan_backward(SGR_OP_MINGRU, k, hx, h0, h0_batch_stride, h, dh, dk, dhx, dh0,
+                             dh0_batch_stride, B, T, D, dtype, workspace, ws_bytes, stream);
+}
+
+sgr_status_t minmax_scan_backward(const void *r, const void *s, const void *x0,
+                                  int64_t x0_batch_stride, const void *x, const void *dx, void *dr,
+                                  void *ds, void *dx0, int64_t dx0_batch_stride, int64_t B,
+                                  int64_t T, int64_t D, sgr_dtype_t dtype, void *workspace,
+                                  size_t ws_bytes, cudaStream_t stream) {
+    return run_scan_backward(SGR_OP_MINMAX, r, s, x0, x0_batch_stride, x, dx, dr, ds, dx0,
+                             dx0_batch_stride, B, T, D, dtype, workspace, ws_bytes, stream);
+}
+
+size_t sgr_backward_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype) {
+    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return 0;
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return 0;
+    if (B <= 0 || T <= 0 || D <= 0) return 0;
+    const Plan a = make_plan(B, T, D, dtype, true, true);
+    const Plan b = make_plan(B, T, D, dtype, false, true);
+    return a.ws_bytes > b.ws_bytes ? a.ws_bytes : b.ws_bytes;
 }
 
 size_t sgr_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype) {

@@ -134,6 +134,49 @@ def minmax_scan(r: torch.Tensor, s: torch.Tensor, x0: Optional[torch.Tensor] = N
     return _scan("minmax_scan", _abi.SGR_OP_MINMAX, r, s, x0, out, workspace)
 
 
+def _scan_backward(fn: str, op: int, p, q, init, fwd, gy, want_dinit: bool, workspace):
+    for t, n in ((p, "first operand"), (q, "second operand"), (fwd, "forward output"),
+                 (gy, "upstream gradient")):
+        _seq(t, f"{fn}: {n}")
+        if t.shape != p.shape or t.dtype != p.dtype or t.device != p.device:
+            raise ValueError(f"{fn}: {n} must match the first operand's shape, dtype and device")
+    dt = _dtype_code(p, fn)
+    B, T, D = p.shape
+    ip, ibs = _rows(init, B, D, p, fn + ": initial state")
+    dp, dq = torch.empty_like(p), torch.empty_like(p)
+    dinit = torch.empty((B, D), dtype=p.dtype, device=p.device) if want_dinit else None
+    need = int(lib().sgr_backward_workspace_size(op, B, T, D, dt))
+    wp, wn = 0, 0
+    if need:
+        ws = workspace if workspace is not None else default_workspace(p.device, need)
+        wp, wn = ws.ptr, ws.nbytes
+    with torch.cuda.device(p.device):
+        code = getattr(lib(), fn)(p.data_ptr(), q.data_ptr(), ip, ibs, fwd.data_ptr(), gy.data_ptr(),
+                                  dp.data_ptr(), dq.data_ptr(),
+                                  dinit.data_ptr() if dinit is not None else 0, D,
+                                  B, T, D, dt, wp, wn, _stream(p.device))
+    check(fn, code)
+    return dp, dq, dinit
+
+
+def mingru_scan_backward(k: torch.Tensor, hx: torch.Tensor, h0: Optional[torch.Tensor],
+                         h: torch.Tensor, dh: torch.Tensor, want_dh0: bool = True,
+                         workspace: Optional[Workspace] = None):
+    """(dk, dhx, dh0) for dL/dh = dh through h = mingru_scan(k, hx, h0); dh0 is
+    (B, D) (or None when want_dh0 is false)."""
+    return _scan_backward("mingru_scan_backward", _abi.SGR_OP_MINGRU, k, hx, h0, h, dh, want_dh0,
+                          workspace)
+
+
+def minmax_scan_backward(r: torch.Tensor, s: torch.Tensor, x0: Optional[torch.Tensor],
+                         x: torch.Tensor, dx: torch.Tensor, want_dx0: bool = True,
+                         workspace: Optional[Workspace] = None):
+    """(dr, ds, dx0) for dL/dx = dx through x = minmax_scan(r, s, x0); equal
+    operands of a min or a max share the gradient evenly."""
+    return _scan_backward("minmax_scan_backward", _abi.SGR_OP_MINMAX, r, s, x0, x, dx, want_dx0,
+                          workspace)
+
+
 def mingru_step(k_t: torch.Tensor, hx_t: torch.Tensor, h_prev: Optional[torch.Tensor] = None,
                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One token: (B, D) rows in (any batch stride, contiguous along D), new

@@ -258,3 +258,86 @@ def test_host_staging_size():
     auto = size(B, T, D)
     assert 6 * (8 << 20) // 2 <= auto <= 6 * (8 << 20) // 2 + (4 << 20)
     assert size(2, 5, 3, op=MINMAX, chunks=2) > 0
+
+
+# ------------------------------------------------------------- gradients
+
+@pytest.mark.parametrize("fn", ["mingru_scan_backward", "minmax_scan_backward"])
+def test_backward_argument_errors(fn):
+    E = _abi.SGR_ERR_INVALID_ARG
+    G, O0, O1, DI = 0x60000000, 0x70000000, 0x80000000, 0x90000000
+
+    def call(p=A, q=Bp, init=None, ibs=0, fwd=C, gy=G, o0=O0, o1=O1, di=None, dbs=0,
+             B=2, T=4, D=8, dt=F32, ws=None, wn=0):
+        return scan(fn, p, q, init, ibs, fwd, gy, o0, o1, di, dbs, B, T, D, dt, ws, wn, None)
+
+    assert call(B=-1) == E
+    assert call(dt=7) == E
+    assert call(ibs=-1) == E
+    assert call(dbs=-8) == E
+    for kw in ({"p": None}, {"q": None}, {"fwd": None}, {"gy": None}, {"o0": None}, {"o1": None}):
+        assert call(**kw) == E
+    assert call(o0=A + 64) == E                   # output on an input
+    assert call(o1=G) == E
+    assert call(o1=O0 + 16) == E                  # the two outputs overlap
+    assert call(di=O1 + 32, dbs=8) == E           # initial-state gradient on an output
+    assert call(di=DI, dbs=4) == E                # its rows would overlap each other
+    for shp in [(0, 4, 4), (2, 4, 0)]:
+        B, T, D = shp
+        assert call(p=None, q=None, fwd=None, gy=None, o0=None, o1=None, B=B, T=T, D=D) == _abi.SGR_OK
+    assert call(B=1 << 40, T=1 << 20, D=1 << 10) == _abi.SGR_ERR_UNSUPPORTED
+    # long sequences need a workspace
+    assert call(B=1, T=1 << 16, D=64) == _abi.SGR_ERR_WORKSPACE
+    need = _abi.lib().sgr_backward_workspace_size(MINGRU, 1, 1 << 16, 64, F32)
+    assert need > 0
+    assert call(B=1, T=1 << 16, D=64, ws=0x50000000, wn=256) == _abi.SGR_ERR_WORKSPACE
+    assert call(B=1, T=1 << 16, D=64, ws=0x50000008, wn=need) == _abi.SGR_ERR_WORKSPACE   # misaligned
+
+
+@pytest.mark.parametrize("shape", [(2, 1000, 96), (1, 777, 36), (3, 129, 40), (1, 1, 1), (2, 300, 7)])
+@pytest.mark.parametrize("dtype", [F32, BF16])
+@pytest.mark.parametrize("aligned", [True, False])
+def test_backward_plan_reverse_indices(shape, dtype, aligned):
+    """Replay the gradient kernel's reverse-time indexing: every (b, t, d) is
+    written exactly once, the state row read (t - 1) is in range or the
+    initial state, and exactly one thread per channel ends at time row 0."""
+    B, T, D = shape
+    pl = _abi.plan(MINGRU, B, T, D, dtype, aligned)   # forward plan: only for V / layout
+    lib = _abi.lib()
+    assert lib.sgr_set_kernel_override(1) == 0       # the tile plan the gradient kernel uses
+    try:
+        pl = _abi.plan(MINGRU, B, T, D, dtype, aligned)
+    finally:
+        lib.sgr_set_kernel_override(0)
+    V, cg, R, W = pl["channels_per_thread"], pl["channel_lanes"], pl["rows_per_thread"], pl["warps"]
+    while R > 1 and R * V > 16:   # the gradient kernel's cap on elements per thread
+        R //= 2
+    J = 32 // cg
+    TR, TC = W * J * R, cg * V
+    n_dt = -(-D // TC)
+    n_chains = B * n_dt
+    n_chunks = -(-T // TR)
+    assert R * V <= 16
+    cover = np.zeros((B, T, D), dtype=np.int32)
+    ends_at_zero = np.zeros((B, D), dtype=np.int32)
+    for tile in range(n_chains * n_chunks):
+        c, chain = divmod(tile, n_chains)
+        b, dt = divmod(chain, n_dt)
+        ct = n_chunks - 1 - c
+        for warp in range(W):
+            for lane in range(32):
+                g, j = lane % cg, lane // cg
+                d0 = dt * TC + g * V
+                if d0 >= D:
+                    continue
+                top = ct * TR + TR - 1 - (warp * J + j) * R
+                for r in range(R):
+                    t = top - r
+                    assert t >= 0
+                    if t < T:
+                        cover[b, t, d0:d0 + V] += 1
+                        assert t - 1 >= -1
+                if top - (R - 1) == 0:
+                    ends_at_zero[b, d0:d0 + V] += 1
+    assert (cover == 1).all()
+    assert (ends_at_zero == 1).all()
