@@ -273,12 +273,64 @@ def measure_row(w, device, steps=10, warmup=3):
     gbs = bytes_ / per / 1e9
     plan = sgr._abi.plan(0 if w.op == "mingru" else 1, w.B, w.T, w.D,
                          0 if w.dtype == "f32" else 1, True)
+    row = {"op": f"{w.op}_scan", "B": w.B, "T": w.T, "D": w.D, "io_dtype": w.dtype,
+           "us_per_launch": round(per * 1e6, 2), "gbs": round(gbs, 1),
+           "gelem_per_s": round(w.n_elems / per / 1e9, 2), "roofline_frac": round(gbs / peak, 4),
+           "bytes_per_launch": bytes_,
+           "tile": f"{plan['tile_rows']}x{plan['tile_channels']}", "n_tiles": plan["n_tiles"]}
+    if bytes_ < 64 << 20:
+        # fits in L2 and is over in microseconds: the host's call overhead shows in
+        # the per-call events, so also time the launches replayed from a CUDA graph
+        stream = torch.cuda.Stream(device)
+        stream.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(stream):
+            fn()
+            stream.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                for _ in range(steps):
+                    fn()
+            graph.replay()
+            stream.synchronize()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            graph.replay()
+            t1.record(stream)
+            stream.synchronize()
+        g_per = t0.elapsed_time(t1) / 1e3 / steps
+        row["us_per_launch_graph"] = round(g_per * 1e6, 2)
+        row["note"] = "fits in L2 (inputs stay cached between launches): latency, not bandwidth"
+        del graph
     del p, q, init, out, ws
-    return {"op": f"{w.op}_scan", "B": w.B, "T": w.T, "D": w.D, "io_dtype": w.dtype,
+    return row
+
+
+def measure_backward_row(w, device, steps=10, warmup=3):
+    """Gradient of one scan (dL/d out given): reads the two inputs, the forward
+    output and the upstream gradient, writes the two input gradients (and the
+    initial state's): 6 (B, T, D) tensors per launch."""
+    import scan_gated_rnns_b200 as sgr
+    p, q, init = generate(w, device=device)
+    fwd = (sgr.mingru_scan if w.op == "mingru" else sgr.minmax_scan)(p, q, init)
+    g = torch.Generator(device=device).manual_seed(w.seed + 17)
+    gy = torch.randn(p.shape, device=device, generator=g).to(p.dtype)
+    op = 0 if w.op == "mingru" else 1
+    dt = 0 if w.dtype == "f32" else 1
+    ws = sgr.Workspace(sgr._abi.lib().sgr_backward_workspace_size(op, w.B, w.T, w.D, dt), device)
+    bwd = sgr.mingru_scan_backward if w.op == "mingru" else sgr.minmax_scan_backward
+    fn = lambda: bwd(p, q, init, fwd, gy, init is not None, workspace=ws)  # noqa: E731
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    total, per = timed_launches(fn, steps, torch.cuda.current_stream(device))
+    bytes_ = 6 * w.n_elems * w.elem_bytes + (2 * w.B * w.D * w.elem_bytes if init is not None else 0)
+    peak, _ = hbm_peak()
+    gbs = bytes_ / per / 1e9
+    del p, q, init, fwd, gy, ws
+    return {"op": f"{w.op}_scan_backward", "B": w.B, "T": w.T, "D": w.D, "io_dtype": w.dtype,
             "us_per_launch": round(per * 1e6, 2), "gbs": round(gbs, 1),
             "gelem_per_s": round(w.n_elems / per / 1e9, 2), "roofline_frac": round(gbs / peak, 4),
-            "bytes_per_launch": bytes_,
-            "tile": f"{plan['tile_rows']}x{plan['tile_channels']}", "n_tiles": plan["n_tiles"]}
+            "bytes_per_launch": bytes_, "kernel": "sgr::scan_backward_kernel"}
 
 
 def measure_step_row(device, B=8, D=1024, calls=200, warmup=10):
@@ -432,6 +484,10 @@ def run_b200(args):
                 rows[name] = measure_row(WORKLOADS[name], device)
                 torch.cuda.empty_cache()
         rows["mingru_step_b8_d1024_f32"] = measure_step_row(device)
+        for name in ("mingru_b8_t4096_d1024_f32_h0", "minmax_b4_t8192_d768_f32",
+                     "mingru_b16_t2048_d4096_bf16_h0"):
+            rows[name.replace("_b", "_backward_b", 1)] = measure_backward_row(WORKLOADS[name], device)
+            torch.cuda.empty_cache()
         line["rows"] = rows
     if world > 1:
         import torch.distributed as dist

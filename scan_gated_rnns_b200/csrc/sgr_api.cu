@@ -134,6 +134,14 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
     p.vec = aligned && (D % vw == 0);
     const int ok = g_override_kind.load();
     p.kind = (p.vec && ok != KIND_TILE && !force_tile) ? KIND_PIPELINED : KIND_TILE;
+    if (p.kind == KIND_PIPELINED && ok == KIND_AUTO) {
+        // under two tiles per persistent block: little to pipeline, and
+        // one plain launch per tile starts sooner (no tensor maps, no
+        // cooperative launch)
+        const int64_t tc = p.esz == 4 ? 32 : 64, tr = 112;
+        const int64_t tiles = B * ((D + tc - 1) / tc) * ((T + tr - 1) / tr);
+        if (tiles < 4 * kAssumedSMs) p.kind = KIND_TILE;
+    }
     const int orr = g_override_r.load();
     if (p.kind == KIND_PIPELINED) {
         // 4 channels per lane (16-byte fp32 / 8-byte bf16 vectors)
