@@ -22,6 +22,10 @@ Functions (all inputs are widened exactly to float64 first):
 ``minmax(r, s, x0=None)``
     MinMax neuron x_{t+1} = max(min(r_t, x_t), s_t); page "MinMax Recurrent
     Neural Cascades" (The model, item 3).
+``mingru_decay(k, hx, h0, dt, lam, log1p_delta=False)``
+    minGRU with time decay: the state is gated by gamma_t = exp(-lam_d u_bt)
+    (u = dt or log1p(dt); lam u > 1e4 wipes it) at each token boundary; page
+    "Your first delta model", Step 5.  ``mingru_decay_backward`` adds dlam.
 ``mingru_backward(k, hx, h0, gy)`` / ``minmax_backward(r, s, x0, gy)``
     gradients of a loss with dL/d out = gy with respect to both inputs and the
     initial state, by the chain rule through the sequential loop (forward
@@ -74,6 +78,11 @@ def _open(path: str):
         fn = getattr(lib, name)
         fn.restype = ctypes.c_int
         fn.argtypes = [dp, dp, dp, i64, dp, dp, dp, dp, i64, i64, i64]
+    lib.oracle_mingru_decay.restype = ctypes.c_int
+    lib.oracle_mingru_decay.argtypes = [dp, dp, dp, i64, dp, i64, dp, ctypes.c_int, dp, i64, i64, i64]
+    lib.oracle_mingru_decay_backward.restype = ctypes.c_int
+    lib.oracle_mingru_decay_backward.argtypes = [dp, dp, dp, i64, dp, i64, dp, ctypes.c_int, dp, dp, dp,
+                                                 dp, dp, i64, i64, i64]
     return lib
 
 
@@ -204,3 +213,39 @@ def mingru_backward(k, hx, h0, gy, threads: int = 1):
 def minmax_backward(r, s, x0, gy, threads: int = 1):
     """(dr, ds, dx0) of a loss with dL/d out = gy (fp64; ties share evenly)."""
     return _run_backward("oracle_minmax_backward", r, s, x0, gy, threads)
+
+
+def _decay_args(dt, lam, B, T, D):
+    dt = _as_f64(dt).reshape(B, T)
+    lam = _as_f64(lam).reshape(D)
+    return dt, lam
+
+
+def mingru_decay(k, hx, h0, dt, lam, log1p_delta: bool = False) -> np.ndarray:
+    """fp64 minGRU with time decay; dt (B, T) gaps, lam (D,) rates."""
+    k, hx = _as_f64(k), _as_f64(hx)
+    B, T, D = k.shape
+    dt, lam = _decay_args(dt, lam, B, T, D)
+    init = _as_f64(h0).reshape(B, D) if h0 is not None else None
+    h = np.empty_like(k)
+    rc = _load().oracle_mingru_decay(_ptr(k), _ptr(hx), _ptr(init) if init is not None else None, D,
+                                     _ptr(dt), T, _ptr(lam), int(log1p_delta), _ptr(h), B, T, D)
+    if rc != 0:
+        raise RuntimeError(f"oracle_mingru_decay returned {rc}")
+    return h
+
+
+def mingru_decay_backward(k, hx, h0, dt, lam, gy, log1p_delta: bool = False):
+    """(dk, dhx, dh0, dlam) of a loss with dL/dh = gy through mingru_decay."""
+    k, hx, gy = _as_f64(k), _as_f64(hx), _as_f64(gy)
+    B, T, D = k.shape
+    dt, lam = _decay_args(dt, lam, B, T, D)
+    init = _as_f64(h0).reshape(B, D) if h0 is not None else None
+    dk, dhx = np.empty_like(k), np.empty_like(k)
+    dh0, dlam = np.empty((B, D)), np.empty(D)
+    rc = _load().oracle_mingru_decay_backward(
+        _ptr(k), _ptr(hx), _ptr(init) if init is not None else None, D, _ptr(dt), T, _ptr(lam),
+        int(log1p_delta), _ptr(gy), _ptr(dk), _ptr(dhx), _ptr(dh0), _ptr(dlam), B, T, D)
+    if rc != 0:
+        raise RuntimeError(f"oracle_mingru_decay_backward returned {rc}")
+    return dk, dhx, dh0, dlam

@@ -295,3 +295,111 @@ int oracle_minmax_backward(const double *r, const double *s,
     free(x);
     return 0;
 }
+
+/* ------------------------------------------------------ minGRU, time decay */
+
+/*
+ * Time decay (page "Your first delta model", Step 5: the decay contract every
+ * mixer accepts): the carried state is gated once per token, at the token
+ * boundary, before that token's own write lands undecayed,
+ *     h <- gamma_t h,   gamma_t = exp(-lambda_d * u_{b,t}),
+ * with u the gap preceding the token (delta_t), or log1p(delta_t) when gaps
+ * are compressed (log1p_delta).  delta_t = 0 gives gamma = exp(0) = 1, no
+ * decay.  A gap with lambda * u > 1e4 wipes the state completely (the page's
+ * clamp; gamma = 0 exactly, with zero derivative).  For the minGRU's vector
+ * state this reads
+ *     h_t = (1 - z_t) gamma_t h_{t-1} + z_t g(hx_t).
+ * delta_t is (B, T) with batch stride dt_bs; lambda is (D,), >= 0.
+ */
+static double decay_gate(double lam, double gap, int log1p_delta)
+{
+    double u = log1p_delta ? log1p(gap) : gap;
+    double x = lam * u;
+    return (x > 1e4) ? 0.0 : exp(-x);
+}
+
+/* d gamma / d lambda = -u gamma (0 where the clamp holds gamma at 0) */
+static double decay_gate_dlam(double lam, double gap, int log1p_delta)
+{
+    double u = log1p_delta ? log1p(gap) : gap;
+    double x = lam * u;
+    return (x > 1e4) ? 0.0 : -u * exp(-x);
+}
+
+int oracle_mingru_decay(const double *k, const double *hx,
+                        const double *h0, int64_t h0_bs,
+                        const double *dt, int64_t dt_bs, const double *lam, int log1p_delta,
+                        double *h, int64_t B, int64_t T, int64_t D)
+{
+    if (B < 0 || T < 0 || D < 0) return 1;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t t = 0; t < T; ++t) {
+            for (int64_t d = 0; d < D; ++d) {
+                int64_t i = (b * T + t) * D + d;
+                double prev;
+                if (t > 0) {
+                    prev = h[i - D];
+                } else {
+                    prev = h0 ? h0[b * h0_bs + d] : 0.0;
+                }
+                double gamma = decay_gate(lam[d], dt[b * dt_bs + t], log1p_delta);
+                h[i] = sigmoid(-k[i]) * (gamma * prev) + sigmoid(k[i]) * g_act(hx[i]);
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Gradients of the decayed recurrence for dL/dh = gy, as oracle_mingru_backward
+ * plus the decay:
+ *   dh_t/dk_t      = z (1 - z) (g - gamma h_{t-1})
+ *   dh_t/dh_{t-1}  = (1 - z) gamma
+ *   dL/dlambda_d   = sum over b, t of delta_t (1 - z_t) h_{t-1} dgamma_t/dlambda
+ * dlam (D,) is overwritten with the sum over the whole batch; dh0, dlam may be NULL.
+ */
+int oracle_mingru_decay_backward(const double *k, const double *hx,
+                                 const double *h0, int64_t h0_bs,
+                                 const double *dt, int64_t dt_bs, const double *lam, int log1p_delta,
+                                 const double *gy, double *dk, double *dhx, double *dh0, double *dlam,
+                                 int64_t B, int64_t T, int64_t D)
+{
+    if (B < 0 || T < 0 || D < 0) return 1;
+    double *h = malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    if (!h) return 2;
+    if (dlam) {
+        for (int64_t d = 0; d < D; ++d) dlam[d] = 0.0;
+    }
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t d = 0; d < D; ++d) {
+            double init = h0 ? h0[b * h0_bs + d] : 0.0;
+            double prev = init;
+            for (int64_t t = 0; t < T; ++t) {
+                int64_t i = (b * T + t) * D + d;
+                double gamma = decay_gate(lam[d], dt[b * dt_bs + t], log1p_delta);
+                prev = sigmoid(-k[i]) * (gamma * prev) + sigmoid(k[i]) * g_act(hx[i]);
+                h[t] = prev;
+            }
+            double back = 0.0;
+            for (int64_t t = T - 1; t >= 0; --t) {
+                int64_t i = (b * T + t) * D + d;
+                double delta = gy[i] + back;
+                double hprev = (t > 0) ? h[t - 1] : init;
+                double gap = dt[b * dt_bs + t];
+                double gamma = decay_gate(lam[d], gap, log1p_delta);
+                double z = sigmoid(k[i]);
+                double one_minus_z = sigmoid(-k[i]);
+                double x = hx[i];
+                double g = g_act(x);
+                double gprime = (x >= 0.0) ? 1.0 : sigmoid(x) * sigmoid(-x);
+                dk[i] = delta * z * one_minus_z * (g - gamma * hprev);
+                dhx[i] = delta * z * gprime;
+                if (dlam) dlam[d] += delta * one_minus_z * hprev * decay_gate_dlam(lam[d], gap, log1p_delta);
+                back = delta * one_minus_z * gamma;
+            }
+            if (dh0) dh0[b * D + d] = back;
+        }
+    }
+    free(h);
+    return 0;
+}

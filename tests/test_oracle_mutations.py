@@ -15,6 +15,7 @@ import pytest
 
 import oracle
 import test_oracle_backward_pins as bpins
+import test_oracle_decay_pins as dpins
 import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(os.path.abspath(oracle.__file__)), "oracle.c")
@@ -65,6 +66,17 @@ MUTANTS = {
     "bwd_minmax_tie_to_s": ("double dout_dm = (m > s[i]) ? 1.0 : ((m == s[i]) ? 0.5 : 0.0);",
                             "double dout_dm = (m > s[i]) ? 1.0 : 0.0;"),
     "bwd_minmax_state_path": ("lam = delta * dout_dm * dm_dx;", "lam = delta * dm_dx;"),
+    # time decay
+    "decay_exponent_sign": ("return (x > 1e4) ? 0.0 : exp(-x);", "return (x > 1e4) ? 0.0 : exp(x);"),
+    "decay_gates_the_write": ("h[i] = sigmoid(-k[i]) * (gamma * prev) + sigmoid(k[i]) * g_act(hx[i]);",
+                              "h[i] = sigmoid(-k[i]) * prev + gamma * sigmoid(k[i]) * g_act(hx[i]);"),
+    "decay_clamp_keeps_state": ("return (x > 1e4) ? 0.0 : exp(-x);", "return (x > 1e4) ? 1.0 : exp(-x);"),
+    "decay_log1p_ignored": ("    double u = log1p_delta ? log1p(gap) : gap;\n    double x = lam * u;\n    return (x > 1e4)",
+                            "    double u = gap; (void)log1p_delta;\n    double x = lam * u;\n    return (x > 1e4)"),
+    "decay_bwd_dk_without_gamma": ("dk[i] = delta * z * one_minus_z * (g - gamma * hprev);",
+                                   "dk[i] = delta * z * one_minus_z * (g - hprev);"),
+    "decay_bwd_dlam_sign": ("return (x > 1e4) ? 0.0 : -u * exp(-x);", "return (x > 1e4) ? 0.0 : u * exp(-x);"),
+    "decay_bwd_state_without_gamma": ("back = delta * one_minus_z * gamma;", "back = delta * one_minus_z;"),
     "bwd_minmax_r_s_swapped": ("dr[i] = delta * dout_dm * dm_dr;\n                ds[i] = delta * dout_ds;",
                                "ds[i] = delta * dout_dm * dm_dr;\n                dr[i] = delta * dout_ds;"),
 }
@@ -101,6 +113,16 @@ def _pin_checks():
     for seed in range(2):
         out.append(lambda sd=seed: bpins.test_minmax_backward_matches_autograd_with_ties(sd))
         out.append(lambda sd=seed: bpins.test_minmax_backward_conserves_gradient(sd))
+    # time-decay pins
+    for wh in (False, True):
+        out.append(lambda a=wh: dpins.test_zero_gap_and_zero_rate_are_the_plain_recurrence(a))
+    out += [dpins.test_wiping_gap_restarts_the_sequence, dpins.test_log1p_delta_compresses_the_gaps,
+            dpins.test_decay_backward_lambda_finite_differences,
+            dpins.test_decay_backward_without_decay_is_the_plain_gradient]
+    for args in [(0.3, 0.7, 0.5, 0.4, 0.8), (-1.2, -0.9, 2.0, 0.1, 0.2)]:
+        out.append(lambda a=args: dpins.test_constant_inputs_closed_form(*a))
+    for flag in (False, True):
+        out.append(lambda f=flag: dpins.test_decay_backward_matches_autograd(f))
     return out
 
 
