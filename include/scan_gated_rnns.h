@@ -167,6 +167,56 @@ SGR_API sgr_status_t mingru_scan_noalloc(const void *k, const void *hx,
                                          void *h, int64_t B, int64_t T, int64_t D,
                                          sgr_dtype_t dtype, cudaStream_t stream);
 
+/* ----------------------------------------------------------- time decay */
+
+/*
+ * mingru_scan_decay -- mingru_scan with time decay (page "Your first delta
+ * model", Step 5: the decay contract the mixers accept -- the carried state
+ * is gated once per token at the token boundary, before that token's own
+ * write lands undecayed).  For the minGRU's vector state:
+ *     h_t = (1 - z_t) gamma_t h_{t-1} + z_t g(hx_t),
+ *     gamma_t = exp(-lambda_d u_{b,t}),  u = delta_t, or log1p(delta_t)
+ *               when log1p_delta != 0 (compresses very large gaps);
+ * delta_t = 0 gives gamma = 1 (no decay); lambda u > 1e4 wipes the state
+ * (gamma = 0 exactly).
+ *   delta_t : fp32 DEVICE array (B, T), the gap preceding each token, >= 0
+ *             and finite; batch stride delta_t_batch_stride (elements, >= T
+ *             when B > 1)
+ *   lambda  : fp32 DEVICE array (D,), decay rates >= 0 (fixed or learnable)
+ * Other arguments, workspace and errors as mingru_scan (the same workspace
+ * size).  Arithmetic fp32; the gate uses the MUFU exp2 like the activations.
+ */
+SGR_API sgr_status_t mingru_scan_decay(const void *k, const void *hx,
+                                       const void *h0, int64_t h0_batch_stride,
+                                       const float *delta_t, int64_t delta_t_batch_stride,
+                                       const float *lambda, int log1p_delta,
+                                       void *h, int64_t B, int64_t T, int64_t D,
+                                       sgr_dtype_t dtype, void *workspace, size_t ws_bytes,
+                                       cudaStream_t stream);
+
+/*
+ * mingru_scan_decay_backward -- gradients through mingru_scan_decay for
+ * dh = dL/dh: dk, dhx, dh0 as mingru_scan_backward (with the gate:
+ * dk_t = delta_t z (1 - z) (g - gamma_t h_{t-1}), state gradient
+ * (1 - z) gamma), and dlambda (fp32 DEVICE (D,), or NULL) = the sum over
+ * b, t of delta_t (1 - z_t) h_{t-1} dgamma_t/dlambda_d with
+ * dgamma/dlambda = -u gamma (0 where the 1e4 clamp wipes).  dlambda is
+ * overwritten; its sums use atomic adds, so their rounding order varies from
+ * run to run.  No gradient with respect to delta_t (the gaps are data).
+ * Workspace: sgr_backward_workspace_size(SGR_OP_MINGRU, ...).
+ */
+SGR_API sgr_status_t mingru_scan_decay_backward(const void *k, const void *hx,
+                                                const void *h0, int64_t h0_batch_stride,
+                                                const float *delta_t, int64_t delta_t_batch_stride,
+                                                const float *lambda, int log1p_delta,
+                                                const void *h, const void *dh,
+                                                void *dk, void *dhx,
+                                                void *dh0, int64_t dh0_batch_stride,
+                                                float *dlambda,
+                                                int64_t B, int64_t T, int64_t D,
+                                                sgr_dtype_t dtype, void *workspace,
+                                                size_t ws_bytes, cudaStream_t stream);
+
 /* ------------------------------------------------------------ gradients */
 
 /*

@@ -73,6 +73,11 @@ SIGNATURES.update({
     "minmax_scan_backward": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _i64,
                                     _i64, _i64, _i64, _int, _vp, _sz, _vp]),
     "sgr_backward_workspace_size": (_sz, [_int, _i64, _i64, _i64, _int]),
+    "mingru_scan_decay": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _vp, _int, _vp, _i64, _i64, _i64,
+                                 _int, _vp, _sz, _vp]),
+    "mingru_scan_decay_backward": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _vp, _int, _vp, _vp, _vp,
+                                          _vp, _vp, _i64, _vp, _i64, _i64, _i64, _int, _vp, _sz,
+                                          _vp]),
     "mingru_scan_host": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _i64, _i64, _int, _int, _vp, _sz, _vp]),
     "minmax_scan_host": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _i64, _i64, _int, _int, _vp, _sz, _vp]),
 })

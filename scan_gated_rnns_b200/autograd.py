@@ -56,6 +56,30 @@ class MinMaxScan(torch.autograd.Function):
         return dr, ds, (_init_grad(dx0, x0) if dx0 is not None else None)
 
 
+class MinGRUDecayScan(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, k, hx, h0, delta_t, lam, log1p_delta):
+        h = ops.mingru_scan_decay(k, hx, h0, delta_t, lam, log1p_delta)
+        ctx.save_for_backward(k, hx, h0, delta_t, lam, h)
+        ctx.log1p_delta = log1p_delta
+        return h
+
+    @staticmethod
+    def backward(ctx, dh):
+        k, hx, h0, delta_t, lam, h = ctx.saved_tensors
+        dk, dhx, dh0, dlam = ops.mingru_scan_decay_backward(
+            k, hx, h0, delta_t, lam, h, dh.contiguous(), ctx.log1p_delta,
+            want_dh0=h0 is not None and ctx.needs_input_grad[2], want_dlam=ctx.needs_input_grad[4])
+        return (dk, dhx, (_init_grad(dh0, h0) if dh0 is not None else None), None, dlam, None)
+
+
+def mingru_scan_decay_fn(k: torch.Tensor, hx: torch.Tensor, h0: Optional[torch.Tensor],
+                         delta_t: torch.Tensor, lam: torch.Tensor,
+                         log1p_delta: bool = False) -> torch.Tensor:
+    """mingru_scan_decay with gradients for k, hx, h0 and lam (not delta_t)."""
+    return MinGRUDecayScan.apply(k, hx, h0, delta_t, lam, log1p_delta)
+
+
 def mingru_scan_fn(k: torch.Tensor, hx: torch.Tensor, h0: Optional[torch.Tensor] = None) -> torch.Tensor:
     """mingru_scan with gradients for k, hx and h0."""
     return MinGRUScan.apply(k, hx, h0)

@@ -31,10 +31,17 @@
 namespace sgr {
 
 struct MinGRUBwd {
+    static constexpr bool kDecay = false;
     // (k, hx, state before the step) -> (A, cP, cQ); the same exp2 / shared
     // reciprocal evaluation of sigmoid(+-|x|) as the forward activations
     static __device__ __forceinline__ void coeffs(float k, float hx, float h, float &A, float &cP,
                                                   float &cQ) {
+        coeffs_gated(k, hx, h, 1.f, A, cP, cQ);
+    }
+    // with the state entering the step gated by gamma (time decay):
+    // out = (1 - z) gamma h + z g, so A = (1 - z) gamma and cP = z (1 - z) (g - gamma h)
+    static __device__ __forceinline__ void coeffs_gated(float k, float hx, float h, float gamma,
+                                                        float &A, float &cP, float &cQ) {
         const float ek = fast_exp2(fabsf(k) * kNegLog2e);
         const float eh = fast_exp2(fabsf(hx) * kNegLog2e);
         const float dk = 1.f + ek, dh = 1.f + eh;
@@ -45,17 +52,22 @@ struct MinGRUBwd {
         const float sh = eh * rh;           // sigmoid(-|hx|)
         const bool kpos = k >= 0.f;
         const float z = kpos ? rk : sk;
-        A = kpos ? sk : rk;
+        A = (kpos ? sk : rk) * gamma;
         const bool hpos = hx >= 0.f;
         const float g = hpos ? hx + 0.5f : sh;
         const float gp = hpos ? 1.f : sh * rh;
-        cP = (sk * rk) * (g - h);
+        cP = (sk * rk) * (g - gamma * h);
         cQ = z * gp;
     }
     static __device__ __forceinline__ float default_state() { return 0.f; }
 };
 
+struct MinGRUDecayBwd : MinGRUBwd {
+    static constexpr bool kDecay = true;
+};
+
 struct MinMaxBwd {
+    static constexpr bool kDecay = false;
     static __device__ __forceinline__ void coeffs(float r, float s, float x, float &A, float &cP,
                                                   float &cQ) {
         const float m = fminf(r, x);
@@ -78,6 +90,7 @@ struct BwdParams {
     void *out1;           // d in1 (B, T, D)
     void *dinit;          // dL/d initial state (B, D) rows or null
     int64_t dinit_bs;
+    float *dlam;          // time decay: dL/d lambda (D,), accumulated (zeroed by the host), or null
 };
 
 // One block per tile, W data warps + 1 carry warp, the tile kernel's lane
@@ -117,7 +130,14 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_backward_kernel(const
         const IO *gy = static_cast<const IO *>(bp.gy);
 
         // rows r = 0..R-1 at time top - r: A, the upstream gradient, cP, cQ
+        // (time decay: and E = (1 - z) h_{t-1} dgamma/dlambda, for dL/dlambda)
         float A[R][V], G[R][V], P[R][V], Q[R][V];
+        float E[BOp::kDecay ? R : 1][V];
+        float lam2[V];
+        if constexpr (BOp::kDecay) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) lam2[v] = decay_lam2(p, d0 + v);
+        }
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const int64_t t = top - r;
@@ -146,10 +166,22 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_backward_kernel(const
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const bool ok = dvalid && (top - r) < p.T;
+            float u = 0.f;
+            if constexpr (BOp::kDecay) {
+                if ((top - r) < p.T) u = decay_u(p, tc.b, top - r);
+            }
 #pragma unroll
             for (int v = 0; v < V; ++v) {
                 float a, cp, cq;
-                BOp::coeffs(A[r][v], P[r][v], Q[r][v], a, cp, cq);
+                if constexpr (BOp::kDecay) {
+                    const float gamma = decay_gamma(lam2[v], u);
+                    BOp::coeffs_gated(A[r][v], P[r][v], Q[r][v], gamma, a, cp, cq);
+                    // dL/dlambda gains delta (1 - z) h_{t-1} dgamma/dlambda
+                    //   = delta A h_{t-1} (-u)   (dgamma/dlambda = -u gamma; 0 where gamma is 0)
+                    E[r][v] = -u * a * Q[r][v];
+                } else {
+                    BOp::coeffs(A[r][v], P[r][v], Q[r][v], a, cp, cq);
+                }
                 a = ok ? a : 1.f;                 // rows past T: identity pair, gy = 0
                 A[r][v] = a;
                 P[r][v] = cp;
@@ -182,9 +214,12 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_backward_kernel(const
         named_barrier_sync(1, NT);   // summaries are in shared memory
         named_barrier_sync(2, NT);   // the carry warp has written the incoming gradients
 
-        float lam[V];
+        float lam[V], dl[V];
 #pragma unroll
-        for (int v = 0; v < V; ++v) lam[v] = Op::apply(excl[v], s_tot[warp][g * V + v].x);
+        for (int v = 0; v < V; ++v) {
+            lam[v] = Op::apply(excl[v], s_tot[warp][g * V + v].x);
+            dl[v] = 0.f;
+        }
         IO *out0 = static_cast<IO *>(p.out);
         IO *out1 = static_cast<IO *>(bp.out1);
 #pragma unroll
@@ -195,12 +230,27 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_backward_kernel(const
                 const float delta = G[r][v] + lam[v];
                 y0[v] = delta * P[r][v];
                 y1[v] = delta * Q[r][v];
+                if constexpr (BOp::kDecay) dl[v] = fmaf(delta, E[r][v], dl[v]);
                 lam[v] = A[r][v] * delta;
             }
             const int64_t t = top - r;
             if (dvalid && t < p.T) {
                 Access<IO, V>::store(out0 + base + t * p.D, y0);
                 Access<IO, V>::store(out1 + base + t * p.D, y1);
+            }
+        }
+        if constexpr (BOp::kDecay) {
+            // dL/dlambda: sum the warp's row groups, one atomic add per channel and warp
+            if (bp.dlam) {
+#pragma unroll
+                for (int off = CG; off < 32; off <<= 1) {
+#pragma unroll
+                    for (int v = 0; v < V; ++v) dl[v] += __shfl_xor_sync(0xffffffffu, dl[v], off);
+                }
+                if (j == 0 && dvalid) {
+#pragma unroll
+                    for (int v = 0; v < V; ++v) atomicAdd(bp.dlam + d0 + v, dl[v]);
+                }
             }
         }
         // the thread holding time row 0 ends with dL/d (initial state)

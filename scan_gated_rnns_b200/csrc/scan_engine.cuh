@@ -68,6 +68,7 @@ __device__ __forceinline__ float fast_rcp(float x) {
 // ------------------------------------------------------------- operators
 
 struct MinGRUOp {
+    static constexpr bool kDecay = false;
     // pair (A, B): state -> A * state + B
     static __device__ __forceinline__ float2 identity() { return make_float2(1.f, 0.f); }
     // (first, then) -> composition
@@ -113,6 +114,7 @@ struct MinGRUOp {
 };
 
 struct MinMaxOp {
+    static constexpr bool kDecay = false;
     // pair (U, L): state -> max(min(state, U), L)
     static __device__ __forceinline__ float2 identity() { return make_float2(INFINITY, -INFINITY); }
     static __device__ __forceinline__ float2 combine(float2 p, float2 q) {
@@ -132,6 +134,23 @@ struct MinMaxOp {
         return make_float2(fmaxf(fminf(x.x, u.x), l.x), fmaxf(fminf(x.y, u.y), l.y));
     }
 };
+
+// minGRU with time decay (page "Your first delta model", Step 5: every mixer
+// takes the decay contract; the carried state is gated once per token at the
+// token boundary, before the token's own write): the state entering token t
+// is gamma_t h_{t-1}, gamma_t = exp(-lambda_d u_bt), u the gap before the
+// token (or log1p of it), so the per-step pair is (a_t gamma_t, b_t).  A gap
+// with lambda u > 1e4 wipes the state (gamma = 0 exactly).
+struct MinGRUDecayOp : MinGRUOp {
+    static constexpr bool kDecay = true;
+};
+
+// gamma = exp(-lambda u) = 2^(lam2 u) with lam2 = -lambda log2 e (<= 0)
+constexpr float kDecayClampLog2 = -1.0e4f * 1.4426950408889634f;
+__device__ __forceinline__ float decay_gamma(float lam2, float u) {
+    const float x = lam2 * u;
+    return x < kDecayClampLog2 ? 0.f : fast_exp2(x);
+}
 
 // ------------------------------------------------------------ memory access
 
@@ -287,7 +306,21 @@ struct ScanParams {
     uint32_t epoch;
     uint32_t spin_limit;  // polls before a chunk gives up waiting
     int64_t drop_tile;    // testing: this tile does not publish (-1: none)
+    // time decay (MinGRUDecayOp only): gaps (B, T) with batch stride, rates (D,)
+    const float *decay_dt;
+    int64_t decay_dt_bs;
+    const float *decay_lam;
+    int decay_log1p;      // u = log1p(gap) instead of the gap
 };
+
+// gap before token t of batch row b, as it enters the gate
+__device__ __forceinline__ float decay_u(const ScanParams &p, int64_t b, int64_t t) {
+    const float g = p.decay_dt[b * p.decay_dt_bs + t];
+    return p.decay_log1p ? log1pf(g) : g;
+}
+__device__ __forceinline__ float decay_lam2(const ScanParams &p, int64_t d) {
+    return d < p.D ? -p.decay_lam[d] * 1.4426950408889634f : 0.f;
+}
 
 // Position of a tile: chunk c along T, chain = b * n_dt + dt.  All < 2^31.
 struct TileCoord {
@@ -586,12 +619,22 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const Sca
         float2 incl[V];
 #pragma unroll
         for (int v = 0; v < V; ++v) incl[v] = Op::identity();
+        float lam2[V];
+        if constexpr (Op::kDecay) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) lam2[v] = decay_lam2(p, d0 + v);
+        }
 #pragma unroll
         for (int r = 0; r < R; ++r) {
+            float u = 0.f;        // rows past T: gamma = 1 keeps the padding pair the identity
+            if constexpr (Op::kDecay) {
+                if (row0 + r < p.T) u = decay_u(p, b, row0 + r);
+            }
 #pragma unroll
             for (int v = 0; v < V; ++v) {
                 float e0, e1;
                 Op::element(x0[r][v], x1[r][v], e0, e1);
+                if constexpr (Op::kDecay) e0 *= decay_gamma(lam2[v], u);
                 x0[r][v] = e0;
                 x1[r][v] = e1;
                 incl[v] = Op::combine(incl[v], make_float2(e0, e1));
@@ -841,6 +884,11 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                 IA[i] = make_float2(Op::identity().x, Op::identity().x);
                 IB[i] = make_float2(Op::identity().y, Op::identity().y);
             }
+            float lam2[V];
+            if constexpr (Op::kDecay) {
+#pragma unroll
+                for (int v = 0; v < V; ++v) lam2[v] = decay_lam2(p, d0 + v);
+            }
             auto rows = [&](auto fullc) {
                 constexpr bool FULL = decltype(fullc)::value;
 #pragma unroll
@@ -848,6 +896,10 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                     float x0[V], x1[V];
                     unpack(*reinterpret_cast<const Vec *>(t0 + r * TC), x0);
                     unpack(*reinterpret_cast<const Vec *>(t1 + r * TC), x1);
+                    float u = 0.f;
+                    if constexpr (Op::kDecay) {
+                        if (row0[SB] + r < p.T) u = decay_u(p, tc.b, row0[SB] + r);
+                    }
                     if (!FULL) {
                         const bool ok = dvalid[SB] && (row0[SB] + r < p.T);
 #pragma unroll
@@ -861,6 +913,10 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                         float a0, b0, a1, b1;
                         Op::element(x0[2 * i], x1[2 * i], a0, b0);
                         Op::element(x0[2 * i + 1], x1[2 * i + 1], a1, b1);
+                        if constexpr (Op::kDecay) {
+                            a0 *= decay_gamma(lam2[2 * i], u);
+                            a1 *= decay_gamma(lam2[2 * i + 1], u);
+                        }
                         PA[SB][r][i] = make_float2(a0, a1);
                         PB[SB][r][i] = make_float2(b0, b1);
                         Op::fold2(IA[i], IB[i], PA[SB][r][i], PB[SB][r][i]);

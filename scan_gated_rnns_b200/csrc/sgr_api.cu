@@ -347,14 +347,43 @@ cudaError_t dispatch(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
     return dispatch_tile_r<Op, IO, VW, 8>(pl, sp, s);
 }
 
+// time-decay arguments of the minGRU scans (null: no decay)
+struct DecayArgs {
+    const float *dt = nullptr;
+    int64_t dt_bs = 0;
+    const float *lam = nullptr;
+    int log1p = 0;
+};
+
+sgr_status_t check_decay(const DecayArgs *dec, int64_t B, int64_t T, int64_t D) {
+    if (!dec) return SGR_OK;
+    if (!dec->dt || !dec->lam || dec->dt_bs < 0) return SGR_ERR_INVALID_ARG;
+    if (B > 1 && dec->dt_bs < T) return SGR_ERR_INVALID_ARG;   // rows of gaps would overlap
+    int64_t tmp = 0;
+    if (!mul_ok(B - 1, dec->dt_bs, &tmp) || !mul_ok(tmp + T, 4, &tmp)) return SGR_ERR_UNSUPPORTED;
+    (void)D;
+    return SGR_OK;
+}
+
+void set_decay(ScanParams &sp, const DecayArgs *dec) {
+    if (!dec) return;
+    sp.decay_dt = dec->dt;
+    sp.decay_dt_bs = dec->dt_bs;
+    sp.decay_lam = dec->lam;
+    sp.decay_log1p = dec->log1p ? 1 : 0;
+}
+
 sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void *init,
                       int64_t init_bs, void *out, int64_t B, int64_t T, int64_t D,
-                      sgr_dtype_t dtype, void *ws, size_t ws_bytes, cudaStream_t stream) {
+                      sgr_dtype_t dtype, void *ws, size_t ws_bytes, cudaStream_t stream,
+                      const DecayArgs *dec = nullptr) {
     if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
     if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return SGR_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || D < 0 || init_bs < 0) return SGR_ERR_INVALID_ARG;
     if (B == 0 || T == 0 || D == 0) return SGR_OK;
     if (!in0 || !in1 || !out) return SGR_ERR_INVALID_ARG;
+    const sgr_status_t dst = check_decay(dec, B, T, D);
+    if (dst != SGR_OK) return dst;
     const int esz = dtype == SGR_BF16 ? 2 : 4;
     int64_t n = 0, nbytes = 0;
     if (!mul_ok(B, T, &n) || !mul_ok(n, D, &n) || !mul_ok(n, esz, &nbytes)) return SGR_ERR_UNSUPPORTED;
@@ -379,6 +408,7 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
     sp.epoch = 0;
     sp.spin_limit = g_spin_limit.load();
     sp.drop_tile = g_drop_tile.load();
+    set_decay(sp, dec);
     if (pl.n_chunks > 1) {
         if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)) return SGR_ERR_WORKSPACE;
         char *w = static_cast<char *>(ws);
@@ -397,7 +427,10 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
         }
     }
     cudaError_t e;
-    if (op == SGR_OP_MINGRU) {
+    if (op == SGR_OP_MINGRU && dec) {
+        e = dtype == SGR_F32 ? dispatch<MinGRUDecayOp, float>(pl, sp, stream)
+                             : dispatch<MinGRUDecayOp, __nv_bfloat16>(pl, sp, stream);
+    } else if (op == SGR_OP_MINGRU) {
         e = dtype == SGR_F32 ? dispatch<MinGRUOp, float>(pl, sp, stream)
                              : dispatch<MinGRUOp, __nv_bfloat16>(pl, sp, stream);
     } else {
@@ -444,11 +477,17 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
                                int64_t init_bs, const void *fwd, const void *gy, void *out0,
                                void *out1, void *dinit, int64_t dinit_bs, int64_t B, int64_t T,
                                int64_t D, sgr_dtype_t dtype, void *ws, size_t ws_bytes,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, const DecayArgs *dec = nullptr,
+                               float *dlam = nullptr) {
     if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
     if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return SGR_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || D < 0 || init_bs < 0 || dinit_bs < 0) return SGR_ERR_INVALID_ARG;
-    if (B == 0 || D == 0) return SGR_OK;
+    if (B == 0 || D == 0) {
+        // no elements: dL/dlambda is zero
+        if (dec && dlam && D > 0 && cudaMemsetAsync(dlam, 0, size_t(D) * sizeof(float), stream) != cudaSuccess)
+            return SGR_ERR_CUDA;
+        return SGR_OK;
+    }
     if (dinit && B > 1 && dinit_bs < D) return SGR_ERR_INVALID_ARG;   // rows would overlap
     const int esz = dtype == SGR_BF16 ? 2 : 4;
     int64_t n = 0, nbytes = 0, tmp = 0;
@@ -457,7 +496,9 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
         if (!mul_ok(B - 1, bs, &tmp) || !mul_ok(tmp + D, esz, &tmp)) return SGR_ERR_UNSUPPORTED;
     const size_t db = dinit ? rows_span(B, D, dinit_bs, esz) : 0;
     if (T == 0) {
-        // no steps: the gradient reaching the initial state is zero
+        // no steps: the gradients reaching the initial state and lambda are zero
+        if (dec && dlam && cudaMemsetAsync(dlam, 0, size_t(D) * sizeof(float), stream) != cudaSuccess)
+            return SGR_ERR_CUDA;
         if (dinit) {
             if (dinit_bs == D || B == 1) {
                 if (cudaMemsetAsync(dinit, 0, size_t(D) * esz * (B == 1 ? 1 : B), stream) != cudaSuccess)
@@ -470,6 +511,8 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
         return SGR_OK;
     }
     if (!in0 || !in1 || !fwd || !gy || !out0 || !out1) return SGR_ERR_INVALID_ARG;
+    const sgr_status_t dst = check_decay(dec, B, T, D);
+    if (dst != SGR_OK) return dst;
     const size_t tb = size_t(nbytes);
     const size_t ib = init ? rows_span(B, D, init_bs, esz) : 0;
     const void *ins[5] = {in0, in1, fwd, gy, init};
@@ -500,6 +543,10 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
     sp.drop_tile = g_drop_tile.load();
     bp.fwd = fwd; bp.gy = gy; bp.init = init; bp.init_bs = init_bs;
     bp.out1 = out1; bp.dinit = dinit; bp.dinit_bs = dinit_bs;
+    set_decay(sp, dec);
+    bp.dlam = dec ? dlam : nullptr;
+    if (bp.dlam && overlaps(bp.dlam, size_t(D) * sizeof(float), out0, tb)) return SGR_ERR_INVALID_ARG;
+    if (bp.dlam && overlaps(bp.dlam, size_t(D) * sizeof(float), out1, tb)) return SGR_ERR_INVALID_ARG;
     if (pl.n_chunks > 1) {
         if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)) return SGR_ERR_WORKSPACE;
         char *w = static_cast<char *>(ws);
@@ -515,8 +562,14 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
             sp.epoch = next_epoch();
         }
     }
+    // dL/dlambda accumulates over the tiles with atomic adds
+    if (bp.dlam && cudaMemsetAsync(bp.dlam, 0, size_t(D) * sizeof(float), stream) != cudaSuccess)
+        return SGR_ERR_CUDA;
     cudaError_t e;
-    if (op == SGR_OP_MINGRU) {
+    if (op == SGR_OP_MINGRU && dec) {
+        e = dtype == SGR_F32 ? dispatch_bwd<MinGRUDecayBwd, float>(pl, bp, stream)
+                             : dispatch_bwd<MinGRUDecayBwd, __nv_bfloat16>(pl, bp, stream);
+    } else if (op == SGR_OP_MINGRU) {
         e = dtype == SGR_F32 ? dispatch_bwd<MinGRUBwd, float>(pl, bp, stream)
                              : dispatch_bwd<MinGRUBwd, __nv_bfloat16>(pl, bp, stream);
     } else {
@@ -595,6 +648,31 @@ sgr_status_t minmax_scan_backward(const void *r, const void *s, const void *x0,
                                   size_t ws_bytes, cudaStream_t stream) {
     return run_scan_backward(SGR_OP_MINMAX, r, s, x0, x0_batch_stride, x, dx, dr, ds, dx0,
                              dx0_batch_stride, B, T, D, dtype, workspace, ws_bytes, stream);
+}
+
+sgr_status_t mingru_scan_decay(const void *k, const void *hx, const void *h0, int64_t h0_batch_stride,
+                               const float *delta_t, int64_t delta_t_batch_stride, const float *lambda,
+                               int log1p_delta, void *h, int64_t B, int64_t T, int64_t D,
+                               sgr_dtype_t dtype, void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    DecayArgs dec;
+    dec.dt = delta_t; dec.dt_bs = delta_t_batch_stride; dec.lam = lambda; dec.log1p = log1p_delta;
+    return run_scan(SGR_OP_MINGRU, k, hx, h0, h0_batch_stride, h, B, T, D, dtype, workspace,
+                    ws_bytes, stream, &dec);
+}
+
+sgr_status_t mingru_scan_decay_backward(const void *k, const void *hx, const void *h0,
+                                        int64_t h0_batch_stride, const float *delta_t,
+                                        int64_t delta_t_batch_stride, const float *lambda,
+                                        int log1p_delta, const void *h, const void *dh, void *dk,
+                                        void *dhx, void *dh0, int64_t dh0_batch_stride,
+                                        float *dlambda, int64_t B, int64_t T, int64_t D,
+                                        sgr_dtype_t dtype, void *workspace, size_t ws_bytes,
+                                        cudaStream_t stream) {
+    DecayArgs dec;
+    dec.dt = delta_t; dec.dt_bs = delta_t_batch_stride; dec.lam = lambda; dec.log1p = log1p_delta;
+    return run_scan_backward(SGR_OP_MINGRU, k, hx, h0, h0_batch_stride, h, dh, dk, dhx, dh0,
+                             dh0_batch_stride, B, T, D, dtype, workspace, ws_bytes, stream, &dec,
+                             dlambda);
 }
 
 size_t sgr_backward_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype) {

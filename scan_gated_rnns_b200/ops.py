@@ -177,6 +177,80 @@ def minmax_scan_backward(r: torch.Tensor, s: torch.Tensor, x0: Optional[torch.Te
                           workspace)
 
 
+def _decay_operands(fn: str, p: torch.Tensor, delta_t: torch.Tensor, lam: torch.Tensor):
+    B, T, D = p.shape
+    for t, n in ((delta_t, "delta_t"), (lam, "lambda")):
+        _need_cuda(t, f"{fn}: {n}")
+        if t.dtype != torch.float32 or t.device != p.device:
+            raise ValueError(f"{fn}: {n} must be float32 on {p.device}")
+    if delta_t.dim() != 2 or tuple(delta_t.shape) != (B, T) or (T > 1 and delta_t.stride(1) != 1):
+        raise ValueError(f"{fn}: delta_t must be (B, T) = ({B}, {T}) with contiguous rows")
+    if lam.dim() != 1 or lam.shape[0] != D or (D > 1 and lam.stride(0) != 1):
+        raise ValueError(f"{fn}: lambda must be a contiguous (D,) vector")
+    return delta_t.data_ptr(), (delta_t.stride(0) if B > 1 else T), lam.data_ptr()
+
+
+def mingru_scan_decay(k: torch.Tensor, hx: torch.Tensor, h0: Optional[torch.Tensor],
+                      delta_t: torch.Tensor, lam: torch.Tensor, log1p_delta: bool = False,
+                      out: Optional[torch.Tensor] = None,
+                      workspace: Optional[Workspace] = None) -> torch.Tensor:
+    """minGRU with time decay: the state is gated by exp(-lam_d u_bt) at every
+    token boundary (u = delta_t, or log1p(delta_t)); delta_t (B, T) and lam (D,)
+    are float32 whatever the I/O dtype."""
+    fn = "mingru_scan_decay"
+    _seq(k, fn + ": k")
+    _seq(hx, fn + ": hx")
+    if k.shape != hx.shape or k.dtype != hx.dtype or k.device != hx.device:
+        raise ValueError(f"{fn}: operands must share shape, dtype and device")
+    dt = _dtype_code(k, fn)
+    B, T, D = k.shape
+    ip, ibs = _rows(h0, B, D, k, fn + ": initial state")
+    gp, gbs, lp = _decay_operands(fn, k, delta_t, lam)
+    if out is None:
+        out = torch.empty_like(k)
+    need = int(lib().sgr_workspace_size(_abi.SGR_OP_MINGRU, B, T, D, dt))
+    wp, wn = 0, 0
+    if need:
+        ws = workspace if workspace is not None else default_workspace(k.device, need)
+        wp, wn = ws.ptr, ws.nbytes
+    with torch.cuda.device(k.device):
+        code = lib().mingru_scan_decay(k.data_ptr(), hx.data_ptr(), ip, ibs, gp, gbs, lp,
+                                       int(bool(log1p_delta)), out.data_ptr(), B, T, D, dt, wp, wn,
+                                       _stream(k.device))
+    check(fn, code)
+    return out
+
+
+def mingru_scan_decay_backward(k, hx, h0, delta_t, lam, h, dh, log1p_delta: bool = False,
+                               want_dh0: bool = True, want_dlam: bool = True,
+                               workspace: Optional[Workspace] = None):
+    """(dk, dhx, dh0, dlam) through mingru_scan_decay for dL/dh = dh."""
+    fn = "mingru_scan_decay_backward"
+    for t, n in ((k, "k"), (hx, "hx"), (h, "h"), (dh, "dh")):
+        _seq(t, f"{fn}: {n}")
+        if t.shape != k.shape or t.dtype != k.dtype or t.device != k.device:
+            raise ValueError(f"{fn}: {n} must match k's shape, dtype and device")
+    dt = _dtype_code(k, fn)
+    B, T, D = k.shape
+    ip, ibs = _rows(h0, B, D, k, fn + ": initial state")
+    gp, gbs, lp = _decay_operands(fn, k, delta_t, lam)
+    dk, dhx = torch.empty_like(k), torch.empty_like(k)
+    dh0 = torch.empty((B, D), dtype=k.dtype, device=k.device) if want_dh0 else None
+    dlam = torch.empty((D,), dtype=torch.float32, device=k.device) if want_dlam else None
+    need = int(lib().sgr_backward_workspace_size(_abi.SGR_OP_MINGRU, B, T, D, dt))
+    wp, wn = 0, 0
+    if need:
+        ws = workspace if workspace is not None else default_workspace(k.device, need)
+        wp, wn = ws.ptr, ws.nbytes
+    with torch.cuda.device(k.device):
+        code = lib().mingru_scan_decay_backward(
+            k.data_ptr(), hx.data_ptr(), ip, ibs, gp, gbs, lp, int(bool(log1p_delta)), h.data_ptr(),
+            dh.data_ptr(), dk.data_ptr(), dhx.data_ptr(), dh0.data_ptr() if dh0 is not None else 0, D,
+            dlam.data_ptr() if dlam is not None else 0, B, T, D, dt, wp, wn, _stream(k.device))
+    check(fn, code)
+    return dk, dhx, dh0, dlam
+
+
 def mingru_step(k_t: torch.Tensor, hx_t: torch.Tensor, h_prev: Optional[torch.Tensor] = None,
                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One token: (B, D) rows in (any batch stride, contiguous along D), new

@@ -341,3 +341,22 @@ def test_backward_plan_reverse_indices(shape, dtype, aligned):
                     ends_at_zero[b, d0:d0 + V] += 1
     assert (cover == 1).all()
     assert (ends_at_zero == 1).all()
+
+
+def test_decay_argument_errors():
+    lib = _abi.lib()
+    E = _abi.SGR_ERR_INVALID_ARG
+    G, L = 0x60000000, 0x70000000
+
+    def call(dt=G, dbs=4, lam=L, B=2, T=4, D=8):
+        return lib.mingru_scan_decay(A, Bp, None, 0, dt, dbs, lam, 0, C, B, T, D, F32, None, 0, None)
+
+    assert call(dt=None) == E
+    assert call(lam=None) == E
+    assert call(dbs=-1) == E
+    assert call(dbs=3) == E              # gap rows of a (B, T) array would overlap
+    assert call(B=0) == _abi.SGR_OK
+    db = lib.mingru_scan_decay_backward
+    args = (A, Bp, None, 0, G, 3, L, 0, C, 0x80000000, 0x90000000, 0xA0000000, None, 0, 0xB0000000,
+            2, 4, 8, F32, None, 0, None)
+    assert db(*args) == E               # overlapping gap rows

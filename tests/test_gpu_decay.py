@@ -1,0 +1,130 @@
+"""GPU parity of the time-decay minGRU (mingru_scan_decay, its gradient and
+the autograd wrapper) against the fp64 decay oracle.
+
+Decay contract (page "Your first delta model", Step 5, read for a vector
+state): h_t = (1 - z_t) gamma_t h_{t-1} + z_t g(hx_t), gamma = exp(-lambda u),
+u = delta_t or log1p(delta_t), lambda u > 1e4 wipes the state.  Forward bar:
+max relative error <= 1e-5 fp32 I/O, <= 2e-2 bf16 I/O (the gaps and rates
+are fp32 either way).  Gradients: error relative to each channel's largest
+gradient, as for the plain gradients; dL/dlambda (sums over the batch and
+time, accumulated with atomic adds) relative to the sum of the magnitudes of
+its terms.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import scan_gated_rnns_b200 as sgr
+from scan_gated_rnns_b200 import _abi
+from scan_gated_rnns_b200.synth import Workload, generate
+
+from parity import TOL, TORCH_DT, rel_err
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+DEV = torch.device("cuda:0")
+TOL_BWD = {"f32": 1e-5, "bf16": 2e-2}
+
+
+@pytest.fixture(autouse=True)
+def _reset_hooks():
+    yield
+    lib = _abi.lib()
+    lib.sgr_set_tile_override(0, 0)
+    lib.sgr_set_kernel_override(0)
+
+
+def channel_scaled_err(got, ref) -> float:
+    got = got.detach().to("cpu", torch.float64).numpy() if hasattr(got, "detach") else np.asarray(got)
+    scale = np.abs(ref).max(axis=1, keepdims=True)
+    if not np.isfinite(got).all():
+        return float("inf")
+    return float((np.abs(got - ref) / np.maximum(scale, 1e-30)).max())
+
+
+def data(B, T, D, dtype, init, seed, gap_scale=1.0, wipe_at=None):
+    k, hx, h0 = generate(Workload("t", "mingru", B, T, D, dtype, seed=seed, init=init))
+    g = torch.Generator().manual_seed(seed + 500)
+    dt = torch.empty(B, T).exponential_(1.0 / gap_scale, generator=g)
+    if wipe_at is not None:
+        dt[:, wipe_at] = 3e4
+    lam = torch.rand(D, generator=g) * 2.0
+    return k, hx, h0, dt, lam
+
+
+SHAPES = [(2, 1024, 512), (3, 1000, 96), (1, 777, 36), (2, 300, 7), (1, 1, 1), (1, 4097, 32)]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("init", [None, "u01_1"])
+@pytest.mark.parametrize("log1p_delta", [False, True])
+def test_decay_forward_matches_oracle(shape, dtype, init, log1p_delta):
+    k, hx, h0, dt, lam = data(*shape, dtype, init, seed=sum(shape) % 101,
+                              gap_scale=20.0 if log1p_delta else 0.5,
+                              wipe_at=shape[1] // 2 if shape[1] > 2 else None)
+    h = sgr.mingru_scan_decay(k.to(DEV), hx.to(DEV), None if h0 is None else h0.to(DEV),
+                              dt.to(DEV), lam.to(DEV), log1p_delta)
+    torch.cuda.synchronize()
+    ref = oracle.mingru_decay(k, hx, h0, dt, lam, log1p_delta)
+    assert h.dtype == TORCH_DT[dtype]
+    assert rel_err(h, ref) <= TOL[dtype]
+
+
+# (kernel, rows per thread): tile kernel, 7- and 15-warp pipelined kernels
+@pytest.mark.parametrize("kernel,r", [(1, 2), (1, 4), (2, 2), (2, 4), (3, 4)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decay_every_kernel(kernel, r, dtype):
+    sgr.set_kernel_override(kernel)
+    sgr.set_tile_override(0, r)
+    k, hx, h0, dt, lam = data(3, 2500, 160, dtype, "u01_1", seed=kernel * 7 + r, wipe_at=1300)
+    h = sgr.mingru_scan_decay(k.to(DEV), hx.to(DEV), h0.to(DEV), dt.to(DEV), lam.to(DEV))
+    torch.cuda.synchronize()
+    assert rel_err(h, oracle.mingru_decay(k, hx, h0, dt, lam)) <= TOL[dtype]
+
+
+def test_decay_zero_gaps_equal_plain_scan():
+    k, hx, h0, dt, lam = data(2, 3000, 256, "f32", "u01_1", seed=3)
+    z = torch.zeros_like(dt)
+    a = sgr.mingru_scan_decay(k.to(DEV), hx.to(DEV), h0.to(DEV), z.to(DEV), lam.to(DEV))
+    b = sgr.mingru_scan(k.to(DEV), hx.to(DEV), h0.to(DEV))
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)    # gamma = 2^0 = 1 exactly: the same arithmetic
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("init", [None, "u01_1"])
+@pytest.mark.parametrize("shape", [(2, 1000, 96), (1, 3001, 40), (3, 200, 7)])
+def test_decay_backward_matches_oracle(dtype, init, shape):
+    k, hx, h0, dt, lam = data(*shape, dtype, init, seed=sum(shape) % 89, wipe_at=shape[1] // 3)
+    g = torch.Generator().manual_seed(77)
+    gy = torch.randn(*shape, generator=g).to(TORCH_DT[dtype])
+    fwd = torch.from_numpy(oracle.mingru_decay(k, hx, h0, dt, lam)).to(TORCH_DT[dtype])
+    dk, dhx, dh0, dlam = sgr.mingru_scan_decay_backward(
+        *(None if t is None else t.to(DEV) for t in (k, hx, h0, dt, lam, fwd, gy)))
+    torch.cuda.synchronize()
+    rk, rhx, rh0, rlam = oracle.mingru_decay_backward(k, hx, h0, dt, lam, gy)
+    assert channel_scaled_err(dk, rk) <= TOL_BWD[dtype]
+    assert channel_scaled_err(dhx, rhx) <= TOL_BWD[dtype]
+    # dlam: against the sum of the magnitudes of its terms (the oracle run on |gy|)
+    _, _, _, mag = oracle.mingru_decay_backward(k, hx, h0, dt, lam, np.abs(gy.double().numpy()))
+    scale = np.maximum(np.abs(mag), 1e-30)
+    assert float((np.abs(dlam.cpu().double().numpy() - rlam) / scale).max()) <= TOL_BWD[dtype] * 10
+
+
+def test_decay_autograd_wrapper_learns_lambda():
+    B, T, D = 2, 800, 64
+    k, hx, h0, dt, lam = data(B, T, D, "f32", "u01_1", seed=41)
+    gy = torch.randn(B, T, D, generator=torch.Generator().manual_seed(4))
+    K, H, H0, L = (t.to(DEV).requires_grad_() for t in (k, hx, h0, lam))
+    y = sgr.mingru_scan_decay_fn(K, H, H0, dt.to(DEV), L)
+    (y * gy.to(DEV)).sum().backward()
+    rk, rhx, rh0, rlam = oracle.mingru_decay_backward(k, hx, h0, dt, lam, gy)
+    assert channel_scaled_err(K.grad, rk) <= TOL_BWD["f32"]
+    assert channel_scaled_err(H.grad, rhx) <= TOL_BWD["f32"]
+    assert np.allclose(H0.grad.cpu().double().numpy(), rh0, rtol=1e-4, atol=1e-6)
+    assert np.allclose(L.grad.cpu().double().numpy(), rlam, rtol=1e-3, atol=1e-4)
