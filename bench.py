@@ -333,6 +333,48 @@ def measure_backward_row(w, device, steps=10, warmup=3):
             "bytes_per_launch": bytes_, "kernel": "sgr::scan_backward_kernel"}
 
 
+def measure_decay_rows(w, device, steps=10, warmup=3):
+    """minGRU with time decay on workload w: forward and gradient.  Gaps
+    delta_t ~ Exp(1) per (b, t), rates lambda ~ U(0, 1) per channel (fp32)."""
+    import scan_gated_rnns_b200 as sgr
+    p, q, init = generate(w, device=device)
+    g = torch.Generator(device=device).manual_seed(w.seed + 29)
+    dt = torch.empty(w.B, w.T, device=device).exponential_(1.0, generator=g)
+    lam = torch.rand(w.D, device=device, generator=g)
+    out = torch.empty_like(p)
+    ws = sgr.Workspace(max(sgr.workspace_size("mingru", w.B, w.T, w.D, p.dtype),
+                           sgr._abi.lib().sgr_backward_workspace_size(0, w.B, w.T, w.D,
+                                                                      0 if w.dtype == "f32" else 1)),
+                       device)
+    fwd = lambda: sgr.mingru_scan_decay(p, q, init, dt, lam, out=out, workspace=ws)  # noqa: E731
+    for _ in range(warmup):
+        fwd()
+    torch.cuda.synchronize()
+    _, per_f = timed_launches(fwd, steps, torch.cuda.current_stream(device))
+    gy = torch.randn(p.shape, device=device, generator=g).to(p.dtype)
+    bwd = lambda: sgr.mingru_scan_decay_backward(p, q, init, dt, lam, out, gy, workspace=ws)  # noqa: E731
+    for _ in range(warmup):
+        bwd()
+    torch.cuda.synchronize()
+    _, per_b = timed_launches(bwd, steps, torch.cuda.current_stream(device))
+    peak, _ = hbm_peak()
+    extra = w.B * w.T * 4 + w.D * 4                     # gaps and rates
+    fb = w.algorithmic_bytes() + extra
+    bb = 6 * w.n_elems * w.elem_bytes + extra + w.D * 4 + \
+        (2 * w.B * w.D * w.elem_bytes if init is not None else 0)
+    del p, q, init, out, ws, gy, dt, lam
+    rows = {}
+    for kind, per, bytes_, kern in (("", per_f, fb, "sgr::scan_kernel"),
+                                    ("_backward", per_b, bb, "sgr::scan_backward_kernel")):
+        gbs = bytes_ / per / 1e9
+        rows[w.name.replace("mingru_", f"mingru_decay{kind}_", 1)] = {
+            "op": f"mingru_scan_decay{kind}", "B": w.B, "T": w.T, "D": w.D, "io_dtype": w.dtype,
+            "us_per_launch": round(per * 1e6, 2), "gbs": round(gbs, 1),
+            "gelem_per_s": round(w.n_elems / per / 1e9, 2), "roofline_frac": round(gbs / peak, 4),
+            "bytes_per_launch": bytes_, "kernel": kern}
+    return rows
+
+
 def measure_step_row(device, B=8, D=1024, calls=200, warmup=10):
     """Decode step on (B, D): latency-bound; microseconds per call."""
     import scan_gated_rnns_b200 as sgr
@@ -488,6 +530,8 @@ def run_b200(args):
                      "mingru_b16_t2048_d4096_bf16_h0"):
             rows[name.replace("_b", "_backward_b", 1)] = measure_backward_row(WORKLOADS[name], device)
             torch.cuda.empty_cache()
+        rows.update(measure_decay_rows(WORKLOADS["mingru_b8_t4096_d1024_f32_h0"], device))
+        torch.cuda.empty_cache()
         line["rows"] = rows
     if world > 1:
         import torch.distributed as dist

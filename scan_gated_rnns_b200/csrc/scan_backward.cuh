@@ -133,7 +133,7 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_backward_kernel(const
         // (time decay: and E = (1 - z) h_{t-1} dgamma/dlambda, for dL/dlambda)
         float A[R][V], G[R][V], P[R][V], Q[R][V];
         float E[BOp::kDecay ? R : 1][V];
-        float lam2[V];
+        [[maybe_unused]] float lam2[V];
         if constexpr (BOp::kDecay) {
 #pragma unroll
             for (int v = 0; v < V; ++v) lam2[v] = decay_lam2(p, d0 + v);
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_backward_kernel(const
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const bool ok = dvalid && (top - r) < p.T;
-            float u = 0.f;
+            [[maybe_unused]] float u = 0.f;
             if constexpr (BOp::kDecay) {
                 if ((top - r) < p.T) u = decay_u(p, tc.b, top - r);
             }

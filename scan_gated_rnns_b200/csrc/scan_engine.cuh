@@ -619,14 +619,14 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const Sca
         float2 incl[V];
 #pragma unroll
         for (int v = 0; v < V; ++v) incl[v] = Op::identity();
-        float lam2[V];
+        [[maybe_unused]] float lam2[V];
         if constexpr (Op::kDecay) {
 #pragma unroll
             for (int v = 0; v < V; ++v) lam2[v] = decay_lam2(p, d0 + v);
         }
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            float u = 0.f;        // rows past T: gamma = 1 keeps the padding pair the identity
+            [[maybe_unused]] float u = 0.f;        // rows past T: gamma = 1 keeps the padding pair the identity
             if constexpr (Op::kDecay) {
                 if (row0 + r < p.T) u = decay_u(p, b, row0 + r);
             }
@@ -801,8 +801,10 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
     // for the carry warp, at the price of holding two tiles' pairs in
     // registers; with 8 rows per thread that no longer fits, so those tiles
     // replay right after their own phase A and the per-tile work (warp scan,
-    // barriers, tile coordinates) is spread over twice the elements.
-    constexpr bool LAG = R < 8;
+    // barriers, tile coordinates) is spread over twice the elements.  The
+    // time-decay gate's per-channel rates and per-row gaps do not fit beside
+    // two tiles' pairs either (register spills measured slower than waiting).
+    constexpr bool LAG = R < 8 && !Op::kDecay;
     constexpr int NB = LAG ? 2 : 1;
     static_assert(sizeof(Vec) == V * sizeof(IO), "vector type matches the vector width");
     static_assert(CG * J == 32 && TC % 32 == 0, "lane layout");
@@ -884,7 +886,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                 IA[i] = make_float2(Op::identity().x, Op::identity().x);
                 IB[i] = make_float2(Op::identity().y, Op::identity().y);
             }
-            float lam2[V];
+            [[maybe_unused]] float lam2[V];
             if constexpr (Op::kDecay) {
 #pragma unroll
                 for (int v = 0; v < V; ++v) lam2[v] = decay_lam2(p, d0 + v);
@@ -896,7 +898,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                     float x0[V], x1[V];
                     unpack(*reinterpret_cast<const Vec *>(t0 + r * TC), x0);
                     unpack(*reinterpret_cast<const Vec *>(t1 + r * TC), x1);
-                    float u = 0.f;
+                    [[maybe_unused]] float u = 0.f;
                     if constexpr (Op::kDecay) {
                         if (row0[SB] + r < p.T) u = decay_u(p, tc.b, row0[SB] + r);
                     }
