@@ -50,7 +50,8 @@ from scan_gated_rnns_b200.synth import BENCH_WORKLOAD, WORKLOADS, generate  # no
 METRIC = "scan HBM GB/s (fraction of B200 peak) and Gelem/s at BxTxD, vs CPU oracle"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["scan_gated_rnns_b200/csrc/scan_engine.cuh", "scan_gated_rnns_b200/csrc/sgr_api.cu"]
+KERNEL_SOURCES = ["scan_gated_rnns_b200/csrc/scan_engine.cuh", "scan_gated_rnns_b200/csrc/scan_backward.cuh",
+                  "scan_gated_rnns_b200/csrc/sgr_api.cu"]
 
 
 # ------------------------------------------------------------------ helpers
@@ -73,10 +74,10 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier pool measurement)"
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, kernel: str = "scan_kernel"):
     """dram bytes per launch from the committed ncu summary of this kernel and
     workload, if it was taken on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", f"scan_kernel_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     fields = {}
@@ -439,6 +440,21 @@ def run_b200(args):
     fn = scan_fn(w, p, q, init, out, ws)
     stream = torch.cuda.current_stream(device)
     bytes_step = w.algorithmic_bytes()
+    kernel_name = "sgr::scan_kernel"
+    if args.pass_ == "backward":
+        # the gradient of the same scan: reads both inputs, the forward output
+        # and dL/d out, writes both input gradients (and the initial state's)
+        fn()
+        g = torch.Generator(device=device).manual_seed(w.seed + 17)
+        gy = torch.randn(p.shape, device=device, generator=g).to(p.dtype)
+        wsb = sgr.Workspace(sgr._abi.lib().sgr_backward_workspace_size(
+            0 if w.op == "mingru" else 1, w.B, w.T, w.D, 0 if w.dtype == "f32" else 1), device)
+        bwd = sgr.mingru_scan_backward if w.op == "mingru" else sgr.minmax_scan_backward
+        fn = lambda: bwd(p, q, init, out, gy, init is not None, workspace=wsb)  # noqa: E731
+        bytes_step = 6 * w.n_elems * w.elem_bytes + (2 * w.B * w.D * w.elem_bytes if init is not None else 0)
+        kernel_name = "sgr::scan_backward_kernel"
+        ws = wsb
+        args.no_e2e = True
 
     for _ in range(args.warmup):
         fn()
@@ -494,8 +510,8 @@ def run_b200(args):
     achieved = bytes_step / launch_max / 1e9
     plan = sgr._abi.plan(0 if w.op == "mingru" else 1, w.B, w.T, w.D, 0 if w.dtype == "f32" else 1, True)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": UNIT,
-                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name),
-                "peak_source": peak_src, "kernel": "sgr::scan_kernel",
+                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name, kernel_name.split("::")[1]),
+                "peak_source": peak_src, "kernel": kernel_name,
                 "bytes_per_launch": bytes_step,
                 "launch_us": round(launch_max * 1e6, 2)}
     line = {
@@ -503,7 +519,8 @@ def run_b200(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(agg["ms_per_step"], 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic (seeded torch generator on the device)",
-        "config": {"workload": w.name, "op": f"{w.op}_scan", "B": w.B, "T": w.T, "D": w.D,
+        "config": {"workload": w.name, "op": f"{w.op}_scan" + ("_backward" if args.pass_ == "backward" else ""),
+                   "B": w.B, "T": w.T, "D": w.D,
                    "io_dtype": w.dtype, "initial_state": init is not None,
                    "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
                    "tile": f"{plan['tile_rows']}x{plan['tile_channels']}", "n_tiles": plan["n_tiles"],
@@ -575,7 +592,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(wall / args.steps * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded torch generator)", "impl": "reference",
-        "config": {"workload": w.name, "op": f"{w.op}_scan", "B": w.B, "T": w.T, "D": w.D,
+        "config": {"workload": w.name, "op": f"{w.op}_scan" + ("_backward" if args.pass_ == "backward" else ""),
+                   "B": w.B, "T": w.T, "D": w.D,
                    "io_dtype": w.dtype, "initial_state": ins is not None, "global_batch": w.B,
                    "seq_len": w.T, "parallelism": "cpu"},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": rows, "kind": "oracle",
@@ -593,6 +611,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
+                    help="time the scan (default) or its gradient kernel on the workload")
     ap.add_argument("--no-rows", action="store_true", help="skip the other hot-path rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
