@@ -167,6 +167,41 @@ SGR_API sgr_status_t mingru_scan_noalloc(const void *k, const void *hx,
                                          void *h, int64_t B, int64_t T, int64_t D,
                                          sgr_dtype_t dtype, cudaStream_t stream);
 
+/* ------------------------------------------- time axis split over devices */
+
+/*
+ * A sequence whose time axis is split into contiguous slices, one per device
+ * (rank r holds steps [t_r, t_{r+1})), is scanned with one exchange: every
+ * slice's summary.  The recurrences compose associatively (page "MinMax
+ * Recurrent Neural Cascades", Key properties: parallel training with
+ * O(log T) depth; the minGRU's affine steps likewise), so a slice is
+ * summarised per channel by one pair -- minGRU: h_end = A h_start + B;
+ * MinMax: x_end = max(min(x_start, U), L) -- and the state entering slice r
+ * is slices 0 .. r-1's pairs applied in order to the initial state.
+ *
+ * sgr_scan_summary: pairs (B, D, 2) fp32 (A, B or U, L), DEVICE, for the
+ *   slice in0, in1 (B, T, D); T = 0 gives the identity pair.  Workspace:
+ *   sgr_summary_workspace_size(B, T, D, dtype) bytes of device memory (no
+ *   initialisation needed).  Reads the inputs once.
+ * sgr_combine_summaries: out (B, D) rows (batch stride out_bs, I/O dtype) =
+ *   the state entering slice `rank`, from pairs (n, B, D, 2) fp32 of all
+ *   slices in rank order (only the first `rank` are read) and the initial
+ *   state init (rows with batch stride init_bs; NULL: the scan's default,
+ *   0 for both).  out may be init (same stride) for an in-place update.
+ * The slice is then scanned with mingru_scan / minmax_scan with that state.
+ * The exchange itself (an all-gather of the (B, D, 2) pairs) is the
+ * caller's: the Python package does it with torch.distributed (NCCL).
+ */
+SGR_API size_t sgr_summary_workspace_size(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype);
+SGR_API sgr_status_t sgr_scan_summary(sgr_op_t op, const void *in0, const void *in1,
+                                      int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
+                                      float *pairs, void *workspace, size_t ws_bytes,
+                                      cudaStream_t stream);
+SGR_API sgr_status_t sgr_combine_summaries(sgr_op_t op, const float *pairs, int64_t rank,
+                                           const void *init, int64_t init_bs,
+                                           void *out, int64_t out_bs, int64_t B, int64_t D,
+                                           sgr_dtype_t dtype, cudaStream_t stream);
+
 /* ----------------------------------------------------------- time decay */
 
 /*

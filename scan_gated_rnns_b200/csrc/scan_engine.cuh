@@ -1125,6 +1125,126 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
     }
 }
 
+// ------------------------------------------------ sequence summaries
+//
+// For a time axis split across devices (each holds a contiguous slice), the
+// one exchange a scan needs is each slice's summary: per channel, the
+// composition of all its steps' pairs (minGRU: h_end = A h_start + B; MinMax:
+// x_end = max(min(x_start, U), L)).  Pass 1 folds segments of `seg` rows per
+// thread (one thread per V channels of one segment, rows walked in order) into
+// partial pairs [n_seg][B][D]; pass 2 folds each channel's partials in segment
+// order into [B][D] pairs.  Both read every input once; no state crosses
+// blocks, so there is no hand-off and no waiting.
+template <class Op, typename IO, int V>
+__global__ void __launch_bounds__(256) scan_summary_kernel(const ScanParams p, int64_t seg,
+                                                           int64_t n_seg, float2 *partial) {
+    constexpr int U = V >= 8 ? 2 : (V >= 4 ? 4 : 8);           // rows loaded ahead per thread
+    const int64_t groups = (p.D + V - 1) / V;                 // channel groups per batch row
+    const int64_t n = p.B * groups * n_seg;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t gch = i % groups;                        // channel group fastest: coalesced rows
+        const int64_t rest = i / groups;
+        const int64_t b = rest % p.B;
+        const int64_t sg = rest / p.B;
+        const int64_t d0 = gch * V;
+        const int64_t t0 = sg * seg;
+        const int64_t t1 = t0 + seg < p.T ? t0 + seg : p.T;
+        const IO *in0 = static_cast<const IO *>(p.in0);
+        const IO *in1 = static_cast<const IO *>(p.in1);
+        const bool whole = d0 + V <= p.D;
+        float2 acc[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = Op::identity();
+        [[maybe_unused]] float lam2[V];
+        if constexpr (Op::kDecay) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) lam2[v] = decay_lam2(p, d0 + v);
+        }
+        for (int64_t t = t0; t < t1; t += U) {
+            // all U rows' loads first (memory-level parallelism), then the fold
+            float x0[U][V], x1[U][V];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t off = (b * p.T + t + u) * p.D + d0;
+                if (t + u < t1 && whole) {
+                    Access<IO, V>::load(in0 + off, x0[u]);
+                    Access<IO, V>::load(in1 + off, x1[u]);
+                } else {
+#pragma unroll
+                    for (int v = 0; v < V; ++v) {
+                        const bool ok = t + u < t1 && d0 + v < p.D;
+                        x0[u][v] = ok ? load_scalar<IO>(in0 + off + v) : Op::pad0();
+                        x1[u][v] = ok ? load_scalar<IO>(in1 + off + v) : Op::pad1();
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                [[maybe_unused]] float gu = 0.f;
+                if constexpr (Op::kDecay) gu = (t + u < t1) ? decay_u(p, b, t + u) : 0.f;
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    float e0, e1;
+                    Op::element(x0[u][v], x1[u][v], e0, e1);
+                    if constexpr (Op::kDecay) e0 *= decay_gamma(lam2[v], gu);
+                    acc[v] = Op::combine(acc[v], make_float2(e0, e1));
+                }
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            if (d0 + v < p.D) partial[(sg * p.B + b) * p.D + d0 + v] = acc[v];
+        }
+    }
+}
+
+// out[g][i] = the pairs partial[g G .. g G + G - 1][i] folded in order (the
+// last group may be shorter); one thread per (group, channel), channels
+// fastest so that every load of a segment's pairs is coalesced.
+template <class Op>
+__global__ void __launch_bounds__(256) fold_partials_kernel(const float2 *partial, int64_t n_seg,
+                                                            int64_t G, int64_t BD, float2 *out) {
+    const int64_t n_groups = (n_seg + G - 1) / G;
+    const int64_t n = (n_groups > 0 ? n_groups : 1) * BD;
+    for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < n;
+         idx += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t grp = idx / BD, i = idx - grp * BD;
+        const int64_t s0 = grp * G;
+        const int64_t s1 = s0 + G < n_seg ? s0 + G : n_seg;
+        float2 acc = Op::identity();
+        int64_t sg = s0;
+        for (; sg + 8 <= s1; sg += 8) {             // eight loads in flight, then fold in order
+            float2 x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = partial[(sg + u) * BD + i];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc = Op::combine(acc, x[u]);
+        }
+        for (; sg < s1; ++sg) acc = Op::combine(acc, partial[sg * BD + i]);
+        out[grp * BD + i] = acc;
+    }
+}
+
+// Incoming state of slice `rank`: the summaries of slices 0 .. rank-1 (stored
+// [n_slices][B][D] pairs) applied in order to the initial state (null:
+// the operator's default), written in the I/O type.
+template <class Op, typename IO>
+__global__ void __launch_bounds__(256) combine_summaries_kernel(const float2 *pairs, int64_t rank,
+                                                                const IO *init, int64_t init_bs,
+                                                                IO *out, int64_t out_bs, int64_t B,
+                                                                int64_t D) {
+    const int64_t BD = B * D;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < BD;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t b = i / D, d = i - b * D;
+        float x = init ? load_scalar<IO>(init + b * init_bs + d) : Op::default_init();
+        for (int64_t r = 0; r < rank; ++r) x = Op::apply(pairs[r * BD + i], x);
+        const float y[1] = {x};
+        Access<IO, 1>::store(out + b * out_bs + d, y);
+    }
+}
+
 // ------------------------------------------------------------ step kernel
 //
 // One token for (B, D) rows: the same per-element arithmetic as the scan's

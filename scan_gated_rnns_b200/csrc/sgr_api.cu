@@ -579,6 +579,60 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
     return e == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
 }
 
+// ---- sequence summaries (time axis split across devices)
+struct SumPlan {
+    int V = 1;
+    int64_t seg = 0, n_seg = 0;
+    size_t ws = 0;
+};
+
+SumPlan make_sum_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned) {
+    SumPlan sp;
+    // one 16-byte vector of channels per thread (4 fp32, 8 bf16)
+    const int vw = dtype == SGR_BF16 ? 8 : 4;
+    sp.V = (aligned && D % vw == 0) ? vw : 1;
+    const int64_t groups = (D + sp.V - 1) / sp.V;
+    // about 4096 threads per SM (two waves), each with rows of loads in flight, and at
+    // most 512 segments so that the second pass (one thread per channel
+    // folding its segments) stays short
+    const int64_t target = int64_t(kAssumedSMs) * 4096;
+    int64_t n_seg = (target + B * groups - 1) / (B * groups);
+    n_seg = std::max<int64_t>(1, std::min<int64_t>({n_seg, (T + 7) / 8, int64_t(512)}));
+    sp.seg = (T + n_seg - 1) / n_seg;
+    sp.n_seg = (T + sp.seg - 1) / sp.seg;
+    // partials, then (more than 32 segments) their folds in groups of 32
+    const int64_t n_mid = sp.n_seg > 32 ? (sp.n_seg + 31) / 32 : 0;
+    sp.ws = align_up(size_t(sp.n_seg + n_mid) * size_t(B) * size_t(D) * sizeof(float2), kAlign);
+    return sp;
+}
+
+template <class Op, typename IO>
+cudaError_t launch_summary(const SumPlan &pl, const ScanParams &sp, float2 *partial, float2 *out,
+                           cudaStream_t s) {
+    const int64_t groups = (sp.D + pl.V - 1) / pl.V;
+    const int64_t n = sp.B * groups * pl.n_seg;
+    const unsigned grid = unsigned(std::min<int64_t>((n + 255) / 256, int64_t(kAssumedSMs) * 16));
+    constexpr int VW = 16 / int(sizeof(IO));
+    if (pl.V == 1) {
+        scan_summary_kernel<Op, IO, 1><<<grid, 256, 0, s>>>(sp, pl.seg, pl.n_seg, partial);
+    } else {
+        scan_summary_kernel<Op, IO, VW><<<grid, 256, 0, s>>>(sp, pl.seg, pl.n_seg, partial);
+    }
+    const int64_t BD = sp.B * sp.D;
+    auto grid_for = [](int64_t n) { return unsigned(std::min<int64_t>((n + 255) / 256, int64_t(kAssumedSMs) * 16)); };
+    if (pl.n_seg > 32) {
+        // two levels, so no thread folds more than 32 pairs in a row
+        const int64_t n_mid = (pl.n_seg + 31) / 32;
+        float2 *mid = partial + pl.n_seg * BD;
+        fold_partials_kernel<Op><<<grid_for(n_mid * BD), 256, 0, s>>>(partial, pl.n_seg, 32, BD, mid);
+        fold_partials_kernel<Op><<<grid_for(BD), 256, 0, s>>>(mid, n_mid, n_mid, BD, out);
+    } else {
+        fold_partials_kernel<Op><<<grid_for(BD), 256, 0, s>>>(partial, pl.n_seg, pl.n_seg > 0 ? pl.n_seg : 1,
+                                                              BD, out);
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 extern "C" {
@@ -673,6 +727,99 @@ sgr_status_t mingru_scan_decay_backward(const void *k, const void *hx, const voi
     return run_scan_backward(SGR_OP_MINGRU, k, hx, h0, h0_batch_stride, h, dh, dk, dhx, dh0,
                              dh0_batch_stride, B, T, D, dtype, workspace, ws_bytes, stream, &dec,
                              dlambda);
+}
+
+size_t sgr_summary_workspace_size(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype) {
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return 0;
+    if (B <= 0 || T <= 0 || D <= 0) return 0;
+    const SumPlan a = make_sum_plan(B, T, D, dtype, true), b = make_sum_plan(B, T, D, dtype, false);
+    return a.ws > b.ws ? a.ws : b.ws;
+}
+
+sgr_status_t sgr_scan_summary(sgr_op_t op, const void *in0, const void *in1, int64_t B, int64_t T,
+                              int64_t D, sgr_dtype_t dtype, float *pairs, void *workspace,
+                              size_t ws_bytes, cudaStream_t stream) {
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
+    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return SGR_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || D < 0) return SGR_ERR_INVALID_ARG;
+    if (B == 0 || D == 0) return SGR_OK;
+    if (!pairs) return SGR_ERR_INVALID_ARG;
+    const int esz = dtype == SGR_BF16 ? 2 : 4;
+    int64_t n = 0, nbytes = 0;
+    if (!mul_ok(B, T, &n) || !mul_ok(n, D, &n) || !mul_ok(n, esz, &nbytes)) return SGR_ERR_UNSUPPORTED;
+    const size_t pb = size_t(B) * size_t(D) * 2 * sizeof(float);
+    if (T == 0) {
+        // no steps: the identity pair (minGRU (1, 0); MinMax (+inf, -inf))
+        const int64_t BD = B * D;
+        const unsigned g = unsigned(std::min<int64_t>((BD + 255) / 256, int64_t(kAssumedSMs) * 16));
+        float2 *out = reinterpret_cast<float2 *>(pairs);
+        if (op == SGR_OP_MINGRU) fold_partials_kernel<MinGRUOp><<<g, 256, 0, stream>>>(nullptr, 0, 1, BD, out);
+        else fold_partials_kernel<MinMaxOp><<<g, 256, 0, stream>>>(nullptr, 0, 1, BD, out);
+        return cudaGetLastError() == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
+    }
+    if (!in0 || !in1) return SGR_ERR_INVALID_ARG;
+    if (overlaps(pairs, pb, in0, size_t(nbytes)) || overlaps(pairs, pb, in1, size_t(nbytes)))
+        return SGR_ERR_INVALID_ARG;
+    const bool aligned = aligned16(in0) && aligned16(in1);
+    const SumPlan pl = make_sum_plan(B, T, D, dtype, aligned);
+    if (!workspace || ws_bytes < pl.ws || !aligned16(workspace)) return SGR_ERR_WORKSPACE;
+    if (overlaps(workspace, pl.ws, pairs, pb)) return SGR_ERR_INVALID_ARG;
+    ScanParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.in0 = in0; sp.in1 = in1; sp.B = B; sp.T = T; sp.D = D;
+    float2 *partial = static_cast<float2 *>(workspace);
+    float2 *out = reinterpret_cast<float2 *>(pairs);
+    cudaError_t e;
+    if (op == SGR_OP_MINGRU) {
+        e = dtype == SGR_F32 ? launch_summary<MinGRUOp, float>(pl, sp, partial, out, stream)
+                             : launch_summary<MinGRUOp, __nv_bfloat16>(pl, sp, partial, out, stream);
+    } else {
+        e = dtype == SGR_F32 ? launch_summary<MinMaxOp, float>(pl, sp, partial, out, stream)
+                             : launch_summary<MinMaxOp, __nv_bfloat16>(pl, sp, partial, out, stream);
+    }
+    return e == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
+}
+
+sgr_status_t sgr_combine_summaries(sgr_op_t op, const float *pairs, int64_t rank, const void *init,
+                                   int64_t init_bs, void *out, int64_t out_bs, int64_t B, int64_t D,
+                                   sgr_dtype_t dtype, cudaStream_t stream) {
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
+    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return SGR_ERR_INVALID_ARG;
+    if (B < 0 || D < 0 || rank < 0 || init_bs < 0 || out_bs < 0) return SGR_ERR_INVALID_ARG;
+    if (B == 0 || D == 0) return SGR_OK;
+    if (!out || (rank > 0 && !pairs)) return SGR_ERR_INVALID_ARG;
+    if (B > 1 && out_bs < D) return SGR_ERR_INVALID_ARG;
+    const int esz = dtype == SGR_BF16 ? 2 : 4;
+    int64_t tmp = 0;
+    for (int64_t bs : {init_bs, out_bs})
+        if (!mul_ok(B - 1, bs, &tmp) || !mul_ok(tmp + D, esz, &tmp)) return SGR_ERR_UNSUPPORTED;
+    if (!mul_ok(rank, B, &tmp) || !mul_ok(tmp, D, &tmp) || !mul_ok(tmp, 8, &tmp)) return SGR_ERR_UNSUPPORTED;
+    const size_t ob = rows_span(B, D, out_bs, esz);
+    if (overlaps(out, ob, pairs, size_t(tmp))) return SGR_ERR_INVALID_ARG;
+    const bool in_place = init == out && init_bs == out_bs;
+    if (init && !in_place && overlaps(out, ob, init, rows_span(B, D, init_bs, esz)))
+        return SGR_ERR_INVALID_ARG;
+    const int64_t BD = B * D;
+    const unsigned grid = unsigned(std::min<int64_t>((BD + 255) / 256, int64_t(kAssumedSMs) * 16));
+    const float2 *pp = reinterpret_cast<const float2 *>(pairs);
+    if (op == SGR_OP_MINGRU) {
+        if (dtype == SGR_F32)
+            combine_summaries_kernel<MinGRUOp, float><<<grid, 256, 0, stream>>>(
+                pp, rank, static_cast<const float *>(init), init_bs, static_cast<float *>(out), out_bs, B, D);
+        else
+            combine_summaries_kernel<MinGRUOp, __nv_bfloat16><<<grid, 256, 0, stream>>>(
+                pp, rank, static_cast<const __nv_bfloat16 *>(init), init_bs,
+                static_cast<__nv_bfloat16 *>(out), out_bs, B, D);
+    } else {
+        if (dtype == SGR_F32)
+            combine_summaries_kernel<MinMaxOp, float><<<grid, 256, 0, stream>>>(
+                pp, rank, static_cast<const float *>(init), init_bs, static_cast<float *>(out), out_bs, B, D);
+        else
+            combine_summaries_kernel<MinMaxOp, __nv_bfloat16><<<grid, 256, 0, stream>>>(
+                pp, rank, static_cast<const __nv_bfloat16 *>(init), init_bs,
+                static_cast<__nv_bfloat16 *>(out), out_bs, B, D);
+    }
+    return cudaGetLastError() == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
 }
 
 size_t sgr_backward_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype) {

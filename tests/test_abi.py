@@ -360,3 +360,29 @@ def test_decay_argument_errors():
     args = (A, Bp, None, 0, G, 3, L, 0, C, 0x80000000, 0x90000000, 0xA0000000, None, 0, 0xB0000000,
             2, 4, 8, F32, None, 0, None)
     assert db(*args) == E               # overlapping gap rows
+
+
+def test_summary_and_combine_argument_errors():
+    lib = _abi.lib()
+    E = _abi.SGR_ERR_INVALID_ARG
+    P, W = 0x60000000, 0x70000000
+    need = lib.sgr_summary_workspace_size(2, 100, 64, F32)
+    assert need > 0 and lib.sgr_summary_workspace_size(0, 100, 64, F32) == 0
+    s = lambda *a: lib.sgr_scan_summary(*a)   # noqa: E731
+    assert s(MINGRU, A, Bp, -1, 100, 64, F32, P, W, need, None) == E
+    assert s(7, A, Bp, 2, 100, 64, F32, P, W, need, None) == E
+    assert s(MINGRU, A, Bp, 2, 100, 64, 9, P, W, need, None) == E
+    assert s(MINGRU, A, Bp, 2, 100, 64, F32, None, W, need, None) == E
+    assert s(MINGRU, None, Bp, 2, 100, 64, F32, P, W, need, None) == E
+    assert s(MINGRU, A, Bp, 2, 100, 64, F32, A + 64, W, need, None) == E      # pairs on an input
+    assert s(MINGRU, A, Bp, 2, 100, 64, F32, P, None, 0, None) == _abi.SGR_ERR_WORKSPACE
+    assert s(MINGRU, A, Bp, 2, 100, 64, F32, P, W, need - 256, None) == _abi.SGR_ERR_WORKSPACE
+    assert s(MINGRU, A, Bp, 2, 100, 64, F32, P, P, need, None) == E           # workspace on the pairs
+    assert s(MINGRU, A, Bp, 0, 100, 64, F32, None, None, 0, None) == _abi.SGR_OK
+    c = lambda *a: lib.sgr_combine_summaries(*a)   # noqa: E731
+    assert c(MINGRU, P, -1, None, 0, C, 64, 2, 64, F32, None) == E
+    assert c(MINGRU, None, 1, None, 0, C, 64, 2, 64, F32, None) == E          # pairs needed for rank > 0
+    assert c(MINGRU, P, 1, None, 0, C, 32, 2, 64, F32, None) == E             # out rows overlap
+    assert c(MINGRU, P, 1, None, 0, P + 8, 64, 2, 64, F32, None) == E         # out on the pairs
+    assert c(MINGRU, P, 1, C + 4, 64, C, 64, 2, 64, F32, None) == E           # out partly on init
+    assert c(MINGRU, P, 1, None, 0, None, 64, 0, 64, F32, None) == _abi.SGR_OK
