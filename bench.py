@@ -376,6 +376,25 @@ def measure_decay_rows(w, device, steps=10, warmup=3):
     return rows
 
 
+def measure_summary_row(w, device, steps=10, warmup=3):
+    """The slice summary of the split-time-axis path (the extra pass a rank
+    makes before the exchange): reads both inputs once."""
+    from scan_gated_rnns_b200 import sharded
+    p, q, _ = generate(w, device=device)
+    fn = lambda: sharded.scan_summary(w.op, p, q)   # noqa: E731
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    _, per = timed_launches(fn, steps, torch.cuda.current_stream(device))
+    bytes_ = 2 * w.n_elems * w.elem_bytes + w.B * w.D * 8
+    peak, _ = hbm_peak()
+    gbs = bytes_ / per / 1e9
+    del p, q
+    return {"op": f"{w.op}_scan_summary", "B": w.B, "T": w.T, "D": w.D, "io_dtype": w.dtype,
+            "us_per_call": round(per * 1e6, 2), "gbs": round(gbs, 1), "roofline_frac": round(gbs / peak, 4),
+            "bytes_per_call": bytes_, "kernel": "sgr::scan_summary_kernel + fold_partials_kernel"}
+
+
 def measure_step_row(device, B=8, D=1024, calls=200, warmup=10):
     """Decode step on (B, D): latency-bound; microseconds per call."""
     import scan_gated_rnns_b200 as sgr
@@ -549,6 +568,9 @@ def run_b200(args):
             torch.cuda.empty_cache()
         rows.update(measure_decay_rows(WORKLOADS["mingru_b8_t4096_d1024_f32_h0"], device))
         torch.cuda.empty_cache()
+        for name in ("mingru_b8_t4096_d1024_f32_h0", "mingru_b1_t131072_d512_f32_h0"):
+            rows[name.replace("mingru_", "mingru_summary_", 1)] = measure_summary_row(WORKLOADS[name], device)
+            torch.cuda.empty_cache()
         line["rows"] = rows
     if world > 1:
         import torch.distributed as dist
