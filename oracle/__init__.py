@@ -26,6 +26,10 @@ Functions (all inputs are widened exactly to float64 first):
     minGRU with time decay: the state is gated by gamma_t = exp(-lam_d u_bt)
     (u = dt or log1p(dt); lam u > 1e4 wipes it) at each token boundary; page
     "Your first delta model", Step 5.  ``mingru_decay_backward`` adds dlam.
+``mingru_projected(x, w, h0=None)``
+    the minGRU layer's input projection and scan: k = x W[:D]^T, hx = x W[D:]^T
+    (fp64 matrix products, numpy), then ``mingru_linear``; page "Mingru
+    Pytorch" (the layer applied to a (B, T, d) input).
 ``mingru_backward(k, hx, h0, gy)`` / ``minmax_backward(r, s, x0, gy)``
     gradients of a loss with dL/d out = gy with respect to both inputs and the
     initial state, by the chain rule through the sequential loop (forward
@@ -249,3 +253,15 @@ def mingru_decay_backward(k, hx, h0, dt, lam, gy, log1p_delta: bool = False):
     if rc != 0:
         raise RuntimeError(f"oracle_mingru_decay_backward returned {rc}")
     return dk, dhx, dh0, dlam
+
+
+def mingru_projected(x, w, h0=None, threads: int = 1) -> np.ndarray:
+    """fp64: the projections k = x w[:D]^T and hx = x w[D:]^T of a (B, T, d_in)
+    input by a (2 D, d_in) weight, then the minGRU recurrence."""
+    x, w = _as_f64(x), _as_f64(w)
+    if x.ndim != 3 or w.ndim != 2 or w.shape[1] != x.shape[2] or w.shape[0] % 2:
+        raise ValueError(f"x must be (B, T, d_in) and w (2 D, d_in), got {x.shape} {w.shape}")
+    D = w.shape[0] // 2
+    k = np.ascontiguousarray(x @ w[:D].T)
+    hx = np.ascontiguousarray(x @ w[D:].T)
+    return mingru_linear(k, hx, h0, threads=threads)

@@ -74,6 +74,8 @@ SIGNATURES.update({
                                     _i64, _i64, _i64, _int, _vp, _sz, _vp]),
     "sgr_backward_workspace_size": (_sz, [_int, _i64, _i64, _i64, _int]),
     "sgr_summary_workspace_size": (_sz, [_i64, _i64, _i64, _int]),
+    "sgr_projected_workspace_size": (_sz, [_i64, _i64, _i64]),
+    "mingru_projected_scan": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp]),
     "sgr_scan_summary": (_int, [_int, _vp, _vp, _i64, _i64, _i64, _int, _vp, _vp, _sz, _vp]),
     "sgr_combine_summaries": (_int, [_int, _vp, _i64, _vp, _i64, _vp, _i64, _i64, _i64, _int, _vp]),
     "mingru_scan_decay": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _vp, _int, _vp, _i64, _i64, _i64,

@@ -2,6 +2,7 @@
 // argument checks, the choice of chunk shape, the workspace layout and the
 // kernel launches.  No allocation, no synchronisation on the scan paths.
 #include "scan_gated_rnns.h"
+#include "projected_scan.cuh"
 #include "scan_backward.cuh"
 #include "scan_engine.cuh"
 
@@ -633,6 +634,98 @@ cudaError_t launch_summary(const SumPlan &pl, const ScanParams &sp, float2 *part
     return cudaGetLastError();
 }
 
+// ---- input projection fused with the scan (projected_scan.cuh)
+size_t projected_ws_bytes(int64_t B, int64_t T, int64_t D) {
+    const int64_t n_chunks = (T + proj::kTR - 1) / proj::kTR;
+    const int64_t n_tiles = n_chunks * B * (D / proj::kTC);
+    return align_up(kAlign + size_t(n_tiles) * 3 * proj::kTC * 8, kAlign);
+}
+
+sgr_status_t run_projected_scan(const void *x, const void *w, const float *h0, int64_t h0_bs, float *h,
+                                int64_t B, int64_t T, int64_t D, int64_t d_in, void *ws, size_t ws_bytes,
+                                cudaStream_t stream) {
+    if (B < 0 || T < 0 || D < 0 || d_in < 0 || h0_bs < 0) return SGR_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || D == 0) return SGR_OK;
+    if (D % proj::kTC != 0 || d_in % proj::kKB != 0 || d_in == 0) return SGR_ERR_UNSUPPORTED;
+    if (!x || !w || !h) return SGR_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w)) return SGR_ERR_INVALID_ARG;
+    int64_t n = 0, xb = 0, hb = 0, wb = 0, tmp = 0;
+    if (!mul_ok(B, T, &n) || !mul_ok(n, d_in, &xb) || !mul_ok(xb, 2, &xb)) return SGR_ERR_UNSUPPORTED;
+    if (!mul_ok(n, D, &hb) || !mul_ok(hb, 4, &hb)) return SGR_ERR_UNSUPPORTED;
+    if (!mul_ok(2 * D, d_in, &wb) || !mul_ok(wb, 2, &wb)) return SGR_ERR_UNSUPPORTED;
+    if (h0 && (!mul_ok(B - 1, h0_bs, &tmp) || !mul_ok(tmp + D, 4, &tmp))) return SGR_ERR_UNSUPPORTED;
+    if (T > (int64_t(1) << 31) - 1 || d_in > (int64_t(1) << 31) - 1 || 2 * D > (int64_t(1) << 31) - 1)
+        return SGR_ERR_UNSUPPORTED;                    // tensor-map coordinates are 32-bit
+    const size_t ib = h0 ? rows_span(B, D, h0_bs, 4) : 0;
+    if (overlaps(h, size_t(hb), x, size_t(xb)) || overlaps(h, size_t(hb), w, size_t(wb)) ||
+        overlaps(h, size_t(hb), h0, ib))
+        return SGR_ERR_INVALID_ARG;
+    const int64_t n_chunks = (T + proj::kTR - 1) / proj::kTR;
+    const int64_t n_dt = D / proj::kTC;
+    const int64_t n_tiles = n_chunks * B * n_dt;
+    if (n_tiles > int64_t(std::numeric_limits<int>::max())) return SGR_ERR_UNSUPPORTED;
+    const size_t need = projected_ws_bytes(B, T, D);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return SGR_ERR_WORKSPACE;
+
+    ProjParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    ScanParams &sp = pp.s;
+    sp.init = h0; sp.init_bs = h0_bs; sp.out = h;
+    sp.B = B; sp.T = T; sp.D = D;
+    sp.n_dt = n_dt; sp.n_chains = B * n_dt; sp.n_chunks = n_chunks; sp.n_tiles = n_tiles;
+    sp.by_chains = make_fastdiv(uint32_t(sp.n_chains));
+    sp.by_dt = make_fastdiv(uint32_t(n_dt));
+    sp.spin_limit = g_spin_limit.load();
+    sp.drop_tile = g_drop_tile.load();
+    char *wsc = static_cast<char *>(ws);
+    sp.status = reinterpret_cast<uint32_t *>(wsc);
+    sp.words = reinterpret_cast<uint64_t *>(wsc + kAlign);
+    pp.d_in = d_in;
+
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (enc == nullptr) return SGR_ERR_CUDA;
+    alignas(64) CUtensorMap map_x, map_w;
+    {
+        const cuuint64_t dims[3] = {cuuint64_t(d_in), cuuint64_t(T), cuuint64_t(B)};
+        const cuuint64_t strides[2] = {cuuint64_t(d_in) * 2, cuuint64_t(T) * cuuint64_t(d_in) * 2};
+        const cuuint32_t box[3] = {cuuint32_t(proj::kKB), cuuint32_t(proj::kTR), 1u};
+        const cuuint32_t es[3] = {1u, 1u, 1u};
+        if (enc(&map_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(x), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return SGR_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {cuuint64_t(d_in), cuuint64_t(2 * D)};
+        const cuuint64_t strides[1] = {cuuint64_t(d_in) * 2};
+        const cuuint32_t box[2] = {cuuint32_t(proj::kKB), cuuint32_t(proj::kTC)};
+        const cuuint32_t es[2] = {1u, 1u};
+        if (enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(w), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return SGR_ERR_CUDA;
+    }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return SGR_ERR_CUDA;
+    if (cs == cudaStreamCaptureStatusActive) {
+        if (cudaMemsetAsync(sp.words, 0, need - kAlign, stream) != cudaSuccess) return SGR_ERR_CUDA;
+        sp.epoch = 1;
+    } else {
+        sp.epoch = next_epoch();
+    }
+    static std::atomic<int> attr_set[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SGR_ERR_CUDA;
+    if (dev < 0 || dev >= 64 || attr_set[dev].load() == 0) {
+        if (cudaFuncSetAttribute(mingru_projected_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(proj::kSmemBytes)) != cudaSuccess)
+            return SGR_ERR_CUDA;
+        if (dev >= 0 && dev < 64) attr_set[dev].store(1);
+    }
+    mingru_projected_scan_kernel<<<unsigned(n_tiles), 256, proj::kSmemBytes, stream>>>(pp, map_x, map_w);
+    return cudaGetLastError() == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -727,6 +820,17 @@ sgr_status_t mingru_scan_decay_backward(const void *k, const void *hx, const voi
     return run_scan_backward(SGR_OP_MINGRU, k, hx, h0, h0_batch_stride, h, dh, dk, dhx, dh0,
                              dh0_batch_stride, B, T, D, dtype, workspace, ws_bytes, stream, &dec,
                              dlambda);
+}
+
+size_t sgr_projected_workspace_size(int64_t B, int64_t T, int64_t D) {
+    if (B <= 0 || T <= 0 || D <= 0 || D % proj::kTC != 0) return 0;
+    return projected_ws_bytes(B, T, D);
+}
+
+sgr_status_t mingru_projected_scan(const void *x, const void *w, const float *h0, int64_t h0_batch_stride,
+                                   float *h, int64_t B, int64_t T, int64_t D, int64_t d_in,
+                                   void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    return run_projected_scan(x, w, h0, h0_batch_stride, h, B, T, D, d_in, workspace, ws_bytes, stream);
 }
 
 size_t sgr_summary_workspace_size(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype) {

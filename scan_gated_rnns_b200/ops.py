@@ -251,6 +251,39 @@ def mingru_scan_decay_backward(k, hx, h0, delta_t, lam, h, dh, log1p_delta: bool
     return dk, dhx, dh0, dlam
 
 
+def mingru_projected_scan(x: torch.Tensor, w: torch.Tensor, h0: Optional[torch.Tensor] = None,
+                          out: Optional[torch.Tensor] = None,
+                          workspace: Optional[Workspace] = None) -> torch.Tensor:
+    """h (B, T, D) float32 = minGRU scan of k = x w[:D]^T, hx = x w[D:]^T, with
+    the projection on the tensor cores in the same kernel (x (B, T, d_in) and
+    w (2 D, d_in) bfloat16; D % 128 == 0, d_in % 64 == 0)."""
+    fn = "mingru_projected_scan"
+    _seq(x, fn + ": x")
+    _need_cuda(w, fn + ": w")
+    if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16 or w.device != x.device:
+        raise ValueError(f"{fn}: x and w must be bfloat16 on one device")
+    if w.dim() != 2 or w.shape[1] != x.shape[2] or w.shape[0] % 2 or not w.is_contiguous():
+        raise ValueError(f"{fn}: w must be a contiguous (2 D, d_in) matrix")
+    B, T, d_in = x.shape
+    D = w.shape[0] // 2
+    like = torch.empty(0, dtype=torch.float32, device=x.device)
+    ip, ibs = _rows(h0, B, D, like, fn + ": h0")
+    if out is None:
+        out = torch.empty((B, T, D), dtype=torch.float32, device=x.device)
+    elif tuple(out.shape) != (B, T, D) or out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError(f"{fn}: out must be a contiguous (B, T, D) float32 tensor")
+    need = int(lib().sgr_projected_workspace_size(B, T, D))
+    wp, wn = 0, 0
+    if need:
+        ws = workspace if workspace is not None else default_workspace(x.device, need)
+        wp, wn = ws.ptr, ws.nbytes
+    with torch.cuda.device(x.device):
+        code = lib().mingru_projected_scan(x.data_ptr(), w.data_ptr(), ip, ibs, out.data_ptr(), B, T, D, d_in,
+                                           wp, wn, _stream(x.device))
+    check(fn, code)
+    return out
+
+
 def mingru_step(k_t: torch.Tensor, hx_t: torch.Tensor, h_prev: Optional[torch.Tensor] = None,
                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One token: (B, D) rows in (any batch stride, contiguous along D), new

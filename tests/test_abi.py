@@ -386,3 +386,23 @@ def test_summary_and_combine_argument_errors():
     assert c(MINGRU, P, 1, None, 0, P + 8, 64, 2, 64, F32, None) == E         # out on the pairs
     assert c(MINGRU, P, 1, C + 4, 64, C, 64, 2, 64, F32, None) == E           # out partly on init
     assert c(MINGRU, P, 1, None, 0, None, 64, 0, 64, F32, None) == _abi.SGR_OK
+
+
+def test_projected_scan_argument_errors():
+    lib = _abi.lib()
+    X, W, H, WS = 0x10000000, 0x20000000, 0x30000000, 0x40000000
+
+    def call(x=X, w=W, h0=None, hbs=0, h=H, B=2, T=10, D=128, d=64, ws=WS, wn=1 << 20):
+        return lib.mingru_projected_scan(x, w, h0, hbs, h, B, T, D, d, ws, wn, None)
+
+    E = _abi.SGR_ERR_INVALID_ARG
+    assert call(B=-1) == E
+    assert call(x=None) == E
+    assert call(x=X + 8) == E                    # x must be 16-byte aligned (tensor map)
+    assert call(D=96) == _abi.SGR_ERR_UNSUPPORTED
+    assert call(d=48) == _abi.SGR_ERR_UNSUPPORTED
+    assert call(h=X + 64) == E                   # output on x
+    assert call(ws=None, wn=0) == _abi.SGR_ERR_WORKSPACE
+    assert call(wn=lib.sgr_projected_workspace_size(2, 10, 128) - 1) == _abi.SGR_ERR_WORKSPACE
+    assert call(B=0) == _abi.SGR_OK
+    assert lib.sgr_projected_workspace_size(2, 10, 96) == 0
