@@ -395,6 +395,66 @@ def measure_summary_row(w, device, steps=10, warmup=3):
             "bytes_per_call": bytes_, "kernel": "sgr::scan_summary_kernel + fold_partials_kernel"}
 
 
+def bf16_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    except Exception:
+        return 1590.0, "fallback (1.59 PFLOP/s earlier pool measurement)"
+
+
+PROJECTED = {"B": 8, "T": 4096, "D": 1024, "d_in": 1024}
+
+
+def projected_inputs(device, B, T, D, d_in, seed=31):
+    g = torch.Generator(device=device).manual_seed(seed)
+    x = torch.randn(B, T, d_in, device=device, generator=g).to(torch.bfloat16)
+    w = (torch.randn(2 * D, d_in, device=device, generator=g) / d_in ** 0.5).to(torch.bfloat16)
+    h0 = torch.rand(B, D, device=device, generator=g) * 0.9 + 0.1
+    return x, w, h0
+
+
+def measure_projected_row(device, steps=10, warmup=3, B=8, T=4096, D=1024, d_in=1024):
+    """The minGRU layer's input projection fused with the scan (tensor cores),
+    against the same work unfused: two cuBLAS bf16 GEMMs writing k and hx,
+    then the bf16 scan."""
+    import scan_gated_rnns_b200 as sgr
+    x, w, h0 = projected_inputs(device, B, T, D, d_in)
+    out = torch.empty(B, T, D, device=device)
+    ws = sgr.Workspace(sgr._abi.lib().sgr_projected_workspace_size(B, T, D), device)
+    fused = lambda: sgr.mingru_projected_scan(x, w, h0, out=out, workspace=ws)  # noqa: E731
+    for _ in range(warmup):
+        fused()
+    torch.cuda.synchronize()
+    _, per = timed_launches(fused, steps, torch.cuda.current_stream(device))
+    k = torch.empty(B, T, D, device=device, dtype=torch.bfloat16)
+    hx = torch.empty_like(k)
+    hb = torch.empty_like(k)
+    wsb = sgr.Workspace(sgr.workspace_size("mingru", B, T, D, torch.bfloat16), device)
+    h0b = h0.to(torch.bfloat16)
+    wk, wh = w[:D], w[D:]
+
+    def unfused():
+        torch.matmul(x, wk.t(), out=k)
+        torch.matmul(x, wh.t(), out=hx)
+        sgr.mingru_scan(k, hx, h0b, out=hb, workspace=wsb)
+
+    for _ in range(warmup):
+        unfused()
+    torch.cuda.synchronize()
+    _, per_u = timed_launches(unfused, steps, torch.cuda.current_stream(device))
+    flops = 2.0 * B * T * d_in * 2 * D
+    peak, src = bf16_peak()
+    del x, w, h0, out, ws, k, hx, hb, wsb
+    return {"op": "mingru_projected_scan", "B": B, "T": T, "D": D, "d_in": d_in, "io_dtype": "bf16 in, f32 out",
+            "us_per_launch": round(per * 1e6, 2), "tflops": round(flops / per / 1e12, 1),
+            "roofline_frac": round(flops / per / 1e12 / peak, 4), "peak_tflops": peak, "peak_source": src,
+            "flops_per_launch": flops, "kernel": "sgr::mingru_projected_scan_kernel (tcgen05)",
+            "unfused_us": round(per_u * 1e6, 2),
+            "unfused": "torch.matmul bf16 x2 (cuBLAS) to k, hx + mingru_scan bf16"}
+
+
 def measure_step_row(device, B=8, D=1024, calls=200, warmup=10):
     """Decode step on (B, D): latency-bound; microseconds per call."""
     import scan_gated_rnns_b200 as sgr
@@ -460,6 +520,17 @@ def run_b200(args):
     stream = torch.cuda.current_stream(device)
     bytes_step = w.algorithmic_bytes()
     kernel_name = "sgr::scan_kernel"
+    if args.pass_ == "projected":
+        # the input projection fused with the scan: x (B, T, d_in) and W (2 D, d_in) bf16
+        P = PROJECTED
+        x, wproj, hp0 = projected_inputs(device, P["B"], P["T"], P["D"], P["d_in"], seed=shard_seed(31, rank))
+        hout = torch.empty(P["B"], P["T"], P["D"], device=device)
+        wsp = sgr.Workspace(sgr._abi.lib().sgr_projected_workspace_size(P["B"], P["T"], P["D"]), device)
+        fn = lambda: sgr.mingru_projected_scan(x, wproj, hp0, out=hout, workspace=wsp)  # noqa: E731
+        bytes_step = 2 * P["B"] * P["T"] * P["d_in"] + 4 * P["D"] * P["d_in"] + 4 * P["B"] * P["T"] * P["D"]
+        kernel_name = "sgr::mingru_projected_scan_kernel"
+        ws = wsp
+        args.no_e2e = True
     if args.pass_ == "backward":
         # the gradient of the same scan: reads both inputs, the forward output
         # and dL/d out, writes both input gradients (and the initial state's)
@@ -533,6 +604,15 @@ def run_b200(args):
                 "peak_source": peak_src, "kernel": kernel_name,
                 "bytes_per_launch": bytes_step,
                 "launch_us": round(launch_max * 1e6, 2)}
+    if args.pass_ == "projected":
+        P = PROJECTED
+        flops = 2.0 * P["B"] * P["T"] * P["d_in"] * 2 * P["D"]
+        tpeak, tsrc = bf16_peak()
+        roofline = {"bound": "tensor", "achieved": round(flops / launch_max / 1e12, 1), "peak": tpeak,
+                    "unit": "TFLOP/s", "frac": round(flops / launch_max / 1e12 / tpeak, 4),
+                    "traffic": recorded_traffic("b8_t4096_d1024_din1024", "mingru_projected_scan_kernel"),
+                    "peak_source": tsrc, "kernel": kernel_name, "flops_per_launch": flops,
+                    "launch_us": round(launch_max * 1e6, 2)}
     line = {
         "metric": METRIC, "value": round(agg["gbs"], 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(agg["ms_per_step"], 4),
@@ -571,6 +651,8 @@ def run_b200(args):
         for name in ("mingru_b8_t4096_d1024_f32_h0", "mingru_b1_t131072_d512_f32_h0"):
             rows[name.replace("mingru_", "mingru_summary_", 1)] = measure_summary_row(WORKLOADS[name], device)
             torch.cuda.empty_cache()
+        rows["mingru_projected_b8_t4096_d1024_din1024"] = measure_projected_row(device)
+        torch.cuda.empty_cache()
         line["rows"] = rows
     if world > 1:
         import torch.distributed as dist
@@ -633,8 +715,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
-                    help="time the scan (default) or its gradient kernel on the workload")
+    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward", "projected"],
+                    help="time the scan (default), its gradient kernel on the workload, or the input "
+                         "projection fused with the scan (B8 T4096 D1024 d_in 1024)")
     ap.add_argument("--no-rows", action="store_true", help="skip the other hot-path rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
