@@ -178,14 +178,14 @@ SGR_API sgr_status_t mingru_scan_noalloc(const void *k, const void *hx,
  *     hx[b, t, c] = sum_j x[b, t, j] W[D + c, j]
  *     h = the minGRU scan of (k, hx) from h0, as mingru_scan
  * k and hx are computed on the tensor cores (bf16 operands, fp32
- * accumulation, tcgen05.mma) in tiles of 128 tokens x 128 channels and
+ * accumulation, tcgen05.mma) in tiles of 64 channels x 256 tokens and
  * consumed in place: they are never written to memory.
  *   x   : bf16 DEVICE (B, T, d_in) contiguous, 16-byte aligned
  *   w   : bf16 DEVICE (2 D, d_in) contiguous, 16-byte aligned (a linear
  *         layer's weight, out_features = 2 D: rows 0..D-1 give k, D..2D-1 hx)
  *   h0  : fp32 DEVICE rows (B, D), batch stride h0_batch_stride, or NULL (0)
  *   h   : fp32 DEVICE (B, T, D) output
- *   D % 128 == 0 and d_in % 64 == 0 (else SGR_ERR_UNSUPPORTED); any T.
+ *   D % 64 == 0 and d_in % 64 == 0 (else SGR_ERR_UNSUPPORTED); any T.
  *   workspace: sgr_projected_workspace_size(B, T, D) bytes, zero-filled once
  *         (same rules as the scans' workspace; always needed).
  */

@@ -2,23 +2,36 @@
 //
 // The layer (page "Mingru Pytorch": a module applied to a (B, T, d) input)
 // computes k and hx from the input by a linear projection and scans them.
-// Here one kernel does both for a tile of 128 tokens x 128 channels:
-//   k[t, c]  = sum_j x[t, j] W[c, j],   hx[t, c] = sum_j x[t, j] W[D + c, j]
+// Here one kernel does both for a tile of 64 channels x 256 tokens:
+//   k[c, t]  = sum_j W[c, j] x[t, j],   hx[c, t] = sum_j W[D + c, j] x[t, j]
 // on the 5th-generation tensor cores (tcgen05.mma, bf16 operands, fp32
 // accumulators in tensor memory, operands staged by the tensor memory
 // accelerator with 128-byte swizzle), then the activations, the tile's scan
 // and the chunk hand-off of the scan engine, and writes h.  k and hx never go
 // to HBM.
 //
-// Warp roles (8 warps): warp 0 loads x and W tiles into a 2-stage ring; warp
-// 1 allocates tensor memory and issues the MMAs (one thread); then all 8
-// warps run the epilogue, for each half of the tile's channels in turn: each
-// thread reads 32 accumulator columns of one token row and writes the (a, b)
-// pairs to shared memory (the ring, idle by then), then owns one channel and
-// a quarter of the rows: folds them, gets the tile's incoming state (warp 0
-// publishes the chunk summary and looks back), replays and stores.  About 99 KB of
-// shared memory and 256 of the 512 tensor-memory columns per block, so two
-// blocks share an SM and one's epilogue runs beside the other's MMAs.
+// The product is taken transposed: the MMA's M side is the tile's 64 k rows
+// and 64 hx rows of W, interleaved in groups of 16 (W rows k 0-15, hx 0-15,
+// k 16-31, hx 16-31, ...), its N side 256 tokens.  Tensor-memory lane = W
+// row, column = token, so every thread that reads the accumulator holds one
+// channel's values along time -- the order of the recurrence -- and the k and
+// hx of a channel sit 16 lanes apart in the same warp, one shuffle from each
+// other.  No shared-memory transpose, and one look-back per tile.
+//
+// Persistent blocks, one per SM (cooperative launch: every look-back waits
+// for a block that is resident), each taking tiles blockIdx.x, blockIdx.x +
+// gridDim.x, ...  Warp 0 streams W and x tiles by TMA into a 4-stage ring
+// (continuing across tiles); one thread of warp 1 issues the MMAs of tile i
+// into one of two accumulators (512 tensor-memory columns in all) while warps
+// 4-19 run the epilogue of tile i-1 from the other.  Epilogue warp (q, g)
+// reads lane quarter q (channels 16q .. 16q+15, k and hx) and columns 64g ..
+// 64g+63; after the exchange each thread owns one channel and 32 consecutive
+// tokens: it computes their (a, b) pairs into registers and folds them; warp
+// 2 combines the eight folds of each channel, publishes the chunk summary,
+// looks back and publishes the state; each thread then replays its tokens
+// from the state before them and stores h.  The carry is warp 2's, so that the
+// look-back's registers do not add to the epilogue threads' (which hold their
+// 32 pairs across it).
 #pragma once
 
 #include "scan_engine.cuh"
@@ -33,22 +46,28 @@ struct ProjParams {
 
 namespace proj {
 
-constexpr int kTR = 128;            // tokens per tile (MMA M)
-constexpr int kTC = 128;            // channels per tile: N = 2 kTC (k and hx)
-constexpr int kN = 2 * kTC;
+constexpr int kTR = 256;            // tokens per tile (MMA N)
+constexpr int kTC = 64;             // channels per tile
+constexpr int kM = 2 * kTC;         // MMA M: k and hx rows of W
+constexpr int kGrp = 16;            // W rows per interleave group
 constexpr int kKB = 64;             // K per stage: one 128-byte swizzle row of bf16
-constexpr int kStages = 2;          // two blocks per SM: one's epilogue overlaps the other's MMAs
-constexpr int kHalf = kTC / 2;      // the epilogue handles the channels in two halves
-constexpr uint32_t kABytes = kTR * kKB * 2;     // 16 KB
-constexpr uint32_t kBBytes = kN * kKB * 2;      // 32 KB
+constexpr int kStages = 4;
+constexpr uint32_t kGrpBytes = kGrp * kKB * 2;  // 2 KB: one group of W rows
+constexpr uint32_t kABytes = kM * kKB * 2;      // 16 KB (W)
+constexpr uint32_t kBBytes = kTR * kKB * 2;     // 32 KB (x)
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr uint32_t kRingBytes = kStages * kStageBytes;            // 96 KB
-constexpr uint32_t kPairBytes = kTR * kHalf * 8;                  // 64 KB, aliases the ring
-static_assert(kPairBytes <= kRingBytes, "pairs fit in the idle ring");
+constexpr uint32_t kRingBytes = kStages * kStageBytes;            // 192 KB
 constexpr uint32_t kBarOffset = kRingBytes;
-// + align slack; barriers; four row-quarter fold results and the incoming states
-constexpr uint32_t kSmemBytes = 1024 + kRingBytes + 256 + 4 * kHalf * 8 + kHalf * 4;
-constexpr uint32_t kTmemCols = 256;
+constexpr int kEpiWarps = 16;                   // warps 4 .. 19
+constexpr int kThreads = (4 + kEpiWarps) * 32;
+constexpr int kSegs = kEpiWarps / 4 * 2;        // 32-token segments of a tile: 8
+// + align slack; barriers; per tile parity: the segments' folds and the
+// channels' incoming states
+constexpr uint32_t kSmemBytes = 1024 + kBarOffset + 256 + 2 * kSegs * kTC * 8 + 2 * kTC * 4;
+static_assert(kSmemBytes <= 227 * 1024, "one block per SM");
+static_assert(kSegs * 32 == kTR && kEpiWarps % 4 == 0, "epilogue covers the tile");
+constexpr uint32_t kAccCols = kTR;              // fp32 accumulator columns per tile
+constexpr uint32_t kTmemCols = 2 * kAccCols;    // two accumulators
 constexpr uint32_t kWaitLimit = 1u << 20;
 
 // K-major operand with 128-byte swizzle: rows of 128 bytes, 8-row groups
@@ -63,8 +82,8 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
 }
 
 // kind::f16 instruction descriptor: bf16 x bf16 -> fp32, both K-major, M x N
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kN >> 3) << 17) |
-                            (uint32_t(kTR >> 4) << 24);
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kTR >> 3) << 17) |
+                            (uint32_t(kM >> 4) << 24);
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
     asm volatile(
@@ -79,7 +98,7 @@ __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, uint32_t lim
     return false;
 }
 
-// 32 consecutive accumulator columns of this thread's row (lane quarter of
+// 32 consecutive accumulator columns of this thread's lane (lane quarter of
 // the warp); completes with tmem_wait
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
@@ -93,42 +112,38 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// the pair of (row r, channel c of the half) in the epilogue buffer: rows of
-// kHalf pairs, channel index xor-ed with the row's low bits so that a warp
-// writing one channel of 32 rows, and a warp reading 32 channels of one row,
-// both touch every bank evenly
-__device__ __forceinline__ uint32_t pair_slot(int r, int c) { return uint32_t(r * kHalf + (c ^ (r & 15))); }
-
 }  // namespace proj
 
-__global__ void __launch_bounds__(256, 2) mingru_projected_scan_kernel(const ProjParams pp,
-                                                                      const __grid_constant__ CUtensorMap map_x,
-                                                                      const __grid_constant__ CUtensorMap map_w) {
+__global__ void __launch_bounds__(proj::kThreads, 1) mingru_projected_scan_kernel(
+    const ProjParams pp, const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w) {
     using namespace proj;
     using Op = MinGRUOp;
-    constexpr int CV = kHalf / 32;          // channels per carry lane within a half
+    constexpr int CV = kTC / 32;            // channels per carry lane
     const ScanParams &p = pp.s;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                             ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOffset);   // full[S], empty[S], done
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kStages + 1);
-    float2 *s_part = reinterpret_cast<float2 *>(smem + kBarOffset + 256);          // [4][kHalf]
-    float *s_hin = reinterpret_cast<float *>(smem + kBarOffset + 256 + 4 * kHalf * 8);
-    float2 *pairs = reinterpret_cast<float2 *>(smem);                   // after the MMAs: the ring's space
+    // full[S], empty[S], acc_full[2], acc_empty[2]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOffset);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kStages + 4);
+    float2 *s_part = reinterpret_cast<float2 *>(smem + kBarOffset + 256);              // [2][kSegs][kTC]
+    float *s_hin = reinterpret_cast<float *>(smem + kBarOffset + 256 + 2 * kSegs * kTC * 8);  // [2][kTC]
     const uint32_t ring = smem_addr(smem);
     auto full = [&](int s) { return smem_addr(&bars[s]); };
     auto empty = [&](int s) { return smem_addr(&bars[kStages + s]); };
-    const uint32_t done = smem_addr(&bars[2 * kStages]);
+    auto acc_full = [&](int a) { return smem_addr(&bars[2 * kStages + a]); };
+    auto acc_empty = [&](int a) { return smem_addr(&bars[2 * kStages + 2 + a]); };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t tile = blockIdx.x;
-    const TileCoord tc = tile_coord(p, uint32_t(tile));
-    const int64_t c = tc.c, b = tc.b, ct = tc.dt, chain = tc.chain;
+    const int64_t G = gridDim.x;
+    const int64_t first = blockIdx.x;
+    const int n_local = int((p.n_tiles - first + G - 1) / G);
     const int n_kb = int(pp.d_in / kKB);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2 * kStages + 1; ++i) mbar_init(smem_addr(&bars[i]), 1);
+        for (int i = 0; i < 2 * kStages + 2; ++i) mbar_init(smem_addr(&bars[i]), 1);
+        // each epilogue warp hands the accumulator back once it has read its part
+        for (int i = 2 * kStages + 2; i < 2 * kStages + 4; ++i) mbar_init(smem_addr(&bars[i]), kEpiWarps);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -141,136 +156,179 @@ __global__ void __launch_bounds__(256, 2) mingru_projected_scan_kernel(const Pro
     asm volatile("tcgen05.fence::after_thread_sync;");
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0 && lane == 0) {
-        // producer: x rows [c kTR, c kTR + kTR) of batch row b; W rows
-        // [ct kTC, +kTC) (k) and [D + ct kTC, +kTC) (hx); K in steps of kKB
-        bool ok = true;
-        for (int kb = 0; kb < n_kb && ok; ++kb) {
-            const int s = kb % kStages;
-            if (kb >= kStages && !wait(empty(s), uint32_t((kb / kStages - 1) & 1), kWaitLimit)) {
-                ok = false;
-                break;
+    if (warp == 0) {
+        if (lane == 0) {
+            // producer: for each tile, the W rows of channels [dt kTC, +kTC) in
+            // interleaved groups (group gi of kind k, k = 0 for k rows, 1 for
+            // hx rows, goes to A row (2 gi + k) kGrp) and x rows [c kTR, +kTR)
+            // of batch row b; K in steps of kKB
+            bool ok = true;
+            int64_t g = 0;                               // K steps issued so far
+            for (int n = 0; n < n_local && ok; ++n) {
+                const TileCoord tc = tile_coord(p, uint32_t(first + int64_t(n) * G));
+                const int w_row = int(int64_t(tc.dt) * kTC);
+                for (int kb = 0; kb < n_kb; ++kb, ++g) {
+                    const int s = int(g % kStages);
+                    if (g >= kStages && !wait(empty(s), uint32_t((g / kStages - 1) & 1), kWaitLimit)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = ring + uint32_t(s) * kStageBytes;
+                    mbar_expect_tx(full(s), kStageBytes);
+#pragma unroll
+                    for (int gi = 0; gi < kTC / kGrp; ++gi) {
+                        tma_load_2d(a_dst + uint32_t(2 * gi) * kGrpBytes, &map_w, kb * kKB, w_row + gi * kGrp, full(s));
+                        tma_load_2d(a_dst + uint32_t(2 * gi + 1) * kGrpBytes, &map_w, kb * kKB,
+                                    int(p.D) + w_row + gi * kGrp, full(s));
+                    }
+                    tma_load_3d(a_dst + kABytes, &map_x, kb * kKB, int(tc.c) * kTR, int(tc.b), full(s));
+                }
             }
-            const uint32_t a_dst = ring + uint32_t(s) * kStageBytes;
-            const uint32_t b_dst = a_dst + kABytes;
-            mbar_expect_tx(full(s), kStageBytes);
-            tma_load_3d(a_dst, &map_x, kb * kKB, int(c) * kTR, int(b), full(s));
-            tma_load_2d(b_dst, &map_w, kb * kKB, int(ct) * kTC, full(s));
-            tma_load_2d(b_dst + kBBytes / 2, &map_w, kb * kKB, int(p.D + ct * kTC), full(s));
+            if (!ok) atomicOr(p.status, kTimeoutBit);
+            // a block never leaves with copies in flight: wait (bounded) for the
+            // last stages issued, which the MMA thread also waits for
+            for (int64_t k = g > kStages ? g - kStages : 0; k < g; ++k)
+                wait(full(int(k % kStages)), uint32_t((k / kStages) & 1), kWaitLimit);
         }
-        if (!ok) atomicOr(p.status, kTimeoutBit);
-    } else if (warp == 1 && lane == 0) {
-        // MMA issuer
-        bool ok = true;
-        for (int kb = 0; kb < n_kb; ++kb) {
-            const int s = kb % kStages;
-            if (!wait(full(s), uint32_t((kb / kStages) & 1), kWaitLimit)) {
-                ok = false;
-                break;
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // MMA issuer: tile n into accumulator n & 1 once the epilogue has read it
+            bool ok = true;
+            int64_t g = 0;
+            for (int n = 0; n < n_local && ok; ++n) {
+                const int a = n & 1;
+                if (n >= 2 && !wait(acc_empty(a), uint32_t((n / 2 - 1) & 1), kWaitLimit)) {
+                    ok = false;
+                    break;
+                }
+                asm volatile("tcgen05.fence::after_thread_sync;");
+                const uint32_t acc = tmem + uint32_t(a) * kAccCols;
+                for (int kb = 0; kb < n_kb; ++kb, ++g) {
+                    const int s = int(g % kStages);
+                    if (!wait(full(s), uint32_t((g / kStages) & 1), kWaitLimit)) {
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;");
+                    const uint32_t a_addr = ring + uint32_t(s) * kStageBytes;
+                    const uint64_t da = sw128_desc(a_addr), db = sw128_desc(a_addr + kABytes);
+#pragma unroll
+                    for (int kk = 0; kk < kKB / 16; ++kk) {
+                        const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
+                        asm volatile(
+                            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                            ::"r"(acc), "l"(da + uint64_t(kk * 2)), "l"(db + uint64_t(kk * 2)), "r"(kIdesc),
+                              "r"(accumulate));
+                    }
+                    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                                 ::"r"(empty(s)) : "memory");
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                             ::"r"(acc_full(a)) : "memory");
             }
+            if (!ok) atomicOr(p.status, kTimeoutBit);
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // the carry warp: for each tile, the chunk hand-off of the scan engine
+        // (publish the summary, look back, publish the state) for the tile's
+        // channels, CV per lane, from the epilogue's segment folds
+        constexpr uint32_t NE = kEpiWarps * 32;
+        const int cl = lane * CV;
+        for (int n = 0; n < n_local; ++n) {
+            const int64_t tile = first + int64_t(n) * G;
+            const TileCoord tc = tile_coord(p, uint32_t(tile));
+            const int64_t c = tc.c, b = tc.b, dt = tc.dt, chain = tc.chain;
+            const float2 *part = s_part + (n & 1) * kSegs * kTC;
+            float *hin_s = s_hin + (n & 1) * kTC;
+            named_barrier_sync(1, NE + 32);
+            float2 total[CV];
+#pragma unroll
+            for (int v = 0; v < CV; ++v) {
+                total[v] = part[cl + v];
+#pragma unroll
+                for (int sg = 1; sg < kSegs; ++sg) total[v] = Op::combine(total[v], part[sg * kTC + cl + v]);
+            }
+            const bool publish = (p.n_chunks > 1) && (int64_t(c) < p.n_chunks - 1) && (tile != p.drop_tile);
+            const int64_t dl = dt * kTC + cl;
+            float hin[CV];
+            if (c == 0) {
+#pragma unroll
+                for (int v = 0; v < CV; ++v) hin[v] = load_init<float>(p, b, dl + v, Op::default_init());
+            } else {
+                if (publish) publish_summary<CV, kTC>(p, tile, cl, total);
+                look_back<Op, float, CV, kTC>(p, c, chain, b, dl, cl, hin);
+            }
+#pragma unroll
+            for (int v = 0; v < CV; ++v) hin_s[cl + v] = hin[v];
+            __syncwarp();
+            named_barrier_arrive(2, NE + 32);
+            if (publish) {
+                float fin[CV];
+#pragma unroll
+                for (int v = 0; v < CV; ++v) fin[v] = Op::apply(total[v], hin[v]);
+                publish_state<CV, kTC>(p, tile, cl, fin);
+            }
+        }
+    } else if (warp >= 4) {
+        // epilogue
+        constexpr uint32_t NE = kEpiWarps * 32;
+        const int q = warp & 3;                      // lane quarter: channels 16q .. 16q+15
+        const int cg = (warp - 4) >> 2;              // column group: tokens 64 cg .. 64 cg + 63
+        const bool hx_lane = lane >= 16;             // this lane reads hx (else k)
+        const int ch = q * kGrp + (lane & 15);       // channel within the tile
+        const int seg = 2 * cg + (hx_lane ? 1 : 0);  // 32-token segment this thread scans
+        const int tok0 = seg * 32;
+        for (int n = 0; n < n_local; ++n) {
+            const int64_t tile = first + int64_t(n) * G;
+            const TileCoord tc = tile_coord(p, uint32_t(tile));
+            const int64_t c = tc.c, b = tc.b, dt = tc.dt;
+            const int a = n & 1;
+            float2 *part = s_part + a * kSegs * kTC;
+            float *hin_s = s_hin + a * kTC;
+            if (!wait(acc_full(a), uint32_t((n / 2) & 1), kWaitLimit)) atomicOr(p.status, kTimeoutBit);
+            __syncwarp();                            // tensor-memory loads are warp-collective
             asm volatile("tcgen05.fence::after_thread_sync;");
-            const uint32_t a_addr = ring + uint32_t(s) * kStageBytes;
-            const uint64_t da = sw128_desc(a_addr), db = sw128_desc(a_addr + kABytes);
+            uint32_t r0[32], r1[32];
+            const uint32_t taddr = tmem + (uint32_t(q * 32) << 16) + uint32_t(a) * kAccCols + uint32_t(cg * 64);
+            tmem_ld32(taddr, r0);
+            tmem_ld32(taddr + 32, r1);
+            tmem_wait();
+            asm volatile("tcgen05.fence::before_thread_sync;");
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty(a)) : "memory");
+
+            // k lanes keep columns 0-31 of the group and take hx of them from the
+            // partner lane; hx lanes keep columns 32-63 and take k of them
+            const int rows = int(p.T - c * kTR < kTR ? p.T - c * kTR : kTR);
+            float av[32], bv[32];
+            float2 fold = Op::identity();
 #pragma unroll
-            for (int kk = 0; kk < kKB / 16; ++kk) {
-                const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-                asm volatile(
-                    "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                    "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                    ::"r"(tmem), "l"(da + uint64_t(kk * 2)), "l"(db + uint64_t(kk * 2)), "r"(kIdesc), "r"(acc));
+            for (int i = 0; i < 32; ++i) {
+                const float sent = __uint_as_float(hx_lane ? r0[i] : r1[i]);
+                const float got = __shfl_xor_sync(0xffffffffu, sent, 16);
+                const float kv = hx_lane ? got : __uint_as_float(r0[i]);
+                const float hv = hx_lane ? __uint_as_float(r1[i]) : got;
+                float x = 1.f, y = 0.f;              // tokens past T: the identity pair
+                if (tok0 + i < rows) Op::element(kv, hv, x, y);
+                av[i] = x;
+                bv[i] = y;
+                fold = Op::combine(fold, make_float2(x, y));
             }
-            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                         ::"r"(empty(s)) : "memory");
-        }
-        if (!ok) atomicOr(p.status, kTimeoutBit);
-        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                     ::"r"(done) : "memory");
-    }
-    __syncwarp();        // lanes 1-31 of warps 0 and 1 wait here for their lane 0's role
-    {
-        // epilogue, all 8 warps (the producer and MMA threads have issued
-        // everything by now).  Warp w reads tensor-memory lane quarter w % 4
-        // (token rows 32 (w % 4) ..) and, of each half of the channels, the
-        // 32 columns w / 4.
-        constexpr uint32_t NE = 256;
-        const int q = warp & 3;
-        const int cs = warp >> 2;
-        const int r = q * 32 + lane;                 // this thread's token row
-        const int64_t t = c * kTR + r;
-        if (!wait(done, 0, kWaitLimit)) atomicOr(p.status, kTimeoutBit);
-        __syncwarp();    // tensor-memory loads are warp-collective
-        asm volatile("tcgen05.fence::after_thread_sync;");
-        // every TMA load has landed and every MMA has read its operands: the
-        // ring's space now holds the pairs, one half of the channels at a time
-        const bool valid = t < p.T;
-        const int ch = threadIdx.x & (kHalf - 1);    // fold and replay: channel of the half ...
-        const int rq = threadIdx.x / kHalf;          // ... and quarter of the rows
-        const int rows = int(p.T - c * kTR < kTR ? p.T - c * kTR : kTR);
-#pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {
-            {
-                // k and hx of 32 channels of this row: both loads in flight, one wait
-                uint32_t kv[32], hv[32];
-                tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(hf * kHalf + cs * 32), kv);
-                tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(kTC + hf * kHalf + cs * 32), hv);
-                tmem_wait();
+            part[seg * kTC + ch] = fold;
+            named_barrier_arrive(1, NE + 32);        // the folds are in shared memory
+            named_barrier_sync(2, NE + 32);          // the carry warp has written the states
+            // replay this thread's tokens from the state before them and store h
+            float st = hin_s[ch];
+            for (int sg = 0; sg < seg; ++sg) st = Op::apply(part[sg * kTC + ch], st);
+            float *out = static_cast<float *>(p.out) + (b * p.T + c * kTR + tok0) * p.D + dt * kTC + ch;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    float a = 1.f, bb = 0.f;         // rows past T: the identity pair
-                    if (valid) Op::element(__uint_as_float(kv[i]), __uint_as_float(hv[i]), a, bb);
-                    pairs[pair_slot(r, cs * 32 + i)] = make_float2(a, bb);
-                }
+            for (int i = 0; i < 32; ++i) {
+                st = Op::step(av[i], bv[i], st);
+                if (tok0 + i < rows) __stcs(out + int64_t(i) * p.D, st);
             }
-            named_barrier_sync(1, NE);
-            // fold this thread's 32 rows of its channel
-            float2 part = Op::identity();
-#pragma unroll 8
-            for (int rr = rq * 32; rr < rq * 32 + 32; ++rr) part = Op::combine(part, pairs[pair_slot(rr, ch)]);
-            s_part[rq * kHalf + ch] = part;
-            named_barrier_sync(2, NE);
-            if (warp == 0) {
-                // the chunk hand-off (scan engine): publish the summary, look back, publish the state
-                const int cl = lane * CV;                 // channel within the half
-                const int ct_ch = hf * kHalf + cl;        // channel within the tile
-                float2 total[CV];
-#pragma unroll
-                for (int v = 0; v < CV; ++v) {
-                    total[v] = s_part[cl + v];
-#pragma unroll
-                    for (int qq = 1; qq < 4; ++qq) total[v] = Op::combine(total[v], s_part[qq * kHalf + cl + v]);
-                }
-                const bool publish = (p.n_chunks > 1) && (c < p.n_chunks - 1) && (tile != p.drop_tile);
-                const int64_t dl = ct * kTC + ct_ch;
-                float hin[CV];
-                if (c == 0) {
-#pragma unroll
-                    for (int v = 0; v < CV; ++v) hin[v] = load_init<float>(p, b, dl + v, Op::default_init());
-                } else {
-                    if (publish) publish_summary<CV, kTC>(p, tile, ct_ch, total);
-                    look_back<Op, float, CV, kTC>(p, c, chain, b, dl, ct_ch, hin);
-                }
-#pragma unroll
-                for (int v = 0; v < CV; ++v) s_hin[cl + v] = hin[v];
-                if (publish) {
-                    float fin[CV];
-#pragma unroll
-                    for (int v = 0; v < CV; ++v) fin[v] = Op::apply(total[v], hin[v]);
-                    publish_state<CV, kTC>(p, tile, ct_ch, fin);
-                }
-            }
-            named_barrier_sync(3, NE);
-            // replay the channel's rows from their incoming state and store h
-            float st = s_hin[ch];
-            for (int qq = 0; qq < rq; ++qq) st = Op::apply(s_part[qq * kHalf + ch], st);
-            float *out = static_cast<float *>(p.out) + (b * p.T + c * kTR) * p.D + ct * kTC + hf * kHalf + ch;
-            const int r1 = rq * 32 + 32 < rows ? rq * 32 + 32 : rows;
-#pragma unroll 4
-            for (int rr = rq * 32; rr < r1; ++rr) {
-                const float2 pr = pairs[pair_slot(rr, ch)];
-                st = Op::step(pr.x, pr.y, st);
-                __stcs(out + int64_t(rr) * p.D, st);
-            }
-            named_barrier_sync(1, NE);                   // the buffer is free for the next half
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;");

@@ -698,7 +698,7 @@ sgr_status_t run_projected_scan(const void *x, const void *w, const float *h0, i
     {
         const cuuint64_t dims[2] = {cuuint64_t(d_in), cuuint64_t(2 * D)};
         const cuuint64_t strides[1] = {cuuint64_t(d_in) * 2};
-        const cuuint32_t box[2] = {cuuint32_t(proj::kKB), cuuint32_t(proj::kTC)};
+        const cuuint32_t box[2] = {cuuint32_t(proj::kKB), cuuint32_t(proj::kGrp)};
         const cuuint32_t es[2] = {1u, 1u};
         if (enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(w), dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -713,16 +713,38 @@ sgr_status_t run_projected_scan(const void *x, const void *w, const float *h0, i
     } else {
         sp.epoch = next_epoch();
     }
-    static std::atomic<int> attr_set[64];
+    // persistent blocks, as many as are resident at once (one per SM: the
+    // block holds all 512 tensor-memory columns), launched cooperatively so
+    // that every look-back waits for a block that is running
+    static std::atomic<int> occ_cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SGR_ERR_CUDA;
-    if (dev < 0 || dev >= 64 || attr_set[dev].load() == 0) {
+    int occ = (dev >= 0 && dev < 64) ? occ_cache[dev].load() : 0;
+    if (occ == 0) {
         if (cudaFuncSetAttribute(mingru_projected_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(proj::kSmemBytes)) != cudaSuccess)
             return SGR_ERR_CUDA;
-        if (dev >= 0 && dev < 64) attr_set[dev].store(1);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, mingru_projected_scan_kernel, proj::kThreads,
+                                                          proj::kSmemBytes) != cudaSuccess)
+            return SGR_ERR_CUDA;
+        if (occ <= 0) return SGR_ERR_UNSUPPORTED;
+        occ = 1;                                       // tensor memory: one block per SM whatever fits
+        if (dev >= 0 && dev < 64) occ_cache[dev].store(occ);
     }
-    mingru_projected_scan_kernel<<<unsigned(n_tiles), 256, proj::kSmemBytes, stream>>>(pp, map_x, map_w);
+    const DeviceInfo di = device_info(dev);
+    if (di.sms <= 0) return SGR_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(std::min<int64_t>(n_tiles, int64_t(di.sms) * occ)));
+    cfg.blockDim = dim3(proj::kThreads);
+    cfg.dynamicSmemBytes = proj::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, mingru_projected_scan_kernel, pp, map_x, map_w) != cudaSuccess)
+        return SGR_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
 }
 

@@ -256,7 +256,7 @@ def mingru_projected_scan(x: torch.Tensor, w: torch.Tensor, h0: Optional[torch.T
                           workspace: Optional[Workspace] = None) -> torch.Tensor:
     """h (B, T, D) float32 = minGRU scan of k = x w[:D]^T, hx = x w[D:]^T, with
     the projection on the tensor cores in the same kernel (x (B, T, d_in) and
-    w (2 D, d_in) bfloat16; D % 128 == 0, d_in % 64 == 0)."""
+    w (2 D, d_in) bfloat16; D % 64 == 0, d_in % 64 == 0)."""
     fn = "mingru_projected_scan"
     _seq(x, fn + ": x")
     _need_cuda(w, fn + ": w")

@@ -37,7 +37,12 @@ def data(B, T, D, d_in, seed, with_h0=True):
 
 
 @pytest.mark.parametrize("shape", [(2, 300, 128, 64), (1, 1000, 256, 128), (3, 129, 128, 256),
-                                   (1, 1, 128, 64), (2, 2049, 256, 512), (4, 128, 384, 64)])
+                                   (1, 1, 128, 64), (2, 2049, 256, 512), (4, 128, 384, 64),
+                                   # more tiles than SMs: each persistent block takes several,
+                                   # both accumulators and the operand ring wrap around
+                                   (4, 4096, 256, 64), (2, 8191, 512, 128),
+                                   # channel counts that are odd multiples of the 64-channel tile
+                                   (3, 700, 64, 64), (2, 513, 192, 128)])
 @pytest.mark.parametrize("with_h0", [False, True])
 def test_projected_scan_matches_oracle(shape, with_h0):
     x, w, h0 = data(*shape, seed=sum(shape) % 97, with_h0=with_h0)
@@ -101,3 +106,23 @@ def test_projected_scan_graph_capture():
             graph.replay()
         s.synchronize()
     assert rel_err(out, oracle.mingru_projected(x, w, h0)) <= TOL_PROJ
+
+
+def test_projected_scan_full_size_sampled_chains():
+    """At the 8 x 4096 tokens x 1024 channels, d_in 1024 layer (2048 tiles,
+    about 14 per persistent block), whole chains of sampled (batch row,
+    channel) pairs against the oracle run on just those weight rows."""
+    B, T, D, d_in = 8, 4096, 1024, 1024
+    g = torch.Generator(device=DEV).manual_seed(11)
+    X = torch.randn(B, T, d_in, device=DEV, generator=g).to(torch.bfloat16)
+    W = (torch.randn(2 * D, d_in, device=DEV, generator=g) / d_in ** 0.5).to(torch.bfloat16)
+    H0 = torch.rand(B, D, device=DEV, generator=g) * 0.9 + 0.1
+    h = sgr.mingru_projected_scan(X, W, H0)
+    torch.cuda.synchronize()
+    x, w, h0, hc = X.cpu(), W.cpu(), H0.cpu(), h.cpu()
+    rng = np.random.default_rng(12)
+    chans = np.concatenate([[0, 127, 128, D - 1], rng.choice(D, 12, replace=False)])
+    for b in (0, 3, B - 1):
+        rows = np.concatenate([chans, D + chans])
+        ref = oracle.mingru_projected(x[b:b + 1], w[rows], h0[b:b + 1, chans], threads=8)
+        assert rel_err(hc[b:b + 1, :, chans], ref) <= TOL_PROJ
