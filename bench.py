@@ -55,6 +55,7 @@ FALLBACK_HBM_GBS = 6650.0
 _ENGINE = "scan_gated_rnns_b200/csrc/scan_engine.cuh"
 KERNEL_SOURCES = {
     "scan_kernel": [_ENGINE],
+    "scan_sequential_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_sequential.cuh"],
     "scan_backward_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_backward.cuh"],
     "mingru_projected_scan_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/projected_scan.cuh"],
 }
@@ -263,6 +264,12 @@ def scan_fn(w, p, q, init, out, ws):
     return lambda: f(p, q, init, out=out, workspace=ws)
 
 
+def plan_kernel(plan) -> str:
+    """The device kernel a scan plan launches (the library's kernel kinds)."""
+    return {1: "sgr::scan_tile_kernel", 2: "sgr::scan_pipelined_kernel", 3: "sgr::scan_pipelined_kernel",
+            4: "sgr::scan_sequential_kernel"}.get(plan["kernel"], "sgr::scan_kernel")
+
+
 def measure_row(w, device, steps=10, warmup=3):
     """One other hot-path row, timed alone (inputs larger than L2 except the
     small shape, which is launch-latency bound)."""
@@ -284,7 +291,7 @@ def measure_row(w, device, steps=10, warmup=3):
     row = {"op": f"{w.op}_scan", "B": w.B, "T": w.T, "D": w.D, "io_dtype": w.dtype,
            "us_per_launch": round(per * 1e6, 2), "gbs": round(gbs, 1),
            "gelem_per_s": round(w.n_elems / per / 1e9, 2), "roofline_frac": round(gbs / peak, 4),
-           "bytes_per_launch": bytes_,
+           "bytes_per_launch": bytes_, "kernel": plan_kernel(plan),
            "tile": f"{plan['tile_rows']}x{plan['tile_channels']}", "n_tiles": plan["n_tiles"]}
     if bytes_ < 64 << 20:
         # fits in L2 and is over in microseconds: the host's call overhead shows in
@@ -527,7 +534,12 @@ def run_b200(args):
     fn = scan_fn(w, p, q, init, out, ws)
     stream = torch.cuda.current_stream(device)
     bytes_step = w.algorithmic_bytes()
+    # the chunked kernels' profiles are filed as scan_kernel; the channel-
+    # sequential kernel (wide batches) under its own name
     kernel_name = "sgr::scan_kernel"
+    if sgr._abi.plan(0 if w.op == "mingru" else 1, w.B, w.T, w.D, 0 if w.dtype == "f32" else 1,
+                     True)["kernel"] == 4:
+        kernel_name = "sgr::scan_sequential_kernel"
     if args.pass_ == "projected":
         # the input projection fused with the scan: x (B, T, d_in) and W (2 D, d_in) bf16
         P = PROJECTED

@@ -65,6 +65,11 @@
  *  by two calls that can run at the same time (e.g. on two streams).
  *  Calls may be captured in a CUDA graph; a captured call zero-fills the flag
  *  region itself inside the graph.
+ *  Wide batches (B x D large enough that groups of 32 channels give every SM
+ *  several warps) are not cut along T at all: each warp scans its 32 channels
+ *  over the whole sequence, and sgr_workspace_size() returns 0.
+ *  A workspace passed to such a call anyway (>= 4 bytes, 16-byte aligned)
+ *  receives the status word of its bounded waits.
  */
 #ifndef SCAN_GATED_RNNS_H
 #define SCAN_GATED_RNNS_H
@@ -418,11 +423,13 @@ SGR_API const char *sgr_version(void);
 SGR_API sgr_status_t sgr_set_tile_override(int channel_lanes, int rows_per_thread);
 
 /*
- * Tuning/testing knob, process-wide: 0 automatic (pipelined kernel for
- * aligned vector-width rows, tile kernel otherwise), 1 force the tile kernel,
- * 2 pipelined with 7 data warps per block (two blocks per SM), 3 pipelined
- * with 15 data warps (one block per SM, tiles twice as long), both wherever
- * the fast path applies.
+ * Tuning/testing knob, process-wide: 0 automatic (for aligned vector-width
+ * rows: the channel-sequential kernel when B x ceil(D / 32) reaches 6 (fp32)
+ * or 9 (bf16) warps per SM, the pipelined kernel otherwise; the tile kernel
+ * for anything else), 1 force the tile kernel, 2 pipelined with 7 data warps
+ * per block (two blocks per SM), 3 pipelined with 15 data warps (one block per
+ * SM, tiles twice as long), 4 channel-sequential (one warp walks the whole
+ * sequence of a group of 32 channels), 2-4 wherever the fast path applies.
  */
 SGR_API sgr_status_t sgr_set_kernel_override(int kernel);
 
@@ -432,7 +439,10 @@ SGR_API sgr_status_t sgr_set_kernel_override(int kernel);
 typedef struct sgr_plan {
     int32_t vector_path;        /* 1: 128-bit loads; 0: scalar variant            */
     int32_t kernel;             /* 1: one block per tile; 2: pipelined persistent,
-                                   7 data warps; 3: pipelined, 15 data warps       */
+                                   7 data warps; 3: pipelined, 15 data warps;
+                                   4: channel-sequential, one warp per channel
+                                   group and the whole of T (one chunk; warps =
+                                   warps per block, stages = load-ring slots)   */
     int32_t channels_per_thread;
     int32_t channel_lanes;      /* lanes across D per warp                         */
     int32_t rows_per_thread;

@@ -90,6 +90,7 @@ SIGNATURES.update({
 KERNEL_TILE = 1
 KERNEL_PIPELINED = 2
 KERNEL_PIPELINED_WIDE = 3
+KERNEL_SEQUENTIAL = 4
 
 _lock = threading.Lock()
 _lib = None

@@ -875,7 +875,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
             base[SB] = (int64_t(tc.b) * p.T) * p.D + d0;
             if (!mbar_wait(bars + 8u * uint32_t(n % S), uint32_t((n / S) & 1), wait_limit)) {
                 wait_limit = 1;
-                if (lane == 0) atomicOr(p.status, kTimeoutBit);
+                if (lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);   // null: one chunk, no workspace
             }
             const IO *t0 = reinterpret_cast<const IO *>(smem + (n % S) * Shape::slot_bytes) +
                            ((warp * J + j) * R) * TC + g * V;

@@ -1,0 +1,198 @@
+// scan_sequential.cuh -- channel-sequential scan for wide batches, sm_100a.
+//
+// When a scan has enough channels (B x D) to give every SM several warps, the
+// time axis needs no splitting at all: each warp takes a group of channels of
+// one batch row and walks t = 0 .. T-1 in order, applying each step's map to
+// the state it holds in registers,
+//   minGRU (page "Mingru Pytorch", log-space minGRU): h <- a_t h + b_t,
+//       a_t = 1 - z_t = sigmoid(-k_t), b_t = z_t g(hx_t);
+//   MinMax neuron (page "MinMax Recurrent Neural Cascades", The model, item 3):
+//       x <- max(min(x, r_t), s_t).
+// This is the chunked scan with one chunk per channel: there is no fold of a
+// chunk into a summary pair, no carry between blocks and no replay, so per
+// element the work is the activations and one step.  The parallel (chunked)
+// kernels in scan_engine.cuh remain for shapes with fewer channels, where the
+// time axis has to be cut to fill the GPU.
+//
+// Layout per warp: a channel group of 32 channels (a 128-byte fp32 or 64-byte
+// bf16 row segment per operand), lane l owning channel l of the group.  The
+// warp streams its rows through a ring of S slots of
+// RB rows in shared memory, both operands of a slot loaded by the tensor
+// memory accelerator (one box of CW channels x RB rows per operand, completion
+// counted on the slot's mbarrier; no multicast); lane 0 refills a slot as soon
+// as the warp has copied it into registers.  Outputs go through two staging
+// buffers of RB rows and leave by tensor-memory-accelerator stores (a bulk
+// group per slot), so no thread computes an output address.  Every warp is
+// independent: no block-wide barrier after set-up.  Rows past T and channels
+// past D are zero-filled on load and clipped on store.
+#pragma once
+
+#include "scan_engine.cuh"
+
+namespace sgr {
+
+constexpr int kSeqRows = 16;          // rows per slot
+constexpr int kSeqOutBufs = 2;
+
+// one channel per lane: a warp's channel group is 32 channels, a 128-byte
+// (fp32) or 64-byte (bf16) row segment per operand.  (Two bf16 channels per
+// lane halve the warps a batch provides; the warps' latency, not their issue
+// rate, bounds this kernel, and 32-channel groups measured 13-40% faster.)
+template <typename IO> constexpr int seq_row_bytes() { return 32 * int(sizeof(IO)); }
+
+// bytes of one warp's shared memory with S load slots of rows of `row_bytes`
+__host__ __device__ constexpr size_t seq_warp_bytes(int S, int row_bytes) {
+    return (size_t(S) * 2 * kSeqRows * row_bytes + size_t(kSeqOutBufs) * kSeqRows * row_bytes +
+            size_t(S) * 8 + 127) / 128 * 128;
+}
+
+// a lane's element of one row in shared memory, widened to / narrowed from fp32
+template <typename IO> struct LaneRow;
+template <> struct LaneRow<float> {
+    static __device__ __forceinline__ float load(uint32_t a) {
+        uint32_t v;
+        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+        return __uint_as_float(v);
+    }
+    static __device__ __forceinline__ void store(uint32_t a, float x) {
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(a), "r"(__float_as_uint(x)) : "memory");
+    }
+};
+template <> struct LaneRow<__nv_bfloat16> {
+    static __device__ __forceinline__ float load(uint32_t a) {
+        uint16_t v;
+        asm volatile("ld.shared.b16 %0, [%1];" : "=h"(v) : "r"(a) : "memory");
+        return __uint_as_float(uint32_t(v) << 16);
+    }
+    static __device__ __forceinline__ void store(uint32_t a, float x) {
+        __nv_bfloat16 h = __float2bfloat16_rn(x);
+        asm volatile("st.shared.b16 [%0], %1;" ::"r"(a), "h"(*reinterpret_cast<uint16_t *>(&h)) : "memory");
+    }
+};
+
+// shared -> global tensor store of one box (a bulk group per call)
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most N of this thread's bulk groups still reading shared memory
+template <int N> __device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+struct SeqParams {
+    ScanParams s;        // operands, sizes, initial state, status word (may be null), decay
+    int64_t n_groups;    // channel groups per batch row
+    int64_t n_warps;     // B * n_groups
+    int slots;           // load ring depth S
+};
+
+// Block: WB independent warps; warp (blockIdx.x WB + w) scans channel group
+// (b, grp) of the batch.  Dynamic shared memory: WB x seq_warp_bytes(S).
+template <class Op, typename IO, int WB>
+__global__ void __launch_bounds__(WB * 32)
+scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap map0,
+                       const __grid_constant__ CUtensorMap map1, const __grid_constant__ CUtensorMap map_out) {
+    using LR = LaneRow<IO>;
+    constexpr int CW = 32;
+    constexpr int kRowBytes = seq_row_bytes<IO>();
+    constexpr uint32_t kOpBytes = kSeqRows * kRowBytes;             // one operand of a slot
+    const ScanParams &p = q.s;
+    extern __shared__ __align__(128) unsigned char smem[];
+
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t gw = int64_t(blockIdx.x) * WB + warp;
+    if (gw >= q.n_warps) return;                                     // no block barrier below
+    const int S = q.slots;
+    const int64_t b = gw / q.n_groups;
+    const int64_t grp = gw - b * q.n_groups;
+    const int x0 = int(grp) * CW;                                    // first channel of the group
+    const int64_t d = int64_t(x0) + lane;                            // the lane's channel
+
+    const uint32_t base = smem_addr(smem) + uint32_t(warp * seq_warp_bytes(S, kRowBytes));
+    const uint32_t ring = base;                                      // S slots: [k rows | hx rows]
+    const uint32_t outb = base + uint32_t(S) * 2 * kOpBytes;         // 2 staging buffers
+    const uint32_t bars = outb + kSeqOutBufs * kOpBytes;             // S mbarriers
+
+    const int n_slots = int((p.T + kSeqRows - 1) / kSeqRows);       // T < 2^31 (host check)
+    auto issue = [&](int i, int s) {                                 // lane 0: rows of slot i into ring slot s
+        const uint32_t dst = ring + uint32_t(s) * 2 * kOpBytes;
+        const uint32_t bar = bars + 8u * uint32_t(s);
+        mbar_expect_tx(bar, 2 * kOpBytes);
+        tma_load_3d(dst, &map0, x0, i * kSeqRows, int(b), bar);
+        tma_load_3d(dst + kOpBytes, &map1, x0, i * kSeqRows, int(b), bar);
+    };
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(bars + 8u * s, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int s = 0; s < S && s < n_slots; ++s) issue(s, s);
+    }
+    __syncwarp();
+
+    float h = load_init<IO>(p, b, d, Op::default_init());           // the lane's state
+    [[maybe_unused]] float lam2 = 0.f;
+    if constexpr (Op::kDecay) lam2 = decay_lam2(p, d);
+
+    uint32_t wait_limit = kMbarLimit;
+    bool bad = false;
+    int s = 0;                 // ring slot of slot i
+    uint32_t phase = 0;        // parity of that slot's current use
+    for (int i = 0; i < n_slots; ++i) {
+        if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
+            // a copy that never lands: record it, make every later output NaN
+            // and stop waiting at length (the kernel still ends)
+            wait_limit = 1;
+            if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
+            bad = true;
+        }
+        const uint32_t src = ring + uint32_t(s) * 2 * kOpBytes + uint32_t(lane) * uint32_t(sizeof(IO));
+        float x0r[kSeqRows], x1r[kSeqRows];
+#pragma unroll
+        for (int r = 0; r < kSeqRows; ++r) {
+            x0r[r] = LR::load(src + r * kRowBytes);
+            x1r[r] = LR::load(src + kOpBytes + r * kRowBytes);
+        }
+        // staging buffer i % 2 is free once the store issued two slots ago
+        // has read it (the warp synchronises just below)
+        if (lane == 0) bulk_wait_read<kSeqOutBufs - 1>();
+        __syncwarp();                                                // the slot is in registers
+        if (lane == 0 && !bad && i + S < n_slots) {
+            fence_proxy_async();
+            issue(i + S, s);
+        }
+        if (++s == S) {
+            s = 0;
+            phase ^= 1u;
+        }
+        const uint32_t obuf = outb + uint32_t(i & (kSeqOutBufs - 1)) * kOpBytes;
+        const uint32_t dst = obuf + uint32_t(lane) * uint32_t(sizeof(IO));
+        // each row's step map (independent of the state), then the step
+#pragma unroll
+        for (int r = 0; r < kSeqRows; ++r) {
+            float a, c;
+            Op::element(x0r[r], x1r[r], a, c);
+            if constexpr (Op::kDecay) {
+                const int64_t t = int64_t(i) * kSeqRows + r;
+                a *= decay_gamma(lam2, t < p.T ? decay_u(p, b, t) : 0.f);
+            }
+            h = Op::step(a, c, h);
+            LR::store(dst + r * kRowBytes, bad ? __int_as_float(0x7fffffff) : h);
+        }
+        fence_proxy_async();                                         // outputs visible to the store
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_3d(&map_out, obuf, x0, i * kSeqRows, int(b));
+            bulk_commit();
+        }
+    }
+    if (lane == 0) bulk_wait_all();
+}
+
+}  // namespace sgr

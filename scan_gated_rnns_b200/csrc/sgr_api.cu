@@ -5,6 +5,7 @@
 #include "projected_scan.cuh"
 #include "scan_backward.cuh"
 #include "scan_engine.cuh"
+#include "scan_sequential.cuh"
 
 #include <algorithm>
 #include <atomic>
@@ -28,7 +29,24 @@ constexpr int kAssumedSMs = 148;     // B200; only used to pick a tile shape
 constexpr int64_t kTargetTiles = 4 * 148;  // tile kernel: prefer >= 4 tiles per SM
 constexpr size_t kAlign = 256;
 
-enum Kind { KIND_AUTO = 0, KIND_TILE = 1, KIND_PIPELINED = 2, KIND_PIPELINED_WIDE = 3 };
+enum Kind { KIND_AUTO = 0, KIND_TILE = 1, KIND_PIPELINED = 2, KIND_PIPELINED_WIDE = 3, KIND_SEQUENTIAL = 4 };
+
+// Channel-sequential kernel (scan_sequential.cuh): one warp per 32-channel
+// group walks the whole sequence.  Chosen when the groups alone give every SM
+// at least kSeqMinWarpsPerSM warps (fp32) or kSeqMinWarpsPerSMHalf (bf16:
+// half the bytes per element, so twice the warps for the same bandwidth);
+// below that the time axis is cut into chunks (measured crossovers: fp32
+// between 3.5 and 5.2 warps per SM (noisy near 5), bf16 between 7 and 10.4).  Shared-memory
+// figures are those of sm_100 (228 KB per SM, 1 KB reserved per block, 227 KB
+// per block at most); the launch reads the device's own.
+constexpr int kSeqMinWarpsPerSM = 6;
+constexpr int kSeqMinWarpsPerSMHalf = 9;
+constexpr int kSeqMaxSlots = 8;
+constexpr int kSeqMinSlots = 2;
+constexpr int kSeqWarpsPerBlock = 1;
+constexpr size_t kAssumedSmemPerSM = 233472;
+constexpr size_t kAssumedSmemReserved = 1024;
+constexpr size_t kAssumedSmemPerBlock = 232448;
 
 std::atomic<int> g_override_cg{0};
 std::atomic<int> g_override_r{0};
@@ -121,6 +139,34 @@ bool make_operand_map(CUtensorMap *map, const void *ptr, int64_t B, int64_t T, i
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Shared memory of the channel-sequential kernel.  With K = ceil(groups /
+// SMs) warps per SM in one wave, each single-warp block asks for about 1/K of
+// the SM's shared memory, so no SM can take more than K of them and the
+// groups spread evenly over the SMs (the block scheduler would otherwise be
+// free to stack more on some SMs and leave others short); the share beyond
+// the staging buffers deepens the load ring, up to kSeqMaxSlots slots.  Past
+// 16 warps per SM the work runs in waves and the ring keeps 4 slots.
+struct SeqLayout {
+    int slots = 4;
+    size_t smem = 0;
+};
+SeqLayout seq_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, size_t reserved,
+                     size_t smem_block_max) {
+    SeqLayout l;
+    const int64_t K = sms > 0 ? (groups + sms - 1) / sms : 1;
+    size_t alloc = seq_warp_bytes(4, row_bytes);
+    if (K >= 1 && K <= 16) {
+        const size_t share = smem_sm / size_t(K);
+        alloc = share > reserved ? (share - reserved) / 128 * 128 : 0;
+    }
+    alloc = std::min(alloc, smem_block_max);
+    int S = kSeqMaxSlots;
+    while (S > kSeqMinSlots && seq_warp_bytes(S, row_bytes) > alloc) --S;
+    l.slots = S;
+    l.smem = std::max(alloc, seq_warp_bytes(S, row_bytes));
+    return l;
+}
+
 // Tile shape of a scan.  Aligned vector-width rows take the pipelined kernel
 // (fp32: 7 x 4 x R rows x 32 channels; bf16: 7 x 2 x R rows x 64 channels;
 // 128-byte row segments); anything else takes the tile kernel's scalar
@@ -134,6 +180,34 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
     const int vw = 16 / p.esz;
     p.vec = aligned && (D % vw == 0);
     const int ok = g_override_kind.load();
+    {
+        // whole sequences per warp when the channel groups fill the GPU
+        const int64_t cw = 32;
+        const int64_t groups = B * ((D + cw - 1) / cw);
+        const bool seq_ok = p.vec && !force_tile && T <= int64_t(std::numeric_limits<int>::max()) &&
+                            B <= int64_t(std::numeric_limits<int>::max());
+        const int min_per_sm = p.esz == 2 ? kSeqMinWarpsPerSMHalf : kSeqMinWarpsPerSM;
+        const bool want = ok == KIND_SEQUENTIAL ||
+                          (ok == KIND_AUTO && groups >= int64_t(min_per_sm) * kAssumedSMs);
+        if (seq_ok && want) {
+            const SeqLayout lay = seq_layout(groups, int(cw) * p.esz, kAssumedSMs, kAssumedSmemPerSM,
+                                             kAssumedSmemReserved, kAssumedSmemPerBlock);
+            p.kind = KIND_SEQUENTIAL;
+            p.V = 1;
+            p.cg = 32;
+            p.r = 1;
+            p.stages = lay.slots;
+            p.warps = kSeqWarpsPerBlock;
+            p.TR = T > 0 ? int(std::min<int64_t>(T, std::numeric_limits<int>::max())) : 0;
+            p.TC = int(cw);
+            p.smem = lay.smem;
+            p.n_dt = (D + cw - 1) / cw;
+            p.n_chains = B * p.n_dt;
+            p.n_chunks = T > 0 ? 1 : 0;
+            p.n_tiles = p.n_chains * p.n_chunks;
+            return p;
+        }
+    }
     p.kind = (p.vec && ok != KIND_TILE && !force_tile) ? KIND_PIPELINED : KIND_TILE;
     if (p.kind == KIND_PIPELINED && ok == KIND_AUTO) {
         // under two tiles per persistent block: little to pipeline, and
@@ -327,9 +401,62 @@ cudaError_t launch_pipelined(const ScanParams &sp_in, cudaStream_t s, int64_t *g
     return e;
 }
 
+// ---- channel-sequential kernel launch: one warp per channel group
+template <class Op, typename IO>
+cudaError_t launch_sequential(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
+    constexpr int WB = kSeqWarpsPerBlock;
+    constexpr int CW = 32;
+    constexpr int kRowBytes = seq_row_bytes<IO>();
+    auto kernel = scan_sequential_kernel<Op, IO, WB>;
+    alignas(64) CUtensorMap map0, map1, map_out;
+    if (!make_operand_map(&map0, sp.in0, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
+        !make_operand_map(&map1, sp.in1, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
+        !make_operand_map(&map_out, sp.out, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows))
+        return cudaErrorInvalidValue;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    // per device, once: the shared-memory figures and the kernel's limit
+    struct Dev { int sms, smem_sm, reserved, smem_block; };
+    static std::atomic<int> ready[64];
+    static Dev info[64];
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (ready[dev].load(std::memory_order_acquire) == 0) {
+        Dev d;
+        if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&d.smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) !=
+            cudaSuccess)
+            return e;
+        if ((e = cudaDeviceGetAttribute(&d.reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess)
+            return e;
+        if ((e = cudaDeviceGetAttribute(&d.smem_block, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+            cudaSuccess)
+            return e;
+        if (d.sms <= 0 || d.smem_block < int(seq_warp_bytes(kSeqMinSlots, kRowBytes)))
+            return cudaErrorInvalidConfiguration;
+        if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_block)) !=
+            cudaSuccess)
+            return e;
+        info[dev] = d;
+        ready[dev].store(1, std::memory_order_release);
+    }
+    const Dev d = info[dev];
+    SeqParams q;
+    q.s = sp;
+    q.n_groups = pl.n_dt;
+    q.n_warps = pl.n_chains;
+    const SeqLayout lay = seq_layout((q.n_warps + WB - 1) / WB * WB, kRowBytes, d.sms, size_t(d.smem_sm),
+                                     size_t(d.reserved), size_t(d.smem_block));
+    q.slots = lay.slots;
+    const int64_t grid = (q.n_warps + WB - 1) / WB;
+    kernel<<<dim3(unsigned(grid)), WB * 32, lay.smem, s>>>(q, map0, map1, map_out);
+    return cudaGetLastError();
+}
+
 template <class Op, typename IO>
 cudaError_t dispatch(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
     constexpr int VW = 16 / int(sizeof(IO));
+    if (pl.kind == KIND_SEQUENTIAL) return launch_sequential<Op, IO>(pl, sp, s);
     if (pl.kind == KIND_PIPELINED) {
         if constexpr (sizeof(IO) == 2) {
             if (pl.r == 8) return launch_pipelined<Op, IO, 4, 8, kPipeWarps>(sp, s, nullptr);
@@ -410,6 +537,10 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
     sp.spin_limit = g_spin_limit.load();
     sp.drop_tile = g_drop_tile.load();
     set_decay(sp, dec);
+    if (pl.kind == KIND_SEQUENTIAL && ws && ws_bytes >= sizeof(uint32_t) && aligned16(ws)) {
+        // no hand-off words; a workspace, when given, still receives the status
+        sp.status = static_cast<uint32_t *>(ws);
+    }
     if (pl.n_chunks > 1) {
         if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)) return SGR_ERR_WORKSPACE;
         char *w = static_cast<char *>(ws);
@@ -1012,7 +1143,7 @@ sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dty
     plan->channel_lanes = p.cg;
     plan->rows_per_thread = p.r;
     plan->warps = p.warps;
-    plan->threads = (plan->warps + 1) * 32;
+    plan->threads = (p.kind == KIND_SEQUENTIAL ? plan->warps : plan->warps + 1) * 32;
     plan->stages = p.stages;
     plan->tile_rows = p.TR;
     plan->tile_channels = p.TC;
@@ -1045,7 +1176,7 @@ sgr_status_t sgr_set_drop_publish(int64_t tile) {
 }
 
 sgr_status_t sgr_set_kernel_override(int kernel) {
-    if (kernel < KIND_AUTO || kernel > KIND_PIPELINED_WIDE) return SGR_ERR_INVALID_ARG;
+    if (kernel < KIND_AUTO || kernel > KIND_SEQUENTIAL) return SGR_ERR_INVALID_ARG;
     g_override_kind.store(kernel);
     return SGR_OK;
 }

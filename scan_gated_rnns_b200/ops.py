@@ -111,7 +111,8 @@ def _scan(fn: str, op: int, p: torch.Tensor, q: torch.Tensor, init, out, workspa
             raise ValueError(f"{fn}: out must match the operands")
     need = int(lib().sgr_workspace_size(op, B, T, D, dt))
     wp, wn = 0, 0
-    if need:
+    if need or workspace is not None:
+        # a workspace given where none is needed still receives the status word
         ws = workspace if workspace is not None else default_workspace(p.device, need)
         wp, wn = ws.ptr, ws.nbytes
     with torch.cuda.device(p.device):
@@ -314,7 +315,9 @@ def set_tile_override(channel_lanes: int = 0, rows_per_thread: int = 0) -> None:
 
 
 def set_kernel_override(kernel: int = 0) -> None:
-    """0 automatic, 1 tile kernel, 2 pipelined kernel (where the fast path applies)."""
+    """0 automatic, 1 tile kernel, 2 pipelined kernel, 3 pipelined with 15-warp
+    blocks, 4 channel-sequential kernel (the last three where the fast path
+    applies)."""
     check("sgr_set_kernel_override", lib().sgr_set_kernel_override(kernel))
 
 

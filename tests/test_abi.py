@@ -109,7 +109,7 @@ def test_workspace_size_and_hooks():
     assert lib.sgr_set_tile_override(3, 0) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_tile_override(0, 3) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_drop_publish(-2) == _abi.SGR_ERR_INVALID_ARG
-    assert lib.sgr_set_kernel_override(4) == _abi.SGR_ERR_INVALID_ARG
+    assert lib.sgr_set_kernel_override(5) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_wait_limit(0) == _abi.SGR_OK
     assert lib.sgr_set_drop_publish(-1) == _abi.SGR_OK
     assert lib.sgr_workspace_init(None, 0, None) == _abi.SGR_OK
@@ -120,9 +120,49 @@ def test_workspace_size_and_hooks():
 # ----------------------------------------------------- index arithmetic
 # The kernel's address formulas, replayed for every block and thread.
 
+SEQ_ROWS = 16            # rows per load slot of the channel-sequential kernel
+
+
+def check_sequential_indices(pl, B, T, D, esz, check_cover):
+    """The channel-sequential kernel: warp gw scans channel group gw % n_groups
+    (32 channels) of batch row gw // n_groups over the whole sequence, in slots
+    of 16 rows loaded and stored as tensor-memory-accelerator boxes of 32
+    channels x 16 rows."""
+    V, CW = pl["channels_per_thread"], pl["tile_channels"]
+    rb = CW * esz                                       # bytes of one operand row of a group
+    assert pl["vector_path"] and V == 1 and CW == 32 and rb in (64, 128)
+    assert pl["channel_lanes"] == 32 and pl["threads"] == 32 * pl["warps"]
+    assert pl["n_chunks"] == 1 and pl["workspace_bytes"] == 0 and pl["tile_rows"] == T
+    n_groups = -(-D // CW)
+    assert pl["n_channel_tiles"] == n_groups and pl["n_chains"] == B * n_groups
+    assert pl["n_tiles"] == pl["n_chains"] < 2 ** 31
+    assert 2 <= pl["stages"] <= 8
+    # a warp's ring, staging buffers and mbarriers fit its block's shared memory
+    warp_bytes = -(-(pl["stages"] * 2 * SEQ_ROWS * rb + 2 * SEQ_ROWS * rb + pl["stages"] * 8) // 128) * 128
+    assert warp_bytes * pl["warps"] <= pl["smem_bytes"] <= 227 * 1024
+    assert (D * esz) % 16 == 0 and T < 2 ** 31 and B < 2 ** 31
+    gw = np.arange(pl["n_chains"], dtype=np.int64)
+    b, grp = gw // n_groups, gw % n_groups
+    x0 = grp * CW
+    assert ((x0 * esz) % 16 == 0).all()                 # box x coordinate 16-byte aligned
+    assert (x0 < D).all() and (b < B).all()
+    n_slots = -(-T // SEQ_ROWS)
+    assert n_slots * SEQ_ROWS < 2 ** 31                 # row coordinates are 32-bit
+    if check_cover:
+        # the store boxes, clipped to the tensor, write every element exactly once
+        cover = np.zeros((B, max(T, 1), D), dtype=np.int32)
+        for w in range(len(gw)):
+            for i in range(n_slots):
+                cover[b[w], i * SEQ_ROWS:min(T, (i + 1) * SEQ_ROWS), x0[w]:min(D, x0[w] + CW)] += 1
+        assert (cover[:, :T] == 1).all(), "every output element is written exactly once"
+
+
 def check_plan_indices(B, T, D, dtype, aligned, check_cover):
     pl = _abi.plan(MINGRU, B, T, D, dtype, aligned)
     esz = 4 if dtype == F32 else 2
+    if pl["kernel"] == _abi.KERNEL_SEQUENTIAL:
+        check_sequential_indices(pl, B, T, D, esz, check_cover)
+        return
     V, cg, R, W = pl["channels_per_thread"], pl["channel_lanes"], pl["rows_per_thread"], pl["warps"]
     J = 32 // cg
     TR, TC = pl["tile_rows"], pl["tile_channels"]
@@ -197,7 +237,7 @@ SMALL_SHAPES = [(2, 1024, 512), (3, 1000, 96), (1, 777, 36), (2, 300, 7), (1, 1,
 @pytest.mark.parametrize("aligned", [True, False])
 @pytest.mark.parametrize("override", [(0, 0, 0), (1, 0, 1), (1, 0, 2), (1, 0, 4), (1, 0, 8),
                                       (2, 0, 2), (2, 0, 4), (2, 0, 8), (3, 0, 2), (3, 0, 4),
-                                      (3, 0, 8)])
+                                      (3, 0, 8), (4, 0, 0)])
 def test_plan_indices_small(shape, dtype, aligned, override):
     lib = _abi.lib()
     assert lib.sgr_set_kernel_override(override[0]) == 0
