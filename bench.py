@@ -56,6 +56,8 @@ _ENGINE = "scan_gated_rnns_b200/csrc/scan_engine.cuh"
 KERNEL_SOURCES = {
     "scan_kernel": [_ENGINE],
     "scan_sequential_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_sequential.cuh"],
+    "scan_sequential_backward_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_backward.cuh",
+                                        "scan_gated_rnns_b200/csrc/scan_sequential.cuh"],
     "scan_backward_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_backward.cuh"],
     "mingru_projected_scan_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/projected_scan.cuh"],
 }
@@ -270,6 +272,14 @@ def plan_kernel(plan) -> str:
             4: "sgr::scan_sequential_kernel"}.get(plan["kernel"], "sgr::scan_kernel")
 
 
+def backward_kernel(w) -> str:
+    """The device kernel the gradient of workload w launches."""
+    import scan_gated_rnns_b200 as sgr
+    kind = sgr._abi.lib().sgr_backward_kernel(0 if w.op == "mingru" else 1, w.B, w.T, w.D,
+                                              0 if w.dtype == "f32" else 1, 1)
+    return "sgr::scan_sequential_backward_kernel" if kind == 4 else "sgr::scan_backward_kernel"
+
+
 def measure_row(w, device, steps=10, warmup=3):
     """One other hot-path row, timed alone (inputs larger than L2 except the
     small shape, which is launch-latency bound)."""
@@ -345,7 +355,7 @@ def measure_backward_row(w, device, steps=10, warmup=3):
     return {"op": f"{w.op}_scan_backward", "B": w.B, "T": w.T, "D": w.D, "io_dtype": w.dtype,
             "us_per_launch": round(per * 1e6, 2), "gbs": round(gbs, 1),
             "gelem_per_s": round(w.n_elems / per / 1e9, 2), "roofline_frac": round(gbs / peak, 4),
-            "bytes_per_launch": bytes_, "kernel": "sgr::scan_backward_kernel"}
+            "bytes_per_launch": bytes_, "kernel": backward_kernel(w)}
 
 
 def measure_decay_rows(w, device, steps=10, warmup=3):
@@ -562,7 +572,7 @@ def run_b200(args):
         bwd = sgr.mingru_scan_backward if w.op == "mingru" else sgr.minmax_scan_backward
         fn = lambda: bwd(p, q, init, out, gy, init is not None, workspace=wsb)  # noqa: E731
         bytes_step = 6 * w.n_elems * w.elem_bytes + (2 * w.B * w.D * w.elem_bytes if init is not None else 0)
-        kernel_name = "sgr::scan_backward_kernel"
+        kernel_name = backward_kernel(w)
         ws = wsb
         args.no_e2e = True
 

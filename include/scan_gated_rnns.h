@@ -467,6 +467,14 @@ typedef struct sgr_plan {
 SGR_API sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D,
                                    sgr_dtype_t dtype, int aligned, sgr_plan_t *plan);
 
+/* Which kernel the gradient of this shape runs (mingru_scan_backward,
+ * minmax_scan_backward and their time-decay forms): 1 the chunked tile kernel,
+ * 4 the channel-sequential kernel (wide batches: one warp walks the whole
+ * sequence of 32 channels backwards); 0 for invalid arguments.  `aligned` says
+ * whether all six (B, T, D) operands would be 16-byte aligned.  Pure host code. */
+SGR_API int sgr_backward_kernel(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
+                                int aligned);
+
 /* ------------------------------------------------------- testing hooks */
 
 /*

@@ -66,6 +66,7 @@ SIGNATURES.update({
     "sgr_set_wait_limit": (_int, [ctypes.c_uint32]),
     "sgr_set_drop_publish": (_int, [_i64]),
     "sgr_set_kernel_override": (_int, [_int]),
+    "sgr_backward_kernel": (_int, [_int, _i64, _i64, _i64, _int, _int]),
     "mingru_scan_noalloc": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _i64, _i64, _int, _vp]),
     "sgr_host_staging_size": (_sz, [_int, _i64, _i64, _i64, _int, _int]),
     "mingru_scan_backward": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _i64,

@@ -27,6 +27,7 @@
 // past D are zero-filled on load and clipped on store.
 #pragma once
 
+#include "scan_backward.cuh"
 #include "scan_engine.cuh"
 
 namespace sgr {
@@ -191,6 +192,176 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
             tma_store_3d(&map_out, obuf, x0, i * kSeqRows, int(b));
             bulk_commit();
         }
+    }
+    if (lane == 0) bulk_wait_all();
+}
+
+}  // namespace sgr
+
+// ------------------------------------------------------- gradients
+//
+// The gradient of either scan walks the sequence backwards (scan_backward.cuh
+// states the recurrence): with lam the gradient reaching out_t from the steps
+// after t, delta = gy_t + lam, d in0_t = delta cP_t, d in1_t = delta cQ_t and
+// lam <- A_t delta, where (A_t, cP_t, cQ_t) are the local partials of step t
+// given the state before it (the forward output one row back, or the initial
+// state at t = 0).  For wide batches each warp does this for its 32 channels
+// from t = T - 1 down to 0 with lam in a register -- no reverse chunking, no
+// look-back.  Slots are rows [j RB, j RB + RB) taken for j from the top down
+// (the top one may run past T: those rows are skipped); per slot the copy
+// engine brings four boxes -- k, hx (or r, s), gy, and the forward output
+// shifted one row back (box starting at row j RB - 1; the row before t = 0
+// is read as zero fill and replaced by the initial state) -- and two boxes of
+// input gradients leave by tensor stores, which never start at a negative row.
+namespace sgr {
+
+constexpr int kSeqBwdIn = 4;        // operands loaded per slot
+constexpr int kSeqBwdOut = 2;       // gradients stored per slot
+
+__host__ __device__ constexpr size_t seq_bwd_warp_bytes(int S, int row_bytes) {
+    return (size_t(S) * kSeqBwdIn * kSeqRows * row_bytes +
+            size_t(kSeqOutBufs) * kSeqBwdOut * kSeqRows * row_bytes + size_t(S) * 8 + 127) / 128 * 128;
+}
+
+struct SeqBwdParams {
+    BwdParams g;         // operands, gradients, initial state, status word (may be null), decay
+    int64_t n_groups;    // channel groups per batch row
+    int64_t n_warps;     // B * n_groups
+    int slots;           // load ring depth S
+};
+
+template <class BOp, typename IO, int WB>
+__global__ void __launch_bounds__(WB * 32)
+scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CUtensorMap map_in0,
+                                const __grid_constant__ CUtensorMap map_in1,
+                                const __grid_constant__ CUtensorMap map_gy,
+                                const __grid_constant__ CUtensorMap map_fwd,
+                                const __grid_constant__ CUtensorMap map_d0,
+                                const __grid_constant__ CUtensorMap map_d1) {
+    using LR = LaneRow<IO>;
+    constexpr int CW = 32;
+    constexpr int kRowBytes = seq_row_bytes<IO>();
+    constexpr uint32_t kOpBytes = kSeqRows * kRowBytes;             // one operand of a slot
+    const BwdParams &bp = q.g;
+    const ScanParams &p = bp.s;
+    extern __shared__ __align__(128) unsigned char smem[];
+
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t gw = int64_t(blockIdx.x) * WB + warp;
+    if (gw >= q.n_warps) return;                                     // no block barrier below
+    const int S = q.slots;
+    const int64_t b = gw / q.n_groups;
+    const int64_t grp = gw - b * q.n_groups;
+    const int x0 = int(grp) * CW;
+    const int64_t d = int64_t(x0) + lane;
+
+    const uint32_t base = smem_addr(smem) + uint32_t(warp * seq_bwd_warp_bytes(S, kRowBytes));
+    const uint32_t ring = base;                                      // S slots: [in0 | in1 | gy | fwd]
+    const uint32_t outb = base + uint32_t(S) * kSeqBwdIn * kOpBytes; // 2 x [d in0 | d in1]
+    const uint32_t bars = outb + kSeqOutBufs * kSeqBwdOut * kOpBytes;
+
+    const int n_slots = int((p.T + kSeqRows - 1) / kSeqRows);       // T < 2^31 (host check)
+    // processing slot i covers time rows [j RB, j RB + RB), j = n_slots - 1 - i
+    auto issue = [&](int i, int s) {
+        const int y = (n_slots - 1 - i) * kSeqRows;
+        const uint32_t dst = ring + uint32_t(s) * kSeqBwdIn * kOpBytes;
+        const uint32_t bar = bars + 8u * uint32_t(s);
+        mbar_expect_tx(bar, kSeqBwdIn * kOpBytes);
+        tma_load_3d(dst, &map_in0, x0, y, int(b), bar);
+        tma_load_3d(dst + kOpBytes, &map_in1, x0, y, int(b), bar);
+        tma_load_3d(dst + 2 * kOpBytes, &map_gy, x0, y, int(b), bar);
+        tma_load_3d(dst + 3 * kOpBytes, &map_fwd, x0, y - 1, int(b), bar);   // state before each row
+    };
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(bars + 8u * s, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int s = 0; s < S && s < n_slots; ++s) issue(s, s);
+    }
+    __syncwarp();
+
+    const float h_init =
+        (bp.init && d < p.D) ? load_scalar<IO>(static_cast<const IO *>(bp.init) + b * bp.init_bs + d)
+                             : BOp::default_state();
+    [[maybe_unused]] float lam2 = 0.f, dl = 0.f;
+    if constexpr (BOp::kDecay) lam2 = decay_lam2(p, d);
+
+    float lam = 0.f;           // dL/d (state after the rows still to walk)
+    uint32_t wait_limit = kMbarLimit;
+    bool bad = false;
+    int s = 0;
+    uint32_t phase = 0;
+    for (int i = 0; i < n_slots; ++i) {
+        const int j = n_slots - 1 - i;
+        if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
+            wait_limit = 1;
+            if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
+            bad = true;
+        }
+        const uint32_t src = ring + uint32_t(s) * kSeqBwdIn * kOpBytes + uint32_t(lane) * uint32_t(sizeof(IO));
+        float xk[kSeqRows], xh[kSeqRows], xg[kSeqRows], xf[kSeqRows];
+#pragma unroll
+        for (int r = 0; r < kSeqRows; ++r) {
+            xk[r] = LR::load(src + r * kRowBytes);
+            xh[r] = LR::load(src + kOpBytes + r * kRowBytes);
+            xg[r] = LR::load(src + 2 * kOpBytes + r * kRowBytes);
+            xf[r] = LR::load(src + 3 * kOpBytes + r * kRowBytes);
+        }
+        if (lane == 0) bulk_wait_read<kSeqOutBufs - 1>();            // staging buffers of slot i - 2
+        __syncwarp();
+        if (lane == 0 && !bad && i + S < n_slots) {
+            fence_proxy_async();
+            issue(i + S, s);
+        }
+        if (++s == S) {
+            s = 0;
+            phase ^= 1u;
+        }
+        if (j == 0) xf[0] = h_init;                                  // the state before t = 0
+        const uint32_t obuf = outb + uint32_t(i & (kSeqOutBufs - 1)) * kSeqBwdOut * kOpBytes;
+        const uint32_t dst = obuf + uint32_t(lane) * uint32_t(sizeof(IO));
+        const int valid = int(p.T - int64_t(j) * kSeqRows);         // rows of the slot inside T (>= 1)
+        auto rows = [&](auto fullc) {
+            constexpr bool FULL = decltype(fullc)::value;
+#pragma unroll
+            for (int r = kSeqRows - 1; r >= 0; --r) {
+                float A, cP, cQ;
+                [[maybe_unused]] float u = 0.f;
+                if constexpr (BOp::kDecay) {
+                    const int64_t t = int64_t(j) * kSeqRows + r;
+                    u = t < p.T ? decay_u(p, b, t) : 0.f;
+                    BOp::coeffs_gated(xk[r], xh[r], xf[r], decay_gamma(lam2, u), A, cP, cQ);
+                } else {
+                    BOp::coeffs(xk[r], xh[r], xf[r], A, cP, cQ);
+                }
+                const float delta = xg[r] + lam;
+                float y0 = delta * cP, y1 = delta * cQ;
+                if (FULL || r < valid) {
+                    lam = A * delta;
+                    // dL/dlambda gains delta (1 - z) h_{t-1} dgamma/dlambda = delta A h_{t-1} (-u)
+                    if constexpr (BOp::kDecay) dl = fmaf(delta, -u * A * xf[r], dl);
+                }
+                if (bad) y0 = y1 = __int_as_float(0x7fffffff);
+                LR::store(dst + r * kRowBytes, y0);
+                LR::store(dst + kOpBytes + r * kRowBytes, y1);
+            }
+        };
+        if (valid >= kSeqRows) rows(std::true_type{});
+        else rows(std::false_type{});
+        fence_proxy_async();                                         // gradients visible to the stores
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_3d(&map_d0, obuf, x0, j * kSeqRows, int(b));
+            tma_store_3d(&map_d1, obuf + kOpBytes, x0, j * kSeqRows, int(b));
+            bulk_commit();
+        }
+    }
+    if (bp.dinit && d < p.D) {
+        const float y[1] = {bad ? __int_as_float(0x7fffffff) : lam};
+        Access<IO, 1>::store(static_cast<IO *>(bp.dinit) + b * bp.dinit_bs + d, y);
+    }
+    if constexpr (BOp::kDecay) {
+        if (bp.dlam && d < p.D) atomicAdd(bp.dlam + d, dl);
     }
     if (lane == 0) bulk_wait_all();
 }

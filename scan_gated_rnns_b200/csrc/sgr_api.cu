@@ -12,6 +12,8 @@
 #include <cstring>
 #include <limits>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 namespace {
 
@@ -41,6 +43,11 @@ enum Kind { KIND_AUTO = 0, KIND_TILE = 1, KIND_PIPELINED = 2, KIND_PIPELINED_WID
 // per block at most); the launch reads the device's own.
 constexpr int kSeqMinWarpsPerSM = 6;
 constexpr int kSeqMinWarpsPerSMHalf = 9;
+// The gradient (four operands in, two out per element, where the chunked
+// gradient kernel is a plain tile kernel) gains from 3 warps per SM in both
+// dtypes (measured: fp32 loses at 2.6 and wins at 3.5, bf16 wins at 3.5 and
+// loses at 1.7).
+constexpr int kSeqBwdMinWarpsPerSM = 3;
 constexpr int kSeqMaxSlots = 8;
 constexpr int kSeqMinSlots = 2;
 constexpr int kSeqWarpsPerBlock = 1;
@@ -150,20 +157,23 @@ struct SeqLayout {
     int slots = 4;
     size_t smem = 0;
 };
+size_t seq_bytes(bool backward, int S, int row_bytes) {
+    return backward ? seq_bwd_warp_bytes(S, row_bytes) : seq_warp_bytes(S, row_bytes);
+}
 SeqLayout seq_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, size_t reserved,
-                     size_t smem_block_max) {
+                     size_t smem_block_max, bool backward = false) {
     SeqLayout l;
     const int64_t K = sms > 0 ? (groups + sms - 1) / sms : 1;
-    size_t alloc = seq_warp_bytes(4, row_bytes);
+    size_t alloc = seq_bytes(backward, 4, row_bytes);
     if (K >= 1 && K <= 16) {
         const size_t share = smem_sm / size_t(K);
         alloc = share > reserved ? (share - reserved) / 128 * 128 : 0;
     }
     alloc = std::min(alloc, smem_block_max);
     int S = kSeqMaxSlots;
-    while (S > kSeqMinSlots && seq_warp_bytes(S, row_bytes) > alloc) --S;
+    while (S > kSeqMinSlots && seq_bytes(backward, S, row_bytes) > alloc) --S;
     l.slots = S;
-    l.smem = std::max(alloc, seq_warp_bytes(S, row_bytes));
+    l.smem = std::max(alloc, seq_bytes(backward, S, row_bytes));
     return l;
 }
 
@@ -401,7 +411,48 @@ cudaError_t launch_pipelined(const ScanParams &sp_in, cudaStream_t s, int64_t *g
     return e;
 }
 
-// ---- channel-sequential kernel launch: one warp per channel group
+// ---- channel-sequential kernels: one warp per channel group
+// Per device: SM count and shared-memory figures, read once; and, once per
+// kernel and device, the kernel's dynamic shared-memory limit raised to the
+// device's maximum per block.
+struct SeqDev {
+    int sms = 0, smem_sm = 0, reserved = 0, smem_block = 0;
+};
+cudaError_t seq_device(const void *kernel, size_t min_bytes, SeqDev *out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    static std::mutex mu;
+    static SeqDev info[64];
+    static bool have[64];
+    static std::vector<std::pair<const void *, int>> raised;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!have[dev]) {
+        SeqDev d;
+        if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&d.smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) !=
+            cudaSuccess)
+            return e;
+        if ((e = cudaDeviceGetAttribute(&d.reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess)
+            return e;
+        if ((e = cudaDeviceGetAttribute(&d.smem_block, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+            cudaSuccess)
+            return e;
+        if (d.sms <= 0) return cudaErrorInvalidConfiguration;
+        info[dev] = d;
+        have[dev] = true;
+    }
+    if (size_t(info[dev].smem_block) < min_bytes) return cudaErrorInvalidConfiguration;
+    if (std::find(raised.begin(), raised.end(), std::make_pair(kernel, dev)) == raised.end()) {
+        if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, info[dev].smem_block)) !=
+            cudaSuccess)
+            return e;
+        raised.emplace_back(kernel, dev);
+    }
+    *out = info[dev];
+    return cudaSuccess;
+}
 template <class Op, typename IO>
 cudaError_t launch_sequential(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
     constexpr int WB = kSeqWarpsPerBlock;
@@ -413,34 +464,9 @@ cudaError_t launch_sequential(const Plan &pl, const ScanParams &sp, cudaStream_t
         !make_operand_map(&map1, sp.in1, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
         !make_operand_map(&map_out, sp.out, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows))
         return cudaErrorInvalidValue;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    SeqDev d;
+    cudaError_t e = seq_device(reinterpret_cast<const void *>(kernel), seq_warp_bytes(kSeqMinSlots, kRowBytes), &d);
     if (e != cudaSuccess) return e;
-    // per device, once: the shared-memory figures and the kernel's limit
-    struct Dev { int sms, smem_sm, reserved, smem_block; };
-    static std::atomic<int> ready[64];
-    static Dev info[64];
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (ready[dev].load(std::memory_order_acquire) == 0) {
-        Dev d;
-        if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-        if ((e = cudaDeviceGetAttribute(&d.smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) !=
-            cudaSuccess)
-            return e;
-        if ((e = cudaDeviceGetAttribute(&d.reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess)
-            return e;
-        if ((e = cudaDeviceGetAttribute(&d.smem_block, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
-            cudaSuccess)
-            return e;
-        if (d.sms <= 0 || d.smem_block < int(seq_warp_bytes(kSeqMinSlots, kRowBytes)))
-            return cudaErrorInvalidConfiguration;
-        if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_block)) !=
-            cudaSuccess)
-            return e;
-        info[dev] = d;
-        ready[dev].store(1, std::memory_order_release);
-    }
-    const Dev d = info[dev];
     SeqParams q;
     q.s = sp;
     q.n_groups = pl.n_dt;
@@ -598,6 +624,51 @@ cudaError_t dispatch_bwd_r(const Plan &pl, const BwdParams &bp, cudaStream_t s) 
     }
 }
 
+// ---- channel-sequential gradient launch (wide batches)
+template <class BOp, typename IO>
+cudaError_t launch_sequential_bwd(const BwdParams &bp, cudaStream_t s) {
+    constexpr int WB = kSeqWarpsPerBlock;
+    constexpr int CW = 32;
+    constexpr int kRowBytes = seq_row_bytes<IO>();
+    auto kernel = scan_sequential_backward_kernel<BOp, IO, WB>;
+    const ScanParams &sp = bp.s;
+    const int esz = int(sizeof(IO));
+    alignas(64) CUtensorMap m_in0, m_in1, m_gy, m_fwd, m_d0, m_d1;
+    if (!make_operand_map(&m_in0, sp.in0, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
+        !make_operand_map(&m_in1, sp.in1, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
+        !make_operand_map(&m_gy, bp.gy, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
+        !make_operand_map(&m_fwd, bp.fwd, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
+        !make_operand_map(&m_d0, sp.out, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
+        !make_operand_map(&m_d1, bp.out1, sp.B, sp.T, sp.D, esz, CW, kSeqRows))
+        return cudaErrorInvalidValue;
+    SeqDev d;
+    cudaError_t e = seq_device(reinterpret_cast<const void *>(kernel), seq_bwd_warp_bytes(kSeqMinSlots, kRowBytes), &d);
+    if (e != cudaSuccess) return e;
+    SeqBwdParams q;
+    q.g = bp;
+    q.n_groups = (sp.D + CW - 1) / CW;
+    q.n_warps = sp.B * q.n_groups;
+    const SeqLayout lay = seq_layout((q.n_warps + WB - 1) / WB * WB, kRowBytes, d.sms, size_t(d.smem_sm),
+                                     size_t(d.reserved), size_t(d.smem_block), true);
+    q.slots = lay.slots;
+    const int64_t grid = (q.n_warps + WB - 1) / WB;
+    kernel<<<dim3(unsigned(grid)), WB * 32, lay.smem, s>>>(q, m_in0, m_in1, m_gy, m_fwd, m_d0, m_d1);
+    return cudaGetLastError();
+}
+
+// whether a gradient of this shape walks whole sequences per warp
+bool seq_backward_planned(int64_t B, int64_t T, int64_t D, int esz, bool aligned) {
+    const int vw = 16 / esz;
+    if (!aligned || D % vw != 0 || T > int64_t(std::numeric_limits<int>::max()) ||
+        B > int64_t(std::numeric_limits<int>::max()))
+        return false;
+    const int ok = g_override_kind.load();
+    if (ok == KIND_SEQUENTIAL) return true;
+    if (ok != KIND_AUTO) return false;
+    const int64_t groups = B * ((D + 31) / 32);
+    return groups >= int64_t(kSeqBwdMinWarpsPerSM) * kAssumedSMs;
+}
+
 template <class BOp, typename IO>
 cudaError_t dispatch_bwd(const Plan &pl, const BwdParams &bp, cudaStream_t s) {
     constexpr int VW = 16 / int(sizeof(IO));
@@ -659,8 +730,9 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
 
     const bool aligned = aligned16(in0) && aligned16(in1) && aligned16(fwd) && aligned16(gy) &&
                          aligned16(out0) && aligned16(out1);
+    const bool seq = seq_backward_planned(B, T, D, esz, aligned);
     const Plan pl = make_plan(B, T, D, dtype, aligned, true);
-    if (pl.n_tiles > int64_t(std::numeric_limits<int>::max())) return SGR_ERR_UNSUPPORTED;
+    if (!seq && pl.n_tiles > int64_t(std::numeric_limits<int>::max())) return SGR_ERR_UNSUPPORTED;
 
     BwdParams bp;
     std::memset(&bp, 0, sizeof(bp));
@@ -679,6 +751,25 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
     bp.dlam = dec ? dlam : nullptr;
     if (bp.dlam && overlaps(bp.dlam, size_t(D) * sizeof(float), out0, tb)) return SGR_ERR_INVALID_ARG;
     if (bp.dlam && overlaps(bp.dlam, size_t(D) * sizeof(float), out1, tb)) return SGR_ERR_INVALID_ARG;
+    if (seq) {
+        // one warp per channel group over the whole sequence: no hand-off
+        // words; a workspace, when given, receives the status word
+        if (ws && ws_bytes >= sizeof(uint32_t) && aligned16(ws)) sp.status = static_cast<uint32_t *>(ws);
+        if (bp.dlam && cudaMemsetAsync(bp.dlam, 0, size_t(D) * sizeof(float), stream) != cudaSuccess)
+            return SGR_ERR_CUDA;
+        cudaError_t e;
+        if (op == SGR_OP_MINGRU && dec) {
+            e = dtype == SGR_F32 ? launch_sequential_bwd<MinGRUDecayBwd, float>(bp, stream)
+                                 : launch_sequential_bwd<MinGRUDecayBwd, __nv_bfloat16>(bp, stream);
+        } else if (op == SGR_OP_MINGRU) {
+            e = dtype == SGR_F32 ? launch_sequential_bwd<MinGRUBwd, float>(bp, stream)
+                                 : launch_sequential_bwd<MinGRUBwd, __nv_bfloat16>(bp, stream);
+        } else {
+            e = dtype == SGR_F32 ? launch_sequential_bwd<MinMaxBwd, float>(bp, stream)
+                                 : launch_sequential_bwd<MinMaxBwd, __nv_bfloat16>(bp, stream);
+        }
+        return e == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
+    }
     if (pl.n_chunks > 1) {
         if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)) return SGR_ERR_WORKSPACE;
         char *w = static_cast<char *>(ws);
@@ -1162,6 +1253,13 @@ sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dty
         plan->div_chains_m = plan->div_chains_s = plan->div_dt_m = plan->div_dt_s = 0;
     }
     return SGR_OK;
+}
+
+int sgr_backward_kernel(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, int aligned) {
+    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return 0;
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return 0;
+    if (B < 0 || T < 0 || D < 0) return 0;
+    return seq_backward_planned(B, T, D, dtype == SGR_BF16 ? 2 : 4, aligned != 0) ? KIND_SEQUENTIAL : KIND_TILE;
 }
 
 sgr_status_t sgr_set_wait_limit(uint32_t polls) {

@@ -446,3 +446,24 @@ def test_projected_scan_argument_errors():
     assert call(wn=lib.sgr_projected_workspace_size(2, 10, 128) - 1) == _abi.SGR_ERR_WORKSPACE
     assert call(B=0) == _abi.SGR_OK
     assert lib.sgr_projected_workspace_size(2, 10, 96) == 0
+
+
+def test_backward_kernel_choice():
+    """The gradient walks whole sequences per warp (kernel 4) from 3 warps of
+    32 channels per SM, on aligned vector-width rows; otherwise the tile
+    kernel (1)."""
+    lib = _abi.lib()
+    assert lib.sgr_backward_kernel(MINGRU, 16, 2048, 4096, BF16, 1) == 4     # 2048 groups
+    assert lib.sgr_backward_kernel(MINGRU, 4, 2048, 4096, BF16, 1) == 4      # 512 groups
+    assert lib.sgr_backward_kernel(MINGRU, 2, 2048, 4096, BF16, 1) == 1      # 256 groups
+    assert lib.sgr_backward_kernel(MINGRU, 8, 4096, 1024, F32, 1) == 1       # 256 groups
+    assert lib.sgr_backward_kernel(MINGRU, 16, 2048, 4096, BF16, 0) == 1     # unaligned
+    assert lib.sgr_backward_kernel(MINGRU, 16, 2048, 4100, BF16, 1) == 1     # D not a vector multiple
+    assert lib.sgr_backward_kernel(9, 16, 2048, 4096, BF16, 1) == 0
+    assert lib.sgr_set_kernel_override(4) == 0
+    try:
+        assert lib.sgr_backward_kernel(MINGRU, 1, 10, 32, F32, 1) == 4
+        assert lib.sgr_backward_kernel(MINGRU, 1, 10, 36, F32, 1) == 4       # partial group, aligned rows
+        assert lib.sgr_backward_kernel(MINGRU, 1, 10, 6, F32, 1) == 1        # rows not 16-byte multiples
+    finally:
+        lib.sgr_set_kernel_override(0)
