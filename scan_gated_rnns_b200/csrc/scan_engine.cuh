@@ -100,6 +100,30 @@ struct MinGRUOp {
         const float g = (hx >= 0.f) ? hx + 0.5f : sg.y;
         b = z * g;
     }
+    // The pairs of two steps (rows) of one channel, each fp32x2 operation
+    // packed across the two steps: two independent dependency chains per
+    // instruction stream, and the same values as element() except that
+    // g(hx) = max(hx + 0.5, sigmoid(hx)), which holds for every hx
+    // (hx + 0.5 - sigmoid(hx) is increasing and 0 at hx = 0; where hx < 0,
+    // sigmoid(hx) = sigmoid(-|hx|)), replaces the compare and select.  Used by
+    // the channel-sequential kernel, where one lane owns one channel.
+    static __device__ __forceinline__ void element_rows(float k0, float hx0, float k1, float hx1, float2 &a,
+                                                        float2 &b) {
+        const float2 ek = make_float2(fast_exp2(fabsf(k0) * kNegLog2e), fast_exp2(fabsf(k1) * kNegLog2e));
+        const float2 eh = make_float2(fast_exp2(fabsf(hx0) * kNegLog2e), fast_exp2(fabsf(hx1) * kNegLog2e));
+        const float2 one = make_float2(1.f, 1.f);
+        const float2 dk = __fadd2_rn(ek, one), dh = __fadd2_rn(eh, one);
+        const float2 pr = __fmul2_rn(dk, dh);
+        const float2 inv = make_float2(fast_rcp(pr.x), fast_rcp(pr.y));   // 1 / ((1 + ek)(1 + eh))
+        const float2 rk = __fmul2_rn(dh, inv), rh = __fmul2_rn(dk, inv);
+        const float2 sk = __fmul2_rn(ek, rk), sh = __fmul2_rn(eh, rh);     // sigmoid(-|k|), sigmoid(-|hx|)
+        const float2 kb = __fadd2_rn(one, make_float2(-sk.x, -sk.y));      // sigmoid(|k|)
+        const bool p0 = k0 >= 0.f, p1 = k1 >= 0.f;
+        a = make_float2(p0 ? sk.x : kb.x, p1 ? sk.y : kb.y);
+        const float2 z = make_float2(p0 ? kb.x : sk.x, p1 ? kb.y : sk.y);
+        const float2 hp = __fadd2_rn(make_float2(hx0, hx1), make_float2(0.5f, 0.5f));
+        b = __fmul2_rn(z, make_float2(fmaxf(hp.x, sh.x), fmaxf(hp.y, sh.y)));
+    }
     // fold a step into a running pair, two channels at once: (A, B) <- (A a, B a + b)
     static __device__ __forceinline__ void fold2(float2 &A, float2 &B, float2 a, float2 b) {
         B = __ffma2_rn(B, a, b);
@@ -124,6 +148,11 @@ struct MinMaxOp {
     static __device__ __forceinline__ float pad0() { return INFINITY; }
     static __device__ __forceinline__ float pad1() { return -INFINITY; }
     static __device__ __forceinline__ void element(float r, float s, float &u, float &l) { u = r; l = s; }
+    static __device__ __forceinline__ void element_rows(float r0, float s0, float r1, float s1, float2 &u,
+                                                        float2 &l) {
+        u = make_float2(r0, r1);
+        l = make_float2(s0, s1);
+    }
     static __device__ __forceinline__ float step(float u, float l, float x) { return fmaxf(fminf(x, u), l); }
     static __device__ __forceinline__ float default_init() { return 0.f; }
     static __device__ __forceinline__ void fold2(float2 &U, float2 &L, float2 u, float2 l) {
@@ -873,6 +902,16 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
             row0[SB] = int(tc.c) * TR + (warp * J + j) * R;
             full[SB] = dvalid[SB] && (row0[SB] + R <= p.T);
             base[SB] = (int64_t(tc.b) * p.T) * p.D + d0;
+            // time decay: the tile's rates and the thread's row gaps are plain
+            // global loads, issued before the wait for the tile so that their
+            // latency overlaps it
+            [[maybe_unused]] float lam2[V], ur[R];
+            if constexpr (Op::kDecay) {
+#pragma unroll
+                for (int v = 0; v < V; ++v) lam2[v] = decay_lam2(p, d0 + v);
+#pragma unroll
+                for (int r = 0; r < R; ++r) ur[r] = row0[SB] + r < p.T ? decay_u(p, tc.b, row0[SB] + r) : 0.f;
+            }
             if (!mbar_wait(bars + 8u * uint32_t(n % S), uint32_t((n / S) & 1), wait_limit)) {
                 wait_limit = 1;
                 if (lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);   // null: one chunk, no workspace
@@ -886,11 +925,6 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                 IA[i] = make_float2(Op::identity().x, Op::identity().x);
                 IB[i] = make_float2(Op::identity().y, Op::identity().y);
             }
-            [[maybe_unused]] float lam2[V];
-            if constexpr (Op::kDecay) {
-#pragma unroll
-                for (int v = 0; v < V; ++v) lam2[v] = decay_lam2(p, d0 + v);
-            }
             auto rows = [&](auto fullc) {
                 constexpr bool FULL = decltype(fullc)::value;
 #pragma unroll
@@ -899,9 +933,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                     unpack(*reinterpret_cast<const Vec *>(t0 + r * TC), x0);
                     unpack(*reinterpret_cast<const Vec *>(t1 + r * TC), x1);
                     [[maybe_unused]] float u = 0.f;
-                    if constexpr (Op::kDecay) {
-                        if (row0[SB] + r < p.T) u = decay_u(p, tc.b, row0[SB] + r);
-                    }
+                    if constexpr (Op::kDecay) u = ur[r];
                     if (!FULL) {
                         const bool ok = dvalid[SB] && (row0[SB] + r < p.T);
 #pragma unroll

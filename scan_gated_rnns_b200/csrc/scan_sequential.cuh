@@ -174,17 +174,22 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
         }
         const uint32_t obuf = outb + uint32_t(i & (kSeqOutBufs - 1)) * kOpBytes;
         const uint32_t dst = obuf + uint32_t(lane) * uint32_t(sizeof(IO));
-        // each row's step map (independent of the state), then the step
+        // the step maps of two rows at a time (independent of the state),
+        // then the two steps
+        static_assert(kSeqRows % 2 == 0, "rows are taken in pairs");
 #pragma unroll
-        for (int r = 0; r < kSeqRows; ++r) {
-            float a, c;
-            Op::element(x0r[r], x1r[r], a, c);
+        for (int r = 0; r < kSeqRows; r += 2) {
+            float2 a, c;
+            Op::element_rows(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
             if constexpr (Op::kDecay) {
                 const int64_t t = int64_t(i) * kSeqRows + r;
-                a *= decay_gamma(lam2, t < p.T ? decay_u(p, b, t) : 0.f);
+                a.x *= decay_gamma(lam2, t < p.T ? decay_u(p, b, t) : 0.f);
+                a.y *= decay_gamma(lam2, t + 1 < p.T ? decay_u(p, b, t + 1) : 0.f);
             }
-            h = Op::step(a, c, h);
+            h = Op::step(a.x, c.x, h);
             LR::store(dst + r * kRowBytes, bad ? __int_as_float(0x7fffffff) : h);
+            h = Op::step(a.y, c.y, h);
+            LR::store(dst + (r + 1) * kRowBytes, bad ? __int_as_float(0x7fffffff) : h);
         }
         fence_proxy_async();                                         // outputs visible to the store
         __syncwarp();
