@@ -492,9 +492,31 @@ def measure_step_row(device, B=8, D=1024, calls=200, warmup=10):
         fn()
     torch.cuda.synchronize()
     total, per = timed_launches(fn, calls, torch.cuda.current_stream(device))
+    # the same steps replayed from a CUDA graph: the device-side time of one
+    # step without the host's per-call overhead (token-by-token decoding
+    # captures its step loop the same way)
+    stream = torch.cuda.Stream(device)
+    stream.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(stream):
+        fn()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for _ in range(calls):
+                fn()
+        graph.replay()
+        stream.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        graph.replay()
+        t1.record(stream)
+        stream.synchronize()
+    g_per = t0.elapsed_time(t1) / 1e3 / calls
+    del graph
     return {"op": "mingru_step", "B": B, "D": D, "io_dtype": "f32",
             "us_per_call": round(total / calls * 1e6, 2),
-            "us_per_launch_event": round(per * 1e6, 2), "bytes_per_call": 4 * 4 * B * D}
+            "us_per_launch_event": round(per * 1e6, 2),
+            "us_per_step_graph": round(g_per * 1e6, 2), "bytes_per_call": 4 * 4 * B * D}
 
 
 def cpu_baseline(w, p, q, init, budget_s: float = 12.0):

@@ -174,22 +174,29 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
         }
         const uint32_t obuf = outb + uint32_t(i & (kSeqOutBufs - 1)) * kOpBytes;
         const uint32_t dst = obuf + uint32_t(lane) * uint32_t(sizeof(IO));
-        // the step maps of two rows at a time (independent of the state),
-        // then the two steps
         static_assert(kSeqRows % 2 == 0, "rows are taken in pairs");
+        if (__any_sync(0xffffffffu, bad)) {
+            // a copy of this or an earlier slot never landed: NaN outputs
+            bad = true;
 #pragma unroll
-        for (int r = 0; r < kSeqRows; r += 2) {
-            float2 a, c;
-            Op::element_rows(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
-            if constexpr (Op::kDecay) {
-                const int64_t t = int64_t(i) * kSeqRows + r;
-                a.x *= decay_gamma(lam2, t < p.T ? decay_u(p, b, t) : 0.f);
-                a.y *= decay_gamma(lam2, t + 1 < p.T ? decay_u(p, b, t + 1) : 0.f);
+            for (int r = 0; r < kSeqRows; ++r) LR::store(dst + r * kRowBytes, __int_as_float(0x7fffffff));
+        } else {
+            // the step maps of two rows at a time (independent of the
+            // state), then the two steps
+#pragma unroll
+            for (int r = 0; r < kSeqRows; r += 2) {
+                float2 a, c;
+                Op::element_rows(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
+                if constexpr (Op::kDecay) {
+                    const int64_t t = int64_t(i) * kSeqRows + r;
+                    a.x *= decay_gamma(lam2, t < p.T ? decay_u(p, b, t) : 0.f);
+                    a.y *= decay_gamma(lam2, t + 1 < p.T ? decay_u(p, b, t + 1) : 0.f);
+                }
+                h = Op::step(a.x, c.x, h);
+                LR::store(dst + r * kRowBytes, h);
+                h = Op::step(a.y, c.y, h);
+                LR::store(dst + (r + 1) * kRowBytes, h);
             }
-            h = Op::step(a.x, c.x, h);
-            LR::store(dst + r * kRowBytes, bad ? __int_as_float(0x7fffffff) : h);
-            h = Op::step(a.y, c.y, h);
-            LR::store(dst + (r + 1) * kRowBytes, bad ? __int_as_float(0x7fffffff) : h);
         }
         fence_proxy_async();                                         // outputs visible to the store
         __syncwarp();
@@ -340,19 +347,28 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
                     BOp::coeffs(xk[r], xh[r], xf[r], A, cP, cQ);
                 }
                 const float delta = xg[r] + lam;
-                float y0 = delta * cP, y1 = delta * cQ;
                 if (FULL || r < valid) {
                     lam = A * delta;
                     // dL/dlambda gains delta (1 - z) h_{t-1} dgamma/dlambda = delta A h_{t-1} (-u)
                     if constexpr (BOp::kDecay) dl = fmaf(delta, -u * A * xf[r], dl);
                 }
-                if (bad) y0 = y1 = __int_as_float(0x7fffffff);
-                LR::store(dst + r * kRowBytes, y0);
-                LR::store(dst + kOpBytes + r * kRowBytes, y1);
+                LR::store(dst + r * kRowBytes, delta * cP);
+                LR::store(dst + kOpBytes + r * kRowBytes, delta * cQ);
             }
         };
-        if (valid >= kSeqRows) rows(std::true_type{});
-        else rows(std::false_type{});
+        if (__any_sync(0xffffffffu, bad)) {
+            // a copy of this or an earlier slot never landed: NaN gradients
+            bad = true;
+#pragma unroll
+            for (int r = 0; r < kSeqRows; ++r) {
+                LR::store(dst + r * kRowBytes, __int_as_float(0x7fffffff));
+                LR::store(dst + kOpBytes + r * kRowBytes, __int_as_float(0x7fffffff));
+            }
+        } else if (valid >= kSeqRows) {
+            rows(std::true_type{});
+        } else {
+            rows(std::false_type{});
+        }
         fence_proxy_async();                                         // gradients visible to the stores
         __syncwarp();
         if (lane == 0) {
