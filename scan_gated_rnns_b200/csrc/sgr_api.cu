@@ -157,11 +157,14 @@ struct SeqLayout {
     int slots = 4;
     size_t smem = 0;
 };
-size_t seq_bytes(bool backward, int S, int row_bytes) {
-    return backward ? seq_bwd_warp_bytes(S, row_bytes) : seq_warp_bytes(S, row_bytes);
+enum SeqKind { SEQ_SCAN = 0, SEQ_BACKWARD = 1, SEQ_FOLD = 2 };
+size_t seq_bytes(int kind, int S, int row_bytes) {
+    return kind == SEQ_BACKWARD ? seq_bwd_warp_bytes(S, row_bytes)
+         : kind == SEQ_FOLD     ? seq_fold_warp_bytes(S, row_bytes)
+                                : seq_warp_bytes(S, row_bytes);
 }
 SeqLayout seq_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, size_t reserved,
-                     size_t smem_block_max, bool backward = false) {
+                     size_t smem_block_max, int backward = SEQ_SCAN) {
     SeqLayout l;
     const int64_t K = sms > 0 ? (groups + sms - 1) / sms : 1;
     size_t alloc = seq_bytes(backward, 4, row_bytes);
@@ -649,7 +652,7 @@ cudaError_t launch_sequential_bwd(const BwdParams &bp, cudaStream_t s) {
     q.n_groups = (sp.D + CW - 1) / CW;
     q.n_warps = sp.B * q.n_groups;
     const SeqLayout lay = seq_layout((q.n_warps + WB - 1) / WB * WB, kRowBytes, d.sms, size_t(d.smem_sm),
-                                     size_t(d.reserved), size_t(d.smem_block), true);
+                                     size_t(d.reserved), size_t(d.smem_block), SEQ_BACKWARD);
     q.slots = lay.slots;
     const int64_t grid = (q.n_warps + WB - 1) / WB;
     kernel<<<dim3(unsigned(grid)), WB * 32, lay.smem, s>>>(q, m_in0, m_in1, m_gy, m_fwd, m_d0, m_d1);
@@ -807,12 +810,32 @@ struct SumPlan {
     int V = 1;
     int64_t seg = 0, n_seg = 0;
     size_t ws = 0;
+    bool seq = false;     // warps folding TMA-fed segments of 32-channel groups
 };
 
+// Aligned vector-width rows: one warp per (segment, 32-channel group),
+// segments whole 16-row slots (at most 512 of them), about 52 warps per SM in
+// all (several waves of short segments; measured against 13-156 on the
+// summary rows: 13 per SM in one wave was best for fp32 B8 x 4096 x 1024 by
+// 2% but 20% slower for bf16 B16 x 2048 x 4096, more than 52 slower for the
+// former).  Otherwise one thread per vector (or channel) per segment.
 SumPlan make_sum_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned) {
     SumPlan sp;
-    // one 16-byte vector of channels per thread (4 fp32, 8 bf16)
     const int vw = dtype == SGR_BF16 ? 8 : 4;
+    if (aligned && D % vw == 0 && T <= int64_t(std::numeric_limits<int>::max()) &&
+        B <= int64_t(std::numeric_limits<int>::max())) {
+        sp.seq = true;
+        const int64_t chains = B * ((D + 31) / 32);
+        const int64_t target = int64_t(52) * kAssumedSMs;
+        const int64_t max_seg = std::min<int64_t>(512, (T + kSeqRows - 1) / kSeqRows);
+        const int64_t n_seg = std::max<int64_t>(1, std::min<int64_t>((target + chains - 1) / chains, max_seg));
+        sp.seg = ((T + n_seg - 1) / n_seg + kSeqRows - 1) / kSeqRows * kSeqRows;
+        sp.n_seg = (T + sp.seg - 1) / sp.seg;
+        const int64_t n_mid = sp.n_seg > 32 ? (sp.n_seg + 31) / 32 : 0;
+        sp.ws = align_up(size_t(sp.n_seg + n_mid) * size_t(B) * size_t(D) * sizeof(float2), kAlign);
+        return sp;
+    }
+    // one 16-byte vector of channels per thread (4 fp32, 8 bf16)
     sp.V = (aligned && D % vw == 0) ? vw : 1;
     const int64_t groups = (D + sp.V - 1) / sp.V;
     // about 4096 threads per SM (two waves), each with rows of loads in flight, and at
@@ -829,17 +852,49 @@ SumPlan make_sum_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool a
     return sp;
 }
 
+// pass 1 on TMA-fed warps: one per (segment, 32-channel group)
+template <class Op, typename IO>
+cudaError_t launch_sequential_fold(const SumPlan &pl, const ScanParams &sp, float2 *partial, cudaStream_t s) {
+    constexpr int WB = kSeqWarpsPerBlock;
+    constexpr int CW = 32;
+    constexpr int kRowBytes = seq_row_bytes<IO>();
+    auto kernel = scan_sequential_fold_kernel<Op, IO, WB>;
+    alignas(64) CUtensorMap map0, map1;
+    if (!make_operand_map(&map0, sp.in0, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
+        !make_operand_map(&map1, sp.in1, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows))
+        return cudaErrorInvalidValue;
+    SeqDev d;
+    cudaError_t e = seq_device(reinterpret_cast<const void *>(kernel), seq_fold_warp_bytes(kSeqMinSlots, kRowBytes), &d);
+    if (e != cudaSuccess) return e;
+    SeqFoldParams q;
+    q.s = sp;
+    q.n_groups = (sp.D + CW - 1) / CW;
+    q.n_warps = pl.n_seg * sp.B * q.n_groups;
+    q.seg_rows = pl.seg;
+    q.partial = partial;
+    const SeqLayout lay = seq_layout((q.n_warps + WB - 1) / WB * WB, kRowBytes, d.sms, size_t(d.smem_sm),
+                                     size_t(d.reserved), size_t(d.smem_block), SEQ_FOLD);
+    q.slots = lay.slots;
+    kernel<<<dim3(unsigned((q.n_warps + WB - 1) / WB)), WB * 32, lay.smem, s>>>(q, map0, map1);
+    return cudaGetLastError();
+}
+
 template <class Op, typename IO>
 cudaError_t launch_summary(const SumPlan &pl, const ScanParams &sp, float2 *partial, float2 *out,
                            cudaStream_t s) {
-    const int64_t groups = (sp.D + pl.V - 1) / pl.V;
-    const int64_t n = sp.B * groups * pl.n_seg;
-    const unsigned grid = unsigned(std::min<int64_t>((n + 255) / 256, int64_t(kAssumedSMs) * 16));
     constexpr int VW = 16 / int(sizeof(IO));
-    if (pl.V == 1) {
-        scan_summary_kernel<Op, IO, 1><<<grid, 256, 0, s>>>(sp, pl.seg, pl.n_seg, partial);
+    if (pl.seq) {
+        const cudaError_t e = launch_sequential_fold<Op, IO>(pl, sp, partial, s);
+        if (e != cudaSuccess) return e;
     } else {
-        scan_summary_kernel<Op, IO, VW><<<grid, 256, 0, s>>>(sp, pl.seg, pl.n_seg, partial);
+        const int64_t groups = (sp.D + pl.V - 1) / pl.V;
+        const int64_t n = sp.B * groups * pl.n_seg;
+        const unsigned grid = unsigned(std::min<int64_t>((n + 255) / 256, int64_t(kAssumedSMs) * 16));
+        if (pl.V == 1) {
+            scan_summary_kernel<Op, IO, 1><<<grid, 256, 0, s>>>(sp, pl.seg, pl.n_seg, partial);
+        } else {
+            scan_summary_kernel<Op, IO, VW><<<grid, 256, 0, s>>>(sp, pl.seg, pl.n_seg, partial);
+        }
     }
     const int64_t BD = sp.B * sp.D;
     auto grid_for = [](int64_t n) { return unsigned(std::min<int64_t>((n + 255) / 256, int64_t(kAssumedSMs) * 16)); };

@@ -416,7 +416,10 @@ def test_summary_and_combine_argument_errors():
     assert s(MINGRU, None, Bp, 2, 100, 64, F32, P, W, need, None) == E
     assert s(MINGRU, A, Bp, 2, 100, 64, F32, A + 64, W, need, None) == E      # pairs on an input
     assert s(MINGRU, A, Bp, 2, 100, 64, F32, P, None, 0, None) == _abi.SGR_ERR_WORKSPACE
-    assert s(MINGRU, A, Bp, 2, 100, 64, F32, P, W, need - 256, None) == _abi.SGR_ERR_WORKSPACE
+    # the size covers both the aligned (warp per segment) and the unaligned
+    # plan; 256 bytes, less than either needs, is rejected for both alignments
+    assert s(MINGRU, A, Bp, 2, 100, 64, F32, P, W, 256, None) == _abi.SGR_ERR_WORKSPACE
+    assert s(MINGRU, A + 4, Bp, 2, 100, 64, F32, P, W, 256, None) == _abi.SGR_ERR_WORKSPACE
     assert s(MINGRU, A, Bp, 2, 100, 64, F32, P, P, need, None) == E           # workspace on the pairs
     assert s(MINGRU, A, Bp, 0, 100, 64, F32, None, None, 0, None) == _abi.SGR_OK
     c = lambda *a: lib.sgr_combine_summaries(*a)   # noqa: E731
