@@ -204,3 +204,21 @@ def test_bf16_workload_chunked_kernel_still_matches():
     chans = sample_channels(w, 48)
     ref = oracle_on_channels("mingru", k, hx, h0, chans)
     assert rel_err(gpu_channels(h, chans), ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("dtype,shape,forced", [
+    ("bf16", (128, 20, 4096), False),   # 16384 groups: ~111 warps per SM, several waves
+    ("f32", (1, 70000, 32), True),      # one warp, 4375 slots: every ring slot reused many times
+])
+def test_sequential_many_waves_and_long_sequences(dtype, shape, forced):
+    if forced:
+        sgr.set_kernel_override(SEQ)
+    pl = plan(*shape, dtype)
+    assert pl["kernel"] == SEQ
+    k, hx, h0 = small("mingru", *shape, dtype, "u01_1", seed=101)
+    h = sgr.mingru_scan(*dev(k, hx, h0))
+    r, s, x0 = small("minmax", *shape, dtype, "u01_1", seed=102)
+    x = sgr.minmax_scan(*dev(r, s, x0))
+    torch.cuda.synchronize()
+    assert rel_err(h, oracle.mingru_linear(k, hx, h0, threads=8)) <= TOL[dtype]
+    assert exact(x, oracle.minmax(r, s, x0, threads=8))
