@@ -5,6 +5,7 @@
 #include "projected_scan.cuh"
 #include "scan_backward.cuh"
 #include "scan_engine.cuh"
+#include "scan_fold.cuh"
 #include "scan_sequential.cuh"
 
 #include <algorithm>
