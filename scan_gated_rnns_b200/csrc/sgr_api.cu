@@ -186,9 +186,13 @@ SeqLayout seq_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, siz
 // 128-byte row segments); anything else takes the tile kernel's scalar
 // variant.  The override knobs select the kernel and the rows per thread.
 // force_tile: the tile kernel whatever the alignment (the gradient kernel,
-// which keeps four values per element live, also caps a thread at 16 elements)
+// which keeps four values per element live, also caps a thread at 16 elements).
+// light_op: the recurrence does next to no arithmetic per element (MinMax), so
+// per-tile work dominates and the longer tiles of 15-warp blocks pay wherever
+// they still give every SM 4 tiles (measured: MinMax B4 x 8192 x 768 fp32 0.81
+// of the copy bandwidth against 0.78 with 7-warp blocks; minGRU slower).
 Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
-               bool force_tile = false) {
+               bool force_tile = false, bool light_op = false) {
     Plan p;
     p.esz = (dtype == SGR_BF16) ? 2 : 4;
     const int vw = 16 / p.esz;
@@ -251,7 +255,8 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
         const int64_t n_chains = B * ((D + p.TC - 1) / p.TC);
         const int64_t tr_wide = int64_t(kPipeWarpsWide) * (32 / p.cg) * p.r;
         const int64_t tiles_wide = n_chains * ((T + tr_wide - 1) / tr_wide);
-        bool wide = n_chains > 0 && 2 * kAssumedSMs >= 8 * n_chains && tiles_wide >= 4 * kAssumedSMs;
+        bool wide = n_chains > 0 && (light_op || 2 * kAssumedSMs >= 8 * n_chains) &&
+                    tiles_wide >= 4 * kAssumedSMs;
         if (ok == KIND_PIPELINED) wide = false;
         if (ok == KIND_PIPELINED_WIDE) wide = true;
         // 8 rows: bf16 only (fp32 tiles of 8 rows exceed the TMA box with 15
@@ -553,7 +558,7 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
         return SGR_ERR_INVALID_ARG;
 
     const bool aligned = aligned16(in0) && aligned16(in1) && aligned16(out);
-    const Plan pl = make_plan(B, T, D, dtype, aligned);
+    const Plan pl = make_plan(B, T, D, dtype, aligned, false, op == SGR_OP_MINMAX);
     if (pl.n_tiles > int64_t(std::numeric_limits<int>::max())) return SGR_ERR_UNSUPPORTED;
 
     ScanParams sp;
@@ -1240,8 +1245,8 @@ size_t sgr_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtyp
     if (dtype != SGR_F32 && dtype != SGR_BF16) return 0;
     if (B <= 0 || T <= 0 || D <= 0) return 0;
     // the vector and the scalar variant may cut T differently: cover both
-    const Plan a = make_plan(B, T, D, dtype, true);
-    const Plan b = make_plan(B, T, D, dtype, false);
+    const Plan a = make_plan(B, T, D, dtype, true, false, op == SGR_OP_MINMAX);
+    const Plan b = make_plan(B, T, D, dtype, false, false, op == SGR_OP_MINMAX);
     return a.ws_bytes > b.ws_bytes ? a.ws_bytes : b.ws_bytes;
 }
 
@@ -1283,7 +1288,7 @@ sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dty
     if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return SGR_ERR_INVALID_ARG;
     if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || D < 0 || !plan) return SGR_ERR_INVALID_ARG;
-    const Plan p = make_plan(B, T, D, dtype, aligned != 0);
+    const Plan p = make_plan(B, T, D, dtype, aligned != 0, false, op == SGR_OP_MINMAX);
     plan->vector_path = p.vec ? 1 : 0;
     plan->kernel = p.kind;
     plan->channels_per_thread = p.V;

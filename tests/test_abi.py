@@ -157,8 +157,8 @@ def check_sequential_indices(pl, B, T, D, esz, check_cover):
         assert (cover[:, :T] == 1).all(), "every output element is written exactly once"
 
 
-def check_plan_indices(B, T, D, dtype, aligned, check_cover):
-    pl = _abi.plan(MINGRU, B, T, D, dtype, aligned)
+def check_plan_indices(B, T, D, dtype, aligned, check_cover, op=MINGRU):
+    pl = _abi.plan(op, B, T, D, dtype, aligned)
     esz = 4 if dtype == F32 else 2
     if pl["kernel"] == _abi.KERNEL_SEQUENTIAL:
         check_sequential_indices(pl, B, T, D, esz, check_cover)
@@ -223,7 +223,7 @@ def check_plan_indices(B, T, D, dtype, aligned, check_cover):
     if n_chunks > 1:
         assert pl["off_words"] >= 4 and pl["off_words"] % 8 == 0
         assert pl["off_words"] + 8 * 3 * TC * n_tiles <= pl["workspace_bytes"]
-        assert _abi.lib().sgr_workspace_size(MINGRU, B, T, D, dtype) >= pl["workspace_bytes"]
+        assert _abi.lib().sgr_workspace_size(op, B, T, D, dtype) >= pl["workspace_bytes"]
     else:
         assert pl["workspace_bytes"] == 0
 
@@ -252,7 +252,8 @@ def test_plan_indices_small(shape, dtype, aligned, override):
 @pytest.mark.parametrize("name", sorted(WORKLOADS))
 def test_plan_indices_workloads(name):
     w = WORKLOADS[name]
-    check_plan_indices(w.B, w.T, w.D, F32 if w.dtype == "f32" else BF16, True, check_cover=False)
+    op = MINGRU if w.op == "mingru" else _abi.SGR_OP_MINMAX
+    check_plan_indices(w.B, w.T, w.D, F32 if w.dtype == "f32" else BF16, True, check_cover=False, op=op)
 
 
 # ------------------------------------------------------- host-buffer scans
@@ -470,3 +471,15 @@ def test_backward_kernel_choice():
         assert lib.sgr_backward_kernel(MINGRU, 1, 10, 6, F32, 1) == 1        # rows not 16-byte multiples
     finally:
         lib.sgr_set_kernel_override(0)
+
+
+def test_minmax_plans_take_the_long_tiles():
+    """MinMax, next to no arithmetic per element, takes the 15-warp pipelined
+    blocks wherever they still give every SM 4 tiles; minGRU on the same
+    shape keeps the 7-warp blocks."""
+    assert _abi.plan(_abi.SGR_OP_MINMAX, 4, 8192, 768, F32, True)["kernel"] == _abi.KERNEL_PIPELINED_WIDE
+    assert _abi.plan(MINGRU, 4, 8192, 768, F32, True)["kernel"] == _abi.KERNEL_PIPELINED
+    lib = _abi.lib()
+    # the size query covers this plan (and the unaligned one)
+    assert lib.sgr_workspace_size(_abi.SGR_OP_MINMAX, 4, 8192, 768, F32) >= \
+        _abi.plan(_abi.SGR_OP_MINMAX, 4, 8192, 768, F32, True)["workspace_bytes"] > 0
