@@ -21,6 +21,10 @@
 // Persistent blocks, one per SM (cooperative launch: every look-back waits
 // for a block that is resident), each taking tiles blockIdx.x, blockIdx.x +
 // gridDim.x, ...  Warp 0 streams W and x tiles by TMA into a 4-stage ring
+// (per stage one box of x and one box of W, the latter through a 4-D view of
+// W -- (K, row in a 16-row group, k or hx, group) -- that lands the tile's
+// rows in the interleaved order above; issuing the W rows as eight 16-row
+// boxes instead measured 11% slower)
 // (continuing across tiles); one thread of warp 1 issues the MMAs of tile i
 // into one of two accumulators (512 tensor-memory columns in all) while warps
 // 4-19 run the epilogue of tile i-1 from the other.  Epilogue warp (q, g)
@@ -85,10 +89,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kTR >> 3) << 17) |
                             (uint32_t(kM >> 4) << 24);
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int x, int y, int z, int w,
+                                            uint32_t bar) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar) : "memory");
 }
 
 // bounded wait; false if the phase did not complete
@@ -175,12 +180,9 @@ __global__ void __launch_bounds__(proj::kThreads, 1) mingru_projected_scan_kerne
                     }
                     const uint32_t a_dst = ring + uint32_t(s) * kStageBytes;
                     mbar_expect_tx(full(s), kStageBytes);
-#pragma unroll
-                    for (int gi = 0; gi < kTC / kGrp; ++gi) {
-                        tma_load_2d(a_dst + uint32_t(2 * gi) * kGrpBytes, &map_w, kb * kKB, w_row + gi * kGrp, full(s));
-                        tma_load_2d(a_dst + uint32_t(2 * gi + 1) * kGrpBytes, &map_w, kb * kKB,
-                                    int(p.D) + w_row + gi * kGrp, full(s));
-                    }
+                    // W viewed as (K, row in group, k/hx, group): one box of
+                    // (kKB, kGrp, 2, kTC / kGrp) lands in the interleaved order
+                    tma_load_4d(a_dst, &map_w, kb * kKB, 0, 0, w_row / kGrp, full(s));
                     tma_load_3d(a_dst + kABytes, &map_x, kb * kKB, int(tc.c) * kTR, int(tc.b), full(s));
                 }
             }

@@ -979,11 +979,14 @@ sgr_status_t run_projected_scan(const void *x, const void *w, const float *h0, i
             return SGR_ERR_CUDA;
     }
     {
-        const cuuint64_t dims[2] = {cuuint64_t(d_in), cuuint64_t(2 * D)};
-        const cuuint64_t strides[1] = {cuuint64_t(d_in) * 2};
-        const cuuint32_t box[2] = {cuuint32_t(proj::kKB), cuuint32_t(proj::kGrp)};
-        const cuuint32_t es[2] = {1u, 1u};
-        if (enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(w), dims, strides, box, es,
+        // W (2 D, d_in) as (d_in, 16 rows of a group, k/hx, D / 16 groups)
+        const cuuint64_t dims[4] = {cuuint64_t(d_in), cuuint64_t(proj::kGrp), 2, cuuint64_t(D / proj::kGrp)};
+        const cuuint64_t strides[3] = {cuuint64_t(d_in) * 2, cuuint64_t(D) * cuuint64_t(d_in) * 2,
+                                       cuuint64_t(proj::kGrp) * cuuint64_t(d_in) * 2};
+        const cuuint32_t box[4] = {cuuint32_t(proj::kKB), cuuint32_t(proj::kGrp), 2u,
+                                   cuuint32_t(proj::kTC / proj::kGrp)};
+        const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+        if (enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(w), dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return SGR_ERR_CUDA;
