@@ -174,12 +174,12 @@ struct MinGRUDecayOp : MinGRUOp {
     static constexpr bool kDecay = true;
 };
 
-// gamma = exp(-lambda u) = 2^(lam2 u) with lam2 = -lambda log2 e (<= 0)
-constexpr float kDecayClampLog2 = -1.0e4f * 1.4426950408889634f;
-__device__ __forceinline__ float decay_gamma(float lam2, float u) {
-    const float x = lam2 * u;
-    return x < kDecayClampLog2 ? 0.f : fast_exp2(x);
-}
+// gamma = exp(-lambda u) = 2^(lam2 u) with lam2 = -lambda log2 e (<= 0).
+// The wipe needs no compare: the MUFU 2^x flushes every result below the
+// normal range to +0, so gamma is exactly 0 for all lambda u above about 87.3
+// (2^-126 = e^-87.3), which includes every gap past the 1e4 clamp; the
+// gradients then see gamma = 0 and dgamma/dlambda = -u gamma = 0 there too.
+__device__ __forceinline__ float decay_gamma(float lam2, float u) { return fast_exp2(lam2 * u); }
 
 // ------------------------------------------------------------ memory access
 
