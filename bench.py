@@ -653,7 +653,7 @@ def run_b200(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(et * 1e3 / e_steps, 3), "steps": e_steps,
                "api": f"{host_fn.__name__} (pinned host tensors in and out, time slices of "
-                      "~8 MB of inputs, uploads/scans/downloads overlapped)",
+                      "about sqrt(input MiB / 4.6) slices, uploads/scans/downloads overlapped)",
                "staging_bytes": nbytes}
         del hp, hq, hi, hout
 

@@ -351,7 +351,9 @@ SGR_API size_t sgr_backward_workspace_size(sgr_op_t op, int64_t B, int64_t T, in
  * data that does not already live on the GPU.
  *
  * The time axis is cut into slices of Tc = ceil(T / n) rows, n = `chunks`
- * (0 picks n so that one slice's inputs are about 8 MB).  Slice i is copied to
+ * (0 picks n = round(sqrt(input MiB / 4.6)): 7 slices for 256 MiB of inputs,
+ * which balances a fixed cost per slice against the pipeline's fill and
+ * drain).  Slice i is copied to
  * the device on a library-owned copy stream, scanned on `stream` with the
  * last row of slice i-1's output as its initial state, and copied back on a
  * second library-owned stream, with two sets of device buffers, so the

@@ -90,7 +90,7 @@ def mingru_scan_host(k: torch.Tensor, hx: torch.Tensor, h0: Optional[torch.Tenso
                      out: Optional[torch.Tensor] = None, chunks: int = 0, device=None,
                      blocking: bool = True) -> torch.Tensor:
     """minGRU scan of host (B, T, D) tensors, computed on the GPU; returns a
-    host tensor.  ``chunks`` = time slices (0: automatic, ~8 MB of inputs each)."""
+    host tensor.  ``chunks`` = time slices (0: automatic, about sqrt(input MiB / 4.6))."""
     return _scan_host("mingru_scan_host", "mingru", k, hx, h0, out, chunks, device, blocking)
 
 

@@ -295,9 +295,10 @@ def test_host_staging_size():
             assert s <= prev
         prev = s
     assert size(B, T, D, chunks=T) == size(B, T, D, chunks=10 * T)    # at most one row per slice
-    # automatic slices hold about 8 MB of inputs: staging stays far below the tensor
+    # automatic slices: n = round(sqrt(input MiB / 4.6)), 7 for these 256 MiB of
+    # inputs; staging stays far below the tensor
     auto = size(B, T, D)
-    assert 6 * (8 << 20) // 2 <= auto <= 6 * (8 << 20) // 2 + (4 << 20)
+    assert auto == size(B, T, D, chunks=7) and auto < 6 * whole // 4
     assert size(2, 5, 3, op=MINMAX, chunks=2) > 0
 
 
