@@ -67,7 +67,10 @@
  *  region itself inside the graph.
  *  Wide batches (B x D large enough that groups of 32 channels give every SM
  *  several warps) are not cut along T at all: each warp scans its 32 channels
- *  over the whole sequence, and sgr_workspace_size() returns 0.
+ *  over the whole sequence, and the plan needs no workspace.  The
+ *  time-decayed minGRU (mingru_scan_decay) is always cut along T when T spans
+ *  several chunks; sgr_workspace_size(SGR_OP_MINGRU, ...) covers it too, so
+ *  it may be > 0 for such shapes.
  *  A workspace passed to such a call anyway (>= 4 bytes, 16-byte aligned)
  *  receives the status word of its bounded waits.
  */
@@ -253,6 +256,11 @@ SGR_API sgr_status_t sgr_combine_summaries(sgr_op_t op, const float *pairs, int6
  *   lambda  : fp32 DEVICE array (D,), decay rates >= 0 (fixed or learnable)
  * Other arguments, workspace and errors as mingru_scan (the same workspace
  * size).  Arithmetic fp32; the gate uses the MUFU exp2 like the activations.
+ * Kernel: never the channel-sequential one (it would wait for the gaps one row
+ * at a time); the chunked kernels with 4 rows per thread, so the plan that
+ * sgr_scan_plan reports for SGR_OP_MINGRU may differ.  With delta_t and lambda
+ * 16-byte aligned (and a batch stride a multiple of 4) the pipelined kernel
+ * brings them in with the copy engine beside the operands.
  */
 SGR_API sgr_status_t mingru_scan_decay(const void *k, const void *hx,
                                        const void *h0, int64_t h0_batch_stride,

@@ -753,13 +753,23 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const Sca
 // warp released before it waited for tile n-1: no cycle.  Every look-back
 // wait is for a tile with a smaller index and blocks are co-resident, so the
 // smallest unfinished tile can always progress.
-template <typename IO, int V, int CG, int R, int S, int W>
+template <typename IO, int V, int CG, int R, int S, int W, bool DEC = false>
 struct PipeShape {
     static constexpr int J = 32 / CG;
     static constexpr int TC = CG * V;
     static constexpr int TR = W * J * R;
     static constexpr size_t op_bytes = size_t(TR) * TC * sizeof(IO);     // one operand of a tile
-    static constexpr size_t slot_bytes = 2 * op_bytes;
+    // time decay through the copy engine: the tile's TC rates, then its TR
+    // row gaps (fp32), follow the two operands in the slot.  Every copy's
+    // shared-memory destination must sit on a 128-byte boundary, a copy box
+    // spans at most 256 elements a dimension and 16-byte multiples of them,
+    // and a gap box starts at a row index whose byte offset is a multiple
+    // of 16 (tiles start at multiples of TR).
+    static constexpr bool dec_boxable = TR % 4 == 0 && TR <= 256 && TC <= 256 && (TC * 4) % 128 == 0;
+    static_assert(op_bytes % 128 == 0, "operand copies land on 128-byte boundaries");
+    static constexpr size_t dec_bytes = DEC ? size_t(TR + TC) * sizeof(float) : 0;
+    static constexpr size_t tx_bytes = 2 * op_bytes + dec_bytes;         // bytes a tile's copies bring
+    static constexpr size_t slot_bytes = (tx_bytes + 127) / 128 * 128;
     static constexpr size_t bar_offset = S * slot_bytes;
     static constexpr size_t cnt_offset = bar_offset + S * 8;          // per-slot reader counts
     static constexpr size_t tot_offset = (cnt_offset + S * 4 + 15) / 16 * 16;        // [2][W][TC] float2
@@ -803,17 +813,35 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tma_load_1d(uint32_t dst, const CUtensorMap *map, int x, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.1d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2}], [%3];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(bar) : "memory");
+}
+
 // bound on mbarrier polls (each try_wait may suspend the thread for up to a
 // microsecond or so); after one wait has run out, later waits of the thread
 // make a single poll, so a broken copy cannot stretch the kernel to n_local
 // full bounds
 constexpr uint32_t kMbarLimit = 1u << 16;
 
-template <class Op, typename IO, int V, int CG, int R, int S, int W, int MINB>
+// DT (time decay only): the gaps and rates come with the tile through the
+// copy engine (map_gap: the (B, T) gaps, map_lam: the (D,) rates), so they
+// hold no registers across the wait and the one-tile lag fits; otherwise
+// they are plain loads and map_gap, map_lam are unused.
+template <class Op, typename IO, int V, int CG, int R, int S, int W, int MINB, bool DT = false>
 __global__ void __launch_bounds__((W + 1) * 32, MINB)
 scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap map0,
-                      const __grid_constant__ CUtensorMap map1) {
-    using Shape = PipeShape<IO, V, CG, R, S, W>;
+                      const __grid_constant__ CUtensorMap map1, const __grid_constant__ CUtensorMap map_gap,
+                      const __grid_constant__ CUtensorMap map_lam) {
+    static_assert(!DT || Op::kDecay, "decay operands through the copy engine need a decay operator");
+    using Shape = PipeShape<IO, V, CG, R, S, W, DT>;
+    static_assert(!DT || Shape::dec_boxable, "decay operands fit copy boxes");
     using Vec = typename VecOf<IO, V>::type;
     constexpr int J = Shape::J;
     constexpr int TC = Shape::TC;
@@ -833,7 +861,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
     // barriers, tile coordinates) is spread over twice the elements.  The
     // time-decay gate's per-channel rates and per-row gaps do not fit beside
     // two tiles' pairs either (register spills measured slower than waiting).
-    constexpr bool LAG = R < 8 && !Op::kDecay;
+    constexpr bool LAG = R < 8 && (!Op::kDecay || DT);
     constexpr int NB = LAG ? 2 : 1;
     static_assert(sizeof(Vec) == V * sizeof(IO), "vector type matches the vector width");
     static_assert(CG * J == 32 && TC % 32 == 0, "lane layout");
@@ -859,9 +887,13 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
         const uint32_t slot = ring + uint32_t((n % S) * Shape::slot_bytes);
         const uint32_t bar = bars + 8u * uint32_t(n % S);
         const int x = int(tc.dt) * TC, y = int(tc.c) * TR, z = int(tc.b);
-        mbar_expect_tx(bar, uint32_t(Shape::slot_bytes));
+        mbar_expect_tx(bar, uint32_t(Shape::tx_bytes));
         tma_load_3d(slot, &map0, x, y, z, bar);
         tma_load_3d(slot + uint32_t(Shape::op_bytes), &map1, x, y, z, bar);
+        if constexpr (DT) {
+            tma_load_1d(slot + uint32_t(2 * Shape::op_bytes), &map_lam, x, bar);
+            tma_load_2d(slot + uint32_t(2 * Shape::op_bytes) + uint32_t(TC) * 4u, &map_gap, y, z, bar);
+        }
     };
 
     if (threadIdx.x == 0) {
@@ -906,7 +938,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
             // global loads, issued before the wait for the tile so that their
             // latency overlaps it
             [[maybe_unused]] float lam2[V], ur[R];
-            if constexpr (Op::kDecay) {
+            if constexpr (Op::kDecay && !DT) {
 #pragma unroll
                 for (int v = 0; v < V; ++v) lam2[v] = decay_lam2(p, d0 + v);
 #pragma unroll
@@ -919,6 +951,11 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
             const IO *t0 = reinterpret_cast<const IO *>(smem + (n % S) * Shape::slot_bytes) +
                            ((warp * J + j) * R) * TC + g * V;
             const IO *t1 = t0 + TR * TC;
+            // DT: the tile's rates (channels past D read 0) and gaps (rows
+            // past T read 0: gamma = 1) in the slot
+            [[maybe_unused]] const float *s_lam =
+                reinterpret_cast<const float *>(smem + (n % S) * Shape::slot_bytes + 2 * Shape::op_bytes);
+            [[maybe_unused]] const float *s_gap = s_lam + TC;
             float2 IA[V2], IB[V2];
 #pragma unroll
             for (int i = 0; i < V2; ++i) {
@@ -933,7 +970,12 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                     unpack(*reinterpret_cast<const Vec *>(t0 + r * TC), x0);
                     unpack(*reinterpret_cast<const Vec *>(t1 + r * TC), x1);
                     [[maybe_unused]] float u = 0.f;
-                    if constexpr (Op::kDecay) u = ur[r];
+                    if constexpr (DT) {
+                        u = s_gap[(warp * J + j) * R + r];
+                        if (p.decay_log1p) u = log1pf(u);
+                    } else if constexpr (Op::kDecay) {
+                        u = ur[r];
+                    }
                     if (!FULL) {
                         const bool ok = dvalid[SB] && (row0[SB] + r < p.T);
 #pragma unroll
@@ -947,7 +989,10 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                         float a0, b0, a1, b1;
                         Op::element(x0[2 * i], x1[2 * i], a0, b0);
                         Op::element(x0[2 * i + 1], x1[2 * i + 1], a1, b1);
-                        if constexpr (Op::kDecay) {
+                        if constexpr (DT) {
+                            a0 *= decay_gamma(s_lam[g * V + 2 * i] * -1.4426950408889634f, u);
+                            a1 *= decay_gamma(s_lam[g * V + 2 * i + 1] * -1.4426950408889634f, u);
+                        } else if constexpr (Op::kDecay) {
                             a0 *= decay_gamma(lam2[2 * i], u);
                             a1 *= decay_gamma(lam2[2 * i + 1], u);
                         }

@@ -191,8 +191,12 @@ SeqLayout seq_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, siz
 // per-tile work dominates and the longer tiles of 15-warp blocks pay wherever
 // they still give every SM 4 tiles (measured: MinMax B4 x 8192 x 768 fp32 0.81
 // of the copy bandwidth against 0.78 with 7-warp blocks; minGRU slower).
+// light_op: the MinMax clamp pair; decay: the time-decayed minGRU, whose
+// per-row gaps the channel-sequential kernel would wait for one row at a
+// time, and whose extra gate per element favours 4 rows per thread in the
+// pipelined kernel (bf16 with 15-warp blocks)
 Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
-               bool force_tile = false, bool light_op = false) {
+               bool force_tile = false, bool light_op = false, bool decay = false) {
     Plan p;
     p.esz = (dtype == SGR_BF16) ? 2 : 4;
     const int vw = 16 / p.esz;
@@ -206,7 +210,7 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
                             B <= int64_t(std::numeric_limits<int>::max());
         const int min_per_sm = p.esz == 2 ? kSeqMinWarpsPerSMHalf : kSeqMinWarpsPerSM;
         const bool want = ok == KIND_SEQUENTIAL ||
-                          (ok == KIND_AUTO && groups >= int64_t(min_per_sm) * kAssumedSMs);
+                          (ok == KIND_AUTO && !decay && groups >= int64_t(min_per_sm) * kAssumedSMs);
         if (seq_ok && want) {
             const SeqLayout lay = seq_layout(groups, int(cw) * p.esz, kAssumedSMs, kAssumedSmemPerSM,
                                              kAssumedSmemReserved, kAssumedSmemPerBlock);
@@ -245,7 +249,7 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
         // elements are half the bytes, so per-tile work (warp scan, barriers,
         // hand-off) weighs twice as much per byte and is spread over twice
         // the rows (replayed without the one-tile lag, see the kernel)
-        p.r = (orr == 2 || orr == 4 || orr == 8) ? orr : (p.esz == 2 ? 8 : 4);
+        p.r = (orr == 2 || orr == 4 || orr == 8) ? orr : (p.esz == 2 && !decay ? 8 : 4);
         p.stages = kStages;
         // Block shape: about (blocks in flight) / n_chains chunks of one
         // channel tile are processed at once and a look-back folds that many
@@ -255,7 +259,7 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
         const int64_t n_chains = B * ((D + p.TC - 1) / p.TC);
         const int64_t tr_wide = int64_t(kPipeWarpsWide) * (32 / p.cg) * p.r;
         const int64_t tiles_wide = n_chains * ((T + tr_wide - 1) / tr_wide);
-        bool wide = n_chains > 0 && (light_op || 2 * kAssumedSMs >= 8 * n_chains) &&
+        bool wide = n_chains > 0 && (light_op || (decay && p.esz == 2) || 2 * kAssumedSMs >= 8 * n_chains) &&
                     tiles_wide >= 4 * kAssumedSMs;
         if (ok == KIND_PIPELINED) wide = false;
         if (ok == KIND_PIPELINED_WIDE) wide = true;
@@ -375,17 +379,48 @@ DeviceInfo device_info(int dev) {
     return d;
 }
 
-template <class Op, typename IO, int V, int R, int W>
-cudaError_t launch_pipelined(const ScanParams &sp_in, cudaStream_t s, int64_t *grid_out) {
+// Tensor maps of a decay's gaps (B, T) fp32 rows with a batch stride and
+// rates (D,) fp32, for boxes of TR gaps of one batch row and TC rates; false
+// when the copy engine cannot take them (16-byte aligned bases and row
+// stride needed), and the kernel then loads them itself.
+bool make_decay_maps(CUtensorMap *gap, CUtensorMap *lam, const ScanParams &sp, int TR, int TC) {
+    if (!sp.decay_dt || !sp.decay_lam || !aligned16(sp.decay_dt) || !aligned16(sp.decay_lam)) return false;
+    if (sp.B > 1 && (sp.decay_dt_bs % 4) != 0) return false;
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (enc == nullptr) return false;
+    {
+        const cuuint64_t dims[2] = {cuuint64_t(sp.T), cuuint64_t(sp.B)};
+        const cuuint64_t row = sp.B > 1 ? cuuint64_t(sp.decay_dt_bs) * 4 : (cuuint64_t(sp.T) * 4 + 15) / 16 * 16;
+        const cuuint64_t strides[1] = {row};
+        const cuuint32_t box[2] = {cuuint32_t(TR), 1u};
+        const cuuint32_t es[2] = {1u, 1u};
+        if (enc(gap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(sp.decay_dt), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    {
+        const cuuint64_t dims[1] = {cuuint64_t(sp.D)};
+        const cuuint64_t strides[1] = {0};
+        const cuuint32_t box[1] = {cuuint32_t(TC)};
+        const cuuint32_t es[1] = {1u};
+        if (enc(lam, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<float *>(sp.decay_lam), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    return true;
+}
+
+template <class Op, typename IO, int V, int R, int W, bool DT>
+cudaError_t launch_pipelined_shape(const ScanParams &sp_in, const CUtensorMap &map0, const CUtensorMap &map1,
+                                   const CUtensorMap &map_gap, const CUtensorMap &map_lam, cudaStream_t s,
+                                   int64_t *grid_out) {
     constexpr int CG = pipe_cg<IO>();
-    using Shape = PipeShape<IO, V, CG, R, kStages, W>;
+    using Shape = PipeShape<IO, V, CG, R, kStages, W, DT>;
     constexpr int MINB = W == kPipeWarps ? 2 : 1;
-    auto kernel = scan_pipelined_kernel<Op, IO, V, CG, R, kStages, W, MINB>;
+    auto kernel = scan_pipelined_kernel<Op, IO, V, CG, R, kStages, W, MINB, DT>;
     constexpr size_t smem = Shape::smem_bytes;
-    alignas(64) CUtensorMap map0, map1;
-    if (!make_operand_map(&map0, sp_in.in0, sp_in.B, sp_in.T, sp_in.D, int(sizeof(IO)), Shape::TC, Shape::TR) ||
-        !make_operand_map(&map1, sp_in.in1, sp_in.B, sp_in.T, sp_in.D, int(sizeof(IO)), Shape::TC, Shape::TR))
-        return cudaErrorInvalidValue;
     constexpr int NT = (W + 1) * 32;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -416,8 +451,23 @@ cudaError_t launch_pipelined(const ScanParams &sp_in, cudaStream_t s, int64_t *g
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kernel, sp, map0, map1);
-    return e;
+    return cudaLaunchKernelEx(&cfg, kernel, sp, map0, map1, map_gap, map_lam);
+}
+
+template <class Op, typename IO, int V, int R, int W>
+cudaError_t launch_pipelined(const ScanParams &sp_in, cudaStream_t s, int64_t *grid_out) {
+    constexpr int CG = pipe_cg<IO>();
+    using Shape = PipeShape<IO, V, CG, R, kStages, W>;
+    alignas(64) CUtensorMap map0, map1, map_gap, map_lam;
+    if (!make_operand_map(&map0, sp_in.in0, sp_in.B, sp_in.T, sp_in.D, int(sizeof(IO)), Shape::TC, Shape::TR) ||
+        !make_operand_map(&map1, sp_in.in1, sp_in.B, sp_in.T, sp_in.D, int(sizeof(IO)), Shape::TC, Shape::TR))
+        return cudaErrorInvalidValue;
+    if constexpr (Op::kDecay && PipeShape<IO, V, CG, R, kStages, W, true>::dec_boxable) {
+        if (make_decay_maps(&map_gap, &map_lam, sp_in, Shape::TR, Shape::TC))
+            return launch_pipelined_shape<Op, IO, V, R, W, true>(sp_in, map0, map1, map_gap, map_lam, s, grid_out);
+    }
+    // no decay operands through the copy engine: the two maps are not read
+    return launch_pipelined_shape<Op, IO, V, R, W, false>(sp_in, map0, map1, map0, map1, s, grid_out);
 }
 
 // ---- channel-sequential kernels: one warp per channel group
@@ -558,7 +608,7 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
         return SGR_ERR_INVALID_ARG;
 
     const bool aligned = aligned16(in0) && aligned16(in1) && aligned16(out);
-    const Plan pl = make_plan(B, T, D, dtype, aligned, false, op == SGR_OP_MINMAX);
+    const Plan pl = make_plan(B, T, D, dtype, aligned, false, op == SGR_OP_MINMAX, dec != nullptr);
     if (pl.n_tiles > int64_t(std::numeric_limits<int>::max())) return SGR_ERR_UNSUPPORTED;
 
     ScanParams sp;
@@ -1247,10 +1297,12 @@ size_t sgr_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtyp
     if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return 0;
     if (dtype != SGR_F32 && dtype != SGR_BF16) return 0;
     if (B <= 0 || T <= 0 || D <= 0) return 0;
-    // the vector and the scalar variant may cut T differently: cover both
-    const Plan a = make_plan(B, T, D, dtype, true, false, op == SGR_OP_MINMAX);
-    const Plan b = make_plan(B, T, D, dtype, false, false, op == SGR_OP_MINMAX);
-    return a.ws_bytes > b.ws_bytes ? a.ws_bytes : b.ws_bytes;
+    // the vector and the scalar variant may cut T differently, and the
+    // time-decayed minGRU may take another kernel: cover them all
+    size_t need = 0;
+    for (int v = 0; v < (op == SGR_OP_MINGRU ? 4 : 2); ++v)
+        need = std::max(need, make_plan(B, T, D, dtype, (v & 1) == 0, false, op == SGR_OP_MINMAX, v >= 2).ws_bytes);
+    return need;
 }
 
 sgr_status_t sgr_workspace_init(void *workspace, size_t ws_bytes, cudaStream_t stream) {

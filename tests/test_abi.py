@@ -101,6 +101,15 @@ def test_step_argument_errors():
     assert lib.mingru_step(A, 8, Bp, 8, None, 0, C, 8, 0, 8, F32, None) == _abi.SGR_OK
 
 
+def test_workspace_covers_the_decayed_plan():
+    # wide batches: the plain plan needs no workspace, the time-decayed scan
+    # (never channel-sequential) is cut along T and needs one
+    for B, dtype in ((16, F32), (24, BF16)):
+        pl = _abi.plan(MINGRU, B, 2048, 2048, dtype, True)
+        assert pl["kernel"] == _abi.KERNEL_SEQUENTIAL and pl["workspace_bytes"] == 0
+        assert _abi.lib().sgr_workspace_size(MINGRU, B, 2048, 2048, dtype) > 0
+
+
 def test_workspace_size_and_hooks():
     lib = _abi.lib()
     assert lib.sgr_workspace_size(MINGRU, 2, 1, 512, F32) == 0      # one chunk

@@ -87,6 +87,46 @@ def test_decay_every_kernel(kernel, r, dtype):
     assert rel_err(h, oracle.mingru_decay(k, hx, h0, dt, lam)) <= TOL[dtype]
 
 
+# Wide batches: the plain scan's plan scans whole sequences per warp, the
+# decayed scan stays on the chunked kernels, and the workspace query covers it.
+@pytest.mark.parametrize("dtype,B", [("f32", 16), ("bf16", 24)])
+def test_decay_wide_batch(dtype, B):
+    T, D = 300, 2048
+    code = _abi.SGR_F32 if dtype == "f32" else _abi.SGR_BF16
+    assert _abi.plan(_abi.SGR_OP_MINGRU, B, T, D, code, True)["kernel"] == _abi.KERNEL_SEQUENTIAL
+    need = sgr.workspace_size("mingru", B, T, D, TORCH_DT[dtype])
+    assert need > 0
+    k, hx, h0, dt, lam = data(B, T, D, dtype, "u01_1", seed=B, wipe_at=150)
+    ws = sgr.Workspace(need, DEV)
+    h = sgr.mingru_scan_decay(k.to(DEV), hx.to(DEV), h0.to(DEV), dt.to(DEV), lam.to(DEV), workspace=ws)
+    torch.cuda.synchronize()
+    assert rel_err(h, oracle.mingru_decay(k, hx, h0, dt, lam)) <= TOL[dtype]
+
+
+# Gaps and rates through the copy engine (16-byte aligned starts, a batch
+# stride that is a multiple of 4) or, otherwise, plain loads: a padded
+# stride, an odd one, an unaligned start of the gaps or of the rates, and a
+# single batch row whose length is not a multiple of 4.
+@pytest.mark.parametrize("B,pad,gap_off,lam_off", [(3, 3, 0, 0), (3, 1, 0, 0), (3, 0, 1, 0),
+                                                   (3, 3, 0, 1), (1, 0, 0, 0)])
+@pytest.mark.parametrize("kernel", [2, 3])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decay_gap_layouts(B, pad, gap_off, lam_off, kernel, dtype):
+    sgr.set_kernel_override(kernel)
+    sgr.set_tile_override(0, 4)
+    T, D = 2501, 160
+    k, hx, h0, dt, lam = data(B, T, D, dtype, "u01_1", seed=11 + pad + gap_off + lam_off, wipe_at=1200)
+    gstore = torch.full((B, T + pad + gap_off), float("nan"), device=DEV)
+    gaps = gstore[:, gap_off:gap_off + T]
+    gaps.copy_(dt.to(DEV))
+    lstore = torch.full((D + lam_off,), float("nan"), device=DEV)
+    rates = lstore[lam_off:]
+    rates.copy_(lam.to(DEV))
+    h = sgr.mingru_scan_decay(k.to(DEV), hx.to(DEV), h0.to(DEV), gaps, rates)
+    torch.cuda.synchronize()
+    assert rel_err(h, oracle.mingru_decay(k, hx, h0, dt, lam)) <= TOL[dtype]
+
+
 def test_decay_zero_gaps_equal_plain_scan():
     k, hx, h0, dt, lam = data(2, 3000, 256, "f32", "u01_1", seed=3)
     z = torch.zeros_like(dt)
