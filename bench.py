@@ -153,6 +153,16 @@ class ClockSampler:
             pw = None
         return sm, rs, pw
 
+    def sample_now(self):
+        """One sample from the calling thread (see timed_launches)."""
+        if not self.ok:
+            return
+        try:
+            sm, rs, pw = self._read()
+            self.samples.append((time.time(), sm, rs, pw))
+        except Exception:
+            pass
+
     def start(self):
         if not self.ok:
             return self
@@ -241,9 +251,13 @@ def aggregate(bytes_per_step: int, elems_per_step: int, steps: int, max_seconds:
 
 # ---------------------------------------------------------------- GPU timing
 
-def timed_launches(fn, steps: int, stream):
+def timed_launches(fn, steps: int, stream, while_busy=None):
     """Time `steps` calls of fn with CUDA events on the launching stream: the
-    whole region and each launch.  Returns (total_s, mean_launch_s)."""
+    whole region and each launch.  Returns (total_s, mean_launch_s).
+    `while_busy`, if given, is called on the host between the last launch
+    being queued and the stream reaching its end (the clock sampler reads
+    NVML there, so that its samples fall inside the timed region however
+    short it is)."""
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     t0 = torch.cuda.Event(enable_timing=True)
@@ -254,6 +268,10 @@ def timed_launches(fn, steps: int, stream):
         fn()
         ends[i].record(stream)
     t1.record(stream)
+    if while_busy is not None:
+        while not t1.query():
+            while_busy()
+            time.sleep(2e-4)
     torch.cuda.synchronize()
     total = t0.elapsed_time(t1) / 1e3
     per = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends)) / 1e3
@@ -623,7 +641,7 @@ def run_b200(args):
     barrier(world, device)
     torch.cuda.synchronize()
     h0 = time.time()
-    total, per_launch = timed_launches(fn, args.steps, stream)
+    total, per_launch = timed_launches(fn, args.steps, stream, while_busy=clocks.sample_now)
     h1 = time.time()
     barrier(world, device)
     clocks.stop()

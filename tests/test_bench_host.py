@@ -58,3 +58,53 @@ def test_cpu_baseline_record():
     assert r["kind"] == "oracle" and r["unit"] == bench.UNIT
     assert r["value"] > 0 and r["cores"] >= 1 and 1 <= r["passes"] <= 50
     assert r["cpu_seconds"] >= 0 and "batch rows" in r["sample"]
+
+
+def test_clock_samples_taken_inside_the_timed_region():
+    # a fake NVML reading: samples from the calling thread carry the reasons
+    # bits, and the summary keeps those inside the window
+    c = bench.ClockSampler.__new__(bench.ClockSampler)
+    c.samples, c.ok, c.max_mhz = [], True, 1965
+    c._read = lambda: (1965, 0x4, 500.0)
+    t0 = bench.time.time()
+    for _ in range(3):
+        c.sample_now()
+    t1 = bench.time.time()
+    c.samples.append((t1 + 10.0, 900, 0x40, 100.0))      # after the window: ignored
+    r = c.summary(t0, t1)
+    assert r["samples"] == 3 and r["window"] == "timed region"
+    assert r["sm_mhz"] == 1965 and r["reasons"] == ["sw_power_cap"] and r["power_w_max"] == 500.0
+    # NVML missing: no samples, clocks reported as unknown
+    c.ok = False
+    c.sample_now()
+    assert c.summary(t0, t1)["sm_mhz"] is None
+
+
+def test_timed_launches_samples_until_the_stream_is_done(monkeypatch):
+    # fake CUDA events: the end event completes after a few queries
+    class Ev:
+        polls = 0
+
+        def __init__(self, enable_timing=True):
+            pass
+
+        def record(self, stream):
+            pass
+
+        def query(self):
+            Ev.polls += 1
+            return Ev.polls > 4
+
+        def elapsed_time(self, other):
+            return 2.0
+
+    monkeypatch.setattr(bench.torch.cuda, "Event", Ev)
+    monkeypatch.setattr(bench.torch.cuda, "synchronize", lambda: None)
+    calls, seen = [], []
+    total, per = bench.timed_launches(lambda: calls.append(1), 3, None, while_busy=lambda: seen.append(1))
+    assert len(calls) == 3 and len(seen) == 4
+    assert total == 2e-3 and per == 2e-3
+    Ev.polls = 0
+    bench.timed_launches(lambda: None, 2, None)             # no sampler: no queries
+    assert Ev.polls == 0
+
