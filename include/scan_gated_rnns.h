@@ -255,7 +255,8 @@ SGR_API sgr_status_t sgr_combine_summaries(sgr_op_t op, const float *pairs, int6
  *             when B > 1)
  *   lambda  : fp32 DEVICE array (D,), decay rates >= 0 (fixed or learnable)
  * Other arguments, workspace and errors as mingru_scan (the same workspace
- * size).  Arithmetic fp32; the gate uses the MUFU exp2 like the activations.
+ * size); h must not overlap delta_t or lambda either (SGR_ERR_INVALID_ARG).
+ * Arithmetic fp32; the gate uses the MUFU exp2 like the activations.
  * Kernel: never the channel-sequential one (it would wait for the gaps one row
  * at a time); the chunked kernels with 4 rows per thread, so the plan that
  * sgr_scan_plan reports for SGR_OP_MINGRU may differ.  With delta_t and lambda
@@ -279,6 +280,8 @@ SGR_API sgr_status_t mingru_scan_decay(const void *k, const void *hx,
  * dgamma/dlambda = -u gamma (0 where the 1e4 clamp wipes).  dlambda is
  * overwritten; its sums use atomic adds, so their rounding order varies from
  * run to run.  No gradient with respect to delta_t (the gaps are data).
+ * No output may overlap delta_t or lambda, and dlambda may overlap no other
+ * operand (SGR_ERR_INVALID_ARG).
  * Workspace: sgr_backward_workspace_size(SGR_OP_MINGRU, ...).
  */
 SGR_API sgr_status_t mingru_scan_decay_backward(const void *k, const void *hx,

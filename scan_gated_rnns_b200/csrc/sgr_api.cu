@@ -578,6 +578,20 @@ sgr_status_t check_decay(const DecayArgs *dec, int64_t B, int64_t T, int64_t D) 
     return SGR_OK;
 }
 
+// bytes the gaps span (B rows of T, batch stride dt_bs; sizes checked by
+// check_decay) and the rates span
+size_t decay_gap_bytes(const DecayArgs &dec, int64_t B, int64_t T) {
+    return size_t((B - 1) * dec.dt_bs + T) * sizeof(float);
+}
+size_t decay_lam_bytes(int64_t D) { return size_t(D) * sizeof(float); }
+
+// an output written while the gaps and rates are still being read must not
+// share memory with them
+bool overlaps_decay(const DecayArgs *dec, const void *out, size_t n, int64_t B, int64_t T, int64_t D) {
+    return dec && (overlaps(out, n, dec->dt, decay_gap_bytes(*dec, B, T)) ||
+                   overlaps(out, n, dec->lam, decay_lam_bytes(D)));
+}
+
 void set_decay(ScanParams &sp, const DecayArgs *dec) {
     if (!dec) return;
     sp.decay_dt = dec->dt;
@@ -604,7 +618,8 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
     if (init && !mul_ok(B - 1, init_bs, &init_span_elems)) return SGR_ERR_UNSUPPORTED;
     const size_t tb = size_t(nbytes);
     const size_t ib = init ? rows_span(B, D, init_bs, esz) : 0;
-    if (overlaps(out, tb, in0, tb) || overlaps(out, tb, in1, tb) || overlaps(out, tb, init, ib))
+    if (overlaps(out, tb, in0, tb) || overlaps(out, tb, in1, tb) || overlaps(out, tb, init, ib) ||
+        overlaps_decay(dec, out, tb, B, T, D))
         return SGR_ERR_INVALID_ARG;
 
     const bool aligned = aligned16(in0) && aligned16(in1) && aligned16(out);
@@ -786,6 +801,19 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
     }
     if (overlaps(out0, tb, out1, tb) || overlaps(out0, tb, dinit, db) || overlaps(out1, tb, dinit, db))
         return SGR_ERR_INVALID_ARG;
+    if (overlaps_decay(dec, out0, tb, B, T, D) || overlaps_decay(dec, out1, tb, B, T, D) ||
+        overlaps_decay(dec, dinit, db, B, T, D))
+        return SGR_ERR_INVALID_ARG;
+    if (dec && dlam) {
+        // dL/dlambda is cleared and accumulated while everything else is read
+        // or written: it shares memory with none of it
+        const size_t lb = decay_lam_bytes(D);
+        if (overlaps_decay(dec, dlam, lb, B, T, D) || overlaps(dlam, lb, out0, tb) ||
+            overlaps(dlam, lb, out1, tb) || overlaps(dlam, lb, dinit, db))
+            return SGR_ERR_INVALID_ARG;
+        for (int i = 0; i < 5; ++i)
+            if (overlaps(dlam, lb, ins[i], in_bytes[i])) return SGR_ERR_INVALID_ARG;
+    }
 
     const bool aligned = aligned16(in0) && aligned16(in1) && aligned16(fwd) && aligned16(gy) &&
                          aligned16(out0) && aligned16(out1);
@@ -808,8 +836,6 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
     bp.out1 = out1; bp.dinit = dinit; bp.dinit_bs = dinit_bs;
     set_decay(sp, dec);
     bp.dlam = dec ? dlam : nullptr;
-    if (bp.dlam && overlaps(bp.dlam, size_t(D) * sizeof(float), out0, tb)) return SGR_ERR_INVALID_ARG;
-    if (bp.dlam && overlaps(bp.dlam, size_t(D) * sizeof(float), out1, tb)) return SGR_ERR_INVALID_ARG;
     if (seq) {
         // one warp per channel group over the whole sequence: no hand-off
         // words; a workspace, when given, receives the status word

@@ -412,6 +412,25 @@ def test_decay_argument_errors():
             2, 4, 8, F32, None, 0, None)
     assert db(*args) == E               # overlapping gap rows
 
+    # outputs sharing memory with the gaps or the rates, and dL/dlambda
+    # sharing memory with any operand: refused before anything is queued
+    span = 2 * 4 * 8 * 4                                       # one (2, 4, 8) fp32 tensor
+    assert call(dt=C + 16) == E
+    assert call(lam=C + span - 4) == E
+    big = dict(B=2, T=1 << 16, D=64, dbs=1 << 16)              # chunked: needs a workspace
+    assert call(dt=C + 2 * (1 << 16) * 64 * 4, **big) == _abi.SGR_ERR_WORKSPACE   # adjacent, no overlap
+    ok = list(args)
+    ok[5] = 4                                                  # gap rows of 4: no overlap among them
+    ok[13] = 8                                                 # dh0 rows of D (used when dh0 is set)
+    for i, v in ((14, A + 4), (14, G + 4), (14, L + 4), (14, 0x90000000 + 4), (14, C + 4),
+                 (10, L), (10, G + 8), (11, L + 16), (12, G)):
+        bad = list(ok)
+        bad[i] = v
+        assert db(*bad) == E, (i, hex(v))
+    ok[15:18] = [2, 1 << 16, 64]
+    ok[5] = 1 << 16
+    assert db(*ok) == _abi.SGR_ERR_WORKSPACE                   # distinct buffers pass the checks
+
 
 def test_summary_and_combine_argument_errors():
     lib = _abi.lib()
