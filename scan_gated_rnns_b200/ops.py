@@ -42,21 +42,24 @@ def _seq(t: torch.Tensor, name: str) -> None:
 
 
 def _rows(t: Optional[torch.Tensor], B: int, D: int, like: torch.Tensor, name: str) -> Tuple[int, int]:
-    """(pointer, batch stride in elements) of a (B, D) or (D,) operand."""
+    """(pointer, batch stride in elements) of a (B, D) or (D,) operand.  (On
+    the decode step's path: one stride tuple and integer device indices keep
+    it to a few attribute reads.)"""
     if t is None:
         return 0, 0
     _need_cuda(t, name)
-    if t.dtype != like.dtype or t.device != like.device:
+    if t.dtype != like.dtype or t.get_device() != like.get_device():
         raise ValueError(f"{name} must have dtype {like.dtype} on {like.device}")
-    if t.dim() == 1:
-        if t.shape[0] != D or (D > 1 and t.stride(0) != 1):
+    st = t.stride()
+    if len(st) == 1:
+        if t.shape[0] != D or (D > 1 and st[0] != 1):
             raise ValueError(f"{name} must be a contiguous (D,) vector")
         return t.data_ptr(), 0
-    if t.dim() != 2 or tuple(t.shape) != (B, D):
+    if len(st) != 2 or t.shape != (B, D):
         raise ValueError(f"{name} must be (B, D) = ({B}, {D}), got {tuple(t.shape)}")
-    if D > 1 and t.stride(1) != 1:
+    if D > 1 and st[1] != 1:
         raise ValueError(f"{name} rows must be contiguous along D")
-    return t.data_ptr(), (t.stride(0) if B > 1 else D)
+    return t.data_ptr(), (st[0] if B > 1 else D)
 
 
 class Workspace:
