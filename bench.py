@@ -290,14 +290,6 @@ def plan_kernel(plan) -> str:
             4: "sgr::scan_sequential_kernel"}.get(plan["kernel"], "sgr::scan_kernel")
 
 
-def decay_kernel(plan) -> str:
-    """The device kernel the time-decayed minGRU launches, given the plain
-    scan's plan: the same, except that it never takes the channel-sequential
-    kernel and runs the pipelined one there (wide batches always have the
-    tiles for it)."""
-    return plan_kernel({"kernel": 2 if plan["kernel"] == 4 else plan["kernel"]})
-
-
 def backward_kernel(w) -> str:
     """The device kernel the gradient of workload w launches."""
     import scan_gated_rnns_b200 as sgr
@@ -414,9 +406,9 @@ def measure_decay_rows(w, device, steps=10, warmup=3):
     bb = 6 * w.n_elems * w.elem_bytes + extra + w.D * 4 + \
         (2 * w.B * w.D * w.elem_bytes if init is not None else 0)
     del p, q, init, out, ws, gy, dt, lam
-    plan = sgr._abi.plan(0, w.B, w.T, w.D, 0 if w.dtype == "f32" else 1, True)
+    plan = sgr._abi.plan(0, w.B, w.T, w.D, 0 if w.dtype == "f32" else 1, True, decay=True)
     rows = {}
-    for kind, per, bytes_, kern in (("", per_f, fb, decay_kernel(plan)),
+    for kind, per, bytes_, kern in (("", per_f, fb, plan_kernel(plan)),
                                     ("_backward", per_b, bb, backward_kernel(w))):
         gbs = bytes_ / per / 1e9
         rows[w.name.replace("mingru_", f"mingru_decay{kind}_", 1)] = {

@@ -480,6 +480,13 @@ typedef struct sgr_plan {
 SGR_API sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D,
                                    sgr_dtype_t dtype, int aligned, sgr_plan_t *plan);
 
+/* The plan of mingru_scan_decay for this shape (the time-decayed minGRU may
+ * take another kernel than sgr_scan_plan(SGR_OP_MINGRU, ...) reports: never
+ * the channel-sequential one, 4 rows per thread).  `aligned` as above.  Pure
+ * host code. */
+SGR_API sgr_status_t sgr_scan_plan_decay(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
+                                         int aligned, sgr_plan_t *plan);
+
 /* Which kernel the gradient of this shape runs (mingru_scan_backward,
  * minmax_scan_backward and their time-decay forms): 1 the chunked tile kernel,
  * 4 the channel-sequential kernel (wide batches: one warp walks the whole

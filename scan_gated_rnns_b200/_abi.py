@@ -63,6 +63,7 @@ class Plan(ctypes.Structure):
 
 SIGNATURES.update({
     "sgr_scan_plan": (_int, [_int, _i64, _i64, _i64, _int, _int, ctypes.POINTER(Plan)]),
+    "sgr_scan_plan_decay": (_int, [_i64, _i64, _i64, _int, _int, ctypes.POINTER(Plan)]),
     "sgr_set_wait_limit": (_int, [ctypes.c_uint32]),
     "sgr_set_drop_publish": (_int, [_i64]),
     "sgr_set_kernel_override": (_int, [_int]),
@@ -116,9 +117,16 @@ def lib():
     return _lib
 
 
-def plan(op: int, B: int, T: int, D: int, dtype: int, aligned: bool = True) -> dict:
+def plan(op: int, B: int, T: int, D: int, dtype: int, aligned: bool = True, decay: bool = False) -> dict:
+    """The library's plan for a scan of this shape; decay: the time-decayed
+    minGRU's (op must then be SGR_OP_MINGRU)."""
     out = Plan()
-    check("sgr_scan_plan", lib().sgr_scan_plan(op, B, T, D, dtype, int(aligned), ctypes.byref(out)))
+    if decay:
+        if op != SGR_OP_MINGRU:
+            raise ValueError("plan: only the minGRU scan has a time-decayed form")
+        check("sgr_scan_plan_decay", lib().sgr_scan_plan_decay(B, T, D, dtype, int(aligned), ctypes.byref(out)))
+    else:
+        check("sgr_scan_plan", lib().sgr_scan_plan(op, B, T, D, dtype, int(aligned), ctypes.byref(out)))
     return out.as_dict()
 
 

@@ -1364,12 +1364,8 @@ const char *sgr_status_string(sgr_status_t s) {
 
 const char *sgr_version(void) { return "scan_gated_rnns_b200 0.1.0 sm_100a"; }
 
-sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
-                           int aligned, sgr_plan_t *plan) {
-    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return SGR_ERR_INVALID_ARG;
-    if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
-    if (B < 0 || T < 0 || D < 0 || !plan) return SGR_ERR_INVALID_ARG;
-    const Plan p = make_plan(B, T, D, dtype, aligned != 0, false, op == SGR_OP_MINMAX);
+namespace {
+void fill_plan(const Plan &p, sgr_plan_t *plan) {
     plan->vector_path = p.vec ? 1 : 0;
     plan->kernel = p.kind;
     plan->channels_per_thread = p.V;
@@ -1394,6 +1390,23 @@ sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dty
     } else {
         plan->div_chains_m = plan->div_chains_s = plan->div_dt_m = plan->div_dt_s = 0;
     }
+}
+}  // namespace
+
+sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
+                           int aligned, sgr_plan_t *plan) {
+    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return SGR_ERR_INVALID_ARG;
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || D < 0 || !plan) return SGR_ERR_INVALID_ARG;
+    fill_plan(make_plan(B, T, D, dtype, aligned != 0, false, op == SGR_OP_MINMAX), plan);
+    return SGR_OK;
+}
+
+sgr_status_t sgr_scan_plan_decay(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, int aligned,
+                                 sgr_plan_t *plan) {
+    if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || D < 0 || !plan) return SGR_ERR_INVALID_ARG;
+    fill_plan(make_plan(B, T, D, dtype, aligned != 0, false, false, true), plan);
     return SGR_OK;
 }
 

@@ -101,6 +101,29 @@ def test_step_argument_errors():
     assert lib.mingru_step(A, 8, Bp, 8, None, 0, C, 8, 0, 8, F32, None) == _abi.SGR_OK
 
 
+def test_decayed_plan():
+    # never the channel-sequential kernel; 4 rows per thread; bf16 with the
+    # 15-warp blocks wherever their tiles still give every SM 4 of them
+    for B, T, D, dtype in ((16, 2048, 2048, F32), (24, 2048, 2048, BF16), (8, 4096, 1024, BF16),
+                           (8, 4096, 1024, F32), (4, 8192, 512, BF16)):
+        plain = _abi.plan(MINGRU, B, T, D, dtype, True)
+        pl = _abi.plan(MINGRU, B, T, D, dtype, True, decay=True)
+        assert pl["kernel"] in (_abi.KERNEL_PIPELINED, _abi.KERNEL_PIPELINED_WIDE), (B, T, D, dtype)
+        assert pl["rows_per_thread"] == 4
+        if dtype == BF16:
+            assert pl["kernel"] == _abi.KERNEL_PIPELINED_WIDE and pl["warps"] == 15
+        assert pl["workspace_bytes"] <= _abi.lib().sgr_workspace_size(MINGRU, B, T, D, dtype)
+        assert plain["kernel"] != _abi.KERNEL_SEQUENTIAL or pl["workspace_bytes"] > 0
+    # small shapes: one launch per tile, as for the plain scan
+    assert _abi.plan(MINGRU, 2, 1024, 512, F32, True, decay=True)["kernel"] == _abi.KERNEL_TILE
+    # unaligned rows: the scalar tile kernel
+    assert _abi.plan(MINGRU, 8, 4096, 1024, F32, False, decay=True)["kernel"] == _abi.KERNEL_TILE
+    with pytest.raises(ValueError):
+        _abi.plan(MINMAX, 8, 4096, 1024, F32, True, decay=True)
+    lib = _abi.lib()
+    assert lib.sgr_scan_plan_decay(8, 4096, 1024, 7, 1, None) == _abi.SGR_ERR_INVALID_ARG
+
+
 def test_workspace_covers_the_decayed_plan():
     # wide batches: the plain plan needs no workspace, the time-decayed scan
     # (never channel-sequential) is cut along T and needs one

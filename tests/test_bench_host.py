@@ -44,13 +44,6 @@ def test_plan_kernel_names():
     assert bench.plan_kernel({"kernel": 4}) == "sgr::scan_sequential_kernel"
 
 
-def test_decay_kernel_names():
-    # the decayed scan keeps the plain plan's kernel except the channel-sequential one
-    assert bench.decay_kernel({"kernel": 4}) == "sgr::scan_pipelined_kernel"
-    assert bench.decay_kernel({"kernel": 3}) == "sgr::scan_pipelined_kernel"
-    assert bench.decay_kernel({"kernel": 1}) == "sgr::scan_tile_kernel"
-
-
 def test_cpu_baseline_record():
     w = Workload("t", "mingru", 2, 64, 32, "f32", seed=3, init="u01_1")
     p, q, i0 = generate(w)
