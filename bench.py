@@ -567,7 +567,13 @@ def cpu_baseline(w, p, q, init, budget_s: float = 12.0, cpu_target_s: float = 12
         fn(ps, qs, ins, threads=threads)
         wall += time.perf_counter() - t0
     bytes_ = (3 * rows * row * w.elem_bytes + (rows * w.D * w.elem_bytes if init is not None else 0)) * passes
+    # the first pass over one batch row ran on one thread: the single-core rate
+    one_bytes = 3 * row * w.elem_bytes + (w.D * w.elem_bytes if init is not None else 0)
+    single = {"value": round(one_bytes / max(one, 1e-9) / 1e9, 4), "unit": UNIT,
+              "gelem_per_s": round(row / max(one, 1e-9) / 1e9, 5), "seconds": round(one, 3),
+              "sample": f"batch row 0 ({w.T}x{w.D} elements), 1 thread, one pass"}
     return {"value": round(bytes_ / wall / 1e9, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "single_thread": single,
             "gelem_per_s": round(passes * rows * row / wall / 1e9, 5), "seconds": round(wall, 2),
             "cpu_seconds": round(wall * threads, 1), "passes": passes,
             "sample": f"batch rows 0..{rows - 1} of the workload ({rows}x{w.T}x{w.D} elements), "

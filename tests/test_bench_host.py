@@ -51,6 +51,8 @@ def test_cpu_baseline_record():
     assert r["kind"] == "oracle" and r["unit"] == bench.UNIT
     assert r["value"] > 0 and r["cores"] >= 1 and 1 <= r["passes"] <= 50
     assert r["cpu_seconds"] >= 0 and "batch rows" in r["sample"]
+    one = r["single_thread"]
+    assert one["value"] > 0 and one["unit"] == bench.UNIT and "1 thread" in one["sample"]
 
 
 def test_clock_samples_taken_inside_the_timed_region():
