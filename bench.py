@@ -538,11 +538,21 @@ def measure_step_row(device, B=8, D=1024, calls=200, warmup=10):
             "us_per_step_graph": round(g_per * 1e6, 2), "bytes_per_call": 4 * 4 * B * D}
 
 
+def usable_cores() -> int:
+    """CPUs this process may run on (its affinity mask where the platform has
+    one, else the logical CPU count), capped at 32 threads."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        n = os.cpu_count() or 1
+    return max(1, min(n, 32))
+
+
 def cpu_baseline(w, p, q, init, budget_s: float = 12.0, cpu_target_s: float = 12.0):
     """The fp64 CPU oracle as it stands, on a bounded sample of the workload:
     whole batch rows (all T and D of each), threads over rows."""
     import oracle
-    cores = max(1, min(os.cpu_count() or 1, 32))
+    cores = usable_cores()
     row = w.T * w.D
     # time one row first, then size the sample to about `budget_s` of wall time
     p1, q1 = p[:1].cpu(), q[:1].cpu()
@@ -578,7 +588,8 @@ def cpu_baseline(w, p, q, init, budget_s: float = 12.0, cpu_target_s: float = 12
             "cpu_seconds": round(wall * threads, 1), "passes": passes,
             "sample": f"batch rows 0..{rows - 1} of the workload ({rows}x{w.T}x{w.D} elements), "
                       f"{passes} pass(es), fp64 {'linear-space minGRU' if w.op == 'mingru' else 'MinMax'} "
-                      f"oracle, {threads} thread(s) over rows; host has {os.cpu_count()} logical CPUs"}
+                      f"oracle, {threads} thread(s) over rows; host has {os.cpu_count()} logical CPUs, "
+                      f"{usable_cores()} usable by this process (affinity mask, capped at 32)"}
 
 
 # ------------------------------------------------------------------- arms
@@ -771,7 +782,7 @@ def run_reference(args):
         p, q, init = generate(w, device=dev)
     else:
         p, q, init = generate(w.scaled(B=1))
-    cores = max(1, min(os.cpu_count() or 1, 32))
+    cores = usable_cores()
     # one step = the oracle over one batch row (T x D elements) per thread
     rows = max(1, min(w.B, cores))
     ps, qs = p[:rows].cpu(), q[:rows].cpu()

@@ -44,6 +44,13 @@ def test_plan_kernel_names():
     assert bench.plan_kernel({"kernel": 4}) == "sgr::scan_sequential_kernel"
 
 
+def test_usable_cores_follow_the_affinity_mask(monkeypatch):
+    monkeypatch.setattr(bench.os, "sched_getaffinity", lambda pid: {0, 2, 5})
+    assert bench.usable_cores() == 3
+    monkeypatch.setattr(bench.os, "sched_getaffinity", lambda pid: set(range(100)))
+    assert bench.usable_cores() == 32
+
+
 def test_cpu_baseline_record():
     w = Workload("t", "mingru", 2, 64, 32, "f32", seed=3, init="u01_1")
     p, q, i0 = generate(w)
