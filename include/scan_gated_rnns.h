@@ -55,24 +55,29 @@
  *
  * Workspace (mingru_scan, minmax_scan)
  * ------------------------------------
- *  Long sequences are cut into chunks of T that run on different thread
- *  blocks; each chunk receives its carried state from the chunks before it
- *  through a small device workspace (flags and per-chunk summaries) that stays
- *  in L2.  sgr_workspace_size() gives the bytes a call needs (0 when the whole
- *  sequence fits one chunk, in which case workspace may be NULL).  Before its
- *  first use a workspace must be zero-filled once (sgr_workspace_init or
- *  cudaMemset); afterwards calls keep it valid.  One workspace must not be used
- *  by two calls that can run at the same time (e.g. on two streams).
- *  Calls may be captured in a CUDA graph; a captured call zero-fills the flag
- *  region itself inside the graph.
+ *  Every non-empty call takes a small device workspace: a 256-byte header
+ *  whose first 4 bytes are the status word of the kernels' bounded waits
+ *  (read by sgr_workspace_status), followed, when the sequence is cut into
+ *  chunks of T that run on different thread blocks, by the words through
+ *  which each chunk receives its carried state from the chunks before it
+ *  (per-chunk summaries and states tagged with the launch; they stay in L2).
+ *  sgr_workspace_size() gives the bytes a call needs: 256 when the whole
+ *  sequence runs as one chunk, more when it is cut; 0 only for an empty
+ *  shape, in which case workspace may be NULL.  Before its first use a
+ *  workspace must be zero-filled once (sgr_workspace_init or cudaMemset);
+ *  afterwards calls keep it valid.  One workspace must not be used by two
+ *  calls that can run at the same time (e.g. on two streams).
+ *  Calls may be captured in a CUDA graph; a captured call zero-fills the
+ *  hand-off words itself inside the graph.  When one block per chunk is
+ *  launched (the tile kernels), the call also zeroes a ticket counter in the
+ *  header on `stream` before the launch: blocks take their chunk numbers from
+ *  it in the order they start, so no chunk ever waits for one whose block has
+ *  not started.
  *  Wide batches (B x D large enough that groups of 32 channels give every SM
  *  several warps) are not cut along T at all: each warp scans its 32 channels
- *  over the whole sequence, and the plan needs no workspace.  The
+ *  over the whole sequence, and the plan needs only the header.  The
  *  time-decayed minGRU (mingru_scan_decay) is always cut along T when T spans
- *  several chunks; sgr_workspace_size(SGR_OP_MINGRU, ...) covers it too, so
- *  it may be > 0 for such shapes.
- *  A workspace passed to such a call anyway (>= 4 bytes, 16-byte aligned)
- *  receives the status word of its bounded waits.
+ *  several chunks; sgr_workspace_size(SGR_OP_MINGRU, ...) covers it too.
  */
 #ifndef SCAN_GATED_RNNS_H
 #define SCAN_GATED_RNNS_H
@@ -168,7 +173,10 @@ SGR_API sgr_status_t mingru_step(const void *k_t, int64_t k_batch_stride,
  * SGR_ERR_WORKSPACE.  The first call on a device looks up the array's device
  * address and zero-fills it on `stream`, so make it before any stream capture.
  * All calls on a device share the array: calls whose kernels can overlap on
- * the GPU race and must not be made.
+ * the GPU race and must not be made.  The array's status word is internal:
+ * each call clears it on `stream` before its launch and nothing reads it
+ * back, so a chunk that gave up waiting (SGR_ERR_TIMEOUT with mingru_scan)
+ * shows only as NaN outputs here.
  */
 SGR_API sgr_status_t mingru_scan_noalloc(const void *k, const void *hx,
                                          const void *h0, int64_t h0_batch_stride,
@@ -218,7 +226,9 @@ SGR_API sgr_status_t mingru_projected_scan(const void *x, const void *w,
  * sgr_scan_summary: pairs (B, D, 2) fp32 (A, B or U, L), DEVICE, for the
  *   slice in0, in1 (B, T, D); T = 0 gives the identity pair.  Workspace:
  *   sgr_summary_workspace_size(B, T, D, dtype) bytes of device memory (no
- *   initialisation needed).  Reads the inputs once.
+ *   initialisation needed): a 256-byte header whose first 4 bytes receive the
+ *   status word of the bounded waits (sgr_workspace_status reads it), then
+ *   per-segment partial pairs.  Reads the inputs once.
  * sgr_combine_summaries: out (B, D) rows (batch stride out_bs, I/O dtype) =
  *   the state entering slice `rank`, from pairs (n, B, D, 2) fp32 of all
  *   slices in rank order (only the first `rank` are read) and the initial
@@ -348,7 +358,8 @@ SGR_API sgr_status_t minmax_scan_backward(const void *r, const void *s,
                                           int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
                                           void *workspace, size_t ws_bytes, cudaStream_t stream);
 
-/* Bytes of workspace a gradient call of this shape needs (0: none).  Pure host code. */
+/* Bytes of workspace a gradient call of this shape needs (at least the 256-byte
+ * header for a non-empty shape).  Pure host code. */
 SGR_API size_t sgr_backward_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D,
                                            sgr_dtype_t dtype);
 
@@ -404,7 +415,8 @@ SGR_API sgr_status_t minmax_scan_host(const void *r, const void *s,
 
 /* ------------------------------------------------------------ workspace */
 
-/* Bytes of workspace a scan of this shape needs (0: none).  Pure host code. */
+/* Bytes of workspace a scan of this shape needs: at least the 256-byte header
+ * for any non-empty shape, 0 for an empty one.  Pure host code. */
 SGR_API size_t sgr_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D,
                           sgr_dtype_t dtype);
 
@@ -469,8 +481,8 @@ typedef struct sgr_plan {
     int64_t n_chunks;           /* tiles along T                                   */
     int64_t n_tiles;            /* n_chains * n_chunks                             */
     uint64_t smem_bytes;        /* dynamic shared memory per block                 */
-    uint64_t workspace_bytes;   /* 0 when n_chunks == 1                            */
-    uint64_t off_words;         /* workspace offset of the hand-off words          */
+    uint64_t workspace_bytes;   /* 256 (the header) when n_chunks == 1             */
+    uint64_t off_words;         /* workspace offset of the hand-off words (256)    */
     uint32_t div_chains_m, div_chains_s;  /* tile -> chunk division constants   */
     uint32_t div_dt_m, div_dt_s;          /* chain -> batch division constants  */
 } sgr_plan_t;

@@ -93,6 +93,8 @@ KERNEL_TILE = 1
 KERNEL_PIPELINED = 2
 KERNEL_PIPELINED_WIDE = 3
 KERNEL_SEQUENTIAL = 4
+KERNEL_SEQUENTIAL_SPLIT = 5
+KERNEL_SEQUENTIAL_PAIR = 6
 
 _lock = threading.Lock()
 _lib = None

@@ -332,6 +332,7 @@ struct ScanParams {
     FastDiv by_dt;        // chain -> (b, dt)
     uint64_t *words;      // [n_tiles][3][TC] hand-off words (workspace)
     uint32_t *status;     // device status word
+    uint32_t *ticket;     // chunk ticket counter, zero at launch (tile kernels), or null: tile = blockIdx.x
     uint32_t epoch;
     uint32_t spin_limit;  // polls before a chunk gives up waiting
     int64_t drop_tile;    // testing: this tile does not publish (-1: none)
@@ -590,6 +591,17 @@ __device__ __forceinline__ void fold_warps(float2 (*s_tot)[TC], int ch, float2 (
     }
 }
 
+// The tile a block works on: the next ticket when the launch hands tiles out
+// in start order (one atomic per block, broadcast through shared memory;
+// every thread of the block must call this), else blockIdx.x.
+__device__ __forceinline__ int64_t take_tile(uint32_t *ticket) {
+    if (ticket == nullptr) return blockIdx.x;
+    __shared__ uint32_t s_ticket;
+    if (threadIdx.x == 0) s_ticket = atomicAdd(ticket, 1u);
+    __syncthreads();
+    return s_ticket;
+}
+
 // -------------------------------------------------------- tile kernel
 //
 // One block per tile (TR rows x TC channels), W data warps + 1 carry warp.
@@ -597,11 +609,15 @@ __device__ __forceinline__ void fold_warps(float2 (*s_tot)[TC], int ch, float2 (
 // 16-byte vector, or 1 for the scalar variant), CG (lanes across channels),
 // R (rows per thread), W (data warps).  J = 32 / CG row groups per warp,
 // TR = W * J * R, TC = CG * V.  Tiles are numbered chain-fastest:
-// blockIdx.x = chunk * n_chains + chain, chain = b * n_dt + dt.  Blocks are
-// dispatched in increasing index order and a block publishes its summary
-// before it waits, so every wait is for a block that started earlier and waits
-// never form a cycle.  Used for the scalar (unaligned) variant and as a
-// cross-check of the pipelined kernel.
+// tile = chunk * n_chains + chain, chain = b * n_dt + dt.  When the sequence
+// spans several chunks a block does not take the tile of its blockIdx: it
+// takes the next number from a ticket counter in the workspace (zeroed in the
+// stream before the launch), so tiles are handed out in the order blocks
+// actually start, whatever order the hardware dispatches them in.  Every
+// look-back then waits only for tiles that running blocks already hold, and
+// a block publishes its summary before it waits, so waits never form a cycle.
+// Used for the scalar (unaligned) variant and as a cross-check of the
+// pipelined kernel.
 template <class Op, typename IO, int V, int CG, int R, int W, int MINB>
 __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const ScanParams p) {
     constexpr int J = 32 / CG;
@@ -616,7 +632,7 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const Sca
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int64_t tile = blockIdx.x;
+    const int64_t tile = take_tile(p.ticket);
 
     if (warp < W) {
         const TileCoord tc = tile_coord(p, uint32_t(tile));

@@ -96,14 +96,33 @@ struct SeqParams {
 
 // Block: WB independent warps; warp (blockIdx.x WB + w) scans channel group
 // (b, grp) of the batch.  Dynamic shared memory: WB x seq_warp_bytes(S).
-template <class Op, typename IO, int WB>
+//
+// SPLIT = 1: a warp's group is 32 channels, lane l owns channel l and walks
+// every row.  SPLIT = 2: a warp's group is 16 channels and each slot's rows
+// are split between the two half-warps, which doubles the warps a batch
+// provides (the kernel is bound by the latency each warp exposes, so twice
+// the warps hide it better) at the price of a fold and a hand-off per slot:
+// lane (c, part) = (lane % 16, lane / 16) owns channel c of rows
+// [8 part, 8 part + 8) of every slot.  Both halves fold their 8 step maps
+// into one pair; the lower half applies its pair to the slot's incoming
+// state, hands the result (the state after row 7) to the upper half with one
+// shuffle, the upper half applies its own pair to it and hands the slot's
+// final state back; then every lane replays its 8 rows from its incoming
+// state and stores them.  This is the chunked scan with two chunks per slot
+// (page "MinMax Recurrent Neural Cascades", Key properties: the pairs
+// compose associatively).  The two halves read rows 256 (bf16) or 512
+// (fp32) bytes apart, a 2-way shared-memory bank conflict per load.
+template <class Op, typename IO, int WB, int SPLIT = 1>
 __global__ void __launch_bounds__(WB * 32)
 scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap map0,
                        const __grid_constant__ CUtensorMap map1, const __grid_constant__ CUtensorMap map_out) {
+    static_assert(SPLIT == 1 || SPLIT == 2, "one or two row groups per slot");
     using LR = LaneRow<IO>;
-    constexpr int CW = 32;
-    constexpr int kRowBytes = seq_row_bytes<IO>();
+    constexpr int CW = 32 / SPLIT;                                   // channels of a warp's group
+    constexpr int LROWS = kSeqRows / SPLIT;                          // rows of a slot per lane
+    constexpr int kRowBytes = CW * int(sizeof(IO));
     constexpr uint32_t kOpBytes = kSeqRows * kRowBytes;             // one operand of a slot
+    static_assert(LROWS % 2 == 0, "rows are taken in pairs");
     const ScanParams &p = q.s;
     extern __shared__ __align__(128) unsigned char smem[];
 
@@ -115,12 +134,15 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
     const int64_t b = gw / q.n_groups;
     const int64_t grp = gw - b * q.n_groups;
     const int x0 = int(grp) * CW;                                    // first channel of the group
-    const int64_t d = int64_t(x0) + lane;                            // the lane's channel
+    const int ch = lane % CW;                                        // the lane's channel in the group
+    const int part = lane / CW;                                      // the lane's rows of a slot
+    const int64_t d = int64_t(x0) + ch;                              // the lane's channel
 
     const uint32_t base = smem_addr(smem) + uint32_t(warp * seq_warp_bytes(S, kRowBytes));
     const uint32_t ring = base;                                      // S slots: [k rows | hx rows]
     const uint32_t outb = base + uint32_t(S) * 2 * kOpBytes;         // 2 staging buffers
     const uint32_t bars = outb + kSeqOutBufs * kOpBytes;             // S mbarriers
+    const uint32_t lane_off = uint32_t(part * LROWS * kRowBytes + ch * int(sizeof(IO)));
 
     const int n_slots = int((p.T + kSeqRows - 1) / kSeqRows);       // T < 2^31 (host check)
     auto issue = [&](int i, int s) {                                 // lane 0: rows of slot i into ring slot s
@@ -137,7 +159,7 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
     }
     __syncwarp();
 
-    float h = load_init<IO>(p, b, d, Op::default_init());           // the lane's state
+    float h = load_init<IO>(p, b, d, Op::default_init());           // state entering the slot
     [[maybe_unused]] float lam2 = 0.f;
     if constexpr (Op::kDecay) lam2 = decay_lam2(p, d);
 
@@ -153,10 +175,10 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
             if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
             bad = true;
         }
-        const uint32_t src = ring + uint32_t(s) * 2 * kOpBytes + uint32_t(lane) * uint32_t(sizeof(IO));
-        float x0r[kSeqRows], x1r[kSeqRows];
+        const uint32_t src = ring + uint32_t(s) * 2 * kOpBytes + lane_off;
+        float x0r[LROWS], x1r[LROWS];
 #pragma unroll
-        for (int r = 0; r < kSeqRows; ++r) {
+        for (int r = 0; r < LROWS; ++r) {
             x0r[r] = LR::load(src + r * kRowBytes);
             x1r[r] = LR::load(src + kOpBytes + r * kRowBytes);
         }
@@ -173,18 +195,17 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
             phase ^= 1u;
         }
         const uint32_t obuf = outb + uint32_t(i & (kSeqOutBufs - 1)) * kOpBytes;
-        const uint32_t dst = obuf + uint32_t(lane) * uint32_t(sizeof(IO));
-        static_assert(kSeqRows % 2 == 0, "rows are taken in pairs");
+        const uint32_t dst = obuf + lane_off;
         if (__any_sync(0xffffffffu, bad)) {
             // a copy of this or an earlier slot never landed: NaN outputs
             bad = true;
 #pragma unroll
-            for (int r = 0; r < kSeqRows; ++r) LR::store(dst + r * kRowBytes, __int_as_float(0x7fffffff));
-        } else {
+            for (int r = 0; r < LROWS; ++r) LR::store(dst + r * kRowBytes, __int_as_float(0x7fffffff));
+        } else if constexpr (SPLIT == 1) {
             // the step maps of two rows at a time (independent of the
             // state), then the two steps
 #pragma unroll
-            for (int r = 0; r < kSeqRows; r += 2) {
+            for (int r = 0; r < LROWS; r += 2) {
                 float2 a, c;
                 Op::element_rows(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
                 if constexpr (Op::kDecay) {
@@ -197,11 +218,185 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
                 h = Op::step(a.y, c.y, h);
                 LR::store(dst + (r + 1) * kRowBytes, h);
             }
+        } else {
+            // the lane's step maps, their fold into one pair, the hand-off
+            // between the two halves, then the replay from the lane's state
+            float am[LROWS], cm[LROWS];
+#pragma unroll
+            for (int r = 0; r < LROWS; r += 2) {
+                float2 a, c;
+                Op::element_rows(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
+                if constexpr (Op::kDecay) {
+                    const int64_t t = int64_t(i) * kSeqRows + part * LROWS + r;
+                    a.x *= decay_gamma(lam2, t < p.T ? decay_u(p, b, t) : 0.f);
+                    a.y *= decay_gamma(lam2, t + 1 < p.T ? decay_u(p, b, t + 1) : 0.f);
+                }
+                am[r] = a.x; cm[r] = c.x;
+                am[r + 1] = a.y; cm[r + 1] = c.y;
+            }
+            float2 P = make_float2(am[0], cm[0]);
+#pragma unroll
+            for (int r = 1; r < LROWS; ++r) P = Op::combine(P, make_float2(am[r], cm[r]));
+            const float lo_out = Op::apply(P, h);                        // lower half: state after row LROWS-1
+            const float from_lo = __shfl_xor_sync(0xffffffffu, lo_out, 16);
+            const float hin = part ? from_lo : h;                        // the lane's incoming state
+            const float out = Op::apply(P, hin);                         // upper half: the slot's final state
+            const float from_hi = __shfl_xor_sync(0xffffffffu, out, 16);
+            h = part ? out : from_hi;
+            float y = hin;
+#pragma unroll
+            for (int r = 0; r < LROWS; ++r) {
+                y = Op::step(am[r], cm[r], y);
+                LR::store(dst + r * kRowBytes, y);
+            }
         }
         fence_proxy_async();                                         // outputs visible to the store
         __syncwarp();
         if (lane == 0) {
             tma_store_3d(&map_out, obuf, x0, i * kSeqRows, int(b));
+            bulk_commit();
+        }
+    }
+    if (lane == 0) bulk_wait_all();
+}
+
+// Two warps per channel group, each slot's rows split between them (wide bf16
+// batches whose 32-channel groups alone leave each SM short of warps): the
+// block's warps w = 0, 1 scan the same 32 channels of one batch row (lane =
+// channel, 64- or 128-byte rows, no bank conflicts), warp w taking rows
+// [32 i + 16 w, 32 i + 16 w + 16) of slot i through its own ring of 16-row
+// boxes.  Each warp folds its 16 step maps into one pair and puts it in
+// shared memory (double-buffered by slot parity); after one named barrier per
+// slot both warps read the other's pair and compose the slot's chain
+// themselves -- h_mid = P0(h), h_end = P1(h_mid) -- so no second hand-off is
+// needed: warp 0 replays its rows from h, warp 1 from h_mid, and both carry
+// h_end into the next slot.  A warp whose copy never landed publishes a NaN
+// pair, so both warps' later outputs turn NaN.  One staging buffer per warp
+// (its previous store has long finished reading it by the time the next
+// slot's outputs are written), which leaves the shared memory to the load
+// ring.  Dynamic shared memory: 2 x seq_pair_warp_bytes(S) + the pair buffers.
+constexpr int kPairWarps = 2;
+__host__ __device__ constexpr size_t seq_pair_warp_bytes(int S, int row_bytes) {
+    return (size_t(S) * 2 * kSeqRows * row_bytes + size_t(kSeqRows) * row_bytes + size_t(S) * 8 + 127) / 128 * 128;
+}
+__host__ __device__ constexpr size_t seq_pair_block_bytes(int S, int row_bytes) {
+    return kPairWarps * seq_pair_warp_bytes(S, row_bytes) + size_t(2) * kPairWarps * 32 * sizeof(float2);
+}
+
+template <class Op, typename IO>
+__global__ void __launch_bounds__(kPairWarps * 32)
+scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorMap map0,
+                            const __grid_constant__ CUtensorMap map1, const __grid_constant__ CUtensorMap map_out) {
+    using LR = LaneRow<IO>;
+    constexpr int CW = 32;
+    constexpr int kRowBytes = CW * int(sizeof(IO));
+    constexpr uint32_t kOpBytes = kSeqRows * kRowBytes;             // one operand of a warp's 16 rows
+    constexpr int kSlotRows = kPairWarps * kSeqRows;                // rows of a slot (both warps)
+    const ScanParams &p = q.s;
+    extern __shared__ __align__(128) unsigned char smem[];
+
+    const int lane = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5;
+    const int64_t gw = blockIdx.x;                                   // one channel group per block
+    if (gw >= q.n_warps) return;                                     // whole block: no barrier is left waiting
+    const int S = q.slots;
+    const int64_t b = gw / q.n_groups;
+    const int64_t grp = gw - b * q.n_groups;
+    const int x0 = int(grp) * CW;
+    const int64_t d = int64_t(x0) + lane;
+
+    const uint32_t base = smem_addr(smem) + uint32_t(w * seq_pair_warp_bytes(S, kRowBytes));
+    const uint32_t ring = base;
+    const uint32_t outb = base + uint32_t(S) * 2 * kOpBytes;        // one staging buffer
+    const uint32_t bars = outb + kOpBytes;
+    float2 *xpair = reinterpret_cast<float2 *>(smem + kPairWarps * seq_pair_warp_bytes(S, kRowBytes));  // [2][2][32]
+
+    const int n_slots = int((p.T + kSlotRows - 1) / kSlotRows);     // T < 2^31 (host check)
+    auto issue = [&](int i, int s) {
+        const uint32_t dst = ring + uint32_t(s) * 2 * kOpBytes;
+        const uint32_t bar = bars + 8u * uint32_t(s);
+        const int y = i * kSlotRows + w * kSeqRows;
+        mbar_expect_tx(bar, 2 * kOpBytes);
+        tma_load_3d(dst, &map0, x0, y, int(b), bar);
+        tma_load_3d(dst + kOpBytes, &map1, x0, y, int(b), bar);
+    };
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(bars + 8u * s, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int s = 0; s < S && s < n_slots; ++s) issue(s, s);
+    }
+    __syncwarp();
+
+    float h = load_init<IO>(p, b, d, Op::default_init());           // state entering the slot
+    [[maybe_unused]] float lam2 = 0.f;
+    if constexpr (Op::kDecay) lam2 = decay_lam2(p, d);
+
+    uint32_t wait_limit = kMbarLimit;
+    bool bad = false;
+    int s = 0;
+    uint32_t phase = 0;
+    for (int i = 0; i < n_slots; ++i) {
+        if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
+            wait_limit = 1;
+            if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
+            bad = true;
+        }
+        const uint32_t src = ring + uint32_t(s) * 2 * kOpBytes + uint32_t(lane) * uint32_t(sizeof(IO));
+        float x0r[kSeqRows], x1r[kSeqRows];
+#pragma unroll
+        for (int r = 0; r < kSeqRows; ++r) {
+            x0r[r] = LR::load(src + r * kRowBytes);
+            x1r[r] = LR::load(src + kOpBytes + r * kRowBytes);
+        }
+        __syncwarp();                                                // the slot is in registers
+        if (lane == 0 && !bad && i + S < n_slots) {
+            fence_proxy_async();
+            issue(i + S, s);
+        }
+        if (++s == S) {
+            s = 0;
+            phase ^= 1u;
+        }
+        bad = __any_sync(0xffffffffu, bad);
+        float am[kSeqRows], cm[kSeqRows];
+#pragma unroll
+        for (int r = 0; r < kSeqRows; r += 2) {
+            float2 a, c;
+            Op::element_rows(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
+            if constexpr (Op::kDecay) {
+                const int64_t t = int64_t(i) * kSlotRows + w * kSeqRows + r;
+                a.x *= decay_gamma(lam2, t < p.T ? decay_u(p, b, t) : 0.f);
+                a.y *= decay_gamma(lam2, t + 1 < p.T ? decay_u(p, b, t + 1) : 0.f);
+            }
+            am[r] = a.x; cm[r] = c.x;
+            am[r + 1] = a.y; cm[r + 1] = c.y;
+        }
+        float2 P = make_float2(am[0], cm[0]);
+#pragma unroll
+        for (int r = 1; r < kSeqRows; ++r) P = Op::combine(P, make_float2(am[r], cm[r]));
+        if (bad) P = make_float2(__int_as_float(0x7fffffff), __int_as_float(0x7fffffff));
+        float2 *xb = xpair + (i & 1) * kPairWarps * 32;
+        xb[w * 32 + lane] = P;
+        named_barrier_sync(1, kPairWarps * 32);                      // both warps' pairs of slot i written
+        const float2 Q = xb[(1 - w) * 32 + lane];
+        const float hmid = Op::apply(w ? Q : P, h);
+        const float hend = Op::apply(w ? P : Q, hmid);
+        float y = w ? hmid : h;
+        h = hend;
+        if (lane == 0) bulk_wait_read<0>();                          // the last slot's store has read the buffer
+        __syncwarp();
+        const uint32_t obuf = outb;
+        const uint32_t dst = obuf + uint32_t(lane) * uint32_t(sizeof(IO));
+#pragma unroll
+        for (int r = 0; r < kSeqRows; ++r) {
+            y = Op::step(am[r], cm[r], y);
+            LR::store(dst + r * kRowBytes, y);
+        }
+        fence_proxy_async();
+        __syncwarp();
+        const int y0 = i * kSlotRows + w * kSeqRows;
+        if (lane == 0 && y0 < p.T) {                                  // no store starts past the tensor
+            tma_store_3d(&map_out, obuf, x0, y0, int(b));
             bulk_commit();
         }
     }

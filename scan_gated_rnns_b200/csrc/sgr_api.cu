@@ -31,8 +31,13 @@ constexpr int kStages = 3;
 constexpr int kAssumedSMs = 148;     // B200; only used to pick a tile shape
 constexpr int64_t kTargetTiles = 4 * 148;  // tile kernel: prefer >= 4 tiles per SM
 constexpr size_t kAlign = 256;
+// Workspace header, [0, 256): the status word of the bounded waits at byte 0,
+// the tile kernels' chunk ticket counter at byte 64 (its own 32-byte sector).
+// Every non-empty scan plan has the header; hand-off words follow it.
+constexpr size_t kTicketOffset = 64;
 
-enum Kind { KIND_AUTO = 0, KIND_TILE = 1, KIND_PIPELINED = 2, KIND_PIPELINED_WIDE = 3, KIND_SEQUENTIAL = 4 };
+enum Kind { KIND_AUTO = 0, KIND_TILE = 1, KIND_PIPELINED = 2, KIND_PIPELINED_WIDE = 3, KIND_SEQUENTIAL = 4,
+            KIND_SEQUENTIAL_SPLIT = 5, KIND_SEQUENTIAL_PAIR = 6 };
 
 // Channel-sequential kernel (scan_sequential.cuh): one warp per 32-channel
 // group walks the whole sequence.  Chosen when the groups alone give every SM
@@ -78,6 +83,7 @@ struct Plan {
     int esz = 4;          // bytes per stored element
     bool vec = false;     // 128-bit path
     int kind = KIND_TILE;
+    int split = 1;        // channel-sequential: row groups per slot (1, or 2 half-warps)
     int V = 1;            // channels per thread
     int cg = 32;          // lanes across channels
     int r = 2;            // rows per thread
@@ -181,6 +187,25 @@ SeqLayout seq_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, siz
     return l;
 }
 
+// the two-warp blocks of scan_sequential_pair_kernel: one block per channel
+// group, the block's share of the SM's shared memory split between its warps
+SeqLayout seq_pair_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, size_t reserved,
+                          size_t smem_block_max) {
+    SeqLayout l;
+    const int64_t K = sms > 0 ? (groups + sms - 1) / sms : 1;
+    size_t alloc = seq_pair_block_bytes(4, row_bytes);
+    if (K >= 1 && K <= 16) {
+        const size_t share = smem_sm / size_t(K);
+        alloc = share > reserved ? (share - reserved) / 128 * 128 : 0;
+    }
+    alloc = std::min(alloc, smem_block_max);
+    int S = kSeqMaxSlots;
+    while (S > kSeqMinSlots && seq_pair_block_bytes(S, row_bytes) > alloc) --S;
+    l.slots = S;
+    l.smem = std::max(alloc, seq_pair_block_bytes(S, row_bytes));
+    return l;
+}
+
 // Tile shape of a scan.  Aligned vector-width rows take the pipelined kernel
 // (fp32: 7 x 4 x R rows x 32 channels; bf16: 7 x 2 x R rows x 64 channels;
 // 128-byte row segments); anything else takes the tile kernel's scalar
@@ -209,24 +234,35 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
         const bool seq_ok = p.vec && !force_tile && T <= int64_t(std::numeric_limits<int>::max()) &&
                             B <= int64_t(std::numeric_limits<int>::max());
         const int min_per_sm = p.esz == 2 ? kSeqMinWarpsPerSMHalf : kSeqMinWarpsPerSM;
-        const bool want = ok == KIND_SEQUENTIAL ||
+        const bool want = ok == KIND_SEQUENTIAL || ok == KIND_SEQUENTIAL_SPLIT || ok == KIND_SEQUENTIAL_PAIR ||
                           (ok == KIND_AUTO && !decay && groups >= int64_t(min_per_sm) * kAssumedSMs);
         if (seq_ok && want) {
-            const SeqLayout lay = seq_layout(groups, int(cw) * p.esz, kAssumedSMs, kAssumedSmemPerSM,
-                                             kAssumedSmemReserved, kAssumedSmemPerBlock);
-            p.kind = KIND_SEQUENTIAL;
+            const bool split = ok == KIND_SEQUENTIAL_SPLIT;
+            const bool pair = ok == KIND_SEQUENTIAL_PAIR;
+            const int64_t gw = split ? cw / 2 : cw;                 // channels per warp
+            const int64_t n_warps = B * ((D + gw - 1) / gw);
+            const SeqLayout lay = pair ? seq_pair_layout(n_warps, int(gw) * p.esz, kAssumedSMs, kAssumedSmemPerSM,
+                                                         kAssumedSmemReserved, kAssumedSmemPerBlock)
+                                       : seq_layout(n_warps, int(gw) * p.esz, kAssumedSMs, kAssumedSmemPerSM,
+                                                    kAssumedSmemReserved, kAssumedSmemPerBlock);
+            p.kind = pair ? KIND_SEQUENTIAL_PAIR : split ? KIND_SEQUENTIAL_SPLIT : KIND_SEQUENTIAL;
+            p.split = (split || pair) ? 2 : 1;
             p.V = 1;
-            p.cg = 32;
-            p.r = 1;
+            p.cg = int(gw);
+            p.r = pair ? kSeqRows : kSeqRows / p.split;            // rows of a slot per lane
             p.stages = lay.slots;
-            p.warps = kSeqWarpsPerBlock;
+            p.warps = pair ? kPairWarps : kSeqWarpsPerBlock;
             p.TR = T > 0 ? int(std::min<int64_t>(T, std::numeric_limits<int>::max())) : 0;
-            p.TC = int(cw);
+            p.TC = int(gw);
             p.smem = lay.smem;
-            p.n_dt = (D + cw - 1) / cw;
+            p.n_dt = (D + gw - 1) / gw;
             p.n_chains = B * p.n_dt;
             p.n_chunks = T > 0 ? 1 : 0;
             p.n_tiles = p.n_chains * p.n_chunks;
+            if (p.n_tiles > 0) {
+                p.off_words = kAlign;                           // the header alone: status word
+                p.ws_bytes = kAlign;
+            }
             return p;
         }
     }
@@ -303,9 +339,10 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
     p.n_chains = B * p.n_dt;
     p.n_chunks = (T + p.TR - 1) / p.TR;
     p.n_tiles = p.n_chains * p.n_chunks;
-    if (p.n_chunks > 1) {
-        p.off_words = kAlign;                                   // [0, 256): status word
-        p.ws_bytes = align_up(p.off_words + size_t(p.n_tiles) * 3 * p.TC * 8, kAlign);
+    if (p.n_tiles > 0) {
+        p.off_words = kAlign;                                   // [0, 256): header
+        p.ws_bytes = kAlign;
+        if (p.n_chunks > 1) p.ws_bytes = align_up(p.off_words + size_t(p.n_tiles) * 3 * p.TC * 8, kAlign);
     }
     return p;
 }
@@ -512,12 +549,12 @@ cudaError_t seq_device(const void *kernel, size_t min_bytes, SeqDev *out) {
     *out = info[dev];
     return cudaSuccess;
 }
-template <class Op, typename IO>
+template <class Op, typename IO, int SPLIT>
 cudaError_t launch_sequential(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
     constexpr int WB = kSeqWarpsPerBlock;
-    constexpr int CW = 32;
-    constexpr int kRowBytes = seq_row_bytes<IO>();
-    auto kernel = scan_sequential_kernel<Op, IO, WB>;
+    constexpr int CW = 32 / SPLIT;
+    constexpr int kRowBytes = CW * int(sizeof(IO));
+    auto kernel = scan_sequential_kernel<Op, IO, WB, SPLIT>;
     alignas(64) CUtensorMap map0, map1, map_out;
     if (!make_operand_map(&map0, sp.in0, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
         !make_operand_map(&map1, sp.in1, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
@@ -539,9 +576,35 @@ cudaError_t launch_sequential(const Plan &pl, const ScanParams &sp, cudaStream_t
 }
 
 template <class Op, typename IO>
+cudaError_t launch_sequential_pair(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
+    constexpr int CW = 32;
+    constexpr int kRowBytes = CW * int(sizeof(IO));
+    auto kernel = scan_sequential_pair_kernel<Op, IO>;
+    alignas(64) CUtensorMap map0, map1, map_out;
+    if (!make_operand_map(&map0, sp.in0, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
+        !make_operand_map(&map1, sp.in1, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
+        !make_operand_map(&map_out, sp.out, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows))
+        return cudaErrorInvalidValue;
+    SeqDev d;
+    cudaError_t e = seq_device(reinterpret_cast<const void *>(kernel), seq_pair_block_bytes(kSeqMinSlots, kRowBytes), &d);
+    if (e != cudaSuccess) return e;
+    SeqParams q;
+    q.s = sp;
+    q.n_groups = pl.n_dt;
+    q.n_warps = pl.n_chains;                  // channel groups: one block each
+    const SeqLayout lay = seq_pair_layout(q.n_warps, kRowBytes, d.sms, size_t(d.smem_sm), size_t(d.reserved),
+                                          size_t(d.smem_block));
+    q.slots = lay.slots;
+    kernel<<<dim3(unsigned(q.n_warps)), kPairWarps * 32, lay.smem, s>>>(q, map0, map1, map_out);
+    return cudaGetLastError();
+}
+
+template <class Op, typename IO>
 cudaError_t dispatch(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
     constexpr int VW = 16 / int(sizeof(IO));
-    if (pl.kind == KIND_SEQUENTIAL) return launch_sequential<Op, IO>(pl, sp, s);
+    if (pl.kind == KIND_SEQUENTIAL) return launch_sequential<Op, IO, 1>(pl, sp, s);
+    if (pl.kind == KIND_SEQUENTIAL_SPLIT) return launch_sequential<Op, IO, 2>(pl, sp, s);
+    if (pl.kind == KIND_SEQUENTIAL_PAIR) return launch_sequential_pair<Op, IO>(pl, sp, s);
     if (pl.kind == KIND_PIPELINED) {
         if constexpr (sizeof(IO) == 2) {
             if (pl.r == 8) return launch_pipelined<Op, IO, 4, 8, kPipeWarps>(sp, s, nullptr);
@@ -637,15 +700,17 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
     sp.spin_limit = g_spin_limit.load();
     sp.drop_tile = g_drop_tile.load();
     set_decay(sp, dec);
-    if (pl.kind == KIND_SEQUENTIAL && ws && ws_bytes >= sizeof(uint32_t) && aligned16(ws)) {
-        // no hand-off words; a workspace, when given, still receives the status
-        sp.status = static_cast<uint32_t *>(ws);
-    }
+    // every plan records its bounded waits in the workspace's status word
+    if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)) return SGR_ERR_WORKSPACE;
+    sp.status = static_cast<uint32_t *>(ws);
     if (pl.n_chunks > 1) {
-        if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)) return SGR_ERR_WORKSPACE;
         char *w = static_cast<char *>(ws);
-        sp.status = reinterpret_cast<uint32_t *>(w);
         sp.words = reinterpret_cast<uint64_t *>(w + pl.off_words);
+        if (pl.kind == KIND_TILE) {
+            // one block per tile: tiles go out by ticket in block start order
+            sp.ticket = reinterpret_cast<uint32_t *>(w + kTicketOffset);
+            if (cudaMemsetAsync(sp.ticket, 0, sizeof(uint32_t), stream) != cudaSuccess) return SGR_ERR_CUDA;
+        }
         cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
         if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return SGR_ERR_CUDA;
         if (cs == cudaStreamCaptureStatusActive) {
@@ -737,7 +802,7 @@ bool seq_backward_planned(int64_t B, int64_t T, int64_t D, int esz, bool aligned
         B > int64_t(std::numeric_limits<int>::max()))
         return false;
     const int ok = g_override_kind.load();
-    if (ok == KIND_SEQUENTIAL) return true;
+    if (ok == KIND_SEQUENTIAL || ok == KIND_SEQUENTIAL_SPLIT || ok == KIND_SEQUENTIAL_PAIR) return true;
     if (ok != KIND_AUTO) return false;
     const int64_t groups = B * ((D + 31) / 32);
     return groups >= int64_t(kSeqBwdMinWarpsPerSM) * kAssumedSMs;
@@ -838,8 +903,9 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
     bp.dlam = dec ? dlam : nullptr;
     if (seq) {
         // one warp per channel group over the whole sequence: no hand-off
-        // words; a workspace, when given, receives the status word
-        if (ws && ws_bytes >= sizeof(uint32_t) && aligned16(ws)) sp.status = static_cast<uint32_t *>(ws);
+        // words; the workspace header receives the status word
+        if (!ws || ws_bytes < kAlign || !aligned16(ws)) return SGR_ERR_WORKSPACE;
+        sp.status = static_cast<uint32_t *>(ws);
         if (bp.dlam && cudaMemsetAsync(bp.dlam, 0, size_t(D) * sizeof(float), stream) != cudaSuccess)
             return SGR_ERR_CUDA;
         cudaError_t e;
@@ -855,11 +921,14 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
         }
         return e == cudaSuccess ? SGR_OK : SGR_ERR_CUDA;
     }
+    if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)) return SGR_ERR_WORKSPACE;
+    sp.status = static_cast<uint32_t *>(ws);
     if (pl.n_chunks > 1) {
-        if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)) return SGR_ERR_WORKSPACE;
         char *w = static_cast<char *>(ws);
-        sp.status = reinterpret_cast<uint32_t *>(w);
         sp.words = reinterpret_cast<uint64_t *>(w + pl.off_words);
+        // one block per tile: tiles go out by ticket in block start order
+        sp.ticket = reinterpret_cast<uint32_t *>(w + kTicketOffset);
+        if (cudaMemsetAsync(sp.ticket, 0, sizeof(uint32_t), stream) != cudaSuccess) return SGR_ERR_CUDA;
         cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
         if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return SGR_ERR_CUDA;
         if (cs == cudaStreamCaptureStatusActive) {
@@ -914,7 +983,7 @@ SumPlan make_sum_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool a
         sp.seg = ((T + n_seg - 1) / n_seg + kSeqRows - 1) / kSeqRows * kSeqRows;
         sp.n_seg = (T + sp.seg - 1) / sp.seg;
         const int64_t n_mid = sp.n_seg > 32 ? (sp.n_seg + 31) / 32 : 0;
-        sp.ws = align_up(size_t(sp.n_seg + n_mid) * size_t(B) * size_t(D) * sizeof(float2), kAlign);
+        sp.ws = kAlign + align_up(size_t(sp.n_seg + n_mid) * size_t(B) * size_t(D) * sizeof(float2), kAlign);
         return sp;
     }
     // one 16-byte vector of channels per thread (4 fp32, 8 bf16)
@@ -928,9 +997,10 @@ SumPlan make_sum_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool a
     n_seg = std::max<int64_t>(1, std::min<int64_t>({n_seg, (T + 7) / 8, int64_t(512)}));
     sp.seg = (T + n_seg - 1) / n_seg;
     sp.n_seg = (T + sp.seg - 1) / sp.seg;
-    // partials, then (more than 32 segments) their folds in groups of 32
+    // the status word's header, the partials, then (more than 32 segments)
+    // their folds in groups of 32
     const int64_t n_mid = sp.n_seg > 32 ? (sp.n_seg + 31) / 32 : 0;
-    sp.ws = align_up(size_t(sp.n_seg + n_mid) * size_t(B) * size_t(D) * sizeof(float2), kAlign);
+    sp.ws = kAlign + align_up(size_t(sp.n_seg + n_mid) * size_t(B) * size_t(D) * sizeof(float2), kAlign);
     return sp;
 }
 
@@ -1255,7 +1325,8 @@ sgr_status_t sgr_scan_summary(sgr_op_t op, const void *in0, const void *in1, int
     ScanParams sp;
     std::memset(&sp, 0, sizeof(sp));
     sp.in0 = in0; sp.in1 = in1; sp.B = B; sp.T = T; sp.D = D;
-    float2 *partial = static_cast<float2 *>(workspace);
+    sp.status = static_cast<uint32_t *>(workspace);                  // header: the status word
+    float2 *partial = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + kAlign);
     float2 *out = reinterpret_cast<float2 *>(pairs);
     cudaError_t e;
     if (op == SGR_OP_MINGRU) {
@@ -1372,7 +1443,8 @@ void fill_plan(const Plan &p, sgr_plan_t *plan) {
     plan->channel_lanes = p.cg;
     plan->rows_per_thread = p.r;
     plan->warps = p.warps;
-    plan->threads = (p.kind == KIND_SEQUENTIAL ? plan->warps : plan->warps + 1) * 32;
+    const bool seq = p.kind == KIND_SEQUENTIAL || p.kind == KIND_SEQUENTIAL_SPLIT || p.kind == KIND_SEQUENTIAL_PAIR;
+    plan->threads = (seq ? plan->warps : plan->warps + 1) * 32;
     plan->stages = p.stages;
     plan->tile_rows = p.TR;
     plan->tile_channels = p.TC;
@@ -1429,7 +1501,7 @@ sgr_status_t sgr_set_drop_publish(int64_t tile) {
 }
 
 sgr_status_t sgr_set_kernel_override(int kernel) {
-    if (kernel < KIND_AUTO || kernel > KIND_SEQUENTIAL) return SGR_ERR_INVALID_ARG;
+    if (kernel < KIND_AUTO || kernel > KIND_SEQUENTIAL_PAIR) return SGR_ERR_INVALID_ARG;
     g_override_kind.store(kernel);
     return SGR_OK;
 }
@@ -1463,9 +1535,12 @@ sgr_status_t sgr_set_tile_override(int channel_lanes, int rows_per_thread) {
 // device current) and zero-fills it on the caller's stream; that first call
 // should therefore come before any stream capture.  All calls on a device
 // share the one array and it keeps the last call's contents; every launch tags
-// its words with a fresh epoch, so nothing needs clearing between calls, but
-// calls whose kernels can overlap on the GPU (e.g. on two streams without an
-// ordering between them) race on the array and must not be made.
+// its hand-off words with a fresh epoch, so those need no clearing between
+// calls, but calls whose kernels can overlap on the GPU (e.g. on two streams
+// without an ordering between them) race on the array and must not be made.
+// The array's status word is the library's own: each call clears it on the
+// stream before its launch, and no entry point reads it back, so for this
+// entry point a chunk that gave up waiting shows only as NaN outputs.
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
@@ -1486,6 +1561,7 @@ extern "C" sgr_status_t mingru_scan_noalloc(const void *k, const void *hx, const
     // scratch this shape needs, for whichever kernel variant the call takes
     const size_t need = sgr_workspace_size(SGR_OP_MINGRU, B, T, D, dtype);
     if (need > kNoAllocScratchBytes) return SGR_ERR_WORKSPACE;
+    if (!k || !hx || !h) return SGR_ERR_INVALID_ARG;
     void *ws = nullptr;
     if (need > 0) {
         int dev = 0;
@@ -1499,6 +1575,8 @@ extern "C" sgr_status_t mingru_scan_noalloc(const void *k, const void *hx, const
             g_noalloc_ptr[dev] = p;
         }
         ws = g_noalloc_ptr[dev];
+        // a bit left by an earlier call's timed-out wait must not linger
+        if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), stream) != cudaSuccess) return SGR_ERR_CUDA;
     }
     return mingru_scan(k, hx, h0, h0_batch_stride, h, B, T, D, dtype, ws,
                        ws ? kNoAllocScratchBytes : 0, stream);

@@ -50,14 +50,31 @@ def test_version_and_status_strings():
 
 
 # ----------------------------------------------------- argument validation
-# Fake device addresses: validation must reject these calls before touching CUDA.
+# Fake device addresses: validation must reject these calls before touching
+# CUDA.  The overlap checks need distinct non-null addresses, so these tests
+# run only where no CUDA device is visible: should a check ever regress, the
+# call then fails to launch (no device) instead of running a kernel on
+# addresses that back nothing.
 A, Bp, C = 0x10000000, 0x20000000, 0x30000000
+
+
+def _device_visible() -> bool:
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:  # noqa: BLE001 - no torch: no device either
+        return False
+
+
+fake_addresses = pytest.mark.skipif(_device_visible(),
+                                    reason="fake device addresses are only passed where no GPU is visible")
 
 
 def scan(fn, *args):
     return getattr(_abi.lib(), fn)(*args)
 
 
+@fake_addresses
 @pytest.mark.parametrize("fn", ["mingru_scan", "minmax_scan"])
 def test_scan_argument_errors(fn):
     E = _abi.SGR_ERR_INVALID_ARG
@@ -89,6 +106,7 @@ def test_scan_argument_errors(fn):
         == _abi.SGR_ERR_UNSUPPORTED
 
 
+@fake_addresses
 def test_step_argument_errors():
     lib = _abi.lib()
     E = _abi.SGR_ERR_INVALID_ARG
@@ -125,23 +143,27 @@ def test_decayed_plan():
 
 
 def test_workspace_covers_the_decayed_plan():
-    # wide batches: the plain plan needs no workspace, the time-decayed scan
-    # (never channel-sequential) is cut along T and needs one
+    # wide batches: the plain plan needs only the workspace header (its status
+    # word), the time-decayed scan (never channel-sequential) is cut along T
+    # and needs hand-off words too
     for B, dtype in ((16, F32), (24, BF16)):
         pl = _abi.plan(MINGRU, B, 2048, 2048, dtype, True)
-        assert pl["kernel"] == _abi.KERNEL_SEQUENTIAL and pl["workspace_bytes"] == 0
-        assert _abi.lib().sgr_workspace_size(MINGRU, B, 2048, 2048, dtype) > 0
+        assert pl["kernel"] in SEQ_KINDS and pl["workspace_bytes"] == WS_HEADER
+        assert _abi.lib().sgr_workspace_size(MINGRU, B, 2048, 2048, dtype) > WS_HEADER
 
 
 def test_workspace_size_and_hooks():
     lib = _abi.lib()
-    assert lib.sgr_workspace_size(MINGRU, 2, 1, 512, F32) == 0      # one chunk
+    assert lib.sgr_workspace_size(MINGRU, 2, 1, 512, F32) == WS_HEADER     # one chunk: the header
+    assert lib.sgr_workspace_size(MINGRU, 0, 1, 512, F32) == 0             # empty shape
     assert lib.sgr_workspace_size(9, 2, 4096, 512, F32) == 0
     assert lib.sgr_workspace_size(MINGRU, 8, 4096, 1024, F32) > 0
     assert lib.sgr_set_tile_override(3, 0) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_tile_override(0, 3) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_drop_publish(-2) == _abi.SGR_ERR_INVALID_ARG
-    assert lib.sgr_set_kernel_override(5) == _abi.SGR_ERR_INVALID_ARG
+    assert lib.sgr_set_kernel_override(7) == _abi.SGR_ERR_INVALID_ARG
+    assert lib.sgr_set_kernel_override(_abi.KERNEL_SEQUENTIAL_SPLIT) == _abi.SGR_OK
+    assert lib.sgr_set_kernel_override(0) == _abi.SGR_OK
     assert lib.sgr_set_wait_limit(0) == _abi.SGR_OK
     assert lib.sgr_set_drop_publish(-1) == _abi.SGR_OK
     assert lib.sgr_workspace_init(None, 0, None) == _abi.SGR_OK
@@ -153,46 +175,70 @@ def test_workspace_size_and_hooks():
 # The kernel's address formulas, replayed for every block and thread.
 
 SEQ_ROWS = 16            # rows per load slot of the channel-sequential kernel
+SEQ_KINDS = (_abi.KERNEL_SEQUENTIAL, _abi.KERNEL_SEQUENTIAL_SPLIT, _abi.KERNEL_SEQUENTIAL_PAIR)
+WS_HEADER = 256          # workspace header: status word at 0, chunk ticket at 64
 
 
 def check_sequential_indices(pl, B, T, D, esz, check_cover):
-    """The channel-sequential kernel: warp gw scans channel group gw % n_groups
-    (32 channels) of batch row gw // n_groups over the whole sequence, in slots
-    of 16 rows loaded and stored as tensor-memory-accelerator boxes of 32
-    channels x 16 rows."""
+    """The channel-sequential kernels: warp gw scans channel group gw % n_groups
+    (32 channels; 16 when each slot's rows are split between the half-warps)
+    of batch row gw // n_groups over the whole sequence, in slots of 16 rows
+    loaded and stored as tensor-memory-accelerator boxes of CW channels x 16
+    rows; lane l owns channel l % CW of the slot rows
+    [(l // CW) R, (l // CW) R + R), R = 16 CW / 32.  With two warps per group
+    (kernel 6) a block's warps w = 0, 1 take rows [32 i + 16 w, 32 i + 16 w + 16)
+    of slot i, lane l channel l."""
     V, CW = pl["channels_per_thread"], pl["tile_channels"]
+    pair = pl["kernel"] == _abi.KERNEL_SEQUENTIAL_PAIR
+    split = 2 if pl["kernel"] == _abi.KERNEL_SEQUENTIAL_SPLIT else 1
     rb = CW * esz                                       # bytes of one operand row of a group
-    assert pl["vector_path"] and V == 1 and CW == 32 and rb in (64, 128)
-    assert pl["channel_lanes"] == 32 and pl["threads"] == 32 * pl["warps"]
-    assert pl["n_chunks"] == 1 and pl["workspace_bytes"] == 0 and pl["tile_rows"] == T
+    assert pl["vector_path"] and V == 1 and CW == 32 // split and rb in (32, 64, 128)
+    assert pl["channel_lanes"] == CW and pl["threads"] == 32 * pl["warps"]
+    assert pl["warps"] == (2 if pair else 1)
+    assert pl["rows_per_thread"] == SEQ_ROWS // split
+    assert pl["n_chunks"] == 1 and pl["workspace_bytes"] == WS_HEADER and pl["tile_rows"] == T
+    # a lane's elements of a slot stay inside its warp's 16 rows of CW channels
+    lane = np.arange(32)
+    off = (lane // CW) * pl["rows_per_thread"] * rb + (lane % CW) * esz
+    assert (off + (pl["rows_per_thread"] - 1) * rb + esz <= SEQ_ROWS * rb).all()
+    assert len(set(zip(lane % CW, lane // CW))) == 32   # no two lanes share an element
     n_groups = -(-D // CW)
     assert pl["n_channel_tiles"] == n_groups and pl["n_chains"] == B * n_groups
     assert pl["n_tiles"] == pl["n_chains"] < 2 ** 31
     assert 2 <= pl["stages"] <= 8
-    # a warp's ring, staging buffers and mbarriers fit its block's shared memory
-    warp_bytes = -(-(pl["stages"] * 2 * SEQ_ROWS * rb + 2 * SEQ_ROWS * rb + pl["stages"] * 8) // 128) * 128
-    assert warp_bytes * pl["warps"] <= pl["smem_bytes"] <= 227 * 1024
+    # the warps' rings, staging buffers and mbarriers fit their block's shared memory
+    S = pl["stages"]
+    if pair:
+        warp_bytes = -(-(S * 2 * SEQ_ROWS * rb + SEQ_ROWS * rb + S * 8) // 128) * 128
+        block_bytes = 2 * warp_bytes + 2 * 2 * 32 * 8      # + the pairs exchanged per slot
+    else:
+        block_bytes = -(-(S * 2 * SEQ_ROWS * rb + 2 * SEQ_ROWS * rb + S * 8) // 128) * 128
+    assert block_bytes <= pl["smem_bytes"] <= 227 * 1024
     assert (D * esz) % 16 == 0 and T < 2 ** 31 and B < 2 ** 31
     gw = np.arange(pl["n_chains"], dtype=np.int64)
     b, grp = gw // n_groups, gw % n_groups
     x0 = grp * CW
     assert ((x0 * esz) % 16 == 0).all()                 # box x coordinate 16-byte aligned
     assert (x0 < D).all() and (b < B).all()
-    n_slots = -(-T // SEQ_ROWS)
-    assert n_slots * SEQ_ROWS < 2 ** 31                 # row coordinates are 32-bit
+    slot_rows = 2 * SEQ_ROWS if pair else SEQ_ROWS
+    n_slots = -(-T // slot_rows)
+    assert n_slots * slot_rows < 2 ** 31                # row coordinates are 32-bit
     if check_cover:
         # the store boxes, clipped to the tensor, write every element exactly once
+        # (a pair warp's box that would start past T is not stored)
         cover = np.zeros((B, max(T, 1), D), dtype=np.int32)
         for w in range(len(gw)):
             for i in range(n_slots):
-                cover[b[w], i * SEQ_ROWS:min(T, (i + 1) * SEQ_ROWS), x0[w]:min(D, x0[w] + CW)] += 1
+                for y0 in ([i * slot_rows, i * slot_rows + SEQ_ROWS] if pair else [i * SEQ_ROWS]):
+                    if y0 < T:
+                        cover[b[w], y0:min(T, y0 + SEQ_ROWS), x0[w]:min(D, x0[w] + CW)] += 1
         assert (cover[:, :T] == 1).all(), "every output element is written exactly once"
 
 
 def check_plan_indices(B, T, D, dtype, aligned, check_cover, op=MINGRU):
     pl = _abi.plan(op, B, T, D, dtype, aligned)
     esz = 4 if dtype == F32 else 2
-    if pl["kernel"] == _abi.KERNEL_SEQUENTIAL:
+    if pl["kernel"] in SEQ_KINDS:
         check_sequential_indices(pl, B, T, D, esz, check_cover)
         return
     V, cg, R, W = pl["channels_per_thread"], pl["channel_lanes"], pl["rows_per_thread"], pl["warps"]
@@ -253,11 +299,12 @@ def check_plan_indices(B, T, D, dtype, aligned, check_cover, op=MINGRU):
     CV = TC // 32
     assert (np.arange(32) * CV + CV - 1 < TC).all()
     if n_chunks > 1:
-        assert pl["off_words"] >= 4 and pl["off_words"] % 8 == 0
+        # hand-off words after the header (status word, chunk ticket)
+        assert pl["off_words"] >= WS_HEADER and pl["off_words"] % 8 == 0
         assert pl["off_words"] + 8 * 3 * TC * n_tiles <= pl["workspace_bytes"]
         assert _abi.lib().sgr_workspace_size(op, B, T, D, dtype) >= pl["workspace_bytes"]
     else:
-        assert pl["workspace_bytes"] == 0
+        assert pl["workspace_bytes"] == WS_HEADER
 
 
 SMALL_SHAPES = [(2, 1024, 512), (3, 1000, 96), (1, 777, 36), (2, 300, 7), (1, 1, 1), (5, 1, 64),
@@ -269,7 +316,7 @@ SMALL_SHAPES = [(2, 1024, 512), (3, 1000, 96), (1, 777, 36), (2, 300, 7), (1, 1,
 @pytest.mark.parametrize("aligned", [True, False])
 @pytest.mark.parametrize("override", [(0, 0, 0), (1, 0, 1), (1, 0, 2), (1, 0, 4), (1, 0, 8),
                                       (2, 0, 2), (2, 0, 4), (2, 0, 8), (3, 0, 2), (3, 0, 4),
-                                      (3, 0, 8), (4, 0, 0)])
+                                      (3, 0, 8), (4, 0, 0), (5, 0, 0), (6, 0, 0)])
 def test_plan_indices_small(shape, dtype, aligned, override):
     lib = _abi.lib()
     assert lib.sgr_set_kernel_override(override[0]) == 0
@@ -290,6 +337,7 @@ def test_plan_indices_workloads(name):
 
 # ------------------------------------------------------- host-buffer scans
 
+@fake_addresses
 @pytest.mark.parametrize("fn", ["mingru_scan_host", "minmax_scan_host"])
 def test_host_scan_argument_errors(fn):
     E = _abi.SGR_ERR_INVALID_ARG
@@ -336,6 +384,7 @@ def test_host_staging_size():
 
 # ------------------------------------------------------------- gradients
 
+@fake_addresses
 @pytest.mark.parametrize("fn", ["mingru_scan_backward", "minmax_scan_backward"])
 def test_backward_argument_errors(fn):
     E = _abi.SGR_ERR_INVALID_ARG
@@ -417,6 +466,7 @@ def test_backward_plan_reverse_indices(shape, dtype, aligned):
     assert (ends_at_zero == 1).all()
 
 
+@fake_addresses
 def test_decay_argument_errors():
     lib = _abi.lib()
     E = _abi.SGR_ERR_INVALID_ARG
@@ -455,6 +505,7 @@ def test_decay_argument_errors():
     assert db(*ok) == _abi.SGR_ERR_WORKSPACE                   # distinct buffers pass the checks
 
 
+@fake_addresses
 def test_summary_and_combine_argument_errors():
     lib = _abi.lib()
     E = _abi.SGR_ERR_INVALID_ARG
@@ -484,6 +535,7 @@ def test_summary_and_combine_argument_errors():
     assert c(MINGRU, P, 1, None, 0, None, 64, 0, 64, F32, None) == _abi.SGR_OK
 
 
+@fake_addresses
 def test_projected_scan_argument_errors():
     lib = _abi.lib()
     X, W, H, WS = 0x10000000, 0x20000000, 0x30000000, 0x40000000
