@@ -54,3 +54,45 @@ def gpu_channels(y: torch.Tensor, chans):
     b = torch.tensor([c[0] for c in chans], device=y.device)
     d = torch.tensor([c[1] for c in chans], device=y.device)
     return y[b, :, d].to("cpu", torch.float64).numpy()
+
+
+def _as_host(x):
+    if hasattr(x, "detach"):
+        return x.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def _fold_channels(a, G):
+    """(B, T, D) -> (B G, T, D / G): channel groups become batch rows, so the
+    oracle's threads (one per batch row) all have work."""
+    B, T, D = a.shape
+    return a.reshape(B, T, G, D // G).transpose(0, 2, 1, 3).reshape(B * G, T, D // G)
+
+
+def _unfold_channels(a, B, G):
+    BG, T, Dg = a.shape
+    return a.reshape(B, G, T, Dg).transpose(0, 2, 1, 3).reshape(B, T, G * Dg)
+
+
+def full_rel_err(op, p, q, init, got, threads=8, rows=2, fn=None):
+    """Max relative error of `got` (B, T, D) against the oracle over EVERY
+    channel and row, evaluated `rows` batch rows at a time (bounded host
+    memory).  `fn` replaces the oracle call (same signature as
+    oracle.mingru_linear) for other recurrences."""
+    B, T, D = p.shape
+    call = fn or (oracle.mingru_linear if op == "mingru" else oracle.minmax)
+    worst = 0.0
+    for b0 in range(0, B, rows):
+        b1 = min(B, b0 + rows)
+        nb = b1 - b0
+        G = 1
+        while nb * G < threads and D % (2 * G) == 0 and D // (2 * G) >= 8:
+            G *= 2
+        P = _fold_channels(_as_host(p[b0:b1]), G)
+        Q = _fold_channels(_as_host(q[b0:b1]), G)
+        I = None
+        if init is not None:
+            I = _as_host(init[b0:b1]).reshape(nb * G, D // G)
+        ref = _unfold_channels(call(P, Q, I, threads=threads), nb, G)
+        worst = max(worst, rel_err(got[b0:b1], ref))
+    return worst

@@ -17,7 +17,7 @@ import torch
 import oracle
 import scan_gated_rnns_b200 as sgr
 from scan_gated_rnns_b200 import _abi
-from scan_gated_rnns_b200.synth import WORKLOADS, Workload, generate, sample_channels
+from scan_gated_rnns_b200.synth import WORKLOADS, Workload, generate
 
 from parity import TORCH_DT
 
@@ -208,28 +208,23 @@ def test_backward_bounded_wait_reports_timeout():
 
 
 def test_backward_workload_b8_t4096_d1024():
-    """The gradient of the benchmark's minGRU workload, at full size, checked on
-    a seeded sample of channels over their full length."""
+    """The gradient of the benchmark's minGRU workload, at full size, on every
+    channel and row: the kernel reads the oracle's forward (rounded to fp32)
+    and is compared with the oracle's gradient of the whole tensor."""
     w = WORKLOADS["mingru_b8_t4096_d1024_f32_h0"]
     K, H, H0 = generate(w, device=DEV)
     g = torch.Generator(device=DEV).manual_seed(5)
     GY = torch.randn(K.shape, device=DEV, generator=g)
-    chans = sample_channels(w, 48)
-    b = torch.tensor([c[0] for c in chans])
-    d = torch.tensor([c[1] for c in chans])
-    kc, hc, gc = (t[b.to(DEV), :, d.to(DEV)].cpu()[:, :, None] for t in (K, H, GY))
-    i0c = H0[b.to(DEV), d.to(DEV)].cpu()[:, None]
-    # forward state for the GPU input: the oracle's forward of the whole tensor is too slow
-    # on the CPU, so h comes from the oracle on the sampled channels and the GPU's own forward
-    # elsewhere; the sampled channels' gradients depend only on their own h
-    Hf = sgr.mingru_scan(K, H, H0)
-    hc_oracle = torch.from_numpy(oracle.mingru_linear(kc, hc, i0c)).float()[:, :, 0]
-    Hf[b.to(DEV), :, d.to(DEV)] = hc_oracle.to(DEV)
+    k, hx, h0, gy = (t.cpu() for t in (K, H, H0, GY))
+    Hf = torch.from_numpy(oracle.mingru_linear(k, hx, h0, threads=8)).float().to(DEV)
     dk, dhx, dh0 = sgr.mingru_scan_backward(K, H, H0, Hf, GY)
     torch.cuda.synchronize()
-    rk, rhx, rh0 = oracle.mingru_backward(kc, hc, i0c, gc)
-    got_k = dk[b.to(DEV), :, d.to(DEV)].cpu()[:, :, None]
-    got_hx = dhx[b.to(DEV), :, d.to(DEV)].cpu()[:, :, None]
-    assert channel_scaled_err(got_k, rk) <= TOL_BWD["f32"]
-    assert channel_scaled_err(got_hx, rhx) <= TOL_BWD["f32"]
-    assert np.allclose(dh0[b.to(DEV), d.to(DEV)].cpu().double().numpy(), rh0[:, 0], rtol=1e-4, atol=1e-6)
+    rk, rhx, rh0 = oracle.mingru_backward(k, hx, h0, gy, threads=8)
+    ek, ehx = channel_scaled_err(dk, rk), channel_scaled_err(dhx, rhx)
+    # dL/dh0 sums signed terms over the whole sequence: its error is measured
+    # against the largest |dL/dh0| of the batch row
+    g0 = dh0.double().cpu().numpy()
+    eh0 = float((np.abs(g0 - rh0) / np.abs(rh0).max(axis=1, keepdims=True)).max())
+    print(f"{w.name} gradient: channel-scaled max error dk {ek:.3e}, dhx {ehx:.3e}, dh0 {eh0:.3e}")
+    assert ek <= TOL_BWD["f32"] and ehx <= TOL_BWD["f32"]
+    assert eh0 <= TOL_BWD["f32"]

@@ -150,10 +150,20 @@ def test_decay_backward_matches_oracle(dtype, init, shape):
     rk, rhx, rh0, rlam = oracle.mingru_decay_backward(k, hx, h0, dt, lam, gy)
     assert channel_scaled_err(dk, rk) <= TOL_BWD[dtype]
     assert channel_scaled_err(dhx, rhx) <= TOL_BWD[dtype]
-    # dlam: against the sum of the magnitudes of its terms (the oracle run on |gy|)
-    _, _, _, mag = oracle.mingru_decay_backward(k, hx, h0, dt, lam, np.abs(gy.double().numpy()))
-    scale = np.maximum(np.abs(mag), 1e-30)
-    assert float((np.abs(dlam.cpu().double().numpy() - rlam) / scale).max()) <= TOL_BWD[dtype] * 10
+    # dlam_d sums B T signed terms: its error is measured against the sum of
+    # the terms' magnitudes (the oracle's dlam for |gy|, every term >= 0)
+    err = lam_err(dlam, rlam, k, hx, h0, dt, lam, gy)
+    print(f"decay gradient {shape} {dtype} init={init}: dlam error {err:.3e} of the summed term magnitudes")
+    assert err <= TOL_BWD[dtype]
+
+
+def lam_err(got, rlam, k, hx, h0, dt, lam, gy) -> float:
+    """max_d |got_d - ref_d| / sum over (b, t) of |term_bt,d|: the oracle's
+    dL/dlambda for |gy| is that sum (every term then has the same sign)."""
+    gabs = np.abs(gy.double().numpy() if hasattr(gy, "double") else np.asarray(gy, np.float64))
+    _, _, _, mag = oracle.mingru_decay_backward(k, hx, h0, dt, lam, gabs)
+    got = got.detach().cpu().double().numpy() if hasattr(got, "detach") else np.asarray(got, np.float64)
+    return float((np.abs(got - rlam) / np.maximum(np.abs(mag), 1e-30)).max())
 
 
 def test_decay_autograd_wrapper_learns_lambda():
@@ -166,5 +176,10 @@ def test_decay_autograd_wrapper_learns_lambda():
     rk, rhx, rh0, rlam = oracle.mingru_decay_backward(k, hx, h0, dt, lam, gy)
     assert channel_scaled_err(K.grad, rk) <= TOL_BWD["f32"]
     assert channel_scaled_err(H.grad, rhx) <= TOL_BWD["f32"]
-    assert np.allclose(H0.grad.cpu().double().numpy(), rh0, rtol=1e-4, atol=1e-6)
-    assert np.allclose(L.grad.cpu().double().numpy(), rlam, rtol=1e-3, atol=1e-4)
+    # dL/dh0 (a signed sum over the sequence) against the largest |dL/dh0| of
+    # its batch row; dL/dlambda against its summed term magnitudes
+    g0 = H0.grad.cpu().double().numpy()
+    e0 = float((np.abs(g0 - rh0) / np.abs(rh0).max(axis=1, keepdims=True)).max())
+    el = lam_err(L.grad, rlam, k, hx, h0, dt, lam, gy)
+    print(f"decay autograd: dh0 error {e0:.3e} (row-scaled), dlam error {el:.3e} (term-magnitude-scaled)")
+    assert e0 <= TOL_BWD["f32"] and el <= TOL_BWD["f32"]

@@ -20,9 +20,9 @@ import torch
 import oracle
 import scan_gated_rnns_b200 as sgr
 from scan_gated_rnns_b200 import _abi
-from scan_gated_rnns_b200.synth import WORKLOADS, Workload, generate, sample_channels
+from scan_gated_rnns_b200.synth import WORKLOADS, Workload, generate
 
-from parity import TOL, TORCH_DT, gpu_channels, oracle_on_channels, rel_err
+from parity import TOL, TORCH_DT, full_rel_err, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -290,17 +290,19 @@ def test_workload_mingru_b2_t1024_d512():
     k, hx, h0 = generate(w, device=DEV)
     h = sgr.mingru_scan(k, hx, h0)
     torch.cuda.synchronize()
-    assert rel_err(h, oracle.mingru_linear(k, hx, h0, threads=8)) <= TOL["f32"]
+    err = rel_err(h, oracle.mingru_linear(k, hx, h0, threads=8))
+    print(f"{w.name}: max relative error {err:.3e} (bar {TOL['f32']:.0e})")
+    assert err <= TOL["f32"]
 
 
 def test_workload_mingru_b8_t4096_d1024_and_steps():
     w = WORKLOADS["mingru_b8_t4096_d1024_f32_h0"]
     K, H, H0 = generate(w, device=DEV)
     full = sgr.mingru_scan(K, H, H0)
-    chans = sample_channels(w, 64)
-    ref = oracle_on_channels("mingru", K, H, H0, chans)
     torch.cuda.synchronize()
-    assert rel_err(gpu_channels(full, chans), ref) <= TOL["f32"]
+    err = full_rel_err("mingru", K, H, H0, full)           # every channel and row
+    print(f"{w.name}: max relative error {err:.3e} (bar {TOL['f32']:.0e})")
+    assert err <= TOL["f32"]
     # first 4000 tokens in parallel, then 96 single-token steps
     pre = sgr.mingru_scan(K[:, :4000].contiguous(), H[:, :4000].contiguous(), H0)
     state = pre[:, -1, :].clone()
@@ -311,7 +313,9 @@ def test_workload_mingru_b8_t4096_d1024_and_steps():
     torch.cuda.synchronize()
     stitched = torch.cat([pre, torch.stack(tail, dim=1)], dim=1)
     assert rel_err(stitched, full.double().cpu().numpy()) <= TOL["f32"]
-    assert rel_err(gpu_channels(stitched, chans), ref) <= TOL["f32"]
+    err = full_rel_err("mingru", K, H, H0, stitched)
+    print(f"{w.name} (4000 scanned + 96 steps): max relative error {err:.3e}")
+    assert err <= TOL["f32"]
 
 
 def test_workload_minmax_b4_t8192_d768():
@@ -326,15 +330,17 @@ def test_workload_long_sequence():
     w = WORKLOADS["mingru_b1_t131072_d512_f32_h0"]
     k, hx, h0 = generate(w, device=DEV)
     h = sgr.mingru_scan(k, hx, h0)
-    chans = sample_channels(w, 48)
-    ref = oracle_on_channels("mingru", k, hx, h0, chans)
-    assert rel_err(gpu_channels(h, chans), ref) <= TOL["f32"]
+    torch.cuda.synchronize()
+    err = full_rel_err("mingru", k, hx, h0, h)             # every channel and row
+    print(f"{w.name}: max relative error {err:.3e} (bar {TOL['f32']:.0e})")
+    assert err <= TOL["f32"]
 
 
 def test_workload_bf16_throughput_shape():
     w = WORKLOADS["mingru_b16_t2048_d4096_bf16_h0"]
     k, hx, h0 = generate(w, device=DEV)
     h = sgr.mingru_scan(k, hx, h0)
-    chans = sample_channels(w, 96)
-    ref = oracle_on_channels("mingru", k, hx, h0, chans)
-    assert rel_err(gpu_channels(h, chans), ref) <= TOL["bf16"]
+    torch.cuda.synchronize()
+    err = full_rel_err("mingru", k, hx, h0, h)             # every channel and row
+    print(f"{w.name}: max relative error {err:.3e} (bar {TOL['bf16']:.0e})")
+    assert err <= TOL["bf16"]
