@@ -35,6 +35,7 @@ import json
 import math
 import os
 import statistics
+import subprocess
 import sys
 import threading
 import time
@@ -287,7 +288,7 @@ def scan_fn(w, p, q, init, out, ws):
 def plan_kernel(plan) -> str:
     """The device kernel a scan plan launches (the library's kernel kinds)."""
     return {1: "sgr::scan_tile_kernel", 2: "sgr::scan_pipelined_kernel", 3: "sgr::scan_pipelined_kernel",
-            4: "sgr::scan_sequential_kernel"}.get(plan["kernel"], "sgr::scan_kernel")
+            4: "sgr::scan_sequential_kernel", 5: "sgr::scan_sequential_kernel (split)"}.get(plan["kernel"], "sgr::scan_kernel")
 
 
 def backward_kernel(w) -> str:
@@ -532,10 +533,37 @@ def measure_step_row(device, B=8, D=1024, calls=200, warmup=10):
         stream.synchronize()
     g_per = t0.elapsed_time(t1) / 1e3 / calls
     del graph
-    return {"op": "mingru_step", "B": B, "D": D, "io_dtype": "f32",
-            "us_per_call": round(total / calls * 1e6, 2),
-            "us_per_launch_event": round(per * 1e6, 2),
-            "us_per_step_graph": round(g_per * 1e6, 2), "bytes_per_call": 4 * 4 * B * D}
+    row = {"op": "mingru_step", "B": B, "D": D, "io_dtype": "f32",
+           "us_per_call": round(total / calls * 1e6, 2),
+           "us_per_launch_event": round(per * 1e6, 2),
+           "us_per_step_graph": round(g_per * 1e6, 2), "bytes_per_call": 4 * 4 * B * D}
+    row["c_host_loop"] = step_host_loop(device, B, D)
+    return row
+
+
+def step_host_loop(device, B, D, steps=2000, warmup=100):
+    """The same decode step called from a plain C++ host loop through the C
+    ABI (scan_gated_rnns_b200/step_latency, built with the library): the
+    per-token cost without Python.  Its own process on the same device."""
+    from scan_gated_rnns_b200 import build as sgr_build
+    exe = sgr_build.STEP_EXE
+    if not os.path.exists(exe):
+        return {"unavailable": "step_latency not built"}
+    env = dict(os.environ)
+    idx = device.index if device.index is not None else 0
+    vis = env.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        env["CUDA_VISIBLE_DEVICES"] = vis.split(",")[idx]
+    else:
+        env["CUDA_VISIBLE_DEVICES"] = str(idx)
+    try:
+        out = subprocess.run([exe, str(B), str(D), str(steps), str(warmup)], env=env, capture_output=True,
+                             text=True, timeout=120)
+    except (OSError, subprocess.TimeoutExpired) as e:
+        return {"unavailable": f"step_latency did not run: {e}"}
+    if out.returncode != 0:
+        return {"unavailable": (out.stderr or out.stdout).strip()[-200:]}
+    return json.loads(out.stdout.strip().splitlines()[-1])
 
 
 def usable_cores() -> int:

@@ -19,6 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsgr.so")
+STEP_EXE = os.path.join(PKG, "step_latency")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
@@ -49,15 +50,30 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not verbose and up_to_date():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    if force or verbose or not up_to_date():
+        tmp = LIB + f".tmp{os.getpid()}"
+        cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, LIB)
+    build_step_latency(force)
     return LIB
+
+
+def build_step_latency(force: bool = False) -> str:
+    """The host-loop decode timer (native/step_latency.cpp), a plain C++
+    program linked against libsgr.so (found next to it at run time)."""
+    src = os.path.join(PKG, "native", "step_latency.cpp")
+    if not force and os.path.exists(STEP_EXE) and \
+            os.path.getmtime(STEP_EXE) >= max(os.path.getmtime(src), os.path.getmtime(LIB)):
+        return STEP_EXE
+    tmp = STEP_EXE + f".tmp{os.getpid()}"
+    cmd = [nvcc(), "-O2", "-std=c++17", "-x", "cu", "-gencode", "arch=compute_100a,code=sm_100a",
+           "-I", INCLUDE, "-o", tmp, src, "-L", PKG, "-lsgr", "-Xlinker", "-rpath=$ORIGIN"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, STEP_EXE)
+    return STEP_EXE
 
 
 if __name__ == "__main__":
