@@ -4,12 +4,12 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl b200|reference] [--no-rows]
 
-A step is one minGRU scan (activations, in-chunk scan, chunk hand-off,
-fix-up, store) over one batch of the workload, with inputs resident in HBM.
-The default workload is the minGRU scan with carried state,
-B=8 T=4096 D=1024 fp32 (k, hx ~ N(0,1), h0 ~ U(0.1,1)).  Its inputs (268 MB)
-and output (134 MB) are larger than the 126 MB L2, so back-to-back steps do
-not hit in L2.
+A step is one minGRU scan (activations, the scan over T, store) over one
+batch of the workload, with inputs resident in HBM.  The default workload is
+the largest single-GPU configuration, the minGRU scan with carried state
+B=16 T=2048 D=4096 with bf16 inputs and output and fp32 arithmetic (k, hx ~
+N(0,1), h0 ~ U(0.1,1)).  Its inputs (537 MB) and output (268 MB) are larger
+than the 126 MB L2, so back-to-back steps do not hit in L2.
 
 Metric: scan HBM GB/s = algorithmic bytes (inputs read once + output written
 once + initial state) per step / time per step, summed over GPUs.  Also
@@ -57,6 +57,7 @@ _ENGINE = "scan_gated_rnns_b200/csrc/scan_engine.cuh"
 KERNEL_SOURCES = {
     "scan_kernel": [_ENGINE],
     "scan_sequential_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_sequential.cuh"],
+    "scan_sequential_pair_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_sequential.cuh"],
     "scan_sequential_backward_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_backward.cuh",
                                         "scan_gated_rnns_b200/csrc/scan_sequential.cuh"],
     "scan_backward_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_backward.cuh"],
@@ -288,7 +289,18 @@ def scan_fn(w, p, q, init, out, ws):
 def plan_kernel(plan) -> str:
     """The device kernel a scan plan launches (the library's kernel kinds)."""
     return {1: "sgr::scan_tile_kernel", 2: "sgr::scan_pipelined_kernel", 3: "sgr::scan_pipelined_kernel",
-            4: "sgr::scan_sequential_kernel", 5: "sgr::scan_sequential_kernel (split)"}.get(plan["kernel"], "sgr::scan_kernel")
+            4: "sgr::scan_sequential_kernel", 5: "sgr::scan_sequential_kernel (split rows)",
+            6: "sgr::scan_sequential_pair_kernel"}.get(plan["kernel"], "sgr::scan_kernel")
+
+
+def profile_kernel(plan) -> str:
+    """The name a plan's kernel is filed under in profiles/: the chunked
+    kernels as scan_kernel, the channel-sequential ones by their own names."""
+    if plan["kernel"] in (4, 5):
+        return "sgr::scan_sequential_kernel"
+    if plan["kernel"] == 6:
+        return "sgr::scan_sequential_pair_kernel"
+    return "sgr::scan_kernel"
 
 
 def backward_kernel(w) -> str:
@@ -640,11 +652,9 @@ def run_b200(args):
     stream = torch.cuda.current_stream(device)
     bytes_step = w.algorithmic_bytes()
     # the chunked kernels' profiles are filed as scan_kernel; the channel-
-    # sequential kernel (wide batches) under its own name
-    kernel_name = "sgr::scan_kernel"
-    if sgr._abi.plan(0 if w.op == "mingru" else 1, w.B, w.T, w.D, 0 if w.dtype == "f32" else 1,
-                     True)["kernel"] == 4:
-        kernel_name = "sgr::scan_sequential_kernel"
+    # sequential kernels (wide batches) under their own names
+    kernel_name = profile_kernel(sgr._abi.plan(0 if w.op == "mingru" else 1, w.B, w.T, w.D,
+                                               0 if w.dtype == "f32" else 1, True))
     if args.pass_ == "projected":
         # the input projection fused with the scan: x (B, T, d_in) and W (2 D, d_in) bf16
         P = PROJECTED

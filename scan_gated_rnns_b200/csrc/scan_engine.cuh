@@ -101,28 +101,33 @@ struct MinGRUOp {
         b = z * g;
     }
     // The pairs of two steps (rows) of one channel, each fp32x2 operation
-    // packed across the two steps: two independent dependency chains per
-    // instruction stream, and the same values as element() except that
-    // g(hx) = max(hx + 0.5, sigmoid(hx)), which holds for every hx
-    // (hx + 0.5 - sigmoid(hx) is increasing and 0 at hx = 0; where hx < 0,
-    // sigmoid(hx) = sigmoid(-|hx|)), replaces the compare and select.  Used by
-    // the channel-sequential kernel, where one lane owns one channel.
+    // packed across the two steps (two independent dependency chains per
+    // instruction stream), for the kernels where one lane owns one channel.
+    // Evaluated without the sign selects of element(): with e = 2^(k log2 e),
+    //   a = sigmoid(-k) = 1 / (1 + e),  z = sigmoid(k) = e a,
+    // both relative-accurate for either sign of k (a product and a quotient
+    // of correctly signed positive terms, no cancellation).  k log2 e is
+    // clamped at 126 so that e stays finite: beyond k ~ 87 that leaves
+    // a = 2^-126 (instead of a smaller positive number) and z = 1, and
+    // k = +inf gives z = 1 exactly, k = -inf gives e = 0, a = 1, z = 0.
+    // g(hx) = max(hx + 0.5, sigmoid(hx)) with sigmoid(hx) = 1 / (1 + 2^(-hx
+    // log2 e)) holds for every hx (hx + 0.5 - sigmoid(hx) is increasing and
+    // 0 at hx = 0); hx = -inf gives 0, large hx gives hx + 0.5.  MUFU work:
+    // 2 exp2 + 2 reciprocals per element, about 5 instructions fewer than
+    // element().
     static __device__ __forceinline__ void element_rows(float k0, float hx0, float k1, float hx1, float2 &a,
                                                         float2 &b) {
-        const float2 ek = make_float2(fast_exp2(fabsf(k0) * kNegLog2e), fast_exp2(fabsf(k1) * kNegLog2e));
-        const float2 eh = make_float2(fast_exp2(fabsf(hx0) * kNegLog2e), fast_exp2(fabsf(hx1) * kNegLog2e));
+        const float2 tk = __fmul2_rn(make_float2(k0, k1), make_float2(-kNegLog2e, -kNegLog2e));
+        const float2 th = __fmul2_rn(make_float2(hx0, hx1), make_float2(kNegLog2e, kNegLog2e));
         const float2 one = make_float2(1.f, 1.f);
-        const float2 dk = __fadd2_rn(ek, one), dh = __fadd2_rn(eh, one);
-        const float2 pr = __fmul2_rn(dk, dh);
-        const float2 inv = make_float2(fast_rcp(pr.x), fast_rcp(pr.y));   // 1 / ((1 + ek)(1 + eh))
-        const float2 rk = __fmul2_rn(dh, inv), rh = __fmul2_rn(dk, inv);
-        const float2 sk = __fmul2_rn(ek, rk), sh = __fmul2_rn(eh, rh);     // sigmoid(-|k|), sigmoid(-|hx|)
-        const float2 kb = __fadd2_rn(one, make_float2(-sk.x, -sk.y));      // sigmoid(|k|)
-        const bool p0 = k0 >= 0.f, p1 = k1 >= 0.f;
-        a = make_float2(p0 ? sk.x : kb.x, p1 ? sk.y : kb.y);
-        const float2 z = make_float2(p0 ? kb.x : sk.x, p1 ? kb.y : sk.y);
+        const float2 ek = make_float2(fast_exp2(fminf(tk.x, 126.f)), fast_exp2(fminf(tk.y, 126.f)));
+        const float2 dk = __fadd2_rn(ek, one);                                  // 1 + e^k
+        const float2 dh = __fadd2_rn(make_float2(fast_exp2(th.x), fast_exp2(th.y)), one);   // 1 + e^-hx
+        a = make_float2(fast_rcp(dk.x), fast_rcp(dk.y));                         // sigmoid(-k)
+        const float2 z = __fmul2_rn(ek, a);                                     // sigmoid(k)
+        const float2 s = make_float2(fast_rcp(dh.x), fast_rcp(dh.y));            // sigmoid(hx)
         const float2 hp = __fadd2_rn(make_float2(hx0, hx1), make_float2(0.5f, 0.5f));
-        b = __fmul2_rn(z, make_float2(fmaxf(hp.x, sh.x), fmaxf(hp.y, sh.y)));
+        b = __fmul2_rn(z, make_float2(fmaxf(hp.x, s.x), fmaxf(hp.y, s.y)));
     }
     // fold a step into a running pair, two channels at once: (A, B) <- (A a, B a + b)
     static __device__ __forceinline__ void fold2(float2 &A, float2 &B, float2 a, float2 b) {

@@ -94,6 +94,16 @@ struct SeqParams {
     int slots;           // load ring depth S
 };
 
+// Time decay in the channel-sequential kernels: the gaps u_t are per (batch
+// row, row), shared by a warp's channels.  A warp's 16 rows of a slot have
+// their gaps spread across the lanes, lane l holding row y0 + (l % 16)'s
+// (0 past T: gamma = 1), loaded one slot ahead so that no step waits for
+// them; each row's gap is then taken from its lane by one shuffle.
+__device__ __forceinline__ float seq_slot_gap(const ScanParams &p, int64_t b, int64_t y0, int lane) {
+    const int64_t t = y0 + (lane & (kSeqRows - 1));
+    return (y0 >= 0 && t < p.T) ? decay_u(p, b, t) : 0.f;
+}
+
 // Block: WB independent warps; warp (blockIdx.x WB + w) scans channel group
 // (b, grp) of the batch.  Dynamic shared memory: WB x seq_warp_bytes(S).
 //
@@ -160,14 +170,19 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
     __syncwarp();
 
     float h = load_init<IO>(p, b, d, Op::default_init());           // state entering the slot
-    [[maybe_unused]] float lam2 = 0.f;
-    if constexpr (Op::kDecay) lam2 = decay_lam2(p, d);
+    [[maybe_unused]] float lam2 = 0.f, gcur = 0.f;
+    if constexpr (Op::kDecay) {
+        lam2 = decay_lam2(p, d);
+        gcur = seq_slot_gap(p, b, 0, lane);
+    }
 
     uint32_t wait_limit = kMbarLimit;
     bool bad = false;
     int s = 0;                 // ring slot of slot i
     uint32_t phase = 0;        // parity of that slot's current use
     for (int i = 0; i < n_slots; ++i) {
+        [[maybe_unused]] float gnext = 0.f;
+        if constexpr (Op::kDecay) gnext = seq_slot_gap(p, b, int64_t(i + 1) * kSeqRows, lane);
         if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
             // a copy that never lands: record it, make every later output NaN
             // and stop waiting at length (the kernel still ends)
@@ -209,9 +224,8 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
                 float2 a, c;
                 Op::element_rows(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
                 if constexpr (Op::kDecay) {
-                    const int64_t t = int64_t(i) * kSeqRows + r;
-                    a.x *= decay_gamma(lam2, t < p.T ? decay_u(p, b, t) : 0.f);
-                    a.y *= decay_gamma(lam2, t + 1 < p.T ? decay_u(p, b, t + 1) : 0.f);
+                    a.x *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r));
+                    a.y *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r + 1));
                 }
                 h = Op::step(a.x, c.x, h);
                 LR::store(dst + r * kRowBytes, h);
@@ -227,9 +241,8 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
                 float2 a, c;
                 Op::element_rows(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
                 if constexpr (Op::kDecay) {
-                    const int64_t t = int64_t(i) * kSeqRows + part * LROWS + r;
-                    a.x *= decay_gamma(lam2, t < p.T ? decay_u(p, b, t) : 0.f);
-                    a.y *= decay_gamma(lam2, t + 1 < p.T ? decay_u(p, b, t + 1) : 0.f);
+                    a.x *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, part * LROWS + r));
+                    a.y *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, part * LROWS + r + 1));
                 }
                 am[r] = a.x; cm[r] = c.x;
                 am[r + 1] = a.y; cm[r + 1] = c.y;
@@ -256,6 +269,7 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
             tma_store_3d(&map_out, obuf, x0, i * kSeqRows, int(b));
             bulk_commit();
         }
+        if constexpr (Op::kDecay) gcur = gnext;
     }
     if (lane == 0) bulk_wait_all();
 }
@@ -328,14 +342,19 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
     __syncwarp();
 
     float h = load_init<IO>(p, b, d, Op::default_init());           // state entering the slot
-    [[maybe_unused]] float lam2 = 0.f;
-    if constexpr (Op::kDecay) lam2 = decay_lam2(p, d);
+    [[maybe_unused]] float lam2 = 0.f, gcur = 0.f;
+    if constexpr (Op::kDecay) {
+        lam2 = decay_lam2(p, d);
+        gcur = seq_slot_gap(p, b, w * kSeqRows, lane);
+    }
 
     uint32_t wait_limit = kMbarLimit;
     bool bad = false;
     int s = 0;
     uint32_t phase = 0;
     for (int i = 0; i < n_slots; ++i) {
+        [[maybe_unused]] float gnext = 0.f;
+        if constexpr (Op::kDecay) gnext = seq_slot_gap(p, b, int64_t(i + 1) * kSlotRows + w * kSeqRows, lane);
         if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
             wait_limit = 1;
             if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
@@ -364,9 +383,8 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
             float2 a, c;
             Op::element_rows(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
             if constexpr (Op::kDecay) {
-                const int64_t t = int64_t(i) * kSlotRows + w * kSeqRows + r;
-                a.x *= decay_gamma(lam2, t < p.T ? decay_u(p, b, t) : 0.f);
-                a.y *= decay_gamma(lam2, t + 1 < p.T ? decay_u(p, b, t + 1) : 0.f);
+                a.x *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r));
+                a.y *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r + 1));
             }
             am[r] = a.x; cm[r] = c.x;
             am[r + 1] = a.y; cm[r + 1] = c.y;
@@ -399,6 +417,7 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
             tma_store_3d(&map_out, obuf, x0, y0, int(b));
             bulk_commit();
         }
+        if constexpr (Op::kDecay) gcur = gnext;
     }
     if (lane == 0) bulk_wait_all();
 }
@@ -490,8 +509,11 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
     const float h_init =
         (bp.init && d < p.D) ? load_scalar<IO>(static_cast<const IO *>(bp.init) + b * bp.init_bs + d)
                              : BOp::default_state();
-    [[maybe_unused]] float lam2 = 0.f, dl = 0.f;
-    if constexpr (BOp::kDecay) lam2 = decay_lam2(p, d);
+    [[maybe_unused]] float lam2 = 0.f, dl = 0.f, gcur = 0.f;
+    if constexpr (BOp::kDecay) {
+        lam2 = decay_lam2(p, d);
+        gcur = seq_slot_gap(p, b, int64_t(n_slots - 1) * kSeqRows, lane);
+    }
 
     float lam = 0.f;           // dL/d (state after the rows still to walk)
     uint32_t wait_limit = kMbarLimit;
@@ -500,6 +522,8 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
     uint32_t phase = 0;
     for (int i = 0; i < n_slots; ++i) {
         const int j = n_slots - 1 - i;
+        [[maybe_unused]] float gnext = 0.f;                         // the gaps of the slot below
+        if constexpr (BOp::kDecay) gnext = seq_slot_gap(p, b, int64_t(j - 1) * kSeqRows, lane);
         if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
             wait_limit = 1;
             if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
@@ -535,8 +559,7 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
                 float A, cP, cQ;
                 [[maybe_unused]] float u = 0.f;
                 if constexpr (BOp::kDecay) {
-                    const int64_t t = int64_t(j) * kSeqRows + r;
-                    u = t < p.T ? decay_u(p, b, t) : 0.f;
+                    u = __shfl_sync(0xffffffffu, gcur, r);
                     BOp::coeffs_gated(xk[r], xh[r], xf[r], decay_gamma(lam2, u), A, cP, cQ);
                 } else {
                     BOp::coeffs(xk[r], xh[r], xf[r], A, cP, cQ);
@@ -571,6 +594,7 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
             tma_store_3d(&map_d1, obuf + kOpBytes, x0, j * kSeqRows, int(b));
             bulk_commit();
         }
+        if constexpr (BOp::kDecay) gcur = gnext;
     }
     if (bp.dinit && d < p.D) {
         const float y[1] = {bad ? __int_as_float(0x7fffffff) : lam};

@@ -39,16 +39,25 @@ constexpr size_t kTicketOffset = 64;
 enum Kind { KIND_AUTO = 0, KIND_TILE = 1, KIND_PIPELINED = 2, KIND_PIPELINED_WIDE = 3, KIND_SEQUENTIAL = 4,
             KIND_SEQUENTIAL_SPLIT = 5, KIND_SEQUENTIAL_PAIR = 6 };
 
-// Channel-sequential kernel (scan_sequential.cuh): one warp per 32-channel
-// group walks the whole sequence.  Chosen when the groups alone give every SM
-// at least kSeqMinWarpsPerSM warps (fp32) or kSeqMinWarpsPerSMHalf (bf16:
-// half the bytes per element, so twice the warps for the same bandwidth);
-// below that the time axis is cut into chunks (measured crossovers: fp32
-// between 3.5 and 5.2 warps per SM (noisy near 5), bf16 between 7 and 10.4).  Shared-memory
+// Channel-sequential kernels (scan_sequential.cuh): each 32-channel group's
+// whole sequence is walked by one warp or by a block of two warps.  Chosen
+// when the groups alone give every SM at least kSeqMinWarpsPerSM of them
+// (fp32) or kSeqMinWarpsPerSMHalf (bf16); below that the time axis is cut
+// into chunks (measured crossovers: fp32 between 3.5 and 5.2 groups per SM,
+// noisy near 5; bf16 between 3.5 and 6.9 with two warps per group).  Shared-memory
 // figures are those of sm_100 (228 KB per SM, 1 KB reserved per block, 227 KB
 // per block at most); the launch reads the device's own.
 constexpr int kSeqMinWarpsPerSM = 6;
-constexpr int kSeqMinWarpsPerSMHalf = 9;
+constexpr int kSeqMinWarpsPerSMHalf = 6;
+// Below these many 32-channel groups per SM, each group takes a block of two
+// warps that split every slot's rows (scan_sequential_pair_kernel): twice the
+// warps hide the latency each one exposes, for a fold and a pair exchange per
+// slot.  Measured on B x 2048 x D (fraction of the copy bandwidth, one warp
+// per group against two): bf16 D 4096 at 6.9 groups per SM 0.53 / 0.58, 13.8:
+// 0.70 / 0.76, 20.8: 0.70 / 0.75, 27.7: 0.84 / 0.76; fp32 D 2048 at 10.4:
+// 0.81 / 0.84, 13.8: 0.84 / 0.86, and D 4096 at 27.7: 0.85 / 0.87.
+constexpr int kSeqPairBelow = 32;
+constexpr int kSeqPairBelowHalf = 24;
 // The gradient (four operands in, two out per element, where the chunked
 // gradient kernel is a plain tile kernel) gains from 3 warps per SM in both
 // dtypes (measured: fp32 loses at 2.6 and wins at 3.5, bf16 wins at 3.5 and
@@ -216,10 +225,10 @@ SeqLayout seq_pair_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm
 // per-tile work dominates and the longer tiles of 15-warp blocks pay wherever
 // they still give every SM 4 tiles (measured: MinMax B4 x 8192 x 768 fp32 0.81
 // of the copy bandwidth against 0.78 with 7-warp blocks; minGRU slower).
-// light_op: the MinMax clamp pair; decay: the time-decayed minGRU, whose
-// per-row gaps the channel-sequential kernel would wait for one row at a
-// time, and whose extra gate per element favours 4 rows per thread in the
-// pipelined kernel (bf16 with 15-warp blocks)
+// decay: the time-decayed minGRU, whose extra gate per element favours 4
+// rows per thread in the pipelined kernel (bf16 with 15-warp blocks); wide
+// decayed batches take the channel-sequential kernels like the plain scan
+// (their gaps arrive one slot ahead, spread across the lanes)
 Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
                bool force_tile = false, bool light_op = false, bool decay = false) {
     Plan p;
@@ -235,10 +244,12 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
                             B <= int64_t(std::numeric_limits<int>::max());
         const int min_per_sm = p.esz == 2 ? kSeqMinWarpsPerSMHalf : kSeqMinWarpsPerSM;
         const bool want = ok == KIND_SEQUENTIAL || ok == KIND_SEQUENTIAL_SPLIT || ok == KIND_SEQUENTIAL_PAIR ||
-                          (ok == KIND_AUTO && !decay && groups >= int64_t(min_per_sm) * kAssumedSMs);
+                          (ok == KIND_AUTO && groups >= int64_t(min_per_sm) * kAssumedSMs);
         if (seq_ok && want) {
             const bool split = ok == KIND_SEQUENTIAL_SPLIT;
-            const bool pair = ok == KIND_SEQUENTIAL_PAIR;
+            const int pair_below = p.esz == 2 ? kSeqPairBelowHalf : kSeqPairBelow;
+            const bool pair = ok == KIND_SEQUENTIAL_PAIR ||
+                              (ok == KIND_AUTO && groups < int64_t(pair_below) * kAssumedSMs);
             const int64_t gw = split ? cw / 2 : cw;                 // channels per warp
             const int64_t n_warps = B * ((D + gw - 1) / gw);
             const SeqLayout lay = pair ? seq_pair_layout(n_warps, int(gw) * p.esz, kAssumedSMs, kAssumedSmemPerSM,

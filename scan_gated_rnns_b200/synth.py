@@ -74,8 +74,9 @@ WORKLOADS = {
     ]
 }
 
-# the workload the benchmark times by default (minGRU scan with carried state)
-BENCH_WORKLOAD = "mingru_b8_t4096_d1024_f32_h0"
+# the workload the benchmark times by default: the largest single-GPU shape,
+# the minGRU scan of B16 x T2048 x D4096 with bf16 I/O and a carried state
+BENCH_WORKLOAD = "mingru_b16_t2048_d4096_bf16_h0"
 
 
 def generate(w: Workload, seed: Optional[int] = None, device="cpu"):

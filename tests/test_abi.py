@@ -120,18 +120,21 @@ def test_step_argument_errors():
 
 
 def test_decayed_plan():
-    # never the channel-sequential kernel; 4 rows per thread; bf16 with the
-    # 15-warp blocks wherever their tiles still give every SM 4 of them
-    for B, T, D, dtype in ((16, 2048, 2048, F32), (24, 2048, 2048, BF16), (8, 4096, 1024, BF16),
-                           (8, 4096, 1024, F32), (4, 8192, 512, BF16)):
+    # wide batches: the channel-sequential kernel the plain scan takes;
+    # otherwise 4 rows per thread, bf16 with the 15-warp blocks wherever their
+    # tiles still give every SM 4 of them
+    for B, T, D, dtype in ((16, 2048, 2048, F32), (24, 2048, 2048, BF16)):
         plain = _abi.plan(MINGRU, B, T, D, dtype, True)
+        pl = _abi.plan(MINGRU, B, T, D, dtype, True, decay=True)
+        assert pl["kernel"] == plain["kernel"] and pl["kernel"] in SEQ_KINDS, (B, T, D, dtype)
+        assert pl["workspace_bytes"] == WS_HEADER
+    for B, T, D, dtype in ((8, 4096, 1024, BF16), (8, 4096, 1024, F32), (4, 8192, 512, BF16)):
         pl = _abi.plan(MINGRU, B, T, D, dtype, True, decay=True)
         assert pl["kernel"] in (_abi.KERNEL_PIPELINED, _abi.KERNEL_PIPELINED_WIDE), (B, T, D, dtype)
         assert pl["rows_per_thread"] == 4
         if dtype == BF16:
             assert pl["kernel"] == _abi.KERNEL_PIPELINED_WIDE and pl["warps"] == 15
         assert pl["workspace_bytes"] <= _abi.lib().sgr_workspace_size(MINGRU, B, T, D, dtype)
-        assert plain["kernel"] != _abi.KERNEL_SEQUENTIAL or pl["workspace_bytes"] > 0
     # small shapes: one launch per tile, as for the plain scan
     assert _abi.plan(MINGRU, 2, 1024, 512, F32, True, decay=True)["kernel"] == _abi.KERNEL_TILE
     # unaligned rows: the scalar tile kernel
@@ -143,13 +146,15 @@ def test_decayed_plan():
 
 
 def test_workspace_covers_the_decayed_plan():
-    # wide batches: the plain plan needs only the workspace header (its status
-    # word), the time-decayed scan (never channel-sequential) is cut along T
-    # and needs hand-off words too
-    for B, dtype in ((16, F32), (24, BF16)):
-        pl = _abi.plan(MINGRU, B, 2048, 2048, dtype, True)
-        assert pl["kernel"] in SEQ_KINDS and pl["workspace_bytes"] == WS_HEADER
-        assert _abi.lib().sgr_workspace_size(MINGRU, B, 2048, 2048, dtype) > WS_HEADER
+    # the size covers the plain and the time-decayed plan of a shape: wide
+    # batches need the header alone for both, narrower ones hand-off words
+    lib = _abi.lib()
+    for B, T, D, dtype in ((16, 2048, 2048, F32), (24, 2048, 2048, BF16), (8, 4096, 1024, BF16),
+                           (1, 1 << 16, 64, F32)):
+        need = lib.sgr_workspace_size(MINGRU, B, T, D, dtype)
+        for decay in (False, True):
+            for aligned in (True, False):
+                assert _abi.plan(MINGRU, B, T, D, dtype, aligned, decay=decay)["workspace_bytes"] <= need
 
 
 def test_workspace_size_and_hooks():

@@ -87,20 +87,27 @@ def test_decay_every_kernel(kernel, r, dtype):
     assert rel_err(h, oracle.mingru_decay(k, hx, h0, dt, lam)) <= TOL[dtype]
 
 
-# Wide batches: the plain scan's plan scans whole sequences per warp, the
-# decayed scan stays on the chunked kernels, and the workspace query covers it.
-@pytest.mark.parametrize("dtype,B", [("f32", 16), ("bf16", 24)])
-def test_decay_wide_batch(dtype, B):
+# Wide batches: the decayed scan takes the channel-sequential kernel the
+# plain scan's plan names (gaps spread across the lanes one slot ahead), its
+# workspace is the status header, and no wait gives up.
+@pytest.mark.parametrize("dtype,B", [("f32", 16), ("bf16", 24), ("bf16", 64)])
+@pytest.mark.parametrize("log1p_delta", [False, True])
+def test_decay_wide_batch(dtype, B, log1p_delta):
     T, D = 300, 2048
     code = _abi.SGR_F32 if dtype == "f32" else _abi.SGR_BF16
-    assert _abi.plan(_abi.SGR_OP_MINGRU, B, T, D, code, True)["kernel"] == _abi.KERNEL_SEQUENTIAL
+    pl = _abi.plan(_abi.SGR_OP_MINGRU, B, T, D, code, True, decay=True)
+    assert pl["kernel"] == _abi.plan(_abi.SGR_OP_MINGRU, B, T, D, code, True)["kernel"]
+    assert pl["kernel"] in (_abi.KERNEL_SEQUENTIAL, _abi.KERNEL_SEQUENTIAL_PAIR)
     need = sgr.workspace_size("mingru", B, T, D, TORCH_DT[dtype])
-    assert need > 0
-    k, hx, h0, dt, lam = data(B, T, D, dtype, "u01_1", seed=B, wipe_at=150)
+    assert need >= pl["workspace_bytes"]
+    k, hx, h0, dt, lam = data(B, T, D, dtype, "u01_1", seed=B, wipe_at=150,
+                              gap_scale=20.0 if log1p_delta else 1.0)
     ws = sgr.Workspace(need, DEV)
-    h = sgr.mingru_scan_decay(k.to(DEV), hx.to(DEV), h0.to(DEV), dt.to(DEV), lam.to(DEV), workspace=ws)
+    h = sgr.mingru_scan_decay(k.to(DEV), hx.to(DEV), h0.to(DEV), dt.to(DEV), lam.to(DEV), log1p_delta,
+                              workspace=ws)
     torch.cuda.synchronize()
-    assert rel_err(h, oracle.mingru_decay(k, hx, h0, dt, lam)) <= TOL[dtype]
+    assert ws.status() == _abi.SGR_OK
+    assert rel_err(h, oracle.mingru_decay(k, hx, h0, dt, lam, log1p_delta)) <= TOL[dtype]
 
 
 # Gaps and rates through the copy engine (16-byte aligned starts, a batch

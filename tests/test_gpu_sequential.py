@@ -66,9 +66,10 @@ SHAPES = [(2, 1, 64), (3, 17, 40), (2, 300, 96), (1, 1000, 200), (4, 129, 8), (2
 @pytest.mark.parametrize("shape", SHAPES)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("init", [None, "u01_1"])
-def test_mingru_sequential_matches_oracle(shape, dtype, init):
-    sgr.set_kernel_override(SEQ)
-    assert plan(*shape, dtype)["kernel"] == SEQ
+@pytest.mark.parametrize("kind", SEQ_KINDS)
+def test_mingru_sequential_matches_oracle(shape, dtype, init, kind):
+    sgr.set_kernel_override(kind)
+    assert plan(*shape, dtype)["kernel"] == kind
     k, hx, h0 = small("mingru", *shape, dtype, init, seed=sum(shape) % 97)
     h = sgr.mingru_scan(*dev(k, hx, h0))
     torch.cuda.synchronize()
@@ -79,16 +80,18 @@ def test_mingru_sequential_matches_oracle(shape, dtype, init):
 @pytest.mark.parametrize("shape", SHAPES)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("init", [None, "u01_1"])
-def test_minmax_sequential_bit_exact(shape, dtype, init):
-    sgr.set_kernel_override(SEQ)
+@pytest.mark.parametrize("kind", SEQ_KINDS)
+def test_minmax_sequential_bit_exact(shape, dtype, init, kind):
+    sgr.set_kernel_override(kind)
     r, s, x0 = small("minmax", *shape, dtype, init, seed=sum(shape) % 89 + 3)
     x = sgr.minmax_scan(*dev(r, s, x0))
     torch.cuda.synchronize()
     assert exact(x, oracle.minmax(r, s, x0, threads=8))
 
 
-def test_minmax_sequential_special_values():
-    sgr.set_kernel_override(SEQ)
+@pytest.mark.parametrize("kind", SEQ_KINDS)
+def test_minmax_sequential_special_values(kind):
+    sgr.set_kernel_override(kind)
     g = torch.Generator().manual_seed(3)
     vals = torch.tensor([-math.inf, -2.0, -0.5, 0.5, 1.0, 3.0, math.inf])
     r = vals[torch.randint(0, 7, (2, 777, 96), generator=g)]
@@ -99,9 +102,10 @@ def test_minmax_sequential_special_values():
     assert exact(x, oracle.minmax(r, s, x0, threads=8))
 
 
-def test_mingru_sequential_gate_closed_forms():
+@pytest.mark.parametrize("kind", SEQ_KINDS)
+def test_mingru_sequential_gate_closed_forms(kind):
     # z = 1 (k = +inf): h_t = g(hx_t); z = 0 (k = -inf): h_t = h_0 exactly
-    sgr.set_kernel_override(SEQ)
+    sgr.set_kernel_override(kind)
     B, T, D = 2, 333, 64
     g = torch.Generator().manual_seed(5)
     hx = torch.randn(B, T, D, generator=g) * 3
@@ -115,8 +119,9 @@ def test_mingru_sequential_gate_closed_forms():
     assert torch.equal(h.cpu(), h0[:, None, :].expand(B, T, D))
 
 
-def test_mingru_sequential_initial_state_layouts():
-    sgr.set_kernel_override(SEQ)
+@pytest.mark.parametrize("kind", SEQ_KINDS)
+def test_mingru_sequential_initial_state_layouts(kind):
+    sgr.set_kernel_override(kind)
     B, T, D = 3, 200, 96
     k, hx, h0 = small("mingru", B, T, D, "f32", "u01_1", seed=11)
     K, H = dev(k, hx)
@@ -133,8 +138,9 @@ def test_mingru_sequential_initial_state_layouts():
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("log1p_delta", [False, True])
-def test_decay_sequential_matches_oracle(dtype, log1p_delta):
-    sgr.set_kernel_override(SEQ)
+@pytest.mark.parametrize("kind", SEQ_KINDS)
+def test_decay_sequential_matches_oracle(dtype, log1p_delta, kind):
+    sgr.set_kernel_override(kind)
     B, T, D = 3, 500, 136
     k, hx, h0 = small("mingru", B, T, D, dtype, "u01_1", seed=61)
     g = torch.Generator().manual_seed(62)
@@ -172,8 +178,9 @@ def test_misaligned_rows_do_not_take_it():
     assert rel_err(h, oracle.mingru_linear(k, hx, h0)) <= TOL["f32"]
 
 
-def test_sequential_graph_capture_replays():
-    sgr.set_kernel_override(SEQ)
+@pytest.mark.parametrize("kind", SEQ_KINDS)
+def test_sequential_graph_capture_replays(kind):
+    sgr.set_kernel_override(kind)
     B, T, D = 2, 300, 128
     k0, hx0, h00 = small("mingru", B, T, D, "bf16", "u01_1", seed=81)
     K, H, H0 = dev(k0, hx0, h00)
@@ -196,9 +203,9 @@ def test_sequential_graph_capture_replays():
 
 def test_bf16_workload_chunked_kernel_still_matches():
     # the full-size bf16 workload through the chunked pipelined kernel (the
-    # automatic choice there is the sequential kernel)
+    # automatic choice there is the two-warp channel-sequential kernel)
     w = WORKLOADS["mingru_b16_t2048_d4096_bf16_h0"]
-    assert plan(w.B, w.T, w.D, "bf16")["kernel"] == SEQ
+    assert plan(w.B, w.T, w.D, "bf16")["kernel"] == _abi.KERNEL_SEQUENTIAL_PAIR
     sgr.set_kernel_override(_abi.KERNEL_PIPELINED)
     k, hx, h0 = generate(w, device=DEV)
     h = sgr.mingru_scan(k, hx, h0)
@@ -209,14 +216,16 @@ def test_bf16_workload_chunked_kernel_still_matches():
 
 
 @pytest.mark.parametrize("dtype,shape,forced", [
-    ("bf16", (128, 20, 4096), False),   # 16384 groups: ~111 warps per SM, several waves
-    ("f32", (1, 70000, 32), True),      # one warp, 4375 slots: every ring slot reused many times
+    ("bf16", (128, 20, 4096), None),    # 16384 groups: ~111 warps per SM, several waves
+    ("f32", (1, 70000, 32), SEQ),       # one warp, 4375 slots: every ring slot reused many times
+    ("f32", (1, 70001, 32), _abi.KERNEL_SEQUENTIAL_PAIR),    # two warps, 2188 slots, a ragged last one
+    ("bf16", (2, 30001, 48), _abi.KERNEL_SEQUENTIAL_SPLIT),  # half-warps, partial channel groups
 ])
 def test_sequential_many_waves_and_long_sequences(dtype, shape, forced):
     if forced:
-        sgr.set_kernel_override(SEQ)
+        sgr.set_kernel_override(forced)
     pl = plan(*shape, dtype)
-    assert pl["kernel"] == SEQ
+    assert pl["kernel"] == (forced or SEQ)
     k, hx, h0 = small("mingru", *shape, dtype, "u01_1", seed=101)
     h = sgr.mingru_scan(*dev(k, hx, h0))
     r, s, x0 = small("minmax", *shape, dtype, "u01_1", seed=102)
