@@ -449,12 +449,16 @@ SGR_API sgr_status_t sgr_set_tile_override(int channel_lanes, int rows_per_threa
 
 /*
  * Tuning/testing knob, process-wide: 0 automatic (for aligned vector-width
- * rows: the channel-sequential kernel when B x ceil(D / 32) reaches 6 (fp32)
- * or 9 (bf16) warps per SM, the pipelined kernel otherwise; the tile kernel
- * for anything else), 1 force the tile kernel, 2 pipelined with 7 data warps
- * per block (two blocks per SM), 3 pipelined with 15 data warps (one block per
- * SM, tiles twice as long), 4 channel-sequential (one warp walks the whole
- * sequence of a group of 32 channels), 2-4 wherever the fast path applies.
+ * rows: a channel-sequential kernel when the 32-channel groups B x ceil(D / 32)
+ * reach 6 per SM -- two warps per group below 24 (bf16) or 32 (fp32) groups
+ * per SM, one warp per group above -- the pipelined kernel otherwise; the tile
+ * kernel for anything else), 1 force the tile kernel, 2 pipelined with 7 data
+ * warps per block (two blocks per SM), 3 pipelined with 15 data warps (one
+ * block per SM, tiles twice as long), 4 channel-sequential with one warp per
+ * group of 32 channels walking the whole sequence, 5 channel-sequential with
+ * each slot's 16 rows split between the two half-warps of a warp (groups of
+ * 16 channels), 6 channel-sequential with two warps per group of 32 channels
+ * splitting each 32-row slot; 2-6 wherever the fast path applies.
  */
 SGR_API sgr_status_t sgr_set_kernel_override(int kernel);
 
@@ -467,7 +471,11 @@ typedef struct sgr_plan {
                                    7 data warps; 3: pipelined, 15 data warps;
                                    4: channel-sequential, one warp per channel
                                    group and the whole of T (one chunk; warps =
-                                   warps per block, stages = load-ring slots)   */
+                                   warps per block, stages = load-ring slots);
+                                   5: the same with 16-channel groups, the rows
+                                   of each slot split between half-warps;
+                                   6: two warps per 32-channel group, each slot
+                                   of 32 rows split between them                */
     int32_t channels_per_thread;
     int32_t channel_lanes;      /* lanes across D per warp                         */
     int32_t rows_per_thread;
