@@ -286,6 +286,9 @@ def scan_fn(w, p, q, init, out, ws):
     return lambda: f(p, q, init, out=out, workspace=ws)
 
 
+PASS_SUFFIX = {"backward": "_backward", "decay": "_decay", "decay_backward": "_decay_backward"}
+
+
 def plan_kernel(plan) -> str:
     """The device kernel a scan plan launches (the library's kernel kinds)."""
     return {1: "sgr::scan_tile_kernel", 2: "sgr::scan_pipelined_kernel", 3: "sgr::scan_pipelined_kernel",
@@ -680,6 +683,34 @@ def run_b200(args):
         kernel_name = backward_kernel(w)
         ws = wsb
         args.no_e2e = True
+    profile_key = w.name
+    if args.pass_ in ("decay", "decay_backward"):
+        # the time-decayed minGRU on the workload: gaps ~ Exp(1) per (b, t),
+        # rates ~ U(0, 1) per channel, fp32 (the decay rows' recipe)
+        if w.op != "mingru":
+            raise SystemExit("bench.py: time decay is a minGRU variant")
+        g = torch.Generator(device=device).manual_seed(w.seed + 29)
+        gaps = torch.empty(w.B, w.T, device=device).exponential_(1.0, generator=g)
+        lam = torch.rand(w.D, device=device, generator=g)
+        code = 0 if w.dtype == "f32" else 1
+        wsd = sgr.Workspace(max(sgr.workspace_size("mingru", w.B, w.T, w.D, p.dtype),
+                                sgr._abi.lib().sgr_backward_workspace_size(0, w.B, w.T, w.D, code)), device)
+        extra = w.B * w.T * 4 + w.D * 4                 # gaps and rates
+        sgr.mingru_scan_decay(p, q, init, gaps, lam, out=out, workspace=wsd)
+        if args.pass_ == "decay":
+            fn = lambda: sgr.mingru_scan_decay(p, q, init, gaps, lam, out=out, workspace=wsd)  # noqa: E731
+            bytes_step = w.algorithmic_bytes() + extra
+            kernel_name = profile_kernel(sgr._abi.plan(0, w.B, w.T, w.D, code, True, decay=True))
+        else:
+            gy = torch.randn(p.shape, device=device, generator=g).to(p.dtype)
+            fn = lambda: sgr.mingru_scan_decay_backward(p, q, init, gaps, lam, out, gy,  # noqa: E731
+                                                        workspace=wsd)
+            bytes_step = 6 * w.n_elems * w.elem_bytes + extra + w.D * 4 + \
+                (2 * w.B * w.D * w.elem_bytes if init is not None else 0)
+            kernel_name = backward_kernel(w)
+        profile_key = w.name.replace("mingru_", "mingru_decay_", 1)
+        ws = wsd
+        args.no_e2e = True
 
     for _ in range(args.warmup):
         fn()
@@ -735,7 +766,7 @@ def run_b200(args):
     achieved = bytes_step / launch_max / 1e9
     plan = sgr._abi.plan(0 if w.op == "mingru" else 1, w.B, w.T, w.D, 0 if w.dtype == "f32" else 1, True)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": UNIT,
-                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name, kernel_name.split("::")[1]),
+                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(profile_key, kernel_name.split("::")[1]),
                 "peak_source": peak_src, "kernel": kernel_name,
                 "bytes_per_launch": bytes_step,
                 "launch_us": round(launch_max * 1e6, 2)}
@@ -753,7 +784,7 @@ def run_b200(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(agg["ms_per_step"], 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic (seeded torch generator on the device)",
-        "config": {"workload": w.name, "op": f"{w.op}_scan" + ("_backward" if args.pass_ == "backward" else ""),
+        "config": {"workload": w.name, "op": f"{w.op}_scan" + PASS_SUFFIX.get(args.pass_, ""),
                    "B": w.B, "T": w.T, "D": w.D,
                    "io_dtype": w.dtype, "initial_state": init is not None,
                    "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
@@ -793,8 +824,9 @@ def run_b200(args):
                      "mingru_b16_t2048_d4096_bf16_h0"):
             rows[name.replace("_b", "_backward_b", 1)] = measure_backward_row(WORKLOADS[name], device)
             torch.cuda.empty_cache()
-        rows.update(measure_decay_rows(WORKLOADS["mingru_b8_t4096_d1024_f32_h0"], device))
-        torch.cuda.empty_cache()
+        for name in ("mingru_b8_t4096_d1024_f32_h0", "mingru_b16_t2048_d4096_bf16_h0"):
+            rows.update(measure_decay_rows(WORKLOADS[name], device))
+            torch.cuda.empty_cache()
         for name in ("mingru_b8_t4096_d1024_f32_h0", "mingru_b1_t131072_d512_f32_h0"):
             rows[name.replace("mingru_", "mingru_summary_", 1)] = measure_summary_row(WORKLOADS[name], device)
             torch.cuda.empty_cache()
@@ -843,7 +875,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(wall / args.steps * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded torch generator)", "impl": "reference",
-        "config": {"workload": w.name, "op": f"{w.op}_scan" + ("_backward" if args.pass_ == "backward" else ""),
+        "config": {"workload": w.name, "op": f"{w.op}_scan" + PASS_SUFFIX.get(args.pass_, ""),
                    "B": w.B, "T": w.T, "D": w.D,
                    "io_dtype": w.dtype, "initial_state": ins is not None, "global_batch": w.B,
                    "seq_len": w.T, "parallelism": "cpu"},
@@ -862,9 +894,11 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward", "projected"],
-                    help="time the scan (default), its gradient kernel on the workload, or the input "
-                         "projection fused with the scan (B8 T4096 D1024 d_in 1024)")
+    ap.add_argument("--pass", dest="pass_", default="forward",
+                    choices=["forward", "backward", "decay", "decay_backward", "projected"],
+                    help="time the scan (default), its gradient kernel on the workload, the time-decayed "
+                         "minGRU or its gradient on the workload, or the input projection fused with the "
+                         "scan (B8 T4096 D1024 d_in 1024)")
     ap.add_argument("--no-rows", action="store_true", help="skip the other hot-path rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")

@@ -97,9 +97,9 @@ struct BwdParams {
 // layout (lane (g, j) of warp w owns channels [g V, g V + V) of processing rows
 // [(w J + j) R, (w J + j) R + R)); processing row rho of a tile is time row
 // ct TR + TR - 1 - rho.  Tiles are numbered chain-fastest in processing order
-// and, when the sequence spans several chunks, handed to blocks by a ticket
-// counter in the order the blocks start (take_tile), so every look-back waits
-// on a tile that a running block already holds.
+// and, when the sequence spans several chunks, handed to persistent blocks by
+// a ticket counter (for_each_ticket), so every look-back waits on a tile that
+// a running block holds.
 template <class BOp, typename IO, int V, int CG, int R, int W, int MINB>
 __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_backward_kernel(const BwdParams bp) {
     constexpr int J = 32 / CG;
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_backward_kernel(const
     const ScanParams &p = bp.s;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int64_t tile = take_tile(p.ticket);
+    for_each_ticket(p.ticket, p.n_tiles, [&](const int64_t tile, auto take_next) {
 
     if (warp < W) {
         const TileCoord tc = tile_coord(p, uint32_t(tile));
@@ -215,6 +215,7 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_backward_kernel(const
         }
         named_barrier_sync(1, NT);   // summaries are in shared memory
         named_barrier_sync(2, NT);   // the carry warp has written the incoming gradients
+        take_next();                 // the tile's look-back is over: take the next ticket
 
         float lam[V], dl[V];
 #pragma unroll
@@ -267,6 +268,7 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_backward_kernel(const
         named_barrier_sync(1, NT);
         carry_tile<Op, IO, CV, TC, W>(p, tile, s_tot, lane, [&] { named_barrier_sync(2, NT); });
     }
+    });
 }
 
 }  // namespace sgr

@@ -129,6 +129,33 @@ struct MinGRUOp {
         const float2 hp = __fadd2_rn(make_float2(hx0, hx1), make_float2(0.5f, 0.5f));
         b = __fmul2_rn(z, make_float2(fmaxf(hp.x, s.x), fmaxf(hp.y, s.y)));
     }
+    // The same pairs with one reciprocal shared by the two gates (3 MUFU
+    // operations per element instead of 4), for bf16 I/O: with
+    // e_k = 2^(min(k log2 e, 120)) and e_h = 2^(-|hx| log2 e) <= 1,
+    // q = 1 / ((1 + e_k)(1 + e_h)) stays a normal number (the product is at
+    // most 2^121), z = e_k (1 + e_h) q = sigmoid(k), a = 1 - z,
+    // sigmoid(-|hx|) = e_h (1 + e_k) q and g = max(hx + 0.5, sigmoid(-|hx|))
+    // (equal to g(hx) for either sign of hx).  a = 1 - z is exact where
+    // k <= 0 (z <= 1/2) and carries an absolute error of an fp32 ulp of 1
+    // where k >> 0: far below the bf16 rounding of the outputs, not enough
+    // for the fp32 bar on long closed-gate stretches, hence bf16 only.
+    // k = -inf gives z = 0 and a = 1 exactly; hx = -inf gives g = 0.
+    static __device__ __forceinline__ void element_rows_lean(float k0, float hx0, float k1, float hx1,
+                                                             float2 &a, float2 &b) {
+        const float2 tk = __fmul2_rn(make_float2(k0, k1), make_float2(-kNegLog2e, -kNegLog2e));
+        const float2 ek = make_float2(fast_exp2(fminf(tk.x, 120.f)), fast_exp2(fminf(tk.y, 120.f)));
+        const float2 eh = make_float2(fast_exp2(fabsf(hx0) * kNegLog2e), fast_exp2(fabsf(hx1) * kNegLog2e));
+        const float2 one = make_float2(1.f, 1.f);
+        const float2 dk = __fadd2_rn(ek, one), dh = __fadd2_rn(eh, one);
+        const float2 pr = __fmul2_rn(dk, dh);
+        const float2 q = make_float2(fast_rcp(pr.x), fast_rcp(pr.y));
+        const float2 z = __fmul2_rn(ek, __fmul2_rn(dh, q));                    // sigmoid(k)
+        a = __ffma2_rn(z, make_float2(-1.f, -1.f), one);                        // sigmoid(-k)
+        const float2 sh = __fmul2_rn(eh, __fmul2_rn(dk, q));                   // sigmoid(-|hx|)
+        const float2 hp = __fadd2_rn(make_float2(hx0, hx1), make_float2(0.5f, 0.5f));
+        b = __fmul2_rn(z, make_float2(fmaxf(hp.x, sh.x), fmaxf(hp.y, sh.y)));
+    }
+    static constexpr bool kLeanRows = true;
     // fold a step into a running pair, two channels at once: (A, B) <- (A a, B a + b)
     static __device__ __forceinline__ void fold2(float2 &A, float2 &B, float2 a, float2 b) {
         B = __ffma2_rn(B, a, b);
@@ -158,6 +185,7 @@ struct MinMaxOp {
         u = make_float2(r0, r1);
         l = make_float2(s0, s1);
     }
+    static constexpr bool kLeanRows = false;
     static __device__ __forceinline__ float step(float u, float l, float x) { return fmaxf(fminf(x, u), l); }
     static __device__ __forceinline__ float default_init() { return 0.f; }
     static __device__ __forceinline__ void fold2(float2 &U, float2 &L, float2 u, float2 l) {
@@ -596,15 +624,36 @@ __device__ __forceinline__ void fold_warps(float2 (*s_tot)[TC], int ch, float2 (
     }
 }
 
-// The tile a block works on: the next ticket when the launch hands tiles out
-// in start order (one atomic per block, broadcast through shared memory;
-// every thread of the block must call this), else blockIdx.x.
-__device__ __forceinline__ int64_t take_tile(uint32_t *ticket) {
-    if (ticket == nullptr) return blockIdx.x;
-    __shared__ uint32_t s_ticket;
-    if (threadIdx.x == 0) s_ticket = atomicAdd(ticket, 1u);
+// The tiles a block works on.  With a ticket counter (the call zeroes it on
+// the stream before the launch) the block takes tickets in increasing order
+// until they run out.  body(tile, take_next) runs on every thread; it calls
+// take_next() once the tile's incoming state is resolved (after its own
+// look-back), and thread 0 then takes the next ticket, so the atomic's
+// latency hides behind the rest of the tile (the replay and stores).  A block
+// never holds a ticket it has not started while it waits: every tile a
+// look-back waits for is held by a running block that is working on it (or
+// has finished it), and tiles wait only for smaller tickets, so waits never
+// form a cycle, and a wait that gives up delays no unrelated tile.  Without
+// a counter: the tile of the block's index.  Every thread of the block must
+// call this; there is a block barrier between tiles.
+template <class Body>
+__device__ __forceinline__ void for_each_ticket(uint32_t *ticket, int64_t n_tiles, Body body) {
+    if (ticket == nullptr) {
+        body(int64_t(blockIdx.x), [] {});
+        return;
+    }
+    __shared__ uint32_t s_next[2];
+    if (threadIdx.x == 0) s_next[0] = atomicAdd(ticket, 1u);
     __syncthreads();
-    return s_ticket;
+    for (int it = 0;; ++it) {
+        const int64_t tile = s_next[it & 1];
+        if (tile >= n_tiles) break;
+        uint32_t *next = &s_next[(it + 1) & 1];
+        body(tile, [&] {
+            if (threadIdx.x == 0) *next = atomicAdd(ticket, 1u);
+        });
+        __syncthreads();                 // shared state reused by the next tile; the next ticket visible
+    }
 }
 
 // -------------------------------------------------------- tile kernel
@@ -615,14 +664,13 @@ __device__ __forceinline__ int64_t take_tile(uint32_t *ticket) {
 // R (rows per thread), W (data warps).  J = 32 / CG row groups per warp,
 // TR = W * J * R, TC = CG * V.  Tiles are numbered chain-fastest:
 // tile = chunk * n_chains + chain, chain = b * n_dt + dt.  When the sequence
-// spans several chunks a block does not take the tile of its blockIdx: it
-// takes the next number from a ticket counter in the workspace (zeroed in the
-// stream before the launch), so tiles are handed out in the order blocks
-// actually start, whatever order the hardware dispatches them in.  Every
-// look-back then waits only for tiles that running blocks already hold, and
-// a block publishes its summary before it waits, so waits never form a cycle.
-// Used for the scalar (unaligned) variant and as a cross-check of the
-// pipelined kernel.
+// spans several chunks the blocks are persistent and take their tiles from a
+// ticket counter in the workspace (for_each_ticket), so tiles are handed out
+// in the order blocks reach them, whatever order the hardware dispatches
+// blocks in.  Every look-back then waits only for tiles that running blocks
+// hold, and a block publishes its summary before it waits, so waits never
+// form a cycle.  Used for the scalar (unaligned) variant, for shapes with few
+// tiles, and as a cross-check of the pipelined kernel.
 template <class Op, typename IO, int V, int CG, int R, int W, int MINB>
 __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const ScanParams p) {
     constexpr int J = 32 / CG;
@@ -637,7 +685,7 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const Sca
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int64_t tile = take_tile(p.ticket);
+    for_each_ticket(p.ticket, p.n_tiles, [&](const int64_t tile, auto take_next) {
 
     if (warp < W) {
         const TileCoord tc = tile_coord(p, uint32_t(tile));
@@ -714,6 +762,7 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const Sca
         }
         named_barrier_sync(1, NT);   // totals are in shared memory
         named_barrier_sync(2, NT);   // the carry warp has written the warp states
+        take_next();                 // the tile's look-back is over: take the next ticket
 
         float st[V];
 #pragma unroll
@@ -733,6 +782,7 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const Sca
         named_barrier_sync(1, NT);
         carry_tile<Op, IO, CV, TC, W>(p, tile, s_tot, lane, [&] { named_barrier_sync(2, NT); });
     }
+    });
 }
 
 // --------------------------------------------------- pipelined kernel

@@ -94,10 +94,19 @@ struct SeqParams {
     int slots;           // load ring depth S
 };
 
+// The step pairs of two rows: bf16 I/O takes the shared-reciprocal form
+// (one MUFU operation fewer per element; these kernels keep the MUFU pipe
+// busy), fp32 I/O the form with relative-accurate gates for either sign.
+template <class Op, typename IO>
+__device__ __forceinline__ void seq_rows(float k0, float hx0, float k1, float hx1, float2 &a, float2 &b) {
+    if constexpr (sizeof(IO) == 2 && Op::kLeanRows) Op::element_rows_lean(k0, hx0, k1, hx1, a, b);
+    else Op::element_rows(k0, hx0, k1, hx1, a, b);
+}
+
 // Time decay in the channel-sequential kernels: the gaps u_t are per (batch
 // row, row), shared by a warp's channels.  A warp's 16 rows of a slot have
 // their gaps spread across the lanes, lane l holding row y0 + (l % 16)'s
-// (0 past T: gamma = 1), loaded one slot ahead so that no step waits for
+// (0 past T: gamma = 1), loaded two slots ahead so that no step waits for
 // them; each row's gap is then taken from its lane by one shuffle.
 __device__ __forceinline__ float seq_slot_gap(const ScanParams &p, int64_t b, int64_t y0, int lane) {
     const int64_t t = y0 + (lane & (kSeqRows - 1));
@@ -171,9 +180,11 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
 
     float h = load_init<IO>(p, b, d, Op::default_init());           // state entering the slot
     [[maybe_unused]] float lam2 = 0.f, gcur = 0.f;
+    [[maybe_unused]] float gnext = 0.f;
     if constexpr (Op::kDecay) {
         lam2 = decay_lam2(p, d);
         gcur = seq_slot_gap(p, b, 0, lane);
+        gnext = seq_slot_gap(p, b, kSeqRows, lane);
     }
 
     uint32_t wait_limit = kMbarLimit;
@@ -181,8 +192,8 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
     int s = 0;                 // ring slot of slot i
     uint32_t phase = 0;        // parity of that slot's current use
     for (int i = 0; i < n_slots; ++i) {
-        [[maybe_unused]] float gnext = 0.f;
-        if constexpr (Op::kDecay) gnext = seq_slot_gap(p, b, int64_t(i + 1) * kSeqRows, lane);
+        [[maybe_unused]] float gnext2 = 0.f;
+        if constexpr (Op::kDecay) gnext2 = seq_slot_gap(p, b, int64_t(i + 2) * kSeqRows, lane);
         if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
             // a copy that never lands: record it, make every later output NaN
             // and stop waiting at length (the kernel still ends)
@@ -222,7 +233,7 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
 #pragma unroll
             for (int r = 0; r < LROWS; r += 2) {
                 float2 a, c;
-                Op::element_rows(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
+                seq_rows<Op, IO>(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
                 if constexpr (Op::kDecay) {
                     a.x *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r));
                     a.y *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r + 1));
@@ -239,7 +250,7 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
 #pragma unroll
             for (int r = 0; r < LROWS; r += 2) {
                 float2 a, c;
-                Op::element_rows(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
+                seq_rows<Op, IO>(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
                 if constexpr (Op::kDecay) {
                     a.x *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, part * LROWS + r));
                     a.y *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, part * LROWS + r + 1));
@@ -269,7 +280,10 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
             tma_store_3d(&map_out, obuf, x0, i * kSeqRows, int(b));
             bulk_commit();
         }
-        if constexpr (Op::kDecay) gcur = gnext;
+        if constexpr (Op::kDecay) {
+            gcur = gnext;
+            gnext = gnext2;
+        }
     }
     if (lane == 0) bulk_wait_all();
 }
@@ -279,12 +293,15 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
 // block's warps w = 0, 1 scan the same 32 channels of one batch row (lane =
 // channel, 64- or 128-byte rows, no bank conflicts), warp w taking rows
 // [32 i + 16 w, 32 i + 16 w + 16) of slot i through its own ring of 16-row
-// boxes.  Each warp folds its 16 step maps into one pair and puts it in
-// shared memory (double-buffered by slot parity); after one named barrier per
+// boxes.  Each warp folds its 16 step maps into one pair -- rows r and r + 8
+// as two chains, one fp32x2 operation advancing both, the running composites
+// kept -- and puts it in shared memory (double-buffered by slot parity); after one named barrier per
 // slot both warps read the other's pair and compose the slot's chain
 // themselves -- h_mid = P0(h), h_end = P1(h_mid) -- so no second hand-off is
-// needed: warp 0 replays its rows from h, warp 1 from h_mid, and both carry
-// h_end into the next slot.  A warp whose copy never landed publishes a NaN
+// needed: warp 0 takes h, warp 1 h_mid as its incoming state, and both carry
+// h_end into the next slot.  A row's output is then its chain's running
+// composite applied to the chain's incoming state, one independent fp32x2
+// operation for two rows (no replay chain).  A warp whose copy never landed publishes a NaN
 // pair, so both warps' later outputs turn NaN.  One staging buffer per warp
 // (its previous store has long finished reading it by the time the next
 // slot's outputs are written), which leaves the shared memory to the load
@@ -343,9 +360,11 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
 
     float h = load_init<IO>(p, b, d, Op::default_init());           // state entering the slot
     [[maybe_unused]] float lam2 = 0.f, gcur = 0.f;
+    [[maybe_unused]] float gnext = 0.f;
     if constexpr (Op::kDecay) {
         lam2 = decay_lam2(p, d);
         gcur = seq_slot_gap(p, b, w * kSeqRows, lane);
+        gnext = seq_slot_gap(p, b, kSlotRows + w * kSeqRows, lane);
     }
 
     uint32_t wait_limit = kMbarLimit;
@@ -353,8 +372,8 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
     int s = 0;
     uint32_t phase = 0;
     for (int i = 0; i < n_slots; ++i) {
-        [[maybe_unused]] float gnext = 0.f;
-        if constexpr (Op::kDecay) gnext = seq_slot_gap(p, b, int64_t(i + 1) * kSlotRows + w * kSeqRows, lane);
+        [[maybe_unused]] float gnext2 = 0.f;
+        if constexpr (Op::kDecay) gnext2 = seq_slot_gap(p, b, int64_t(i + 2) * kSlotRows + w * kSeqRows, lane);
         if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
             wait_limit = 1;
             if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
@@ -377,21 +396,28 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
             phase ^= 1u;
         }
         bad = __any_sync(0xffffffffu, bad);
-        float am[kSeqRows], cm[kSeqRows];
+        // rows r and r + 8 as two chains, each fp32x2 operation spanning
+        // both: the step maps of the pair, then the running composites from
+        // the start of each chain (PA, PB: the pair mapping the chain's
+        // incoming state to row r's, resp. row r + 8's, output)
+        constexpr int H = kSeqRows / 2;
+        float2 PA[H], PB[H];
+        float2 A = make_float2(Op::identity().x, Op::identity().x);
+        float2 Bc = make_float2(Op::identity().y, Op::identity().y);
 #pragma unroll
-        for (int r = 0; r < kSeqRows; r += 2) {
+        for (int r = 0; r < H; ++r) {
             float2 a, c;
-            Op::element_rows(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
+            seq_rows<Op, IO>(x0r[r], x1r[r], x0r[r + H], x1r[r + H], a, c);
             if constexpr (Op::kDecay) {
                 a.x *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r));
-                a.y *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r + 1));
+                a.y *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r + H));
             }
-            am[r] = a.x; cm[r] = c.x;
-            am[r + 1] = a.y; cm[r + 1] = c.y;
+            Op::fold2(A, Bc, a, c);
+            PA[r] = A;
+            PB[r] = Bc;
         }
-        float2 P = make_float2(am[0], cm[0]);
-#pragma unroll
-        for (int r = 1; r < kSeqRows; ++r) P = Op::combine(P, make_float2(am[r], cm[r]));
+        // the warp's 16 rows: the first chain, then the second
+        float2 P = Op::combine(make_float2(A.x, Bc.x), make_float2(A.y, Bc.y));
         if (bad) P = make_float2(__int_as_float(0x7fffffff), __int_as_float(0x7fffffff));
         float2 *xb = xpair + (i & 1) * kPairWarps * 32;
         xb[w * 32 + lane] = P;
@@ -399,16 +425,20 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
         const float2 Q = xb[(1 - w) * 32 + lane];
         const float hmid = Op::apply(w ? Q : P, h);
         const float hend = Op::apply(w ? P : Q, hmid);
-        float y = w ? hmid : h;
+        const float hin = w ? hmid : h;                              // this warp's incoming state
         h = hend;
+        // incoming states of the two chains: the warp's, and the state after row 7
+        float2 hh = make_float2(hin, Op::apply(make_float2(A.x, Bc.x), hin));
+        if (bad) hh = make_float2(__int_as_float(0x7fffffff), __int_as_float(0x7fffffff));   // NaN outputs
         if (lane == 0) bulk_wait_read<0>();                          // the last slot's store has read the buffer
         __syncwarp();
         const uint32_t obuf = outb;
         const uint32_t dst = obuf + uint32_t(lane) * uint32_t(sizeof(IO));
 #pragma unroll
-        for (int r = 0; r < kSeqRows; ++r) {
-            y = Op::step(am[r], cm[r], y);
-            LR::store(dst + r * kRowBytes, y);
+        for (int r = 0; r < H; ++r) {
+            const float2 y = Op::step2(PA[r], PB[r], hh);           // rows r and r + 8, independent
+            LR::store(dst + r * kRowBytes, y.x);
+            LR::store(dst + (r + H) * kRowBytes, y.y);
         }
         fence_proxy_async();
         __syncwarp();
@@ -417,7 +447,10 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
             tma_store_3d(&map_out, obuf, x0, y0, int(b));
             bulk_commit();
         }
-        if constexpr (Op::kDecay) gcur = gnext;
+        if constexpr (Op::kDecay) {
+            gcur = gnext;
+            gnext = gnext2;
+        }
     }
     if (lane == 0) bulk_wait_all();
 }
@@ -510,9 +543,11 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
         (bp.init && d < p.D) ? load_scalar<IO>(static_cast<const IO *>(bp.init) + b * bp.init_bs + d)
                              : BOp::default_state();
     [[maybe_unused]] float lam2 = 0.f, dl = 0.f, gcur = 0.f;
+    [[maybe_unused]] float gnext = 0.f;
     if constexpr (BOp::kDecay) {
         lam2 = decay_lam2(p, d);
         gcur = seq_slot_gap(p, b, int64_t(n_slots - 1) * kSeqRows, lane);
+        gnext = seq_slot_gap(p, b, int64_t(n_slots - 2) * kSeqRows, lane);
     }
 
     float lam = 0.f;           // dL/d (state after the rows still to walk)
@@ -522,8 +557,8 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
     uint32_t phase = 0;
     for (int i = 0; i < n_slots; ++i) {
         const int j = n_slots - 1 - i;
-        [[maybe_unused]] float gnext = 0.f;                         // the gaps of the slot below
-        if constexpr (BOp::kDecay) gnext = seq_slot_gap(p, b, int64_t(j - 1) * kSeqRows, lane);
+        [[maybe_unused]] float gnext2 = 0.f;                        // the gaps two slots below
+        if constexpr (BOp::kDecay) gnext2 = seq_slot_gap(p, b, int64_t(j - 2) * kSeqRows, lane);
         if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
             wait_limit = 1;
             if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
@@ -594,7 +629,10 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
             tma_store_3d(&map_d1, obuf + kOpBytes, x0, j * kSeqRows, int(b));
             bulk_commit();
         }
-        if constexpr (BOp::kDecay) gcur = gnext;
+        if constexpr (BOp::kDecay) {
+            gcur = gnext;
+            gnext = gnext2;
+        }
     }
     if (bp.dinit && d < p.D) {
         const float y[1] = {bad ? __int_as_float(0x7fffffff) : lam};

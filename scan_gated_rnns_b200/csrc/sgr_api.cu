@@ -383,33 +383,6 @@ size_t rows_span(int64_t B, int64_t D, int64_t bs, int esz) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// ---- tile kernel launch
-template <class Op, typename IO, int V, int CG, int R>
-cudaError_t launch_tile(const ScanParams &sp, cudaStream_t s) {
-    if constexpr (R * V > 32) {
-        return cudaErrorInvalidConfiguration;   // never planned (see make_plan)
-    } else {
-        // registers a data thread keeps live: its tile (2RV), one pair per
-        // channel (2V) and about 24 for addressing; blocks of 256 threads
-        constexpr int NEED = 2 * R * V + 2 * V + 24;
-        constexpr int MINB = NEED <= 56 ? 4 : (NEED <= 72 ? 3 : 2);
-        scan_tile_kernel<Op, IO, V, CG, R, kWarps, MINB>
-            <<<dim3(unsigned(sp.n_tiles)), (kWarps + 1) * 32, 0, s>>>(sp);
-        return cudaGetLastError();
-    }
-}
-
-template <class Op, typename IO, int V, int CG>
-cudaError_t dispatch_tile_r(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
-    switch (pl.r) {
-        case 1: return launch_tile<Op, IO, V, CG, 1>(sp, s);
-        case 2: return launch_tile<Op, IO, V, CG, 2>(sp, s);
-        case 4: return launch_tile<Op, IO, V, CG, 4>(sp, s);
-        default: return launch_tile<Op, IO, V, CG, 8>(sp, s);
-    }
-}
-
-// ---- pipelined kernel launch: persistent, co-resident blocks
 struct DeviceInfo {
     int sms = 0;
 };
@@ -426,6 +399,67 @@ DeviceInfo device_info(int dev) {
     }
     return d;
 }
+
+// ---- tile kernel launch
+// Blocks of a tile-kernel launch: one per tile without a ticket counter;
+// with one, as many as stay resident at once (the blocks loop over tickets),
+// from the kernel's occupancy on the current device, read once per kernel
+// and device.
+template <class Kernel>
+cudaError_t tile_grid(Kernel kernel, int threads, int64_t n_tiles, bool ticket, int64_t *grid) {
+    *grid = n_tiles;
+    if (!ticket) return cudaSuccess;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    static std::mutex mu;
+    static std::vector<std::pair<std::pair<const void *, int>, int>> cache;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_pair(reinterpret_cast<const void *>(kernel), dev);
+    int per_sm = 0;
+    for (const auto &c : cache)
+        if (c.first == key) per_sm = c.second;
+    if (per_sm == 0) {
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0)) != cudaSuccess) return e;
+        if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+        cache.emplace_back(key, per_sm);
+    }
+    const DeviceInfo di = device_info(dev);
+    if (di.sms <= 0) return cudaErrorInvalidDevice;
+    *grid = std::min<int64_t>(n_tiles, int64_t(per_sm) * di.sms);
+    return cudaSuccess;
+}
+
+template <class Op, typename IO, int V, int CG, int R>
+cudaError_t launch_tile(const ScanParams &sp, cudaStream_t s) {
+    if constexpr (R * V > 32) {
+        return cudaErrorInvalidConfiguration;   // never planned (see make_plan)
+    } else {
+        // registers a data thread keeps live: its tile (2RV), one pair per
+        // channel (2V) and about 24 for addressing; blocks of 256 threads
+        constexpr int NEED = 2 * R * V + 2 * V + 24;
+        constexpr int MINB = NEED <= 56 ? 4 : (NEED <= 72 ? 3 : 2);
+        auto kernel = scan_tile_kernel<Op, IO, V, CG, R, kWarps, MINB>;
+        int64_t grid = 0;
+        const cudaError_t e = tile_grid(kernel, (kWarps + 1) * 32, sp.n_tiles, sp.ticket != nullptr, &grid);
+        if (e != cudaSuccess) return e;
+        kernel<<<dim3(unsigned(grid)), (kWarps + 1) * 32, 0, s>>>(sp);
+        return cudaGetLastError();
+    }
+}
+
+template <class Op, typename IO, int V, int CG>
+cudaError_t dispatch_tile_r(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
+    switch (pl.r) {
+        case 1: return launch_tile<Op, IO, V, CG, 1>(sp, s);
+        case 2: return launch_tile<Op, IO, V, CG, 2>(sp, s);
+        case 4: return launch_tile<Op, IO, V, CG, 4>(sp, s);
+        default: return launch_tile<Op, IO, V, CG, 8>(sp, s);
+    }
+}
+
+// ---- pipelined kernel launch: persistent, co-resident blocks
 
 // Tensor maps of a decay's gaps (B, T) fp32 rows with a batch stride and
 // rates (D,) fp32, for boxes of TR gaps of one batch row and TC rates; false
@@ -758,8 +792,11 @@ cudaError_t launch_bwd_tile(const BwdParams &bp, cudaStream_t s) {
         // pair per channel and about 24 for addressing; blocks of 256 threads
         constexpr int NEED = 4 * R * V + 2 * V + 24;
         constexpr int MINB = NEED <= 56 ? 4 : (NEED <= 72 ? 3 : 2);
-        scan_backward_kernel<BOp, IO, V, CG, R, kWarps, MINB>
-            <<<unsigned(bp.s.n_tiles), (kWarps + 1) * 32, 0, s>>>(bp);
+        auto kernel = scan_backward_kernel<BOp, IO, V, CG, R, kWarps, MINB>;
+        int64_t grid = 0;
+        const cudaError_t e = tile_grid(kernel, (kWarps + 1) * 32, bp.s.n_tiles, bp.s.ticket != nullptr, &grid);
+        if (e != cudaSuccess) return e;
+        kernel<<<unsigned(grid), (kWarps + 1) * 32, 0, s>>>(bp);
         return cudaGetLastError();
     }
 }
