@@ -134,7 +134,7 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_backward_kernel(const
         // rows r = 0..R-1 at time top - r: A, the upstream gradient, cP, cQ
         // (time decay: and E = (1 - z) h_{t-1} dgamma/dlambda, for dL/dlambda)
         float A[R][V], G[R][V], P[R][V], Q[R][V];
-        float E[BOp::kDecay ? R : 1][V];
+        [[maybe_unused]] float E[BOp::kDecay ? R : 1][V];
         [[maybe_unused]] float lam2[V];
         if constexpr (BOp::kDecay) {
 #pragma unroll

@@ -41,9 +41,15 @@ constexpr int kSeqOutBufs = 2;
 // rate, bounds this kernel, and 32-channel groups measured 13-40% faster.)
 template <typename IO> constexpr int seq_row_bytes() { return 32 * int(sizeof(IO)); }
 
+// Time decay through the copy engine: each slot carries its 16 rows' gaps
+// (a 64-byte box of the (B, T) gap array) in a 128-byte area after its
+// operand boxes, so they land with the slot on its mbarrier.
+constexpr uint32_t kSeqGapBytes = 128;
+
 // bytes of one warp's shared memory with S load slots of rows of `row_bytes`
-__host__ __device__ constexpr size_t seq_warp_bytes(int S, int row_bytes) {
-    return (size_t(S) * 2 * kSeqRows * row_bytes + size_t(kSeqOutBufs) * kSeqRows * row_bytes +
+// (gap: the per-slot gap area, 0 or kSeqGapBytes)
+__host__ __device__ constexpr size_t seq_warp_bytes(int S, int row_bytes, size_t gap = 0) {
+    return (size_t(S) * (2 * kSeqRows * row_bytes + gap) + size_t(kSeqOutBufs) * kSeqRows * row_bytes +
             size_t(S) * 8 + 127) / 128 * 128;
 }
 
@@ -112,6 +118,12 @@ __device__ __forceinline__ float seq_slot_gap(const ScanParams &p, int64_t b, in
     const int64_t t = y0 + (lane & (kSeqRows - 1));
     return (y0 >= 0 && t < p.T) ? decay_u(p, b, t) : 0.f;
 }
+// the same gap from a slot's gap area (rows past T were zero-filled: gamma = 1)
+__device__ __forceinline__ float seq_smem_gap(const ScanParams &p, uint32_t gaps, int lane) {
+    float g;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(g) : "r"(gaps + 4u * uint32_t(lane & (kSeqRows - 1))) : "memory");
+    return p.decay_log1p ? log1pf(g) : g;
+}
 
 // Block: WB independent warps; warp (blockIdx.x WB + w) scans channel group
 // (b, grp) of the batch.  Dynamic shared memory: WB x seq_warp_bytes(S).
@@ -131,11 +143,14 @@ __device__ __forceinline__ float seq_slot_gap(const ScanParams &p, int64_t b, in
 // (page "MinMax Recurrent Neural Cascades", Key properties: the pairs
 // compose associatively).  The two halves read rows 256 (bf16) or 512
 // (fp32) bytes apart, a 2-way shared-memory bank conflict per load.
-template <class Op, typename IO, int WB, int SPLIT = 1>
+template <class Op, typename IO, int WB, int SPLIT = 1, bool DT = false>
 __global__ void __launch_bounds__(WB * 32)
 scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap map0,
-                       const __grid_constant__ CUtensorMap map1, const __grid_constant__ CUtensorMap map_out) {
+                       const __grid_constant__ CUtensorMap map1, const __grid_constant__ CUtensorMap map_out,
+                       const __grid_constant__ CUtensorMap map_gap) {
     static_assert(SPLIT == 1 || SPLIT == 2, "one or two row groups per slot");
+    static_assert(!DT || Op::kDecay, "gaps through the copy engine need a decay operator");
+    constexpr uint32_t kGap = DT ? kSeqGapBytes : 0;
     using LR = LaneRow<IO>;
     constexpr int CW = 32 / SPLIT;                                   // channels of a warp's group
     constexpr int LROWS = kSeqRows / SPLIT;                          // rows of a slot per lane
@@ -157,19 +172,21 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
     const int part = lane / CW;                                      // the lane's rows of a slot
     const int64_t d = int64_t(x0) + ch;                              // the lane's channel
 
-    const uint32_t base = smem_addr(smem) + uint32_t(warp * seq_warp_bytes(S, kRowBytes));
-    const uint32_t ring = base;                                      // S slots: [k rows | hx rows]
-    const uint32_t outb = base + uint32_t(S) * 2 * kOpBytes;         // 2 staging buffers
+    constexpr uint32_t kSlot = 2 * kOpBytes + kGap;                 // [k rows | hx rows | gaps]
+    const uint32_t base = smem_addr(smem) + uint32_t(warp * seq_warp_bytes(S, kRowBytes, kGap));
+    const uint32_t ring = base;                                      // S slots
+    const uint32_t outb = base + uint32_t(S) * kSlot;                // 2 staging buffers
     const uint32_t bars = outb + kSeqOutBufs * kOpBytes;             // S mbarriers
     const uint32_t lane_off = uint32_t(part * LROWS * kRowBytes + ch * int(sizeof(IO)));
 
     const int n_slots = int((p.T + kSeqRows - 1) / kSeqRows);       // T < 2^31 (host check)
     auto issue = [&](int i, int s) {                                 // lane 0: rows of slot i into ring slot s
-        const uint32_t dst = ring + uint32_t(s) * 2 * kOpBytes;
+        const uint32_t dst = ring + uint32_t(s) * kSlot;
         const uint32_t bar = bars + 8u * uint32_t(s);
-        mbar_expect_tx(bar, 2 * kOpBytes);
+        mbar_expect_tx(bar, 2 * kOpBytes + (DT ? kSeqRows * 4 : 0));
         tma_load_3d(dst, &map0, x0, i * kSeqRows, int(b), bar);
         tma_load_3d(dst + kOpBytes, &map1, x0, i * kSeqRows, int(b), bar);
+        if constexpr (DT) tma_load_2d(dst + 2 * kOpBytes, &map_gap, i * kSeqRows, int(b), bar);
     };
     if (lane == 0) {
         for (int s = 0; s < S; ++s) mbar_init(bars + 8u * s, 1);
@@ -183,8 +200,10 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
     [[maybe_unused]] float gnext = 0.f;
     if constexpr (Op::kDecay) {
         lam2 = decay_lam2(p, d);
-        gcur = seq_slot_gap(p, b, 0, lane);
-        gnext = seq_slot_gap(p, b, kSeqRows, lane);
+        if constexpr (!DT) {
+            gcur = seq_slot_gap(p, b, 0, lane);
+            gnext = seq_slot_gap(p, b, kSeqRows, lane);
+        }
     }
 
     uint32_t wait_limit = kMbarLimit;
@@ -193,7 +212,7 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
     uint32_t phase = 0;        // parity of that slot's current use
     for (int i = 0; i < n_slots; ++i) {
         [[maybe_unused]] float gnext2 = 0.f;
-        if constexpr (Op::kDecay) gnext2 = seq_slot_gap(p, b, int64_t(i + 2) * kSeqRows, lane);
+        if constexpr (Op::kDecay && !DT) gnext2 = seq_slot_gap(p, b, int64_t(i + 2) * kSeqRows, lane);
         if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
             // a copy that never lands: record it, make every later output NaN
             // and stop waiting at length (the kernel still ends)
@@ -201,13 +220,14 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
             if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
             bad = true;
         }
-        const uint32_t src = ring + uint32_t(s) * 2 * kOpBytes + lane_off;
+        const uint32_t src = ring + uint32_t(s) * kSlot + lane_off;
         float x0r[LROWS], x1r[LROWS];
 #pragma unroll
         for (int r = 0; r < LROWS; ++r) {
             x0r[r] = LR::load(src + r * kRowBytes);
             x1r[r] = LR::load(src + kOpBytes + r * kRowBytes);
         }
+        if constexpr (DT) gcur = seq_smem_gap(p, ring + uint32_t(s) * kSlot + 2 * kOpBytes, lane);
         // staging buffer i % 2 is free once the store issued two slots ago
         // has read it (the warp synchronises just below)
         if (lane == 0) bulk_wait_read<kSeqOutBufs - 1>();
@@ -280,7 +300,7 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
             tma_store_3d(&map_out, obuf, x0, i * kSeqRows, int(b));
             bulk_commit();
         }
-        if constexpr (Op::kDecay) {
+        if constexpr (Op::kDecay && !DT) {
             gcur = gnext;
             gnext = gnext2;
         }
@@ -307,17 +327,21 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
 // slot's outputs are written), which leaves the shared memory to the load
 // ring.  Dynamic shared memory: 2 x seq_pair_warp_bytes(S) + the pair buffers.
 constexpr int kPairWarps = 2;
-__host__ __device__ constexpr size_t seq_pair_warp_bytes(int S, int row_bytes) {
-    return (size_t(S) * 2 * kSeqRows * row_bytes + size_t(kSeqRows) * row_bytes + size_t(S) * 8 + 127) / 128 * 128;
+__host__ __device__ constexpr size_t seq_pair_warp_bytes(int S, int row_bytes, size_t gap = 0) {
+    return (size_t(S) * (2 * kSeqRows * row_bytes + gap) + size_t(kSeqRows) * row_bytes + size_t(S) * 8 + 127) /
+           128 * 128;
 }
-__host__ __device__ constexpr size_t seq_pair_block_bytes(int S, int row_bytes) {
-    return kPairWarps * seq_pair_warp_bytes(S, row_bytes) + size_t(2) * kPairWarps * 32 * sizeof(float2);
+__host__ __device__ constexpr size_t seq_pair_block_bytes(int S, int row_bytes, size_t gap = 0) {
+    return kPairWarps * seq_pair_warp_bytes(S, row_bytes, gap) + size_t(2) * kPairWarps * 32 * sizeof(float2);
 }
 
-template <class Op, typename IO>
+template <class Op, typename IO, bool DT = false>
 __global__ void __launch_bounds__(kPairWarps * 32)
 scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorMap map0,
-                            const __grid_constant__ CUtensorMap map1, const __grid_constant__ CUtensorMap map_out) {
+                            const __grid_constant__ CUtensorMap map1, const __grid_constant__ CUtensorMap map_out,
+                            const __grid_constant__ CUtensorMap map_gap) {
+    static_assert(!DT || Op::kDecay, "gaps through the copy engine need a decay operator");
+    constexpr uint32_t kGap = DT ? kSeqGapBytes : 0;
     using LR = LaneRow<IO>;
     constexpr int CW = 32;
     constexpr int kRowBytes = CW * int(sizeof(IO));
@@ -336,20 +360,22 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
     const int x0 = int(grp) * CW;
     const int64_t d = int64_t(x0) + lane;
 
-    const uint32_t base = smem_addr(smem) + uint32_t(w * seq_pair_warp_bytes(S, kRowBytes));
+    constexpr uint32_t kSlot = 2 * kOpBytes + kGap;                 // [k rows | hx rows | gaps]
+    const uint32_t base = smem_addr(smem) + uint32_t(w * seq_pair_warp_bytes(S, kRowBytes, kGap));
     const uint32_t ring = base;
-    const uint32_t outb = base + uint32_t(S) * 2 * kOpBytes;        // one staging buffer
+    const uint32_t outb = base + uint32_t(S) * kSlot;               // one staging buffer
     const uint32_t bars = outb + kOpBytes;
-    float2 *xpair = reinterpret_cast<float2 *>(smem + kPairWarps * seq_pair_warp_bytes(S, kRowBytes));  // [2][2][32]
+    float2 *xpair = reinterpret_cast<float2 *>(smem + kPairWarps * seq_pair_warp_bytes(S, kRowBytes, kGap));  // [2][2][32]
 
     const int n_slots = int((p.T + kSlotRows - 1) / kSlotRows);     // T < 2^31 (host check)
     auto issue = [&](int i, int s) {
-        const uint32_t dst = ring + uint32_t(s) * 2 * kOpBytes;
+        const uint32_t dst = ring + uint32_t(s) * kSlot;
         const uint32_t bar = bars + 8u * uint32_t(s);
         const int y = i * kSlotRows + w * kSeqRows;
-        mbar_expect_tx(bar, 2 * kOpBytes);
+        mbar_expect_tx(bar, 2 * kOpBytes + (DT ? kSeqRows * 4 : 0));
         tma_load_3d(dst, &map0, x0, y, int(b), bar);
         tma_load_3d(dst + kOpBytes, &map1, x0, y, int(b), bar);
+        if constexpr (DT) tma_load_2d(dst + 2 * kOpBytes, &map_gap, y, int(b), bar);
     };
     if (lane == 0) {
         for (int s = 0; s < S; ++s) mbar_init(bars + 8u * s, 1);
@@ -363,8 +389,10 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
     [[maybe_unused]] float gnext = 0.f;
     if constexpr (Op::kDecay) {
         lam2 = decay_lam2(p, d);
-        gcur = seq_slot_gap(p, b, w * kSeqRows, lane);
-        gnext = seq_slot_gap(p, b, kSlotRows + w * kSeqRows, lane);
+        if constexpr (!DT) {
+            gcur = seq_slot_gap(p, b, w * kSeqRows, lane);
+            gnext = seq_slot_gap(p, b, kSlotRows + w * kSeqRows, lane);
+        }
     }
 
     uint32_t wait_limit = kMbarLimit;
@@ -373,19 +401,21 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
     uint32_t phase = 0;
     for (int i = 0; i < n_slots; ++i) {
         [[maybe_unused]] float gnext2 = 0.f;
-        if constexpr (Op::kDecay) gnext2 = seq_slot_gap(p, b, int64_t(i + 2) * kSlotRows + w * kSeqRows, lane);
+        if constexpr (Op::kDecay && !DT)
+            gnext2 = seq_slot_gap(p, b, int64_t(i + 2) * kSlotRows + w * kSeqRows, lane);
         if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
             wait_limit = 1;
             if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
             bad = true;
         }
-        const uint32_t src = ring + uint32_t(s) * 2 * kOpBytes + uint32_t(lane) * uint32_t(sizeof(IO));
+        const uint32_t src = ring + uint32_t(s) * kSlot + uint32_t(lane) * uint32_t(sizeof(IO));
         float x0r[kSeqRows], x1r[kSeqRows];
 #pragma unroll
         for (int r = 0; r < kSeqRows; ++r) {
             x0r[r] = LR::load(src + r * kRowBytes);
             x1r[r] = LR::load(src + kOpBytes + r * kRowBytes);
         }
+        if constexpr (DT) gcur = seq_smem_gap(p, ring + uint32_t(s) * kSlot + 2 * kOpBytes, lane);
         __syncwarp();                                                // the slot is in registers
         if (lane == 0 && !bad && i + S < n_slots) {
             fence_proxy_async();
@@ -447,7 +477,7 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
             tma_store_3d(&map_out, obuf, x0, y0, int(b));
             bulk_commit();
         }
-        if constexpr (Op::kDecay) {
+        if constexpr (Op::kDecay && !DT) {
             gcur = gnext;
             gnext = gnext2;
         }
@@ -477,8 +507,8 @@ namespace sgr {
 constexpr int kSeqBwdIn = 4;        // operands loaded per slot
 constexpr int kSeqBwdOut = 2;       // gradients stored per slot
 
-__host__ __device__ constexpr size_t seq_bwd_warp_bytes(int S, int row_bytes) {
-    return (size_t(S) * kSeqBwdIn * kSeqRows * row_bytes +
+__host__ __device__ constexpr size_t seq_bwd_warp_bytes(int S, int row_bytes, size_t gap = 0) {
+    return (size_t(S) * (kSeqBwdIn * kSeqRows * row_bytes + gap) +
             size_t(kSeqOutBufs) * kSeqBwdOut * kSeqRows * row_bytes + size_t(S) * 8 + 127) / 128 * 128;
 }
 
@@ -489,14 +519,17 @@ struct SeqBwdParams {
     int slots;           // load ring depth S
 };
 
-template <class BOp, typename IO, int WB>
+template <class BOp, typename IO, int WB, bool DT = false>
 __global__ void __launch_bounds__(WB * 32)
 scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CUtensorMap map_in0,
                                 const __grid_constant__ CUtensorMap map_in1,
                                 const __grid_constant__ CUtensorMap map_gy,
                                 const __grid_constant__ CUtensorMap map_fwd,
                                 const __grid_constant__ CUtensorMap map_d0,
-                                const __grid_constant__ CUtensorMap map_d1) {
+                                const __grid_constant__ CUtensorMap map_d1,
+                                const __grid_constant__ CUtensorMap map_gap) {
+    static_assert(!DT || BOp::kDecay, "gaps through the copy engine need a decay operator");
+    constexpr uint32_t kGap = DT ? kSeqGapBytes : 0;
     using LR = LaneRow<IO>;
     constexpr int CW = 32;
     constexpr int kRowBytes = seq_row_bytes<IO>();
@@ -515,22 +548,24 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
     const int x0 = int(grp) * CW;
     const int64_t d = int64_t(x0) + lane;
 
-    const uint32_t base = smem_addr(smem) + uint32_t(warp * seq_bwd_warp_bytes(S, kRowBytes));
-    const uint32_t ring = base;                                      // S slots: [in0 | in1 | gy | fwd]
-    const uint32_t outb = base + uint32_t(S) * kSeqBwdIn * kOpBytes; // 2 x [d in0 | d in1]
+    constexpr uint32_t kSlot = kSeqBwdIn * kOpBytes + kGap;         // [in0 | in1 | gy | fwd | gaps]
+    const uint32_t base = smem_addr(smem) + uint32_t(warp * seq_bwd_warp_bytes(S, kRowBytes, kGap));
+    const uint32_t ring = base;
+    const uint32_t outb = base + uint32_t(S) * kSlot;                // 2 x [d in0 | d in1]
     const uint32_t bars = outb + kSeqOutBufs * kSeqBwdOut * kOpBytes;
 
     const int n_slots = int((p.T + kSeqRows - 1) / kSeqRows);       // T < 2^31 (host check)
     // processing slot i covers time rows [j RB, j RB + RB), j = n_slots - 1 - i
     auto issue = [&](int i, int s) {
         const int y = (n_slots - 1 - i) * kSeqRows;
-        const uint32_t dst = ring + uint32_t(s) * kSeqBwdIn * kOpBytes;
+        const uint32_t dst = ring + uint32_t(s) * kSlot;
         const uint32_t bar = bars + 8u * uint32_t(s);
-        mbar_expect_tx(bar, kSeqBwdIn * kOpBytes);
+        mbar_expect_tx(bar, kSeqBwdIn * kOpBytes + (DT ? kSeqRows * 4 : 0));
         tma_load_3d(dst, &map_in0, x0, y, int(b), bar);
         tma_load_3d(dst + kOpBytes, &map_in1, x0, y, int(b), bar);
         tma_load_3d(dst + 2 * kOpBytes, &map_gy, x0, y, int(b), bar);
         tma_load_3d(dst + 3 * kOpBytes, &map_fwd, x0, y - 1, int(b), bar);   // state before each row
+        if constexpr (DT) tma_load_2d(dst + kSeqBwdIn * kOpBytes, &map_gap, y, int(b), bar);
     };
     if (lane == 0) {
         for (int s = 0; s < S; ++s) mbar_init(bars + 8u * s, 1);
@@ -546,8 +581,10 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
     [[maybe_unused]] float gnext = 0.f;
     if constexpr (BOp::kDecay) {
         lam2 = decay_lam2(p, d);
-        gcur = seq_slot_gap(p, b, int64_t(n_slots - 1) * kSeqRows, lane);
-        gnext = seq_slot_gap(p, b, int64_t(n_slots - 2) * kSeqRows, lane);
+        if constexpr (!DT) {
+            gcur = seq_slot_gap(p, b, int64_t(n_slots - 1) * kSeqRows, lane);
+            gnext = seq_slot_gap(p, b, int64_t(n_slots - 2) * kSeqRows, lane);
+        }
     }
 
     float lam = 0.f;           // dL/d (state after the rows still to walk)
@@ -558,13 +595,13 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
     for (int i = 0; i < n_slots; ++i) {
         const int j = n_slots - 1 - i;
         [[maybe_unused]] float gnext2 = 0.f;                        // the gaps two slots below
-        if constexpr (BOp::kDecay) gnext2 = seq_slot_gap(p, b, int64_t(j - 2) * kSeqRows, lane);
+        if constexpr (BOp::kDecay && !DT) gnext2 = seq_slot_gap(p, b, int64_t(j - 2) * kSeqRows, lane);
         if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
             wait_limit = 1;
             if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
             bad = true;
         }
-        const uint32_t src = ring + uint32_t(s) * kSeqBwdIn * kOpBytes + uint32_t(lane) * uint32_t(sizeof(IO));
+        const uint32_t src = ring + uint32_t(s) * kSlot + uint32_t(lane) * uint32_t(sizeof(IO));
         float xk[kSeqRows], xh[kSeqRows], xg[kSeqRows], xf[kSeqRows];
 #pragma unroll
         for (int r = 0; r < kSeqRows; ++r) {
@@ -573,6 +610,7 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
             xg[r] = LR::load(src + 2 * kOpBytes + r * kRowBytes);
             xf[r] = LR::load(src + 3 * kOpBytes + r * kRowBytes);
         }
+        if constexpr (DT) gcur = seq_smem_gap(p, ring + uint32_t(s) * kSlot + kSeqBwdIn * kOpBytes, lane);
         if (lane == 0) bulk_wait_read<kSeqOutBufs - 1>();            // staging buffers of slot i - 2
         __syncwarp();
         if (lane == 0 && !bad && i + S < n_slots) {
@@ -629,7 +667,7 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
             tma_store_3d(&map_d1, obuf + kOpBytes, x0, j * kSeqRows, int(b));
             bulk_commit();
         }
-        if constexpr (BOp::kDecay) {
+        if constexpr (BOp::kDecay && !DT) {
             gcur = gnext;
             gnext = gnext2;
         }

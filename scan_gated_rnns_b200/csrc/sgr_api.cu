@@ -174,44 +174,45 @@ struct SeqLayout {
     size_t smem = 0;
 };
 enum SeqKind { SEQ_SCAN = 0, SEQ_BACKWARD = 1, SEQ_FOLD = 2 };
-size_t seq_bytes(int kind, int S, int row_bytes) {
-    return kind == SEQ_BACKWARD ? seq_bwd_warp_bytes(S, row_bytes)
+size_t seq_bytes(int kind, int S, int row_bytes, size_t gap) {
+    return kind == SEQ_BACKWARD ? seq_bwd_warp_bytes(S, row_bytes, gap)
          : kind == SEQ_FOLD     ? seq_fold_warp_bytes(S, row_bytes)
-                                : seq_warp_bytes(S, row_bytes);
+                                : seq_warp_bytes(S, row_bytes, gap);
 }
+// gap: per-slot bytes of time-decay gaps brought by the copy engine (0 or kSeqGapBytes)
 SeqLayout seq_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, size_t reserved,
-                     size_t smem_block_max, int backward = SEQ_SCAN) {
+                     size_t smem_block_max, int backward = SEQ_SCAN, size_t gap = 0) {
     SeqLayout l;
     const int64_t K = sms > 0 ? (groups + sms - 1) / sms : 1;
-    size_t alloc = seq_bytes(backward, 4, row_bytes);
+    size_t alloc = seq_bytes(backward, 4, row_bytes, gap);
     if (K >= 1 && K <= 16) {
         const size_t share = smem_sm / size_t(K);
         alloc = share > reserved ? (share - reserved) / 128 * 128 : 0;
     }
     alloc = std::min(alloc, smem_block_max);
     int S = kSeqMaxSlots;
-    while (S > kSeqMinSlots && seq_bytes(backward, S, row_bytes) > alloc) --S;
+    while (S > kSeqMinSlots && seq_bytes(backward, S, row_bytes, gap) > alloc) --S;
     l.slots = S;
-    l.smem = std::max(alloc, seq_bytes(backward, S, row_bytes));
+    l.smem = std::max(alloc, seq_bytes(backward, S, row_bytes, gap));
     return l;
 }
 
 // the two-warp blocks of scan_sequential_pair_kernel: one block per channel
 // group, the block's share of the SM's shared memory split between its warps
 SeqLayout seq_pair_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, size_t reserved,
-                          size_t smem_block_max) {
+                          size_t smem_block_max, size_t gap = 0) {
     SeqLayout l;
     const int64_t K = sms > 0 ? (groups + sms - 1) / sms : 1;
-    size_t alloc = seq_pair_block_bytes(4, row_bytes);
+    size_t alloc = seq_pair_block_bytes(4, row_bytes, gap);
     if (K >= 1 && K <= 16) {
         const size_t share = smem_sm / size_t(K);
         alloc = share > reserved ? (share - reserved) / 128 * 128 : 0;
     }
     alloc = std::min(alloc, smem_block_max);
     int S = kSeqMaxSlots;
-    while (S > kSeqMinSlots && seq_pair_block_bytes(S, row_bytes) > alloc) --S;
+    while (S > kSeqMinSlots && seq_pair_block_bytes(S, row_bytes, gap) > alloc) --S;
     l.slots = S;
-    l.smem = std::max(alloc, seq_pair_block_bytes(S, row_bytes));
+    l.smem = std::max(alloc, seq_pair_block_bytes(S, row_bytes, gap));
     return l;
 }
 
@@ -252,10 +253,11 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
                               (ok == KIND_AUTO && groups < int64_t(pair_below) * kAssumedSMs);
             const int64_t gw = split ? cw / 2 : cw;                 // channels per warp
             const int64_t n_warps = B * ((D + gw - 1) / gw);
+            const size_t gap = decay ? kSeqGapBytes : 0;
             const SeqLayout lay = pair ? seq_pair_layout(n_warps, int(gw) * p.esz, kAssumedSMs, kAssumedSmemPerSM,
-                                                         kAssumedSmemReserved, kAssumedSmemPerBlock)
+                                                         kAssumedSmemReserved, kAssumedSmemPerBlock, gap)
                                        : seq_layout(n_warps, int(gw) * p.esz, kAssumedSMs, kAssumedSmemPerSM,
-                                                    kAssumedSmemReserved, kAssumedSmemPerBlock);
+                                                    kAssumedSmemReserved, kAssumedSmemPerBlock, SEQ_SCAN, gap);
             p.kind = pair ? KIND_SEQUENTIAL_PAIR : split ? KIND_SEQUENTIAL_SPLIT : KIND_SEQUENTIAL;
             p.split = (split || pair) ? 2 : 1;
             p.V = 1;
@@ -494,6 +496,25 @@ bool make_decay_maps(CUtensorMap *gap, CUtensorMap *lam, const ScanParams &sp, i
     return true;
 }
 
+// Tensor map of a decay's gaps for the channel-sequential kernels: boxes of
+// 16 gaps of one batch row (64 bytes); false when the copy engine cannot take
+// the array (16-byte aligned base and row stride needed), and the kernels
+// then load the gaps themselves.
+bool make_seq_gap_map(CUtensorMap *gap, const ScanParams &sp) {
+    if (!sp.decay_dt || !aligned16(sp.decay_dt)) return false;
+    if (sp.B > 1 && (sp.decay_dt_bs % 4) != 0) return false;
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[2] = {cuuint64_t(sp.T), cuuint64_t(sp.B)};
+    const cuuint64_t row = sp.B > 1 ? cuuint64_t(sp.decay_dt_bs) * 4 : (cuuint64_t(sp.T) * 4 + 15) / 16 * 16;
+    const cuuint64_t strides[1] = {row};
+    const cuuint32_t box[2] = {cuuint32_t(kSeqRows), 1u};
+    const cuuint32_t es[2] = {1u, 1u};
+    return enc(gap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(sp.decay_dt), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <class Op, typename IO, int V, int R, int W, bool DT>
 cudaError_t launch_pipelined_shape(const ScanParams &sp_in, const CUtensorMap &map0, const CUtensorMap &map1,
                                    const CUtensorMap &map_gap, const CUtensorMap &map_lam, cudaStream_t s,
@@ -594,54 +615,81 @@ cudaError_t seq_device(const void *kernel, size_t min_bytes, SeqDev *out) {
     *out = info[dev];
     return cudaSuccess;
 }
-template <class Op, typename IO, int SPLIT>
-cudaError_t launch_sequential(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
+template <class Op, typename IO, int SPLIT, bool DT>
+cudaError_t launch_sequential_dt(const Plan &pl, const ScanParams &sp, const CUtensorMap &map0,
+                                 const CUtensorMap &map1, const CUtensorMap &map_out, const CUtensorMap &map_gap,
+                                 cudaStream_t s) {
     constexpr int WB = kSeqWarpsPerBlock;
     constexpr int CW = 32 / SPLIT;
     constexpr int kRowBytes = CW * int(sizeof(IO));
-    auto kernel = scan_sequential_kernel<Op, IO, WB, SPLIT>;
-    alignas(64) CUtensorMap map0, map1, map_out;
-    if (!make_operand_map(&map0, sp.in0, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
-        !make_operand_map(&map1, sp.in1, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
-        !make_operand_map(&map_out, sp.out, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows))
-        return cudaErrorInvalidValue;
+    constexpr size_t kGap = DT ? kSeqGapBytes : 0;
+    auto kernel = scan_sequential_kernel<Op, IO, WB, SPLIT, DT>;
     SeqDev d;
-    cudaError_t e = seq_device(reinterpret_cast<const void *>(kernel), seq_warp_bytes(kSeqMinSlots, kRowBytes), &d);
+    cudaError_t e = seq_device(reinterpret_cast<const void *>(kernel), seq_warp_bytes(kSeqMinSlots, kRowBytes, kGap), &d);
     if (e != cudaSuccess) return e;
     SeqParams q;
     q.s = sp;
     q.n_groups = pl.n_dt;
     q.n_warps = pl.n_chains;
     const SeqLayout lay = seq_layout((q.n_warps + WB - 1) / WB * WB, kRowBytes, d.sms, size_t(d.smem_sm),
-                                     size_t(d.reserved), size_t(d.smem_block));
+                                     size_t(d.reserved), size_t(d.smem_block), SEQ_SCAN, kGap);
     q.slots = lay.slots;
     const int64_t grid = (q.n_warps + WB - 1) / WB;
-    kernel<<<dim3(unsigned(grid)), WB * 32, lay.smem, s>>>(q, map0, map1, map_out);
+    kernel<<<dim3(unsigned(grid)), WB * 32, lay.smem, s>>>(q, map0, map1, map_out, map_gap);
     return cudaGetLastError();
 }
 
-template <class Op, typename IO>
-cudaError_t launch_sequential_pair(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
-    constexpr int CW = 32;
-    constexpr int kRowBytes = CW * int(sizeof(IO));
-    auto kernel = scan_sequential_pair_kernel<Op, IO>;
-    alignas(64) CUtensorMap map0, map1, map_out;
+template <class Op, typename IO, int SPLIT>
+cudaError_t launch_sequential(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
+    constexpr int CW = 32 / SPLIT;
+    alignas(64) CUtensorMap map0, map1, map_out, map_gap;
     if (!make_operand_map(&map0, sp.in0, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
         !make_operand_map(&map1, sp.in1, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
         !make_operand_map(&map_out, sp.out, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows))
         return cudaErrorInvalidValue;
+    if constexpr (Op::kDecay) {
+        if (make_seq_gap_map(&map_gap, sp))
+            return launch_sequential_dt<Op, IO, SPLIT, true>(pl, sp, map0, map1, map_out, map_gap, s);
+    }
+    // no gaps through the copy engine: the kernel does not read map_gap
+    return launch_sequential_dt<Op, IO, SPLIT, false>(pl, sp, map0, map1, map_out, map0, s);
+}
+
+template <class Op, typename IO, bool DT>
+cudaError_t launch_sequential_pair_dt(const Plan &pl, const ScanParams &sp, const CUtensorMap &map0,
+                                      const CUtensorMap &map1, const CUtensorMap &map_out,
+                                      const CUtensorMap &map_gap, cudaStream_t s) {
+    constexpr int kRowBytes = 32 * int(sizeof(IO));
+    constexpr size_t kGap = DT ? kSeqGapBytes : 0;
+    auto kernel = scan_sequential_pair_kernel<Op, IO, DT>;
     SeqDev d;
-    cudaError_t e = seq_device(reinterpret_cast<const void *>(kernel), seq_pair_block_bytes(kSeqMinSlots, kRowBytes), &d);
+    cudaError_t e = seq_device(reinterpret_cast<const void *>(kernel),
+                               seq_pair_block_bytes(kSeqMinSlots, kRowBytes, kGap), &d);
     if (e != cudaSuccess) return e;
     SeqParams q;
     q.s = sp;
     q.n_groups = pl.n_dt;
     q.n_warps = pl.n_chains;                  // channel groups: one block each
     const SeqLayout lay = seq_pair_layout(q.n_warps, kRowBytes, d.sms, size_t(d.smem_sm), size_t(d.reserved),
-                                          size_t(d.smem_block));
+                                          size_t(d.smem_block), kGap);
     q.slots = lay.slots;
-    kernel<<<dim3(unsigned(q.n_warps)), kPairWarps * 32, lay.smem, s>>>(q, map0, map1, map_out);
+    kernel<<<dim3(unsigned(q.n_warps)), kPairWarps * 32, lay.smem, s>>>(q, map0, map1, map_out, map_gap);
     return cudaGetLastError();
+}
+
+template <class Op, typename IO>
+cudaError_t launch_sequential_pair(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
+    constexpr int CW = 32;
+    alignas(64) CUtensorMap map0, map1, map_out, map_gap;
+    if (!make_operand_map(&map0, sp.in0, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
+        !make_operand_map(&map1, sp.in1, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows) ||
+        !make_operand_map(&map_out, sp.out, sp.B, sp.T, sp.D, int(sizeof(IO)), CW, kSeqRows))
+        return cudaErrorInvalidValue;
+    if constexpr (Op::kDecay) {
+        if (make_seq_gap_map(&map_gap, sp))
+            return launch_sequential_pair_dt<Op, IO, true>(pl, sp, map0, map1, map_out, map_gap, s);
+    }
+    return launch_sequential_pair_dt<Op, IO, false>(pl, sp, map0, map1, map_out, map0, s);
 }
 
 template <class Op, typename IO>
@@ -812,35 +860,49 @@ cudaError_t dispatch_bwd_r(const Plan &pl, const BwdParams &bp, cudaStream_t s) 
 }
 
 // ---- channel-sequential gradient launch (wide batches)
-template <class BOp, typename IO>
-cudaError_t launch_sequential_bwd(const BwdParams &bp, cudaStream_t s) {
+template <class BOp, typename IO, bool DT>
+cudaError_t launch_sequential_bwd_dt(const BwdParams &bp, const CUtensorMap (&m)[7], cudaStream_t s) {
     constexpr int WB = kSeqWarpsPerBlock;
     constexpr int CW = 32;
     constexpr int kRowBytes = seq_row_bytes<IO>();
-    auto kernel = scan_sequential_backward_kernel<BOp, IO, WB>;
+    constexpr size_t kGap = DT ? kSeqGapBytes : 0;
+    auto kernel = scan_sequential_backward_kernel<BOp, IO, WB, DT>;
     const ScanParams &sp = bp.s;
-    const int esz = int(sizeof(IO));
-    alignas(64) CUtensorMap m_in0, m_in1, m_gy, m_fwd, m_d0, m_d1;
-    if (!make_operand_map(&m_in0, sp.in0, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
-        !make_operand_map(&m_in1, sp.in1, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
-        !make_operand_map(&m_gy, bp.gy, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
-        !make_operand_map(&m_fwd, bp.fwd, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
-        !make_operand_map(&m_d0, sp.out, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
-        !make_operand_map(&m_d1, bp.out1, sp.B, sp.T, sp.D, esz, CW, kSeqRows))
-        return cudaErrorInvalidValue;
     SeqDev d;
-    cudaError_t e = seq_device(reinterpret_cast<const void *>(kernel), seq_bwd_warp_bytes(kSeqMinSlots, kRowBytes), &d);
+    cudaError_t e =
+        seq_device(reinterpret_cast<const void *>(kernel), seq_bwd_warp_bytes(kSeqMinSlots, kRowBytes, kGap), &d);
     if (e != cudaSuccess) return e;
     SeqBwdParams q;
     q.g = bp;
     q.n_groups = (sp.D + CW - 1) / CW;
     q.n_warps = sp.B * q.n_groups;
     const SeqLayout lay = seq_layout((q.n_warps + WB - 1) / WB * WB, kRowBytes, d.sms, size_t(d.smem_sm),
-                                     size_t(d.reserved), size_t(d.smem_block), SEQ_BACKWARD);
+                                     size_t(d.reserved), size_t(d.smem_block), SEQ_BACKWARD, kGap);
     q.slots = lay.slots;
     const int64_t grid = (q.n_warps + WB - 1) / WB;
-    kernel<<<dim3(unsigned(grid)), WB * 32, lay.smem, s>>>(q, m_in0, m_in1, m_gy, m_fwd, m_d0, m_d1);
+    kernel<<<dim3(unsigned(grid)), WB * 32, lay.smem, s>>>(q, m[0], m[1], m[2], m[3], m[4], m[5], m[6]);
     return cudaGetLastError();
+}
+
+template <class BOp, typename IO>
+cudaError_t launch_sequential_bwd(const BwdParams &bp, cudaStream_t s) {
+    constexpr int CW = 32;
+    const ScanParams &sp = bp.s;
+    const int esz = int(sizeof(IO));
+    // k, hx (or r, s), dL/dh, the forward output, d in0, d in1, the gaps
+    alignas(64) CUtensorMap m[7];
+    if (!make_operand_map(&m[0], sp.in0, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
+        !make_operand_map(&m[1], sp.in1, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
+        !make_operand_map(&m[2], bp.gy, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
+        !make_operand_map(&m[3], bp.fwd, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
+        !make_operand_map(&m[4], sp.out, sp.B, sp.T, sp.D, esz, CW, kSeqRows) ||
+        !make_operand_map(&m[5], bp.out1, sp.B, sp.T, sp.D, esz, CW, kSeqRows))
+        return cudaErrorInvalidValue;
+    if constexpr (BOp::kDecay) {
+        if (make_seq_gap_map(&m[6], sp)) return launch_sequential_bwd_dt<BOp, IO, true>(bp, m, s);
+    }
+    m[6] = m[0];                              // not read without gaps through the copy engine
+    return launch_sequential_bwd_dt<BOp, IO, false>(bp, m, s);
 }
 
 // whether a gradient of this shape walks whole sequences per warp

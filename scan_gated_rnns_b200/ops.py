@@ -319,8 +319,9 @@ def set_tile_override(channel_lanes: int = 0, rows_per_thread: int = 0) -> None:
 
 def set_kernel_override(kernel: int = 0) -> None:
     """0 automatic, 1 tile kernel, 2 pipelined kernel, 3 pipelined with 15-warp
-    blocks, 4 channel-sequential kernel (the last three where the fast path
-    applies)."""
+    blocks, 4 channel-sequential kernel (one warp per 32-channel group), 5 the
+    same with each slot's rows split between half-warps, 6 two warps per
+    32-channel group (2-6 where the fast path applies)."""
     check("sgr_set_kernel_override", lib().sgr_set_kernel_override(kernel))
 
 

@@ -134,6 +134,35 @@ def test_decay_gap_layouts(B, pad, gap_off, lam_off, kernel, dtype):
     assert rel_err(h, oracle.mingru_decay(k, hx, h0, dt, lam)) <= TOL[dtype]
 
 
+# The channel-sequential kernels take the gaps through the copy engine when
+# the gap array allows it (16-byte aligned start, batch stride a multiple of
+# 4) and load them themselves otherwise: both, forward and gradient.
+@pytest.mark.parametrize("B,pad,gap_off", [(3, 0, 0), (3, 3, 0), (3, 1, 0), (3, 0, 1), (1, 0, 0)])
+@pytest.mark.parametrize("kernel", [4, 5, 6])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decay_sequential_gap_layouts(B, pad, gap_off, kernel, dtype):
+    sgr.set_kernel_override(kernel)
+    T, D = 1001, 96
+    k, hx, h0, dt, lam = data(B, T, D, dtype, "u01_1", seed=21 + pad + gap_off + kernel, wipe_at=500)
+    gstore = torch.full((B, T + pad + gap_off), float("nan"), device=DEV)
+    gaps = gstore[:, gap_off:gap_off + T]
+    gaps.copy_(dt.to(DEV))
+    h = sgr.mingru_scan_decay(k.to(DEV), hx.to(DEV), h0.to(DEV), gaps, lam.to(DEV))
+    torch.cuda.synchronize()
+    assert rel_err(h, oracle.mingru_decay(k, hx, h0, dt, lam)) <= TOL[dtype]
+    # the gradient (channel-sequential for these kinds) with the same gap layout
+    g = torch.Generator().manual_seed(9)
+    gy = torch.randn(B, T, D, generator=g).to(TORCH_DT[dtype])
+    fwd = torch.from_numpy(oracle.mingru_decay(k, hx, h0, dt, lam)).to(TORCH_DT[dtype])
+    dk, dhx, dh0, dlam = sgr.mingru_scan_decay_backward(k.to(DEV), hx.to(DEV), h0.to(DEV), gaps, lam.to(DEV),
+                                                        fwd.to(DEV), gy.to(DEV))
+    torch.cuda.synchronize()
+    rk, rhx, rh0, rlam = oracle.mingru_decay_backward(k, hx, h0, dt, lam, gy)
+    assert channel_scaled_err(dk, rk) <= TOL_BWD[dtype]
+    assert channel_scaled_err(dhx, rhx) <= TOL_BWD[dtype]
+    assert lam_err(dlam, rlam, k, hx, h0, dt, lam, gy) <= TOL_BWD[dtype]
+
+
 def test_decay_zero_gaps_equal_plain_scan():
     k, hx, h0, dt, lam = data(2, 3000, 256, "f32", "u01_1", seed=3)
     z = torch.zeros_like(dt)
