@@ -61,6 +61,8 @@ KERNEL_SOURCES = {
     "scan_sequential_backward_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_backward.cuh",
                                         "scan_gated_rnns_b200/csrc/scan_sequential.cuh"],
     "scan_backward_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_backward.cuh"],
+    "scan_pipelined_backward_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_backward.cuh",
+                                       "scan_gated_rnns_b200/csrc/scan_pipelined_backward.cuh"],
     "mingru_projected_scan_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/projected_scan.cuh"],
 }
 
@@ -311,7 +313,8 @@ def backward_kernel(w) -> str:
     import scan_gated_rnns_b200 as sgr
     kind = sgr._abi.lib().sgr_backward_kernel(0 if w.op == "mingru" else 1, w.B, w.T, w.D,
                                               0 if w.dtype == "f32" else 1, 1)
-    return "sgr::scan_sequential_backward_kernel" if kind == 4 else "sgr::scan_backward_kernel"
+    return {4: "sgr::scan_sequential_backward_kernel",
+            2: "sgr::scan_pipelined_backward_kernel"}.get(kind, "sgr::scan_backward_kernel")
 
 
 def measure_row(w, device, steps=10, warmup=3):
@@ -433,6 +436,46 @@ def measure_decay_rows(w, device, steps=10, warmup=3):
             "gelem_per_s": round(w.n_elems / per / 1e9, 2), "roofline_frac": round(gbs / peak, 4),
             "bytes_per_launch": bytes_, "kernel": kern}
     return rows
+
+
+def measure_log_row(w, device, steps=10, warmup=3):
+    """The minGRU scan evaluated in log space (mingru_scan_log) beside the
+    linear pairs on the same inputs: once with the linear scan's own plan and
+    once forced onto the chunked kernel the log-space scan runs, so that the
+    two times differ only in the evaluation domain."""
+    import scan_gated_rnns_b200 as sgr
+    p, q, init = generate(w, device=device)
+    out = torch.empty_like(p)
+    ws = sgr.Workspace(max(sgr.workspace_size("mingru_log", w.B, w.T, w.D, p.dtype),
+                           sgr.workspace_size("mingru", w.B, w.T, w.D, p.dtype)), device)
+    dt = 0 if w.dtype == "f32" else 1
+    plan = sgr._abi.plan(sgr._abi.SGR_OP_MINGRU_LOG, w.B, w.T, w.D, dt)
+    stream = torch.cuda.current_stream(device)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        return timed_launches(fn, steps, stream)[1]
+
+    per_log = timed(lambda: sgr.mingru_scan_log(p, q, init, out=out, workspace=ws))
+    per_lin = timed(lambda: sgr.mingru_scan(p, q, init, out=out, workspace=ws))
+    sgr.set_kernel_override(plan["kernel"])
+    try:
+        per_same = timed(lambda: sgr.mingru_scan(p, q, init, out=out, workspace=ws))
+    finally:
+        sgr.set_kernel_override(0)
+    lin_plan = sgr._abi.plan(0, w.B, w.T, w.D, dt)
+    bytes_ = w.algorithmic_bytes()
+    peak, _ = hbm_peak()
+    gbs = bytes_ / per_log / 1e9
+    del p, q, init, out, ws
+    return {"op": "mingru_scan_log", "B": w.B, "T": w.T, "D": w.D, "io_dtype": w.dtype,
+            "us_per_launch": round(per_log * 1e6, 2), "gbs": round(gbs, 1),
+            "gelem_per_s": round(w.n_elems / per_log / 1e9, 2), "roofline_frac": round(gbs / peak, 4),
+            "bytes_per_launch": bytes_, "kernel": plan_kernel(plan) + " (log-space pairs)",
+            "linear_same_kernel_us": round(per_same * 1e6, 2),
+            "linear_us": round(per_lin * 1e6, 2), "linear_kernel": plan_kernel(lin_plan)}
 
 
 def measure_summary_row(w, device, steps=10, warmup=3):
@@ -829,6 +872,9 @@ def run_b200(args):
             torch.cuda.empty_cache()
         for name in ("mingru_b8_t4096_d1024_f32_h0", "mingru_b1_t131072_d512_f32_h0"):
             rows[name.replace("mingru_", "mingru_summary_", 1)] = measure_summary_row(WORKLOADS[name], device)
+            torch.cuda.empty_cache()
+        for name in ("mingru_b8_t4096_d1024_f32_h0", "mingru_b16_t2048_d4096_bf16_h0"):
+            rows[name.replace("mingru_", "mingru_log_", 1)] = measure_log_row(WORKLOADS[name], device)
             torch.cuda.empty_cache()
         rows["mingru_projected_b8_t4096_d1024_din1024"] = measure_projected_row(device)
         torch.cuda.empty_cache()

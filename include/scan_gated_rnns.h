@@ -74,10 +74,12 @@
  *  it in the order they start, so no chunk ever waits for one whose block has
  *  not started.
  *  Wide batches (B x D large enough that groups of 32 channels give every SM
- *  several warps) are not cut along T at all: each warp scans its 32 channels
- *  over the whole sequence, and the plan needs only the header.  The
- *  time-decayed minGRU (mingru_scan_decay) is always cut along T when T spans
- *  several chunks; sgr_workspace_size(SGR_OP_MINGRU, ...) covers it too.
+ *  several warps) are not cut along T at all: each warp (or pair of warps)
+ *  scans its 32 channels over the whole sequence, and the plan needs only the
+ *  header.  The time-decayed minGRU (mingru_scan_decay) follows the same
+ *  plans; sgr_workspace_size(SGR_OP_MINGRU, ...) covers it too.  The
+ *  log-space minGRU (mingru_scan_log) is always cut along T when T spans
+ *  several chunks: size its workspace with SGR_OP_MINGRU_LOG.
  */
 #ifndef SCAN_GATED_RNNS_H
 #define SCAN_GATED_RNNS_H
@@ -112,7 +114,9 @@ typedef enum sgr_status {
 
 typedef enum sgr_dtype { SGR_F32 = 0, SGR_BF16 = 1 } sgr_dtype_t;
 
-typedef enum sgr_op { SGR_OP_MINGRU = 0, SGR_OP_MINMAX = 1 } sgr_op_t;
+/* SGR_OP_MINGRU_LOG names mingru_scan_log for sgr_workspace_size and
+ * sgr_scan_plan only (it has no gradient, summary or step entry points). */
+typedef enum sgr_op { SGR_OP_MINGRU = 0, SGR_OP_MINMAX = 1, SGR_OP_MINGRU_LOG = 2 } sgr_op_t;
 
 /* ---------------------------------------------------------------- scans */
 
@@ -125,6 +129,27 @@ typedef enum sgr_op { SGR_OP_MINGRU = 0, SGR_OP_MINMAX = 1 } sgr_op_t;
  *   workspace: see above; ws_bytes >= sgr_workspace_size(SGR_OP_MINGRU, ...).
  */
 SGR_API sgr_status_t mingru_scan(const void *k, const void *hx,
+                         const void *h0, int64_t h0_batch_stride,
+                         void *h, int64_t B, int64_t T, int64_t D,
+                         sgr_dtype_t dtype, void *workspace, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/*
+ * mingru_scan_log -- the same result as mingru_scan, evaluated in log space
+ * (page "Mingru Pytorch", Requirements & limits: the log-space numerically
+ * stable minGRU): the chunked kernels carry log2 h_t through pairs
+ * (sum of log a, logaddexp of log b) and exponentiate at the store.  Kept as
+ * the measured alternative to the linear pairs mingru_scan evaluates: more
+ * MUFU work per element and an error that grows with the log-state's range.
+ * Arguments, layout, ownership and errors as mingru_scan, except:
+ *   h0       : optional initial state, h0 > 0 (0 allowed: log h = -inf);
+ *              h0 < 0 has no logarithm and gives NaN outputs.
+ *   workspace: ws_bytes >= sgr_workspace_size(SGR_OP_MINGRU_LOG, ...); the
+ *              sequence is cut into chunks whatever the batch width (no
+ *              channel-sequential kernel), so wide batches need more than
+ *              sgr_workspace_size(SGR_OP_MINGRU, ...).
+ */
+SGR_API sgr_status_t mingru_scan_log(const void *k, const void *hx,
                          const void *h0, int64_t h0_batch_stride,
                          void *h, int64_t B, int64_t T, int64_t D,
                          sgr_dtype_t dtype, void *workspace, size_t ws_bytes,
@@ -508,10 +533,16 @@ SGR_API sgr_status_t sgr_scan_plan_decay(int64_t B, int64_t T, int64_t D, sgr_dt
                                          int aligned, sgr_plan_t *plan);
 
 /* Which kernel the gradient of this shape runs (mingru_scan_backward,
- * minmax_scan_backward and their time-decay forms): 1 the chunked tile kernel,
- * 4 the channel-sequential kernel (wide batches: one warp walks the whole
- * sequence of 32 channels backwards); 0 for invalid arguments.  `aligned` says
- * whether all six (B, T, D) operands would be 16-byte aligned.  Pure host code. */
+ * minmax_scan_backward and their time-decay forms): 1 the chunked tile kernel
+ * (blocks take chunks by ticket), 2 the pipelined gradient (persistent blocks
+ * fed by the copy engine; aligned vector-width rows with at least two tiles of
+ * 120 rows per SM; the decayed gradient runs tiles of 56 rows, two blocks per
+ * SM), 4 the channel-sequential kernel (wide batches, from 5 groups of 32
+ * channels per SM: one warp walks the whole sequence of 32 channels
+ * backwards); 0 for invalid arguments.
+ * `aligned` says whether all six (B, T, D) operands would be 16-byte aligned.
+ * Kernel override 2 or 3 forces the pipelined gradient wherever the rows allow
+ * it.  Pure host code. */
 SGR_API int sgr_backward_kernel(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
                                 int aligned);
 

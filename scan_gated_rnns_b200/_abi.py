@@ -24,6 +24,7 @@ SGR_BF16 = 1
 
 SGR_OP_MINGRU = 0
 SGR_OP_MINMAX = 1
+SGR_OP_MINGRU_LOG = 2
 
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -33,6 +34,7 @@ _int = ctypes.c_int
 SIGNATURES = {
     "mingru_scan": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _i64, _i64, _int, _vp, _sz, _vp]),
     "minmax_scan": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _i64, _i64, _int, _vp, _sz, _vp]),
+    "mingru_scan_log": (_int, [_vp, _vp, _vp, _i64, _vp, _i64, _i64, _i64, _int, _vp, _sz, _vp]),
     "mingru_step": (_int, [_vp, _i64, _vp, _i64, _vp, _i64, _vp, _i64, _i64, _i64, _int, _vp]),
     "sgr_workspace_size": (_sz, [_int, _i64, _i64, _i64, _int]),
     "sgr_workspace_init": (_int, [_vp, _sz, _vp]),

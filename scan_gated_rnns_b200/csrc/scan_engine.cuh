@@ -64,6 +64,12 @@ __device__ __forceinline__ float fast_rcp(float x) {
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// log2(x) by the MUFU approximation (x <= 0 gives -inf / NaN)
+__device__ __forceinline__ float fast_lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // ------------------------------------------------------------- operators
 
@@ -167,6 +173,10 @@ struct MinGRUOp {
     static __device__ __forceinline__ float step(float a, float b, float x) { return fmaf(a, x, b); }
     // initial state when none is given
     static __device__ __forceinline__ float default_init() { return 0.f; }
+    // the carried state is the state itself (see MinGRULogOp)
+    static constexpr bool kLogSpace = false;
+    static __device__ __forceinline__ float state_in(float h) { return h; }
+    static __device__ __forceinline__ float state_out(float s) { return s; }
 };
 
 struct MinMaxOp {
@@ -195,6 +205,68 @@ struct MinMaxOp {
     static __device__ __forceinline__ float2 step2(float2 u, float2 l, float2 x) {
         return make_float2(fmaxf(fminf(x.x, u.x), l.x), fmaxf(fminf(x.y, u.y), l.y));
     }
+    static constexpr bool kLogSpace = false;
+    static __device__ __forceinline__ float state_in(float h) { return h; }
+    static __device__ __forceinline__ float state_out(float s) { return s; }
+};
+
+// log2(2^x + 2^y), exact at -inf: the larger term plus log2(1 + 2^-(gap));
+// both -inf gives -inf (not the NaN of -inf - -inf).  2 MUFU operations.
+__device__ __forceinline__ float lse2(float x, float y) {
+    const float m = fmaxf(x, y);
+    const float r = m + fast_lg2(1.f + fast_exp2(fminf(x, y) - m));
+    return m == -INFINITY ? m : r;
+}
+
+// minGRU evaluated in log space, the form the page's layer computes (page
+// "Mingru Pytorch", Requirements & limits: the log-space numerically stable
+// minGRU): with log a_t = -softplus(k_t), log b_t = log z_t + log g(hx_t),
+//   log h_t = logaddexp(log a_t + log h_{t-1}, log b_t),
+// which unrolled is a*_t + logcumsumexp(log b_s - a*_s) with a*_t the running
+// sum of log a.  A pair (LA, LB) maps a log-state x to logaddexp(LA + x, LB);
+// composing two steps adds the LA and takes the logaddexp of the LB shifted by
+// the later LA, so the scan engine's chunk hand-off, look-back and replay
+// carry it unchanged, with the state held as log2 h (h = 0 is -inf) and
+// exponentiated only at the store.  All logs are base 2 (the MUFU's): per
+// element 4 MUFU operations for the activations, 2 for the fold and 3 for the
+// replay and the store, against 3-4 in all for the linear pairs.  Kept as the
+// measured alternative to the linear evaluation, not the default.
+//   softplus2(k) = log2(1 + 2^(k log2 e)) = max(kl, 0) + log2(1 + 2^-|kl|),
+//   LA = -softplus2(k),  log2 z = min(kl, 0) - log2(1 + 2^-|kl|),
+//   log2 g(hx) = log2(hx + 0.5) (hx >= 0), hl - log2(1 + 2^hl) (hx < 0),
+// kl = k log2 e, hl = hx log2 e.  k = -inf gives the identity (0, -inf).
+struct MinGRULogOp {
+    static constexpr bool kDecay = false;
+    static constexpr bool kLeanRows = false;
+    static constexpr bool kLogSpace = true;
+    static __device__ __forceinline__ float2 identity() { return make_float2(0.f, -INFINITY); }
+    static __device__ __forceinline__ float2 combine(float2 p, float2 q) {
+        return make_float2(p.x + q.x, lse2(p.y + q.x, q.y));
+    }
+    static __device__ __forceinline__ float apply(float2 p, float x) { return lse2(p.x + x, p.y); }
+    static __device__ __forceinline__ float pad0() { return -INFINITY; }
+    static __device__ __forceinline__ float pad1() { return 0.f; }
+    static __device__ __forceinline__ void element(float k, float hx, float &la, float &lb) {
+        const float kl = k * -kNegLog2e, hl = hx * -kNegLog2e;
+        const float lk = fast_lg2(1.f + fast_exp2(-fabsf(kl)));
+        const bool hpos = hx >= 0.f;
+        const float lg = fast_lg2(hpos ? hx + 0.5f : 1.f + fast_exp2(hl));
+        la = -(fmaxf(kl, 0.f) + lk);
+        lb = (fminf(kl, 0.f) - lk) + (hpos ? lg : hl - lg);
+    }
+    static __device__ __forceinline__ void fold2(float2 &A, float2 &B, float2 a, float2 b) {
+        B = make_float2(lse2(B.x + a.x, b.x), lse2(B.y + a.y, b.y));
+        A = make_float2(A.x + a.x, A.y + a.y);
+    }
+    static __device__ __forceinline__ float2 step2(float2 a, float2 b, float2 h) {
+        return make_float2(lse2(a.x + h.x, b.x), lse2(a.y + h.y, b.y));
+    }
+    static __device__ __forceinline__ float step(float a, float b, float x) { return lse2(a + x, b); }
+    static __device__ __forceinline__ float default_init() { return 0.f; }
+    // the carried state is log2 h: taken from an initial state (h > 0; 0
+    // gives -inf) and returned to h at the store
+    static __device__ __forceinline__ float state_in(float h) { return fast_lg2(h); }
+    static __device__ __forceinline__ float state_out(float s) { return fast_exp2(s); }
 };
 
 // minGRU with time decay (page "Your first delta model", Step 5: every mixer
@@ -479,7 +551,7 @@ __device__ __forceinline__ bool resolve_window(const ScanParams &p, int64_t q, c
         if (qq < 0) {
 #pragma unroll
             for (int v = 0; v < CV; ++v)
-                hin[v] = Op::apply(M[v], load_init<IO>(p, b, d_first + v, Op::default_init()));
+                hin[v] = Op::apply(M[v], Op::state_in(load_init<IO>(p, b, d_first + v, Op::default_init())));
             done = true;
             continue;
         }
@@ -580,7 +652,7 @@ __device__ __forceinline__ void carry_tile(const ScanParams &p, int64_t tile, fl
     float hin[CV];
     if (c == 0) {
 #pragma unroll
-        for (int v = 0; v < CV; ++v) hin[v] = load_init<IO>(p, b, dl + v, Op::default_init());
+        for (int v = 0; v < CV; ++v) hin[v] = Op::state_in(load_init<IO>(p, b, dl + v, Op::default_init()));
     } else {
         if (publish) publish_summary<CV, TC>(p, tile, ch, total);
         look_back<Op, IO, CV, TC>(p, c, chain, b, dl, ch, hin);
@@ -773,7 +845,7 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const Sca
 #pragma unroll
             for (int v = 0; v < V; ++v) {
                 st[v] = Op::step(x0[r][v], x1[r][v], st[v]);
-                y[v] = st[v];
+                y[v] = Op::state_out(st[v]);
             }
             const int64_t t = row0 + r;
             if (dvalid && t < p.T) Access<IO, V>::store(out + base + t * p.D, y);
@@ -1156,8 +1228,8 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
 #pragma unroll
                 for (int i = 0; i < V2; ++i) {
                     st[i] = Op::step2(PA[SB][r][i], PB[SB][r][i], st[i]);
-                    y[2 * i] = st[i].x;
-                    y[2 * i + 1] = st[i].y;
+                    y[2 * i] = Op::state_out(st[i].x);
+                    y[2 * i + 1] = Op::state_out(st[i].y);
                 }
                 if (full[SB] || (dvalid[SB] && row0[SB] + r < p.T)) Access<IO, V>::store(dst, y);
                 dst += p.D;
@@ -1211,7 +1283,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
             if (tc.c == 0) {
 #pragma unroll
                 for (int v = 0; v < CV; ++v)
-                    init[v] = load_init<IO>(p, tc.b, int64_t(tc.dt) * TC + ch + v, Op::default_init());
+                    init[v] = Op::state_in(load_init<IO>(p, tc.b, int64_t(tc.dt) * TC + ch + v, Op::default_init()));
             } else {
                 load_window<CV, TC, KW>(p, int64_t(tc.c) - 1, tc.chain, ch, win);
             }

@@ -150,6 +150,7 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
                        const __grid_constant__ CUtensorMap map_gap) {
     static_assert(SPLIT == 1 || SPLIT == 2, "one or two row groups per slot");
     static_assert(!DT || Op::kDecay, "gaps through the copy engine need a decay operator");
+    static_assert(!Op::kLogSpace, "the channel-sequential kernels carry linear states");
     constexpr uint32_t kGap = DT ? kSeqGapBytes : 0;
     using LR = LaneRow<IO>;
     constexpr int CW = 32 / SPLIT;                                   // channels of a warp's group
@@ -341,6 +342,7 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
                             const __grid_constant__ CUtensorMap map1, const __grid_constant__ CUtensorMap map_out,
                             const __grid_constant__ CUtensorMap map_gap) {
     static_assert(!DT || Op::kDecay, "gaps through the copy engine need a decay operator");
+    static_assert(!Op::kLogSpace, "the channel-sequential kernels carry linear states");
     constexpr uint32_t kGap = DT ? kSeqGapBytes : 0;
     using LR = LaneRow<IO>;
     constexpr int CW = 32;

@@ -6,6 +6,7 @@
 #include "scan_backward.cuh"
 #include "scan_engine.cuh"
 #include "scan_fold.cuh"
+#include "scan_pipelined_backward.cuh"
 #include "scan_sequential.cuh"
 
 #include <algorithm>
@@ -58,11 +59,13 @@ constexpr int kSeqMinWarpsPerSMHalf = 6;
 // 0.81 / 0.84, 13.8: 0.84 / 0.86, and D 4096 at 27.7: 0.85 / 0.87.
 constexpr int kSeqPairBelow = 32;
 constexpr int kSeqPairBelowHalf = 24;
-// The gradient (four operands in, two out per element, where the chunked
-// gradient kernel is a plain tile kernel) gains from 3 warps per SM in both
-// dtypes (measured: fp32 loses at 2.6 and wins at 3.5, bf16 wins at 3.5 and
-// loses at 1.7).
-constexpr int kSeqBwdMinWarpsPerSM = 3;
+// The gradient (four operands in, two out per element) walks whole sequences
+// from 5 warps per SM: against the pipelined gradient it loses at 3.5 groups
+// per SM (bf16 B4 x 2048 x 4096 150 us against 101 us; fp32 B8 x 2048 x 2048
+// a tie, its decayed form 194 against 182 us) and wins at 6.9 (bf16 B8:
+// 177 against 183 us, decayed 224 against 247; fp32 B16 x 2048 x 2048 289
+// against 306, decayed 308 against 349).
+constexpr int kSeqBwdMinWarpsPerSM = 5;
 constexpr int kSeqMaxSlots = 8;
 constexpr int kSeqMinSlots = 2;
 constexpr int kSeqWarpsPerBlock = 1;
@@ -229,9 +232,14 @@ SeqLayout seq_pair_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm
 // decay: the time-decayed minGRU, whose extra gate per element favours 4
 // rows per thread in the pipelined kernel (bf16 with 15-warp blocks); wide
 // decayed batches take the channel-sequential kernels like the plain scan
-// (their gaps arrive one slot ahead, spread across the lanes)
+// (each slot's gaps arrive with it through the copy engine, or, for gap
+// arrays the copy engine cannot address, spread across the lanes two slots
+// ahead)
+// chunked_only: never the channel-sequential kernels (the log-space minGRU,
+// which only the chunked kernels evaluate)
 Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
-               bool force_tile = false, bool light_op = false, bool decay = false) {
+               bool force_tile = false, bool light_op = false, bool decay = false,
+               bool chunked_only = false) {
     Plan p;
     p.esz = (dtype == SGR_BF16) ? 2 : 4;
     const int vw = 16 / p.esz;
@@ -241,7 +249,7 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
         // whole sequences per warp when the channel groups fill the GPU
         const int64_t cw = 32;
         const int64_t groups = B * ((D + cw - 1) / cw);
-        const bool seq_ok = p.vec && !force_tile && T <= int64_t(std::numeric_limits<int>::max()) &&
+        const bool seq_ok = p.vec && !force_tile && !chunked_only && T <= int64_t(std::numeric_limits<int>::max()) &&
                             B <= int64_t(std::numeric_limits<int>::max());
         const int min_per_sm = p.esz == 2 ? kSeqMinWarpsPerSMHalf : kSeqMinWarpsPerSM;
         const bool want = ok == KIND_SEQUENTIAL || ok == KIND_SEQUENTIAL_SPLIT || ok == KIND_SEQUENTIAL_PAIR ||
@@ -695,9 +703,14 @@ cudaError_t launch_sequential_pair(const Plan &pl, const ScanParams &sp, cudaStr
 template <class Op, typename IO>
 cudaError_t dispatch(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
     constexpr int VW = 16 / int(sizeof(IO));
-    if (pl.kind == KIND_SEQUENTIAL) return launch_sequential<Op, IO, 1>(pl, sp, s);
-    if (pl.kind == KIND_SEQUENTIAL_SPLIT) return launch_sequential<Op, IO, 2>(pl, sp, s);
-    if (pl.kind == KIND_SEQUENTIAL_PAIR) return launch_sequential_pair<Op, IO>(pl, sp, s);
+    if constexpr (!Op::kLogSpace) {
+        if (pl.kind == KIND_SEQUENTIAL) return launch_sequential<Op, IO, 1>(pl, sp, s);
+        if (pl.kind == KIND_SEQUENTIAL_SPLIT) return launch_sequential<Op, IO, 2>(pl, sp, s);
+        if (pl.kind == KIND_SEQUENTIAL_PAIR) return launch_sequential_pair<Op, IO>(pl, sp, s);
+    } else {
+        if (pl.kind == KIND_SEQUENTIAL || pl.kind == KIND_SEQUENTIAL_SPLIT || pl.kind == KIND_SEQUENTIAL_PAIR)
+            return cudaErrorInvalidConfiguration;    // never planned (chunked_only)
+    }
     if (pl.kind == KIND_PIPELINED) {
         if constexpr (sizeof(IO) == 2) {
             if (pl.r == 8) return launch_pipelined<Op, IO, 4, 8, kPipeWarps>(sp, s, nullptr);
@@ -761,7 +774,8 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
                       sgr_dtype_t dtype, void *ws, size_t ws_bytes, cudaStream_t stream,
                       const DecayArgs *dec = nullptr) {
     if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
-    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return SGR_ERR_INVALID_ARG;
+    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX && op != SGR_OP_MINGRU_LOG) return SGR_ERR_INVALID_ARG;
+    if (op == SGR_OP_MINGRU_LOG && dec) return SGR_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || D < 0 || init_bs < 0) return SGR_ERR_INVALID_ARG;
     if (B == 0 || T == 0 || D == 0) return SGR_OK;
     if (!in0 || !in1 || !out) return SGR_ERR_INVALID_ARG;
@@ -779,7 +793,8 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
         return SGR_ERR_INVALID_ARG;
 
     const bool aligned = aligned16(in0) && aligned16(in1) && aligned16(out);
-    const Plan pl = make_plan(B, T, D, dtype, aligned, false, op == SGR_OP_MINMAX, dec != nullptr);
+    const Plan pl = make_plan(B, T, D, dtype, aligned, false, op == SGR_OP_MINMAX, dec != nullptr,
+                              op == SGR_OP_MINGRU_LOG);
     if (pl.n_tiles > int64_t(std::numeric_limits<int>::max())) return SGR_ERR_UNSUPPORTED;
 
     ScanParams sp;
@@ -823,6 +838,9 @@ sgr_status_t run_scan(sgr_op_t op, const void *in0, const void *in1, const void 
     } else if (op == SGR_OP_MINGRU) {
         e = dtype == SGR_F32 ? dispatch<MinGRUOp, float>(pl, sp, stream)
                              : dispatch<MinGRUOp, __nv_bfloat16>(pl, sp, stream);
+    } else if (op == SGR_OP_MINGRU_LOG) {
+        e = dtype == SGR_F32 ? dispatch<MinGRULogOp, float>(pl, sp, stream)
+                             : dispatch<MinGRULogOp, __nv_bfloat16>(pl, sp, stream);
     } else {
         e = dtype == SGR_F32 ? dispatch<MinMaxOp, float>(pl, sp, stream)
                              : dispatch<MinMaxOp, __nv_bfloat16>(pl, sp, stream);
@@ -918,9 +936,130 @@ bool seq_backward_planned(int64_t B, int64_t T, int64_t D, int esz, bool aligned
     return groups >= int64_t(kSeqBwdMinWarpsPerSM) * kAssumedSMs;
 }
 
+// ---- pipelined gradient (narrow batches, aligned vector-width rows)
+// fp32 32 channels x 2 rows per thread, bf16 64 channels x 4 rows per thread;
+// 15 data warps + 1 carry warp, one block per SM, tiles of 120 rows (four
+// operand boxes per ring slot, 3 slots: about 190 KB of shared memory), or 7
+// data warps, two blocks per SM, tiles of 56 rows.  The plain gradients take
+// the 15-warp blocks (fp32 B8 x 4096 x 1024: 140 against 150 us; MinMax
+// B4 x 8192 x 768: 119 against 135 us).  The decayed one, whose longer phase
+// A each block's carry warp waits behind, takes the 7-warp blocks where the
+// channel tiles give the blocks in flight little look-back depth (fp32 B8 x
+// 4096 x 1024, 256 chains: 187 against 195 us; bf16, 128 chains: 142
+// against 150) and the 15-warp ones where the depth grows (fp32 B4 x 8192 x
+// 768, 96 chains: 150 against 158 us).
+template <typename IO> constexpr int bwd_pipe_r() { return sizeof(IO) == 4 ? 2 : 4; }
+template <typename IO, bool DT = false, int W = kPipeWarpsWide>
+using BwdPipeShape = PipeBwdShape<IO, 4, pipe_cg<IO>(), bwd_pipe_r<IO>(), kStages, W, DT>;
+
+// The gradient's tile plan: the pipelined kernel for aligned vector-width
+// rows with at least two tiles per SM (override 2 or 3 forces it wherever the
+// rows allow), else the ticketed tile kernel (make_plan with force_tile).
+// decay: the time-decayed gradient (7-warp blocks).
+Plan make_bwd_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned, bool decay = false) {
+    const int esz = dtype == SGR_BF16 ? 2 : 4;
+    const int vw = 16 / esz;
+    const int ok = g_override_kind.load();
+    const bool vec = aligned && D % vw == 0 && T < int64_t(std::numeric_limits<int>::max()) / 2;
+    if (vec && (ok == KIND_AUTO || ok == KIND_PIPELINED || ok == KIND_PIPELINED_WIDE)) {
+        Plan p;
+        p.esz = esz;
+        p.vec = true;
+        p.kind = KIND_PIPELINED;
+        p.V = 4;
+        p.cg = esz == 4 ? 8 : 16;
+        p.TC = p.cg * p.V;
+        p.r = esz == 4 ? 2 : 4;
+        p.stages = kStages;
+        // blocks of 15 data warps, one per SM, or of 7, two per SM (override
+        // 2; decay with at least 0.8 chains per SM)
+        const int64_t chains = B * ((D + (esz == 4 ? 32 : 64) - 1) / (esz == 4 ? 32 : 64));
+        const bool narrow = ok == KIND_PIPELINED || (ok == KIND_AUTO && decay && 5 * chains >= 4 * kAssumedSMs);
+        p.warps = narrow ? kPipeWarps : kPipeWarpsWide;
+        p.TR = p.warps * (32 / p.cg) * p.r;
+        p.smem = narrow ? (esz == 4 ? BwdPipeShape<float, false, kPipeWarps>::smem_bytes
+                                    : BwdPipeShape<__nv_bfloat16, false, kPipeWarps>::smem_bytes)
+                        : (esz == 4 ? BwdPipeShape<float>::smem_bytes : BwdPipeShape<__nv_bfloat16>::smem_bytes);
+        p.n_dt = (D + p.TC - 1) / p.TC;
+        p.n_chains = B * p.n_dt;
+        p.n_chunks = (T + p.TR - 1) / p.TR;
+        p.n_tiles = p.n_chains * p.n_chunks;
+        if (p.n_tiles > 0) {
+            p.off_words = kAlign;
+            p.ws_bytes = kAlign;
+            if (p.n_chunks > 1) p.ws_bytes = align_up(p.off_words + size_t(p.n_tiles) * 3 * p.TC * 8, kAlign);
+        }
+        if (ok != KIND_AUTO || p.n_tiles >= 2 * kAssumedSMs) return p;
+    }
+    return make_plan(B, T, D, dtype, aligned, true);
+}
+
+template <class BOp, typename IO, bool DT, int W>
+cudaError_t launch_pipelined_bwd_shape(const BwdParams &bp, const CUtensorMap (&m)[6], cudaStream_t s) {
+    constexpr int CG = pipe_cg<IO>();
+    constexpr int R = bwd_pipe_r<IO>();
+    using Shape = BwdPipeShape<IO, DT, W>;
+    auto kernel = scan_pipelined_backward_kernel<BOp, IO, 4, CG, R, kStages, W, W == kPipeWarps ? 2 : 1, DT>;
+    constexpr size_t smem = Shape::smem_bytes;
+    constexpr int NT = (W + 1) * 32;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    // per-device one-time set-up of the shared-memory limit and occupancy
+    static std::atomic<int> occ_cache[64];
+    int occ = (dev >= 0 && dev < 64) ? occ_cache[dev].load() : 0;
+    if (occ == 0) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, NT, smem);
+        if (e != cudaSuccess) return e;
+        if (occ <= 0) return cudaErrorInvalidConfiguration;
+        if (dev >= 0 && dev < 64) occ_cache[dev].store(occ);
+    }
+    const DeviceInfo di = device_info(dev);
+    if (di.sms <= 0) return cudaErrorInvalidDevice;
+    const int64_t grid = std::min<int64_t>(bp.s.n_tiles, int64_t(di.sms) * occ);
+    BwdParams args = bp;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(grid));
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args, m[0], m[1], m[2], m[3], m[4], m[5]);
+}
+
+template <class BOp, typename IO, int W>
+cudaError_t launch_pipelined_bwd(const BwdParams &bp, cudaStream_t s) {
+    using Shape = BwdPipeShape<IO, false, W>;
+    const ScanParams &sp = bp.s;
+    const int esz = int(sizeof(IO));
+    // k, hx (or r, s), dL/dh, the forward output; the decay's gaps and rates
+    alignas(64) CUtensorMap m[6];
+    if (!make_operand_map(&m[0], sp.in0, sp.B, sp.T, sp.D, esz, Shape::TC, Shape::TR) ||
+        !make_operand_map(&m[1], sp.in1, sp.B, sp.T, sp.D, esz, Shape::TC, Shape::TR) ||
+        !make_operand_map(&m[2], bp.gy, sp.B, sp.T, sp.D, esz, Shape::TC, Shape::TR) ||
+        !make_operand_map(&m[3], bp.fwd, sp.B, sp.T, sp.D, esz, Shape::TC, Shape::TR))
+        return cudaErrorInvalidValue;
+    if constexpr (BOp::kDecay && BwdPipeShape<IO, true, W>::dec_boxable) {
+        if (make_decay_maps(&m[4], &m[5], sp, Shape::TR, Shape::TC))
+            return launch_pipelined_bwd_shape<BOp, IO, true, W>(bp, m, s);
+    }
+    m[4] = m[0];                              // not read without decay operands through the copy engine
+    m[5] = m[0];
+    return launch_pipelined_bwd_shape<BOp, IO, false, W>(bp, m, s);
+}
+
 template <class BOp, typename IO>
 cudaError_t dispatch_bwd(const Plan &pl, const BwdParams &bp, cudaStream_t s) {
     constexpr int VW = 16 / int(sizeof(IO));
+    if (pl.kind == KIND_PIPELINED)
+        return pl.warps == kPipeWarps ? launch_pipelined_bwd<BOp, IO, kPipeWarps>(bp, s)
+                                      : launch_pipelined_bwd<BOp, IO, kPipeWarpsWide>(bp, s);
     if (!pl.vec) return dispatch_bwd_r<BOp, IO, 1, 32>(pl, bp, s);
     return dispatch_bwd_r<BOp, IO, VW, 8>(pl, bp, s);
 }
@@ -993,7 +1132,7 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
     const bool aligned = aligned16(in0) && aligned16(in1) && aligned16(fwd) && aligned16(gy) &&
                          aligned16(out0) && aligned16(out1);
     const bool seq = seq_backward_planned(B, T, D, esz, aligned);
-    const Plan pl = make_plan(B, T, D, dtype, aligned, true);
+    const Plan pl = make_bwd_plan(B, T, D, dtype, aligned, dec != nullptr);
     if (!seq && pl.n_tiles > int64_t(std::numeric_limits<int>::max())) return SGR_ERR_UNSUPPORTED;
 
     BwdParams bp;
@@ -1036,9 +1175,11 @@ sgr_status_t run_scan_backward(sgr_op_t op, const void *in0, const void *in1, co
     if (pl.n_chunks > 1) {
         char *w = static_cast<char *>(ws);
         sp.words = reinterpret_cast<uint64_t *>(w + pl.off_words);
-        // one block per tile: tiles go out by ticket in block start order
-        sp.ticket = reinterpret_cast<uint32_t *>(w + kTicketOffset);
-        if (cudaMemsetAsync(sp.ticket, 0, sizeof(uint32_t), stream) != cudaSuccess) return SGR_ERR_CUDA;
+        if (pl.kind == KIND_TILE) {
+            // tile kernel: tiles go out by ticket in block start order
+            sp.ticket = reinterpret_cast<uint32_t *>(w + kTicketOffset);
+            if (cudaMemsetAsync(sp.ticket, 0, sizeof(uint32_t), stream) != cudaSuccess) return SGR_ERR_CUDA;
+        }
         cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
         if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return SGR_ERR_CUDA;
         if (cs == cudaStreamCaptureStatusActive) {
@@ -1301,6 +1442,13 @@ sgr_status_t mingru_scan(const void *k, const void *hx, const void *h0, int64_t 
                     ws_bytes, stream);
 }
 
+sgr_status_t mingru_scan_log(const void *k, const void *hx, const void *h0, int64_t h0_batch_stride,
+                             void *h, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
+                             void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    return run_scan(SGR_OP_MINGRU_LOG, k, hx, h0, h0_batch_stride, h, B, T, D, dtype, workspace,
+                    ws_bytes, stream);
+}
+
 sgr_status_t minmax_scan(const void *r, const void *s, const void *x0, int64_t x0_batch_stride,
                          void *x, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
                          void *workspace, size_t ws_bytes, cudaStream_t stream) {
@@ -1495,15 +1643,20 @@ size_t sgr_backward_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D,
     if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return 0;
     if (dtype != SGR_F32 && dtype != SGR_BF16) return 0;
     if (B <= 0 || T <= 0 || D <= 0) return 0;
-    const Plan a = make_plan(B, T, D, dtype, true, true);
-    const Plan b = make_plan(B, T, D, dtype, false, true);
-    return a.ws_bytes > b.ws_bytes ? a.ws_bytes : b.ws_bytes;
+    // the aligned and unaligned plans, plain and decayed (shorter tiles)
+    size_t need = 0;
+    for (int v = 0; v < 4; ++v)
+        need = std::max(need, make_bwd_plan(B, T, D, dtype, (v & 1) == 0, v >= 2).ws_bytes);
+    return need;
 }
 
 size_t sgr_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype) {
-    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return 0;
+    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX && op != SGR_OP_MINGRU_LOG) return 0;
     if (dtype != SGR_F32 && dtype != SGR_BF16) return 0;
     if (B <= 0 || T <= 0 || D <= 0) return 0;
+    if (op == SGR_OP_MINGRU_LOG)
+        return std::max(make_plan(B, T, D, dtype, true, false, false, false, true).ws_bytes,
+                        make_plan(B, T, D, dtype, false, false, false, false, true).ws_bytes);
     // the vector and the scalar variant may cut T differently, and the
     // time-decayed minGRU may take another kernel: cover them all
     size_t need = 0;
@@ -1577,10 +1730,11 @@ void fill_plan(const Plan &p, sgr_plan_t *plan) {
 
 sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
                            int aligned, sgr_plan_t *plan) {
-    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return SGR_ERR_INVALID_ARG;
+    if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX && op != SGR_OP_MINGRU_LOG) return SGR_ERR_INVALID_ARG;
     if (dtype != SGR_F32 && dtype != SGR_BF16) return SGR_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || D < 0 || !plan) return SGR_ERR_INVALID_ARG;
-    fill_plan(make_plan(B, T, D, dtype, aligned != 0, false, op == SGR_OP_MINMAX), plan);
+    fill_plan(make_plan(B, T, D, dtype, aligned != 0, false, op == SGR_OP_MINMAX, false, op == SGR_OP_MINGRU_LOG),
+              plan);
     return SGR_OK;
 }
 
@@ -1596,7 +1750,8 @@ int sgr_backward_kernel(sgr_op_t op, int64_t B, int64_t T, int64_t D, sgr_dtype_
     if (op != SGR_OP_MINGRU && op != SGR_OP_MINMAX) return 0;
     if (dtype != SGR_F32 && dtype != SGR_BF16) return 0;
     if (B < 0 || T < 0 || D < 0) return 0;
-    return seq_backward_planned(B, T, D, dtype == SGR_BF16 ? 2 : 4, aligned != 0) ? KIND_SEQUENTIAL : KIND_TILE;
+    if (seq_backward_planned(B, T, D, dtype == SGR_BF16 ? 2 : 4, aligned != 0)) return KIND_SEQUENTIAL;
+    return make_bwd_plan(B, T, D, dtype, aligned != 0).kind;
 }
 
 sgr_status_t sgr_set_wait_limit(uint32_t polls) {

@@ -84,7 +84,7 @@ _cache = {}
 
 
 def workspace_size(op: str, B: int, T: int, D: int, dtype: torch.dtype) -> int:
-    opc = {"mingru": _abi.SGR_OP_MINGRU, "minmax": _abi.SGR_OP_MINMAX}[op]
+    opc = {"mingru": _abi.SGR_OP_MINGRU, "minmax": _abi.SGR_OP_MINMAX, "mingru_log": _abi.SGR_OP_MINGRU_LOG}[op]
     return int(lib().sgr_workspace_size(opc, B, T, D, _DT[dtype]))
 
 
@@ -130,6 +130,13 @@ def mingru_scan(k: torch.Tensor, hx: torch.Tensor, h0: Optional[torch.Tensor] = 
     """h (B, T, D): minGRU over the time axis of pre-activations k, hx (B, T, D),
     with optional initial state h0 (B, D) or (D,)."""
     return _scan("mingru_scan", _abi.SGR_OP_MINGRU, k, hx, h0, out, workspace)
+
+
+def mingru_scan_log(k: torch.Tensor, hx: torch.Tensor, h0: Optional[torch.Tensor] = None,
+                    out: Optional[torch.Tensor] = None, workspace: Optional[Workspace] = None) -> torch.Tensor:
+    """mingru_scan's result evaluated in log space (log2 h carried through the
+    chunked kernels); h0 must be >= 0."""
+    return _scan("mingru_scan_log", _abi.SGR_OP_MINGRU_LOG, k, hx, h0, out, workspace)
 
 
 def minmax_scan(r: torch.Tensor, s: torch.Tensor, x0: Optional[torch.Tensor] = None,
@@ -321,7 +328,9 @@ def set_kernel_override(kernel: int = 0) -> None:
     """0 automatic, 1 tile kernel, 2 pipelined kernel, 3 pipelined with 15-warp
     blocks, 4 channel-sequential kernel (one warp per 32-channel group), 5 the
     same with each slot's rows split between half-warps, 6 two warps per
-    32-channel group (2-6 where the fast path applies)."""
+    32-channel group (2-6 where the fast path applies).  Gradients: 1 the tile
+    kernel, 2 the pipelined gradient with 7-warp blocks (two per SM), 3 with
+    15-warp blocks (one per SM), 4 the channel-sequential gradient."""
     check("sgr_set_kernel_override", lib().sgr_set_kernel_override(kernel))
 
 

@@ -562,14 +562,19 @@ def test_projected_scan_argument_errors():
 
 
 def test_backward_kernel_choice():
-    """The gradient walks whole sequences per warp (kernel 4) from 3 warps of
-    32 channels per SM, on aligned vector-width rows; otherwise the tile
-    kernel (1)."""
+    """The gradient walks whole sequences per warp (kernel 4) from 5 warps of
+    32 channels per SM, on aligned vector-width rows; below that, on aligned
+    vector-width rows, the pipelined gradient (2) once it has two tiles per SM;
+    otherwise the tile kernel (1)."""
     lib = _abi.lib()
     assert lib.sgr_backward_kernel(MINGRU, 16, 2048, 4096, BF16, 1) == 4     # 2048 groups
-    assert lib.sgr_backward_kernel(MINGRU, 4, 2048, 4096, BF16, 1) == 4      # 512 groups
-    assert lib.sgr_backward_kernel(MINGRU, 2, 2048, 4096, BF16, 1) == 1      # 256 groups
-    assert lib.sgr_backward_kernel(MINGRU, 8, 4096, 1024, F32, 1) == 1       # 256 groups
+    assert lib.sgr_backward_kernel(MINGRU, 8, 2048, 4096, BF16, 1) == 4      # 1024 groups
+    assert lib.sgr_backward_kernel(MINGRU, 4, 2048, 4096, BF16, 1) == 2      # 512 groups
+    assert lib.sgr_backward_kernel(MINGRU, 2, 2048, 4096, BF16, 1) == 2      # 256 groups, 2304 tiles
+    assert lib.sgr_backward_kernel(MINGRU, 8, 4096, 1024, F32, 1) == 2       # 256 groups, 8960 tiles
+    assert lib.sgr_backward_kernel(_abi.SGR_OP_MINMAX, 4, 8192, 768, F32, 1) == 2
+    assert lib.sgr_backward_kernel(MINGRU, 2, 1024, 512, F32, 1) == 1       # 288 tiles: one launch per tile
+    assert lib.sgr_backward_kernel(MINGRU, 8, 4096, 1024, F32, 0) == 1       # unaligned
     assert lib.sgr_backward_kernel(MINGRU, 16, 2048, 4096, BF16, 0) == 1     # unaligned
     assert lib.sgr_backward_kernel(MINGRU, 16, 2048, 4100, BF16, 1) == 1     # D not a vector multiple
     assert lib.sgr_backward_kernel(9, 16, 2048, 4096, BF16, 1) == 0
@@ -582,6 +587,38 @@ def test_backward_kernel_choice():
         lib.sgr_set_kernel_override(0)
 
 
+def test_log_space_plan():
+    """mingru_scan_log runs the chunked kernels at any batch width: its plan is
+    never channel-sequential, and its workspace size covers it where the
+    linear scan of a wide batch needs only the header.  Gradients, summaries
+    and the decayed form do not take it."""
+    lib = _abi.lib()
+    LOG = _abi.SGR_OP_MINGRU_LOG
+    for B, T, D, dt in [(16, 2048, 4096, BF16), (8, 4096, 1024, F32), (2, 1000, 96, F32), (64, 512, 2048, F32)]:
+        for aligned in (True, False):
+            pl = _abi.plan(LOG, B, T, D, dt, aligned)
+            assert pl["kernel"] in (_abi.KERNEL_TILE, _abi.KERNEL_PIPELINED, _abi.KERNEL_PIPELINED_WIDE)
+            assert lib.sgr_workspace_size(LOG, B, T, D, dt) >= pl["workspace_bytes"]
+    assert _abi.plan(MINGRU, 16, 2048, 4096, BF16)["workspace_bytes"] == WS_HEADER
+    assert lib.sgr_workspace_size(LOG, 16, 2048, 4096, BF16) > WS_HEADER
+    assert lib.sgr_backward_workspace_size(LOG, 8, 4096, 1024, F32) == 0
+    assert lib.sgr_backward_kernel(LOG, 8, 4096, 1024, F32, 1) == 0
+
+
+@fake_addresses
+def test_log_space_argument_errors():
+    E = _abi.SGR_ERR_INVALID_ARG
+    fn = "mingru_scan_log"
+    assert scan(fn, A, Bp, None, 0, C, -1, 4, 4, F32, None, 0, None) == E
+    assert scan(fn, None, Bp, None, 0, C, 1, 4, 4, F32, None, 0, None) == E
+    assert scan(fn, A, Bp, None, 0, A + 16, 1, 4, 4, F32, None, 0, None) == E
+    for shp in [(0, 4, 4), (2, 0, 4), (2, 4, 0)]:
+        assert scan(fn, None, None, None, 0, None, *shp, F32, None, 0, None) == _abi.SGR_OK
+    # a wide batch: the linear scan's header-only workspace is too small here
+    assert scan(fn, A, Bp, None, 0, C, 16, 2048, 4096, BF16, 0x50000000, WS_HEADER, None) \
+        == _abi.SGR_ERR_WORKSPACE
+
+
 def test_minmax_plans_take_the_long_tiles():
     """MinMax, next to no arithmetic per element, takes the 15-warp pipelined
     blocks wherever they still give every SM 4 tiles; minGRU on the same
@@ -592,3 +629,75 @@ def test_minmax_plans_take_the_long_tiles():
     # the size query covers this plan (and the unaligned one)
     assert lib.sgr_workspace_size(_abi.SGR_OP_MINMAX, 4, 8192, 768, F32) >= \
         _abi.plan(_abi.SGR_OP_MINMAX, 4, 8192, 768, F32, True)["workspace_bytes"] > 0
+
+
+@pytest.mark.parametrize("shape", [(2, 1000, 96), (1, 3001, 40), (1, 121, 64), (2, 7, 32), (3, 250, 160),
+                                   (8, 4096, 1024)])
+@pytest.mark.parametrize("dtype", [F32, BF16])
+@pytest.mark.parametrize("override,W", [(2, 7), (3, 15)])
+def test_pipelined_backward_indices(shape, dtype, override, W):
+    """The pipelined gradient (persistent blocks, four copy boxes per tile):
+    tiles numbered chain-fastest in processing order, processing chunk c
+    covering time chunk n_chunks - 1 - c; boxes of TC x TR at (dt TC, ct TR, b),
+    the forward output's one row earlier; lane (g, j) of warp w owns channels
+    [g V, g V + V) of processing rows [(w J + j) R, (w J + j) R + R), processing
+    row rho at slot row TR - 1 - rho.  Every slot row read is inside the slot,
+    every (b, t, d) is written exactly once, exactly one thread per channel
+    ends at time row 0, and the workspace covers the hand-off words.
+    Override 2 takes blocks of 7 data warps (two per SM), 3 of 15 (one)."""
+    B, T, D = shape
+    esz = 4 if dtype == F32 else 2
+    if D % (16 // esz):
+        pytest.skip("vector rows only")
+    lib = _abi.lib()
+    assert lib.sgr_set_kernel_override(override) == 0
+    try:
+        assert lib.sgr_backward_kernel(MINGRU, B, T, D, dtype, 1) == 2
+        need = lib.sgr_backward_workspace_size(MINGRU, B, T, D, dtype)
+    finally:
+        lib.sgr_set_kernel_override(0)
+    cg, V = (8 if dtype == F32 else 16), 4
+    R = 2 if dtype == F32 else 4
+    J = 32 // cg
+    TC, TR = cg * V, W * J * R
+    assert TR == 8 * W and (TC * esz) % 16 == 0 and TC <= 256 and TR <= 256
+    assert TR % 4 == 0                       # the decay gaps' box starts at ct TR: a 16-byte multiple
+    n_dt = -(-D // TC)
+    n_chains, n_chunks = B * n_dt, -(-T // TR)
+    n_tiles = n_chains * n_chunks
+    assert n_tiles < 2 ** 31 and n_chunks * TR < 2 ** 31
+    if n_chunks > 1:
+        assert need >= WS_HEADER + 8 * 3 * TC * n_tiles
+    # a slot: four operand boxes, then (decay) TC rates and TR gaps; 3 slots
+    slot = -(-(4 * TR * TC * esz + (TR + TC) * 4) // 128) * 128
+    smem = 3 * slot + 3 * 8 + 3 * 4 + 16 + 2 * W * TC * 8 + 2 * TC * 8 + 2 * TC * 4 + 2 * TC * 4 + 16
+    assert smem * (2 if W == 7 else 1) <= 228 * 1024 - 2 * 1024   # blocks per SM, 1 KB reserved each
+    tile = np.arange(n_tiles, dtype=np.int64)[:, None, None]
+    warp = np.arange(W, dtype=np.int64)[None, :, None]
+    lane = np.arange(32, dtype=np.int64)[None, None, :]
+    c, chain = tile // n_chains, tile % n_chains
+    b, dt = chain // n_dt, chain % n_dt
+    ct = n_chunks - 1 - c
+    assert (ct * TR - 1 >= -1).all()         # the forward output's box starts at row -1 at the earliest
+    g, j = lane % cg, lane // cg
+    d0 = dt * TC + g * V
+    rho0 = (warp * J + j) * R
+    top = ct * TR + TR - 1 - rho0
+    assert ((TR - 1 - rho0 - (R - 1)) >= 0).all() and ((TR - 1 - rho0) < TR).all()
+    ends = (top - (R - 1) == 0) & (d0 < D)
+    cnt0 = np.zeros((B, D), dtype=np.int32)
+    bb, dd = np.broadcast_to(b, ends.shape)[ends], np.broadcast_to(d0, ends.shape)[ends]
+    for v in range(V):
+        np.add.at(cnt0, (bb, dd + v), 1)
+    assert (cnt0 == 1).all(), "one thread per channel ends at time row 0"
+    if B * T * D <= 1 << 22:
+        cover = np.zeros((B, T, D), dtype=np.int32)
+        for r in range(R):
+            t = top - r
+            ok = (t < T) & (d0 < D)
+            tt = np.broadcast_to(t, ok.shape)[ok]
+            b2, d2 = np.broadcast_to(b, ok.shape)[ok], np.broadcast_to(d0, ok.shape)[ok]
+            assert (tt >= 0).all()
+            for v in range(V):
+                np.add.at(cover, (b2, tt, d2 + v), 1)
+        assert (cover == 1).all(), "every element's gradient is written exactly once"

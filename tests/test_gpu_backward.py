@@ -95,10 +95,44 @@ def test_backward_matches_oracle(op, shape, dtype, init):
     assert dp.dtype == TORCH_DT[dtype] and dp.shape == p.shape
     assert channel_scaled_err(dp, rp) <= TOL_BWD[dtype]
     assert channel_scaled_err(dq, rq) <= TOL_BWD[dtype]
-    # the initial-state gradient: relative to its own magnitude per channel
-    scale = np.maximum(np.abs(rinit), np.abs(gy.double().numpy()).sum(axis=1) * 1e-3)
-    err = np.abs(dinit.double().cpu().numpy() - rinit) / np.maximum(scale, 1e-30)
-    assert err.max() <= TOL_BWD[dtype] * 10
+    assert row_scaled_err(dinit, rinit) <= TOL_BWD[dtype]
+
+
+def row_scaled_err(got, ref) -> float:
+    """dL/d(initial state), (B, D): a signed sum over the whole sequence, so
+    measured against the largest |dL/dh0| of the same batch row."""
+    got = got.detach().double().cpu().numpy() if hasattr(got, "detach") else np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    scale = np.maximum(np.abs(ref).max(axis=1, keepdims=True), 1e-30)
+    return float((np.abs(got - ref) / scale).max())
+
+
+# The pipelined gradient (persistent blocks, copy-engine ring; the automatic
+# choice for aligned narrow batches with at least two tiles per SM), forced on
+# shapes with ragged sequences and channel tiles, one-tile sequences, a single
+# row and short sequences.
+PIPE_SHAPES = [(2, 1000, 96), (1, 3001, 40), (3, 250, 160), (1, 121, 64), (2, 7, 32), (4, 240, 8)]
+
+
+@pytest.mark.parametrize("op", ["mingru", "minmax"])
+@pytest.mark.parametrize("shape", PIPE_SHAPES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("init", [None, "u01_1"])
+@pytest.mark.parametrize("kernel", [2, 3])
+def test_pipelined_backward_matches_oracle(op, shape, dtype, init, kernel):
+    """kernel 2: blocks of 7 data warps (two per SM); 3: of 15 (one per SM)."""
+    B, T, D = shape
+    if dtype == "bf16" and D % 8:
+        pytest.skip("bf16 vector rows need D % 8 == 0")
+    sgr.set_kernel_override(kernel)
+    code = _abi.SGR_F32 if dtype == "f32" else _abi.SGR_BF16
+    assert _abi.lib().sgr_backward_kernel(0 if op == "mingru" else 1, B, T, D, code, 1) == 2
+    p, q, i0, fwd, gy = inputs(op, *shape, dtype, init, seed=sum(shape) % 811 + 5)
+    dp, dq, dinit = gpu_backward(op, p, q, i0, fwd, gy)
+    rp, rq, rinit = oracle_backward(op, p, q, i0, gy)
+    assert channel_scaled_err(dp, rp) <= TOL_BWD[dtype]
+    assert channel_scaled_err(dq, rq) <= TOL_BWD[dtype]
+    assert row_scaled_err(dinit, rinit) <= TOL_BWD[dtype]
 
 
 @pytest.mark.parametrize("op", ["mingru", "minmax"])
@@ -134,7 +168,10 @@ def test_minmax_backward_ties_match_oracle():
     assert not (both & distinct & (fwd.numpy() != s.numpy())).any()
 
 
-def test_backward_initial_state_layouts():
+@pytest.mark.parametrize("kernel", [0, 2])
+def test_backward_initial_state_layouts(kernel):
+    # 0: automatic (the tile kernel at this size), 2: the pipelined gradient
+    sgr.set_kernel_override(kernel)
     B, T, D = 3, 600, 96
     p, q, i0, fwd, gy = inputs("mingru", B, T, D, "f32", "u01_1", seed=11)
     P, Q, F, G = (t.to(DEV) for t in (p, q, fwd, gy))
@@ -155,7 +192,7 @@ def test_backward_initial_state_layouts():
     torch.cuda.synchronize()
     rk, rhx, rh0 = oracle.mingru_backward(p, q, i0, gy)
     assert channel_scaled_err(dk, rk) <= TOL_BWD["f32"]
-    assert np.allclose(dwide[:, D:2 * D].cpu().double().numpy(), rh0, rtol=1e-4, atol=1e-6)
+    assert row_scaled_err(dwide[:, D:2 * D], rh0) <= TOL_BWD["f32"]
     assert bool((dwide[:, :D] == 7.0).all()) and bool((dwide[:, 2 * D:] == 7.0).all())
     # T = 0: the initial-state gradient is zero
     dh0 = torch.full((B, D), 5.0, device=DEV)
@@ -184,7 +221,8 @@ def test_autograd_wrappers(op, h0_kind):
     assert channel_scaled_err(Q.grad, rq) <= TOL_BWD["f32"]
     if I is not None:
         want = rinit if init.dim() == 2 else rinit.sum(0)
-        assert np.allclose(I.grad.cpu().double().numpy(), want, rtol=1e-4, atol=1e-6)
+        got = I.grad.cpu().double().numpy()
+        assert row_scaled_err(got.reshape(-1, D), np.asarray(want).reshape(-1, D)) <= TOL_BWD["f32"]
 
 
 def test_backward_bounded_wait_reports_timeout():

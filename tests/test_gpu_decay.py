@@ -132,6 +132,47 @@ def test_decay_gap_layouts(B, pad, gap_off, lam_off, kernel, dtype):
     h = sgr.mingru_scan_decay(k.to(DEV), hx.to(DEV), h0.to(DEV), gaps, rates)
     torch.cuda.synchronize()
     assert rel_err(h, oracle.mingru_decay(k, hx, h0, dt, lam)) <= TOL[dtype]
+    # the pipelined gradient (2: 7-warp blocks, 3: 15-warp blocks) with the
+    # same layouts: gaps and rates in its ring slots or by plain loads
+    assert _abi.lib().sgr_backward_kernel(0, B, T, D, _abi.SGR_F32 if dtype == "f32" else _abi.SGR_BF16, 1) == 2
+    g = torch.Generator().manual_seed(13 + pad)
+    gy = torch.randn(B, T, D, generator=g).to(TORCH_DT[dtype])
+    fwd = torch.from_numpy(oracle.mingru_decay(k, hx, h0, dt, lam)).to(TORCH_DT[dtype])
+    dk, dhx, dh0, dlam = sgr.mingru_scan_decay_backward(k.to(DEV), hx.to(DEV), h0.to(DEV), gaps, rates,
+                                                        fwd.to(DEV), gy.to(DEV))
+    torch.cuda.synchronize()
+    rk, rhx, rh0, rlam = oracle.mingru_decay_backward(k, hx, h0, dt, lam, gy)
+    assert channel_scaled_err(dk, rk) <= TOL_BWD[dtype]
+    assert channel_scaled_err(dhx, rhx) <= TOL_BWD[dtype]
+    e0 = float((np.abs(dh0.cpu().double().numpy() - rh0) / np.abs(rh0).max(axis=1, keepdims=True)).max())
+    assert e0 <= TOL_BWD[dtype]
+    assert lam_err(dlam, rlam, k, hx, h0, dt, lam, gy) <= TOL_BWD[dtype]
+
+
+@pytest.mark.parametrize("log1p_delta", [False, True])
+def test_decay_workload_gradient_every_channel(log1p_delta):
+    """The decayed gradient on the B8 x 4096 x 1024 fp32 workload (the
+    pipelined gradient with 7-warp blocks, gaps and rates in its ring slots)
+    against the oracle on every channel."""
+    B, T, D = 8, 4096, 1024
+    assert _abi.lib().sgr_backward_kernel(0, B, T, D, _abi.SGR_F32, 1) == 2
+    k, hx, h0, dt, lam = data(B, T, D, "f32", "u01_1", seed=61, gap_scale=20.0 if log1p_delta else 1.0,
+                              wipe_at=2000)
+    g = torch.Generator().manual_seed(62)
+    gy = torch.randn(B, T, D, generator=g)
+    fwd = torch.from_numpy(oracle.mingru_decay(k, hx, h0, dt, lam, log1p_delta)).float()
+    dk, dhx, dh0, dlam = sgr.mingru_scan_decay_backward(k.to(DEV), hx.to(DEV), h0.to(DEV), dt.to(DEV),
+                                                        lam.to(DEV), fwd.to(DEV), gy.to(DEV), log1p_delta)
+    torch.cuda.synchronize()
+    rk, rhx, rh0, rlam = oracle.mingru_decay_backward(k, hx, h0, dt, lam, gy, log1p_delta)
+    ek, eh = channel_scaled_err(dk, rk), channel_scaled_err(dhx, rhx)
+    e0 = float((np.abs(dh0.cpu().double().numpy() - rh0) / np.abs(rh0).max(axis=1, keepdims=True)).max())
+    gabs = np.abs(gy.double().numpy())
+    _, _, _, mag = oracle.mingru_decay_backward(k, hx, h0, dt, lam, gabs, log1p_delta)
+    el = float((np.abs(dlam.cpu().double().numpy() - rlam) / np.maximum(np.abs(mag), 1e-30)).max())
+    print(f"decayed gradient B8 x 4096 x 1024 log1p={log1p_delta}: dk {ek:.3e}, dhx {eh:.3e}, "
+          f"dh0 {e0:.3e} (scaled), dlam {el:.3e} of the summed term magnitudes")
+    assert max(ek, eh, e0, el) <= TOL_BWD["f32"]
 
 
 # The channel-sequential kernels take the gaps through the copy engine when

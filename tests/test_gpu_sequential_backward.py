@@ -84,10 +84,11 @@ def test_sequential_backward_matches_oracle(op, shape, dtype, init):
     assert dp.dtype == TORCH_DT[dtype] and dp.shape == p.shape
     assert channel_scaled_err(dp, rp) <= TOL_BWD[dtype]
     assert channel_scaled_err(dq, rq) <= TOL_BWD[dtype]
-    # the initial-state gradient, relative to its own magnitude per channel
-    scale = np.maximum(np.abs(rinit), np.abs(gy.double().numpy()).sum(axis=1) * 1e-3)
-    err = np.abs(dinit.double().cpu().numpy() - rinit) / np.maximum(scale, 1e-30)
-    assert err.max() <= TOL_BWD[dtype] * 10
+    # the initial-state gradient (a signed sum over the sequence), against the
+    # largest |dL/dh0| of its batch row
+    got = dinit.double().cpu().numpy()
+    scale = np.maximum(np.abs(rinit).max(axis=1, keepdims=True), 1e-30)
+    assert float((np.abs(got - rinit) / scale).max()) <= TOL_BWD[dtype]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -109,7 +110,7 @@ def test_sequential_decay_backward_matches_oracle(dtype, log1p_delta):
     assert channel_scaled_err(dhx, rhx) <= TOL_BWD[dtype]
     _, _, _, mag = oracle.mingru_decay_backward(k, hx, h0, dt, lam, np.abs(gy.double().numpy()), log1p_delta)
     scale = np.maximum(np.abs(mag), 1e-30)
-    assert float((np.abs(dlam.cpu().double().numpy() - rlam) / scale).max()) <= TOL_BWD[dtype] * 10
+    assert float((np.abs(dlam.cpu().double().numpy() - rlam) / scale).max()) <= TOL_BWD[dtype]
 
 
 def test_wide_batch_gradient_selects_it_and_matches():
@@ -127,4 +128,7 @@ def test_wide_batch_gradient_selects_it_and_matches():
     tp, tq, tinit = sgr.mingru_scan_backward(*dev(p, q, i0, fwd, gy))
     torch.cuda.synchronize()
     assert channel_scaled_err(tp, rp) <= TOL_BWD["bf16"]
-    assert torch.allclose(tinit.float(), dinit.float(), rtol=2e-2, atol=1e-3)
+    # both initial-state gradients against the oracle's, per batch row
+    for d0 in (dinit, tinit):
+        got = d0.double().cpu().numpy()
+        assert float((np.abs(got - rinit) / np.abs(rinit).max(axis=1, keepdims=True)).max()) <= TOL_BWD["bf16"]
