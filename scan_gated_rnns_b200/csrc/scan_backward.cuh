@@ -59,6 +59,38 @@ struct MinGRUBwd {
         cP = (sk * rk) * (g - gamma * h);
         cQ = z * gp;
     }
+    // the same for two elements, the arithmetic in packed fp32x2 operations
+    // (the MUFU operations and the sign selects stay per element)
+    static __device__ __forceinline__ void coeffs_gated2(float2 k, float2 hx, float2 h, float2 gamma,
+                                                         float2 &A, float2 &cP, float2 &cQ) {
+        const float2 c = make_float2(kNegLog2e, kNegLog2e), one = make_float2(1.f, 1.f);
+        const float2 tk = __fmul2_rn(make_float2(fabsf(k.x), fabsf(k.y)), c);
+        const float2 th = __fmul2_rn(make_float2(fabsf(hx.x), fabsf(hx.y)), c);
+        const float2 ek = make_float2(fast_exp2(tk.x), fast_exp2(tk.y));
+        const float2 eh = make_float2(fast_exp2(th.x), fast_exp2(th.y));
+        const float2 dk = __fadd2_rn(ek, one), dh = __fadd2_rn(eh, one);
+        const float2 pr = __fmul2_rn(dk, dh);
+        const float2 inv = make_float2(fast_rcp(pr.x), fast_rcp(pr.y));
+        const float2 rk = __fmul2_rn(dh, inv);           // sigmoid(|k|)
+        const float2 rh = __fmul2_rn(dk, inv);           // sigmoid(|hx|)
+        const float2 sk = __fmul2_rn(ek, rk);            // sigmoid(-|k|)
+        const float2 sh = __fmul2_rn(eh, rh);            // sigmoid(-|hx|)
+        const bool kp0 = k.x >= 0.f, kp1 = k.y >= 0.f;
+        const bool hp0 = hx.x >= 0.f, hp1 = hx.y >= 0.f;
+        const float2 z = make_float2(kp0 ? rk.x : sk.x, kp1 ? rk.y : sk.y);
+        A = __fmul2_rn(make_float2(kp0 ? sk.x : rk.x, kp1 ? sk.y : rk.y), gamma);
+        const float2 hp = __fadd2_rn(hx, make_float2(0.5f, 0.5f));
+        const float2 shrh = __fmul2_rn(sh, rh);
+        const float2 g = make_float2(hp0 ? hp.x : sh.x, hp1 ? hp.y : sh.y);
+        const float2 gp = make_float2(hp0 ? 1.f : shrh.x, hp1 ? 1.f : shrh.y);
+        const float2 gmh = __ffma2_rn(make_float2(-gamma.x, -gamma.y), h, g);    // g - gamma h
+        cP = __fmul2_rn(__fmul2_rn(sk, rk), gmh);
+        cQ = __fmul2_rn(z, gp);
+    }
+    static __device__ __forceinline__ void coeffs2(float2 k, float2 hx, float2 h, float2 &A, float2 &cP,
+                                                   float2 &cQ) {
+        coeffs_gated2(k, hx, h, make_float2(1.f, 1.f), A, cP, cQ);
+    }
     static __device__ __forceinline__ float default_state() { return 0.f; }
 };
 
@@ -76,6 +108,11 @@ struct MinMaxBwd {
         A = dout_dm * (1.f - dm_dr);
         cP = dout_dm * dm_dr;
         cQ = 1.f - dout_dm;
+    }
+    static __device__ __forceinline__ void coeffs2(float2 r, float2 s, float2 x, float2 &A, float2 &cP,
+                                                   float2 &cQ) {
+        coeffs(r.x, s.x, x.x, A.x, cP.x, cQ.x);
+        coeffs(r.y, s.y, x.y, A.y, cP.y, cQ.y);
     }
     static __device__ __forceinline__ float default_state() { return 0.f; }
 };

@@ -279,6 +279,22 @@ struct MinGRUDecayOp : MinGRUOp {
     static constexpr bool kDecay = true;
 };
 
+// The step pairs of two elements (two channels of a row in the pipelined
+// kernel) in packed fp32x2 operations: bf16 I/O takes the shared-reciprocal
+// form, fp32 I/O the form with relative-accurate gates for either sign; the
+// log-space operator evaluates them one by one.
+template <class Op, typename IO>
+__device__ __forceinline__ void element_pair(float k0, float hx0, float k1, float hx1, float2 &a, float2 &b) {
+    if constexpr (Op::kLogSpace) {
+        Op::element(k0, hx0, a.x, b.x);
+        Op::element(k1, hx1, a.y, b.y);
+    } else if constexpr (sizeof(IO) == 2 && Op::kLeanRows) {
+        Op::element_rows_lean(k0, hx0, k1, hx1, a, b);
+    } else {
+        Op::element_rows(k0, hx0, k1, hx1, a, b);
+    }
+}
+
 // gamma = exp(-lambda u) = 2^(lam2 u) with lam2 = -lambda log2 e (<= 0).
 // The wipe needs no compare: the MUFU 2^x flushes every result below the
 // normal range to +0, so gamma is exactly 0 for all lambda u above about 87.3
@@ -1129,19 +1145,19 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                     }
 #pragma unroll
                     for (int i = 0; i < V2; ++i) {
-                        float a0, b0, a1, b1;
-                        Op::element(x0[2 * i], x1[2 * i], a0, b0);
-                        Op::element(x0[2 * i + 1], x1[2 * i + 1], a1, b1);
+                        float2 a2, b2;
+                        element_pair<Op, IO>(x0[2 * i], x1[2 * i], x0[2 * i + 1], x1[2 * i + 1], a2, b2);
                         if constexpr (DT) {
-                            a0 *= decay_gamma(s_lam[g * V + 2 * i] * -1.4426950408889634f, u);
-                            a1 *= decay_gamma(s_lam[g * V + 2 * i + 1] * -1.4426950408889634f, u);
+                            const float2 l2 = __fmul2_rn(*reinterpret_cast<const float2 *>(s_lam + g * V + 2 * i),
+                                                         make_float2(kNegLog2e, kNegLog2e));
+                            const float2 e = __fmul2_rn(l2, make_float2(u, u));
+                            a2 = __fmul2_rn(a2, make_float2(fast_exp2(e.x), fast_exp2(e.y)));
                         } else if constexpr (Op::kDecay) {
-                            a0 *= decay_gamma(lam2[2 * i], u);
-                            a1 *= decay_gamma(lam2[2 * i + 1], u);
+                            a2 = __fmul2_rn(a2, make_float2(decay_gamma(lam2[2 * i], u), decay_gamma(lam2[2 * i + 1], u)));
                         }
-                        PA[SB][r][i] = make_float2(a0, a1);
-                        PB[SB][r][i] = make_float2(b0, b1);
-                        Op::fold2(IA[i], IB[i], PA[SB][r][i], PB[SB][r][i]);
+                        PA[SB][r][i] = a2;
+                        PB[SB][r][i] = b2;
+                        Op::fold2(IA[i], IB[i], a2, b2);
                     }
                 }
             };

@@ -87,6 +87,7 @@ scan_pipelined_backward_kernel(const BwdParams bp, const __grid_constant__ CUten
     constexpr int TC = Shape::TC;
     constexpr int TR = Shape::TR;
     constexpr int CV = TC / 32;
+    constexpr int V2 = V / 2;                 // channel pairs of a thread (packed fp32x2 work)
     constexpr uint32_t NT = (W + 1) * 32;
     constexpr bool kDec = BOp::kDecay;
     // as in the forward kernel: fp32 I/O folds the warp summaries in the last
@@ -230,12 +231,16 @@ scan_pipelined_backward_kernel(const BwdParams bp, const __grid_constant__ CUten
                 }
             }
 
-            // per element: A, gy, cP, cQ (and the dL/dlambda factor) for phase B
-            float A[R][V], Gy[R][V], P[R][V], Q[R][V];
-            [[maybe_unused]] float Ed[kDec ? R : 1][V];
-            float2 incl[V];
+            // per element: A, gy, cP, cQ (and the dL/dlambda factor) for phase B,
+            // held as pairs of neighbouring channels for packed fp32x2 work
+            float2 A[R][V2], Gy[R][V2], P[R][V2], Q[R][V2];
+            [[maybe_unused]] float2 Ed[kDec ? R : 1][V2];
+            float2 IA[V2], IB[V2];             // the fold of the thread's rows, per channel pair
 #pragma unroll
-            for (int v = 0; v < V; ++v) incl[v] = Op::identity();
+            for (int i = 0; i < V2; ++i) {
+                IA[i] = make_float2(1.f, 1.f);
+                IB[i] = make_float2(0.f, 0.f);
+            }
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 const int64_t t = top - r;
@@ -252,23 +257,37 @@ scan_pipelined_backward_kernel(const BwdParams bp, const __grid_constant__ CUten
                 [[maybe_unused]] float u = 0.f;
                 if constexpr (kDec) u = ur[r];
 #pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    float a, cp, cq;
+                for (int i = 0; i < V2; ++i) {
+                    const float2 k2 = make_float2(xk[2 * i], xk[2 * i + 1]);
+                    const float2 h2 = make_float2(xh[2 * i], xh[2 * i + 1]);
+                    const float2 f2 = make_float2(xf[2 * i], xf[2 * i + 1]);
+                    float2 a, cp, cq;
                     if constexpr (kDec) {
-                        BOp::coeffs_gated(xk[v], xh[v], xf[v], decay_gamma(lam2[v], u), a, cp, cq);
+                        const float2 gam = make_float2(decay_gamma(lam2[2 * i], u), decay_gamma(lam2[2 * i + 1], u));
+                        BOp::coeffs_gated2(k2, h2, f2, gam, a, cp, cq);
                         // dL/dlambda gains delta A h_{t-1} (-u)
-                        Ed[r][v] = ok ? -u * a * xf[v] : 0.f;
+                        const float2 e = __fmul2_rn(__fmul2_rn(a, f2), make_float2(-u, -u));
+                        Ed[r][i] = ok ? e : make_float2(0.f, 0.f);
                     } else {
-                        BOp::coeffs(xk[v], xh[v], xf[v], a, cp, cq);
+                        BOp::coeffs2(k2, h2, f2, a, cp, cq);
                     }
-                    a = ok ? a : 1.f;                 // rows past T, channels past D: the identity pair
-                    const float gv = ok ? xg[v] : 0.f;
-                    A[r][v] = a;
-                    Gy[r][v] = gv;
-                    P[r][v] = cp;
-                    Q[r][v] = cq;
-                    incl[v] = Op::combine(incl[v], make_float2(a, a * gv));
+                    // rows past T, channels past D: the identity pair
+                    a = ok ? a : make_float2(1.f, 1.f);
+                    const float2 gv = ok ? make_float2(xg[2 * i], xg[2 * i + 1]) : make_float2(0.f, 0.f);
+                    A[r][i] = a;
+                    Gy[r][i] = gv;
+                    P[r][i] = cp;
+                    Q[r][i] = cq;
+                    // (IA, IB) <- (IA a, IB a + a gy)
+                    IB[i] = __ffma2_rn(IB[i], a, __fmul2_rn(a, gv));
+                    IA[i] = __fmul2_rn(IA[i], a);
                 }
+            }
+            float2 incl[V];
+#pragma unroll
+            for (int i = 0; i < V2; ++i) {
+                incl[2 * i] = make_float2(IA[i].x, IB[i].x);
+                incl[2 * i + 1] = make_float2(IA[i].y, IB[i].y);
             }
             // scan across the J row groups of the warp
 #pragma unroll
@@ -325,29 +344,42 @@ scan_pipelined_backward_kernel(const BwdParams bp, const __grid_constant__ CUten
 
             // ---- phase B: replay lam from the thread's incoming gradient
             named_barrier_sync(3 + BUF, NT);
-            float lam[V];
-            [[maybe_unused]] float dl[V];
+            float2 lam[V2];
+            [[maybe_unused]] float2 dl2[V2];
 #pragma unroll
-            for (int v = 0; v < V; ++v) {
-                const int c0 = g * V + v;
-                lam[v] = Op::apply(ex[v], Op::apply(s_tot[BUF][warp][c0], s_hin[BUF][c0]));
-                if constexpr (kDec) dl[v] = 0.f;
+            for (int i = 0; i < V2; ++i) {
+                const int c0 = g * V + 2 * i;
+                lam[i] = make_float2(Op::apply(ex[2 * i], Op::apply(s_tot[BUF][warp][c0], s_hin[BUF][c0])),
+                                     Op::apply(ex[2 * i + 1], Op::apply(s_tot[BUF][warp][c0 + 1], s_hin[BUF][c0 + 1])));
+                if constexpr (kDec) dl2[i] = make_float2(0.f, 0.f);
             }
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 float y0[V], y1[V];
 #pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    const float delta = Gy[r][v] + lam[v];
-                    y0[v] = delta * P[r][v];
-                    y1[v] = delta * Q[r][v];
-                    if constexpr (kDec) dl[v] = fmaf(delta, Ed[r][v], dl[v]);
-                    lam[v] = A[r][v] * delta;
+                for (int i = 0; i < V2; ++i) {
+                    const float2 delta = __fadd2_rn(Gy[r][i], lam[i]);
+                    const float2 a0 = __fmul2_rn(delta, P[r][i]);
+                    const float2 a1 = __fmul2_rn(delta, Q[r][i]);
+                    y0[2 * i] = a0.x;
+                    y0[2 * i + 1] = a0.y;
+                    y1[2 * i] = a1.x;
+                    y1[2 * i + 1] = a1.y;
+                    if constexpr (kDec) dl2[i] = __ffma2_rn(delta, Ed[r][i], dl2[i]);
+                    lam[i] = __fmul2_rn(A[r][i], delta);
                 }
                 const int64_t t = top - r;
                 if (dvalid && t < p.T) {
                     Access<IO, V>::store(out0 + base + t * p.D, y0);
                     Access<IO, V>::store(out1 + base + t * p.D, y1);
+                }
+            }
+            [[maybe_unused]] float dl[V];
+            if constexpr (kDec) {
+#pragma unroll
+                for (int i = 0; i < V2; ++i) {
+                    dl[2 * i] = dl2[i].x;
+                    dl[2 * i + 1] = dl2[i].y;
                 }
             }
             if constexpr (kDec) {
@@ -390,7 +422,7 @@ scan_pipelined_backward_kernel(const BwdParams bp, const __grid_constant__ CUten
             if (bp.dinit && dvalid && top - (R - 1) == 0) {
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
-                    const float y[1] = {lam[v]};
+                    const float y[1] = {(v & 1) ? lam[v / 2].y : lam[v / 2].x};
                     Access<IO, 1>::store(static_cast<IO *>(bp.dinit) + int64_t(tc.b) * bp.dinit_bs + d0 + v, y);
                 }
             }

@@ -531,6 +531,7 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
                                 const __grid_constant__ CUtensorMap map_d1,
                                 const __grid_constant__ CUtensorMap map_gap) {
     static_assert(!DT || BOp::kDecay, "gaps through the copy engine need a decay operator");
+    static_assert(kSeqRows % 2 == 0, "rows are taken in pairs");
     constexpr uint32_t kGap = DT ? kSeqGapBytes : 0;
     using LR = LaneRow<IO>;
     constexpr int CW = 32;
@@ -627,26 +628,45 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
         const uint32_t obuf = outb + uint32_t(i & (kSeqOutBufs - 1)) * kSeqBwdOut * kOpBytes;
         const uint32_t dst = obuf + uint32_t(lane) * uint32_t(sizeof(IO));
         const int valid = int(p.T - int64_t(j) * kSeqRows);         // rows of the slot inside T (>= 1)
+        // rows r and r - 1 as the two halves of packed fp32x2 operations
+        // (coefficients, outputs, dL/dlambda terms); the gradient itself
+        // runs through them one row at a time
         auto rows = [&](auto fullc) {
             constexpr bool FULL = decltype(fullc)::value;
 #pragma unroll
-            for (int r = kSeqRows - 1; r >= 0; --r) {
-                float A, cP, cQ;
-                [[maybe_unused]] float u = 0.f;
+            for (int r = kSeqRows - 1; r >= 1; r -= 2) {
+                const float2 k2 = make_float2(xk[r], xk[r - 1]);
+                const float2 h2 = make_float2(xh[r], xh[r - 1]);
+                const float2 f2 = make_float2(xf[r], xf[r - 1]);
+                float2 A, cP, cQ;
+                [[maybe_unused]] float2 u2 = make_float2(0.f, 0.f);
                 if constexpr (BOp::kDecay) {
-                    u = __shfl_sync(0xffffffffu, gcur, r);
-                    BOp::coeffs_gated(xk[r], xh[r], xf[r], decay_gamma(lam2, u), A, cP, cQ);
+                    u2 = make_float2(__shfl_sync(0xffffffffu, gcur, r), __shfl_sync(0xffffffffu, gcur, r - 1));
+                    BOp::coeffs_gated2(k2, h2, f2, make_float2(decay_gamma(lam2, u2.x), decay_gamma(lam2, u2.y)),
+                                       A, cP, cQ);
                 } else {
-                    BOp::coeffs(xk[r], xh[r], xf[r], A, cP, cQ);
+                    BOp::coeffs2(k2, h2, f2, A, cP, cQ);
                 }
-                const float delta = xg[r] + lam;
-                if (FULL || r < valid) {
-                    lam = A * delta;
+                float2 delta;
+                delta.x = xg[r] + lam;
+                if (FULL || r < valid) lam = A.x * delta.x;
+                delta.y = xg[r - 1] + lam;
+                if (FULL || r - 1 < valid) lam = A.y * delta.y;
+                if constexpr (BOp::kDecay) {
                     // dL/dlambda gains delta (1 - z) h_{t-1} dgamma/dlambda = delta A h_{t-1} (-u)
-                    if constexpr (BOp::kDecay) dl = fmaf(delta, -u * A * xf[r], dl);
+                    float2 e = __fmul2_rn(__fmul2_rn(A, f2), make_float2(-u2.x, -u2.y));
+                    if (!FULL) {
+                        if (r >= valid) e.x = 0.f;
+                        if (r - 1 >= valid) e.y = 0.f;
+                    }
+                    const float2 de = __fmul2_rn(delta, e);
+                    dl += de.x + de.y;
                 }
-                LR::store(dst + r * kRowBytes, delta * cP);
-                LR::store(dst + kOpBytes + r * kRowBytes, delta * cQ);
+                const float2 o0 = __fmul2_rn(delta, cP), o1 = __fmul2_rn(delta, cQ);
+                LR::store(dst + r * kRowBytes, o0.x);
+                LR::store(dst + (r - 1) * kRowBytes, o0.y);
+                LR::store(dst + kOpBytes + r * kRowBytes, o1.x);
+                LR::store(dst + kOpBytes + (r - 1) * kRowBytes, o1.y);
             }
         };
         if (__any_sync(0xffffffffu, bad)) {
