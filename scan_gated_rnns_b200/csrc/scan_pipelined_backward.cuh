@@ -265,8 +265,9 @@ scan_pipelined_backward_kernel(const BwdParams bp, const __grid_constant__ CUten
                     if constexpr (kDec) {
                         const float2 gam = make_float2(decay_gamma(lam2[2 * i], u), decay_gamma(lam2[2 * i + 1], u));
                         BOp::coeffs_gated2(k2, h2, f2, gam, a, cp, cq);
-                        // dL/dlambda gains delta A h_{t-1} (-u)
-                        const float2 e = __fmul2_rn(__fmul2_rn(a, f2), make_float2(-u, -u));
+                        // dL/dlambda gains delta A h_{t-1} (-u) = (A delta) (-u h_{t-1}):
+                        // the second factor here, the first in phase B
+                        const float2 e = __fmul2_rn(f2, make_float2(-u, -u));
                         Ed[r][i] = ok ? e : make_float2(0.f, 0.f);
                     } else {
                         BOp::coeffs2(k2, h2, f2, a, cp, cq);
@@ -365,8 +366,8 @@ scan_pipelined_backward_kernel(const BwdParams bp, const __grid_constant__ CUten
                     y0[2 * i + 1] = a0.y;
                     y1[2 * i] = a1.x;
                     y1[2 * i + 1] = a1.y;
-                    if constexpr (kDec) dl2[i] = __ffma2_rn(delta, Ed[r][i], dl2[i]);
                     lam[i] = __fmul2_rn(A[r][i], delta);
+                    if constexpr (kDec) dl2[i] = __ffma2_rn(lam[i], Ed[r][i], dl2[i]);
                 }
                 const int64_t t = top - r;
                 if (dvalid && t < p.T) {

@@ -508,10 +508,15 @@ namespace sgr {
 
 constexpr int kSeqBwdIn = 4;        // operands loaded per slot
 constexpr int kSeqBwdOut = 2;       // gradients stored per slot
+// Staging buffers of the gradients: a slot's buffer is written again three
+// slots later, so a store has two slots' work to finish reading it (with
+// two buffers, the plain gradient's warps waited on their stores of two
+// slots back: 26% of the sampled stalls on the bf16 throughput workload).
+constexpr int kSeqBwdOutBufs = 3;
 
 __host__ __device__ constexpr size_t seq_bwd_warp_bytes(int S, int row_bytes, size_t gap = 0) {
     return (size_t(S) * (kSeqBwdIn * kSeqRows * row_bytes + gap) +
-            size_t(kSeqOutBufs) * kSeqBwdOut * kSeqRows * row_bytes + size_t(S) * 8 + 127) / 128 * 128;
+            size_t(kSeqBwdOutBufs) * kSeqBwdOut * kSeqRows * row_bytes + size_t(S) * 8 + 127) / 128 * 128;
 }
 
 struct SeqBwdParams {
@@ -554,8 +559,8 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
     constexpr uint32_t kSlot = kSeqBwdIn * kOpBytes + kGap;         // [in0 | in1 | gy | fwd | gaps]
     const uint32_t base = smem_addr(smem) + uint32_t(warp * seq_bwd_warp_bytes(S, kRowBytes, kGap));
     const uint32_t ring = base;
-    const uint32_t outb = base + uint32_t(S) * kSlot;                // 2 x [d in0 | d in1]
-    const uint32_t bars = outb + kSeqOutBufs * kSeqBwdOut * kOpBytes;
+    const uint32_t outb = base + uint32_t(S) * kSlot;                // 3 x [d in0 | d in1]
+    const uint32_t bars = outb + kSeqBwdOutBufs * kSeqBwdOut * kOpBytes;
 
     const int n_slots = int((p.T + kSeqRows - 1) / kSeqRows);       // T < 2^31 (host check)
     // processing slot i covers time rows [j RB, j RB + RB), j = n_slots - 1 - i
@@ -614,7 +619,7 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
             xf[r] = LR::load(src + 3 * kOpBytes + r * kRowBytes);
         }
         if constexpr (DT) gcur = seq_smem_gap(p, ring + uint32_t(s) * kSlot + kSeqBwdIn * kOpBytes, lane);
-        if (lane == 0) bulk_wait_read<kSeqOutBufs - 1>();            // staging buffers of slot i - 2
+        if (lane == 0) bulk_wait_read<kSeqBwdOutBufs - 1>();         // staging buffers of slot i - 3
         __syncwarp();
         if (lane == 0 && !bad && i + S < n_slots) {
             fence_proxy_async();
@@ -625,7 +630,7 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
             phase ^= 1u;
         }
         if (j == 0) xf[0] = h_init;                                  // the state before t = 0
-        const uint32_t obuf = outb + uint32_t(i & (kSeqOutBufs - 1)) * kSeqBwdOut * kOpBytes;
+        const uint32_t obuf = outb + uint32_t(i % kSeqBwdOutBufs) * kSeqBwdOut * kOpBytes;
         const uint32_t dst = obuf + uint32_t(lane) * uint32_t(sizeof(IO));
         const int valid = int(p.T - int64_t(j) * kSeqRows);         // rows of the slot inside T (>= 1)
         // rows r and r - 1 as the two halves of packed fp32x2 operations
@@ -647,19 +652,22 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
                 } else {
                     BOp::coeffs2(k2, h2, f2, A, cP, cQ);
                 }
-                float2 delta;
+                float2 delta, lamn;
                 delta.x = xg[r] + lam;
                 if (FULL || r < valid) lam = A.x * delta.x;
+                lamn.x = lam;
                 delta.y = xg[r - 1] + lam;
                 if (FULL || r - 1 < valid) lam = A.y * delta.y;
+                lamn.y = lam;
                 if constexpr (BOp::kDecay) {
-                    // dL/dlambda gains delta (1 - z) h_{t-1} dgamma/dlambda = delta A h_{t-1} (-u)
-                    float2 e = __fmul2_rn(__fmul2_rn(A, f2), make_float2(-u2.x, -u2.y));
+                    // dL/dlambda gains delta (1 - z) h_{t-1} dgamma/dlambda
+                    //   = delta A h_{t-1} (-u) = (A delta) (-u h_{t-1})
+                    float2 e = __fmul2_rn(f2, make_float2(-u2.x, -u2.y));
                     if (!FULL) {
                         if (r >= valid) e.x = 0.f;
                         if (r - 1 >= valid) e.y = 0.f;
                     }
-                    const float2 de = __fmul2_rn(delta, e);
+                    const float2 de = __fmul2_rn(lamn, e);
                     dl += de.x + de.y;
                 }
                 const float2 o0 = __fmul2_rn(delta, cP), o1 = __fmul2_rn(delta, cQ);
