@@ -288,7 +288,7 @@ def scan_fn(w, p, q, init, out, ws):
     return lambda: f(p, q, init, out=out, workspace=ws)
 
 
-PASS_SUFFIX = {"backward": "_backward", "decay": "_decay", "decay_backward": "_decay_backward"}
+PASS_SUFFIX = {"backward": "_backward", "decay": "_decay", "decay_backward": "_decay_backward", "log": "_log"}
 
 
 def plan_kernel(plan) -> str:
@@ -727,6 +727,19 @@ def run_b200(args):
         ws = wsb
         args.no_e2e = True
     profile_key = w.name
+    if args.pass_ == "log":
+        # the same scan evaluated in log space (mingru_scan_log), for the
+        # comparison of evaluation domains
+        if w.op != "mingru":
+            raise SystemExit("bench.py: the log-space evaluation is a minGRU form")
+        wsl = sgr.Workspace(sgr.workspace_size("mingru_log", w.B, w.T, w.D, p.dtype), device)
+        fn = lambda: sgr.mingru_scan_log(p, q, init, out=out, workspace=wsl)  # noqa: E731
+        kernel_name = plan_kernel(sgr._abi.plan(sgr._abi.SGR_OP_MINGRU_LOG, w.B, w.T, w.D,
+                                                0 if w.dtype == "f32" else 1, True))
+        kernel_name = "sgr::scan_kernel" if "sequential" not in kernel_name else kernel_name
+        profile_key = w.name.replace("mingru_", "mingru_log_", 1)
+        ws = wsl
+        args.no_e2e = True
     if args.pass_ in ("decay", "decay_backward"):
         # the time-decayed minGRU on the workload: gaps ~ Exp(1) per (b, t),
         # rates ~ U(0, 1) per channel, fp32 (the decay rows' recipe)
@@ -941,10 +954,10 @@ def main(argv=None):
     ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--pass", dest="pass_", default="forward",
-                    choices=["forward", "backward", "decay", "decay_backward", "projected"],
+                    choices=["forward", "backward", "decay", "decay_backward", "projected", "log"],
                     help="time the scan (default), its gradient kernel on the workload, the time-decayed "
-                         "minGRU or its gradient on the workload, or the input projection fused with the "
-                         "scan (B8 T4096 D1024 d_in 1024)")
+                         "minGRU or its gradient on the workload, the input projection fused with the "
+                         "scan (B8 T4096 D1024 d_in 1024), or the minGRU scan evaluated in log space")
     ap.add_argument("--no-rows", action="store_true", help="skip the other hot-path rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")

@@ -229,9 +229,11 @@ SeqLayout seq_pair_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm
 // per-tile work dominates and the longer tiles of 15-warp blocks pay wherever
 // they still give every SM 4 tiles (measured: MinMax B4 x 8192 x 768 fp32 0.81
 // of the copy bandwidth against 0.78 with 7-warp blocks; minGRU slower).
-// decay: the time-decayed minGRU, whose extra gate per element favours 4
-// rows per thread in the pipelined kernel (bf16 with 15-warp blocks); wide
-// decayed batches take the channel-sequential kernels like the plain scan
+// decay: the time-decayed minGRU, which takes the plain scan's plans (bf16:
+// 8 rows per thread in 7-warp blocks, measured 78.3 against 82.4 us with 4
+// rows in 15-warp blocks on B8 x 4096 x 1024, 41.5 against 45.5 us on B2 x
+// 2048 x 4096, 47.5 against 47.7 us on B4 x 8192 x 512); wide decayed
+// batches take the channel-sequential kernels like the plain scan
 // (each slot's gaps arrive with it through the copy engine, or, for gap
 // arrays the copy engine cannot address, spread across the lanes two slots
 // ahead)
@@ -306,7 +308,7 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
         // elements are half the bytes, so per-tile work (warp scan, barriers,
         // hand-off) weighs twice as much per byte and is spread over twice
         // the rows (replayed without the one-tile lag, see the kernel)
-        p.r = (orr == 2 || orr == 4 || orr == 8) ? orr : (p.esz == 2 && !decay ? 8 : 4);
+        p.r = (orr == 2 || orr == 4 || orr == 8) ? orr : (p.esz == 2 ? 8 : 4);
         p.stages = kStages;
         // Block shape: about (blocks in flight) / n_chains chunks of one
         // channel tile are processed at once and a look-back folds that many
@@ -316,7 +318,7 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
         const int64_t n_chains = B * ((D + p.TC - 1) / p.TC);
         const int64_t tr_wide = int64_t(kPipeWarpsWide) * (32 / p.cg) * p.r;
         const int64_t tiles_wide = n_chains * ((T + tr_wide - 1) / tr_wide);
-        bool wide = n_chains > 0 && (light_op || (decay && p.esz == 2) || 2 * kAssumedSMs >= 8 * n_chains) &&
+        bool wide = n_chains > 0 && (light_op || 2 * kAssumedSMs >= 8 * n_chains) &&
                     tiles_wide >= 4 * kAssumedSMs;
         if (ok == KIND_PIPELINED) wide = false;
         if (ok == KIND_PIPELINED_WIDE) wide = true;

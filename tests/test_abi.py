@@ -120,20 +120,20 @@ def test_step_argument_errors():
 
 
 def test_decayed_plan():
-    # wide batches: the channel-sequential kernel the plain scan takes;
-    # otherwise 4 rows per thread, bf16 with the 15-warp blocks wherever their
-    # tiles still give every SM 4 of them
+    # the decayed scan takes the plain scan's plan: wide batches the
+    # channel-sequential kernel, otherwise the pipelined kernel with the
+    # plain scan's rows per thread (4 fp32, 8 bf16) and block shape
     for B, T, D, dtype in ((16, 2048, 2048, F32), (24, 2048, 2048, BF16)):
         plain = _abi.plan(MINGRU, B, T, D, dtype, True)
         pl = _abi.plan(MINGRU, B, T, D, dtype, True, decay=True)
         assert pl["kernel"] == plain["kernel"] and pl["kernel"] in SEQ_KINDS, (B, T, D, dtype)
         assert pl["workspace_bytes"] == WS_HEADER
     for B, T, D, dtype in ((8, 4096, 1024, BF16), (8, 4096, 1024, F32), (4, 8192, 512, BF16)):
+        plain = _abi.plan(MINGRU, B, T, D, dtype, True)
         pl = _abi.plan(MINGRU, B, T, D, dtype, True, decay=True)
         assert pl["kernel"] in (_abi.KERNEL_PIPELINED, _abi.KERNEL_PIPELINED_WIDE), (B, T, D, dtype)
-        assert pl["rows_per_thread"] == 4
-        if dtype == BF16:
-            assert pl["kernel"] == _abi.KERNEL_PIPELINED_WIDE and pl["warps"] == 15
+        assert pl["rows_per_thread"] == (4 if dtype == F32 else 8)
+        assert (pl["kernel"], pl["warps"], pl["tile_rows"]) == (plain["kernel"], plain["warps"], plain["tile_rows"])
         assert pl["workspace_bytes"] <= _abi.lib().sgr_workspace_size(MINGRU, B, T, D, dtype)
     # small shapes: one launch per tile, as for the plain scan
     assert _abi.plan(MINGRU, 2, 1024, 512, F32, True, decay=True)["kernel"] == _abi.KERNEL_TILE
