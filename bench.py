@@ -58,6 +58,7 @@ KERNEL_SOURCES = {
     "scan_kernel": [_ENGINE],
     "scan_sequential_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_sequential.cuh"],
     "scan_sequential_pair_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_sequential.cuh"],
+    "scan_sequential_pair2_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_sequential.cuh"],
     "scan_sequential_backward_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_backward.cuh",
                                         "scan_gated_rnns_b200/csrc/scan_sequential.cuh"],
     "scan_backward_kernel": [_ENGINE, "scan_gated_rnns_b200/csrc/scan_backward.cuh"],
@@ -295,7 +296,8 @@ def plan_kernel(plan) -> str:
     """The device kernel a scan plan launches (the library's kernel kinds)."""
     return {1: "sgr::scan_tile_kernel", 2: "sgr::scan_pipelined_kernel", 3: "sgr::scan_pipelined_kernel",
             4: "sgr::scan_sequential_kernel", 5: "sgr::scan_sequential_kernel (split rows)",
-            6: "sgr::scan_sequential_pair_kernel"}.get(plan["kernel"], "sgr::scan_kernel")
+            6: "sgr::scan_sequential_pair_kernel",
+            7: "sgr::scan_sequential_pair2_kernel"}.get(plan["kernel"], "sgr::scan_kernel")
 
 
 def profile_kernel(plan) -> str:
@@ -305,6 +307,8 @@ def profile_kernel(plan) -> str:
         return "sgr::scan_sequential_kernel"
     if plan["kernel"] == 6:
         return "sgr::scan_sequential_pair_kernel"
+    if plan["kernel"] == 7:
+        return "sgr::scan_sequential_pair2_kernel"
     return "sgr::scan_kernel"
 
 

@@ -476,14 +476,16 @@ SGR_API sgr_status_t sgr_set_tile_override(int channel_lanes, int rows_per_threa
  * Tuning/testing knob, process-wide: 0 automatic (for aligned vector-width
  * rows: a channel-sequential kernel when the 32-channel groups B x ceil(D / 32)
  * reach 6 per SM -- two warps per group below 24 (bf16) or 32 (fp32) groups
- * per SM, one warp per group above -- the pipelined kernel otherwise; the tile
+ * per SM, above that one warp per group (fp32) or two warps per group of 64
+ * channels (bf16) -- the pipelined kernel otherwise; the tile
  * kernel for anything else), 1 force the tile kernel, 2 pipelined with 7 data
  * warps per block (two blocks per SM), 3 pipelined with 15 data warps (one
  * block per SM, tiles twice as long), 4 channel-sequential with one warp per
  * group of 32 channels walking the whole sequence, 5 channel-sequential with
  * each slot's 16 rows split between the two half-warps of a warp (groups of
  * 16 channels), 6 channel-sequential with two warps per group of 32 channels
- * splitting each 32-row slot; 2-6 wherever the fast path applies.
+ * splitting each 32-row slot, 7 the same with groups of 64 channels, two
+ * per lane (bf16 I/O; fp32 takes 6); 2-7 wherever the fast path applies.
  */
 SGR_API sgr_status_t sgr_set_kernel_override(int kernel);
 
@@ -500,7 +502,9 @@ typedef struct sgr_plan {
                                    5: the same with 16-channel groups, the rows
                                    of each slot split between half-warps;
                                    6: two warps per 32-channel group, each slot
-                                   of 32 rows split between them                */
+                                   of 32 rows split between them; 7: the same
+                                   with 64-channel groups, two channels per
+                                   lane (bf16)                                  */
     int32_t channels_per_thread;
     int32_t channel_lanes;      /* lanes across D per warp                         */
     int32_t rows_per_thread;

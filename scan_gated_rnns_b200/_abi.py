@@ -97,6 +97,7 @@ KERNEL_PIPELINED_WIDE = 3
 KERNEL_SEQUENTIAL = 4
 KERNEL_SEQUENTIAL_SPLIT = 5
 KERNEL_SEQUENTIAL_PAIR = 6
+KERNEL_SEQUENTIAL_PAIR2 = 7
 
 _lock = threading.Lock()
 _lib = None

@@ -487,6 +487,206 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
     if (lane == 0) bulk_wait_all();
 }
 
+// The two-warp kernel with two channels per lane (bf16 I/O): a block scans a
+// group of 64 channels of one batch row, lane l owning channels 2l and
+// 2l + 1, so each operand row of a warp is one 128-byte segment read as one
+// 32-bit shared load per lane, and each output row is written as one packed
+// bf16 pair.  Everything else follows scan_sequential_pair_kernel: warp w
+// takes rows [32 i + 16 w, 32 i + 16 w + 16) of slot i through its own ring,
+// folds them -- here four chains per lane (two channels x rows r and r + 8),
+// advanced as two fp32x2 operations per row pair -- exchanges its two pairs
+// with the other warp after one named barrier per slot, and writes each row
+// as its chain's running composite applied to the chain's incoming state.
+// The channel pair doubles each warp's independent work while the batch
+// provides half the warps.
+constexpr int kPair2Channels = 64;
+__host__ __device__ constexpr size_t seq_pair2_block_bytes(int S, size_t gap = 0) {
+    return kPairWarps * seq_pair_warp_bytes(S, kPair2Channels * 2, gap) + size_t(2) * kPairWarps * 32 * sizeof(float4);
+}
+
+// two bf16 channels of one row: (low, high) halves as fp32
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void sts_bf16x2(uint32_t a, float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(a), "r"(*reinterpret_cast<const uint32_t *>(&h)) : "memory");
+}
+
+template <class Op, bool DT = false>
+__global__ void __launch_bounds__(kPairWarps * 32)
+scan_sequential_pair2_kernel(const SeqParams q, const __grid_constant__ CUtensorMap map0,
+                             const __grid_constant__ CUtensorMap map1, const __grid_constant__ CUtensorMap map_out,
+                             const __grid_constant__ CUtensorMap map_gap) {
+    static_assert(!DT || Op::kDecay, "gaps through the copy engine need a decay operator");
+    static_assert(!Op::kLogSpace, "the channel-sequential kernels carry linear states");
+    using IO = __nv_bfloat16;
+    constexpr uint32_t kGap = DT ? kSeqGapBytes : 0;
+    constexpr int CW = kPair2Channels;
+    constexpr int kRowBytes = CW * int(sizeof(IO));                 // 128
+    constexpr uint32_t kOpBytes = kSeqRows * kRowBytes;             // one operand of a warp's 16 rows
+    constexpr int kSlotRows = kPairWarps * kSeqRows;
+    constexpr int H = kSeqRows / 2;
+    const ScanParams &p = q.s;
+    extern __shared__ __align__(128) unsigned char smem[];
+
+    const int lane = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5;
+    const int64_t gw = blockIdx.x;
+    if (gw >= q.n_warps) return;
+    const int S = q.slots;
+    const int64_t b = gw / q.n_groups;
+    const int64_t grp = gw - b * q.n_groups;
+    const int x0 = int(grp) * CW;
+    const int64_t d = int64_t(x0) + 2 * lane;                       // the lane's first channel
+
+    constexpr uint32_t kSlot = 2 * kOpBytes + kGap;
+    const uint32_t base = smem_addr(smem) + uint32_t(w * seq_pair_warp_bytes(S, kRowBytes, kGap));
+    const uint32_t ring = base;
+    const uint32_t outb = base + uint32_t(S) * kSlot;
+    const uint32_t bars = outb + kOpBytes;
+    float4 *xpair = reinterpret_cast<float4 *>(smem + kPairWarps * seq_pair_warp_bytes(S, kRowBytes, kGap));  // [2][2][32]
+
+    const int n_slots = int((p.T + kSlotRows - 1) / kSlotRows);
+    auto issue = [&](int i, int s) {
+        const uint32_t dst = ring + uint32_t(s) * kSlot;
+        const uint32_t bar = bars + 8u * uint32_t(s);
+        const int y = i * kSlotRows + w * kSeqRows;
+        mbar_expect_tx(bar, 2 * kOpBytes + (DT ? kSeqRows * 4 : 0));
+        tma_load_3d(dst, &map0, x0, y, int(b), bar);
+        tma_load_3d(dst + kOpBytes, &map1, x0, y, int(b), bar);
+        if constexpr (DT) tma_load_2d(dst + 2 * kOpBytes, &map_gap, y, int(b), bar);
+    };
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(bars + 8u * s, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int s = 0; s < S && s < n_slots; ++s) issue(s, s);
+    }
+    __syncwarp();
+
+    // states entering the slot (channels d, d + 1; past D: the default)
+    float2 h = make_float2(load_init<IO>(p, b, d, Op::default_init()), load_init<IO>(p, b, d + 1, Op::default_init()));
+    [[maybe_unused]] float2 lam2 = make_float2(0.f, 0.f);
+    [[maybe_unused]] float gcur = 0.f, gnext = 0.f;
+    if constexpr (Op::kDecay) {
+        lam2 = make_float2(d < p.D ? decay_lam2(p, d) : 0.f, d + 1 < p.D ? decay_lam2(p, d + 1) : 0.f);
+        if constexpr (!DT) {
+            gcur = seq_slot_gap(p, b, w * kSeqRows, lane);
+            gnext = seq_slot_gap(p, b, kSlotRows + w * kSeqRows, lane);
+        }
+    }
+
+    uint32_t wait_limit = kMbarLimit;
+    bool bad = false;
+    int s = 0;
+    uint32_t phase = 0;
+    for (int i = 0; i < n_slots; ++i) {
+        [[maybe_unused]] float gnext2 = 0.f;
+        if constexpr (Op::kDecay && !DT)
+            gnext2 = seq_slot_gap(p, b, int64_t(i + 2) * kSlotRows + w * kSeqRows, lane);
+        if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
+            wait_limit = 1;
+            if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
+            bad = true;
+        }
+        const uint32_t src = ring + uint32_t(s) * kSlot + uint32_t(lane) * 4u;
+        uint32_t x0r[kSeqRows], x1r[kSeqRows];
+#pragma unroll
+        for (int r = 0; r < kSeqRows; ++r) {
+            x0r[r] = lds32(src + r * kRowBytes);
+            x1r[r] = lds32(src + kOpBytes + r * kRowBytes);
+        }
+        if constexpr (DT) gcur = seq_smem_gap(p, ring + uint32_t(s) * kSlot + 2 * kOpBytes, lane);
+        __syncwarp();                                                // the slot is in registers
+        if (lane == 0 && !bad && i + S < n_slots) {
+            fence_proxy_async();
+            issue(i + S, s);
+        }
+        if (++s == S) {
+            s = 0;
+            phase ^= 1u;
+        }
+        bad = __any_sync(0xffffffffu, bad);
+        // four chains: (channels d, d + 1) x (rows r, r + 8); L = rows 0-7,
+        // U = rows 8-15, each an fp32x2 over the two channels
+        float2 PAL[H], PBL[H], PAU[H], PBU[H];
+        float2 AL = make_float2(Op::identity().x, Op::identity().x), BL = make_float2(Op::identity().y, Op::identity().y);
+        float2 AU = AL, BU = BL;
+#pragma unroll
+        for (int r = 0; r < H; ++r) {
+            const float2 kl = unpack_bf16x2(x0r[r]), hl = unpack_bf16x2(x1r[r]);
+            const float2 ku = unpack_bf16x2(x0r[r + H]), hu = unpack_bf16x2(x1r[r + H]);
+            float2 al, cl, au, cu;
+            seq_rows<Op, IO>(kl.x, hl.x, kl.y, hl.y, al, cl);
+            seq_rows<Op, IO>(ku.x, hu.x, ku.y, hu.y, au, cu);
+            if constexpr (Op::kDecay) {
+                const float ul = __shfl_sync(0xffffffffu, gcur, r), uu = __shfl_sync(0xffffffffu, gcur, r + H);
+                al = __fmul2_rn(al, make_float2(decay_gamma(lam2.x, ul), decay_gamma(lam2.y, ul)));
+                au = __fmul2_rn(au, make_float2(decay_gamma(lam2.x, uu), decay_gamma(lam2.y, uu)));
+            }
+            Op::fold2(AL, BL, al, cl);
+            Op::fold2(AU, BU, au, cu);
+            PAL[r] = AL;
+            PBL[r] = BL;
+            PAU[r] = AU;
+            PBU[r] = BU;
+        }
+        // the warp's 16 rows per channel: the first chain, then the second
+        float4 P;
+        {
+            const float2 p0 = Op::combine(make_float2(AL.x, BL.x), make_float2(AU.x, BU.x));
+            const float2 p1 = Op::combine(make_float2(AL.y, BL.y), make_float2(AU.y, BU.y));
+            P = make_float4(p0.x, p0.y, p1.x, p1.y);
+        }
+        if (bad) P = make_float4(__int_as_float(0x7fffffff), __int_as_float(0x7fffffff), __int_as_float(0x7fffffff),
+                                 __int_as_float(0x7fffffff));
+        float4 *xb = xpair + (i & 1) * kPairWarps * 32;
+        xb[w * 32 + lane] = P;
+        named_barrier_sync(1, kPairWarps * 32);
+        const float4 Q = xb[(1 - w) * 32 + lane];
+        const float4 F = w ? Q : P, L = w ? P : Q;                  // first and second half of the slot
+        const float2 hmid = make_float2(Op::apply(make_float2(F.x, F.y), h.x), Op::apply(make_float2(F.z, F.w), h.y));
+        const float2 hend =
+            make_float2(Op::apply(make_float2(L.x, L.y), hmid.x), Op::apply(make_float2(L.z, L.w), hmid.y));
+        const float2 hin = w ? hmid : h;
+        h = hend;
+        // incoming states of the upper chains: after row 7 of each channel
+        float2 hu = make_float2(Op::apply(make_float2(AL.x, BL.x), hin.x), Op::apply(make_float2(AL.y, BL.y), hin.y));
+        float2 hl = hin;
+        if (bad) {
+            hl = make_float2(__int_as_float(0x7fffffff), __int_as_float(0x7fffffff));
+            hu = hl;
+        }
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        const uint32_t dst = outb + uint32_t(lane) * 4u;
+#pragma unroll
+        for (int r = 0; r < H; ++r) {
+            const float2 yl = Op::step2(PAL[r], PBL[r], hl);
+            const float2 yu = Op::step2(PAU[r], PBU[r], hu);
+            sts_bf16x2(dst + r * kRowBytes, yl.x, yl.y);
+            sts_bf16x2(dst + (r + H) * kRowBytes, yu.x, yu.y);
+        }
+        fence_proxy_async();
+        __syncwarp();
+        const int y0 = i * kSlotRows + w * kSeqRows;
+        if (lane == 0 && y0 < p.T) {
+            tma_store_3d(&map_out, outb, x0, y0, int(b));
+            bulk_commit();
+        }
+        if constexpr (Op::kDecay && !DT) {
+            gcur = gnext;
+            gnext = gnext2;
+        }
+    }
+    if (lane == 0) bulk_wait_all();
+}
+
 }  // namespace sgr
 
 // ------------------------------------------------------- gradients

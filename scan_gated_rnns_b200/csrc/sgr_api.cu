@@ -38,7 +38,10 @@ constexpr size_t kAlign = 256;
 constexpr size_t kTicketOffset = 64;
 
 enum Kind { KIND_AUTO = 0, KIND_TILE = 1, KIND_PIPELINED = 2, KIND_PIPELINED_WIDE = 3, KIND_SEQUENTIAL = 4,
-            KIND_SEQUENTIAL_SPLIT = 5, KIND_SEQUENTIAL_PAIR = 6 };
+            KIND_SEQUENTIAL_SPLIT = 5, KIND_SEQUENTIAL_PAIR = 6, KIND_SEQUENTIAL_PAIR2 = 7 };
+bool seq_kind(int k) {
+    return k == KIND_SEQUENTIAL || k == KIND_SEQUENTIAL_SPLIT || k == KIND_SEQUENTIAL_PAIR || k == KIND_SEQUENTIAL_PAIR2;
+}
 
 // Channel-sequential kernels (scan_sequential.cuh): each 32-channel group's
 // whole sequence is walked by one warp or by a block of two warps.  Chosen
@@ -59,6 +62,12 @@ constexpr int kSeqMinWarpsPerSMHalf = 6;
 // 0.81 / 0.84, 13.8: 0.84 / 0.86, and D 4096 at 27.7: 0.85 / 0.87.
 constexpr int kSeqPairBelow = 32;
 constexpr int kSeqPairBelowHalf = 24;
+// From kSeqPairBelowHalf groups per SM, bf16 takes two warps per group of 64
+// channels, two channels per lane (scan_sequential_pair2_kernel): the same
+// warps as one per 32-channel group, fewer instructions per element.  Measured
+// (us, one warp per 32 / two per 32 / two per 64 channels): B32 x 2048 x 4096
+// (27.7 groups per SM) 301.6 / 315.9 / 289.2; below, the 32-channel pairs
+// win: B24 (20.8) 248.3 / 238.1 / 250.4, B16 (13.8) 162.3 / 158.2 / 172.5.
 // The gradient (four operands in, two out per element) walks whole sequences
 // from 5 warps per SM: against the pipelined gradient it loses at 3.5 groups
 // per SM (bf16 B4 x 2048 x 4096 150 us against 101 us; fp32 B8 x 2048 x 2048
@@ -202,20 +211,22 @@ SeqLayout seq_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, siz
 
 // the two-warp blocks of scan_sequential_pair_kernel: one block per channel
 // group, the block's share of the SM's shared memory split between its warps
+// wide: the two-channels-per-lane form (64-channel groups, float4 exchange)
 SeqLayout seq_pair_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, size_t reserved,
-                          size_t smem_block_max, size_t gap = 0) {
+                          size_t smem_block_max, size_t gap = 0, bool wide = false) {
+    auto bytes = [&](int S) { return wide ? seq_pair2_block_bytes(S, gap) : seq_pair_block_bytes(S, row_bytes, gap); };
     SeqLayout l;
     const int64_t K = sms > 0 ? (groups + sms - 1) / sms : 1;
-    size_t alloc = seq_pair_block_bytes(4, row_bytes, gap);
+    size_t alloc = bytes(4);
     if (K >= 1 && K <= 16) {
         const size_t share = smem_sm / size_t(K);
         alloc = share > reserved ? (share - reserved) / 128 * 128 : 0;
     }
     alloc = std::min(alloc, smem_block_max);
     int S = kSeqMaxSlots;
-    while (S > kSeqMinSlots && seq_pair_block_bytes(S, row_bytes, gap) > alloc) --S;
+    while (S > kSeqMinSlots && bytes(S) > alloc) --S;
     l.slots = S;
-    l.smem = std::max(alloc, seq_pair_block_bytes(S, row_bytes, gap));
+    l.smem = std::max(alloc, bytes(S));
     return l;
 }
 
@@ -254,24 +265,29 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
         const bool seq_ok = p.vec && !force_tile && !chunked_only && T <= int64_t(std::numeric_limits<int>::max()) &&
                             B <= int64_t(std::numeric_limits<int>::max());
         const int min_per_sm = p.esz == 2 ? kSeqMinWarpsPerSMHalf : kSeqMinWarpsPerSM;
-        const bool want = ok == KIND_SEQUENTIAL || ok == KIND_SEQUENTIAL_SPLIT || ok == KIND_SEQUENTIAL_PAIR ||
-                          (ok == KIND_AUTO && groups >= int64_t(min_per_sm) * kAssumedSMs);
+        const bool want = seq_kind(ok) || (ok == KIND_AUTO && groups >= int64_t(min_per_sm) * kAssumedSMs);
         if (seq_ok && want) {
             const bool split = ok == KIND_SEQUENTIAL_SPLIT;
             const int pair_below = p.esz == 2 ? kSeqPairBelowHalf : kSeqPairBelow;
-            const bool pair = ok == KIND_SEQUENTIAL_PAIR ||
+            // two channels per lane: bf16 only; automatic from kSeqPairBelowHalf
+            // groups per SM, where it keeps the one-warp kernel's warp count
+            // with fewer instructions and 128-byte rows
+            const bool wide = p.esz == 2 && (ok == KIND_SEQUENTIAL_PAIR2 ||
+                                             (ok == KIND_AUTO && groups >= int64_t(pair_below) * kAssumedSMs));
+            const bool pair = wide || ok == KIND_SEQUENTIAL_PAIR || ok == KIND_SEQUENTIAL_PAIR2 ||
                               (ok == KIND_AUTO && groups < int64_t(pair_below) * kAssumedSMs);
-            const int64_t gw = split ? cw / 2 : cw;                 // channels per warp
+            const int64_t gw = wide ? int64_t(kPair2Channels) : split ? cw / 2 : cw;   // channels per warp
             const int64_t n_warps = B * ((D + gw - 1) / gw);
             const size_t gap = decay ? kSeqGapBytes : 0;
             const SeqLayout lay = pair ? seq_pair_layout(n_warps, int(gw) * p.esz, kAssumedSMs, kAssumedSmemPerSM,
-                                                         kAssumedSmemReserved, kAssumedSmemPerBlock, gap)
+                                                         kAssumedSmemReserved, kAssumedSmemPerBlock, gap, wide)
                                        : seq_layout(n_warps, int(gw) * p.esz, kAssumedSMs, kAssumedSmemPerSM,
                                                     kAssumedSmemReserved, kAssumedSmemPerBlock, SEQ_SCAN, gap);
-            p.kind = pair ? KIND_SEQUENTIAL_PAIR : split ? KIND_SEQUENTIAL_SPLIT : KIND_SEQUENTIAL;
+            p.kind = wide ? KIND_SEQUENTIAL_PAIR2 : pair ? KIND_SEQUENTIAL_PAIR : split ? KIND_SEQUENTIAL_SPLIT
+                                                                                         : KIND_SEQUENTIAL;
             p.split = (split || pair) ? 2 : 1;
-            p.V = 1;
-            p.cg = int(gw);
+            p.V = wide ? 2 : 1;
+            p.cg = int(gw / p.V);                                  // lanes across a group's channels
             p.r = pair ? kSeqRows : kSeqRows / p.split;            // rows of a slot per lane
             p.stages = lay.slots;
             p.warps = pair ? kPairWarps : kSeqWarpsPerBlock;
@@ -702,6 +718,41 @@ cudaError_t launch_sequential_pair(const Plan &pl, const ScanParams &sp, cudaStr
     return launch_sequential_pair_dt<Op, IO, false>(pl, sp, map0, map1, map_out, map0, s);
 }
 
+template <class Op, bool DT>
+cudaError_t launch_sequential_pair2_dt(const Plan &pl, const ScanParams &sp, const CUtensorMap &map0,
+                                       const CUtensorMap &map1, const CUtensorMap &map_out,
+                                       const CUtensorMap &map_gap, cudaStream_t s) {
+    constexpr size_t kGap = DT ? kSeqGapBytes : 0;
+    auto kernel = scan_sequential_pair2_kernel<Op, DT>;
+    SeqDev d;
+    cudaError_t e = seq_device(reinterpret_cast<const void *>(kernel), seq_pair2_block_bytes(kSeqMinSlots, kGap), &d);
+    if (e != cudaSuccess) return e;
+    SeqParams q;
+    q.s = sp;
+    q.n_groups = pl.n_dt;
+    q.n_warps = pl.n_chains;                  // channel groups: one block each
+    const SeqLayout lay = seq_pair_layout(q.n_warps, kPair2Channels * 2, d.sms, size_t(d.smem_sm), size_t(d.reserved),
+                                          size_t(d.smem_block), kGap, true);
+    q.slots = lay.slots;
+    kernel<<<dim3(unsigned(q.n_warps)), kPairWarps * 32, lay.smem, s>>>(q, map0, map1, map_out, map_gap);
+    return cudaGetLastError();
+}
+
+template <class Op>
+cudaError_t launch_sequential_pair2(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
+    constexpr int CW = kPair2Channels;
+    alignas(64) CUtensorMap map0, map1, map_out, map_gap;
+    if (!make_operand_map(&map0, sp.in0, sp.B, sp.T, sp.D, 2, CW, kSeqRows) ||
+        !make_operand_map(&map1, sp.in1, sp.B, sp.T, sp.D, 2, CW, kSeqRows) ||
+        !make_operand_map(&map_out, sp.out, sp.B, sp.T, sp.D, 2, CW, kSeqRows))
+        return cudaErrorInvalidValue;
+    if constexpr (Op::kDecay) {
+        if (make_seq_gap_map(&map_gap, sp))
+            return launch_sequential_pair2_dt<Op, true>(pl, sp, map0, map1, map_out, map_gap, s);
+    }
+    return launch_sequential_pair2_dt<Op, false>(pl, sp, map0, map1, map_out, map0, s);
+}
+
 template <class Op, typename IO>
 cudaError_t dispatch(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
     constexpr int VW = 16 / int(sizeof(IO));
@@ -709,9 +760,12 @@ cudaError_t dispatch(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
         if (pl.kind == KIND_SEQUENTIAL) return launch_sequential<Op, IO, 1>(pl, sp, s);
         if (pl.kind == KIND_SEQUENTIAL_SPLIT) return launch_sequential<Op, IO, 2>(pl, sp, s);
         if (pl.kind == KIND_SEQUENTIAL_PAIR) return launch_sequential_pair<Op, IO>(pl, sp, s);
+        if (pl.kind == KIND_SEQUENTIAL_PAIR2) {
+            if constexpr (sizeof(IO) == 2) return launch_sequential_pair2<Op>(pl, sp, s);
+            else return cudaErrorInvalidConfiguration;   // never planned (bf16 only)
+        }
     } else {
-        if (pl.kind == KIND_SEQUENTIAL || pl.kind == KIND_SEQUENTIAL_SPLIT || pl.kind == KIND_SEQUENTIAL_PAIR)
-            return cudaErrorInvalidConfiguration;    // never planned (chunked_only)
+        if (seq_kind(pl.kind)) return cudaErrorInvalidConfiguration;    // never planned (chunked_only)
     }
     if (pl.kind == KIND_PIPELINED) {
         if constexpr (sizeof(IO) == 2) {
@@ -932,7 +986,7 @@ bool seq_backward_planned(int64_t B, int64_t T, int64_t D, int esz, bool aligned
         B > int64_t(std::numeric_limits<int>::max()))
         return false;
     const int ok = g_override_kind.load();
-    if (ok == KIND_SEQUENTIAL || ok == KIND_SEQUENTIAL_SPLIT || ok == KIND_SEQUENTIAL_PAIR) return true;
+    if (seq_kind(ok)) return true;
     if (ok != KIND_AUTO) return false;
     const int64_t groups = B * ((D + 31) / 32);
     return groups >= int64_t(kSeqBwdMinWarpsPerSM) * kAssumedSMs;
@@ -1708,7 +1762,7 @@ void fill_plan(const Plan &p, sgr_plan_t *plan) {
     plan->channel_lanes = p.cg;
     plan->rows_per_thread = p.r;
     plan->warps = p.warps;
-    const bool seq = p.kind == KIND_SEQUENTIAL || p.kind == KIND_SEQUENTIAL_SPLIT || p.kind == KIND_SEQUENTIAL_PAIR;
+    const bool seq = seq_kind(p.kind);
     plan->threads = (seq ? plan->warps : plan->warps + 1) * 32;
     plan->stages = p.stages;
     plan->tile_rows = p.TR;
@@ -1768,7 +1822,7 @@ sgr_status_t sgr_set_drop_publish(int64_t tile) {
 }
 
 sgr_status_t sgr_set_kernel_override(int kernel) {
-    if (kernel < KIND_AUTO || kernel > KIND_SEQUENTIAL_PAIR) return SGR_ERR_INVALID_ARG;
+    if (kernel < KIND_AUTO || kernel > KIND_SEQUENTIAL_PAIR2) return SGR_ERR_INVALID_ARG;
     g_override_kind.store(kernel);
     return SGR_OK;
 }

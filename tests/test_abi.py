@@ -166,7 +166,7 @@ def test_workspace_size_and_hooks():
     assert lib.sgr_set_tile_override(3, 0) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_tile_override(0, 3) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_drop_publish(-2) == _abi.SGR_ERR_INVALID_ARG
-    assert lib.sgr_set_kernel_override(7) == _abi.SGR_ERR_INVALID_ARG
+    assert lib.sgr_set_kernel_override(8) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_kernel_override(_abi.KERNEL_SEQUENTIAL_SPLIT) == _abi.SGR_OK
     assert lib.sgr_set_kernel_override(0) == _abi.SGR_OK
     assert lib.sgr_set_wait_limit(0) == _abi.SGR_OK
@@ -180,7 +180,8 @@ def test_workspace_size_and_hooks():
 # The kernel's address formulas, replayed for every block and thread.
 
 SEQ_ROWS = 16            # rows per load slot of the channel-sequential kernel
-SEQ_KINDS = (_abi.KERNEL_SEQUENTIAL, _abi.KERNEL_SEQUENTIAL_SPLIT, _abi.KERNEL_SEQUENTIAL_PAIR)
+SEQ_KINDS = (_abi.KERNEL_SEQUENTIAL, _abi.KERNEL_SEQUENTIAL_SPLIT, _abi.KERNEL_SEQUENTIAL_PAIR,
+             _abi.KERNEL_SEQUENTIAL_PAIR2)
 WS_HEADER = 256          # workspace header: status word at 0, chunk ticket at 64
 
 
@@ -192,21 +193,32 @@ def check_sequential_indices(pl, B, T, D, esz, check_cover):
     rows; lane l owns channel l % CW of the slot rows
     [(l // CW) R, (l // CW) R + R), R = 16 CW / 32.  With two warps per group
     (kernel 6) a block's warps w = 0, 1 take rows [32 i + 16 w, 32 i + 16 w + 16)
-    of slot i, lane l channel l."""
+    of slot i, lane l channel l.  Kernel 7 (bf16): the same with groups of 64
+    channels, lane l owning channels 2 l and 2 l + 1 (one 32-bit word of a
+    128-byte row)."""
     V, CW = pl["channels_per_thread"], pl["tile_channels"]
-    pair = pl["kernel"] == _abi.KERNEL_SEQUENTIAL_PAIR
+    pair2 = pl["kernel"] == _abi.KERNEL_SEQUENTIAL_PAIR2
+    pair = pl["kernel"] == _abi.KERNEL_SEQUENTIAL_PAIR or pair2
     split = 2 if pl["kernel"] == _abi.KERNEL_SEQUENTIAL_SPLIT else 1
     rb = CW * esz                                       # bytes of one operand row of a group
-    assert pl["vector_path"] and V == 1 and CW == 32 // split and rb in (32, 64, 128)
-    assert pl["channel_lanes"] == CW and pl["threads"] == 32 * pl["warps"]
+    if pair2:
+        assert esz == 2 and V == 2 and CW == 64 and rb == 128
+    else:
+        assert V == 1 and CW == 32 // split and rb in (32, 64, 128)
+    assert pl["vector_path"] and pl["channel_lanes"] * V == CW and pl["threads"] == 32 * pl["warps"]
     assert pl["warps"] == (2 if pair else 1)
     assert pl["rows_per_thread"] == SEQ_ROWS // split
     assert pl["n_chunks"] == 1 and pl["workspace_bytes"] == WS_HEADER and pl["tile_rows"] == T
     # a lane's elements of a slot stay inside its warp's 16 rows of CW channels
     lane = np.arange(32)
-    off = (lane // CW) * pl["rows_per_thread"] * rb + (lane % CW) * esz
-    assert (off + (pl["rows_per_thread"] - 1) * rb + esz <= SEQ_ROWS * rb).all()
-    assert len(set(zip(lane % CW, lane // CW))) == 32   # no two lanes share an element
+    if pair2:
+        off = lane * 4                                  # channels 2 l, 2 l + 1: one 32-bit word
+        assert (off + (SEQ_ROWS - 1) * rb + 4 <= SEQ_ROWS * rb).all() and (off % 4 == 0).all()
+        assert len(set(off.tolist())) == 32
+    else:
+        off = (lane // CW) * pl["rows_per_thread"] * rb + (lane % CW) * esz
+        assert (off + (pl["rows_per_thread"] - 1) * rb + esz <= SEQ_ROWS * rb).all()
+        assert len(set(zip(lane % CW, lane // CW))) == 32   # no two lanes share an element
     n_groups = -(-D // CW)
     assert pl["n_channel_tiles"] == n_groups and pl["n_chains"] == B * n_groups
     assert pl["n_tiles"] == pl["n_chains"] < 2 ** 31
@@ -215,7 +227,7 @@ def check_sequential_indices(pl, B, T, D, esz, check_cover):
     S = pl["stages"]
     if pair:
         warp_bytes = -(-(S * 2 * SEQ_ROWS * rb + SEQ_ROWS * rb + S * 8) // 128) * 128
-        block_bytes = 2 * warp_bytes + 2 * 2 * 32 * 8      # + the pairs exchanged per slot
+        block_bytes = 2 * warp_bytes + 2 * 2 * 32 * (16 if pair2 else 8)   # + the pairs exchanged per slot
     else:
         block_bytes = -(-(S * 2 * SEQ_ROWS * rb + 2 * SEQ_ROWS * rb + S * 8) // 128) * 128
     assert block_bytes <= pl["smem_bytes"] <= 227 * 1024
@@ -321,7 +333,7 @@ SMALL_SHAPES = [(2, 1024, 512), (3, 1000, 96), (1, 777, 36), (2, 300, 7), (1, 1,
 @pytest.mark.parametrize("aligned", [True, False])
 @pytest.mark.parametrize("override", [(0, 0, 0), (1, 0, 1), (1, 0, 2), (1, 0, 4), (1, 0, 8),
                                       (2, 0, 2), (2, 0, 4), (2, 0, 8), (3, 0, 2), (3, 0, 4),
-                                      (3, 0, 8), (4, 0, 0), (5, 0, 0), (6, 0, 0)])
+                                      (3, 0, 8), (4, 0, 0), (5, 0, 0), (6, 0, 0), (7, 0, 0)])
 def test_plan_indices_small(shape, dtype, aligned, override):
     lib = _abi.lib()
     assert lib.sgr_set_kernel_override(override[0]) == 0

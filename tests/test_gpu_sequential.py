@@ -32,7 +32,9 @@ if not torch.cuda.is_available():
 
 DEV = torch.device("cuda:0")
 SEQ = _abi.KERNEL_SEQUENTIAL
-SEQ_KINDS = (_abi.KERNEL_SEQUENTIAL, _abi.KERNEL_SEQUENTIAL_SPLIT, _abi.KERNEL_SEQUENTIAL_PAIR)
+# 7: two channels per lane, bf16 only (fp32 takes kind 6 under that override)
+SEQ_KINDS = (_abi.KERNEL_SEQUENTIAL, _abi.KERNEL_SEQUENTIAL_SPLIT, _abi.KERNEL_SEQUENTIAL_PAIR,
+             _abi.KERNEL_SEQUENTIAL_PAIR2)
 
 
 @pytest.fixture(autouse=True)
@@ -69,7 +71,8 @@ SHAPES = [(2, 1, 64), (3, 17, 40), (2, 300, 96), (1, 1000, 200), (4, 129, 8), (2
 @pytest.mark.parametrize("kind", SEQ_KINDS)
 def test_mingru_sequential_matches_oracle(shape, dtype, init, kind):
     sgr.set_kernel_override(kind)
-    assert plan(*shape, dtype)["kernel"] == kind
+    want = _abi.KERNEL_SEQUENTIAL_PAIR if (kind == _abi.KERNEL_SEQUENTIAL_PAIR2 and dtype == "f32") else kind
+    assert plan(*shape, dtype)["kernel"] == want
     k, hx, h0 = small("mingru", *shape, dtype, init, seed=sum(shape) % 97)
     h = sgr.mingru_scan(*dev(k, hx, h0))
     torch.cuda.synchronize()
@@ -216,7 +219,8 @@ def test_bf16_workload_chunked_kernel_still_matches():
 
 
 @pytest.mark.parametrize("dtype,shape,forced", [
-    ("bf16", (128, 20, 4096), None),    # 16384 groups: ~111 warps per SM, several waves
+    ("bf16", (128, 20, 4096), None),    # 8192 groups of 64 channels (kernel 7): several waves
+    ("bf16", (128, 20, 4096), SEQ),     # 16384 warps: ~111 per SM, several waves
     ("f32", (1, 70000, 32), SEQ),       # one warp, 4375 slots: every ring slot reused many times
     ("f32", (1, 70001, 32), _abi.KERNEL_SEQUENTIAL_PAIR),    # two warps, 2188 slots, a ragged last one
     ("bf16", (2, 30001, 48), _abi.KERNEL_SEQUENTIAL_SPLIT),  # half-warps, partial channel groups
@@ -225,7 +229,7 @@ def test_sequential_many_waves_and_long_sequences(dtype, shape, forced):
     if forced:
         sgr.set_kernel_override(forced)
     pl = plan(*shape, dtype)
-    assert pl["kernel"] == (forced or SEQ)
+    assert pl["kernel"] == (forced or _abi.KERNEL_SEQUENTIAL_PAIR2)
     k, hx, h0 = small("mingru", *shape, dtype, "u01_1", seed=101)
     h = sgr.mingru_scan(*dev(k, hx, h0))
     r, s, x0 = small("minmax", *shape, dtype, "u01_1", seed=102)
