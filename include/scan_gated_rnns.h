@@ -384,7 +384,9 @@ SGR_API sgr_status_t minmax_scan_backward(const void *r, const void *s,
                                           void *workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* Bytes of workspace a gradient call of this shape needs (at least the 256-byte
- * header for a non-empty shape).  Pure host code. */
+ * header for a non-empty shape; it covers the plain and the time-decayed
+ * gradient).  0 for SGR_OP_MINGRU_LOG, which has no gradient.  Pure host
+ * code. */
 SGR_API size_t sgr_backward_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D,
                                            sgr_dtype_t dtype);
 
@@ -441,7 +443,9 @@ SGR_API sgr_status_t minmax_scan_host(const void *r, const void *s,
 /* ------------------------------------------------------------ workspace */
 
 /* Bytes of workspace a scan of this shape needs: at least the 256-byte header
- * for any non-empty shape, 0 for an empty one.  Pure host code. */
+ * for any non-empty shape, 0 for an empty one or an unknown op.  op selects
+ * mingru_scan (and mingru_scan_decay), minmax_scan, or mingru_scan_log
+ * (SGR_OP_MINGRU_LOG).  Pure host code. */
 SGR_API size_t sgr_workspace_size(sgr_op_t op, int64_t B, int64_t T, int64_t D,
                           sgr_dtype_t dtype);
 
