@@ -136,7 +136,10 @@ struct BwdParams {
 // ct TR + TR - 1 - rho.  Tiles are numbered chain-fastest in processing order
 // and, when the sequence spans several chunks, handed to persistent blocks by
 // a ticket counter (for_each_ticket), so every look-back waits on a tile that
-// a running block holds.
+// a running block holds.  It runs the gradients the copy-engine-fed kernels
+// do not take: unaligned rows and shapes with under two tiles per SM (aligned
+// narrow batches take scan_pipelined_backward.cuh, wide ones the
+// channel-sequential gradient).
 template <class BOp, typename IO, int V, int CG, int R, int W, int MINB>
 __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_backward_kernel(const BwdParams bp) {
     constexpr int J = 32 / CG;

@@ -17,8 +17,9 @@
 // The minGRU log-space formula h = exp(a* + logcumsumexp(log z + log g - a*))
 // is the closed form of the same affine composition; evaluating the pairs in
 // linear space gives that function with fp32 errors relative to each term
-// (no cancellation: all terms are positive) and with 3 MUFU ops per element
-// instead of about 7.
+// (no cancellation: all terms are positive) and with 3-4 MUFU ops per
+// element instead of about 9 for the log-space pairs (MinGRULogOp below,
+// kept as the measured alternative).
 //
 // Work decomposition (one thread block = one tile of TR rows x TC channels):
 //   load   : each thread loads R consecutive rows x V channels of both inputs
@@ -875,9 +876,9 @@ __global__ void __launch_bounds__((W + 1) * 32, MINB) scan_tile_kernel(const Sca
 
 // --------------------------------------------------- pipelined kernel
 //
-// Persistent blocks (co-resident, cooperative launch, two per SM), each owning
-// tiles blockIdx.x, blockIdx.x + gridDim.x, ... in order.  7 data warps and
-// one carry warp.  A tile is TR x TC with TC = CG * V channels (V = 4) and
+// Persistent blocks (co-resident, cooperative launch), each owning tiles
+// blockIdx.x, blockIdx.x + gridDim.x, ... in order: 7 data warps and one
+// carry warp with two blocks per SM, or 15 and one with one block per SM.  A tile is TR x TC with TC = CG * V channels (V = 4) and
 // TR = W * J * R rows (J = 32 / CG row groups per warp): lane (g, j) =
 // (lane % CG, lane / CG) of warp w owns channels [g V, g V + V) of rows
 // [(w J + j) R, (w J + j) R + R).  Narrow tiles (128-byte rows) keep the chunk

@@ -25,14 +25,16 @@
 // tile is time row ct TR + TR - 1 - rho, which the slot holds at row
 // TR - 1 - rho.  Phase A: the local partials (A, cP, cQ) of every element and
 // the pair (A, A gy), the fold of the thread's R rows, the scan across the
-// warp's J row groups and the warp summary, as in the forward kernel.  The
+// warp's J row groups and the warp summary, as in the forward kernel; the
+// arithmetic runs on pairs of neighbouring channels (packed fp32x2).  The
 // four values per element (A, gy, cP, cQ; with decay also the dL/dlambda
-// factor) stay in registers, so phase B of a tile follows its own phase A
-// (no one-tile lag): replay lam from the thread's incoming gradient, write
-// both input gradients with streaming stores, the initial state's gradient
-// from the thread that ends at time row 0, and dL/dlambda with one atomic
-// add per channel and warp.  Carry warp: the forward kernel's, with the
-// affine operator.
+// factor -u h_{t-1}) stay in registers, so phase B of a tile follows its own
+// phase A (no one-tile lag): replay lam from the thread's incoming gradient,
+// write both input gradients with streaming stores, the initial state's
+// gradient from the thread that ends at time row 0, and the dL/dlambda
+// terms, summed over the tile in shared memory and added with one atomic
+// per channel and tile.  Carry warp: the forward kernel's, with the affine
+// operator.
 #pragma once
 
 #include "scan_backward.cuh"

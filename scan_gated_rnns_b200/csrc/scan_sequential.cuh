@@ -14,8 +14,11 @@
 // kernels in scan_engine.cuh remain for shapes with fewer channels, where the
 // time axis has to be cut to fill the GPU.
 //
-// Layout per warp: a channel group of 32 channels (a 128-byte fp32 or 64-byte
-// bf16 row segment per operand), lane l owning channel l of the group.  The
+// Layout per warp (the one-warp kernel; the two-warp kernels below split
+// each slot's rows between a pair of warps, and the bf16 form with 64-channel
+// groups gives each lane two channels): a channel group of 32 channels (a
+// 128-byte fp32 or 64-byte bf16 row segment per operand), lane l owning
+// channel l of the group.  The
 // warp streams its rows through a ring of S slots of
 // RB rows in shared memory, both operands of a slot loaded by the tensor
 // memory accelerator (one box of CW channels x RB rows per operand, completion
@@ -112,8 +115,10 @@ __device__ __forceinline__ void seq_rows(float k0, float hx0, float k1, float hx
 // Time decay in the channel-sequential kernels: the gaps u_t are per (batch
 // row, row), shared by a warp's channels.  A warp's 16 rows of a slot have
 // their gaps spread across the lanes, lane l holding row y0 + (l % 16)'s
-// (0 past T: gamma = 1), loaded two slots ahead so that no step waits for
-// them; each row's gap is then taken from its lane by one shuffle.
+// (0 past T: gamma = 1) -- read from the slot's gap box where the copy engine
+// brings it (seq_smem_gap), else loaded two slots ahead (seq_slot_gap) so
+// that no step waits for them; each row's gap is then taken from its lane by
+// one shuffle.
 __device__ __forceinline__ float seq_slot_gap(const ScanParams &p, int64_t b, int64_t y0, int lane) {
     const int64_t t = y0 + (lane & (kSeqRows - 1));
     return (y0 >= 0 && t < p.T) ? decay_u(p, b, t) : 0.f;

@@ -204,17 +204,21 @@ def test_sequential_graph_capture_replays(kind):
         assert rel_err(out, oracle.mingru_linear(k, hx, h0, threads=8)) <= TOL["bf16"]
 
 
-def test_bf16_workload_chunked_kernel_still_matches():
-    # the full-size bf16 workload through the chunked pipelined kernel (the
-    # automatic choice there is the two-warp channel-sequential kernel)
+@pytest.mark.parametrize("kind,label", [(_abi.KERNEL_PIPELINED, "the chunked kernel"),
+                                        (_abi.KERNEL_SEQUENTIAL_PAIR2, "64-channel warp pairs")])
+def test_bf16_workload_other_kernels_still_match(kind, label):
+    # the full-size bf16 workload through the chunked pipelined kernel and the
+    # two-channels-per-lane kernel (the automatic choice there is the two-warp
+    # channel-sequential kernel with 32-channel groups)
     w = WORKLOADS["mingru_b16_t2048_d4096_bf16_h0"]
     assert plan(w.B, w.T, w.D, "bf16")["kernel"] == _abi.KERNEL_SEQUENTIAL_PAIR
-    sgr.set_kernel_override(_abi.KERNEL_PIPELINED)
+    sgr.set_kernel_override(kind)
+    assert plan(w.B, w.T, w.D, "bf16")["kernel"] == kind
     k, hx, h0 = generate(w, device=DEV)
     h = sgr.mingru_scan(k, hx, h0)
     torch.cuda.synchronize()
     err = full_rel_err("mingru", k, hx, h0, h)             # every channel and row
-    print(f"{w.name} through the chunked kernel: max relative error {err:.3e}")
+    print(f"{w.name} through {label}: max relative error {err:.3e}")
     assert err <= TOL["bf16"]
 
 
