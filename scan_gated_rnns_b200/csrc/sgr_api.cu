@@ -1003,10 +1003,18 @@ bool seq_backward_planned(int64_t B, int64_t T, int64_t D, int esz, bool aligned
 // channel tiles give the blocks in flight little look-back depth (fp32 B8 x
 // 4096 x 1024, 256 chains: 187 against 195 us; bf16, 128 chains: 142
 // against 150) and the 15-warp ones where the depth grows (fp32 B4 x 8192 x
-// 768, 96 chains: 150 against 158 us).
-template <typename IO> constexpr int bwd_pipe_r() { return sizeof(IO) == 4 ? 2 : 4; }
-template <typename IO, bool DT = false, int W = kPipeWarpsWide>
-using BwdPipeShape = PipeBwdShape<IO, 4, pipe_cg<IO>(), bwd_pipe_r<IO>(), kStages, W, DT>;
+// 768, 96 chains: 150 against 158 us).  The fp32 decayed gradient takes
+// 7-warp blocks with 4 rows per thread (16 elements, one block per SM,
+// 112-row tiles) at any chain count: the per-tile work is spread over twice
+// the elements, measured 182.8 against 186.5 us (7-warp, 2 rows) and 193.1
+// (15-warp) on B8 x 4096 x 1024, 143.9 against 156.7 and 149.5 on
+// B4 x 8192 x 768, 188.9 against 197.2 and 194.1 on B2 x 8192 x 2048.
+template <typename IO, bool DECAY = false, int W = kPipeWarpsWide>
+constexpr int bwd_pipe_r() { return (sizeof(IO) == 2 || (DECAY && W == kPipeWarps)) ? 4 : 2; }
+template <typename IO, bool DECAY, int W>
+constexpr int bwd_pipe_minb() { return (W == kPipeWarps && !(sizeof(IO) == 4 && DECAY)) ? 2 : 1; }
+template <typename IO, bool DT = false, int W = kPipeWarpsWide, bool DECAY = false>
+using BwdPipeShape = PipeBwdShape<IO, 4, pipe_cg<IO>(), bwd_pipe_r<IO, DECAY, W>(), kStages, W, DT>;
 
 // The gradient's tile plan: the pipelined kernel for aligned vector-width
 // rows with at least two tiles per SM (override 2 or 3 forces it wherever the
@@ -1025,17 +1033,24 @@ Plan make_bwd_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool alig
         p.V = 4;
         p.cg = esz == 4 ? 8 : 16;
         p.TC = p.cg * p.V;
-        p.r = esz == 4 ? 2 : 4;
         p.stages = kStages;
         // blocks of 15 data warps, one per SM, or of 7, two per SM (override
-        // 2; decay with at least 0.8 chains per SM)
+        // 2; bf16 decay with at least 0.8 chains per SM); the fp32 decayed
+        // gradient always takes 7-warp blocks, one per SM with 4 rows per
+        // thread
         const int64_t chains = B * ((D + (esz == 4 ? 32 : 64) - 1) / (esz == 4 ? 32 : 64));
-        const bool narrow = ok == KIND_PIPELINED || (ok == KIND_AUTO && decay && 5 * chains >= 4 * kAssumedSMs);
+        const bool narrow = ok == KIND_PIPELINED ||
+                            (ok == KIND_AUTO && decay && (esz == 4 || 5 * chains >= 4 * kAssumedSMs));
         p.warps = narrow ? kPipeWarps : kPipeWarpsWide;
+        p.r = (esz == 2 || (decay && narrow)) ? 4 : 2;
         p.TR = p.warps * (32 / p.cg) * p.r;
-        p.smem = narrow ? (esz == 4 ? BwdPipeShape<float, false, kPipeWarps>::smem_bytes
-                                    : BwdPipeShape<__nv_bfloat16, false, kPipeWarps>::smem_bytes)
-                        : (esz == 4 ? BwdPipeShape<float>::smem_bytes : BwdPipeShape<__nv_bfloat16>::smem_bytes);
+        if (esz == 4)
+            p.smem = narrow ? (decay ? BwdPipeShape<float, false, kPipeWarps, true>::smem_bytes
+                                     : BwdPipeShape<float, false, kPipeWarps>::smem_bytes)
+                            : BwdPipeShape<float>::smem_bytes;
+        else
+            p.smem = narrow ? BwdPipeShape<__nv_bfloat16, false, kPipeWarps>::smem_bytes
+                            : BwdPipeShape<__nv_bfloat16>::smem_bytes;
         p.n_dt = (D + p.TC - 1) / p.TC;
         p.n_chains = B * p.n_dt;
         p.n_chunks = (T + p.TR - 1) / p.TR;
@@ -1053,9 +1068,9 @@ Plan make_bwd_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool alig
 template <class BOp, typename IO, bool DT, int W>
 cudaError_t launch_pipelined_bwd_shape(const BwdParams &bp, const CUtensorMap (&m)[6], cudaStream_t s) {
     constexpr int CG = pipe_cg<IO>();
-    constexpr int R = bwd_pipe_r<IO>();
-    using Shape = BwdPipeShape<IO, DT, W>;
-    auto kernel = scan_pipelined_backward_kernel<BOp, IO, 4, CG, R, kStages, W, W == kPipeWarps ? 2 : 1, DT>;
+    constexpr int R = bwd_pipe_r<IO, BOp::kDecay, W>();
+    using Shape = BwdPipeShape<IO, DT, W, BOp::kDecay>;
+    auto kernel = scan_pipelined_backward_kernel<BOp, IO, 4, CG, R, kStages, W, bwd_pipe_minb<IO, BOp::kDecay, W>(), DT>;
     constexpr size_t smem = Shape::smem_bytes;
     constexpr int NT = (W + 1) * 32;
     int dev = 0;
@@ -1091,7 +1106,7 @@ cudaError_t launch_pipelined_bwd_shape(const BwdParams &bp, const CUtensorMap (&
 
 template <class BOp, typename IO, int W>
 cudaError_t launch_pipelined_bwd(const BwdParams &bp, cudaStream_t s) {
-    using Shape = BwdPipeShape<IO, false, W>;
+    using Shape = BwdPipeShape<IO, false, W, BOp::kDecay>;
     const ScanParams &sp = bp.s;
     const int esz = int(sizeof(IO));
     // k, hx (or r, s), dL/dh, the forward output; the decay's gaps and rates
@@ -1101,7 +1116,7 @@ cudaError_t launch_pipelined_bwd(const BwdParams &bp, cudaStream_t s) {
         !make_operand_map(&m[2], bp.gy, sp.B, sp.T, sp.D, esz, Shape::TC, Shape::TR) ||
         !make_operand_map(&m[3], bp.fwd, sp.B, sp.T, sp.D, esz, Shape::TC, Shape::TR))
         return cudaErrorInvalidValue;
-    if constexpr (BOp::kDecay && BwdPipeShape<IO, true, W>::dec_boxable) {
+    if constexpr (BOp::kDecay && BwdPipeShape<IO, true, W, true>::dec_boxable) {
         if (make_decay_maps(&m[4], &m[5], sp, Shape::TR, Shape::TC))
             return launch_pipelined_bwd_shape<BOp, IO, true, W>(bp, m, s);
     }
