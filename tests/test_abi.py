@@ -532,6 +532,7 @@ def test_summary_and_combine_argument_errors():
     s = lambda *a: lib.sgr_scan_summary(*a)   # noqa: E731
     assert s(MINGRU, A, Bp, -1, 100, 64, F32, P, W, need, None) == E
     assert s(7, A, Bp, 2, 100, 64, F32, P, W, need, None) == E
+    assert s(_abi.SGR_OP_MINGRU_LOG, A, Bp, 2, 100, 64, F32, P, W, need, None) == E   # linear pairs only
     assert s(MINGRU, A, Bp, 2, 100, 64, 9, P, W, need, None) == E
     assert s(MINGRU, A, Bp, 2, 100, 64, F32, None, W, need, None) == E
     assert s(MINGRU, None, Bp, 2, 100, 64, F32, P, W, need, None) == E
@@ -550,6 +551,7 @@ def test_summary_and_combine_argument_errors():
     assert c(MINGRU, P, 1, None, 0, P + 8, 64, 2, 64, F32, None) == E         # out on the pairs
     assert c(MINGRU, P, 1, C + 4, 64, C, 64, 2, 64, F32, None) == E           # out partly on init
     assert c(MINGRU, P, 1, None, 0, None, 64, 0, 64, F32, None) == _abi.SGR_OK
+    assert c(_abi.SGR_OP_MINGRU_LOG, P, 1, None, 0, C, 64, 2, 64, F32, None) == E
 
 
 @fake_addresses
