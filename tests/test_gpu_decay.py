@@ -182,7 +182,7 @@ def test_decay_workload_gradient_every_channel(log1p_delta):
 # the gap array allows it (16-byte aligned start, batch stride a multiple of
 # 4) and load them themselves otherwise: both, forward and gradient.
 @pytest.mark.parametrize("B,pad,gap_off", [(3, 0, 0), (3, 3, 0), (3, 1, 0), (3, 0, 1), (1, 0, 0)])
-@pytest.mark.parametrize("kernel", [4, 5, 6])
+@pytest.mark.parametrize("kernel", [4, 5, 6, 7])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_decay_sequential_gap_layouts(B, pad, gap_off, kernel, dtype):
     sgr.set_kernel_override(kernel)
