@@ -1116,6 +1116,20 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
             [[maybe_unused]] const float *s_lam =
                 reinterpret_cast<const float *>(smem + (n % S) * Shape::slot_bytes + 2 * Shape::op_bytes);
             [[maybe_unused]] const float *s_gap = s_lam + TC;
+            // DT: the thread's rates (as lam2 pairs) and its R row gaps, read
+            // once per tile
+            [[maybe_unused]] float2 l2p[V2];
+            if constexpr (DT) {
+#pragma unroll
+                for (int i = 0; i < V2; ++i)
+                    l2p[i] = __fmul2_rn(*reinterpret_cast<const float2 *>(s_lam + g * V + 2 * i),
+                                        make_float2(kNegLog2e, kNegLog2e));
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    ur[r] = s_gap[(warp * J + j) * R + r];
+                    if (p.decay_log1p) ur[r] = log1pf(ur[r]);
+                }
+            }
             float2 IA[V2], IB[V2];
 #pragma unroll
             for (int i = 0; i < V2; ++i) {
@@ -1130,12 +1144,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                     unpack(*reinterpret_cast<const Vec *>(t0 + r * TC), x0);
                     unpack(*reinterpret_cast<const Vec *>(t1 + r * TC), x1);
                     [[maybe_unused]] float u = 0.f;
-                    if constexpr (DT) {
-                        u = s_gap[(warp * J + j) * R + r];
-                        if (p.decay_log1p) u = log1pf(u);
-                    } else if constexpr (Op::kDecay) {
-                        u = ur[r];
-                    }
+                    if constexpr (Op::kDecay) u = ur[r];
                     if (!FULL) {
                         const bool ok = dvalid[SB] && (row0[SB] + r < p.T);
 #pragma unroll
@@ -1149,9 +1158,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                         float2 a2, b2;
                         element_pair<Op, IO>(x0[2 * i], x1[2 * i], x0[2 * i + 1], x1[2 * i + 1], a2, b2);
                         if constexpr (DT) {
-                            const float2 l2 = __fmul2_rn(*reinterpret_cast<const float2 *>(s_lam + g * V + 2 * i),
-                                                         make_float2(kNegLog2e, kNegLog2e));
-                            const float2 e = __fmul2_rn(l2, make_float2(u, u));
+                            const float2 e = __fmul2_rn(l2p[i], make_float2(u, u));
                             a2 = __fmul2_rn(a2, make_float2(fast_exp2(e.x), fast_exp2(e.y)));
                         } else if constexpr (Op::kDecay) {
                             a2 = __fmul2_rn(a2, make_float2(decay_gamma(lam2[2 * i], u), decay_gamma(lam2[2 * i + 1], u)));
