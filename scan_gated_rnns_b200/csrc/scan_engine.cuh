@@ -1079,10 +1079,11 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
         // channels per float2
         float2 PA[NB][R][V2], PB[NB][R][V2];
         float2 E[NB][V];     // the thread's exclusive prefix within its warp, per channel
-        int64_t base[NB];    // global offset of the thread's first element of the tile
-        int row0[NB];        // first row (along T) of the thread's rows
-        bool full[NB];       // all R rows and V channels of the thread inside the tensor
-        bool dvalid[NB];
+        // per tile buffer, what phase B needs: the thread's first output
+        // element and how many of its R rows lie inside the tensor (0 for
+        // channels past D)
+        IO *dstb[NB];
+        int nval[NB];
         uint32_t wait_limit = kMbarLimit;
 
         auto phaseA = [&](int n, auto bufc) {
@@ -1090,10 +1091,12 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
             constexpr int SB = LAG ? BUF : 0;
             const TileCoord tc = tile_coord(p, uint32_t(first + int64_t(n) * G));
             const int64_t d0 = int64_t(tc.dt) * TC + g * V;
-            dvalid[SB] = d0 < p.D;
-            row0[SB] = int(tc.c) * TR + (warp * J + j) * R;
-            full[SB] = dvalid[SB] && (row0[SB] + R <= p.T);
-            base[SB] = (int64_t(tc.b) * p.T) * p.D + d0;
+            const bool dvalid = d0 < p.D;
+            const int row0 = int(tc.c) * TR + (warp * J + j) * R;
+            const int64_t left = p.T - row0;
+            nval[SB] = dvalid ? int(left < R ? (left > 0 ? left : 0) : R) : 0;
+            const bool full = nval[SB] == R;
+            dstb[SB] = out + (int64_t(tc.b) * p.T + row0) * p.D + d0;
             // time decay: the tile's rates and the thread's row gaps are plain
             // global loads, issued before the wait for the tile so that their
             // latency overlaps it
@@ -1102,7 +1105,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
 #pragma unroll
                 for (int v = 0; v < V; ++v) lam2[v] = decay_lam2(p, d0 + v);
 #pragma unroll
-                for (int r = 0; r < R; ++r) ur[r] = row0[SB] + r < p.T ? decay_u(p, tc.b, row0[SB] + r) : 0.f;
+                for (int r = 0; r < R; ++r) ur[r] = row0 + r < p.T ? decay_u(p, tc.b, row0 + r) : 0.f;
             }
             if (!mbar_wait(bars + 8u * uint32_t(n % S), uint32_t((n / S) & 1), wait_limit)) {
                 wait_limit = 1;
@@ -1146,7 +1149,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                     [[maybe_unused]] float u = 0.f;
                     if constexpr (Op::kDecay) u = ur[r];
                     if (!FULL) {
-                        const bool ok = dvalid[SB] && (row0[SB] + r < p.T);
+                        const bool ok = r < nval[SB];
 #pragma unroll
                         for (int v = 0; v < V; ++v) {
                             x0[v] = ok ? x0[v] : Op::pad0();
@@ -1169,7 +1172,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                     }
                 }
             };
-            if (full[SB]) rows(std::true_type{});
+            if (full) rows(std::true_type{});
             else rows(std::false_type{});
             float2 incl[V];
 #pragma unroll
@@ -1245,7 +1248,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                 const float w1 = Op::apply(s_tot[BUF][warp][c0 + 1], s_hin[BUF][c0 + 1]);
                 st[i] = make_float2(Op::apply(E[SB][2 * i], w0), Op::apply(E[SB][2 * i + 1], w1));
             }
-            IO *dst = out + base[SB] + int64_t(row0[SB]) * p.D;
+            IO *dst = dstb[SB];
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 float y[V];
@@ -1255,7 +1258,7 @@ scan_pipelined_kernel(const ScanParams p, const __grid_constant__ CUtensorMap ma
                     y[2 * i] = Op::state_out(st[i].x);
                     y[2 * i + 1] = Op::state_out(st[i].y);
                 }
-                if (full[SB] || (dvalid[SB] && row0[SB] + r < p.T)) Access<IO, V>::store(dst, y);
+                if (r < nval[SB]) Access<IO, V>::store(dst, y);
                 dst += p.D;
             }
         };
