@@ -297,7 +297,8 @@ def plan_kernel(plan) -> str:
     return {1: "sgr::scan_tile_kernel", 2: "sgr::scan_pipelined_kernel", 3: "sgr::scan_pipelined_kernel",
             4: "sgr::scan_sequential_kernel", 5: "sgr::scan_sequential_kernel (split rows)",
             6: "sgr::scan_sequential_pair_kernel",
-            7: "sgr::scan_sequential_pair2_kernel"}.get(plan["kernel"], "sgr::scan_kernel")
+            7: "sgr::scan_sequential_pair2_kernel",
+            8: "sgr::scan_sequential_pair2_kernel (four warps)"}.get(plan["kernel"], "sgr::scan_kernel")
 
 
 def profile_kernel(plan) -> str:
@@ -307,7 +308,7 @@ def profile_kernel(plan) -> str:
         return "sgr::scan_sequential_kernel"
     if plan["kernel"] == 6:
         return "sgr::scan_sequential_pair_kernel"
-    if plan["kernel"] == 7:
+    if plan["kernel"] in (7, 8):
         return "sgr::scan_sequential_pair2_kernel"
     return "sgr::scan_kernel"
 

@@ -489,7 +489,9 @@ SGR_API sgr_status_t sgr_set_tile_override(int channel_lanes, int rows_per_threa
  * each slot's 16 rows split between the two half-warps of a warp (groups of
  * 16 channels), 6 channel-sequential with two warps per group of 32 channels
  * splitting each 32-row slot, 7 the same with groups of 64 channels, two
- * per lane (bf16 I/O; fp32 takes 6); 2-7 wherever the fast path applies.
+ * per lane (bf16 I/O; fp32 takes 6), 8 as 7 with four warps per group, 8
+ * rows of each slot each (bf16 I/O; fp32 takes 6); 2-8 wherever the fast
+ * path applies.
  */
 SGR_API sgr_status_t sgr_set_kernel_override(int kernel);
 
@@ -508,7 +510,8 @@ typedef struct sgr_plan {
                                    6: two warps per 32-channel group, each slot
                                    of 32 rows split between them; 7: the same
                                    with 64-channel groups, two channels per
-                                   lane (bf16)                                  */
+                                   lane (bf16); 8: as 7 with four warps per
+                                   group, 8 rows of each slot per warp          */
     int32_t channels_per_thread;
     int32_t channel_lanes;      /* lanes across D per warp                         */
     int32_t rows_per_thread;

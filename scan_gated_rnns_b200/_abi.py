@@ -98,6 +98,7 @@ KERNEL_SEQUENTIAL = 4
 KERNEL_SEQUENTIAL_SPLIT = 5
 KERNEL_SEQUENTIAL_PAIR = 6
 KERNEL_SEQUENTIAL_PAIR2 = 7
+KERNEL_SEQUENTIAL_QUAD = 8
 
 _lock = threading.Lock()
 _lib = None

@@ -333,9 +333,9 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
 // slot's outputs are written), which leaves the shared memory to the load
 // ring.  Dynamic shared memory: 2 x seq_pair_warp_bytes(S) + the pair buffers.
 constexpr int kPairWarps = 2;
-__host__ __device__ constexpr size_t seq_pair_warp_bytes(int S, int row_bytes, size_t gap = 0) {
-    return (size_t(S) * (2 * kSeqRows * row_bytes + gap) + size_t(kSeqRows) * row_bytes + size_t(S) * 8 + 127) /
-           128 * 128;
+// rows: a warp's rows of a slot (16; 8 in the four-warp blocks)
+__host__ __device__ constexpr size_t seq_pair_warp_bytes(int S, int row_bytes, size_t gap = 0, int rows = kSeqRows) {
+    return (size_t(S) * (2 * rows * row_bytes + gap) + size_t(rows) * row_bytes + size_t(S) * 8 + 127) / 128 * 128;
 }
 __host__ __device__ constexpr size_t seq_pair_block_bytes(int S, int row_bytes, size_t gap = 0) {
     return kPairWarps * seq_pair_warp_bytes(S, row_bytes, gap) + size_t(2) * kPairWarps * 32 * sizeof(float2);
@@ -496,17 +496,23 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
 // group of 64 channels of one batch row, lane l owning channels 2l and
 // 2l + 1, so each operand row of a warp is one 128-byte segment read as one
 // 32-bit shared load per lane, and each output row is written as one packed
-// bf16 pair.  Everything else follows scan_sequential_pair_kernel: warp w
-// takes rows [32 i + 16 w, 32 i + 16 w + 16) of slot i through its own ring,
-// folds them -- here four chains per lane (two channels x rows r and r + 8),
+// bf16 pair.  Everything else follows scan_sequential_pair_kernel: with NW
+// warps per block and RW = 32 / NW rows per warp, warp w takes rows
+// [32 i + RW w, 32 i + RW w + RW) of slot i through its own ring, folds them
+// -- here four chains per lane (two channels x rows r and r + RW / 2),
 // advanced as two fp32x2 operations per row pair -- exchanges its two pairs
-// with the other warp after one named barrier per slot, and writes each row
-// as its chain's running composite applied to the chain's incoming state.
-// The channel pair doubles each warp's independent work while the batch
-// provides half the warps.
+// with the other warps after one named barrier per slot (each warp composes
+// the slot's NW pairs in row order from the slot's incoming state, keeping
+// the state in front of its own rows), and writes each row as its chain's
+// running composite applied to the chain's incoming state.  The channel pair
+// doubles each warp's independent work while the batch provides half the
+// warps; four warps per group (8 rows each) bring the warp count back to
+// that of the 32-channel pairs.
 constexpr int kPair2Channels = 64;
-__host__ __device__ constexpr size_t seq_pair2_block_bytes(int S, size_t gap = 0) {
-    return kPairWarps * seq_pair_warp_bytes(S, kPair2Channels * 2, gap) + size_t(2) * kPairWarps * 32 * sizeof(float4);
+constexpr int kQuadWarps = 4;
+__host__ __device__ constexpr size_t seq_pair2_block_bytes(int S, size_t gap = 0, int NW = kPairWarps) {
+    return size_t(NW) * seq_pair_warp_bytes(S, kPair2Channels * 2, gap, 32 / NW) +
+           size_t(2) * size_t(NW) * 32 * sizeof(float4);
 }
 
 // two bf16 channels of one row: (low, high) halves as fp32
@@ -523,20 +529,22 @@ __device__ __forceinline__ void sts_bf16x2(uint32_t a, float lo, float hi) {
     asm volatile("st.shared.b32 [%0], %1;" ::"r"(a), "r"(*reinterpret_cast<const uint32_t *>(&h)) : "memory");
 }
 
-template <class Op, bool DT = false>
-__global__ void __launch_bounds__(kPairWarps * 32)
+template <class Op, bool DT = false, int NW = kPairWarps>
+__global__ void __launch_bounds__(NW * 32)
 scan_sequential_pair2_kernel(const SeqParams q, const __grid_constant__ CUtensorMap map0,
                              const __grid_constant__ CUtensorMap map1, const __grid_constant__ CUtensorMap map_out,
                              const __grid_constant__ CUtensorMap map_gap) {
     static_assert(!DT || Op::kDecay, "gaps through the copy engine need a decay operator");
     static_assert(!Op::kLogSpace, "the channel-sequential kernels carry linear states");
+    static_assert(NW == kPairWarps || NW == kQuadWarps, "two or four warps per group");
     using IO = __nv_bfloat16;
     constexpr uint32_t kGap = DT ? kSeqGapBytes : 0;
     constexpr int CW = kPair2Channels;
+    constexpr int RW = 32 / NW;                                     // a warp's rows of a slot
     constexpr int kRowBytes = CW * int(sizeof(IO));                 // 128
-    constexpr uint32_t kOpBytes = kSeqRows * kRowBytes;             // one operand of a warp's 16 rows
-    constexpr int kSlotRows = kPairWarps * kSeqRows;
-    constexpr int H = kSeqRows / 2;
+    constexpr uint32_t kOpBytes = RW * kRowBytes;                   // one operand of a warp's rows
+    constexpr int kSlotRows = NW * RW;
+    constexpr int H = RW / 2;
     const ScanParams &p = q.s;
     extern __shared__ __align__(128) unsigned char smem[];
 
@@ -550,18 +558,19 @@ scan_sequential_pair2_kernel(const SeqParams q, const __grid_constant__ CUtensor
     const int x0 = int(grp) * CW;
     const int64_t d = int64_t(x0) + 2 * lane;                       // the lane's first channel
 
+    // the slot's gap box is 16 rows (a warp of four-warp blocks uses 8 of them)
     constexpr uint32_t kSlot = 2 * kOpBytes + kGap;
-    const uint32_t base = smem_addr(smem) + uint32_t(w * seq_pair_warp_bytes(S, kRowBytes, kGap));
+    const uint32_t base = smem_addr(smem) + uint32_t(w * seq_pair_warp_bytes(S, kRowBytes, kGap, RW));
     const uint32_t ring = base;
     const uint32_t outb = base + uint32_t(S) * kSlot;
     const uint32_t bars = outb + kOpBytes;
-    float4 *xpair = reinterpret_cast<float4 *>(smem + kPairWarps * seq_pair_warp_bytes(S, kRowBytes, kGap));  // [2][2][32]
+    float4 *xpair = reinterpret_cast<float4 *>(smem + NW * seq_pair_warp_bytes(S, kRowBytes, kGap, RW));  // [2][NW][32]
 
     const int n_slots = int((p.T + kSlotRows - 1) / kSlotRows);
     auto issue = [&](int i, int s) {
         const uint32_t dst = ring + uint32_t(s) * kSlot;
         const uint32_t bar = bars + 8u * uint32_t(s);
-        const int y = i * kSlotRows + w * kSeqRows;
+        const int y = i * kSlotRows + w * RW;
         mbar_expect_tx(bar, 2 * kOpBytes + (DT ? kSeqRows * 4 : 0));
         tma_load_3d(dst, &map0, x0, y, int(b), bar);
         tma_load_3d(dst + kOpBytes, &map1, x0, y, int(b), bar);
@@ -581,8 +590,8 @@ scan_sequential_pair2_kernel(const SeqParams q, const __grid_constant__ CUtensor
     if constexpr (Op::kDecay) {
         lam2 = make_float2(d < p.D ? decay_lam2(p, d) : 0.f, d + 1 < p.D ? decay_lam2(p, d + 1) : 0.f);
         if constexpr (!DT) {
-            gcur = seq_slot_gap(p, b, w * kSeqRows, lane);
-            gnext = seq_slot_gap(p, b, kSlotRows + w * kSeqRows, lane);
+            gcur = seq_slot_gap(p, b, w * RW, lane);
+            gnext = seq_slot_gap(p, b, kSlotRows + w * RW, lane);
         }
     }
 
@@ -593,16 +602,16 @@ scan_sequential_pair2_kernel(const SeqParams q, const __grid_constant__ CUtensor
     for (int i = 0; i < n_slots; ++i) {
         [[maybe_unused]] float gnext2 = 0.f;
         if constexpr (Op::kDecay && !DT)
-            gnext2 = seq_slot_gap(p, b, int64_t(i + 2) * kSlotRows + w * kSeqRows, lane);
+            gnext2 = seq_slot_gap(p, b, int64_t(i + 2) * kSlotRows + w * RW, lane);
         if (!mbar_wait(bars + 8u * uint32_t(s), phase, wait_limit)) {
             wait_limit = 1;
             if (!bad && lane == 0 && p.status) atomicOr(p.status, kTimeoutBit);
             bad = true;
         }
         const uint32_t src = ring + uint32_t(s) * kSlot + uint32_t(lane) * 4u;
-        uint32_t x0r[kSeqRows], x1r[kSeqRows];
+        uint32_t x0r[RW], x1r[RW];
 #pragma unroll
-        for (int r = 0; r < kSeqRows; ++r) {
+        for (int r = 0; r < RW; ++r) {
             x0r[r] = lds32(src + r * kRowBytes);
             x1r[r] = lds32(src + kOpBytes + r * kRowBytes);
         }
@@ -617,8 +626,8 @@ scan_sequential_pair2_kernel(const SeqParams q, const __grid_constant__ CUtensor
             phase ^= 1u;
         }
         bad = __any_sync(0xffffffffu, bad);
-        // four chains: (channels d, d + 1) x (rows r, r + 8); L = rows 0-7,
-        // U = rows 8-15, each an fp32x2 over the two channels
+        // four chains: (channels d, d + 1) x (rows r, r + H); L = rows
+        // [0, H), U = rows [H, RW), each an fp32x2 over the two channels
         float2 PAL[H], PBL[H], PAU[H], PBU[H];
         float2 AL = make_float2(Op::identity().x, Op::identity().x), BL = make_float2(Op::identity().y, Op::identity().y);
         float2 AU = AL, BU = BL;
@@ -641,7 +650,7 @@ scan_sequential_pair2_kernel(const SeqParams q, const __grid_constant__ CUtensor
             PAU[r] = AU;
             PBU[r] = BU;
         }
-        // the warp's 16 rows per channel: the first chain, then the second
+        // the warp's RW rows per channel: the first chain, then the second
         float4 P;
         {
             const float2 p0 = Op::combine(make_float2(AL.x, BL.x), make_float2(AU.x, BU.x));
@@ -650,17 +659,20 @@ scan_sequential_pair2_kernel(const SeqParams q, const __grid_constant__ CUtensor
         }
         if (bad) P = make_float4(__int_as_float(0x7fffffff), __int_as_float(0x7fffffff), __int_as_float(0x7fffffff),
                                  __int_as_float(0x7fffffff));
-        float4 *xb = xpair + (i & 1) * kPairWarps * 32;
+        // the slot's pairs in row order (double-buffered by slot parity: a
+        // buffer is written again two slots later, after every warp has read
+        // it and passed the next slot's barrier)
+        float4 *xb = xpair + (i & 1) * NW * 32;
         xb[w * 32 + lane] = P;
-        named_barrier_sync(1, kPairWarps * 32);
-        const float4 Q = xb[(1 - w) * 32 + lane];
-        const float4 F = w ? Q : P, L = w ? P : Q;                  // first and second half of the slot
-        const float2 hmid = make_float2(Op::apply(make_float2(F.x, F.y), h.x), Op::apply(make_float2(F.z, F.w), h.y));
-        const float2 hend =
-            make_float2(Op::apply(make_float2(L.x, L.y), hmid.x), Op::apply(make_float2(L.z, L.w), hmid.y));
-        const float2 hin = w ? hmid : h;
-        h = hend;
-        // incoming states of the upper chains: after row 7 of each channel
+        named_barrier_sync(1, NW * 32);
+        float2 hin = h;
+#pragma unroll
+        for (int j = 0; j < NW; ++j) {
+            const float4 Pj = j == w ? P : xb[j * 32 + lane];
+            if (j == w) hin = h;                                     // the state in front of this warp's rows
+            h = make_float2(Op::apply(make_float2(Pj.x, Pj.y), h.x), Op::apply(make_float2(Pj.z, Pj.w), h.y));
+        }
+        // incoming states of the upper chains: after row H - 1 of each channel
         float2 hu = make_float2(Op::apply(make_float2(AL.x, BL.x), hin.x), Op::apply(make_float2(AL.y, BL.y), hin.y));
         float2 hl = hin;
         if (bad) {
@@ -679,7 +691,7 @@ scan_sequential_pair2_kernel(const SeqParams q, const __grid_constant__ CUtensor
         }
         fence_proxy_async();
         __syncwarp();
-        const int y0 = i * kSlotRows + w * kSeqRows;
+        const int y0 = i * kSlotRows + w * RW;
         if (lane == 0 && y0 < p.T) {
             tma_store_3d(&map_out, outb, x0, y0, int(b));
             bulk_commit();

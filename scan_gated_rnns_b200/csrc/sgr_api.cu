@@ -38,9 +38,10 @@ constexpr size_t kAlign = 256;
 constexpr size_t kTicketOffset = 64;
 
 enum Kind { KIND_AUTO = 0, KIND_TILE = 1, KIND_PIPELINED = 2, KIND_PIPELINED_WIDE = 3, KIND_SEQUENTIAL = 4,
-            KIND_SEQUENTIAL_SPLIT = 5, KIND_SEQUENTIAL_PAIR = 6, KIND_SEQUENTIAL_PAIR2 = 7 };
+            KIND_SEQUENTIAL_SPLIT = 5, KIND_SEQUENTIAL_PAIR = 6, KIND_SEQUENTIAL_PAIR2 = 7, KIND_SEQUENTIAL_QUAD = 8 };
 bool seq_kind(int k) {
-    return k == KIND_SEQUENTIAL || k == KIND_SEQUENTIAL_SPLIT || k == KIND_SEQUENTIAL_PAIR || k == KIND_SEQUENTIAL_PAIR2;
+    return k == KIND_SEQUENTIAL || k == KIND_SEQUENTIAL_SPLIT || k == KIND_SEQUENTIAL_PAIR ||
+           k == KIND_SEQUENTIAL_PAIR2 || k == KIND_SEQUENTIAL_QUAD;
 }
 
 // Channel-sequential kernels (scan_sequential.cuh): each 32-channel group's
@@ -68,6 +69,19 @@ constexpr int kSeqPairBelowHalf = 24;
 // (us, one warp per 32 / two per 32 / two per 64 channels): B32 x 2048 x 4096
 // (27.7 groups per SM) 301.6 / 315.9 / 289.2; below, the 32-channel pairs
 // win: B24 (20.8) 248.3 / 238.1 / 250.4, B16 (13.8) 162.3 / 158.2 / 172.5.
+// Four warps per group of 64 channels (8 rows of each slot per warp, the
+// same kernel): the warps of the 32-channel pairs with the per-element work
+// of the 64-channel ones.  Measured on B x 2048 x 4096 bf16 (us, two warps
+// per 32 / two per 64 / four per 64 channels): minGRU B20 (17.3 groups per
+// SM) 205.3 / 197.2 / 199.1, B24 238.1 / 240.1 / 231.9, B32 313.9 / 276.5 /
+// 289.2; decayed B16 182.8 / 205.3 / 184.0, B20 234.0 / 248.3 / 229.3, B24
+// 287.4 / 295.4 / 270.9, B28 327.1 / 334.2 / 313.9, B32 350.7 / 340.5 / 338.0;
+// MinMax B8 82.5 / 76.2 / 76.5, B12 137.6 / 121.3 / 125.4, B16 156.2 / 162.3 /
+// 154.1, B24 227.9 / 227.6 / 219.6, B32 309.7 / 289.2 / 277.0.  Chosen for
+// bf16 MinMax wherever a channel-sequential kernel runs, and for the minGRU
+// from kSeqQuadFrom groups per SM: up to kSeqPairBelowHalf for the plain
+// scan (two warps per 64 channels above), throughout for the decayed one.
+constexpr int kSeqQuadFrom = 16;
 // The gradient (four operands in, two out per element) walks whole sequences
 // from 5 warps per SM: against the pipelined gradient it loses at 3.5 groups
 // per SM (bf16 B4 x 2048 x 4096 150 us against 101 us; fp32 B8 x 2048 x 2048
@@ -212,9 +226,12 @@ SeqLayout seq_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, siz
 // the two-warp blocks of scan_sequential_pair_kernel: one block per channel
 // group, the block's share of the SM's shared memory split between its warps
 // wide: the two-channels-per-lane form (64-channel groups, float4 exchange)
+// with nw warps per group
 SeqLayout seq_pair_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, size_t reserved,
-                          size_t smem_block_max, size_t gap = 0, bool wide = false) {
-    auto bytes = [&](int S) { return wide ? seq_pair2_block_bytes(S, gap) : seq_pair_block_bytes(S, row_bytes, gap); };
+                          size_t smem_block_max, size_t gap = 0, bool wide = false, int nw = kPairWarps) {
+    auto bytes = [&](int S) {
+        return wide ? seq_pair2_block_bytes(S, gap, nw) : seq_pair_block_bytes(S, row_bytes, gap);
+    };
     SeqLayout l;
     const int64_t K = sms > 0 ? (groups + sms - 1) / sms : 1;
     size_t alloc = bytes(4);
@@ -244,7 +261,8 @@ SeqLayout seq_pair_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm
 // 8 rows per thread in 7-warp blocks, measured 78.3 against 82.4 us with 4
 // rows in 15-warp blocks on B8 x 4096 x 1024, 41.5 against 45.5 us on B2 x
 // 2048 x 4096, 47.5 against 47.7 us on B4 x 8192 x 512); wide decayed
-// batches take the channel-sequential kernels like the plain scan
+// batches take the channel-sequential kernels like the plain scan, bf16 ones
+// from kSeqQuadFrom groups per SM with four warps per 64-channel group
 // (each slot's gaps arrive with it through the copy engine, or, for gap
 // arrays the copy engine cannot address, spread across the lanes two slots
 // ahead)
@@ -272,25 +290,32 @@ Plan make_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned,
             // two channels per lane: bf16 only; automatic from kSeqPairBelowHalf
             // groups per SM, where it keeps the one-warp kernel's warp count
             // with fewer instructions and 128-byte rows
-            const bool wide = p.esz == 2 && (ok == KIND_SEQUENTIAL_PAIR2 ||
+            // four warps per group of 64 channels (8 rows of each slot per warp)
+            const bool auto_quad = p.esz == 2 && ok == KIND_AUTO &&
+                                   (light_op || (groups >= int64_t(kSeqQuadFrom) * kAssumedSMs &&
+                                                 (decay || groups < int64_t(pair_below) * kAssumedSMs)));
+            const bool wide = p.esz == 2 && (ok == KIND_SEQUENTIAL_PAIR2 || ok == KIND_SEQUENTIAL_QUAD || auto_quad ||
                                              (ok == KIND_AUTO && groups >= int64_t(pair_below) * kAssumedSMs));
+            const bool quad = wide && (ok == KIND_SEQUENTIAL_QUAD || auto_quad);
+            const int nw = quad ? kQuadWarps : kPairWarps;
             const bool pair = wide || ok == KIND_SEQUENTIAL_PAIR || ok == KIND_SEQUENTIAL_PAIR2 ||
+                              ok == KIND_SEQUENTIAL_QUAD ||
                               (ok == KIND_AUTO && groups < int64_t(pair_below) * kAssumedSMs);
             const int64_t gw = wide ? int64_t(kPair2Channels) : split ? cw / 2 : cw;   // channels per warp
             const int64_t n_warps = B * ((D + gw - 1) / gw);
             const size_t gap = decay ? kSeqGapBytes : 0;
             const SeqLayout lay = pair ? seq_pair_layout(n_warps, int(gw) * p.esz, kAssumedSMs, kAssumedSmemPerSM,
-                                                         kAssumedSmemReserved, kAssumedSmemPerBlock, gap, wide)
+                                                         kAssumedSmemReserved, kAssumedSmemPerBlock, gap, wide, nw)
                                        : seq_layout(n_warps, int(gw) * p.esz, kAssumedSMs, kAssumedSmemPerSM,
                                                     kAssumedSmemReserved, kAssumedSmemPerBlock, SEQ_SCAN, gap);
-            p.kind = wide ? KIND_SEQUENTIAL_PAIR2 : pair ? KIND_SEQUENTIAL_PAIR : split ? KIND_SEQUENTIAL_SPLIT
-                                                                                         : KIND_SEQUENTIAL;
+            p.kind = quad ? KIND_SEQUENTIAL_QUAD : wide ? KIND_SEQUENTIAL_PAIR2 : pair ? KIND_SEQUENTIAL_PAIR
+                                                      : split ? KIND_SEQUENTIAL_SPLIT : KIND_SEQUENTIAL;
             p.split = (split || pair) ? 2 : 1;
             p.V = wide ? 2 : 1;
             p.cg = int(gw / p.V);                                  // lanes across a group's channels
-            p.r = pair ? kSeqRows : kSeqRows / p.split;            // rows of a slot per lane
+            p.r = pair ? 32 / nw : kSeqRows / p.split;             // rows of a slot per lane
             p.stages = lay.slots;
-            p.warps = pair ? kPairWarps : kSeqWarpsPerBlock;
+            p.warps = pair ? nw : kSeqWarpsPerBlock;
             p.TR = T > 0 ? int(std::min<int64_t>(T, std::numeric_limits<int>::max())) : 0;
             p.TC = int(gw);
             p.smem = lay.smem;
@@ -718,39 +743,43 @@ cudaError_t launch_sequential_pair(const Plan &pl, const ScanParams &sp, cudaStr
     return launch_sequential_pair_dt<Op, IO, false>(pl, sp, map0, map1, map_out, map0, s);
 }
 
-template <class Op, bool DT>
+template <class Op, bool DT, int NW>
 cudaError_t launch_sequential_pair2_dt(const Plan &pl, const ScanParams &sp, const CUtensorMap &map0,
                                        const CUtensorMap &map1, const CUtensorMap &map_out,
                                        const CUtensorMap &map_gap, cudaStream_t s) {
     constexpr size_t kGap = DT ? kSeqGapBytes : 0;
-    auto kernel = scan_sequential_pair2_kernel<Op, DT>;
+    auto kernel = scan_sequential_pair2_kernel<Op, DT, NW>;
     SeqDev d;
-    cudaError_t e = seq_device(reinterpret_cast<const void *>(kernel), seq_pair2_block_bytes(kSeqMinSlots, kGap), &d);
+    cudaError_t e =
+        seq_device(reinterpret_cast<const void *>(kernel), seq_pair2_block_bytes(kSeqMinSlots, kGap, NW), &d);
     if (e != cudaSuccess) return e;
     SeqParams q;
     q.s = sp;
     q.n_groups = pl.n_dt;
     q.n_warps = pl.n_chains;                  // channel groups: one block each
     const SeqLayout lay = seq_pair_layout(q.n_warps, kPair2Channels * 2, d.sms, size_t(d.smem_sm), size_t(d.reserved),
-                                          size_t(d.smem_block), kGap, true);
+                                          size_t(d.smem_block), kGap, true, NW);
     q.slots = lay.slots;
-    kernel<<<dim3(unsigned(q.n_warps)), kPairWarps * 32, lay.smem, s>>>(q, map0, map1, map_out, map_gap);
+    kernel<<<dim3(unsigned(q.n_warps)), NW * 32, lay.smem, s>>>(q, map0, map1, map_out, map_gap);
     return cudaGetLastError();
 }
 
-template <class Op>
+// NW warps per group of 64 channels, each taking 32 / NW rows of a slot (the
+// height of the operand and output boxes)
+template <class Op, int NW>
 cudaError_t launch_sequential_pair2(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
     constexpr int CW = kPair2Channels;
+    constexpr int RW = 32 / NW;
     alignas(64) CUtensorMap map0, map1, map_out, map_gap;
-    if (!make_operand_map(&map0, sp.in0, sp.B, sp.T, sp.D, 2, CW, kSeqRows) ||
-        !make_operand_map(&map1, sp.in1, sp.B, sp.T, sp.D, 2, CW, kSeqRows) ||
-        !make_operand_map(&map_out, sp.out, sp.B, sp.T, sp.D, 2, CW, kSeqRows))
+    if (!make_operand_map(&map0, sp.in0, sp.B, sp.T, sp.D, 2, CW, RW) ||
+        !make_operand_map(&map1, sp.in1, sp.B, sp.T, sp.D, 2, CW, RW) ||
+        !make_operand_map(&map_out, sp.out, sp.B, sp.T, sp.D, 2, CW, RW))
         return cudaErrorInvalidValue;
     if constexpr (Op::kDecay) {
         if (make_seq_gap_map(&map_gap, sp))
-            return launch_sequential_pair2_dt<Op, true>(pl, sp, map0, map1, map_out, map_gap, s);
+            return launch_sequential_pair2_dt<Op, true, NW>(pl, sp, map0, map1, map_out, map_gap, s);
     }
-    return launch_sequential_pair2_dt<Op, false>(pl, sp, map0, map1, map_out, map0, s);
+    return launch_sequential_pair2_dt<Op, false, NW>(pl, sp, map0, map1, map_out, map0, s);
 }
 
 template <class Op, typename IO>
@@ -760,9 +789,13 @@ cudaError_t dispatch(const Plan &pl, const ScanParams &sp, cudaStream_t s) {
         if (pl.kind == KIND_SEQUENTIAL) return launch_sequential<Op, IO, 1>(pl, sp, s);
         if (pl.kind == KIND_SEQUENTIAL_SPLIT) return launch_sequential<Op, IO, 2>(pl, sp, s);
         if (pl.kind == KIND_SEQUENTIAL_PAIR) return launch_sequential_pair<Op, IO>(pl, sp, s);
-        if (pl.kind == KIND_SEQUENTIAL_PAIR2) {
-            if constexpr (sizeof(IO) == 2) return launch_sequential_pair2<Op>(pl, sp, s);
-            else return cudaErrorInvalidConfiguration;   // never planned (bf16 only)
+        if (pl.kind == KIND_SEQUENTIAL_PAIR2 || pl.kind == KIND_SEQUENTIAL_QUAD) {
+            if constexpr (sizeof(IO) == 2) {
+                if (pl.kind == KIND_SEQUENTIAL_QUAD) return launch_sequential_pair2<Op, kQuadWarps>(pl, sp, s);
+                return launch_sequential_pair2<Op, kPairWarps>(pl, sp, s);
+            } else {
+                return cudaErrorInvalidConfiguration;    // never planned (bf16 only)
+            }
         }
     } else {
         if (seq_kind(pl.kind)) return cudaErrorInvalidConfiguration;    // never planned (chunked_only)
@@ -1837,7 +1870,7 @@ sgr_status_t sgr_set_drop_publish(int64_t tile) {
 }
 
 sgr_status_t sgr_set_kernel_override(int kernel) {
-    if (kernel < KIND_AUTO || kernel > KIND_SEQUENTIAL_PAIR2) return SGR_ERR_INVALID_ARG;
+    if (kernel < KIND_AUTO || kernel > KIND_SEQUENTIAL_QUAD) return SGR_ERR_INVALID_ARG;
     g_override_kind.store(kernel);
     return SGR_OK;
 }

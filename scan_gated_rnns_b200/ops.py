@@ -329,7 +329,8 @@ def set_kernel_override(kernel: int = 0) -> None:
     blocks, 4 channel-sequential kernel (one warp per 32-channel group), 5 the
     same with each slot's rows split between half-warps, 6 two warps per
     32-channel group, 7 two warps per 64-channel group, two channels per lane
-    (bf16; 2-7 where the fast path applies).  Gradients: 1 the tile
+    (bf16), 8 four warps per 64-channel group (bf16; 2-8 where the fast path
+    applies).  Gradients: 1 the tile
     kernel, 2 the pipelined gradient with 7-warp blocks (two per SM), 3 with
     15-warp blocks (one per SM), 4 the channel-sequential gradient."""
     check("sgr_set_kernel_override", lib().sgr_set_kernel_override(kernel))

@@ -128,6 +128,10 @@ def test_decayed_plan():
         pl = _abi.plan(MINGRU, B, T, D, dtype, True, decay=True)
         assert pl["kernel"] == plain["kernel"] and pl["kernel"] in SEQ_KINDS, (B, T, D, dtype)
         assert pl["workspace_bytes"] == WS_HEADER
+    # bf16 from 16 groups per SM: four warps per 64-channel group
+    for B, want in ((16, _abi.KERNEL_SEQUENTIAL_PAIR), (20, _abi.KERNEL_SEQUENTIAL_QUAD),
+                    (32, _abi.KERNEL_SEQUENTIAL_QUAD)):
+        assert _abi.plan(MINGRU, B, 2048, 4096, BF16, True, decay=True)["kernel"] == want, B
     for B, T, D, dtype in ((8, 4096, 1024, BF16), (8, 4096, 1024, F32), (4, 8192, 512, BF16)):
         plain = _abi.plan(MINGRU, B, T, D, dtype, True)
         pl = _abi.plan(MINGRU, B, T, D, dtype, True, decay=True)
@@ -166,7 +170,7 @@ def test_workspace_size_and_hooks():
     assert lib.sgr_set_tile_override(3, 0) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_tile_override(0, 3) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_drop_publish(-2) == _abi.SGR_ERR_INVALID_ARG
-    assert lib.sgr_set_kernel_override(8) == _abi.SGR_ERR_INVALID_ARG
+    assert lib.sgr_set_kernel_override(9) == _abi.SGR_ERR_INVALID_ARG
     assert lib.sgr_set_kernel_override(_abi.KERNEL_SEQUENTIAL_SPLIT) == _abi.SGR_OK
     assert lib.sgr_set_kernel_override(0) == _abi.SGR_OK
     assert lib.sgr_set_wait_limit(0) == _abi.SGR_OK
@@ -181,7 +185,7 @@ def test_workspace_size_and_hooks():
 
 SEQ_ROWS = 16            # rows per load slot of the channel-sequential kernel
 SEQ_KINDS = (_abi.KERNEL_SEQUENTIAL, _abi.KERNEL_SEQUENTIAL_SPLIT, _abi.KERNEL_SEQUENTIAL_PAIR,
-             _abi.KERNEL_SEQUENTIAL_PAIR2)
+             _abi.KERNEL_SEQUENTIAL_PAIR2, _abi.KERNEL_SEQUENTIAL_QUAD)
 WS_HEADER = 256          # workspace header: status word at 0, chunk ticket at 64
 
 
@@ -195,25 +199,29 @@ def check_sequential_indices(pl, B, T, D, esz, check_cover):
     (kernel 6) a block's warps w = 0, 1 take rows [32 i + 16 w, 32 i + 16 w + 16)
     of slot i, lane l channel l.  Kernel 7 (bf16): the same with groups of 64
     channels, lane l owning channels 2 l and 2 l + 1 (one 32-bit word of a
-    128-byte row)."""
+    128-byte row); kernel 8: kernel 7 with four warps per group, warp w taking
+    rows [32 i + 8 w, 32 i + 8 w + 8) of slot i (boxes of 8 rows)."""
     V, CW = pl["channels_per_thread"], pl["tile_channels"]
-    pair2 = pl["kernel"] == _abi.KERNEL_SEQUENTIAL_PAIR2
+    quad = pl["kernel"] == _abi.KERNEL_SEQUENTIAL_QUAD
+    pair2 = pl["kernel"] == _abi.KERNEL_SEQUENTIAL_PAIR2 or quad
     pair = pl["kernel"] == _abi.KERNEL_SEQUENTIAL_PAIR or pair2
     split = 2 if pl["kernel"] == _abi.KERNEL_SEQUENTIAL_SPLIT else 1
+    nw = 4 if quad else 2 if pair else 1                # warps per group
+    rw = 32 // nw if pair else SEQ_ROWS                 # a warp's rows of a slot (box height)
     rb = CW * esz                                       # bytes of one operand row of a group
     if pair2:
         assert esz == 2 and V == 2 and CW == 64 and rb == 128
     else:
         assert V == 1 and CW == 32 // split and rb in (32, 64, 128)
     assert pl["vector_path"] and pl["channel_lanes"] * V == CW and pl["threads"] == 32 * pl["warps"]
-    assert pl["warps"] == (2 if pair else 1)
-    assert pl["rows_per_thread"] == SEQ_ROWS // split
+    assert pl["warps"] == nw
+    assert pl["rows_per_thread"] == (rw if pair else SEQ_ROWS // split)
     assert pl["n_chunks"] == 1 and pl["workspace_bytes"] == WS_HEADER and pl["tile_rows"] == T
-    # a lane's elements of a slot stay inside its warp's 16 rows of CW channels
+    # a lane's elements of a slot stay inside its warp's rw rows of CW channels
     lane = np.arange(32)
     if pair2:
         off = lane * 4                                  # channels 2 l, 2 l + 1: one 32-bit word
-        assert (off + (SEQ_ROWS - 1) * rb + 4 <= SEQ_ROWS * rb).all() and (off % 4 == 0).all()
+        assert (off + (rw - 1) * rb + 4 <= rw * rb).all() and (off % 4 == 0).all()
         assert len(set(off.tolist())) == 32
     else:
         off = (lane // CW) * pl["rows_per_thread"] * rb + (lane % CW) * esz
@@ -226,8 +234,8 @@ def check_sequential_indices(pl, B, T, D, esz, check_cover):
     # the warps' rings, staging buffers and mbarriers fit their block's shared memory
     S = pl["stages"]
     if pair:
-        warp_bytes = -(-(S * 2 * SEQ_ROWS * rb + SEQ_ROWS * rb + S * 8) // 128) * 128
-        block_bytes = 2 * warp_bytes + 2 * 2 * 32 * (16 if pair2 else 8)   # + the pairs exchanged per slot
+        warp_bytes = -(-(S * 2 * rw * rb + rw * rb + S * 8) // 128) * 128
+        block_bytes = nw * warp_bytes + 2 * nw * 32 * (16 if pair2 else 8)   # + the pairs exchanged per slot
     else:
         block_bytes = -(-(S * 2 * SEQ_ROWS * rb + 2 * SEQ_ROWS * rb + S * 8) // 128) * 128
     assert block_bytes <= pl["smem_bytes"] <= 227 * 1024
@@ -246,9 +254,9 @@ def check_sequential_indices(pl, B, T, D, esz, check_cover):
         cover = np.zeros((B, max(T, 1), D), dtype=np.int32)
         for w in range(len(gw)):
             for i in range(n_slots):
-                for y0 in ([i * slot_rows, i * slot_rows + SEQ_ROWS] if pair else [i * SEQ_ROWS]):
+                for y0 in ([i * slot_rows + rw * v for v in range(nw)] if pair else [i * SEQ_ROWS]):
                     if y0 < T:
-                        cover[b[w], y0:min(T, y0 + SEQ_ROWS), x0[w]:min(D, x0[w] + CW)] += 1
+                        cover[b[w], y0:min(T, y0 + rw), x0[w]:min(D, x0[w] + CW)] += 1
         assert (cover[:, :T] == 1).all(), "every output element is written exactly once"
 
 
@@ -333,7 +341,8 @@ SMALL_SHAPES = [(2, 1024, 512), (3, 1000, 96), (1, 777, 36), (2, 300, 7), (1, 1,
 @pytest.mark.parametrize("aligned", [True, False])
 @pytest.mark.parametrize("override", [(0, 0, 0), (1, 0, 1), (1, 0, 2), (1, 0, 4), (1, 0, 8),
                                       (2, 0, 2), (2, 0, 4), (2, 0, 8), (3, 0, 2), (3, 0, 4),
-                                      (3, 0, 8), (4, 0, 0), (5, 0, 0), (6, 0, 0), (7, 0, 0)])
+                                      (3, 0, 8), (4, 0, 0), (5, 0, 0), (6, 0, 0), (7, 0, 0),
+                                      (8, 0, 0)])
 def test_plan_indices_small(shape, dtype, aligned, override):
     lib = _abi.lib()
     assert lib.sgr_set_kernel_override(override[0]) == 0
@@ -631,6 +640,24 @@ def test_log_space_argument_errors():
     # a wide batch: the linear scan's header-only workspace is too small here
     assert scan(fn, A, Bp, None, 0, C, 16, 2048, 4096, BF16, 0x50000000, WS_HEADER, None) \
         == _abi.SGR_ERR_WORKSPACE
+
+
+def test_bf16_channel_sequential_kind_choice():
+    # B x 2048 x 4096 bf16 (B x 0.86 groups of 32 channels per SM): the minGRU
+    # takes two warps per 32 channels below 16 groups per SM, four warps per
+    # 64 channels up to 24, two per 64 channels above; MinMax four per 64
+    # channels throughout; fp32 never the 64-channel forms
+    for B, want in ((8, _abi.KERNEL_SEQUENTIAL_PAIR), (16, _abi.KERNEL_SEQUENTIAL_PAIR),
+                    (20, _abi.KERNEL_SEQUENTIAL_QUAD), (24, _abi.KERNEL_SEQUENTIAL_QUAD),
+                    (28, _abi.KERNEL_SEQUENTIAL_PAIR2), (32, _abi.KERNEL_SEQUENTIAL_PAIR2)):
+        assert _abi.plan(MINGRU, B, 2048, 4096, BF16, True)["kernel"] == want, B
+    for B in (8, 16, 32):
+        assert _abi.plan(_abi.SGR_OP_MINMAX, B, 2048, 4096, BF16, True)["kernel"] == _abi.KERNEL_SEQUENTIAL_QUAD, B
+    for B in (8, 16, 32):
+        assert _abi.plan(MINGRU, B, 2048, 4096, F32, True)["kernel"] in (_abi.KERNEL_SEQUENTIAL,
+                                                                          _abi.KERNEL_SEQUENTIAL_PAIR)
+        assert _abi.plan(_abi.SGR_OP_MINMAX, B, 2048, 4096, F32, True)["kernel"] in (_abi.KERNEL_SEQUENTIAL,
+                                                                                    _abi.KERNEL_SEQUENTIAL_PAIR)
 
 
 def test_minmax_plans_take_the_long_tiles():

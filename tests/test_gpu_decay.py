@@ -99,8 +99,10 @@ def test_decay_wide_batch(dtype, B, log1p_delta):
     T, D = 300, 2048
     code = _abi.SGR_F32 if dtype == "f32" else _abi.SGR_BF16
     pl = _abi.plan(_abi.SGR_OP_MINGRU, B, T, D, code, True, decay=True)
-    assert pl["kernel"] == _abi.plan(_abi.SGR_OP_MINGRU, B, T, D, code, True)["kernel"]
-    assert pl["kernel"] in (_abi.KERNEL_SEQUENTIAL, _abi.KERNEL_SEQUENTIAL_PAIR, _abi.KERNEL_SEQUENTIAL_PAIR2)
+    plain = _abi.plan(_abi.SGR_OP_MINGRU, B, T, D, code, True)["kernel"]
+    # bf16 from 16 groups per SM: four warps per 64-channel group
+    assert pl["kernel"] == (_abi.KERNEL_SEQUENTIAL_QUAD if dtype == "bf16" and B * D / 32 >= 16 * 148 else plain)
+    assert pl["kernel"] in (_abi.KERNEL_SEQUENTIAL, _abi.KERNEL_SEQUENTIAL_PAIR, _abi.KERNEL_SEQUENTIAL_QUAD)
     need = sgr.workspace_size("mingru", B, T, D, TORCH_DT[dtype])
     assert need >= pl["workspace_bytes"]
     k, hx, h0, dt, lam = data(B, T, D, dtype, "u01_1", seed=B, wipe_at=150,
@@ -182,7 +184,7 @@ def test_decay_workload_gradient_every_channel(log1p_delta):
 # the gap array allows it (16-byte aligned start, batch stride a multiple of
 # 4) and load them themselves otherwise: both, forward and gradient.
 @pytest.mark.parametrize("B,pad,gap_off", [(3, 0, 0), (3, 3, 0), (3, 1, 0), (3, 0, 1), (1, 0, 0)])
-@pytest.mark.parametrize("kernel", [4, 5, 6, 7])
+@pytest.mark.parametrize("kernel", [4, 5, 6, 7, 8])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_decay_sequential_gap_layouts(B, pad, gap_off, kernel, dtype):
     sgr.set_kernel_override(kernel)

@@ -118,7 +118,8 @@ def test_log_scan_plan_is_chunked_and_sized():
     B, T, D = 16, 2048, 4096
     lin = _abi.plan(_abi.SGR_OP_MINGRU, B, T, D, _abi.SGR_BF16)
     log = _abi.plan(_abi.SGR_OP_MINGRU_LOG, B, T, D, _abi.SGR_BF16)
-    assert lin["kernel"] in (_abi.KERNEL_SEQUENTIAL, _abi.KERNEL_SEQUENTIAL_PAIR, _abi.KERNEL_SEQUENTIAL_PAIR2)
+    assert lin["kernel"] in (_abi.KERNEL_SEQUENTIAL, _abi.KERNEL_SEQUENTIAL_PAIR, _abi.KERNEL_SEQUENTIAL_PAIR2,
+                             _abi.KERNEL_SEQUENTIAL_QUAD)
     assert log["kernel"] in (_abi.KERNEL_PIPELINED, _abi.KERNEL_PIPELINED_WIDE)
     assert sgr.workspace_size("mingru_log", B, T, D, torch.bfloat16) >= log["workspace_bytes"] > 256
     assert np.isfinite(log["n_tiles"])

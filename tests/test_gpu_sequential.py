@@ -32,9 +32,11 @@ if not torch.cuda.is_available():
 
 DEV = torch.device("cuda:0")
 SEQ = _abi.KERNEL_SEQUENTIAL
-# 7: two channels per lane, bf16 only (fp32 takes kind 6 under that override)
+# 7, 8: two channels per lane (two or four warps per group), bf16 only (fp32
+# takes kind 6 under those overrides)
 SEQ_KINDS = (_abi.KERNEL_SEQUENTIAL, _abi.KERNEL_SEQUENTIAL_SPLIT, _abi.KERNEL_SEQUENTIAL_PAIR,
-             _abi.KERNEL_SEQUENTIAL_PAIR2)
+             _abi.KERNEL_SEQUENTIAL_PAIR2, _abi.KERNEL_SEQUENTIAL_QUAD)
+WIDE_KINDS = (_abi.KERNEL_SEQUENTIAL_PAIR2, _abi.KERNEL_SEQUENTIAL_QUAD)
 
 
 @pytest.fixture(autouse=True)
@@ -71,7 +73,7 @@ SHAPES = [(2, 1, 64), (3, 17, 40), (2, 300, 96), (1, 1000, 200), (4, 129, 8), (2
 @pytest.mark.parametrize("kind", SEQ_KINDS)
 def test_mingru_sequential_matches_oracle(shape, dtype, init, kind):
     sgr.set_kernel_override(kind)
-    want = _abi.KERNEL_SEQUENTIAL_PAIR if (kind == _abi.KERNEL_SEQUENTIAL_PAIR2 and dtype == "f32") else kind
+    want = _abi.KERNEL_SEQUENTIAL_PAIR if (kind in WIDE_KINDS and dtype == "f32") else kind
     assert plan(*shape, dtype)["kernel"] == want
     k, hx, h0 = small("mingru", *shape, dtype, init, seed=sum(shape) % 97)
     h = sgr.mingru_scan(*dev(k, hx, h0))
@@ -205,7 +207,8 @@ def test_sequential_graph_capture_replays(kind):
 
 
 @pytest.mark.parametrize("kind,label", [(_abi.KERNEL_PIPELINED, "the chunked kernel"),
-                                        (_abi.KERNEL_SEQUENTIAL_PAIR2, "64-channel warp pairs")])
+                                        (_abi.KERNEL_SEQUENTIAL_PAIR2, "64-channel warp pairs"),
+                                        (_abi.KERNEL_SEQUENTIAL_QUAD, "64-channel groups of four warps")])
 def test_bf16_workload_other_kernels_still_match(kind, label):
     # the full-size bf16 workload through the chunked pipelined kernel and the
     # two-channels-per-lane kernel (the automatic choice there is the two-warp
