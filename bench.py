@@ -256,17 +256,32 @@ def aggregate(bytes_per_step: int, elems_per_step: int, steps: int, max_seconds:
 
 # ---------------------------------------------------------------- GPU timing
 
-def timed_launches(fn, steps: int, stream, while_busy=None):
+# GPU cycles of the spin queued ahead of a device-timed region (~50 us at
+# the B200's 1965 MHz boost clock)
+LEAD_CYCLES = 100_000
+
+
+def timed_launches(fn, steps: int, stream, while_busy=None, lead: bool = True):
     """Time `steps` calls of fn with CUDA events on the launching stream: the
     whole region and each launch.  Returns (total_s, mean_launch_s).
     `while_busy`, if given, is called on the host between the last launch
     being queued and the stream reaching its end (the clock sampler reads
     NVML there, so that its samples fall inside the timed region however
-    short it is)."""
+    short it is).  lead: a short GPU spin is queued before the start event,
+    so that the host has queued the first launches by the time the stream
+    reaches it; otherwise, after the synchronize that precedes every timed
+    region, the first interval would hold the host's ~20 us of launch
+    latency on an idle GPU as well as the kernel (measured: the first of 20
+    back-to-back launches 100 us against 76 us for the rest).  Off for the
+    end-to-end and per-call timings, whose host work is part of what they
+    measure."""
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    if lead:
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(LEAD_CYCLES)
     t0.record(stream)
     for i in range(steps):
         starts[i].record(stream)
@@ -574,7 +589,7 @@ def measure_step_row(device, B=8, D=1024, calls=200, warmup=10):
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
-    total, per = timed_launches(fn, calls, torch.cuda.current_stream(device))
+    total, per = timed_launches(fn, calls, torch.cuda.current_stream(device), lead=False)
     # the same steps replayed from a CUDA graph: the device-side time of one
     # step without the host's per-call overhead (token-by-token decoding
     # captures its step loop the same way)
@@ -808,7 +823,7 @@ def run_b200(args):
         torch.cuda.synchronize()
         barrier(world, device)
         e_steps = max(1, min(args.steps, 10))
-        et, _ = timed_launches(e2e_step, e_steps, stream)
+        et, _ = timed_launches(e2e_step, e_steps, stream, lead=False)
         barrier(world, device)
         et = reduce_max(et, world, device)
         h2d = hp.numel() * hp.element_size() + hq.numel() * hq.element_size() + \

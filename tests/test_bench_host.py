@@ -102,11 +102,14 @@ def test_timed_launches_samples_until_the_stream_is_done(monkeypatch):
 
     monkeypatch.setattr(bench.torch.cuda, "Event", Ev)
     monkeypatch.setattr(bench.torch.cuda, "synchronize", lambda: None)
+    spins = []
+    monkeypatch.setattr(bench.torch.cuda, "_sleep", lambda cycles: spins.append(cycles))
     calls, seen = [], []
     total, per = bench.timed_launches(lambda: calls.append(1), 3, None, while_busy=lambda: seen.append(1))
     assert len(calls) == 3 and len(seen) == 4
     assert total == 2e-3 and per == 2e-3
+    assert spins == [bench.LEAD_CYCLES]                      # one spin ahead of the start event
     Ev.polls = 0
-    bench.timed_launches(lambda: None, 2, None)             # no sampler: no queries
-    assert Ev.polls == 0
+    bench.timed_launches(lambda: None, 2, None, lead=False)  # no sampler: no queries; no spin
+    assert Ev.polls == 0 and spins == [bench.LEAD_CYCLES]
 
