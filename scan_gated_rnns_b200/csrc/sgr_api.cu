@@ -29,6 +29,11 @@ constexpr int kWarps = 7;
 constexpr int kPipeWarps = 7;        // two blocks per SM
 constexpr int kPipeWarpsWide = 15;   // one block per SM, tiles twice as long
 constexpr int kStages = 3;
+// the fp32 time-decayed gradient: two blocks of 6 data warps + 1 carry warp per
+// SM, 4 rows per thread, a 2-slot ring (three slots of its 96-row tiles
+// would not leave room for a second block)
+constexpr int kPipeWarpsDecayBwd = 6;
+constexpr int kStagesDecayBwd = 2;
 constexpr int kAssumedSMs = 148;     // B200; only used to pick a tile shape
 constexpr int64_t kTargetTiles = 4 * 148;  // tile kernel: prefer >= 4 tiles per SM
 constexpr size_t kAlign = 256;
@@ -1036,23 +1041,33 @@ bool seq_backward_planned(int64_t B, int64_t T, int64_t D, int esz, bool aligned
 // channel tiles give the blocks in flight little look-back depth (fp32 B8 x
 // 4096 x 1024, 256 chains: 187 against 195 us; bf16, 128 chains: 142
 // against 150) and the 15-warp ones where the depth grows (fp32 B4 x 8192 x
-// 768, 96 chains: 150 against 158 us).  The fp32 decayed gradient takes
-// 7-warp blocks with 4 rows per thread (16 elements, one block per SM,
-// 112-row tiles) at any chain count: the per-tile work is spread over twice
-// the elements, measured 182.8 against 186.5 us (7-warp, 2 rows) and 193.1
-// (15-warp) on B8 x 4096 x 1024, 143.9 against 156.7 and 149.5 on
-// B4 x 8192 x 768, 188.9 against 197.2 and 194.1 on B2 x 8192 x 2048.
+// 768, 96 chains: 150 against 158 us).  The fp32 decayed gradient takes 4
+// rows per thread (16 elements: the per-tile work is spread over twice the
+// elements) in blocks of 6 data warps + 1 carry warp, two per SM (96-row
+// tiles, a 2-slot ring of about 49 KB slots, 128 registers per thread):
+// with 12 data warps per SM instead of 7 the latency each one exposes is
+// hidden, measured 154.0 against 184.6 us for one 7-warp block per SM with
+// 4 rows (override 2) on B8 x 4096 x 1024, 126.4 against 143.7 on
+// B4 x 8192 x 768, 370.5 against 472.4 on B1 x 131072 x 512 (the 7-warp,
+// 4-row blocks had measured 182.8 against 186.5 us for 2 rows and 193.1
+// for 15-warp blocks on B8 x 4096 x 1024).
 template <typename IO, bool DECAY = false, int W = kPipeWarpsWide>
-constexpr int bwd_pipe_r() { return (sizeof(IO) == 2 || (DECAY && W == kPipeWarps)) ? 4 : 2; }
+constexpr int bwd_pipe_r() {
+    return (sizeof(IO) == 2 || (DECAY && (W == kPipeWarps || W == kPipeWarpsDecayBwd))) ? 4 : 2;
+}
 template <typename IO, bool DECAY, int W>
-constexpr int bwd_pipe_minb() { return (W == kPipeWarps && !(sizeof(IO) == 4 && DECAY)) ? 2 : 1; }
+constexpr int bwd_pipe_minb() {
+    return W == kPipeWarpsDecayBwd || (W == kPipeWarps && !(sizeof(IO) == 4 && DECAY)) ? 2 : 1;
+}
+template <int W>
+constexpr int bwd_pipe_stages() { return W == kPipeWarpsDecayBwd ? kStagesDecayBwd : kStages; }
 template <typename IO, bool DT = false, int W = kPipeWarpsWide, bool DECAY = false>
-using BwdPipeShape = PipeBwdShape<IO, 4, pipe_cg<IO>(), bwd_pipe_r<IO, DECAY, W>(), kStages, W, DT>;
+using BwdPipeShape = PipeBwdShape<IO, 4, pipe_cg<IO>(), bwd_pipe_r<IO, DECAY, W>(), bwd_pipe_stages<W>(), W, DT>;
 
 // The gradient's tile plan: the pipelined kernel for aligned vector-width
 // rows with at least two tiles per SM (override 2 or 3 forces it wherever the
 // rows allow), else the ticketed tile kernel (make_plan with force_tile).
-// decay: the time-decayed gradient (7-warp blocks).
+// decay: the time-decayed gradient (fp32: two 6-warp blocks per SM).
 Plan make_bwd_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned, bool decay = false) {
     const int esz = dtype == SGR_BF16 ? 2 : 4;
     const int vw = 16 / esz;
@@ -1069,18 +1084,24 @@ Plan make_bwd_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool alig
         p.stages = kStages;
         // blocks of 15 data warps, one per SM, or of 7, two per SM (override
         // 2; bf16 decay with at least 0.8 chains per SM); the fp32 decayed
-        // gradient always takes 7-warp blocks, one per SM with 4 rows per
-        // thread
+        // gradient takes 4 rows per thread: two 6-warp blocks per SM, or
+        // under override 2 one 7-warp block per SM
         const int64_t chains = B * ((D + (esz == 4 ? 32 : 64) - 1) / (esz == 4 ? 32 : 64));
         const bool narrow = ok == KIND_PIPELINED ||
                             (ok == KIND_AUTO && decay && (esz == 4 || 5 * chains >= 4 * kAssumedSMs));
         p.warps = narrow ? kPipeWarps : kPipeWarpsWide;
         p.r = (esz == 2 || (decay && narrow)) ? 4 : 2;
+        // the fp32 decayed gradient by default: two 6-warp blocks per SM
+        if (esz == 4 && decay && ok == KIND_AUTO) {
+            p.warps = kPipeWarpsDecayBwd;
+            p.stages = kStagesDecayBwd;
+        }
         p.TR = p.warps * (32 / p.cg) * p.r;
         if (esz == 4)
-            p.smem = narrow ? (decay ? BwdPipeShape<float, false, kPipeWarps, true>::smem_bytes
-                                     : BwdPipeShape<float, false, kPipeWarps>::smem_bytes)
-                            : BwdPipeShape<float>::smem_bytes;
+            p.smem = p.warps == kPipeWarpsDecayBwd ? BwdPipeShape<float, false, kPipeWarpsDecayBwd, true>::smem_bytes
+                     : narrow ? (decay ? BwdPipeShape<float, false, kPipeWarps, true>::smem_bytes
+                                       : BwdPipeShape<float, false, kPipeWarps>::smem_bytes)
+                              : BwdPipeShape<float>::smem_bytes;
         else
             p.smem = narrow ? BwdPipeShape<__nv_bfloat16, false, kPipeWarps>::smem_bytes
                             : BwdPipeShape<__nv_bfloat16>::smem_bytes;
@@ -1103,7 +1124,8 @@ cudaError_t launch_pipelined_bwd_shape(const BwdParams &bp, const CUtensorMap (&
     constexpr int CG = pipe_cg<IO>();
     constexpr int R = bwd_pipe_r<IO, BOp::kDecay, W>();
     using Shape = BwdPipeShape<IO, DT, W, BOp::kDecay>;
-    auto kernel = scan_pipelined_backward_kernel<BOp, IO, 4, CG, R, kStages, W, bwd_pipe_minb<IO, BOp::kDecay, W>(), DT>;
+    auto kernel = scan_pipelined_backward_kernel<BOp, IO, 4, CG, R, bwd_pipe_stages<W>(), W,
+                                                 bwd_pipe_minb<IO, BOp::kDecay, W>(), DT>;
     constexpr size_t smem = Shape::smem_bytes;
     constexpr int NT = (W + 1) * 32;
     int dev = 0;
@@ -1161,9 +1183,13 @@ cudaError_t launch_pipelined_bwd(const BwdParams &bp, cudaStream_t s) {
 template <class BOp, typename IO>
 cudaError_t dispatch_bwd(const Plan &pl, const BwdParams &bp, cudaStream_t s) {
     constexpr int VW = 16 / int(sizeof(IO));
-    if (pl.kind == KIND_PIPELINED)
+    if (pl.kind == KIND_PIPELINED) {
+        if constexpr (BOp::kDecay && sizeof(IO) == 4) {
+            if (pl.warps == kPipeWarpsDecayBwd) return launch_pipelined_bwd<BOp, IO, kPipeWarpsDecayBwd>(bp, s);
+        }
         return pl.warps == kPipeWarps ? launch_pipelined_bwd<BOp, IO, kPipeWarps>(bp, s)
                                       : launch_pipelined_bwd<BOp, IO, kPipeWarpsWide>(bp, s);
+    }
     if (!pl.vec) return dispatch_bwd_r<BOp, IO, 1, 32>(pl, bp, s);
     return dispatch_bwd_r<BOp, IO, VW, 8>(pl, bp, s);
 }

@@ -742,3 +742,40 @@ def test_pipelined_backward_indices(shape, dtype, override, W):
             for v in range(V):
                 np.add.at(cover, (b2, tt, d2 + v), 1)
         assert (cover == 1).all(), "every element's gradient is written exactly once"
+
+
+@pytest.mark.parametrize("shape", [(8, 4096, 1024), (4, 8192, 768), (1, 131072, 512), (3, 2501, 160)])
+def test_decayed_fp32_gradient_plan(shape):
+    """The fp32 time-decayed gradient's automatic plan: blocks of 6 data warps
+    + 1 carry warp, two per SM, 4 rows per thread (96-row tiles) and a 2-slot
+    ring.  Two blocks' shared memory fit an SM, a tile's gap box starts on a
+    16-byte boundary, the tiles cover every time row once, and the workspace
+    size covers its hand-off words."""
+    B, T, D = shape
+    W, R, S, cg, V = 6, 4, 2, 8, 4
+    J = 32 // cg
+    TC, TR = cg * V, W * J * R
+    assert TR == 96 and TR % 4 == 0          # the gaps' box starts at ct TR: a 16-byte multiple
+    n_dt, n_chunks = -(-D // TC), -(-T // TR)
+    n_tiles = B * n_dt * n_chunks
+    # the kernel's shared-memory layout: S slots (four operand boxes, then TC
+    # rates and TR gaps), mbarriers, reader counts, warp and tile summaries,
+    # incoming gradients, dL/dlambda sums and their warp count
+    slot = -(-(4 * TR * TC * 4 + (TR + TC) * 4) // 128) * 128
+    cnt = S * slot + S * 8
+    tot = -(-(cnt + S * 4) // 16) * 16
+    smem = tot + 2 * W * TC * 8 + 2 * TC * 8 + 2 * TC * 4 + 2 * TC * 4 + 16
+    assert 2 * (smem + 1024) <= 228 * 1024          # two blocks per SM, 1 KB reserved each
+    assert 2 * (W + 1) * 32 * 128 <= 65536          # at 128 registers per thread
+    # processing rows of a tile: every time row of a chain exactly once
+    rows = np.zeros(n_chunks * TR, dtype=np.int32)
+    for ct in range(n_chunks):
+        for w in range(W):
+            for j in range(J):
+                rho0 = (w * J + j) * R
+                top = ct * TR + TR - 1 - rho0
+                rows[top - R + 1:top + 1] += 1
+    assert (rows == 1).all()
+    need = _abi.lib().sgr_backward_workspace_size(MINGRU, B, T, D, F32)
+    if n_chunks > 1 and n_tiles >= 2 * 148:
+        assert need >= WS_HEADER + 8 * 3 * TC * n_tiles
