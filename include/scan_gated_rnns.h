@@ -537,18 +537,24 @@ SGR_API sgr_status_t sgr_scan_plan(sgr_op_t op, int64_t B, int64_t T, int64_t D,
                                    sgr_dtype_t dtype, int aligned, sgr_plan_t *plan);
 
 /* The plan of mingru_scan_decay for this shape (the time-decayed minGRU may
- * take another kernel than sgr_scan_plan(SGR_OP_MINGRU, ...) reports: never
- * the channel-sequential one, 4 rows per thread).  `aligned` as above.  Pure
- * host code. */
+ * take another kernel than sgr_scan_plan(SGR_OP_MINGRU, ...) reports, with
+ * bf16 I/O only: four warps per 64-channel group from 16 groups of 32
+ * channels per SM, and 8 rows per thread in 7-warp blocks of the chunked
+ * kernels).  `aligned` as above.
+ * Pure host code. */
 SGR_API sgr_status_t sgr_scan_plan_decay(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype,
                                          int aligned, sgr_plan_t *plan);
 
 /* Which kernel the gradient of this shape runs (mingru_scan_backward,
  * minmax_scan_backward and their time-decay forms): 1 the chunked tile kernel
  * (blocks take chunks by ticket), 2 the pipelined gradient (persistent blocks
- * fed by the copy engine; aligned vector-width rows with at least two tiles of
- * 120 rows per SM; the decayed gradient runs tiles of 56 rows, two blocks per
- * SM), 4 the channel-sequential kernel (wide batches, from 5 groups of 32
+ * fed by the copy engine; aligned vector-width rows with at least two tiles
+ * per block: fp32 two blocks of 6 data warps per SM with 96-row tiles for the
+ * decayed gradient and, below 1.5 chains of 32 channels per SM, the plain
+ * ones, else one block of 15 data warps per SM with 120-row tiles; the
+ * fp32 decayed gradient with too few tiles for two blocks takes one 7-warp
+ * block per SM with 112-row tiles, the bf16 one two 7-warp blocks per SM with
+ * 56-row tiles from 0.8 chains per SM), 4 the channel-sequential kernel (wide batches, from 5 groups of 32
  * channels per SM: one warp walks the whole sequence of 32 channels
  * backwards); 0 for invalid arguments.
  * `aligned` says whether all six (B, T, D) operands would be 16-byte aligned.

@@ -29,11 +29,11 @@ constexpr int kWarps = 7;
 constexpr int kPipeWarps = 7;        // two blocks per SM
 constexpr int kPipeWarpsWide = 15;   // one block per SM, tiles twice as long
 constexpr int kStages = 3;
-// the fp32 time-decayed gradient: two blocks of 6 data warps + 1 carry warp per
-// SM, 4 rows per thread, a 2-slot ring (three slots of its 96-row tiles
+// the fp32 pipelined gradients: two blocks of 6 data warps + 1 carry warp per
+// SM, 4 rows per thread, a 2-slot ring (three slots of their 96-row tiles
 // would not leave room for a second block)
-constexpr int kPipeWarpsDecayBwd = 6;
-constexpr int kStagesDecayBwd = 2;
+constexpr int kBwdPairWarps = 6;
+constexpr int kBwdPairStages = 2;
 constexpr int kAssumedSMs = 148;     // B200; only used to pick a tile shape
 constexpr int64_t kTargetTiles = 4 * 148;  // tile kernel: prefer >= 4 tiles per SM
 constexpr size_t kAlign = 256;
@@ -1050,24 +1050,33 @@ bool seq_backward_planned(int64_t B, int64_t T, int64_t D, int esz, bool aligned
 // 4 rows (override 2) on B8 x 4096 x 1024, 126.4 against 143.7 on
 // B4 x 8192 x 768, 370.5 against 472.4 on B1 x 131072 x 512 (the 7-warp,
 // 4-row blocks had measured 182.8 against 186.5 us for 2 rows and 193.1
-// for 15-warp blocks on B8 x 4096 x 1024).
+// for 15-warp blocks on B8 x 4096 x 1024).  The plain fp32 gradients take
+// the same blocks below 1.5 chains per SM (us, two 6-warp blocks against
+// one 15-warp block, minGRU / MinMax): B4 x 8192 x 768 111.1 / 109.2
+// against 119.3 / 116.2, B1 x 131072 x 512 307.7 / 301.7 against
+// 371.2 / 361.1; at B8 x 4096 x 1024 (1.7 chains per SM) 143.3 / 143.8
+// against 139.5 / 147.3.
 template <typename IO, bool DECAY = false, int W = kPipeWarpsWide>
 constexpr int bwd_pipe_r() {
-    return (sizeof(IO) == 2 || (DECAY && (W == kPipeWarps || W == kPipeWarpsDecayBwd))) ? 4 : 2;
+    return (sizeof(IO) == 2 || W == kBwdPairWarps || (DECAY && W == kPipeWarps)) ? 4 : 2;
 }
 template <typename IO, bool DECAY, int W>
 constexpr int bwd_pipe_minb() {
-    return W == kPipeWarpsDecayBwd || (W == kPipeWarps && !(sizeof(IO) == 4 && DECAY)) ? 2 : 1;
+    return W == kBwdPairWarps || (W == kPipeWarps && !(sizeof(IO) == 4 && DECAY)) ? 2 : 1;
 }
 template <int W>
-constexpr int bwd_pipe_stages() { return W == kPipeWarpsDecayBwd ? kStagesDecayBwd : kStages; }
+constexpr int bwd_pipe_stages() { return W == kBwdPairWarps ? kBwdPairStages : kStages; }
 template <typename IO, bool DT = false, int W = kPipeWarpsWide, bool DECAY = false>
 using BwdPipeShape = PipeBwdShape<IO, 4, pipe_cg<IO>(), bwd_pipe_r<IO, DECAY, W>(), bwd_pipe_stages<W>(), W, DT>;
 
 // The gradient's tile plan: the pipelined kernel for aligned vector-width
-// rows with at least two tiles per SM (override 2 or 3 forces it wherever the
-// rows allow), else the ticketed tile kernel (make_plan with force_tile).
-// decay: the time-decayed gradient (fp32: two 6-warp blocks per SM).
+// rows with at least two tiles per block (override 2 or 3 forces it wherever
+// the rows allow), else the ticketed tile kernel (make_plan with force_tile).
+// fp32 takes two 6-warp blocks per SM where that gives every block two
+// tiles -- the decayed gradient at any chain count, the plain ones below 1.5
+// chains of 32 channels per SM -- else (and under an override) the blocks
+// below.
+// decay: the time-decayed gradient.
 Plan make_bwd_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool aligned, bool decay = false) {
     const int esz = dtype == SGR_BF16 ? 2 : 4;
     const int vw = 16 / esz;
@@ -1081,39 +1090,45 @@ Plan make_bwd_plan(int64_t B, int64_t T, int64_t D, sgr_dtype_t dtype, bool alig
         p.V = 4;
         p.cg = esz == 4 ? 8 : 16;
         p.TC = p.cg * p.V;
-        p.stages = kStages;
-        // blocks of 15 data warps, one per SM, or of 7, two per SM (override
-        // 2; bf16 decay with at least 0.8 chains per SM); the fp32 decayed
-        // gradient takes 4 rows per thread: two 6-warp blocks per SM, or
-        // under override 2 one 7-warp block per SM
-        const int64_t chains = B * ((D + (esz == 4 ? 32 : 64) - 1) / (esz == 4 ? 32 : 64));
-        const bool narrow = ok == KIND_PIPELINED ||
-                            (ok == KIND_AUTO && decay && (esz == 4 || 5 * chains >= 4 * kAssumedSMs));
-        p.warps = narrow ? kPipeWarps : kPipeWarpsWide;
-        p.r = (esz == 2 || (decay && narrow)) ? 4 : 2;
-        // the fp32 decayed gradient by default: two 6-warp blocks per SM
-        if (esz == 4 && decay && ok == KIND_AUTO) {
-            p.warps = kPipeWarpsDecayBwd;
-            p.stages = kStagesDecayBwd;
-        }
-        p.TR = p.warps * (32 / p.cg) * p.r;
-        if (esz == 4)
-            p.smem = p.warps == kPipeWarpsDecayBwd ? BwdPipeShape<float, false, kPipeWarpsDecayBwd, true>::smem_bytes
-                     : narrow ? (decay ? BwdPipeShape<float, false, kPipeWarps, true>::smem_bytes
-                                       : BwdPipeShape<float, false, kPipeWarps>::smem_bytes)
-                              : BwdPipeShape<float>::smem_bytes;
-        else
-            p.smem = narrow ? BwdPipeShape<__nv_bfloat16, false, kPipeWarps>::smem_bytes
-                            : BwdPipeShape<__nv_bfloat16>::smem_bytes;
         p.n_dt = (D + p.TC - 1) / p.TC;
         p.n_chains = B * p.n_dt;
-        p.n_chunks = (T + p.TR - 1) / p.TR;
-        p.n_tiles = p.n_chains * p.n_chunks;
-        if (p.n_tiles > 0) {
-            p.off_words = kAlign;
-            p.ws_bytes = kAlign;
-            if (p.n_chunks > 1) p.ws_bytes = align_up(p.off_words + size_t(p.n_tiles) * 3 * p.TC * 8, kAlign);
+        // tiles of `warps` data warps x (32 / cg) row groups x r rows
+        auto shape = [&](int warps, int r, int stages, size_t smem) {
+            p.warps = warps;
+            p.r = r;
+            p.stages = stages;
+            p.smem = smem;
+            p.TR = warps * (32 / p.cg) * r;
+            p.n_chunks = (T + p.TR - 1) / p.TR;
+            p.n_tiles = p.n_chains * p.n_chunks;
+            p.off_words = 0;
+            p.ws_bytes = 0;
+            if (p.n_tiles > 0) {
+                p.off_words = kAlign;
+                p.ws_bytes = kAlign;
+                if (p.n_chunks > 1) p.ws_bytes = align_up(p.off_words + size_t(p.n_tiles) * 3 * p.TC * 8, kAlign);
+            }
+        };
+        const int64_t chains = B * ((D + (esz == 4 ? 32 : 64) - 1) / (esz == 4 ? 32 : 64));
+        if (esz == 4 && ok == KIND_AUTO && (decay || 2 * chains < 3 * kAssumedSMs)) {
+            shape(kBwdPairWarps, 4, kBwdPairStages, BwdPipeShape<float, false, kBwdPairWarps>::smem_bytes);
+            if (p.n_tiles >= 4 * kAssumedSMs) return p;
         }
+        // blocks of 15 data warps, one per SM, or of 7, two per SM (override
+        // 2; bf16 decay with at least 0.8 chains per SM); the fp32 decayed
+        // gradient with 7-warp blocks takes 4 rows per thread, one block per SM
+        const bool narrow = ok == KIND_PIPELINED ||
+                            (ok == KIND_AUTO && decay && (esz == 4 || 5 * chains >= 4 * kAssumedSMs));
+        const int r = (esz == 2 || (decay && narrow)) ? 4 : 2;
+        size_t smem;
+        if (esz == 4)
+            smem = narrow ? (decay ? BwdPipeShape<float, false, kPipeWarps, true>::smem_bytes
+                                   : BwdPipeShape<float, false, kPipeWarps>::smem_bytes)
+                          : BwdPipeShape<float>::smem_bytes;
+        else
+            smem = narrow ? BwdPipeShape<__nv_bfloat16, false, kPipeWarps>::smem_bytes
+                          : BwdPipeShape<__nv_bfloat16>::smem_bytes;
+        shape(narrow ? kPipeWarps : kPipeWarpsWide, r, kStages, smem);
         if (ok != KIND_AUTO || p.n_tiles >= 2 * kAssumedSMs) return p;
     }
     return make_plan(B, T, D, dtype, aligned, true);
@@ -1184,8 +1199,8 @@ template <class BOp, typename IO>
 cudaError_t dispatch_bwd(const Plan &pl, const BwdParams &bp, cudaStream_t s) {
     constexpr int VW = 16 / int(sizeof(IO));
     if (pl.kind == KIND_PIPELINED) {
-        if constexpr (BOp::kDecay && sizeof(IO) == 4) {
-            if (pl.warps == kPipeWarpsDecayBwd) return launch_pipelined_bwd<BOp, IO, kPipeWarpsDecayBwd>(bp, s);
+        if constexpr (sizeof(IO) == 4) {
+            if (pl.warps == kBwdPairWarps) return launch_pipelined_bwd<BOp, IO, kBwdPairWarps>(bp, s);
         }
         return pl.warps == kPipeWarps ? launch_pipelined_bwd<BOp, IO, kPipeWarps>(bp, s)
                                       : launch_pipelined_bwd<BOp, IO, kPipeWarpsWide>(bp, s);

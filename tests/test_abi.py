@@ -596,7 +596,7 @@ def test_backward_kernel_choice():
     assert lib.sgr_backward_kernel(MINGRU, 2, 2048, 4096, BF16, 1) == 2      # 256 groups, 2304 tiles
     assert lib.sgr_backward_kernel(MINGRU, 8, 4096, 1024, F32, 1) == 2       # 256 groups, 8960 tiles
     assert lib.sgr_backward_kernel(_abi.SGR_OP_MINMAX, 4, 8192, 768, F32, 1) == 2
-    assert lib.sgr_backward_kernel(MINGRU, 2, 1024, 512, F32, 1) == 1       # 288 tiles: one launch per tile
+    assert lib.sgr_backward_kernel(MINGRU, 2, 1024, 512, F32, 1) == 1       # 352 tiles of 96 rows, 288 of 120
     assert lib.sgr_backward_kernel(MINGRU, 8, 4096, 1024, F32, 0) == 1       # unaligned
     assert lib.sgr_backward_kernel(MINGRU, 16, 2048, 4096, BF16, 0) == 1     # unaligned
     assert lib.sgr_backward_kernel(MINGRU, 16, 2048, 4100, BF16, 1) == 1     # D not a vector multiple
@@ -744,13 +744,16 @@ def test_pipelined_backward_indices(shape, dtype, override, W):
         assert (cover == 1).all(), "every element's gradient is written exactly once"
 
 
-@pytest.mark.parametrize("shape", [(8, 4096, 1024), (4, 8192, 768), (1, 131072, 512), (3, 2501, 160)])
-def test_decayed_fp32_gradient_plan(shape):
-    """The fp32 time-decayed gradient's automatic plan: blocks of 6 data warps
-    + 1 carry warp, two per SM, 4 rows per thread (96-row tiles) and a 2-slot
-    ring.  Two blocks' shared memory fit an SM, a tile's gap box starts on a
-    16-byte boundary, the tiles cover every time row once, and the workspace
-    size covers its hand-off words."""
+@pytest.mark.parametrize("shape", [(8, 4096, 1024), (4, 8192, 768), (1, 131072, 512), (3, 2501, 640),
+                                   (3, 2501, 160)])
+def test_fp32_gradient_pair_plan(shape):
+    """The fp32 gradients' automatic plan where it gives every block two
+    tiles (the decayed gradient at any chain count, the plain ones below 1.5
+    chains of 32 channels per SM): blocks of 6 data warps + 1 carry warp, two
+    per SM, 4 rows per thread (96-row tiles) and a 2-slot ring.  Two blocks' shared memory (with
+    the time decay's rates and gaps in every slot) fit an SM, a tile's gap box
+    starts on a 16-byte boundary, the tiles cover every time row once, and
+    the workspace size covers the hand-off words."""
     B, T, D = shape
     W, R, S, cg, V = 6, 4, 2, 8, 4
     J = 32 // cg
@@ -776,6 +779,10 @@ def test_decayed_fp32_gradient_plan(shape):
                 top = ct * TR + TR - 1 - rho0
                 rows[top - R + 1:top + 1] += 1
     assert (rows == 1).all()
-    need = _abi.lib().sgr_backward_workspace_size(MINGRU, B, T, D, F32)
-    if n_chunks > 1 and n_tiles >= 2 * 148:
-        assert need >= WS_HEADER + 8 * 3 * TC * n_tiles
+    lib = _abi.lib()
+    kind = lib.sgr_backward_kernel(MINGRU, B, T, D, F32, 1)
+    wide = B * n_dt * -(-T // 120) >= 2 * 148     # 15-warp blocks, 120-row tiles
+    if n_tiles >= 4 * 148:                   # two tiles per block: the decayed gradient's plan
+        assert lib.sgr_backward_workspace_size(MINGRU, B, T, D, F32) >= WS_HEADER + 8 * 3 * TC * n_tiles
+    # the plain gradient (what the kernel query reports)
+    assert kind == (2 if (n_tiles >= 4 * 148 and 2 * B * n_dt < 3 * 148) or wide else 1)

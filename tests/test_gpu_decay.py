@@ -128,7 +128,9 @@ def test_decay_gap_layouts(B, pad, gap_off, lam_off, kernel, dtype):
         pytest.skip("the automatic bf16 plans take the tile kernels at this size")
     sgr.set_kernel_override(kernel)
     sgr.set_tile_override(0, 4)
-    T, D = 2501, 160
+    # the automatic fp32 plan takes two 6-warp blocks per SM from two tiles
+    # per block (592 tiles of 96 rows): 3 x 20 chains of 32 channels
+    T, D = 2501, 640 if kernel == 0 else 160
     k, hx, h0, dt, lam = data(B, T, D, dtype, "u01_1", seed=11 + pad + gap_off + lam_off, wipe_at=1200)
     gstore = torch.full((B, T + pad + gap_off), float("nan"), device=DEV)
     gaps = gstore[:, gap_off:gap_off + T]
@@ -140,11 +142,10 @@ def test_decay_gap_layouts(B, pad, gap_off, lam_off, kernel, dtype):
     torch.cuda.synchronize()
     assert rel_err(h, oracle.mingru_decay(k, hx, h0, dt, lam)) <= TOL[dtype]
     # the pipelined gradient (2: 7-warp blocks, 3: 15-warp blocks; 0: the
-    # automatic plan, for fp32 two 6-warp blocks per SM where the three batch
-    # rows give it enough tiles, else the tile kernel) with the same layouts:
-    # gaps and rates in its ring slots or by plain loads
-    want = 2 if kernel or B == 3 else 1
-    assert _abi.lib().sgr_backward_kernel(0, B, T, D, _abi.SGR_F32 if dtype == "f32" else _abi.SGR_BF16, 1) == want
+    # automatic plan, two 6-warp blocks per SM with three batch rows, one
+    # 7-warp block per SM with one) with the same layouts: gaps and rates in
+    # its ring slots or by plain loads
+    assert _abi.lib().sgr_backward_kernel(0, B, T, D, _abi.SGR_F32 if dtype == "f32" else _abi.SGR_BF16, 1) == 2
     g = torch.Generator().manual_seed(13 + pad)
     gy = torch.randn(B, T, D, generator=g).to(TORCH_DT[dtype])
     fwd = torch.from_numpy(oracle.mingru_decay(k, hx, h0, dt, lam)).to(TORCH_DT[dtype])
