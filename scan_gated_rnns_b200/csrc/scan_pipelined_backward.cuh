@@ -265,7 +265,9 @@ scan_pipelined_backward_kernel(const BwdParams bp, const __grid_constant__ CUten
                     const float2 f2 = make_float2(xf[2 * i], xf[2 * i + 1]);
                     float2 a, cp, cq;
                     if constexpr (kDec) {
-                        const float2 gam = make_float2(decay_gamma(lam2[2 * i], u), decay_gamma(lam2[2 * i + 1], u));
+                        // the two gates' exponents in one packed multiply
+                        const float2 ge = __fmul2_rn(make_float2(lam2[2 * i], lam2[2 * i + 1]), make_float2(u, u));
+                        const float2 gam = make_float2(fast_exp2(ge.x), fast_exp2(ge.y));
                         BOp::coeffs_gated2(k2, h2, f2, gam, a, cp, cq);
                         // dL/dlambda gains delta A h_{t-1} (-u) = (A delta) (-u h_{t-1}):
                         // the second factor here, the first in phase B

@@ -123,6 +123,12 @@ __device__ __forceinline__ float seq_slot_gap(const ScanParams &p, int64_t b, in
     const int64_t t = y0 + (lane & (kSeqRows - 1));
     return (y0 >= 0 && t < p.T) ? decay_u(p, b, t) : 0.f;
 }
+// the decay gates of two elements with their exponents in one packed
+// multiply: (2^(l.x u.x), 2^(l.y u.y)), each product as decay_gamma's
+__device__ __forceinline__ float2 decay_gamma2(float2 l, float2 u) {
+    const float2 e = __fmul2_rn(l, u);
+    return make_float2(fast_exp2(e.x), fast_exp2(e.y));
+}
 // the same gap from a slot's gap area (rows past T were zero-filled: gamma = 1)
 __device__ __forceinline__ float seq_smem_gap(const ScanParams &p, uint32_t gaps, int lane) {
     float g;
@@ -261,8 +267,9 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
                 float2 a, c;
                 seq_rows<Op, IO>(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
                 if constexpr (Op::kDecay) {
-                    a.x *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r));
-                    a.y *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r + 1));
+                    a = __fmul2_rn(a, decay_gamma2(make_float2(lam2, lam2),
+                                                   make_float2(__shfl_sync(0xffffffffu, gcur, r),
+                                                               __shfl_sync(0xffffffffu, gcur, r + 1))));
                 }
                 h = Op::step(a.x, c.x, h);
                 LR::store(dst + r * kRowBytes, h);
@@ -278,8 +285,9 @@ scan_sequential_kernel(const SeqParams q, const __grid_constant__ CUtensorMap ma
                 float2 a, c;
                 seq_rows<Op, IO>(x0r[r], x1r[r], x0r[r + 1], x1r[r + 1], a, c);
                 if constexpr (Op::kDecay) {
-                    a.x *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, part * LROWS + r));
-                    a.y *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, part * LROWS + r + 1));
+                    a = __fmul2_rn(a, decay_gamma2(make_float2(lam2, lam2),
+                                                   make_float2(__shfl_sync(0xffffffffu, gcur, part * LROWS + r),
+                                                               __shfl_sync(0xffffffffu, gcur, part * LROWS + r + 1))));
                 }
                 am[r] = a.x; cm[r] = c.x;
                 am[r + 1] = a.y; cm[r + 1] = c.y;
@@ -446,8 +454,9 @@ scan_sequential_pair_kernel(const SeqParams q, const __grid_constant__ CUtensorM
             float2 a, c;
             seq_rows<Op, IO>(x0r[r], x1r[r], x0r[r + H], x1r[r + H], a, c);
             if constexpr (Op::kDecay) {
-                a.x *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r));
-                a.y *= decay_gamma(lam2, __shfl_sync(0xffffffffu, gcur, r + H));
+                a = __fmul2_rn(a, decay_gamma2(make_float2(lam2, lam2),
+                                               make_float2(__shfl_sync(0xffffffffu, gcur, r),
+                                                           __shfl_sync(0xffffffffu, gcur, r + H))));
             }
             Op::fold2(A, Bc, a, c);
             PA[r] = A;
@@ -640,8 +649,8 @@ scan_sequential_pair2_kernel(const SeqParams q, const __grid_constant__ CUtensor
             seq_rows<Op, IO>(ku.x, hu.x, ku.y, hu.y, au, cu);
             if constexpr (Op::kDecay) {
                 const float ul = __shfl_sync(0xffffffffu, gcur, r), uu = __shfl_sync(0xffffffffu, gcur, r + H);
-                al = __fmul2_rn(al, make_float2(decay_gamma(lam2.x, ul), decay_gamma(lam2.y, ul)));
-                au = __fmul2_rn(au, make_float2(decay_gamma(lam2.x, uu), decay_gamma(lam2.y, uu)));
+                al = __fmul2_rn(al, decay_gamma2(lam2, make_float2(ul, ul)));
+                au = __fmul2_rn(au, decay_gamma2(lam2, make_float2(uu, uu)));
             }
             Op::fold2(AL, BL, al, cl);
             Op::fold2(AU, BU, au, cu);
@@ -864,8 +873,7 @@ scan_sequential_backward_kernel(const SeqBwdParams q, const __grid_constant__ CU
                 [[maybe_unused]] float2 u2 = make_float2(0.f, 0.f);
                 if constexpr (BOp::kDecay) {
                     u2 = make_float2(__shfl_sync(0xffffffffu, gcur, r), __shfl_sync(0xffffffffu, gcur, r - 1));
-                    BOp::coeffs_gated2(k2, h2, f2, make_float2(decay_gamma(lam2, u2.x), decay_gamma(lam2, u2.y)),
-                                       A, cP, cQ);
+                    BOp::coeffs_gated2(k2, h2, f2, decay_gamma2(make_float2(lam2, lam2), u2), A, cP, cQ);
                 } else {
                     BOp::coeffs2(k2, h2, f2, A, cP, cQ);
                 }

@@ -587,8 +587,8 @@ def test_projected_scan_argument_errors():
 def test_backward_kernel_choice():
     """The gradient walks whole sequences per warp (kernel 4) from 5 warps of
     32 channels per SM, on aligned vector-width rows; below that, on aligned
-    vector-width rows, the pipelined gradient (2) once it has two tiles per SM;
-    otherwise the tile kernel (1)."""
+    vector-width rows, the pipelined gradient (2) once it has two tiles per
+    block; otherwise the tile kernel (1)."""
     lib = _abi.lib()
     assert lib.sgr_backward_kernel(MINGRU, 16, 2048, 4096, BF16, 1) == 4     # 2048 groups
     assert lib.sgr_backward_kernel(MINGRU, 8, 2048, 4096, BF16, 1) == 4      # 1024 groups
