@@ -96,6 +96,14 @@ constexpr int kSeqQuadFrom = 16;
 constexpr int kSeqBwdMinWarpsPerSM = 5;
 constexpr int kSeqMaxSlots = 8;
 constexpr int kSeqMinSlots = 2;
+// The blocks of two or four warps per channel group keep two slots per warp
+// whatever their share of the shared memory: a shallower ring measured
+// faster than a deeper one (bf16 B x 2048 x 4096, us, two slots against
+// the share's 3 at B16 / 8 at B8: minGRU 158.3 against 160.1 and 102.8
+// against 105.1, decayed 184.7 against 184.6 and 115.4 against 119.2,
+// MinMax 76.2 against 77.3 at B8), while half the blocks at a time with
+// twice the share (a deeper ring, two waves) measured 193.0 at B16.
+constexpr int kSeqPairMaxSlots = 2;
 constexpr int kSeqWarpsPerBlock = 1;
 constexpr size_t kAssumedSmemPerSM = 233472;
 constexpr size_t kAssumedSmemReserved = 1024;
@@ -229,7 +237,8 @@ SeqLayout seq_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, siz
 }
 
 // the two-warp blocks of scan_sequential_pair_kernel: one block per channel
-// group, the block's share of the SM's shared memory split between its warps
+// group asking for its share of the SM's shared memory (so that the groups
+// spread evenly), of which its warps' rings take kSeqPairMaxSlots slots
 // wide: the two-channels-per-lane form (64-channel groups, float4 exchange)
 // with nw warps per group
 SeqLayout seq_pair_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm, size_t reserved,
@@ -245,7 +254,7 @@ SeqLayout seq_pair_layout(int64_t groups, int row_bytes, int sms, size_t smem_sm
         alloc = share > reserved ? (share - reserved) / 128 * 128 : 0;
     }
     alloc = std::min(alloc, smem_block_max);
-    int S = kSeqMaxSlots;
+    int S = kSeqPairMaxSlots;
     while (S > kSeqMinSlots && bytes(S) > alloc) --S;
     l.slots = S;
     l.smem = std::max(alloc, bytes(S));
