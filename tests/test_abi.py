@@ -231,6 +231,8 @@ def check_sequential_indices(pl, B, T, D, esz, check_cover):
     assert pl["n_channel_tiles"] == n_groups and pl["n_chains"] == B * n_groups
     assert pl["n_tiles"] == pl["n_chains"] < 2 ** 31
     assert 2 <= pl["stages"] <= 8
+    if pair:
+        assert pl["stages"] == 2                        # the pair kernels keep two slots per warp
     # the warps' rings, staging buffers and mbarriers fit their block's shared memory
     S = pl["stages"]
     if pair:
